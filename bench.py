@@ -1,0 +1,364 @@
+"""Benchmark of the NSA forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload nsa_64k]
+
+A step is one full NSA prefill forward (phi of K and V, compressed attention +
+group-summed block scores + top-k, selected-block attention, sliding window +
+gated combine) over the T = 65536 synthetic workload (B = 1, 64 query heads in
+4 KV groups of 16, d_k = 192, d_v = 128, top-16 of 64-token blocks, window 512).
+Inputs are resident in HBM when the timed region starts; L2 is flushed (a
+256 MB write) before every timed step, outside its CUDA events.  Rank 0 prints
+one JSON line.  With N > 1 every rank runs its own replica (the path does not
+shard across GPUs); value = tokens of all ranks / max-over-ranks time.
+
+--impl reference times the CPU oracle (the fp64 restatement of the pages in
+oracle/) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "NSA fwd tokens/s @T=64K and % bf16 tensor peak; decode GB/s vs HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L, S, BSEL = 32, 16, 64
+STAGES = ["phi_k", "phi_v", "cmp_select", "slc_attn", "swa_combine"]
+
+
+# ----------------------------------------------------------------------------- work counts
+
+def n_cmp(T):
+    return 0 if T < L else (T - L) // S + 1
+
+
+def nsa_flops(T, h_q, h_kv, d_k, d_v, top_k, window, B=1):
+    """Algorithmic FLOPs per stage: 2*(q.k pairs)*d_k + 2*(p.v pairs)*d_v over the pairs the
+    method evaluates (causal structure exact, no padding, no recomputation), plus phi."""
+    t = torch.arange(T, dtype=torch.float64)
+    nvis = torch.where(t < L - 1, torch.zeros_like(t), torch.clamp(torch.div(t - L + 1, S, rounding_mode="floor") + 1,
+                                                                  max=n_cmp(T)))
+    nb = torch.div(t, BSEL, rounding_mode="floor") + 1
+    slc = torch.where(nb <= top_k, t + 1, 64.0 * (top_k - 1) + torch.remainder(t, BSEL) + 1)
+    win = torch.clamp(t + 1, max=window)
+    per_pair = 2.0 * (d_k + d_v) * h_q * B
+    nc = n_cmp(T)
+    phi_k = 2.0 * B * nc * h_kv * L * d_k * d_k
+    phi_v = 2.0 * B * nc * h_kv * L * d_v * d_v
+    return {"phi_k": phi_k, "phi_v": phi_v, "cmp_select": float(nvis.sum()) * per_pair,
+            "slc_attn": float(slc.sum()) * per_pair, "swa_combine": float(win.sum()) * per_pair}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples nvidia-smi every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        if shutil.which("nvidia-smi"):
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu)],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+def cpu_workload():
+    c = synth.WORKLOADS["nsa_64k"]
+    return synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=0)
+
+
+def oracle_rate(x, n_sample, seed, threads):
+    """Oracle tokens/s on the 64K workload: phi over the whole sequence, timed, plus the three
+    branches on n_sample uniformly drawn query tokens, timed and scaled to all T tokens."""
+    import oracle
+    c = synth.WORKLOADS["nsa_64k"]
+    torch.set_num_threads(threads)
+    g = torch.Generator().manual_seed(seed)
+    toks = sorted(torch.randint(0, c["T"], (n_sample,), generator=g).tolist())
+    t0 = time.perf_counter()
+    kc = oracle.compress_cache(x.k, x.w_k, L, S)
+    vc = oracle.compress_cache(x.v, x.w_v, L, S)
+    t_phi = time.perf_counter() - t0
+    G = c["h_q"] // c["h_kv"]
+    q, k, v, gates = (oracle.nsa_oracle._f64(a) for a in (x.q, x.k, x.v, x.gates))
+    scale = 1.0 / math.sqrt(c["d_k"])
+    t0 = time.perf_counter()
+    for t in toks:
+        for gi in range(c["h_kv"]):
+            hs = slice(gi * G, (gi + 1) * G)
+            oracle.nsa_token(q[0, t, hs], k[0, :, gi], v[0, :, gi], kc[0, :, gi], vc[0, :, gi], gates[0, t, hs], t,
+                             l=L, s=S, b=BSEL, k=c["top_k"], w=c["window"], scale=scale)
+    t_tok = time.perf_counter() - t0
+    total = t_phi + t_tok * c["T"] / n_sample
+    return c["T"] / total, {"t_phi_s": round(t_phi, 3), "t_sample_s": round(t_tok, 3), "n_sample": n_sample}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    threads = os.cpu_count() or 1
+    c = synth.WORKLOADS["nsa_64k"]
+    n = args.ref_sample
+    rates = []
+    x = cpu_workload()
+    for i in range(args.warmup + args.steps):
+        r, info = oracle_rate(x, n, seed=100 + i, threads=threads)
+        if i >= args.warmup:
+            rates.append(r)
+    val = statistics.mean(rates)
+    sample = (f"per step: phi over all {c['T']} tokens plus all three branches for {n} uniformly drawn query "
+              f"tokens (64 heads), branch time scaled to {c['T']} tokens")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * c["T"] / val,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(c, "nsa_64k"),
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(c, name):
+    return {"workload": f"{name}: NSA forward B={c['B']} T={c['T']} h_q={c['h_q']} h_kv={c['h_kv']} "
+                        f"d_k={c['d_k']} d_v={c['d_v']} l=32 s=16 sel_block=64 top_k={c['top_k']} "
+                        f"window={c['window']} bf16",
+            "global_batch": c["B"], "seq_len": c["T"], "parallelism": "replicas",
+            "l2": "inputs 1.8 GB > 126 MB L2, plus a 256 MB L2 flush before every timed step (outside the events)"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args, rank, world, local_rank):
+    import block_sparse_attention_compress_b200 as nsa
+    from block_sparse_attention_compress_b200.torch_ops import NSAForward
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    c = synth.WORKLOADS[args.workload]
+    B, T, hq, hkv, dk, dv = c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"]
+    x = synth.nsa_inputs(B, T, hq, hkv, dk, dv, seed=rank, device=dev)
+    f = NSAForward(B, T, hq, hkv, dk, dv, x.w_k, x.w_v, top_k=c["top_k"], window=c["window"], device=dev)
+    out = torch.empty((B, T, hq, dv), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    nstage = len(STAGES) + 1
+    ev_sets = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    for evs in ev_sets:            # torch creates the CUDA event on first record
+        for e in evs:
+            e.record(stream)
+    torch.cuda.synchronize()
+    handles = [ctypes_array(ev) for ev in ev_sets]
+
+    def step(i=None):
+        if i is None:
+            f.cfg.stage_events, f.cfg.n_stage_events = None, 0
+        else:
+            f.cfg.stage_events, f.cfg.n_stage_events = handles[i][0], nstage
+        nsa.nsa_forward(x.q, x.k, x.v, x.gates, f.cfg, out)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(i)
+        torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    per_stage = {s: [] for s in STAGES}
+    step_ms = []
+    for evs in ev_sets:
+        step_ms.append(evs[0].elapsed_time(evs[-1]))
+        for j, s in enumerate(STAGES):
+            per_stage[s].append(evs[j].elapsed_time(evs[j + 1]))
+    my_ms = sum(step_ms)
+    total_ms = allreduce_max(my_ms, world, dev)
+    tokens = world * B * T * args.steps
+    value = tokens / (total_ms / 1000.0)
+
+    flops = nsa_flops(T, hq, hkv, dk, dv, c["top_k"], c["window"], B)
+    stage_mean = {s: statistics.mean(v) for s, v in per_stage.items()}
+    dom = max(stage_mean, key=stage_mean.get)
+    peaks, src = load_peaks()
+    ach = flops[dom] / (stage_mean[dom] * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    total_flops = sum(flops.values())
+    result = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; distributions of the workload)",
+        "config": workload_config(c, args.workload),
+        "tflops_computed": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12,
+        "frac_of_bf16_peak": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                     "frac": ach / peak, "traffic": None,
+                     "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside the step)"},
+        "stages_ms": {s: round(v, 4) for s, v in stage_mean.items()},
+        "stage_tflops": {s: round(flops[s] / (stage_mean[s] * 1e-3) / 1e12, 1) for s in STAGES},
+        "gpu_launches": len(STAGES) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, f, x, out, dev, world)
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        r, info = oracle_rate(cpu_workload(), args.ref_sample, seed=7, threads=os.cpu_count() or 1)
+        result["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+                                  "sample": f"phi over all {T} tokens plus the three branches for "
+                                            f"{args.ref_sample} uniformly drawn query tokens, scaled to {T} tokens",
+                                  **info}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(args, f, x, out, dev, world):
+    """Same step through the public API with inputs in pinned host memory: H2D copies of
+    q, k, v, gates, the forward, and the D2H copy of the output, all inside the timed region."""
+    import block_sparse_attention_compress_b200 as nsa
+    host_in = [t.cpu().pin_memory() for t in (x.q, x.k, x.v, x.gates)]
+    host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dev_in = [torch.empty_like(t, device=dev) for t in host_in]
+    f.cfg.stage_events, f.cfg.n_stage_events = None, 0
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = host_out.numel() * host_out.element_size()
+
+    def step():
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        nsa.nsa_forward(*dev_in, f.cfg, out)
+        host_out.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = allreduce_max(t0.elapsed_time(t1), world, dev)
+    tokens = world * out.shape[0] * out.shape[1] * args.steps
+    return {"value": tokens / (ms / 1000.0), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+def ctypes_array(events):
+    import ctypes
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), arr
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def allreduce_max(v, world, dev):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="nsa_64k", choices=["nsa_64k", "nsa_8k", "nsa_tiny"])
+    ap.add_argument("--ref-sample", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,140 @@
+"""Python binding of libnsa, the B200 Native Sparse Attention library.
+
+Argument marshalling only: every function here forwards to the C entry point
+of the same name (include/nsa.h) with raw device pointers taken from torch
+tensors, and the current torch CUDA stream unless one is given.  All
+arithmetic runs in the library's CUDA kernels; if ``libnsa.so`` has not been
+built, importing the entry points raises instead of falling back to anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnsa.so")
+
+NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
+NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
+
+EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_forward", "nsa_decode", "nsa_status_string")
+
+
+class NsaConfig(ctypes.Structure):
+    """Mirror of ``nsa_config`` in include/nsa.h (field order and types must match)."""
+    _fields_ = [
+        ("mode", ctypes.c_int32),
+        ("batch", ctypes.c_int32), ("seqlen", ctypes.c_int32), ("h_q", ctypes.c_int32),
+        ("h_kv", ctypes.c_int32), ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
+        ("cmp_block", ctypes.c_int32), ("cmp_stride", ctypes.c_int32), ("sel_block", ctypes.c_int32),
+        ("top_k", ctypes.c_int32), ("window", ctypes.c_int32),
+        ("force_first", ctypes.c_int32), ("force_local", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+        ("w_cmp_k", ctypes.c_void_p), ("w_cmp_v", ctypes.c_void_p),
+        ("sel_idx_out", ctypes.c_void_p),
+        ("kc_out", ctypes.c_void_p), ("vc_out", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("n_stage_events", ctypes.c_int32),
+    ]
+
+
+class NsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {nsa_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libnsa.so from the package directory (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is not built; run `python -m block_sparse_attention_compress_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    cfgp = ctypes.POINTER(NsaConfig)
+    lib.nsa_workspace_size.argtypes = [cfgp, ctypes.c_int]
+    lib.nsa_workspace_size.restype = sz
+    lib.nsa_compress.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
+    lib.nsa_compress.restype = ctypes.c_int
+    lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
+    lib.nsa_forward.restype = ctypes.c_int
+    lib.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, cfgp, vp, vp]
+    lib.nsa_decode.restype = ctypes.c_int
+    lib.nsa_status_string.argtypes = [ctypes.c_int]
+    lib.nsa_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_contiguous():
+        raise ValueError("tensors passed to libnsa must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream, *tensors) -> int | None:
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+    for t in tensors:
+        if t is not None and not isinstance(t, int) and t.is_cuda:
+            return torch.cuda.current_stream(t.device).cuda_stream
+    return None
+
+
+def make_config(**fields) -> NsaConfig:
+    """Build an NsaConfig; tensors given for pointer fields are replaced by their addresses."""
+    cfg = NsaConfig()
+    defaults = dict(mode=NSA_MODE_NSA, cmp_block=32, cmp_stride=16, sel_block=64, top_k=16, window=512,
+                    force_first=1, force_local=1, softmax_scale=0.0)
+    defaults.update(fields)
+    for name, val in defaults.items():
+        if name in ("w_cmp_k", "w_cmp_v", "sel_idx_out", "kc_out", "vc_out", "workspace"):
+            val = _ptr(val)
+        setattr(cfg, name, val)
+    return cfg
+
+
+def nsa_status_string(status: int) -> str:
+    return load_library().nsa_status_string(int(status)).decode()
+
+
+def nsa_workspace_size(cfg: NsaConfig, decode_batch: int = 0) -> int:
+    return int(load_library().nsa_workspace_size(ctypes.byref(cfg), int(decode_batch)))
+
+
+def _check(status: int, where: str) -> int:
+    if status != NSA_OK:
+        raise NsaError(status, where)
+    return status
+
+
+def nsa_compress(x, w, out, l: int = 32, s: int = 16, stream=None, check: bool = True) -> int:
+    """phi over [B, T, H, d] -> out [B, N_c, H, d_out] (see include/nsa.h)."""
+    B, T, H, d = x.shape
+    st = load_library().nsa_compress(_ptr(x), _ptr(w), B, T, H, d, w.shape[1], l, s, _ptr(out),
+                                     _stream(stream, x))
+    return _check(st, "nsa_compress") if check else st
+
+
+def nsa_forward(q, k, v, gates, cfg: NsaConfig, out, stream=None, check: bool = True) -> int:
+    st = load_library().nsa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), ctypes.byref(cfg), _ptr(out),
+                                    _stream(stream, q))
+    return _check(st, "nsa_forward") if check else st
+
+
+def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, max_seqlen: int, gates, cfg: NsaConfig, out,
+               stream=None, check: bool = True) -> int:
+    st = load_library().nsa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(kc_cache), _ptr(vc_cache),
+                                   _ptr(seqlens), int(max_seqlen), _ptr(gates), ctypes.byref(cfg), _ptr(out),
+                                   _stream(stream, q))
+    return _check(st, "nsa_decode") if check else st

@@ -1,0 +1,120 @@
+// K1: block compression phi ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5: every
+// block of l tokens becomes one key and one value vector; "一文比较 Kimi 和 Deepseek 的两篇
+// 稀疏注意力机制论文", "Deepseek 的论文核心点": a learned map compresses each block).
+//
+// out[b, i, h, :] = vec(x[b, s*i : s*i+l, h, :]) @ w, vec token-major (index r*d + c).
+// As a GEMM: M = N_c windows per (b, h), N = d_out, K = l*d.  The A operand is
+// never materialised: window i, k-chunk (r, c0) is read straight from x
+// (each 64-wide k-chunk lies inside one token because d % 64 == 0).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nsa {
+
+namespace {
+constexpr int kBM = 64, kBN = 64, kBK = 64, kThreads = 128;
+
+template <int D, int DOUT>
+__global__ void __launch_bounds__(kThreads)
+compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
+                int l, int s, int nc, __nv_bfloat16* __restrict__ out) {
+  __shared__ __align__(128) __nv_bfloat16 sA[2][kBM * kBK];
+  __shared__ __align__(128) __nv_bfloat16 sB[2][kBK * kBN];
+  using Swz = SwzTile<kBK>;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int i0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
+  const int bh = blockIdx.z, b = bh / H, h = bh % H;
+  const int nk = l * D / kBK;
+
+  auto load = [&](int kc, int buf) {
+    const int kk0 = kc * kBK;
+    const int r = kk0 / D, c0 = kk0 % D;
+#pragma unroll
+    for (int e = tid; e < kBM * (kBK / 8); e += kThreads) {
+      const int row = e >> 3, ch = e & 7;
+      const int i = i0 + row;
+      const bool ok = i < nc;
+      const __nv_bfloat16* src =
+          x + (((size_t)b * T + (ok ? (size_t)s * i + r : 0)) * H + h) * D + c0 + ch * 8;
+      cp_async16(&sA[buf][Swz::offset(row, ch)], src, ok);
+    }
+#pragma unroll
+    for (int e = tid; e < kBK * (kBN / 8); e += kThreads) {
+      const int row = e >> 3, ch = e & 7;
+      const __nv_bfloat16* src = w + (size_t)(kk0 + row) * DOUT + n0 + ch * 8;
+      cp_async16(&sB[buf][Swz::offset(row, ch)], src, true);
+    }
+  };
+
+  float acc[kBN / 8][4];
+#pragma unroll
+  for (int j = 0; j < kBN / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+
+  load(0, 0);
+  cp_async_commit();
+  for (int kc = 0; kc < nk; ++kc) {
+    if (kc + 1 < nk) load(kc + 1, (kc + 1) & 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    const int buf = kc & 1;
+#pragma unroll
+    for (int ks = 0; ks < kBK / 16; ++ks) {
+      uint32_t a[4];
+      {
+        const int row = warp * 16 + (lane & 15);
+        const int ch = 2 * ks + (lane >> 4);
+        ldsm_x4(a[0], a[1], a[2], a[3], smem_u32(&sA[buf][Swz::offset(row, ch)]));
+      }
+#pragma unroll
+      for (int np = 0; np < kBN / 16; ++np) {
+        uint32_t b0, b1, b2, b3;
+        const int krow = ks * 16 + (lane & 15);
+        const int ch = 2 * np + (lane >> 4);
+        ldsm_x4_t(b0, b1, b2, b3, smem_u32(&sB[buf][Swz::offset(krow, ch)]));
+        mma16816(acc[2 * np], a, b0, b1);
+        mma16816(acc[2 * np + 1], a, b2, b3);
+      }
+    }
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+
+  const int gl = lane >> 2, cq = lane & 3;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int i = i0 + warp * 16 + gl + half * 8;
+    if (i >= nc) continue;
+    __nv_bfloat16* dst = out + (((size_t)b * nc + i) * H + h) * DOUT + n0;
+#pragma unroll
+    for (int j = 0; j < kBN / 8; ++j) {
+      const uint32_t v = pack_bf16(acc[j][2 * half], acc[j][2 * half + 1]);
+      *reinterpret_cast<uint32_t*>(dst + j * 8 + 2 * cq) = v;
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch(const void* x, const void* w, int B, int T, int H, int l, int s, int nc, void* out,
+                   cudaStream_t st) {
+  dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
+  compress_kernel<D, D><<<grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                   static_cast<const __nv_bfloat16*>(w), T, H, l, s, nc,
+                                                   static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
+                            cudaStream_t st) {
+  const int nc = T < l ? 0 : (T - l) / s + 1;
+  if (nc == 0 || B == 0 || H == 0) return cudaSuccess;
+  switch (d) {
+    case 64: return launch<64>(x, w, B, T, H, l, s, nc, out, st);
+    case 128: return launch<128>(x, w, B, T, H, l, s, nc, out, st);
+    case 192: return launch<192>(x, w, B, T, H, l, s, nc, out, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace nsa

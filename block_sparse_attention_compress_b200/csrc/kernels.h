@@ -1,0 +1,38 @@
+// Internal launch wrappers (host side) of the NSA kernels.  Every wrapper
+// launches on `st`, returns cudaGetLastError(), and expects arguments that
+// nsa_api.cu has already validated.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace nsa {
+
+// K1: phi for every (b, h): out [B, N_c, H, d] bf16 (l = 32, s = 16 validated).
+cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
+                            cudaStream_t st);
+
+struct FwdArgs {
+  const void* q;      // [B, T, Hq, dk] bf16
+  const void* k;      // [B, T, Hkv, dk]
+  const void* v;      // [B, T, Hkv, dv]
+  const void* gates;  // [B, T, Hq, 3]
+  const void* kc;     // [B, nc, Hkv, dk]
+  const void* vc;     // [B, nc, Hkv, dv]
+  float* acc;         // [B, T, Hq, dv] fp32 scratch: gated compressed + selected outputs
+  int32_t* idx;       // [B, Hkv, T, top_k]
+  void* out;          // [B, T, Hq, dv] bf16
+  int B, T, Hq, Hkv, G, dk, dv, nc;
+  int top_k, window, force_first, force_local;
+  float scale_log2;   // softmax scale * log2(e)
+};
+
+// K2: compressed attention (writes acc = g_cmp * o_cmp) + group-summed block
+// scores + top-k (writes idx).
+cudaError_t launch_cmp_select(const FwdArgs& a, cudaStream_t st);
+// K3: selected-block attention (acc += g_slc * o_slc).
+cudaError_t launch_slc_attn(const FwdArgs& a, cudaStream_t st);
+// K4 + K5: sliding window and gated combine (out = bf16(acc + g_win * o_win)).
+cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st);
+
+}  // namespace nsa

@@ -1,0 +1,176 @@
+// C ABI of the NSA library: argument validation, workspace carving and the
+// launch sequence on the caller's stream.  See include/nsa.h for the contract.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/nsa.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxTokensNsa = 65536;   // 1024 selection blocks per token (top-k kept in shared memory)
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int n_cmp(int T, int l, int s) { return T < l ? 0 : (T - l) / s + 1; }
+
+bool dims_supported(int dk, int dv) {
+  return (dk == 64 && dv == 64) || (dk == 128 && dv == 128) || (dk == 192 && dv == 128);
+}
+
+// Shape checks common to every entry point.  Returns NSA_OK or the error to report.
+nsa_status check_cfg(const nsa_config* c) {
+  if (!c) return NSA_ERR_INVALID_ARG;
+  if (c->mode != NSA_MODE_NSA && c->mode != NSA_MODE_MOBA) return NSA_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->seqlen < 1 || c->h_q < 1 || c->h_kv < 1 || c->d_k < 1 || c->d_v < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (c->h_q % c->h_kv) return NSA_ERR_INVALID_ARG;
+  if (c->top_k < 0 || c->sel_block < 1) return NSA_ERR_INVALID_ARG;
+  if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return NSA_ERR_INVALID_ARG;
+  if (c->mode == NSA_MODE_NSA) {
+    if (c->cmp_block < 1 || c->cmp_stride < 1 || c->window < 1) return NSA_ERR_INVALID_ARG;
+    if ((c->force_first != 0 && c->force_first != 1) || (c->force_local != 0 && c->force_local != 1))
+      return NSA_ERR_INVALID_ARG;
+    if (c->top_k < 1 || c->top_k < c->force_first + c->force_local) return NSA_ERR_INVALID_ARG;
+    if (c->sel_block % c->cmp_stride) return NSA_ERR_INVALID_ARG;
+    if (!c->w_cmp_k || !c->w_cmp_v || !aligned16(c->w_cmp_k) || !aligned16(c->w_cmp_v))
+      return NSA_ERR_INVALID_ARG;
+    if (c->cmp_block != 32 || c->cmp_stride != 16 || c->sel_block != 64) return NSA_ERR_UNSUPPORTED;
+    if (c->h_q / c->h_kv > 16 || !dims_supported(c->d_k, c->d_v) || c->top_k > 32) return NSA_ERR_UNSUPPORTED;
+    if (c->seqlen > kMaxTokensNsa) return NSA_ERR_UNSUPPORTED;
+  } else {
+    if (c->h_q != c->h_kv || c->d_k != c->d_v) return NSA_ERR_INVALID_ARG;
+    return NSA_ERR_UNSUPPORTED;
+  }
+  if ((c->sel_idx_out && !aligned16(c->sel_idx_out)) || (c->kc_out && !aligned16(c->kc_out)) ||
+      (c->vc_out && !aligned16(c->vc_out)))
+    return NSA_ERR_INVALID_ARG;
+  return NSA_OK;
+}
+
+struct FwdLayout {
+  size_t kc, vc, idx, acc, total;
+};
+
+FwdLayout forward_layout(const nsa_config* c) {
+  const size_t B = c->batch, T = c->seqlen, nc = n_cmp(c->seqlen, c->cmp_block, c->cmp_stride);
+  FwdLayout L{};
+  size_t off = 0;
+  L.kc = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
+  L.vc = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
+  L.idx = off; off = align_up(off + B * c->h_kv * T * c->top_k * 4);
+  L.acc = off; off = align_up(off + B * T * c->h_q * c->d_v * 4);
+  L.total = off;
+  return L;
+}
+
+nsa_status check_workspace(const nsa_config* c, size_t need) {
+  if (need == 0) return NSA_OK;
+  if (!c->workspace || (reinterpret_cast<uintptr_t>(c->workspace) % kAlign)) return NSA_ERR_WORKSPACE;
+  if (c->workspace_bytes < need) return NSA_ERR_WORKSPACE;
+  return NSA_OK;
+}
+
+nsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA; }
+
+// Records the caller's measurement events between kernels (see stage_events in nsa.h).
+struct StageMarks {
+  void* const* ev;
+  int n, next;
+  StageMarks(const nsa_config* c, int kernels)
+      : ev(c->stage_events), n(c->stage_events && c->n_stage_events >= kernels + 1 ? kernels + 1 : 0), next(0) {}
+  cudaError_t mark(cudaStream_t s) {
+    if (next >= n) return cudaSuccess;
+    return cudaEventRecord(static_cast<cudaEvent_t>(ev[next++]), s);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* nsa_status_string(nsa_status s) {
+  switch (s) {
+    case NSA_OK: return "NSA_OK";
+    case NSA_ERR_INVALID_ARG: return "NSA_ERR_INVALID_ARG";
+    case NSA_ERR_UNSUPPORTED: return "NSA_ERR_UNSUPPORTED";
+    case NSA_ERR_WORKSPACE: return "NSA_ERR_WORKSPACE";
+    case NSA_ERR_CUDA: return "NSA_ERR_CUDA";
+    case NSA_ERR_TIMEOUT: return "NSA_ERR_TIMEOUT";
+  }
+  return "NSA_ERR_UNKNOWN";
+}
+
+size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch) {
+  if (check_cfg(cfg) != NSA_OK || decode_batch < 0) return 0;
+  if (decode_batch == 0) return forward_layout(cfg).total;
+  return 0;
+}
+
+nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t T, int32_t H, int32_t d, int32_t d_out,
+                        int32_t l, int32_t s, void* out, void* stream) {
+  if (!x || !w || !out || B < 1 || T < 1 || H < 1 || d < 1 || d_out < 1 || l < 1 || s < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return NSA_ERR_INVALID_ARG;
+  if (l != 32 || s != 16 || d_out != d || (d != 64 && d != 128 && d != 192)) return NSA_ERR_UNSUPPORTED;
+  return from_cuda(nsa::launch_compress(x, w, B, T, H, d, l, s, out, static_cast<cudaStream_t>(stream)));
+}
+
+nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* gates, const nsa_config* cfg,
+                       void* out, void* stream) {
+  nsa_status st = check_cfg(cfg);
+  if (st != NSA_OK) return st;
+  if (!q || !k || !v || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return NSA_ERR_INVALID_ARG;
+  if (cfg->mode == NSA_MODE_NSA && (!gates || (reinterpret_cast<uintptr_t>(gates) & 1u)))
+    return NSA_ERR_INVALID_ARG;
+  const FwdLayout L = forward_layout(cfg);
+  st = check_workspace(cfg, L.total);
+  if (st != NSA_OK) return st;
+
+  auto ws = static_cast<uint8_t*>(cfg->workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nsa::FwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.gates = gates; a.out = out;
+  a.B = cfg->batch; a.T = cfg->seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
+  a.dk = cfg->d_k; a.dv = cfg->d_v; a.nc = n_cmp(cfg->seqlen, cfg->cmp_block, cfg->cmp_stride);
+  a.top_k = cfg->top_k; a.window = cfg->window;
+  a.force_first = cfg->force_first; a.force_local = cfg->force_local;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  void* kc = cfg->kc_out ? cfg->kc_out : ws + L.kc;
+  void* vc = cfg->vc_out ? cfg->vc_out : ws + L.vc;
+  a.kc = kc; a.vc = vc;
+  a.idx = cfg->sel_idx_out ? cfg->sel_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  a.acc = reinterpret_cast<float*>(ws + L.acc);
+
+  StageMarks marks(cfg, 5);
+  cudaError_t e = marks.mark(s);
+  if (e == cudaSuccess)
+    e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, kc, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess)
+    e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, cfg->cmp_block, cfg->cmp_stride, vc, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_cmp_select(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_slc_attn(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_swa_combine(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  return from_cuda(e);
+}
+
+nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* kc_cache,
+                      const void* vc_cache, const int32_t* seqlens, int32_t max_seqlen, const void* gates,
+                      const nsa_config* cfg, void* out, void* stream) {
+  nsa_status st = check_cfg(cfg);
+  if (st != NSA_OK) return st;
+  (void)q; (void)k_cache; (void)v_cache; (void)kc_cache; (void)vc_cache; (void)seqlens; (void)max_seqlen;
+  (void)gates; (void)out; (void)stream;
+  return NSA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

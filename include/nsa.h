@@ -1,0 +1,179 @@
+/*
+ * nsa.h -- C ABI of the B200 (sm_100a) Native Sparse Attention library.
+ *
+ * The operations are those described on these pages (cited by title and section):
+ *   [NOTES] zjai.club episode notes, "逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文
+ *           （含投屏版）——“硬件上的暴力美学”", §5-§10, §13-§17.
+ *   [BLOG]  sunshychen.top, "一文比较 Kimi 和 Deepseek 的两篇稀疏注意力机制论文",
+ *           sections "Kimi 的论文核心点" and "Deepseek 的论文核心点".
+ *   [EN]    youtublog.net/en, "Songlin Yang Explains Attention Mechanisms from
+ *           DeepSeek, Kimi, and MiniMax" (paragraphs on the three branches and GQA).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned, contiguous, row-major device pointers whose
+ *     base is 16-byte aligned.  bf16 unless stated.  The library allocates
+ *     and frees nothing; scratch memory is the caller's `workspace`.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  The return value reports only what the host can see:
+ *     argument validation (nothing is launched when it fails), a workspace
+ *     that is too small, and launch errors.  Faults inside a kernel surface
+ *     at the caller's next synchronisation.
+ *   - Stateless and re-entrant: concurrent calls on different streams are
+ *     safe when their outputs and workspaces do not overlap.
+ *   - Shapes: B batch, T tokens, H_q query heads, H_kv KV heads, G = H_q/H_kv
+ *     query heads per KV head (query head h uses KV head h / G), d_k, d_v.
+ */
+#ifndef NSA_H_
+#define NSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NSA_API __attribute__((visibility("default")))
+#else
+#define NSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NSA_OK = 0,
+  NSA_ERR_INVALID_ARG = 1,  /* a null pointer, a bad shape or an inconsistent config */
+  NSA_ERR_UNSUPPORTED = 2,  /* a legal config these kernels do not implement */
+  NSA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than nsa_workspace_size() */
+  NSA_ERR_CUDA = 4,         /* a kernel launch failed (cudaGetLastError) */
+  NSA_ERR_TIMEOUT = 5       /* reserved for bounded device-side waits (none in this version) */
+} nsa_status;
+
+typedef enum {
+  NSA_MODE_NSA = 0,   /* compressed + selected + sliding-window branches, gated sum */
+  NSA_MODE_MOBA = 1   /* MoBA: mean-pooled block keys, per-head top-k plus the own block */
+} nsa_mode;
+
+/*
+ * Problem description.  Fields marked (NSA) are ignored in MoBA mode.
+ *
+ *   mode          nsa_mode.
+ *   batch, seqlen B and T of the prefill (nsa_forward); in nsa_decode,
+ *                 `batch` is the number of sequences and `seqlen` the capacity
+ *                 L_max of the caches (their second dimension).
+ *   h_q, h_kv     query and KV heads; h_q % h_kv == 0.  MoBA needs h_q == h_kv.
+ *   d_k, d_v      head dims.  Implemented: NSA (d_k,d_v) in {(64,64),(128,128),
+ *                 (192,128)}, G <= 16; MoBA d_k = d_v = 128.
+ *   cmp_block,    (NSA) compression block l and stride s ([NOTES] §5: each block
+ *   cmp_stride    of l tokens becomes one key and one value).  Implemented: 32, 16.
+ *   sel_block     selection block size b: 64 for NSA ([NOTES] §17: 64-token blocks,
+ *                 top-16), the MoBA block size (512 in [NOTES] §17) for MoBA.
+ *   top_k         NSA: blocks per (token, KV head), forced ones included (<= 32).
+ *                 MoBA: past blocks per (token, head), the own block excluded (<= 7).
+ *   window        (NSA) sliding window w: the last w tokens including the query.
+ *   force_first,  (NSA) always select block 0 / the query's own block (0 or 1);
+ *   force_local   top_k >= force_first + force_local.
+ *   softmax_scale scale of q.k in every attention; 0 means 1/sqrt(d_k).
+ *   w_cmp_k       (NSA) phi weights for keys, bf16 [l*d_k, d_k]: compressed key
+ *                 i = vec(K[s*i : s*i+l]) @ w_cmp_k, vec token-major (index r*d+c).
+ *   w_cmp_v       (NSA) phi weights for values, bf16 [l*d_v, d_v].
+ *   sel_idx_out   optional int32 output of the chosen blocks: NSA [B, H_kv, T, top_k],
+ *                 MoBA [B, H_q, T, top_k+1]; ascending, padded with -1.  NULL: not written.
+ *   kc_out,vc_out optional bf16 outputs of the compressed keys/values
+ *                 [B, N_c, H_kv, d_k|d_v], N_c = (T-l)/s+1 (0 if T < l).  NULL: kept
+ *                 in the workspace.
+ *   workspace,    caller-owned device scratch, 256-byte aligned, at least
+ *   workspace_bytes nsa_workspace_size(cfg, 0) bytes (nsa_decode: (cfg, batch)).
+ *   stage_events  optional, for measurement: an array of n_stage_events cudaEvent_t
+ *   n_stage_events handles.  When n_stage_events >= (kernels launched) + 1, event 0 is
+ *                 recorded on `stream` before the first kernel and event i after the
+ *                 i-th, so that cudaEventElapsedTime gives each kernel's duration.
+ *                 nsa_forward launches 5 kernels in NSA mode (phi of K, phi of V,
+ *                 compressed attention + selection, selected attention, window +
+ *                 combine).  NULL or too few: nothing is recorded.
+ */
+typedef struct {
+  int32_t mode;
+  int32_t batch, seqlen, h_q, h_kv, d_k, d_v;
+  int32_t cmp_block, cmp_stride, sel_block, top_k, window;
+  int32_t force_first, force_local;
+  float softmax_scale;
+  const void* w_cmp_k;
+  const void* w_cmp_v;
+  int32_t* sel_idx_out;
+  void* kc_out;
+  void* vc_out;
+  void* workspace;
+  size_t workspace_bytes;
+  void* const* stage_events;
+  int32_t n_stage_events;
+} nsa_config;
+
+/* Bytes of workspace nsa_forward (decode_batch == 0) or nsa_decode
+ * (decode_batch == number of sequences) needs for `cfg`; 0 if cfg is invalid. */
+NSA_API size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch);
+
+/*
+ * nsa_compress -- block compression phi ([NOTES] §5; [BLOG] "Deepseek 的论文核心点":
+ * each block of l tokens is mapped to one short key or value vector).
+ *   x    bf16 [B, T, H, d]      keys or values
+ *   w    bf16 [l*d, d_out]      phi weights (one matrix for all heads)
+ *   out  bf16 [B, N_c, H, d_out] with N_c = (T-l)/s+1; row i = vec(x[s*i : s*i+l]) @ w,
+ *        accumulated in fp32, rounded once to bf16.
+ * Implemented: d in {64,128,192}, d_out == d, (l, s) = (32, 16).
+ */
+NSA_API nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t T, int32_t H, int32_t d,
+                        int32_t d_out, int32_t l, int32_t s, void* out, void* stream);
+
+/*
+ * nsa_forward -- prefill forward.
+ *   q     bf16 [B, T, H_q, d_k]
+ *   k     bf16 [B, T, H_kv, d_k]
+ *   v     bf16 [B, T, H_kv, d_v]
+ *   gates bf16 [B, T, H_q, 3] (NSA; order compressed, selected, window) -- per-token
+ *         per-head branch weights ([NOTES] §6: each branch output is scaled by a gate
+ *         computed from the current token, then the three are added).  NULL in MoBA mode.
+ *   out   bf16 [B, T, H_q, d_v]
+ *
+ * NSA mode, for every token t and query head h (group g = h / G):
+ *   o_cmp  softmax attention over the compressed blocks i with s*i+l-1 <= t ([NOTES] §5);
+ *   score  per 64-token block j: sum over the group's heads and over the visible
+ *          compressed blocks i whose span meets block j of their probabilities
+ *          ([NOTES] §8; [BLOG] "Deepseek 的论文核心点");
+ *   idx    the top_k blocks by score (forced blocks first, ties to the lower index),
+ *          shared by the whole group ([NOTES] §7-§8);
+ *   o_slc  softmax attention over the tokens u <= t of the chosen blocks;
+ *   o_win  softmax attention over u in [t-w+1, t];
+ *   out    g_cmp*o_cmp + g_slc*o_slc + g_win*o_win, rounded to bf16.
+ * MoBA mode, per token t and head h ([BLOG] "Kimi 的论文核心点"; [NOTES] §16-§17):
+ *   the top_k complete past blocks j < t/b by q.mean(K_j) plus the own block t/b,
+ *   one softmax over their tokens u <= t.
+ */
+NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* gates,
+                       const nsa_config* cfg, void* out, void* stream);
+
+/*
+ * nsa_decode -- one decode step per sequence ([NOTES] §13: decoding is bound by
+ * the KV bytes read per step).  NSA mode only.
+ *   q         bf16 [B, H_q, d_k]        the new token's queries
+ *   k_cache   bf16 [B, L_max, H_kv, d_k], v_cache bf16 [B, L_max, H_kv, d_v]
+ *   kc_cache  bf16 [B, N_c(L_max), H_kv, d_k], vc_cache [.., d_v]: phi of the caches
+ *             (nsa_compress); only the first N_c(seqlens[b]) rows are read.
+ *   seqlens   int32 [B] device: tokens in sequence b's cache including the new one
+ *             (1 <= seqlens[b] <= L_max); the query sits at position seqlens[b]-1.
+ *   max_seqlen an upper bound of seqlens (host), <= cfg->seqlen.
+ *   gates     bf16 [B, H_q, 3];  out bf16 [B, H_q, d_v].
+ * cfg->batch = B, cfg->seqlen = L_max; sel_idx_out (optional) is [B, H_kv, top_k].
+ */
+NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache,
+                      const void* kc_cache, const void* vc_cache, const int32_t* seqlens,
+                      int32_t max_seqlen, const void* gates, const nsa_config* cfg,
+                      void* out, void* stream);
+
+/* Human-readable name of a status code (static storage). */
+NSA_API const char* nsa_status_string(nsa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_H_ */

@@ -1,0 +1,139 @@
+"""The C-ABI library on the CPU: it loads, exports every entry point
+include/nsa.h declares, its config struct matches the ctypes mirror, and
+host-side validation answers without launching anything (no GPU needed)."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import block_sparse_attention_compress_b200 as nsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_sparse_attention_compress_b200 import build
+    build.build()
+    return nsa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nsa_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(names) == set(nsa.EXPORTED)
+    out = subprocess.run(["nm", "-D", "--defined-only", nsa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT\s+(nsa_\w+)", out))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_config_layout_matches_header():
+    src = r"""
+    #include <stddef.h>
+    #include <stdio.h>
+    #include "nsa.h"
+    int main(void) {
+      printf("%zu", sizeof(nsa_config));
+    #define F(x) printf(" %s=%zu", #x, offsetof(nsa_config, x));
+      F(mode) F(batch) F(seqlen) F(h_q) F(h_kv) F(d_k) F(d_v) F(cmp_block) F(cmp_stride) F(sel_block)
+      F(top_k) F(window) F(force_first) F(force_local) F(softmax_scale) F(w_cmp_k) F(w_cmp_v)
+      F(sel_idx_out) F(kc_out) F(vc_out) F(workspace) F(workspace_bytes) F(stage_events) F(n_stage_events)
+      return 0;
+    }
+    """
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "l.c")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", os.path.join(d, "l")], check=True)
+        got = subprocess.run([os.path.join(d, "l")], capture_output=True, text=True, check=True).stdout.split()
+    assert int(got[0]) == ctypes.sizeof(nsa.NsaConfig)
+    for item in got[1:]:
+        name, off = item.split("=")
+        assert getattr(nsa.NsaConfig, name).offset == int(off), name
+
+
+def _cfg(**kw):
+    base = dict(batch=1, seqlen=1024, h_q=4, h_kv=1, d_k=64, d_v=64, top_k=4, window=128,
+                w_cmp_k=0x1000, w_cmp_v=0x2000)
+    base.update(kw)
+    return nsa.make_config(**base)
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["NSA_OK", "NSA_ERR_INVALID_ARG", "NSA_ERR_UNSUPPORTED", "NSA_ERR_WORKSPACE",
+                                 "NSA_ERR_CUDA", "NSA_ERR_TIMEOUT"]):
+        assert nsa.nsa_status_string(code) == name
+
+
+def test_workspace_size_of_the_workloads(lib):
+    c = _cfg()
+    # kc 63*64*2, vc same, idx 1*1024*4*4, acc 1024*4*64*4 (each rounded up to 256 B)
+    up = lambda x: (x + 255) // 256 * 256
+    assert nsa.nsa_workspace_size(c) == 2 * up(63 * 64 * 2) + up(1024 * 4 * 4) + up(1024 * 4 * 64 * 4)
+    big = _cfg(seqlen=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512)
+    assert nsa.nsa_workspace_size(big) > 65536 * 64 * 128 * 4
+    assert nsa.nsa_workspace_size(_cfg(h_q=6, h_kv=4)) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(h_q=6, h_kv=4), nsa.NSA_ERR_INVALID_ARG),
+    (dict(batch=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(top_k=1), nsa.NSA_ERR_INVALID_ARG),            # fewer than the two forced blocks
+    (dict(window=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(w_cmp_k=0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(w_cmp_k=0x1004), nsa.NSA_ERR_INVALID_ARG),     # misaligned weights
+    (dict(softmax_scale=-1.0), nsa.NSA_ERR_INVALID_ARG),
+    (dict(mode=7), nsa.NSA_ERR_INVALID_ARG),
+    (dict(sel_block=40), nsa.NSA_ERR_INVALID_ARG),       # not a multiple of the stride
+    (dict(cmp_block=64, cmp_stride=32), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(h_q=32, h_kv=1), nsa.NSA_ERR_UNSUPPORTED),     # group of 32 heads
+    (dict(d_k=96, d_v=96), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(seqlen=65537), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(top_k=33), nsa.NSA_ERR_UNSUPPORTED),
+])
+def test_forward_rejects_bad_configs_without_launching(lib, kw, status):
+    c = _cfg(**kw)
+    st = nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0x40000, c, 0x50000, check=False)
+    assert st == status
+
+
+def test_forward_rejects_null_and_misaligned_tensors(lib):
+    c = _cfg(workspace=0x100000, workspace_bytes=1 << 30)
+    assert nsa.nsa_forward(0, 0x20000, 0x30000, 0x40000, c, 0x50000, check=False) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_forward(0x10008, 0x20000, 0x30000, 0x40000, c, 0x50000, check=False) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0, c, 0x50000, check=False) == nsa.NSA_ERR_INVALID_ARG
+
+
+def test_forward_rejects_small_or_misaligned_workspace(lib):
+    c = _cfg()
+    need = nsa.nsa_workspace_size(c)
+    for ws, nbytes in [(0, 0), (0x100000, need - 1), (0x100080, need)]:
+        c.workspace, c.workspace_bytes = ws, nbytes
+        st = nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0x40000, c, 0x50000, check=False)
+        assert st == nsa.NSA_ERR_WORKSPACE
+
+
+def test_compress_rejects_bad_arguments(lib):
+    L = lib
+    assert L.nsa_compress(0, 0x1000, 1, 64, 1, 64, 64, 32, 16, 0x2000, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress(0x1000, 0x2000, 1, 64, 1, 64, 64, 16, 8, 0x3000, None) == nsa.NSA_ERR_UNSUPPORTED
+    assert L.nsa_compress(0x1000, 0x2000, 1, 64, 1, 96, 96, 32, 16, 0x3000, None) == nsa.NSA_ERR_UNSUPPORTED
+    assert L.nsa_compress(0x1000, 0x2000, 0, 64, 1, 64, 64, 32, 16, 0x3000, None) == nsa.NSA_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(nsa, "_lib", None)
+    monkeypatch.setattr(nsa, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        nsa.load_library()

@@ -1,0 +1,154 @@
+"""GPU parity of the NSA prefill forward (nsa_compress / nsa_forward through
+the C ABI) against the fp64 CPU oracle on the same seeded inputs."""
+import pytest
+import torch
+
+import oracle
+import synth
+from block_sparse_attention_compress_b200 import build
+from block_sparse_attention_compress_b200.torch_ops import NSAForward, compress_torch
+from tests.helpers import assert_close, idx_agreement, token_mask
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+
+
+def run_gpu(x, top_k, window, gates=None, **kw):
+    B, T, hq, dk = x.q.shape
+    hkv, dv = x.k.shape[2], x.v.shape[3]
+    dev = [t.to(DEV) for t in (x.q, x.k, x.v, x.gates if gates is None else gates, x.w_k, x.w_v)]
+    f = NSAForward(B, T, hq, hkv, dk, dv, dev[4], dev[5], top_k=top_k, window=window, **kw)
+    out = f(*dev[:4])
+    torch.cuda.synchronize()
+    return out.cpu(), f.idx.cpu(), f.kc.cpu(), f.vc.cpu()
+
+
+def check_against_oracle(x, top_k, window, tokens=None, gates=None, min_exact=0.97):
+    B, T, hq, dk = x.q.shape
+    hkv = x.k.shape[2]
+    G = hq // hkv
+    g = x.gates if gates is None else gates
+    out, idx, kc, vc = run_gpu(x, top_k, window, gates=g)
+    ref = oracle.nsa_forward(x.q, x.k, x.v, g, x.w_k, x.w_v, top_k=top_k, window=window, tokens=tokens)
+    toks = ref["tokens"]
+    # compressed K/V: bf16 rounding of the same products, at most one bf16 step apart
+    exact_kc = oracle.compress_cache(x.k, x.w_k, 32, 16, round_kc=False)
+    ulp = exact_kc.abs() * 2 ** -7 + 1e-6
+    assert ((kc.double() - exact_kc).abs() <= ulp).all()
+    assert (kc.double() == ref["kc"]).double().mean() > 0.99
+    gi = idx[:, :, toks]
+    exact, swapped = idx_agreement(gi, ref["idx"], ref["score"], tokens=toks)
+    assert exact >= min_exact * gi.shape[0] * gi.shape[1] * gi.shape[2]
+    mask = token_mask((B, len(toks), hq), swapped, G)
+    return assert_close(out[:, toks], ref["out"], mask=mask.unsqueeze(-1).expand(-1, -1, -1, out.shape[-1]),
+                        what="out"), len(swapped)
+
+
+def test_compress_matches_oracle():
+    x = synth.nsa_inputs(2, 1000, 16, 2, 192, 128, seed=11)
+    for t, w in ((x.k, x.w_k), (x.v, x.w_v)):
+        got = compress_torch(t.to(DEV), w.to(DEV)).cpu().double()
+        exact = oracle.compress_cache(t, w, 32, 16, round_kc=False)
+        assert got.shape == exact.shape
+        assert ((got - exact).abs() <= exact.abs() * 2 ** -7 + 1e-6).all()
+        assert (got == oracle.round_bf16(exact)).double().mean() > 0.99
+
+
+def test_tiny_workload_full():
+    c = synth.WORKLOADS["nsa_tiny"]
+    x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=0)
+    check_against_oracle(x, c["top_k"], c["window"])
+
+
+@pytest.mark.parametrize("branch", [0, 1, 2])
+def test_tiny_each_branch_alone(branch):
+    c = synth.WORKLOADS["nsa_tiny"]
+    x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=0)
+    gates = synth.one_hot_gates(1, c["T"], c["h_q"], branch)
+    check_against_oracle(x, c["top_k"], c["window"], gates=gates)
+
+
+def test_ragged_multi_group_full():
+    """T not a multiple of the 8-token tile, the 64-token block or the stride;
+    four groups of 16 heads with the 192/128 head dims; batch 2."""
+    x = synth.nsa_inputs(2, 1001, 64, 4, 192, 128, seed=12)
+    check_against_oracle(x, 16, 200)
+
+
+@pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 47, 48, 64, 65])
+def test_short_sequences(T):
+    """No compressed block (T < 32), exactly one, and the first few selection blocks."""
+    x = synth.nsa_inputs(1, T, 16, 1, 192, 128, seed=13)
+    check_against_oracle(x, 16, 512, min_exact=1.0)
+
+
+def test_all_blocks_selected_is_full_attention():
+    """top_k covering every block with only the selection gate on equals full causal attention."""
+    T = 700
+    x = synth.nsa_inputs(1, T, 16, 1, 192, 128, seed=14)
+    gates = synth.one_hot_gates(1, T, 16, 1)
+    out, idx, _, _ = run_gpu(x, T // 64 + 1, 64, gates=gates)
+    assert (idx[0, 0, T - 1] == torch.arange(T // 64 + 1, dtype=torch.int32)).all()
+    G = 16
+    q, k, v = x.q[0].double(), x.k[0].double(), x.v[0].double()
+    kk = k.repeat_interleave(G, dim=1).transpose(0, 1)
+    vv = v.repeat_interleave(G, dim=1).transpose(0, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.transpose(0, 1), kk, vv, is_causal=True).transpose(0, 1)
+    assert_close(out[0], ref, what="full causal")
+
+
+def test_window_of_T_is_full_attention():
+    T = 600
+    x = synth.nsa_inputs(1, T, 16, 1, 192, 128, seed=15)
+    gates = synth.one_hot_gates(1, T, 16, 2)
+    out, _, _, _ = run_gpu(x, 16, T, gates=gates)
+    q, k, v = x.q[0].double(), x.k[0].double(), x.v[0].double()
+    kk = k.repeat_interleave(16, dim=1).transpose(0, 1)
+    vv = v.repeat_interleave(16, dim=1).transpose(0, 1)
+    ref = torch.nn.functional.scaled_dot_product_attention(q.transpose(0, 1), kk, vv, is_causal=True).transpose(0, 1)
+    assert_close(out[0], ref, what="window = T")
+
+
+def test_zero_gates_give_zero():
+    x = synth.nsa_inputs(1, 300, 16, 1, 192, 128, seed=16)
+    out, _, _, _ = run_gpu(x, 16, 128, gates=torch.zeros(1, 300, 16, 3, dtype=torch.bfloat16))
+    assert torch.equal(out, torch.zeros_like(out))
+
+
+def test_deterministic_and_causal():
+    """Two runs are bitwise equal; changing tokens after t leaves rows <= t bitwise unchanged."""
+    T, t0 = 900, 500
+    x = synth.nsa_inputs(1, T, 64, 4, 192, 128, seed=17)
+    a = run_gpu(x, 16, 256)
+    b = run_gpu(x, 16, 256)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    x.k[:, t0 + 1:] = 3.0
+    x.v[:, t0 + 1:] = -2.0
+    c = run_gpu(x, 16, 256)
+    assert torch.equal(a[0][:, : t0 + 1], c[0][:, : t0 + 1])
+    assert torch.equal(a[1][:, :, : t0 + 1], c[1][:, :, : t0 + 1])
+
+
+def sampled_tokens(T, n, seed):
+    g = torch.Generator().manual_seed(seed)
+    fixed = [0, 31, 63, 64, 511, 512, T // 2, T - 1]
+    rnd = torch.randint(0, T, (n,), generator=g).tolist()
+    return sorted(set(t for t in fixed + rnd if t < T))
+
+
+def test_prefill_8k_sampled():
+    c = synth.WORKLOADS["nsa_8k"]
+    x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=0)
+    check_against_oracle(x, c["top_k"], c["window"], tokens=sampled_tokens(c["T"], 120, 1))
+
+
+def test_prefill_64k_sampled():
+    """The 64K workload in the launch configuration the benchmark times."""
+    c = synth.WORKLOADS["nsa_64k"]
+    x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=0)
+    check_against_oracle(x, c["top_k"], c["window"], tokens=sampled_tokens(c["T"], 90, 2))

@@ -64,3 +64,20 @@ def token_mask(shape_bn_h, swapped, G):
     for (b, g, i) in swapped:
         m[b, i, g * G:(g + 1) * G] = False
     return m
+
+
+def assert_phi_close(got, x, w, what="phi"):
+    """GPU phi (fp32 accumulation, one bf16 rounding) against the exact fp64 map:
+    |got - exact| <= 2^-8 |exact| (the rounding) + 2^-17 * (|x| @ |w|) (fp32 accumulation
+    over l*d terms).  Also most entries round to exactly the same bf16 value."""
+    import oracle
+    exact = oracle.compress_cache(x, w, 32, 16, round_kc=False)
+    mag = oracle.compress_cache(x.double().abs(), w.double().abs(), 32, 16, round_kc=False)
+    got = got.detach().cpu().double()
+    assert got.shape == exact.shape, what
+    if exact.numel() == 0:
+        return
+    bad = (got - exact).abs() > exact.abs() * 2 ** -8 + mag * 2 ** -17
+    assert not bad.any(), f"{what}: {int(bad.sum())} entries off"
+    differ = int((got != oracle.round_bf16(exact)).sum())
+    assert differ <= max(8, exact.numel() // 100), f"{what}: {differ} of {exact.numel()} differ after rounding"

@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libnsa.so")
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
 NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
 
-EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_forward", "nsa_decode", "nsa_status_string")
+EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_forward", "nsa_decode", "nsa_forward_noalloc",
+            "nsa_status_string")
 
 
 class NsaConfig(ctypes.Structure):
@@ -65,6 +66,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_forward.restype = ctypes.c_int
     lib.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, cfgp, vp, vp]
     lib.nsa_decode.restype = ctypes.c_int
+    lib.nsa_forward_noalloc.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
+    lib.nsa_forward_noalloc.restype = ctypes.c_int
     lib.nsa_status_string.argtypes = [ctypes.c_int]
     lib.nsa_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -138,3 +141,10 @@ def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, max_seqlen: int
                                    _ptr(seqlens), int(max_seqlen), _ptr(gates), ctypes.byref(cfg), _ptr(out),
                                    _stream(stream, q))
     return _check(st, "nsa_decode") if check else st
+
+
+def nsa_forward_noalloc(q, k, v, gates, cfg: NsaConfig, out, stream=None, check: bool = True) -> int:
+    """nsa_forward with the library's own fixed scratch array instead of cfg.workspace."""
+    st = load_library().nsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), ctypes.byref(cfg), _ptr(out),
+                                            _stream(stream, q))
+    return _check(st, "nsa_forward_noalloc") if check else st

@@ -169,6 +169,34 @@ NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_
                       int32_t max_seqlen, const void* gates, const nsa_config* cfg,
                       void* out, void* stream);
 
+/*
+ * nsa_forward_noalloc -- nsa_forward for callers that cannot allocate device memory.
+ * The pages have no counterpart: this is a library convenience, not part of the method.
+ *
+ * Some callers are handed only their input and output buffers and cannot call
+ * cudaMalloc: a plugin inside a host application that owns every device allocation,
+ * or latency-critical code that must not allocate because cudaMalloc can synchronise
+ * the device.  This entry point computes exactly what nsa_forward computes, with its
+ * scratch in one fixed device array compiled into the library instead of the caller's
+ * workspace (cfg->workspace and cfg->workspace_bytes are ignored).
+ *   - Limit: the scratch array holds 32 MiB (33554432 bytes), and every GPU that loads
+ *     the library keeps it until the process exits.  A problem whose
+ *     nsa_workspace_size(cfg, 0) exceeds it is rejected with NSA_ERR_WORKSPACE before
+ *     anything runs.  32 MiB covers, for example, 1024 tokens with 4 query heads of
+ *     d_v = 64, or about 1000 tokens with 64 query heads of d_v = 128.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before
+ *     any stream capture.
+ *   - It allocates nothing and frees nothing.  Every call shares the one array, which
+ *     keeps the previous call's contents; nothing in it needs to start at zero, since
+ *     each call writes every scratch byte it later reads.  Calls whose execution
+ *     overlaps on the GPU (different streams, or different host threads) race on the
+ *     array: serialise them.
+ * Arguments, layouts and the other status codes are those of nsa_forward.
+ */
+NSA_API nsa_status nsa_forward_noalloc(const void* q, const void* k, const void* v, const void* gates,
+                                       const nsa_config* cfg, void* out, void* stream);
+
 /* Human-readable name of a status code (static storage). */
 NSA_API const char* nsa_status_string(nsa_status s);
 

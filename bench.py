@@ -270,6 +270,11 @@ def run_ours(args, rank, world, local_rank):
     }
     if not args.no_e2e:
         result["e2e"] = run_e2e(args, f, x, out, dev, world)
+    if not args.no_decode:
+        del x, f, out, flush
+        torch.cuda.empty_cache()
+        result["decode"] = run_decode_bench(args, dev, world)
+        result["gpu_launches"] += result["decode"]["gpu_launches"]
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         r, info = oracle_rate(cpu_workload(), args.ref_sample, seed=7, threads=os.cpu_count() or 1)
         result["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
@@ -278,6 +283,67 @@ def run_ours(args, rank, world, local_rank):
                                   **info}
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def decode_bytes(idx, seqlens, h_q, d_k, d_v, window):
+    """Algorithmic HBM bytes of one decode step: for every (sequence, group) the visible
+    compressed keys/values, the union of the chosen blocks' tokens and the window's tokens
+    (each K/V row once), plus q, gates and out."""
+    B, H_kv, k = idx.shape
+    row = (d_k + d_v) * 2
+    total = 0
+    for b in range(B):
+        L = int(seqlens[b])
+        t = L - 1
+        nvis = 0 if L < 32 else (t - 31) // 16 + 1
+        for g in range(H_kv):
+            toks = set(range(max(0, t - window + 1), t + 1))
+            for j in idx[b, g].tolist():
+                if j >= 0:
+                    toks.update(range(64 * j, min(64 * j + 64, t + 1)))
+            total += nvis * row + len(toks) * row
+        total += h_q * (d_k * 2 + 3 * 2 + d_v * 2)
+    return total
+
+
+def run_decode_bench(args, dev, world):
+    """One decode step per sequence of the 32 x 65536 workload; L2 flushed before each step."""
+    import block_sparse_attention_compress_b200 as nsa
+    from block_sparse_attention_compress_b200.torch_ops import compress_torch
+    c = synth.WORKLOADS["nsa_decode"]
+    B, L, hq, hkv, dk, dv = c["B"], c["L"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"]
+    d = synth.decode_inputs(B, L, hq, hkv, dk, dv, seed=0, device=dev)
+    kc, vc = compress_torch(d.k_cache, d.w_k), compress_torch(d.v_cache, d.w_v)
+    idx = torch.empty((B, hkv, c["top_k"]), dtype=torch.int32, device=dev)
+    out = torch.empty((B, hq, dv), dtype=torch.bfloat16, device=dev)
+    cfg = nsa.make_config(batch=B, seqlen=L, h_q=hq, h_kv=hkv, d_k=dk, d_v=dv, top_k=c["top_k"], window=c["window"],
+                          w_cmp_k=d.w_k, w_cmp_v=d.w_v, sel_idx_out=idx)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    step = lambda: nsa.nsa_decode(d.q, d.k_cache, d.v_cache, kc, vc, d.seqlens, L, d.gates, cfg, out)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    mean_ms = allreduce_max(statistics.mean(ms), world, dev)
+    nbytes = decode_bytes(idx.cpu(), d.seqlens.cpu(), hq, dk, dv, c["window"])
+    peaks, src = load_peaks()
+    gbs = nbytes / (mean_ms * 1e-3) / 1e9
+    return {"workload": f"nsa_decode: B={B} sequences x L={L} cache, h_q={hq} h_kv={hkv} d_k={dk} d_v={dv} "
+                        f"top_k={c['top_k']} window={c['window']}, one new token each",
+            "us_per_step": mean_ms * 1e3, "tokens_per_s": world * B / (mean_ms * 1e-3),
+            "bytes_per_step": nbytes, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0, "bound": "hbm",
+            "peak_source": f"{src} hbm_gbs", "gpu_launches": args.steps,
+            "l2": "256 MB flush before every timed step (outside the events)"}
 
 
 def run_e2e(args, f, x, out, dev, world):
@@ -342,6 +408,7 @@ def main():
     ap.add_argument("--ref-sample", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -1,0 +1,512 @@
+// K6: one decode step ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §13: a decode step
+// is bound by the KV bytes it reads; the group-shared choice reads each chosen block
+// once for all of the group's heads).
+//
+// One CTA = one (sequence, KV group); its 8 warps hold the group's G <= 16 query heads
+// as the 16 rows of m16n8k16 tiles.  Everything happens in one launch:
+//   A  warp w streams compressed blocks [512w, 512w+512) through its own two-stage
+//      shared-memory ring (16 blocks = 10 KB per stage): online softmax for o_cmp and,
+//      per head, the running sums of exp(s - m) per 64-token selection block
+//      (rescaled whenever that head's running max grows);
+//   M  the warps' states are merged: per-head log-sum-exp, the group-summed
+//      normalised block scores, top-k (forced blocks first, ties to the lower
+//      index), and o_cmp;
+//   B  the selected blocks (two per warp), then the window (one chunk per warp),
+//      each with its own softmax, merged the same way;
+//   C  out = g_cmp*o_cmp + g_slc*o_slc + g_win*o_win, rounded to bf16.
+// Loads are 16-byte cp.async of whole K/V rows (coalesced, each row 384 + 256 bytes).
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nsa {
+
+namespace {
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRows = 16;            // rows per stage tile
+constexpr int kRange = 512;          // compressed blocks per warp
+constexpr int kJ = kRange / 4 + 1;   // selection blocks touched by one warp's range
+constexpr int kMaxSel = 1024;
+constexpr int kL = 32, kS = 16, kSel = 64;
+
+template <int DK, int DV>
+struct Smem {
+  static constexpr size_t kStage = (size_t)kRows * (DK + DV) * 2;               // one tile (K then V)
+  static constexpr size_t kRing = (size_t)kWarps * 2 * kStage;                   // per-warp double buffer
+  static constexpr size_t kPart = (size_t)kWarps * 16 * kJ * 4;                  // per-warp per-head block sums
+  static constexpr size_t kPersist =
+      ((size_t)(kWarps * 16 * 2 + kWarps * 16 + kMaxSel + 32 + 3 * 16 * DV) * 4 + 127) / 128 * 128;
+  static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (DV + 2) * 4;
+  static constexpr size_t kPhaseB = kPersist + (kRing > kMergeBytes ? kRing : kMergeBytes);
+  static constexpr size_t kTotal = (kRing + kPart) > kPhaseB ? (kRing + kPart) : kPhaseB;
+  static_assert(kTotal <= 232448, "decode shared memory");
+  static_assert(kPersist + kMergeBytes <= kRing, "o_cmp merge must not touch the per-warp block sums");
+};
+
+__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+// Online-softmax state of one warp: rows gl and gl+8 (two heads per lane quad).
+template <int DV>
+struct State {
+  float m0, m1, l0, l1;
+  float o[DV / 8][4];
+  __device__ void init() {
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < DV / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  }
+};
+
+template <int DK, int DV>
+struct Tile {
+  __nv_bfloat16* k;  // [kRows][DK] swizzled
+  __nv_bfloat16* v;  // [kRows][DV] swizzled
+};
+
+// Issue the copies of rows [r0, r0+16) of a K/V source into a stage; rows >= n are zero-filled.
+template <int DK, int DV, class RowK, class RowV>
+__device__ __forceinline__ void load_rows(Tile<DK, DV> st, int r0, int n, RowK rowk, RowV rowv, int lane) {
+  for (int e = lane; e < kRows * (DK / 8); e += 32) {
+    const int r = e / (DK / 8), ch = e % (DK / 8);
+    const bool ok = r0 + r < n;
+    cp_async16(st.k + SwzTile<DK>::offset(r, ch), rowk(ok ? r0 + r : 0) + ch * 8, ok);
+  }
+  for (int e = lane; e < kRows * (DV / 8); e += 32) {
+    const int r = e / (DV / 8), ch = e % (DV / 8);
+    const bool ok = r0 + r < n;
+    cp_async16(st.v + SwzTile<DV>::offset(r, ch), rowv(ok ? r0 + r : 0) + ch * 8, ok);
+  }
+}
+
+// S = Q K^T for one 16-row tile (two n-tiles), already scaled to log2 units.
+template <int DK>
+__device__ __forceinline__ void qk_tile(const uint32_t (&qf)[DK / 16][4], const __nv_bfloat16* k, float (&s)[2][4],
+                                        float scale_log2, int lane) {
+#pragma unroll
+  for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < DK / 16; ++ks) {
+    uint32_t b0, b1, b2, b3;
+    const int row = (lane & 7) + ((lane >> 4) << 3);
+    const int ch = 2 * ks + ((lane >> 3) & 1);
+    ldsm_x4(b0, b1, b2, b3, smem_u32(k + SwzTile<DK>::offset(row, ch)));
+    mma16816(s[0], qf[ks], b0, b1);
+    mma16816(s[1], qf[ks], b2, b3);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[j][e] *= scale_log2;
+}
+
+// O += P V for one 16-row tile; P given as probabilities in the C-fragment layout.
+template <int DV>
+__device__ __forceinline__ void pv_tile(const float (&p)[2][4], const __nv_bfloat16* v, float (&o)[DV / 8][4],
+                                        int lane) {
+  uint32_t a[4];
+  a[0] = pack_bf16(p[0][0], p[0][1]);
+  a[1] = pack_bf16(p[0][2], p[0][3]);
+  a[2] = pack_bf16(p[1][0], p[1][1]);
+  a[3] = pack_bf16(p[1][2], p[1][3]);
+#pragma unroll
+  for (int np = 0; np < DV / 16; ++np) {
+    uint32_t b0, b1, b2, b3;
+    const int row = lane & 15;
+    const int ch = 2 * np + (lane >> 4);
+    ldsm_x4_t(b0, b1, b2, b3, smem_u32(v + SwzTile<DV>::offset(row, ch)));
+    mma16816(o[2 * np], a, b0, b1);
+    mma16816(o[2 * np + 1], a, b2, b3);
+  }
+}
+
+// Online-softmax update of `st` with the masked logits `s` (masked entries are -inf);
+// on return `s` holds exp2(s - m_new).  Returns the per-row rescale factors.
+template <int DV>
+__device__ __forceinline__ void softmax_update(State<DV>& st, float (&s)[2][4], float& c0, float& c1) {
+  float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+  float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+  mx0 = warp_max4(mx0);
+  mx1 = warp_max4(mx1);
+  const float n0 = fmaxf(st.m0, mx0), n1 = fmaxf(st.m1, mx1);
+  const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
+  c0 = exp2f(st.m0 - b0);
+  c1 = exp2f(st.m1 - b1);
+  float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    s[j][0] = exp2f(s[j][0] - b0); s[j][1] = exp2f(s[j][1] - b0);
+    s[j][2] = exp2f(s[j][2] - b1); s[j][3] = exp2f(s[j][3] - b1);
+    sum0 += s[j][0] + s[j][1];
+    sum1 += s[j][2] + s[j][3];
+  }
+  st.l0 = st.l0 * c0 + warp_sum4(sum0);
+  st.l1 = st.l1 * c1 + warp_sum4(sum1);
+  st.m0 = n0;
+  st.m1 = n1;
+#pragma unroll
+  for (int j = 0; j < DV / 8; ++j) {
+    st.o[j][0] *= c0; st.o[j][1] *= c0; st.o[j][2] *= c1; st.o[j][3] *= c1;
+  }
+}
+
+// Stream rows [0, n) of a K/V source through the warp's ring with one softmax.
+template <int DK, int DV, class RowK, class RowV, class Valid>
+__device__ void attend_rows(const uint32_t (&qf)[DK / 16][4], State<DV>& st, Tile<DK, DV> ring0,
+                            Tile<DK, DV> ring1, int n, RowK rowk, RowV rowv, Valid valid, float scale_log2,
+                            int lane) {
+  const int ntiles = (n + kRows - 1) / kRows;
+  if (ntiles == 0) return;
+  load_rows<DK, DV>(ring0, 0, n, rowk, rowv, lane);
+  cp_async_commit();
+  for (int it = 0; it < ntiles; ++it) {
+    if (it + 1 < ntiles) load_rows<DK, DV>((it + 1) & 1 ? ring1 : ring0, (it + 1) * kRows, n, rowk, rowv, lane);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncwarp();
+    const Tile<DK, DV> cur = (it & 1) ? ring1 : ring0;
+    float s[2][4];
+    qk_tile<DK>(qf, cur.k, s, scale_log2, lane);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int r = it * kRows + j * 8 + 2 * (lane & 3) + e;
+        if (!(r < n && valid(r))) { s[j][e] = -INFINITY; s[j][2 + e] = -INFINITY; }
+      }
+    float c0, c1;
+    softmax_update<DV>(st, s, c0, c1);
+    pv_tile<DV>(s, cur.v, st.o, lane);
+    __syncwarp();
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+}
+
+// Merge the 8 warps' states into o (normalised) for rows < G; result in sOut [16][DV].
+// sScratch must hold kWarps*16*DV floats + kWarps*16*2 floats.
+template <int DV>
+__device__ void merge_states(const State<DV>& st, float* sScratch, float* sOut, int G, int warp, int lane) {
+  const int gl = lane >> 2, cq = lane & 3;
+  float* sO = sScratch;
+  float* sML = sScratch + kWarps * 16 * DV;
+  __syncthreads();   // every warp is done with its stage ring, which the scratch overlays
+#pragma unroll
+  for (int j = 0; j < DV / 8; ++j) {
+    sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq] = st.o[j][0];
+    sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq + 1] = st.o[j][1];
+    sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq] = st.o[j][2];
+    sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq + 1] = st.o[j][3];
+  }
+  if (cq == 0) {
+    sML[(warp * 16 + gl) * 2] = st.m0;
+    sML[(warp * 16 + gl) * 2 + 1] = st.l0;
+    sML[(warp * 16 + gl + 8) * 2] = st.m1;
+    sML[(warp * 16 + gl + 8) * 2 + 1] = st.l1;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * DV; e += kThreads) {
+    const int r = e / DV, c = e % DV;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sML[(w * 16 + r) * 2]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float f = exp2f(sML[(w * 16 + r) * 2] - M);
+        L += f * sML[(w * 16 + r) * 2 + 1];
+        O += f * sO[(w * 16 + r) * DV + c];
+      }
+    }
+    sOut[r * DV + c] = L > 0.f ? O / L : 0.f;
+  }
+  __syncthreads();
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kcache,
+              const __nv_bfloat16* __restrict__ vcache, const __nv_bfloat16* __restrict__ kccache,
+              const __nv_bfloat16* __restrict__ vccache, const int32_t* __restrict__ seqlens,
+              const __nv_bfloat16* __restrict__ gates, __nv_bfloat16* __restrict__ out, int32_t* __restrict__ idx_out,
+              int Lmax, int Ncmax, int max_seqlen, int Hq, int Hkv, int G, int top_k, int window, int force_first,
+              int force_local, float scale_log2) {
+  using SM = Smem<DK, DV>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gl = lane >> 2, cq = lane & 3;
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int L = min(max(seqlens[b], 1), max_seqlen);
+  const int t = L - 1;
+  const int nvis = t < kL - 1 ? 0 : min(Ncmax, (t - kL + 1) / kS + 1);
+  const bool rv0 = gl < G, rv1 = gl + 8 < G;
+
+  Tile<DK, DV> ring0{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)warp * 2 * SM::kStage), nullptr};
+  ring0.v = ring0.k + kRows * DK;
+  Tile<DK, DV> ring1{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)warp * 2 * SM::kStage + SM::kStage), nullptr};
+  ring1.v = ring1.k + kRows * DK;
+  float* part = reinterpret_cast<float*>(smem + SM::kRing) + (size_t)warp * 16 * kJ;   // [16][kJ]
+
+  uint32_t qf[DK / 16][4];
+  {
+    const __nv_bfloat16* q0 = q + ((size_t)b * Hq + g * G + gl) * DK;
+    const __nv_bfloat16* q1 = q0 + 8 * DK;
+#pragma unroll
+    for (int ks = 0; ks < DK / 16; ++ks) {
+      qf[ks][0] = rv0 ? ld_u32(q0 + ks * 16 + 2 * cq) : 0u;
+      qf[ks][1] = rv1 ? ld_u32(q1 + ks * 16 + 2 * cq) : 0u;
+      qf[ks][2] = rv0 ? ld_u32(q0 + ks * 16 + 8 + 2 * cq) : 0u;
+      qf[ks][3] = rv1 ? ld_u32(q1 + ks * 16 + 8 + 2 * cq) : 0u;
+    }
+  }
+
+  // ---------------- A: compressed blocks of this warp ----------------
+  for (int e = lane; e < 16 * kJ; e += 32) part[e] = 0.f;
+  __syncwarp();
+  State<DV> st;
+  st.init();
+  const int i_lo = warp * kRange;
+  const int n_a = max(0, min(nvis - i_lo, kRange));
+  {
+    auto rowk = [&](int r) { return kccache + (((size_t)b * Ncmax + i_lo + r) * Hkv + g) * DK; };
+    auto rowv = [&](int r) { return vccache + (((size_t)b * Ncmax + i_lo + r) * Hkv + g) * DV; };
+    const int ntiles = (n_a + kRows - 1) / kRows;
+    if (ntiles > 0) {
+      load_rows<DK, DV>(ring0, 0, n_a, rowk, rowv, lane);
+      cp_async_commit();
+    }
+    for (int it = 0; it < ntiles; ++it) {
+      if (it + 1 < ntiles) load_rows<DK, DV>((it + 1) & 1 ? ring1 : ring0, (it + 1) * kRows, n_a, rowk, rowv, lane);
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncwarp();
+      const Tile<DK, DV> cur = (it & 1) ? ring1 : ring0;
+      float s[2][4];
+      qk_tile<DK>(qf, cur.k, s, scale_log2, lane);
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+          if (it * kRows + j * 8 + 2 * cq + e >= n_a) { s[j][e] = -INFINITY; s[j][2 + e] = -INFINITY; }
+      float c0, c1;
+      softmax_update<DV>(st, s, c0, c1);
+      // rescale this head's block sums when its running max grew (rare after the first tiles)
+      if (rv0 && c0 != 1.f)
+        for (int jj = cq; jj < kJ; jj += 4) part[gl * kJ + jj] *= c0;
+      if (rv1 && c1 != 1.f)
+        for (int jj = cq; jj < kJ; jj += 4) part[(gl + 8) * kJ + jj] *= c1;
+      __syncwarp();
+      // block sums: local compressed index il = 16*it + 8*nt + 2*cq + e goes to selection
+      // block il/4 and, when il % 4 == 3, also to il/4 + 1 (two passes keep lanes apart)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int jb = 4 * it + 2 * nt + (cq >> 1);
+        float a0 = s[nt][0] + s[nt][1], a1 = s[nt][2] + s[nt][3];
+        a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+        if ((cq & 1) == 0) {
+          if (rv0) part[gl * kJ + jb] += a0;
+          if (rv1) part[(gl + 8) * kJ + jb] += a1;
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int jb = 4 * it + 2 * nt + (cq >> 1) + 1;
+        if (cq & 1) {
+          if (rv0) part[gl * kJ + jb] += s[nt][1];
+          if (rv1) part[(gl + 8) * kJ + jb] += s[nt][3];
+        }
+      }
+      pv_tile<DV>(s, cur.v, st.o, lane);
+      __syncwarp();
+    }
+    cp_async_wait<0>();
+  }
+  __syncthreads();
+
+  // ---------------- M: merge, scores, top-k, o_cmp ----------------
+  // Small persistent buffers sit at the bottom (over the dead phase-A rings); above them one
+  // union region serves the cross-warp merges and, in phase B, the stage rings.
+  float* sML = reinterpret_cast<float*>(smem);                         // [8][16][2] m, l
+  float* sCoef = sML + kWarps * 16 * 2;                                // [8][16]
+  float* sScore = sCoef + kWarps * 16;                                 // [kMaxSel]
+  int* sIdx = reinterpret_cast<int*>(sScore + kMaxSel);                // [32]
+  float* sOcmp = reinterpret_cast<float*>(sIdx + 32);                  // [16][DV]
+  float* sOslc = sOcmp + 16 * DV;                                      // [16][DV]
+  float* sOwin = sOslc + 16 * DV;                                      // [16][DV]
+  uint8_t* uni = smem + SM::kPersist;                                  // merge scratch / phase-B rings
+  float* sMerge = reinterpret_cast<float*>(uni);
+  if (cq == 0) {
+    sML[(warp * 16 + gl) * 2] = st.m0;
+    sML[(warp * 16 + gl) * 2 + 1] = st.l0;
+    sML[(warp * 16 + gl + 8) * 2] = st.m1;
+    sML[(warp * 16 + gl + 8) * 2 + 1] = st.l1;
+  }
+  __syncthreads();
+  if (tid < 16) {   // per-head log-sum-exp (log2 units) and each warp's coefficient
+    const int r = tid;
+    float M = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sML[(w * 16 + r) * 2]);
+    float Ls = 0.f;
+    if (M != -INFINITY)
+      for (int w = 0; w < kWarps; ++w) Ls += exp2f(sML[(w * 16 + r) * 2] - M) * sML[(w * 16 + r) * 2 + 1];
+    const float lse = (r < G && Ls > 0.f) ? M + __log2f(Ls) : INFINITY;
+    for (int w = 0; w < kWarps; ++w) sCoef[w * 16 + r] = exp2f(sML[(w * 16 + r) * 2] - lse);
+  }
+  __syncthreads();
+  const int nb = t / kSel + 1;
+  {
+    const float* partAll = reinterpret_cast<const float*>(smem + SM::kRing);
+    for (int J = tid; J < nb; J += kThreads) {
+      const int w = J / (kRange / 4), jj = J - w * (kRange / 4);
+      float sc = 0.f;
+      for (int r = 0; r < G; ++r) {
+        sc += sCoef[w * 16 + r] * partAll[((size_t)w * 16 + r) * kJ + jj];
+        if (jj == 0 && w > 0) sc += sCoef[(w - 1) * 16 + r] * partAll[((size_t)(w - 1) * 16 + r) * kJ + kJ - 1];
+      }
+      sScore[J] = sc;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {   // top-k over the nb eligible blocks
+    if (nb <= top_k) {
+      for (int j = lane; j < top_k; j += 32) sIdx[j] = j < nb ? j : -1;
+    } else {
+      const int own = t / kSel;
+      uint32_t taken = 0;
+      int nforced = 0;
+      if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
+      if (force_local && !(force_first && own == 0)) {
+        if (lane == (own & 31)) taken |= 1u << (own >> 5);
+        ++nforced;
+      }
+      const int mmax = (nb + 31) >> 5;
+      for (int r = nforced; r < top_k; ++r) {
+        float bs = -FLT_MAX;
+        int bj = 0x7fffffff;
+        for (int m = 0; m < mmax; ++m) {
+          const int j = lane + 32 * m;
+          if (j < nb && !((taken >> m) & 1u)) {
+            const float sc = sScore[j];
+            if (sc > bs) { bs = sc; bj = j; }
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+          const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+          if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; }
+        }
+        if (bj != 0x7fffffff && lane == (bj & 31)) taken |= 1u << (bj >> 5);
+      }
+      int pos = 0;
+      for (int m = 0; m < mmax; ++m) {
+        const bool sel = (taken >> m) & 1u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+        if (sel) sIdx[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * m;
+        pos += __popc(bal);
+      }
+      for (int j = pos + lane; j < top_k; j += 32) sIdx[j] = -1;
+    }
+  }
+  __syncthreads();
+  if (idx_out)
+    for (int j = tid; j < top_k; j += kThreads) idx_out[((size_t)b * Hkv + g) * top_k + j] = sIdx[j];
+  // o_cmp: each warp's o scaled by its coefficient, summed over warps
+  {
+    float* sO = sMerge;
+#pragma unroll
+    for (int j = 0; j < DV / 8; ++j) {
+      const float f0 = sCoef[warp * 16 + gl], f1 = sCoef[warp * 16 + gl + 8];
+      sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq] = st.o[j][0] * f0;
+      sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq + 1] = st.o[j][1] * f0;
+      sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq] = st.o[j][2] * f1;
+      sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq + 1] = st.o[j][3] * f1;
+    }
+    __syncthreads();
+    for (int e = tid; e < 16 * DV; e += kThreads) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) acc += sO[w * 16 * DV + e];
+      sOcmp[e] = acc;
+    }
+    __syncthreads();
+  }
+
+  // ---------------- B: selected blocks, then the window ----------------
+  Tile<DK, DV> rb0{reinterpret_cast<__nv_bfloat16*>(uni + (size_t)warp * 2 * SM::kStage), nullptr};
+  rb0.v = rb0.k + kRows * DK;
+  Tile<DK, DV> rb1{reinterpret_cast<__nv_bfloat16*>(uni + (size_t)warp * 2 * SM::kStage + SM::kStage), nullptr};
+  rb1.v = rb1.k + kRows * DK;
+  const int own = t / kSel;
+  {
+    // warp w takes the chosen blocks at positions 2w and 2w+1 (and more when top_k > 16)
+    st.init();
+    for (int p = warp; p < top_k; p += kWarps) {
+      const int j = sIdx[p];
+      if (j < 0) continue;
+      const int jb = min(j, own);
+      const int u0 = jb * kSel;
+      const int n = min(kSel, t - u0 + 1);
+      auto rowk = [&](int r) { return kcache + (((size_t)b * Lmax + u0 + r) * Hkv + g) * DK; };
+      auto rowv = [&](int r) { return vcache + (((size_t)b * Lmax + u0 + r) * Hkv + g) * DV; };
+      attend_rows<DK, DV>(qf, st, rb0, rb1, n, rowk, rowv, [](int) { return true; }, scale_log2, lane);
+    }
+    merge_states<DV>(st, sMerge, sOslc, G, warp, lane);
+  }
+  {
+    st.init();
+    const int lo = max(0, t - window + 1);
+    const int nwin = t - lo + 1;
+    const int chunk = (nwin + kWarps - 1) / kWarps;
+    const int r0 = min(nwin, warp * chunk);
+    const int n = min(nwin, r0 + chunk) - r0;
+    auto rowk = [&](int r) { return kcache + (((size_t)b * Lmax + lo + r0 + r) * Hkv + g) * DK; };
+    auto rowv = [&](int r) { return vcache + (((size_t)b * Lmax + lo + r0 + r) * Hkv + g) * DV; };
+    attend_rows<DK, DV>(qf, st, rb0, rb1, n, rowk, rowv, [](int) { return true; }, scale_log2, lane);
+    merge_states<DV>(st, sMerge, sOwin, G, warp, lane);
+  }
+
+  // ---------------- C: gated combine ----------------
+  for (int e = tid; e < G * DV; e += kThreads) {
+    const int r = e / DV, c = e % DV;
+    const size_t row = (size_t)b * Hq + g * G + r;
+    const float g0 = __bfloat162float(gates[row * 3]), g1 = __bfloat162float(gates[row * 3 + 1]),
+                g2 = __bfloat162float(gates[row * 3 + 2]);
+    out[row * DV + c] = __float2bfloat16_rn(g0 * sOcmp[e] + g1 * sOslc[e] + g2 * sOwin[e]);
+  }
+}
+
+template <int DK, int DV>
+cudaError_t launch(const DecodeArgs& a, cudaStream_t st) {
+  const size_t smem = Smem<DK, DV>::kTotal;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid(a.Hkv, a.B);
+  decode_kernel<DK, DV><<<grid, kThreads, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.kc),
+      static_cast<const __nv_bfloat16*>(a.vc), a.seqlens, static_cast<const __nv_bfloat16*>(a.gates),
+      static_cast<__nv_bfloat16*>(a.out), a.idx, a.Lmax, a.Ncmax, a.max_seqlen, a.Hq, a.Hkv, a.G, a.top_k, a.window,
+      a.force_first, a.force_local, a.scale_log2);
+  return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st) {
+  if (a.dk == 64 && a.dv == 64) return launch<64, 64>(a, st);
+  if (a.dk == 128 && a.dv == 128) return launch<128, 128>(a, st);
+  if (a.dk == 192 && a.dv == 128) return launch<192, 128>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nsa

@@ -35,4 +35,22 @@ cudaError_t launch_slc_attn(const FwdArgs& a, cudaStream_t st);
 // K4 + K5: sliding window and gated combine (out = bf16(acc + g_win * o_win)).
 cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st);
 
+struct DecodeArgs {
+  const void* q;        // [B, Hq, dk]
+  const void* k;        // [B, Lmax, Hkv, dk]
+  const void* v;        // [B, Lmax, Hkv, dv]
+  const void* kc;       // [B, Ncmax, Hkv, dk]
+  const void* vc;       // [B, Ncmax, Hkv, dv]
+  const int32_t* seqlens;
+  const void* gates;    // [B, Hq, 3]
+  void* out;            // [B, Hq, dv]
+  int32_t* idx;         // [B, Hkv, top_k] or null
+  int B, Lmax, Ncmax, max_seqlen, Hq, Hkv, G, dk, dv;
+  int top_k, window, force_first, force_local;
+  float scale_log2;
+};
+
+// K6: one decode step per sequence, all branches in one launch.
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
+
 }  // namespace nsa

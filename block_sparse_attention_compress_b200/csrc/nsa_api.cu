@@ -106,7 +106,7 @@ const char* nsa_status_string(nsa_status s) {
 size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch) {
   if (check_cfg(cfg) != NSA_OK || decode_batch < 0) return 0;
   if (decode_batch == 0) return forward_layout(cfg).total;
-  return 0;
+  return 0;   // nsa_decode keeps everything on chip
 }
 
 nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t T, int32_t H, int32_t d, int32_t d_out,
@@ -168,9 +168,27 @@ nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache, c
                       const nsa_config* cfg, void* out, void* stream) {
   nsa_status st = check_cfg(cfg);
   if (st != NSA_OK) return st;
-  (void)q; (void)k_cache; (void)v_cache; (void)kc_cache; (void)vc_cache; (void)seqlens; (void)max_seqlen;
-  (void)gates; (void)out; (void)stream;
-  return NSA_ERR_UNSUPPORTED;
+  if (cfg->mode != NSA_MODE_NSA) return NSA_ERR_UNSUPPORTED;
+  if (!q || !k_cache || !v_cache || !kc_cache || !vc_cache || !seqlens || !gates || !out) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(kc_cache) || !aligned16(vc_cache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(gates) & 1u))
+    return NSA_ERR_INVALID_ARG;
+  if (max_seqlen < 1 || max_seqlen > cfg->seqlen) return NSA_ERR_INVALID_ARG;
+  nsa::DecodeArgs a{};
+  a.q = q; a.k = k_cache; a.v = v_cache; a.kc = kc_cache; a.vc = vc_cache; a.seqlens = seqlens;
+  a.gates = gates; a.out = out; a.idx = cfg->sel_idx_out;
+  a.B = cfg->batch; a.Lmax = cfg->seqlen; a.Ncmax = n_cmp(cfg->seqlen, cfg->cmp_block, cfg->cmp_stride);
+  a.max_seqlen = max_seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
+  a.dk = cfg->d_k; a.dv = cfg->d_v; a.top_k = cfg->top_k; a.window = cfg->window;
+  a.force_first = cfg->force_first; a.force_local = cfg->force_local;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  StageMarks marks(cfg, 1);
+  cudaError_t e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_decode(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  return from_cuda(e);
 }
 
 }  // extern "C"

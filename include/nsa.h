@@ -108,8 +108,8 @@ typedef struct {
   int32_t n_stage_events;
 } nsa_config;
 
-/* Bytes of workspace nsa_forward (decode_batch == 0) or nsa_decode
- * (decode_batch == number of sequences) needs for `cfg`; 0 if cfg is invalid. */
+/* Bytes of workspace nsa_forward (decode_batch == 0) needs for `cfg`; 0 if cfg is invalid.
+ * nsa_decode (decode_batch > 0) needs none: the result is 0 and its workspace fields are ignored. */
 NSA_API size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch);
 
 /*
@@ -159,10 +159,14 @@ NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, cons
  *   kc_cache  bf16 [B, N_c(L_max), H_kv, d_k], vc_cache [.., d_v]: phi of the caches
  *             (nsa_compress); only the first N_c(seqlens[b]) rows are read.
  *   seqlens   int32 [B] device: tokens in sequence b's cache including the new one
- *             (1 <= seqlens[b] <= L_max); the query sits at position seqlens[b]-1.
- *   max_seqlen an upper bound of seqlens (host), <= cfg->seqlen.
+ *             (1 <= seqlens[b] <= max_seqlen); the query sits at position seqlens[b]-1.
+ *             Values outside that range are clamped into it on the device.
+ *   max_seqlen an upper bound of seqlens (host), 1 <= max_seqlen <= cfg->seqlen <= 65536.
  *   gates     bf16 [B, H_q, 3];  out bf16 [B, H_q, d_v].
  * cfg->batch = B, cfg->seqlen = L_max; sel_idx_out (optional) is [B, H_kv, top_k].
+ * One launch (stage_events: 1 kernel): per (sequence, KV head), compressed attention with
+ * the group-summed block scores and top-k, then the selected blocks and the window,
+ * then the gated sum -- the same arithmetic as the last row of nsa_forward.
  */
 NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache,
                       const void* kc_cache, const void* vc_cache, const int32_t* seqlens,

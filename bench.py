@@ -63,6 +63,17 @@ def nsa_flops(T, h_q, h_kv, d_k, d_v, top_k, window, B=1):
             "slc_attn": float(slc.sum()) * per_pair, "swa_combine": float(win.sum()) * per_pair}
 
 
+def moba_flops(T, H, d, block, top_k, B=1):
+    """MoBA: 2*(q.k + p.v pairs)*d over the chosen past blocks and the causal own block, plus the
+    unscaled q . mean-key scores over every complete past block."""
+    t = torch.arange(T, dtype=torch.float64)
+    J = torch.div(t, block, rounding_mode="floor")
+    pairs = torch.clamp(J, max=top_k) * block + torch.remainder(t, block) + 1
+    attn = float(pairs.sum()) * 2.0 * (2 * d) * H * B
+    score = float(J.sum()) * 2.0 * d * H * B
+    return attn, score
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -275,6 +286,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         result["decode"] = run_decode_bench(args, dev, world)
         result["gpu_launches"] += result["decode"]["gpu_launches"]
+    if not args.no_moba:
+        torch.cuda.empty_cache()
+        result["moba"] = run_moba_bench(args, dev, world)
+        result["gpu_launches"] += result["moba"]["gpu_launches"]
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         r, info = oracle_rate(cpu_workload(), args.ref_sample, seed=7, threads=os.cpu_count() or 1)
         result["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
@@ -346,6 +361,49 @@ def run_decode_bench(args, dev, world):
             "l2": "256 MB flush before every timed step (outside the events)"}
 
 
+def run_moba_bench(args, dev, world):
+    """MoBA forward of the 128K-token, 32-head workload (stage times from the library's events)."""
+    import block_sparse_attention_compress_b200 as nsa
+    c = synth.WORKLOADS["moba_128k"]
+    B, T, H, d = 1, c["T"], c["h"], c["d"]
+    x = synth.moba_inputs(B, T, H, d, seed=0, device=dev)
+    out = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
+    cfg = nsa.make_config(mode=nsa.NSA_MODE_MOBA, batch=B, seqlen=T, h_q=H, h_kv=H, d_k=d, d_v=d,
+                          sel_block=c["block"], top_k=c["top_k"])
+    ws = torch.empty(nsa.nsa_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    names = ["block_means", "select", "lists", "past_attn", "own_merge"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    for es in evs:
+        for e in es:
+            e.record()
+    torch.cuda.synchronize()
+    handles = [ctypes_array(es) for es in evs]
+    for _ in range(args.warmup):
+        flush.zero_()
+        cfg.stage_events, cfg.n_stage_events = None, 0
+        nsa.nsa_forward(x.q, x.k, x.v, None, cfg, out)
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        cfg.stage_events, cfg.n_stage_events = handles[i][0], len(names) + 1
+        nsa.nsa_forward(x.q, x.k, x.v, None, cfg, out)
+    torch.cuda.synchronize()
+    step_ms = statistics.mean(es[0].elapsed_time(es[-1]) for es in evs)
+    stages = {n: statistics.mean(es[j].elapsed_time(es[j + 1]) for es in evs) for j, n in enumerate(names)}
+    ms = allreduce_max(step_ms, world, dev)
+    attn, score = moba_flops(T, H, d, c["block"], c["top_k"], B)
+    peaks, src = load_peaks()
+    return {"workload": f"moba_128k: B=1 T={T} heads={H} d={d} block={c['block']} top_k={c['top_k']} + own block",
+            "ms_per_step": ms, "tokens_per_s": world * B * T / (ms * 1e-3),
+            "tflops_computed": (attn + score) / (ms * 1e-3) / 1e12,
+            "frac_of_bf16_peak": (attn + score) / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "stages_ms": {n: round(v, 4) for n, v in stages.items()},
+            "gpu_launches": 6 * args.steps}
+
+
 def run_e2e(args, f, x, out, dev, world):
     """Same step through the public API with inputs in pinned host memory: H2D copies of
     q, k, v, gates, the forward, and the D2H copy of the output, all inside the timed region."""
@@ -409,6 +467,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-moba", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -53,4 +53,27 @@ struct DecodeArgs {
 // K6: one decode step per sequence, all branches in one launch.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
+struct MobaLayout {
+  size_t kbar, idx, counts, offsets, chunks, fill, list, part_lse, part_o, total;
+};
+// Workspace carve-up of MoBA mode (each region 256-byte aligned).
+MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k);
+
+struct MobaArgs {
+  const void* q;        // [B, T, H, 128]
+  const void* k;
+  const void* v;
+  void* out;            // [B, T, H, 128]
+  int32_t* idx;         // [B, H, T, top_k + 1] or null (then kept in the workspace)
+  void* workspace;      // moba_layout(...).total bytes
+  int B, T, H, bsz, top_k;
+  float scale_log2;
+  cudaError_t (*mark)(void*, cudaStream_t);   // optional stage marker (measurement events)
+  void* mark_ctx;
+};
+
+// MoBA mode: block means, selection, per-block query lists, past-block attention,
+// own-block attention + merge.
+cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st);
+
 }  // namespace nsa

@@ -1,0 +1,562 @@
+// MoBA mode ("一文比较 Kimi 和 Deepseek 的两篇稀疏注意力机制论文", "Kimi 的论文核心点": every
+// query attends to its own block with a causal staircase and to the past blocks whose
+// mean-pooled key scores highest against it; "逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文"
+// §16-§17: mean pooling, no parameters, every head chooses for itself, 512-token blocks,
+// top 3; the queries that chose one KV block are gathered so the block is read once).
+//
+// Five launches on the caller's stream:
+//   M1 block means      kbar[b, j, h, :] = mean of the keys of block j (fp32);
+//   M2 select           per 64-token tile and head: score_j = q . kbar_j for the past blocks
+//                       (kbar split into two bf16 halves so the tensor-core dot product keeps
+//                       fp32 accuracy), running top-k per row, idx = [past ascending.., own];
+//                       counts the queries that chose each (b, h, j);
+//   M3 lists            one CTA: exclusive scans of the counts (list offsets, 64-query chunks);
+//                       then every choice is scattered into its (b, h, j) list as t*8 + slot;
+//   M4 past attention   persistent CTAs walk the 64-query chunks: gather the chunk's queries,
+//                       stream block j's 512 keys (no mask: every key is in the past), write
+//                       per-query normalised o (bf16) and its log-sum-exp per slot;
+//   M5 own + merge      per 64-token tile and head: causal attention inside the own block,
+//                       then the partials of the past slots are merged in; out in bf16.
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nsa {
+
+namespace {
+constexpr int D = 128;            // head dim of this mode
+constexpr int kQ = 64;            // queries per tile / chunk (4 warps x 16 rows)
+constexpr int kThreads = 128;
+constexpr int kKT = 64;           // keys per shared-memory tile
+constexpr int kMaxK = 7;          // past blocks per query
+
+__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+__device__ __forceinline__ void load_q_frag(uint32_t (&qf)[D / 16][4], const __nv_bfloat16* q0, const __nv_bfloat16* q1,
+                                            bool r0, bool r1, int cq) {
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks) {
+    qf[ks][0] = r0 ? ld_u32(q0 + ks * 16 + 2 * cq) : 0u;
+    qf[ks][1] = r1 ? ld_u32(q1 + ks * 16 + 2 * cq) : 0u;
+    qf[ks][2] = r0 ? ld_u32(q0 + ks * 16 + 8 + 2 * cq) : 0u;
+    qf[ks][3] = r1 ? ld_u32(q1 + ks * 16 + 8 + 2 * cq) : 0u;
+  }
+}
+
+// S (16 x 64) += Q K^T from a swizzled [64][D] bf16 tile.
+__device__ __forceinline__ void qk64(const uint32_t (&qf)[D / 16][4], const __nv_bfloat16* k, float (&s)[8][4],
+                                     int lane) {
+#pragma unroll
+  for (int ks = 0; ks < D / 16; ++ks)
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      uint32_t b0, b1, b2, b3;
+      const int row = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+      const int ch = 2 * ks + ((lane >> 3) & 1);
+      ldsm_x4(b0, b1, b2, b3, smem_u32(k + SwzTile<D>::offset(row, ch)));
+      mma16816(s[2 * np], qf[ks], b0, b1);
+      mma16816(s[2 * np + 1], qf[ks], b2, b3);
+    }
+}
+
+// O (16 x D) += P V with P (16 x 64) in C-fragment layout.
+__device__ __forceinline__ void pv64(const float (&p)[8][4], const __nv_bfloat16* v, float (&o)[D / 8][4], int lane) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    uint32_t a[4];
+    a[0] = pack_bf16(p[2 * kk][0], p[2 * kk][1]);
+    a[1] = pack_bf16(p[2 * kk][2], p[2 * kk][3]);
+    a[2] = pack_bf16(p[2 * kk + 1][0], p[2 * kk + 1][1]);
+    a[3] = pack_bf16(p[2 * kk + 1][2], p[2 * kk + 1][3]);
+#pragma unroll
+    for (int np = 0; np < D / 16; ++np) {
+      uint32_t b0, b1, b2, b3;
+      const int row = kk * 16 + (lane & 15);
+      const int ch = 2 * np + (lane >> 4);
+      ldsm_x4_t(b0, b1, b2, b3, smem_u32(v + SwzTile<D>::offset(row, ch)));
+      mma16816(o[2 * np], a, b0, b1);
+      mma16816(o[2 * np + 1], a, b2, b3);
+    }
+  }
+}
+
+// One online-softmax step for rows (gl, gl+8) with masked logits (-inf) already in log2 units.
+__device__ __forceinline__ void online(float (&s)[8][4], float& m0, float& m1, float& l0, float& l1,
+                                       float (&o)[D / 8][4]) {
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    mx0 = fmaxf(mx0, fmaxf(s[j][0], s[j][1]));
+    mx1 = fmaxf(mx1, fmaxf(s[j][2], s[j][3]));
+  }
+  mx0 = warp_max4(mx0);
+  mx1 = warp_max4(mx1);
+  const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+  const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
+  const float c0 = exp2f(m0 - b0), c1 = exp2f(m1 - b1);
+  float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    s[j][0] = exp2f(s[j][0] - b0); s[j][1] = exp2f(s[j][1] - b0);
+    s[j][2] = exp2f(s[j][2] - b1); s[j][3] = exp2f(s[j][3] - b1);
+    sum0 += s[j][0] + s[j][1];
+    sum1 += s[j][2] + s[j][3];
+  }
+  l0 = l0 * c0 + warp_sum4(sum0);
+  l1 = l1 * c1 + warp_sum4(sum1);
+  m0 = n0;
+  m1 = n1;
+#pragma unroll
+  for (int j = 0; j < D / 8; ++j) {
+    o[j][0] *= c0; o[j][1] *= c0; o[j][2] *= c1; o[j][3] *= c1;
+  }
+}
+
+// ------------------------------------------------------------------ M1
+__global__ void __launch_bounds__(D) moba_mean_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ kbar,
+                                                      int T, int H, int bsz, int nblk) {
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, c = threadIdx.x;
+  const int u0 = j * bsz, u1 = min(T, u0 + bsz);
+  float acc = 0.f;
+  for (int u = u0; u < u1; ++u) acc += __bfloat162float(k[(((size_t)b * T + u) * H + h) * D + c]);
+  kbar[(((size_t)b * nblk + j) * H + h) * D + c] = acc / (float)(u1 - u0);
+}
+
+// ------------------------------------------------------------------ M2
+// Keeps the k best (score desc, index asc) of the values offered to it.
+struct TopK {
+  float v[kMaxK];
+  int j[kMaxK];
+  __device__ void init() {
+#pragma unroll
+    for (int i = 0; i < kMaxK; ++i) { v[i] = -FLT_MAX; j[i] = 0x7fffffff; }
+  }
+  __device__ static bool better(float a, int ja, float b, int jb) { return a > b || (a == b && ja < jb); }
+  __device__ void offer(float val, int idx, int k) {   // list sorted best-first in [0, k), 1 <= k <= kMaxK
+    if (!better(val, idx, v[k - 1], j[k - 1])) return;
+    int p = k - 1;
+    while (p > 0 && better(val, idx, v[p - 1], j[p - 1])) {
+      v[p] = v[p - 1];
+      j[p] = j[p - 1];
+      --p;
+    }
+    v[p] = val;
+    j[p] = idx;
+  }
+};
+
+__global__ void __launch_bounds__(kThreads) moba_select_kernel(
+    const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar, int32_t* __restrict__ idx,
+    int32_t* __restrict__ counts, int T, int H, int bsz, int nblk, int top_k) {
+  __shared__ __align__(128) __nv_bfloat16 sHi[kKT * D];
+  __shared__ __align__(128) __nv_bfloat16 sLo[kKT * D];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
+  const int t0 = blockIdx.x * kQ, h = blockIdx.y, b = blockIdx.z;
+  const int J = t0 / bsz;                      // own block, the same for the whole tile (bsz % 64 == 0)
+  const int ta = t0 + warp * 16 + gl, tb = ta + 8;
+  uint32_t qf[D / 16][4];
+  load_q_frag(qf, q + (((size_t)b * T + min(ta, T - 1)) * H + h) * D, q + (((size_t)b * T + min(tb, T - 1)) * H + h) * D,
+              ta < T, tb < T, cq);
+  TopK k0, k1;
+  k0.init();
+  k1.init();
+  const int kk = min(top_k, J);
+  if (J > top_k && top_k > 0) {
+    for (int j0 = 0; j0 < J; j0 += kKT) {
+      __syncthreads();
+      for (int e = tid; e < kKT * (D / 8); e += kThreads) {   // fp32 means -> bf16 hi + bf16 lo
+        const int r = e / (D / 8), ch = e % (D / 8);
+        const int j = j0 + r;
+        float x[8];
+        if (j < J) {
+          const float4* src = reinterpret_cast<const float4*>(kbar + (((size_t)b * nblk + j) * H + h) * D + ch * 8);
+          const float4 a = src[0], c = src[1];
+          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = 0.f;
+        }
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+          const float2 hf = __bfloat1622float2(h2);
+          hi[i] = *reinterpret_cast<const uint32_t*>(&h2);
+          lo[i] = pack_bf16(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+        }
+        *reinterpret_cast<uint4*>(sHi + SwzTile<D>::offset(r, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(sLo + SwzTile<D>::offset(r, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      __syncthreads();
+      float s[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+      qk64(qf, sHi, s, lane);
+      qk64(qf, sLo, s, lane);
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = j0 + nt * 8 + 2 * cq + e;
+          if (j < J) {
+            k0.offer(s[nt][e], j, kk);
+            k1.offer(s[nt][2 + e], j, kk);
+          }
+        }
+    }
+  }
+  // merge the quad's four lists: kk rounds of a quad-wide argmax
+  int sel0[kMaxK + 1], sel1[kMaxK + 1];
+  if (J <= top_k) {
+    for (int i = 0; i < kk; ++i) sel0[i] = sel1[i] = i;
+  } else if (kk > 0) {
+    int p0 = 0, p1 = 0;
+    for (int r = 0; r < kk; ++r) {
+      float bv0 = p0 < kk ? k0.v[p0] : -FLT_MAX, bv1 = p1 < kk ? k1.v[p1] : -FLT_MAX;
+      int bj0 = p0 < kk ? k0.j[p0] : 0x7fffffff, bj1 = p1 < kk ? k1.j[p1] : 0x7fffffff;
+#pragma unroll
+      for (int off = 1; off < 4; off <<= 1) {
+        const float ov0 = __shfl_xor_sync(0xffffffffu, bv0, off), ov1 = __shfl_xor_sync(0xffffffffu, bv1, off);
+        const int oj0 = __shfl_xor_sync(0xffffffffu, bj0, off), oj1 = __shfl_xor_sync(0xffffffffu, bj1, off);
+        if (TopK::better(ov0, oj0, bv0, bj0)) { bv0 = ov0; bj0 = oj0; }
+        if (TopK::better(ov1, oj1, bv1, bj1)) { bv1 = ov1; bj1 = oj1; }
+      }
+      sel0[r] = bj0;
+      sel1[r] = bj1;
+      if (p0 < kk && k0.j[p0] == bj0) ++p0;   // indices are unique across the quad's lanes
+      if (p1 < kk && k1.j[p1] == bj1) ++p1;
+    }
+  }
+  // ascending order (kk <= 7)
+  for (int a = 1; a < kk; ++a)
+    for (int c = a; c > 0 && sel0[c - 1] > sel0[c]; --c) { const int x = sel0[c]; sel0[c] = sel0[c - 1]; sel0[c - 1] = x; }
+  for (int a = 1; a < kk; ++a)
+    for (int c = a; c > 0 && sel1[c - 1] > sel1[c]; --c) { const int x = sel1[c]; sel1[c] = sel1[c - 1]; sel1[c - 1] = x; }
+  if (cq == 0) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int t = half ? tb : ta;
+      if (t >= T) continue;
+      const int* sel = half ? sel1 : sel0;
+      int32_t* dst = idx + (((size_t)b * H + h) * T + t) * (top_k + 1);
+      for (int i = 0; i < kk; ++i) {
+        dst[i] = sel[i];
+        atomicAdd(&counts[((size_t)b * H + h) * nblk + sel[i]], 1);
+      }
+      dst[kk] = J;
+      for (int i = kk + 1; i <= top_k; ++i) dst[i] = -1;
+    }
+  }
+}
+
+// ------------------------------------------------------------------ M3
+// Exclusive scans over all (b, h, j): list offsets and 64-query chunk starts (one CTA).
+__global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets, int32_t* __restrict__ chunks,
+                                                         int32_t* __restrict__ fill, int E) {
+  __shared__ int32_t s0[1024], s1[1024];
+  __shared__ int32_t carry0, carry1;
+  if (threadIdx.x == 0) { carry0 = 0; carry1 = 0; }
+  __syncthreads();
+  for (int base = 0; base < E; base += 1024) {
+    const int e = base + threadIdx.x;
+    const int c = e < E ? counts[e] : 0;
+    s0[threadIdx.x] = c;
+    s1[threadIdx.x] = (c + kQ - 1) / kQ;
+    __syncthreads();
+    for (int off = 1; off < 1024; off <<= 1) {   // Hillis-Steele inclusive scan
+      const int a0 = threadIdx.x >= off ? s0[threadIdx.x - off] : 0;
+      const int a1 = threadIdx.x >= off ? s1[threadIdx.x - off] : 0;
+      __syncthreads();
+      s0[threadIdx.x] += a0;
+      s1[threadIdx.x] += a1;
+      __syncthreads();
+    }
+    if (e < E) {
+      offsets[e] = carry0 + s0[threadIdx.x] - c;
+      chunks[e] = carry1 + s1[threadIdx.x] - (c + kQ - 1) / kQ;
+      fill[e] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 1023) { carry0 += s0[1023]; carry1 += s1[1023]; }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) { offsets[E] = carry0; chunks[E] = carry1; }
+}
+
+__global__ void moba_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ offsets,
+                                    int32_t* __restrict__ fill, int32_t* __restrict__ list, int T, int H, int nblk,
+                                    int top_k, int bsz) {
+  const size_t n = (size_t)gridDim.y * T;   // (b*H + h) rows of T tokens
+  const int bh = blockIdx.y;
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+    const int32_t* row = idx + ((size_t)bh * T + t) * (top_k + 1);
+    const int own = t / bsz;
+    for (int s = 0; s < top_k; ++s) {
+      const int j = row[s];
+      if (j < 0 || j >= own) break;
+      const size_t e = (size_t)bh * nblk + j;
+      const int pos = offsets[e] + atomicAdd(&fill[e], 1);
+      list[pos] = t * 8 + s;
+    }
+  }
+  (void)n;
+}
+
+// ------------------------------------------------------------------ M4
+__global__ void __launch_bounds__(kThreads) moba_past_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, const int32_t* __restrict__ chunks,
+    const int32_t* __restrict__ list, __nv_bfloat16* __restrict__ part_o, float* __restrict__ part_lse, int T, int H,
+    int nblk, int bsz, int top_k, int E, float scale_log2) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);             // [2][64][D]
+  __nv_bfloat16* sV = sK + 2 * kKT * D;                                    // [2][64][D]
+  __shared__ int32_t sList[kQ];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
+  const int total = chunks[E];
+  for (int c = blockIdx.x; c < total; c += gridDim.x) {
+    // (b, h, j) whose chunk range holds c: last e with chunks[e] <= c (binary search)
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (chunks[mid] <= c) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int bh = e / nblk, j = e % nblk, b = bh / H, h = bh % H;
+    const int first = (c - chunks[e]) * kQ;
+    const int nq = min(kQ, counts[e] - first);
+    __syncthreads();
+    if (tid < kQ) sList[tid] = tid < nq ? list[offsets[e] + first + tid] : -1;
+    __syncthreads();
+    const int ea = sList[warp * 16 + gl], eb = sList[warp * 16 + gl + 8];
+    const int ta = ea >> 3, tb = eb >> 3;
+    uint32_t qf[D / 16][4];
+    load_q_frag(qf, q + (((size_t)b * T + (ea >= 0 ? ta : 0)) * H + h) * D,
+                q + (((size_t)b * T + (eb >= 0 ? tb : 0)) * H + h) * D, ea >= 0, eb >= 0, cq);
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    const int u0 = j * bsz;
+    const int ntiles = bsz / kKT;
+    auto load = [&](int it, int buf) {
+      for (int x = tid; x < kKT * (D / 8); x += kThreads) {
+        const int r = x / (D / 8), ch = x % (D / 8);
+        const size_t row = ((size_t)b * T + u0 + it * kKT + r) * H + h;
+        cp_async16(sK + buf * kKT * D + SwzTile<D>::offset(r, ch), k + row * D + ch * 8, true);
+        cp_async16(sV + buf * kKT * D + SwzTile<D>::offset(r, ch), v + row * D + ch * 8, true);
+      }
+    };
+    load(0, 0);
+    cp_async_commit();
+    for (int it = 0; it < ntiles; ++it) {
+      if (it + 1 < ntiles) load(it + 1, (it + 1) & 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncthreads();
+      float s[8][4];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+      qk64(qf, sK + (it & 1) * kKT * D, s, lane);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int x = 0; x < 4; ++x) s[i][x] *= scale_log2;
+      online(s, m0, m1, l0, l1, o);
+      pv64(s, sV + (it & 1) * kKT * D, o, lane);
+      __syncthreads();
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int ent = half ? eb : ea;
+      if (ent < 0) continue;
+      const int t = ent >> 3, slot = ent & 7;
+      const float l = half ? l1 : l0, m = half ? m1 : m0;
+      const float inv = 1.f / l;
+      const size_t base = (((size_t)b * T + t) * H + h) * top_k + slot;
+      __nv_bfloat16* dst = part_o + base * D;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i)
+        *reinterpret_cast<uint32_t*>(dst + i * 8 + 2 * cq) =
+            pack_bf16(o[i][2 * half] * inv, o[i][2 * half + 1] * inv);
+      if (cq == 0) part_lse[base] = m + __log2f(l);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ M5
+__global__ void __launch_bounds__(kThreads) moba_own_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    const int32_t* __restrict__ idx, const __nv_bfloat16* __restrict__ part_o, const float* __restrict__ part_lse,
+    __nv_bfloat16* __restrict__ out, int T, int H, int bsz, int top_k, float scale_log2) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* sV = sK + 2 * kKT * D;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
+  const int t0 = blockIdx.x * kQ, h = blockIdx.y, b = blockIdx.z;
+  const int J = t0 / bsz, u0 = J * bsz;
+  const int ta = t0 + warp * 16 + gl, tb = ta + 8;
+  const int t_last = min(T - 1, t0 + kQ - 1);
+  uint32_t qf[D / 16][4];
+  load_q_frag(qf, q + (((size_t)b * T + min(ta, T - 1)) * H + h) * D, q + (((size_t)b * T + min(tb, T - 1)) * H + h) * D,
+              ta < T, tb < T, cq);
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[D / 8][4];
+#pragma unroll
+  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  const int ntiles = (t_last - u0) / kKT + 1;
+  auto load = [&](int it, int buf) {
+    for (int x = tid; x < kKT * (D / 8); x += kThreads) {
+      const int r = x / (D / 8), ch = x % (D / 8);
+      const int u = u0 + it * kKT + r;
+      const bool ok = u <= t_last;
+      const size_t row = ((size_t)b * T + (ok ? u : t_last)) * H + h;
+      cp_async16(sK + buf * kKT * D + SwzTile<D>::offset(r, ch), k + row * D + ch * 8, ok);
+      cp_async16(sV + buf * kKT * D + SwzTile<D>::offset(r, ch), v + row * D + ch * 8, ok);
+    }
+  };
+  load(0, 0);
+  cp_async_commit();
+  for (int it = 0; it < ntiles; ++it) {
+    if (it + 1 < ntiles) load(it + 1, (it + 1) & 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    __syncthreads();
+    float s[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
+    qk64(qf, sK + (it & 1) * kKT * D, s, lane);
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int u = u0 + it * kKT + nt * 8 + 2 * cq + e;
+        s[nt][e] = u <= ta ? s[nt][e] * scale_log2 : -INFINITY;
+        s[nt][2 + e] = u <= tb ? s[nt][2 + e] * scale_log2 : -INFINITY;
+      }
+    online(s, m0, m1, l0, l1, o);
+    pv64(s, sV + (it & 1) * kKT * D, o, lane);
+    __syncthreads();
+  }
+  cp_async_wait<0>();
+  // merge the past slots (each a normalised o with its log-sum-exp) into the own-block state
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int t = half ? tb : ta;
+    if (t >= T) continue;
+    const int32_t* row = idx + (((size_t)b * H + h) * T + t) * (top_k + 1);
+    float m = half ? m1 : m0, l = half ? l1 : l0;   // own block: m finite (t itself is always visible)
+    float lse[kMaxK];
+    int np = 0;
+    for (int s = 0; s < top_k; ++s) {
+      const int j = row[s];
+      if (j < 0 || j >= J) break;
+      lse[np++] = part_lse[(((size_t)b * T + t) * H + h) * top_k + s];
+    }
+    float M = m + __log2f(l);
+    for (int s = 0; s < np; ++s) M = fmaxf(M, lse[s]);
+    const float w_own = exp2f(m - M);        // multiplies the unnormalised own o (sum l)
+    float wsum = l * w_own;
+    float ws[kMaxK];
+    for (int s = 0; s < np; ++s) { ws[s] = exp2f(lse[s] - M); wsum += ws[s]; }
+    const float inv = 1.f / wsum;
+    __nv_bfloat16* dst = out + (((size_t)b * T + t) * H + h) * D;
+    const __nv_bfloat16* po = part_o + (((size_t)b * T + t) * H + h) * top_k * D;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) {
+      float x0 = o[i][2 * half] * w_own, x1 = o[i][2 * half + 1] * w_own;
+      for (int s = 0; s < np; ++s) {
+        const __nv_bfloat162 p2 = *reinterpret_cast<const __nv_bfloat162*>(po + s * D + i * 8 + 2 * cq);
+        const float2 pf = __bfloat1622float2(p2);
+        x0 += ws[s] * pf.x;
+        x1 += ws[s] * pf.y;
+      }
+      *reinterpret_cast<uint32_t*>(dst + i * 8 + 2 * cq) = pack_bf16(x0 * inv, x1 * inv);
+    }
+  }
+}
+
+constexpr size_t kAttnSmem = 4ull * kKT * D * 2;   // K and V, double buffered: 64 KB
+
+}  // namespace
+
+MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  MobaLayout L{};
+  const size_t nblk = (T + bsz - 1) / bsz;
+  const size_t E = (size_t)B * H * nblk;
+  size_t off = 0;
+  L.kbar = off; off = up(off + (size_t)B * nblk * H * D * 4);
+  L.idx = off; off = up(off + (size_t)B * H * T * (top_k + 1) * 4);
+  L.counts = off; off = up(off + E * 4);
+  L.offsets = off; off = up(off + (E + 1) * 4);
+  L.chunks = off; off = up(off + (E + 1) * 4);
+  L.fill = off; off = up(off + E * 4);
+  L.list = off; off = up(off + (size_t)B * H * T * top_k * 4);
+  L.part_lse = off; off = up(off + (size_t)B * T * H * top_k * 4);
+  L.part_o = off; off = up(off + (size_t)B * T * H * top_k * D * 2);
+  L.total = off;
+  return L;
+}
+
+cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(moba_past_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moba_own_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int nblk = (a.T + a.bsz - 1) / a.bsz;
+  const int E = a.B * a.H * nblk;
+  const MobaLayout L = moba_layout(a.B, a.T, a.H, a.bsz, a.top_k);
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  int32_t* idx = a.idx ? a.idx : reinterpret_cast<int32_t*>(ws + L.idx);
+  int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+  int32_t* chunks = reinterpret_cast<int32_t*>(ws + L.chunks);
+  int32_t* fill = reinterpret_cast<int32_t*>(ws + L.fill);
+  int32_t* list = reinterpret_cast<int32_t*>(ws + L.list);
+  float* part_lse = reinterpret_cast<float*>(ws + L.part_lse);
+  __nv_bfloat16* part_o = reinterpret_cast<__nv_bfloat16*>(ws + L.part_o);
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(a.v);
+  cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)E * 4, st);
+  if (e != cudaSuccess) return e;
+  if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
+  moba_mean_kernel<<<dim3(nblk, a.H, a.B), D, 0, st>>>(k, kbar, a.T, a.H, a.bsz, nblk);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
+  moba_select_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, 0, st>>>(q, kbar, idx, counts, a.T, a.H, a.bsz,
+                                                                              nblk, a.top_k);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
+  moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, E);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  moba_scatter_kernel<<<dim3((a.T + 255) / 256, a.B * a.H), 256, 0, st>>>(idx, offsets, fill, list, a.T, a.H, nblk,
+                                                                         a.top_k, a.bsz);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (a.top_k > 0) {
+    moba_past_kernel<<<sms * 3, kThreads, kAttnSmem, st>>>(q, k, v, counts, offsets, chunks, list, part_o, part_lse,
+                                                           a.T, a.H, nblk, a.bsz, a.top_k, E, a.scale_log2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
+  moba_own_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kAttnSmem, st>>>(
+      q, k, v, idx, part_o, part_lse, static_cast<__nv_bfloat16*>(a.out), a.T, a.H, a.bsz, a.top_k, a.scale_log2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.mark) e = a.mark(a.mark_ctx, st);
+  return e;
+}
+
+}  // namespace nsa

@@ -11,6 +11,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxTokensNsa = 65536;   // 1024 selection blocks per token (top-k kept in shared memory)
+constexpr int kMaxTokensMoba = 1 << 20;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -42,7 +43,7 @@ nsa_status check_cfg(const nsa_config* c) {
     if (c->seqlen > kMaxTokensNsa) return NSA_ERR_UNSUPPORTED;
   } else {
     if (c->h_q != c->h_kv || c->d_k != c->d_v) return NSA_ERR_INVALID_ARG;
-    return NSA_ERR_UNSUPPORTED;
+    if (c->d_k != 128 || c->sel_block % 64 || c->top_k > 7 || c->seqlen > kMaxTokensMoba) return NSA_ERR_UNSUPPORTED;
   }
   if ((c->sel_idx_out && !aligned16(c->sel_idx_out)) || (c->kc_out && !aligned16(c->kc_out)) ||
       (c->vc_out && !aligned16(c->vc_out)))
@@ -66,6 +67,11 @@ FwdLayout forward_layout(const nsa_config* c) {
   return L;
 }
 
+size_t workspace_bytes(const nsa_config* c) {
+  if (c->mode == NSA_MODE_MOBA) return nsa::moba_layout(c->batch, c->seqlen, c->h_q, c->sel_block, c->top_k).total;
+  return forward_layout(c).total;
+}
+
 nsa_status check_workspace(const nsa_config* c, size_t need) {
   if (need == 0) return NSA_OK;
   if (!c->workspace || (reinterpret_cast<uintptr_t>(c->workspace) % kAlign)) return NSA_ERR_WORKSPACE;
@@ -87,6 +93,21 @@ struct StageMarks {
   }
 };
 
+cudaError_t mark_trampoline(void* ctx, cudaStream_t s) { return static_cast<StageMarks*>(ctx)->mark(s); }
+
+nsa_status moba_forward(const void* q, const void* k, const void* v, const nsa_config* cfg, void* out,
+                        cudaStream_t s) {
+  StageMarks marks(cfg, 5);
+  nsa::MobaArgs a{};
+  a.q = q; a.k = k; a.v = v; a.out = out; a.idx = cfg->sel_idx_out; a.workspace = cfg->workspace;
+  a.B = cfg->batch; a.T = cfg->seqlen; a.H = cfg->h_q; a.bsz = cfg->sel_block; a.top_k = cfg->top_k;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.mark = mark_trampoline;
+  a.mark_ctx = &marks;
+  return from_cuda(nsa::launch_moba(a, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -105,7 +126,7 @@ const char* nsa_status_string(nsa_status s) {
 
 size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch) {
   if (check_cfg(cfg) != NSA_OK || decode_batch < 0) return 0;
-  if (decode_batch == 0) return forward_layout(cfg).total;
+  if (decode_batch == 0) return workspace_bytes(cfg);
   return 0;   // nsa_decode keeps everything on chip
 }
 
@@ -126,9 +147,10 @@ nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* 
     return NSA_ERR_INVALID_ARG;
   if (cfg->mode == NSA_MODE_NSA && (!gates || (reinterpret_cast<uintptr_t>(gates) & 1u)))
     return NSA_ERR_INVALID_ARG;
-  const FwdLayout L = forward_layout(cfg);
-  st = check_workspace(cfg, L.total);
+  st = check_workspace(cfg, workspace_bytes(cfg));
   if (st != NSA_OK) return st;
+  if (cfg->mode == NSA_MODE_MOBA) return moba_forward(q, k, v, cfg, out, static_cast<cudaStream_t>(stream));
+  const FwdLayout L = forward_layout(cfg);
 
   auto ws = static_cast<uint8_t*>(cfg->workspace);
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -62,7 +62,8 @@ typedef enum {
  *                 L_max of the caches (their second dimension).
  *   h_q, h_kv     query and KV heads; h_q % h_kv == 0.  MoBA needs h_q == h_kv.
  *   d_k, d_v      head dims.  Implemented: NSA (d_k,d_v) in {(64,64),(128,128),
- *                 (192,128)}, G <= 16; MoBA d_k = d_v = 128.
+ *                 (192,128)}, G <= 16, T <= 65536; MoBA d_k = d_v = 128, sel_block a
+ *                 multiple of 64, T <= 2^20.
  *   cmp_block,    (NSA) compression block l and stride s ([NOTES] §5: each block
  *   cmp_stride    of l tokens becomes one key and one value).  Implemented: 32, 16.
  *   sel_block     selection block size b: 64 for NSA ([NOTES] §17: 64-token blocks,
@@ -87,9 +88,11 @@ typedef enum {
  *   n_stage_events handles.  When n_stage_events >= (kernels launched) + 1, event 0 is
  *                 recorded on `stream` before the first kernel and event i after the
  *                 i-th, so that cudaEventElapsedTime gives each kernel's duration.
- *                 nsa_forward launches 5 kernels in NSA mode (phi of K, phi of V,
+ *                 nsa_forward has 5 stages in NSA mode (phi of K, phi of V,
  *                 compressed attention + selection, selected attention, window +
- *                 combine).  NULL or too few: nothing is recorded.
+ *                 combine) and 5 in MoBA mode (block means, selection, query lists,
+ *                 past-block attention, own block + merge); nsa_decode has 1.
+ *                 NULL or too few: nothing is recorded.
  */
 typedef struct {
   int32_t mode;

@@ -1,0 +1,484 @@
+// K2 on the 5th-generation tensor cores: compressed attention + group-summed block
+// scores + top-k ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5, §8; "一文比较 Kimi 和
+// Deepseek 的两篇稀疏注意力机制论文", "Deepseek 的论文核心点": the selection scores come
+// from the compressed attention and the group's heads add them before one top-k).
+//
+// One CTA = one KV group g and 8 consecutive tokens; its 128 query rows (token-major,
+// 16 heads per token) are one tcgen05 M=128 tile held in shared memory.  The group's
+// compressed keys/values stream through shared memory by TMA in tiles of 128 blocks.
+//   pass A   S = Q Kc^T into TMEM (rows = (token, head)); each softmax thread owns a
+//            row and keeps its running max and sum -> log-sum-exp per row.
+//   pass B   S^T = Kc Q^T into TMEM (rows = compressed blocks, columns = (token, head)):
+//            each softmax thread owns one compressed block, forms the normalised
+//            probabilities of its 128 columns, adds each token's 16 heads in registers
+//            (the group sum), folds them into 64-token selection-block scores, and
+//            writes P^T (bf16) to shared memory; O^T = Vc^T P^T accumulates in TMEM
+//            (rows = value dims), already normalised, so no rescaling is ever needed.
+//   top-k    per token over the selection-block scores in shared memory.
+//   epilogue acc[t, h, :] = g_cmp * o_cmp, read from O^T (each thread one value dim).
+// Warp roles: 0 TMA producer, 1 MMA issuer (and TMEM owner), 4-7 softmax / epilogue
+// (warp 4+q owns TMEM lanes 32q..32q+31).  Every wait is bounded (see tc.cuh); on a
+// timeout the kernel records an error word, stops issuing work, and frees its TMEM.
+#include <cfloat>
+
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace nsa {
+
+namespace {
+constexpr int kThreads = 256;
+constexpr int kTok = 8;            // tokens per CTA
+constexpr int kRowsM = 128;        // query rows per CTA (8 tokens x 16 heads)
+constexpr int kBlk = 128;          // compressed blocks per tile
+constexpr int kKcSlots = 3;        // ring of 64-column Kc slices
+constexpr int kMaxSel = 1024;
+constexpr int kL = 32, kS = 16, kSel = 64;
+constexpr uint32_t kSlice = kBlk * 128;          // one 64-column slice of a 128-row tile: 16 KB
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+
+enum Err { kErrQ = 1, kErrKcFull, kErrKcEmpty, kErrVcFull, kErrVcEmpty, kErrSFull, kErrSEmpty, kErrPFull,
+           kErrPEmpty, kErrOFull };
+
+template <int DK, int DV>
+struct Smem {
+  static constexpr int kQSlices = DK / 64, kVSlices = DV / 64;
+  static constexpr uint32_t kQ = 0;                                         // Q: kQSlices x 16 KB
+  static constexpr uint32_t kKc = kQ + kQSlices * kSlice;                   // Kc ring: kKcSlots x 16 KB
+  static constexpr uint32_t kVc = kKc + kKcSlots * kSlice;                  // Vc: 2 buffers x kVSlices x 16 KB
+  static constexpr uint32_t kP = kVc + 2 * kVSlices * kSlice;               // P^T: 2 x 16 KB (N = 128 rows)
+  static constexpr uint32_t kScore = kP + 2 * kSlice;                       // [8][1024] fp32
+  static constexpr uint32_t kLse = kScore + kTok * kMaxSel * 4;             // [128] fp32
+  static constexpr uint32_t kGate = kLse + kRowsM * 4;                      // [128] fp32
+  static constexpr uint32_t kBar = kGate + kRowsM * 4;                      // mbarriers
+  static constexpr int kNumBars = 1 + 2 * kKcSlots + 2 * 2 + 2 * 2 + 2 + 1;
+  static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
+  static constexpr uint32_t kBytes = kTmemSlot + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;                         // room to align the base to 1 KB
+  static_assert(kAlloc <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ int n_visible(int t, int nc) { return t < kL - 1 ? 0 : min(nc, (t - kL + 1) / kS + 1); }
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// Barrier among the softmax warps that also ANDs `pred` across them, so that every warp
+// takes the same branch afterwards (no warp can be left waiting at a later barrier).
+__device__ __forceinline__ bool vote_all(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+                     const __grid_constant__ CUtensorMap tm_vc, const __nv_bfloat16* __restrict__ gates,
+                     float* __restrict__ acc, int32_t* __restrict__ idx_out, int T, int Hq, int Hkv, int nc, int top_k,
+                     int force_first, int force_local, float scale_log2, int* __restrict__ err) {
+  using SM = Smem<DK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + SM::kQ;
+  uint8_t* sKc = smem + SM::kKc;
+  uint8_t* sVc = smem + SM::kVc;
+  uint8_t* sP = smem + SM::kP;
+  float* sScore = reinterpret_cast<float*>(smem + SM::kScore);
+  float* sLse = reinterpret_cast<float*>(smem + SM::kLse);
+  float* sGate = reinterpret_cast<float*>(smem + SM::kGate);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+  uint64_t* bar_q = bars;
+  uint64_t* kc_full = bars + 1;
+  uint64_t* kc_empty = kc_full + kKcSlots;
+  uint64_t* vc_full = kc_empty + kKcSlots;
+  uint64_t* vc_empty = vc_full + 2;
+  uint64_t* s_full = vc_empty + 2;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* p_empty = p_full + 1;
+  uint64_t* o_full = p_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tok_tiles = (T + kTok - 1) / kTok;
+  const int t0 = (n_tok_tiles - 1 - (int)blockIdx.x) * kTok;   // longest rows first
+  const int g = blockIdx.y, b = blockIdx.z;
+  const int t_last = min(t0 + kTok - 1, T - 1);
+  const int ntiles = (n_visible(t_last, nc) + kBlk - 1) / kBlk;
+
+  if (tid == 0) {
+    tc::mbar_init(bar_q, 1);
+    for (int i = 0; i < kKcSlots; ++i) { tc::mbar_init(kc_full + i, 1); tc::mbar_init(kc_empty + i, 1); }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(vc_full + i, 1);
+      tc::mbar_init(vc_empty + i, 1);
+      tc::mbar_init(s_full + i, 1);
+      tc::mbar_init(s_empty + i, 4);
+    }
+    tc::mbar_init(p_full, 4);
+    tc::mbar_init(p_empty, 1);
+    tc::mbar_init(o_full, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_kc);
+      tc::prefetch_tmap(&tm_vc);
+      tc::mbar_expect_tx(bar_q, SM::kQSlices * kSlice);
+      for (int s = 0; s < SM::kQSlices; ++s) tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, g * 16, b * T + t0);
+      int fill = 0;   // Kc slice fills so far
+      bool ok = true;
+      for (int pass = 0; pass < 2 && ok; ++pass) {
+        for (int n = 0; n < ntiles && ok; ++n) {
+          const int row = b * nc + n * kBlk;
+          for (int s = 0; s < SM::kQSlices && ok; ++s, ++fill) {
+            const int slot = fill % kKcSlots;
+            ok = tc::mbar_wait(kc_empty + slot, ((fill / kKcSlots) & 1) ^ 1, err, kErrKcEmpty);
+            if (!ok) break;
+            tc::mbar_expect_tx(kc_full + slot, kSlice);
+            tc::tma_load_3d(sKc + slot * kSlice, &tm_kc, kc_full + slot, s * 64, g, row);
+          }
+          if (pass == 1 && ok) {
+            const int vb = n & 1;
+            ok = tc::mbar_wait(vc_empty + vb, ((n >> 1) & 1) ^ 1, err, kErrVcEmpty);
+            if (!ok) break;
+            tc::mbar_expect_tx(vc_full + vb, SM::kVSlices * kSlice);
+            for (int s = 0; s < SM::kVSlices; ++s)
+              tc::tma_load_3d(sVc + (vb * SM::kVSlices + s) * kSlice, &tm_vc, vc_full + vb, s * 64, g, row);
+          }
+        }
+      }
+      // before leaving, let the copies still in flight land (bounded)
+      for (int i = 0; i < kKcSlots && i < fill; ++i) {
+        const int f = fill - 1 - i;
+        tc::mbar_wait(kc_full + (f % kKcSlots), (f / kKcSlots) & 1, err, kErrKcFull);
+      }
+      for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (tc::elect_one()) {
+      const uint32_t idA = tc::idesc_bf16(128, 128, 0, 0);     // S  = Q  Kc^T   (both K-major)
+      const uint32_t idPV = tc::idesc_bf16(128, 128, 1, 1);    // O^T = Vc^T P^T (both MN-major)
+      bool ok = tc::mbar_wait(bar_q, 0, err, kErrQ);
+      tc::tc_fence_after();
+      int use = 0;    // S buffer uses over both passes
+      int fill = 0;   // Kc slices consumed
+      auto issue_s = [&](int pass) -> bool {
+        const int sb = use & 1;
+        if (!tc::mbar_wait(s_empty + sb, ((use >> 1) & 1) ^ 1, err, kErrSEmpty)) return false;
+        tc::tc_fence_after();
+        const uint32_t d = tmem + (sb ? kColS1 : kColS0);
+        for (int s = 0; s < SM::kQSlices; ++s, ++fill) {
+          const int slot = fill % kKcSlots;
+          if (!tc::mbar_wait(kc_full + slot, (fill / kKcSlots) & 1, err, kErrKcFull)) return false;
+          tc::tc_fence_after();
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t dq = tc::sdesc(sQ + s * kSlice + ks * 32, 16, 1024);
+            const uint64_t dk = tc::sdesc(sKc + slot * kSlice + ks * 32, 16, 1024);
+            if (pass == 0) tc::mma_ss(d, dq, dk, idA, (s | ks) != 0);
+            else tc::mma_ss(d, dk, dq, idA, (s | ks) != 0);
+          }
+          tc::mma_commit(kc_empty + slot);
+        }
+        tc::mma_commit(s_full + sb);
+        ++use;
+        return true;
+      };
+      for (int n = 0; n < ntiles && ok; ++n) ok = issue_s(0);
+      if (ok && ntiles > 0) ok = issue_s(1);
+      for (int n = 0; n < ntiles && ok; ++n) {
+        if (n + 1 < ntiles) ok = issue_s(1);
+        if (!ok) break;
+        ok = tc::mbar_wait(p_full, n & 1, err, kErrPFull) && tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint8_t* vb = sVc + (n & 1) * SM::kVSlices * kSlice;
+        for (int ks = 0; ks < kBlk / 16; ++ks) {
+          const uint64_t da = tc::sdesc(vb + ks * 16 * 128, kSlice, 1024);
+          const uint64_t db = tc::sdesc(sP + ks * 16 * 128, kSlice, 1024);
+          tc::mma_ss(tmem + kColO, da, db, idPV, (n | ks) != 0);
+        }
+        tc::mma_commit(p_empty);
+        tc::mma_commit(vc_empty + (n & 1));
+      }
+      if (ok && ntiles > 0) tc::mma_commit(o_full);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int r = tid - 128;                     // TMEM lane owned by this thread
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
+    const int my_tok = r / 16;                   // pass A: this thread's row = (token, head)
+    const int my_t = t0 + my_tok;
+    const int my_nvis = my_t < T ? n_visible(my_t, nc) : 0;
+    int nvis_tok[kTok], nb_tok[kTok];   // visible compressed blocks and eligible selection blocks per token
+#pragma unroll
+    for (int k = 0; k < kTok; ++k) {
+      nvis_tok[k] = (t0 + k < T) ? n_visible(t0 + k, nc) : 0;
+      nb_tok[k] = (t0 + k < T) ? (t0 + k) / kSel + 1 : 0;
+    }
+    bool ok = true;
+    int use = 0;
+    // gates of the 128 rows (g_cmp), zeroed scores
+    {
+      const int t = t0 + my_tok, h = g * 16 + (r % 16);
+      sGate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3]) : 0.f;
+      for (int i = r; i < kTok * kMaxSel; i += 128) sScore[i] = 0.f;
+    }
+    // pass A: log-sum-exp of this thread's row
+    float m = -INFINITY, l = 0.f;
+    for (int n = 0; n < ntiles && ok; ++n, ++use) {
+      const int sb = use & 1;
+      ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const uint32_t base = lane_addr + (sb ? kColS1 : kColS0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+        float v[32];
+        tc::tmem_ld16(base + c0, *reinterpret_cast<float(*)[16]>(v));
+        tc::tmem_ld16(base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+        tc::tmem_wait_ld();
+        float cm = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int i = n * kBlk + c0 + j;
+          v[j] = i < my_nvis ? v[j] * scale_log2 : -INFINITY;
+          cm = fmaxf(cm, v[j]);
+        }
+        const float mn = fmaxf(m, cm);
+        if (mn != -INFINITY) {
+          float sum = 0.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sum += ex2(v[j] - mn);
+          l = l * ex2(m - mn) + sum;
+          m = mn;
+        }
+      }
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(s_empty + sb);
+    }
+    sLse[r] = (my_t < T && l > 0.f) ? m + __log2f(l) : INFINITY;
+    named_sync(1, 128);
+    // pass B: probabilities, P^T, block scores
+    ok = vote_all(1, 128, ok);
+    for (int n = 0; n < ntiles && ok; ++n, ++use) {
+      const int sb = use & 1;
+      ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+      if (ok && n > 0) ok = tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty);
+      ok = vote_all(1, 128, ok);
+      if (!ok) break;
+      tc::tc_fence_after();
+      const uint32_t base = lane_addr + (sb ? kColS1 : kColS0);
+      const int i = n * kBlk + r;                // this thread's compressed block
+      float tok_sum[kTok];
+      uint8_t* prow0 = sP + r * 128;             // N-block 0 (rows 0..63 of the query tile)
+      uint8_t* prow1 = sP + kSlice + r * 128;    // N-block 1 (rows 64..127)
+#pragma unroll
+      for (int k = 0; k < kTok; ++k) {
+        float v[16];
+        tc::tmem_ld16(base + k * 16, v);
+        tc::tmem_wait_ld();
+        const bool vis = i < nvis_tok[k];
+        float s = 0.f;
+        uint32_t pk[8];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          const float p0 = vis ? ex2(v[j] * scale_log2 - sLse[k * 16 + j]) : 0.f;
+          const float p1 = vis ? ex2(v[j + 1] * scale_log2 - sLse[k * 16 + j + 1]) : 0.f;
+          s += p0 + p1;
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+          pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+        }
+        tok_sum[k] = s;
+        // columns k*16 .. k*16+15 are chunks 2*(k%4), 2*(k%4)+1 of N-block k/4
+        uint8_t* prow = (k < 4) ? prow0 : prow1;
+        const int c0 = 2 * (k & 3);
+        *reinterpret_cast<uint4*>(prow + ((c0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(prow + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      }
+      tc::tc_fence_before();
+      tc::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(s_empty + sb);
+        tc::mbar_arrive(p_full);
+      }
+      // selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Phase 1: each group
+      // of four lanes adds its own four blocks plus the lane just below it; phase 2: lane 31
+      // hands its block (i % 4 == 3) to the first selection block of the next warp or tile.
+      const int wq = warp - 4;
+      const int j0 = n * (kBlk / 4) + wq * 8;    // first selection block of this warp
+#pragma unroll
+      for (int k = 0; k < kTok; ++k) {
+        const float v = tok_sum[k];
+        float g4 = v + __shfl_xor_sync(0xffffffffu, v, 1);
+        g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
+        const float prev = __shfl_up_sync(0xffffffffu, v, 1);
+        const int j = j0 + (lane >> 2);
+        if ((lane & 3) == 0 && j < nb_tok[k]) sScore[k * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
+      }
+      named_sync(1, 128);
+      if (lane == 31) {
+#pragma unroll
+        for (int k = 0; k < kTok; ++k)
+          if (j0 + 8 < nb_tok[k]) sScore[k * kMaxSel + j0 + 8] += tok_sum[k];
+      }
+      named_sync(1, 128);
+    }
+    named_sync(1, 128);
+
+    // top-k: warp wq takes tokens wq and wq+4
+    const int wq = warp - 4;
+    for (int k = wq; k < kTok && ok; k += 4) {
+      const int t = t0 + k;
+      if (t >= T) continue;
+      const float* score = sScore + k * kMaxSel;
+      const int nb = t / kSel + 1;
+      int32_t* dst = idx_out + (((size_t)b * Hkv + g) * T + t) * top_k;
+      if (nb <= top_k) {
+        for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
+        continue;
+      }
+      const int own = t / kSel;
+      uint32_t taken = 0;
+      int nforced = 0;
+      if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
+      if (force_local && !(force_first && own == 0)) {
+        if (lane == (own & 31)) taken |= 1u << (own >> 5);
+        ++nforced;
+      }
+      const int mmax = (nb + 31) >> 5;
+      for (int rr = nforced; rr < top_k; ++rr) {
+        float bs = -FLT_MAX;
+        int bj = 0x7fffffff;
+        for (int mm = 0; mm < mmax; ++mm) {
+          const int j = lane + 32 * mm;
+          if (j < nb && !((taken >> mm) & 1u)) {
+            const float sc = score[j];
+            if (sc > bs) { bs = sc; bj = j; }
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+          const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+          if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; }
+        }
+        if (bj != 0x7fffffff && lane == (bj & 31)) taken |= 1u << (bj >> 5);
+      }
+      int pos = 0;
+      for (int mm = 0; mm < mmax; ++mm) {
+        const bool sel = (taken >> mm) & 1u;
+        const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+        if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
+        pos += __popc(bal);
+      }
+      for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
+    }
+
+    // epilogue: thread r owns value dim r of O^T; column c = (token c/16, head c%16)
+    if (ok && ntiles > 0) ok = tc::mbar_wait(o_full, 0, err, kErrOFull);
+    if (ok) {
+      tc::tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < kRowsM; c0 += 16) {
+        float v[16];
+        if (ntiles > 0) {
+          tc::tmem_ld16(lane_addr + kColO + c0, v);
+          tc::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0.f;
+        }
+        const int k = c0 / 16, t = t0 + k;
+        if (t < T && r < DV) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const size_t row = ((size_t)b * T + t) * Hq + g * 16 + j;
+            acc[row * DV + r] = sGate[c0 + j] * v[j];
+          }
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int DK, int DV>
+cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
+  using SM = Smem<DK, DV>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(cmp_select_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)SM::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap mq, mkc, mvc;
+  const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
+  const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
+  const uint32_t bq[3] = {64, 16, kTok};
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
+  const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
+  const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
+  const uint32_t bkv[3] = {64, 1, kBlk};
+  if (!make_tmap_bf16(&mq, a.q, 3, dq, sq, bq)) return cudaErrorInvalidValue;
+  if (a.nc > 0) {
+    if (!make_tmap_bf16(&mkc, a.kc, 3, dk3, sk3, bkv) || !make_tmap_bf16(&mvc, a.vc, 3, dv3, sv3, bkv))
+      return cudaErrorInvalidValue;
+  } else {
+    mkc = mq;   // never dereferenced: no tile is loaded when there is no compressed block
+    mvc = mq;
+  }
+  dim3 grid((a.T + kTok - 1) / kTok, a.Hkv, a.B);
+  cmp_select_tc_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
+      mq, mkc, mvc, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, a.T, a.Hq, a.Hkv, a.nc, a.top_k,
+      a.force_first, a.force_local, a.scale_log2, a.err);
+  return cudaGetLastError();
+}
+}  // namespace
+
+bool cmp_select_tc_supported(const FwdArgs& a) {
+  return a.G == 16 && a.dv == 128 && (a.dk == 128 || a.dk == 192) && a.T <= kMaxSel * kSel && a.err != nullptr;
+}
+
+cudaError_t launch_cmp_select_tc(const FwdArgs& a, cudaStream_t st) {
+  if (a.dk == 192) return launch_tc<192, 128>(a, st);
+  return launch_tc<128, 128>(a, st);
+}
+
+}  // namespace nsa

@@ -25,11 +25,15 @@ struct FwdArgs {
   int B, T, Hq, Hkv, G, dk, dv, nc;
   int top_k, window, force_first, force_local;
   float scale_log2;   // softmax scale * log2(e)
+  int* err;           // device word, zeroed before the launches; nonzero = a bounded wait timed out
 };
 
 // K2: compressed attention (writes acc = g_cmp * o_cmp) + group-summed block
 // scores + top-k (writes idx).
 cudaError_t launch_cmp_select(const FwdArgs& a, cudaStream_t st);
+// K2 on tcgen05 + TMA (G == 16, d_v == 128, d_k in {128, 192}).
+bool cmp_select_tc_supported(const FwdArgs& a);
+cudaError_t launch_cmp_select_tc(const FwdArgs& a, cudaStream_t st);
 // K3: selected-block attention (acc += g_slc * o_slc).
 cudaError_t launch_slc_attn(const FwdArgs& a, cudaStream_t st);
 // K4 + K5: sliding window and gated combine (out = bf16(acc + g_win * o_win)).

@@ -52,13 +52,14 @@ nsa_status check_cfg(const nsa_config* c) {
 }
 
 struct FwdLayout {
-  size_t kc, vc, idx, acc, total;
+  size_t err, kc, vc, idx, acc, total;
 };
 
 FwdLayout forward_layout(const nsa_config* c) {
   const size_t B = c->batch, T = c->seqlen, nc = n_cmp(c->seqlen, c->cmp_block, c->cmp_stride);
   FwdLayout L{};
   size_t off = 0;
+  L.err = off; off = align_up(off + 4);
   L.kc = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
   L.vc = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
   L.idx = off; off = align_up(off + B * c->h_kv * T * c->top_k * 4);
@@ -167,9 +168,11 @@ nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* 
   a.kc = kc; a.vc = vc;
   a.idx = cfg->sel_idx_out ? cfg->sel_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   a.acc = reinterpret_cast<float*>(ws + L.acc);
+  a.err = reinterpret_cast<int*>(ws + L.err);
 
   StageMarks marks(cfg, 5);
-  cudaError_t e = marks.mark(s);
+  cudaError_t e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = marks.mark(s);
   if (e == cudaSuccess)
     e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, kc, s);
   if (e == cudaSuccess) e = marks.mark(s);

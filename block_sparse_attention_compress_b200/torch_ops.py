@@ -35,6 +35,11 @@ class NSAForward:
         self.cfg.workspace = self.workspace.data_ptr()
         self.cfg.workspace_bytes = nbytes
 
+    def device_status(self) -> int:
+        """The workspace's status word after a synchronised call: 0, or the code of a
+        device-side wait that timed out."""
+        return int(self.workspace[:4].view(torch.int32).item())
+
     def __call__(self, q, k, v, gates, out=None):
         B, T, h_q, h_kv, d_k, d_v = self.shape
         if out is None:

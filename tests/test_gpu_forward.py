@@ -25,6 +25,7 @@ def run_gpu(x, top_k, window, gates=None, **kw):
     f = NSAForward(B, T, hq, hkv, dk, dv, dev[4], dev[5], top_k=top_k, window=window, **kw)
     out = f(*dev[:4])
     torch.cuda.synchronize()
+    assert f.device_status() == 0
     return out.cpu(), f.idx.cpu(), f.kc.cpu(), f.vc.cpu()
 
 

@@ -255,6 +255,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     for (int n = 0; n < ntiles && ok; ++n, ++use) {
       const int sb = use & 1;
       ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+      ok = __all_sync(0xffffffffu, ok);   // reconverge before the warp-wide TMEM loads
       if (!ok) break;
       tc::tc_fence_after();
       const uint32_t base = lane_addr + (sb ? kColS1 : kColS0);
@@ -405,6 +406,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
     // epilogue: thread r owns value dim r of O^T; column c = (token c/16, head c%16)
     if (ok && ntiles > 0) ok = tc::mbar_wait(o_full, 0, err, kErrOFull);
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc::tc_fence_after();
 #pragma unroll 1

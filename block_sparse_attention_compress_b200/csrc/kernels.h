@@ -36,6 +36,8 @@ bool cmp_select_tc_supported(const FwdArgs& a);
 cudaError_t launch_cmp_select_tc(const FwdArgs& a, cudaStream_t st);
 // K3: selected-block attention (acc += g_slc * o_slc).
 cudaError_t launch_slc_attn(const FwdArgs& a, cudaStream_t st);
+bool slc_attn_tma_supported(const FwdArgs& a);
+cudaError_t launch_slc_attn_tma(const FwdArgs& a, cudaStream_t st);
 // K4 + K5: sliding window and gated combine (out = bf16(acc + g_win * o_win)).
 cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st);
 

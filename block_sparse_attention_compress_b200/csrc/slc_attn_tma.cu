@@ -1,0 +1,344 @@
+// K3, streaming version: selected-block attention fed by TMA
+// ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5: the top-k blocks are expanded to
+// all their tokens; §10: the group's heads share every loaded block).
+//
+// Persistent CTAs walk the (KV group, batch, token) items, group-major so that the
+// CTAs running at the same time share one group's K/V in L2.  Warp 4 is a TMA
+// producer: for every chosen block of every item it copies the whole 64-token K and V
+// block (128-byte swizzle, 64-column boxes) into a 4-slot ring of 40 KB slots.  Warps
+// 0-3 each take 16 of the 64 keys of every block, with the group's G <= 16 heads as
+// the 16 rows of warp-level m16n8k16 MMAs and an online softmax; at the end of an
+// item their four states are merged and acc += g_slc * o_slc is written.  The ring
+// runs across item boundaries, so the loads of the next token overlap the merge.
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace nsa {
+
+namespace {
+constexpr int kConsumers = 4;
+constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kBlk = 64;
+constexpr int kSlots = 4;
+constexpr int kCtasPerSm = 1;
+constexpr uint32_t kBox = kBlk * 128;   // one 64-row x 64-column box: 8 KB
+
+template <int DK, int DV>
+struct Smem {
+  static constexpr uint32_t kSlotBytes = (DK / 64 + DV / 64) * kBox;
+  static constexpr uint32_t kRing = 0;
+  // merge scratch: every warp leaves, for each of the other three warps, the 32-column
+  // slice that warp owns ([writer][owner slot][16 rows][DV/4]), plus its m and l per row
+  static constexpr uint32_t kMerge = kRing + kSlots * kSlotBytes;
+  static constexpr uint32_t kBar = kMerge + kConsumers * 3 * 16 * (DV / 4) * 4 + kConsumers * 16 * 2 * 4;
+  static constexpr uint32_t kBytes = kBar + 2 * kSlots * 8;
+  static constexpr uint32_t kAlloc = kBytes + 1024;
+  static_assert(kAlloc * kCtasPerSm <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+__device__ __forceinline__ bool vote_all(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
+// byte offset of (row, 16-byte chunk c of a 64-column box) in a 128-byte-swizzled box
+__device__ __forceinline__ uint32_t swz(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gates,
+                    const int32_t* __restrict__ idx, float* __restrict__ acc, int B, int T, int Hq, int Hkv, int G,
+                    int top_k, float scale_log2, int* __restrict__ err) {
+  using SM = Smem<DK, DV>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+  uint64_t* empty = full + kSlots;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      tc::mbar_init(full + s, 1);
+      tc::mbar_init(empty + s, kConsumers);
+    }
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  const long total = (long)Hkv * B * T;
+
+  if (warp == kConsumers) {
+    // ---------------------------------------------------------------- producer
+    // (the whole warp runs the loop; lane 0 issues the copies)
+    if (lane == 0) {
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+    }
+    long fill = 0;
+    bool ok = true;
+    for (long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const int g = (int)(it / ((long)B * T));
+      const int bt = (int)(it % ((long)B * T));
+      const int b = bt / T, t = bt % T;
+      const int mine = lane < top_k ? idx[(((size_t)b * Hkv + g) * T + t) * top_k + lane] : -1;
+      for (int jj = 0; jj < top_k && ok; ++jj) {
+        const int j = __shfl_sync(0xffffffffu, mine, jj);
+        if (j < 0) break;
+        const int jb = min(j, t / kBlk);
+        const int slot = (int)(fill % kSlots);
+        ok = tc::mbar_wait(empty + slot, (uint32_t)(((fill / kSlots) & 1) ^ 1), err, 21);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0) {
+          uint8_t* dst = smem + SM::kRing + slot * SM::kSlotBytes;
+          tc::mbar_expect_tx(full + slot, SM::kSlotBytes);
+          for (int s = 0; s < DK / 64; ++s)
+            tc::tma_load_3d(dst + s * kBox, &tm_k, full + slot, s * 64, g, b * T + jb * kBlk);
+          for (int s = 0; s < DV / 64; ++s)
+            tc::tma_load_3d(dst + (DK / 64 + s) * kBox, &tm_v, full + slot, s * 64, g, b * T + jb * kBlk);
+        }
+        __syncwarp();
+        ++fill;
+      }
+    }
+    if (lane == 0)
+      for (long f = fill - 1; f >= 0 && f >= fill - kSlots; --f)   // let copies in flight land
+        tc::mbar_wait(full + (f % kSlots), (uint32_t)((f / kSlots) & 1), err, 22);
+  } else {
+    // ---------------------------------------------------------------- consumers
+    const int gl = lane >> 2, cq = lane & 3;
+    float* sO = reinterpret_cast<float*>(smem + SM::kMerge);
+    float* sML = sO + kConsumers * 16 * DV;
+    long use = 0;
+    bool ok = true;
+    for (long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+      const int g = (int)(it / ((long)B * T));
+      const int bt = (int)(it % ((long)B * T));
+      const int b = bt / T, t = bt % T;
+      const int mine = lane < top_k ? idx[(((size_t)b * Hkv + g) * T + t) * top_k + lane] : -1;
+      const bool rv0 = gl < G, rv1 = gl + 8 < G;
+      uint32_t qf[DK / 16][4];
+      {
+        const __nv_bfloat16* q0 = q + (((size_t)b * T + t) * Hq + g * G + gl) * DK;
+        const __nv_bfloat16* q1 = q0 + 8 * DK;
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          qf[ks][0] = rv0 ? ld_u32(q0 + ks * 16 + 2 * cq) : 0u;
+          qf[ks][1] = rv1 ? ld_u32(q1 + ks * 16 + 2 * cq) : 0u;
+          qf[ks][2] = rv0 ? ld_u32(q0 + ks * 16 + 8 + 2 * cq) : 0u;
+          qf[ks][3] = rv1 ? ld_u32(q1 + ks * 16 + 8 + 2 * cq) : 0u;
+        }
+      }
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+      float o[DV / 8][4];
+#pragma unroll
+      for (int j = 0; j < DV / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+      for (int jj = 0; jj < top_k; ++jj) {
+        const int j = __shfl_sync(0xffffffffu, mine, jj);
+        if (j < 0) break;
+        const int jb = min(j, t / kBlk);
+        const int slot = (int)(use % kSlots);
+        ok = tc::mbar_wait(full + slot, (uint32_t)((use / kSlots) & 1), err, 23);
+        ok = __all_sync(0xffffffffu, ok);   // reconverge the warp before ldmatrix / mma
+        if (!ok) break;
+        const uint8_t* kb = smem + SM::kRing + slot * SM::kSlotBytes;
+        const uint8_t* vb = kb + (DK / 64) * kBox;
+        const int u0 = jb * kBlk + warp * 16;      // this warp's 16 keys
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int ks = 0; ks < DK / 16; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          const int row = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int c = 2 * (ks & 3) + ((lane >> 3) & 1);
+          ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (ks >> 2) * kBox + swz(row, c)));
+          mma16816(s[0], qf[ks], b0, b1);
+          mma16816(s[1], qf[ks], b2, b3);
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int u = u0 + x * 8 + 2 * cq + e;
+            const bool vis = u <= t;
+            s[x][e] = vis ? s[x][e] * scale_log2 : -INFINITY;
+            s[x][2 + e] = vis ? s[x][2 + e] * scale_log2 : -INFINITY;
+            mx0 = fmaxf(mx0, s[x][e]);
+            mx1 = fmaxf(mx1, s[x][2 + e]);
+          }
+        mx0 = warp_max4(mx0);
+        mx1 = warp_max4(mx1);
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        const float base0 = n0 == -INFINITY ? 0.f : n0, base1 = n1 == -INFINITY ? 0.f : n1;
+        const float c0 = exp2f(m0 - base0), c1 = exp2f(m1 - base1);
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int x = 0; x < 2; ++x)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            s[x][e] = exp2f(s[x][e] - base0);
+            s[x][2 + e] = exp2f(s[x][2 + e] - base1);
+            sum0 += s[x][e];
+            sum1 += s[x][2 + e];
+          }
+        l0 = l0 * c0 + warp_sum4(sum0);
+        l1 = l1 * c1 + warp_sum4(sum1);
+        m0 = n0;
+        m1 = n1;
+#pragma unroll
+        for (int x = 0; x < DV / 8; ++x) {
+          o[x][0] *= c0; o[x][1] *= c0; o[x][2] *= c1; o[x][3] *= c1;
+        }
+        uint32_t a[4];
+        a[0] = pack_bf16(s[0][0], s[0][1]);
+        a[1] = pack_bf16(s[0][2], s[0][3]);
+        a[2] = pack_bf16(s[1][0], s[1][1]);
+        a[3] = pack_bf16(s[1][2], s[1][3]);
+#pragma unroll
+        for (int np = 0; np < DV / 16; ++np) {
+          uint32_t b0, b1, b2, b3;
+          const int row = warp * 16 + (lane & 15);
+          const int c = 2 * (np & 3) + (lane >> 4);
+          ldsm_x4_t(b0, b1, b2, b3, smem_u32(vb + (np >> 2) * kBox + swz(row, c)));
+          mma16816(o[2 * np], a, b0, b1);
+          mma16816(o[2 * np + 1], a, b2, b3);
+        }
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty + slot);
+        ++use;
+      }
+      ok = vote_all(1, kConsumers * 32, ok);
+      if (!ok) break;
+      // merge the four warps' partial states: warp w owns value columns [w*DV/4, (w+1)*DV/4)
+      {
+        constexpr int kNt = DV / 8 / kConsumers;            // n-tiles (8 columns) per owned slice
+        float* sX = reinterpret_cast<float*>(smem + SM::kMerge);
+        float* sMl = sX + kConsumers * 3 * 16 * (DV / 4);
+        auto xaddr = [&](int writer, int owner, int row, int col_in_slice) {
+          const int slot = owner - (owner > writer);      // owner's position among the writer's three peers
+          return sX + (((writer * 3 + slot) * 16 + row) * (DV / 4) + col_in_slice);
+        };
+#pragma unroll
+        for (int x = 0; x < DV / 8; ++x) {
+          const int owner = x / kNt;
+          if (owner == warp) continue;
+          const int cs = (x % kNt) * 8 + 2 * cq;
+          *reinterpret_cast<float2*>(xaddr(warp, owner, gl, cs)) = make_float2(o[x][0], o[x][1]);
+          *reinterpret_cast<float2*>(xaddr(warp, owner, gl + 8, cs)) = make_float2(o[x][2], o[x][3]);
+        }
+        if (cq == 0) {
+          sMl[(warp * 16 + gl) * 2] = m0;
+          sMl[(warp * 16 + gl) * 2 + 1] = l0;
+          sMl[(warp * 16 + gl + 8) * 2] = m1;
+          sMl[(warp * 16 + gl + 8) * 2 + 1] = l1;
+        }
+        // the accumulator values this lane updates (prefetched before the barrier)
+        const size_t row0 = ((size_t)b * T + t) * Hq + g * G;
+        float2 prev[2][kNt];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int xx = 0; xx < kNt; ++xx) {
+            const int r = gl + 8 * hh;
+            const int c = warp * (DV / 4) + xx * 8 + 2 * cq;
+            prev[hh][xx] = r < G ? *reinterpret_cast<const float2*>(acc + (row0 + r) * DV + c) : make_float2(0.f, 0.f);
+          }
+        named_sync(1, kConsumers * 32);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int r = gl + 8 * hh;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sMl[(w * 16 + r) * 2]);
+          float f[kConsumers], L = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumers; ++w) {
+            f[w] = M == -INFINITY ? 0.f : exp2f(sMl[(w * 16 + r) * 2] - M);
+            L += f[w] * sMl[(w * 16 + r) * 2 + 1];
+          }
+          if (r >= G) continue;
+          const float gs = __bfloat162float(gates[(row0 + r) * 3 + 1]);
+          const float scl = L > 0.f ? gs / L : 0.f;
+          float fw = f[0];
+#pragma unroll
+          for (int w = 1; w < kConsumers; ++w) fw = w == warp ? f[w] : fw;
+#pragma unroll
+          for (int x = 0; x < DV / 8; ++x) {
+            if (x / kNt != warp) continue;               // x stays a compile-time index into o
+            const int xx = x % kNt;
+            const int cs = xx * 8 + 2 * cq;
+            float ox = fw * o[x][2 * hh], oy = fw * o[x][2 * hh + 1];
+#pragma unroll
+            for (int w = 0; w < kConsumers; ++w) {
+              if (w == warp) continue;
+              const float2 pv = *reinterpret_cast<const float2*>(xaddr(w, warp, r, cs));
+              ox += f[w] * pv.x;
+              oy += f[w] * pv.y;
+            }
+            const int c = warp * (DV / 4) + cs;
+            float2 pr = prev[hh][0];
+#pragma unroll
+            for (int y = 1; y < kNt; ++y) pr = y == xx ? prev[hh][y] : pr;
+            *reinterpret_cast<float2*>(acc + (row0 + r) * DV + c) = make_float2(pr.x + scl * ox, pr.y + scl * oy);
+          }
+        }
+      }
+      named_sync(1, kConsumers * 32);
+    }
+  }
+  __syncthreads();
+}
+
+template <int DK, int DV>
+cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
+  using SM = Smem<DK, DV>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(slc_attn_tma_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap mk, mv;
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
+  const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
+  const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
+  const uint32_t box[3] = {64, 1, kBlk};
+  if (!make_tmap_bf16(&mk, a.k, 3, dk3, sk3, box) || !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, box))
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long total = (long)a.Hkv * a.B * a.T;
+  const int grid = (int)(total < (long)sms * kCtasPerSm ? total : (long)sms * kCtasPerSm);
+  slc_attn_tma_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
+      mk, mv, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B,
+      a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, a.err);
+  return cudaGetLastError();
+}
+}  // namespace
+
+bool slc_attn_tma_supported(const FwdArgs& a) {
+  return a.err != nullptr && a.G <= 16 && (a.dk == 64 || a.dk == 128 || a.dk == 192) && (a.dv == 64 || a.dv == 128);
+}
+
+cudaError_t launch_slc_attn_tma(const FwdArgs& a, cudaStream_t st) {
+  if (a.dk == 192 && a.dv == 128) return launch_tma<192, 128>(a, st);
+  if (a.dk == 128 && a.dv == 128) return launch_tma<128, 128>(a, st);
+  if (a.dk == 64 && a.dv == 64) return launch_tma<64, 64>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nsa

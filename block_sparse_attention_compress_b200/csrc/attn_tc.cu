@@ -1,4 +1,4 @@
-// K2 on the 5th-generation tensor cores: compressed attention + group-summed block
+// K2 and K4 on the 5th-generation tensor cores.  K2: compressed attention + group-summed block
 // scores + top-k ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5, §8; "一文比较 Kimi 和
 // Deepseek 的两篇稀疏注意力机制论文", "Deepseek 的论文核心点": the selection scores come
 // from the compressed attention and the group's heads add them before one top-k).
@@ -84,12 +84,16 @@ __device__ __forceinline__ bool vote_all(int id, int n, bool pred) {
   return r != 0;
 }
 
-template <int DK, int DV>
+// kWin = false: compressed branch (keys = compressed blocks, scores + top-k, acc = g_cmp * o).
+// kWin = true:  sliding window (keys = tokens [t0-w+1, t0+7], each row masked to its own
+//               window, out = bf16(acc + g_win * o)).
+template <int DK, int DV, bool kWin>
 __global__ void __launch_bounds__(kThreads, 1)
-cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
-                     const __grid_constant__ CUtensorMap tm_vc, const __nv_bfloat16* __restrict__ gates,
-                     float* __restrict__ acc, int32_t* __restrict__ idx_out, int T, int Hq, int Hkv, int nc, int top_k,
-                     int force_first, int force_local, float scale_log2, int* __restrict__ err) {
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
+               const __grid_constant__ CUtensorMap tm_vc, const __nv_bfloat16* __restrict__ gates,
+               float* __restrict__ acc, int32_t* __restrict__ idx_out, __nv_bfloat16* __restrict__ out, int T, int Hq,
+               int Hkv, int nc, int top_k, int force_first, int force_local, int window, float scale_log2,
+               int* __restrict__ err) {
   using SM = Smem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -118,7 +122,10 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int t0 = (n_tok_tiles - 1 - (int)blockIdx.x) * kTok;   // longest rows first
   const int g = blockIdx.y, b = blockIdx.z;
   const int t_last = min(t0 + kTok - 1, T - 1);
-  const int ntiles = (n_visible(t_last, nc) + kBlk - 1) / kBlk;
+  // keys: compressed blocks 0.. (kWin = false) or tokens kv_lo.. (kWin = true)
+  const int kv_lo = kWin ? max(0, t0 - window + 1) : 0;
+  const int ntiles = kWin ? (t_last - kv_lo + kBlk) / kBlk : (n_visible(t_last, nc) + kBlk - 1) / kBlk;
+  const int kv_rows = kWin ? T : nc;   // rows per batch in the key/value tensor maps
 
   if (tid == 0) {
     tc::mbar_init(bar_q, 1);
@@ -155,7 +162,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       bool ok = true;
       for (int pass = 0; pass < 2 && ok; ++pass) {
         for (int n = 0; n < ntiles && ok; ++n) {
-          const int row = b * nc + n * kBlk;
+          const int row = b * kv_rows + kv_lo + n * kBlk;
           for (int s = 0; s < SM::kQSlices && ok; ++s, ++fill) {
             const int slot = fill % kKcSlots;
             ok = tc::mbar_wait(kc_empty + slot, ((fill / kKcSlots) & 1) ^ 1, err, kErrKcEmpty);
@@ -235,20 +242,25 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
     const int my_tok = r / 16;                   // pass A: this thread's row = (token, head)
     const int my_t = t0 + my_tok;
-    const int my_nvis = my_t < T ? n_visible(my_t, nc) : 0;
-    int nvis_tok[kTok], nb_tok[kTok];   // visible compressed blocks and eligible selection blocks per token
+    // key range of this row: compressed blocks [0, my_hi) or tokens [my_lo, my_hi)
+    const int my_lo = kWin ? max(0, my_t - window + 1) : 0;
+    const int my_hi = my_t < T ? (kWin ? my_t + 1 : n_visible(my_t, nc)) : 0;
+    int lo_tok[kTok], hi_tok[kTok], nb_tok[kTok];   // key range per token; eligible selection blocks
 #pragma unroll
     for (int k = 0; k < kTok; ++k) {
-      nvis_tok[k] = (t0 + k < T) ? n_visible(t0 + k, nc) : 0;
-      nb_tok[k] = (t0 + k < T) ? (t0 + k) / kSel + 1 : 0;
+      const bool in = t0 + k < T;
+      lo_tok[k] = kWin ? max(0, t0 + k - window + 1) : 0;
+      hi_tok[k] = in ? (kWin ? t0 + k + 1 : n_visible(t0 + k, nc)) : 0;
+      nb_tok[k] = in ? (t0 + k) / kSel + 1 : 0;
     }
     bool ok = true;
     int use = 0;
     // gates of the 128 rows (g_cmp), zeroed scores
     {
       const int t = t0 + my_tok, h = g * 16 + (r % 16);
-      sGate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3]) : 0.f;
-      for (int i = r; i < kTok * kMaxSel; i += 128) sScore[i] = 0.f;
+      sGate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3 + (kWin ? 2 : 0)]) : 0.f;
+      if (!kWin)
+        for (int i = r; i < kTok * kMaxSel; i += 128) sScore[i] = 0.f;
     }
     // pass A: log-sum-exp of this thread's row
     float m = -INFINITY, l = 0.f;
@@ -268,8 +280,8 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         float cm = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int i = n * kBlk + c0 + j;
-          v[j] = i < my_nvis ? v[j] * scale_log2 : -INFINITY;
+          const int i = kv_lo + n * kBlk + c0 + j;
+          v[j] = (i >= my_lo && i < my_hi) ? v[j] * scale_log2 : -INFINITY;
           cm = fmaxf(cm, v[j]);
         }
         const float mn = fmaxf(m, cm);
@@ -297,7 +309,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       if (!ok) break;
       tc::tc_fence_after();
       const uint32_t base = lane_addr + (sb ? kColS1 : kColS0);
-      const int i = n * kBlk + r;                // this thread's compressed block
+      const int i = kv_lo + n * kBlk + r;        // this thread's key (compressed block or token)
       float tok_sum[kTok];
       uint8_t* prow0 = sP + r * 128;             // N-block 0 (rows 0..63 of the query tile)
       uint8_t* prow1 = sP + kSlice + r * 128;    // N-block 1 (rows 64..127)
@@ -306,7 +318,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         float v[16];
         tc::tmem_ld16(base + k * 16, v);
         tc::tmem_wait_ld();
-        const bool vis = i < nvis_tok[k];
+        const bool vis = i >= lo_tok[k] && i < hi_tok[k];
         float s = 0.f;
         uint32_t pk[8];
 #pragma unroll
@@ -317,7 +329,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
           pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
         }
-        tok_sum[k] = s;
+        if (!kWin) tok_sum[k] = s;
         // columns k*16 .. k*16+15 are chunks 2*(k%4), 2*(k%4)+1 of N-block k/4
         uint8_t* prow = (k < 4) ? prow0 : prow1;
         const int c0 = 2 * (k & 3);
@@ -331,6 +343,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tc::mbar_arrive(s_empty + sb);
         tc::mbar_arrive(p_full);
       }
+      if (kWin) continue;
       // selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Phase 1: each group
       // of four lanes adds its own four blocks plus the lane just below it; phase 2: lane 31
       // hands its block (i % 4 == 3) to the first selection block of the next warp or tile.
@@ -357,7 +370,7 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
     // top-k: warp wq takes tokens wq and wq+4
     const int wq = warp - 4;
-    for (int k = wq; k < kTok && ok; k += 4) {
+    for (int k = wq; k < kTok && ok && !kWin; k += 4) {
       const int t = t0 + k;
       if (t >= T) continue;
       const float* score = sScore + k * kMaxSel;
@@ -424,7 +437,8 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const size_t row = ((size_t)b * T + t) * Hq + g * 16 + j;
-            acc[row * DV + r] = sGate[c0 + j] * v[j];
+            if (kWin) out[row * DV + r] = __float2bfloat16_rn(acc[row * DV + r] + sGate[c0 + j] * v[j]);
+            else acc[row * DV + r] = sGate[c0 + j] * v[j];
           }
         }
       }
@@ -439,37 +453,40 @@ cmp_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   }
 }
 
-template <int DK, int DV>
+template <int DK, int DV, bool kWin>
 cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   using SM = Smem<DK, DV>;
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(cmp_select_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV, kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::kAlloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  CUtensorMap mq, mkc, mvc;
+  const int rows = kWin ? a.T : a.nc;
+  const void* kp = kWin ? a.k : a.kc;
+  const void* vp = kWin ? a.v : a.vc;
+  CUtensorMap mq, mk, mv;
   const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
   const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
   const uint32_t bq[3] = {64, 16, kTok};
-  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * rows};
   const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
-  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * rows};
   const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
   const uint32_t bkv[3] = {64, 1, kBlk};
   if (!make_tmap_bf16(&mq, a.q, 3, dq, sq, bq)) return cudaErrorInvalidValue;
-  if (a.nc > 0) {
-    if (!make_tmap_bf16(&mkc, a.kc, 3, dk3, sk3, bkv) || !make_tmap_bf16(&mvc, a.vc, 3, dv3, sv3, bkv))
+  if (rows > 0) {
+    if (!make_tmap_bf16(&mk, kp, 3, dk3, sk3, bkv) || !make_tmap_bf16(&mv, vp, 3, dv3, sv3, bkv))
       return cudaErrorInvalidValue;
   } else {
-    mkc = mq;   // never dereferenced: no tile is loaded when there is no compressed block
-    mvc = mq;
+    mk = mq;   // never dereferenced: no tile is loaded when there is no key
+    mv = mq;
   }
   dim3 grid((a.T + kTok - 1) / kTok, a.Hkv, a.B);
-  cmp_select_tc_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
-      mq, mkc, mvc, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, a.T, a.Hq, a.Hkv, a.nc, a.top_k,
-      a.force_first, a.force_local, a.scale_log2, a.err);
+  attn_tc_kernel<DK, DV, kWin><<<grid, kThreads, SM::kAlloc, st>>>(
+      mq, mk, mv, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, static_cast<__nv_bfloat16*>(a.out), a.T,
+      a.Hq, a.Hkv, a.nc, a.top_k, a.force_first, a.force_local, a.window, a.scale_log2, a.err);
   return cudaGetLastError();
 }
 }  // namespace
@@ -479,8 +496,15 @@ bool cmp_select_tc_supported(const FwdArgs& a) {
 }
 
 cudaError_t launch_cmp_select_tc(const FwdArgs& a, cudaStream_t st) {
-  if (a.dk == 192) return launch_tc<192, 128>(a, st);
-  return launch_tc<128, 128>(a, st);
+  if (a.dk == 192) return launch_tc<192, 128, false>(a, st);
+  return launch_tc<128, 128, false>(a, st);
+}
+
+bool swa_tc_supported(const FwdArgs& a) { return cmp_select_tc_supported(a); }
+
+cudaError_t launch_swa_tc(const FwdArgs& a, cudaStream_t st) {
+  if (a.dk == 192) return launch_tc<192, 128, true>(a, st);
+  return launch_tc<128, 128, true>(a, st);
 }
 
 }  // namespace nsa

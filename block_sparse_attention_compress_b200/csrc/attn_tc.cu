@@ -16,8 +16,9 @@
 //            (rows = value dims), already normalised, so no rescaling is ever needed.
 //   top-k    per token over the selection-block scores in shared memory.
 //   epilogue acc[t, h, :] = g_cmp * o_cmp, read from O^T (each thread one value dim).
-// Warp roles: 0 TMA producer, 1 MMA issuer (and TMEM owner), 4-7 softmax / epilogue
-// (warp 4+q owns TMEM lanes 32q..32q+31).  Every wait is bounded (see tc.cuh); on a
+// Warp roles: 8 TMA producer, 9 MMA issuer (and TMEM owner), 0-7 softmax / epilogue in
+// two groups of four (warp w owns TMEM lanes 32*(w%4)..+31; group w/4 takes one half of
+// every tile's 128 columns: in the second pass that half is exactly four tokens).  Every wait is bounded (see tc.cuh); on a
 // timeout the kernel records an error word, stops issuing work, and frees its TMEM.
 #include <cfloat>
 
@@ -27,7 +28,9 @@
 namespace nsa {
 
 namespace {
-constexpr int kThreads = 256;
+constexpr int kSoftWarps = 8;                 // two groups of four softmax warps
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kTok = 8;            // tokens per CTA
 constexpr int kRowsM = 128;        // query rows per CTA (8 tokens x 16 heads)
 constexpr int kBlk = 128;          // compressed blocks per tile
@@ -51,6 +54,7 @@ struct Smem {
   static constexpr uint32_t kScore = kP + 2 * kSlice;                       // [8][1024] fp32
   static constexpr uint32_t kLse = kScore + kTok * kMaxSel * 4;             // [128] fp32
   static constexpr uint32_t kGate = kLse + kRowsM * 4;                      // [128] fp32
+  static constexpr uint32_t kML = kP;                                       // [2][128][2] fp32, while P^T is unused
   static constexpr uint32_t kBar = kGate + kRowsM * 4;                      // mbarriers
   static constexpr int kNumBars = 1 + 2 * kKcSlots + 2 * 2 + 2 * 2 + 2 + 1;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
@@ -104,6 +108,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   float* sScore = reinterpret_cast<float*>(smem + SM::kScore);
   float* sLse = reinterpret_cast<float*>(smem + SM::kLse);
   float* sGate = reinterpret_cast<float*>(smem + SM::kGate);
+  float* sML = reinterpret_cast<float*>(smem + SM::kML);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* bar_q = bars;
   uint64_t* kc_full = bars + 1;
@@ -134,14 +139,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(vc_full + i, 1);
       tc::mbar_init(vc_empty + i, 1);
       tc::mbar_init(s_full + i, 1);
-      tc::mbar_init(s_empty + i, 4);
+      tc::mbar_init(s_empty + i, kSoftWarps);
     }
-    tc::mbar_init(p_full, 4);
+    tc::mbar_init(p_full, kSoftWarps);
     tc::mbar_init(p_empty, 1);
     tc::mbar_init(o_full, 1);
     tc::fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc::tmem_alloc(tmem_slot, kTmemCols);
     tc::tmem_relinquish();
   }
@@ -150,7 +155,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
+  if (warp == kTmaWarp) {
     // ------------------------------------------------------------ TMA producer
     if (tc::elect_one()) {
       tc::prefetch_tmap(&tm_q);
@@ -187,7 +192,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (tc::elect_one()) {
       const uint32_t idA = tc::idesc_bf16(128, 128, 0, 0);     // S  = Q  Kc^T   (both K-major)
@@ -236,51 +241,48 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
       if (ok && ntiles > 0) tc::mma_commit(o_full);
     }
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int r = tid - 128;                     // TMEM lane owned by this thread
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp - 4)) << 16);
-    const int my_tok = r / 16;                   // pass A: this thread's row = (token, head)
-    const int my_t = t0 + my_tok;
-    // key range of this row: compressed blocks [0, my_hi) or tokens [my_lo, my_hi)
-    const int my_lo = kWin ? max(0, my_t - window + 1) : 0;
-    const int my_hi = my_t < T ? (kWin ? my_t + 1 : n_visible(my_t, nc)) : 0;
-    int lo_tok[kTok], hi_tok[kTok], nb_tok[kTok];   // key range per token; eligible selection blocks
-#pragma unroll
-    for (int k = 0; k < kTok; ++k) {
-      const bool in = t0 + k < T;
-      lo_tok[k] = kWin ? max(0, t0 + k - window + 1) : 0;
-      hi_tok[k] = in ? (kWin ? t0 + k + 1 : n_visible(t0 + k, nc)) : 0;
-      nb_tok[k] = in ? (t0 + k) / kSel + 1 : 0;
-    }
+    // Two groups of four warps; group gr takes columns [64*gr, 64*gr+64) of every tile.
+    // Warp quarter q = warp % 4 owns TMEM lanes 32q..32q+31; r is this thread's lane.
+    const int gr = warp >> 2, q4 = warp & 3;
+    const int r = 32 * q4 + lane;
+    const int col0 = 64 * gr;
+    const int gbar = 1 + gr;                     // named barrier of this group (128 threads)
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
     bool ok = true;
     int use = 0;
-    // gates of the 128 rows (g_cmp), zeroed scores
-    {
-      const int t = t0 + my_tok, h = g * 16 + (r % 16);
+    if (gr == 0) {   // gates of the 128 rows
+      const int t = t0 + r / 16, h = g * 16 + (r % 16);
       sGate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3 + (kWin ? 2 : 0)]) : 0.f;
-      if (!kWin)
-        for (int i = r; i < kTok * kMaxSel; i += 128) sScore[i] = 0.f;
     }
-    // pass A: log-sum-exp of this thread's row
-    float m = -INFINITY, l = 0.f;
-    for (int n = 0; n < ntiles && ok; ++n, ++use) {
-      const int sb = use & 1;
-      ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
-      ok = __all_sync(0xffffffffu, ok);   // reconverge before the warp-wide TMEM loads
-      if (!ok) break;
-      tc::tc_fence_after();
-      const uint32_t base = lane_addr + (sb ? kColS1 : kColS0);
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
-        float v[32];
-        tc::tmem_ld16(base + c0, *reinterpret_cast<float(*)[16]>(v));
-        tc::tmem_ld16(base + c0 + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+    if (!kWin)
+      for (int i = gr * 128 + r; i < kTok * kMaxSel; i += 256) sScore[i] = 0.f;
+
+    // pass A: this thread's row r = (token r/16, head r%16), its half of every tile's columns
+    {
+      const int my_t = t0 + r / 16;
+      const int my_lo = kWin ? max(0, my_t - window + 1) : 0;
+      const int my_hi = my_t < T ? (kWin ? my_t + 1 : n_visible(my_t, nc)) : 0;
+      float m = -INFINITY, l = 0.f;
+      for (int n = 0; n < ntiles && ok; ++n, ++use) {
+        const int sb = use & 1;
+        ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+        ok = __all_sync(0xffffffffu, ok);      // reconverge before the warp-wide TMEM loads
+        if (!ok) break;
+        tc::tc_fence_after();
+        const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
+        float v[64];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
         tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(s_empty + sb);
         float cm = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int i = kv_lo + n * kBlk + c0 + j;
+        for (int j = 0; j < 64; ++j) {
+          const int i = kv_lo + n * kBlk + col0 + j;
           v[j] = (i >= my_lo && i < my_hi) ? v[j] * scale_log2 : -INFINITY;
           cm = fmaxf(cm, v[j]);
         }
@@ -288,54 +290,70 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (mn != -INFINITY) {
           float sum = 0.f;
 #pragma unroll
-          for (int j = 0; j < 32; ++j) sum += ex2(v[j] - mn);
+          for (int j = 0; j < 64; ++j) sum += ex2(v[j] - mn);
           l = l * ex2(m - mn) + sum;
           m = mn;
         }
       }
-      tc::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(s_empty + sb);
+      sML[(gr * 128 + r) * 2] = m;
+      sML[(gr * 128 + r) * 2 + 1] = l;
     }
-    sLse[r] = (my_t < T && l > 0.f) ? m + __log2f(l) : INFINITY;
-    named_sync(1, 128);
-    // pass B: probabilities, P^T, block scores
-    ok = vote_all(1, 128, ok);
-    for (int n = 0; n < ntiles && ok; ++n, ++use) {
+    ok = vote_all(3, kSoftWarps * 32, ok);
+    if (gr == 0) {
+      const float m0 = sML[r * 2], l0 = sML[r * 2 + 1], m1 = sML[(128 + r) * 2], l1 = sML[(128 + r) * 2 + 1];
+      const float M = fmaxf(m0, m1);
+      const float L = M == -INFINITY ? 0.f : l0 * ex2(m0 - M) + l1 * ex2(m1 - M);
+      sLse[r] = (t0 + r / 16 < T && L > 0.f) ? M + __log2f(L) : INFINITY;
+    }
+    named_sync(3, kSoftWarps * 32);
+
+    // pass B: this thread's key r of every tile; columns = tokens 4*gr .. 4*gr+3, 16 heads each
+    int lo_tok[4], hi_tok[4], nb_tok[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int t = t0 + 4 * gr + k;
+      const bool in = t < T;
+      lo_tok[k] = kWin ? max(0, t - window + 1) : 0;
+      hi_tok[k] = in ? (kWin ? t + 1 : n_visible(t, nc)) : 0;
+      nb_tok[k] = in ? t / kSel + 1 : 0;
+    }
+    uint8_t* prow = sP + gr * kSlice + r * 128;   // row r of N-block gr of P^T
+    for (int n = 0; n < ntiles; ++n, ++use) {
       const int sb = use & 1;
-      ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
-      if (ok && n > 0) ok = tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty);
-      ok = vote_all(1, 128, ok);
+      if (ok) ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+      ok = vote_all(3, kSoftWarps * 32, ok);   // all eight warps leave together or not at all
       if (!ok) break;
       tc::tc_fence_after();
-      const uint32_t base = lane_addr + (sb ? kColS1 : kColS0);
-      const int i = kv_lo + n * kBlk + r;        // this thread's key (compressed block or token)
-      float tok_sum[kTok];
-      uint8_t* prow0 = sP + r * 128;             // N-block 0 (rows 0..63 of the query tile)
-      uint8_t* prow1 = sP + kSlice + r * 128;    // N-block 1 (rows 64..127)
+      const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
+      float v[64];
 #pragma unroll
-      for (int k = 0; k < kTok; ++k) {
-        float v[16];
-        tc::tmem_ld16(base + k * 16, v);
-        tc::tmem_wait_ld();
+      for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+      tc::tmem_wait_ld();
+      const int i = kv_lo + n * kBlk + r;        // this thread's key (compressed block or token)
+      float tok_sum[4];
+      uint32_t pk[32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
         const bool vis = i >= lo_tok[k] && i < hi_tok[k];
         float s = 0.f;
-        uint32_t pk[8];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
-          const float p0 = vis ? ex2(v[j] * scale_log2 - sLse[k * 16 + j]) : 0.f;
-          const float p1 = vis ? ex2(v[j + 1] * scale_log2 - sLse[k * 16 + j + 1]) : 0.f;
+          const float p0 = vis ? ex2(v[16 * k + j] * scale_log2 - sLse[col0 + 16 * k + j]) : 0.f;
+          const float p1 = vis ? ex2(v[16 * k + j + 1] * scale_log2 - sLse[col0 + 16 * k + j + 1]) : 0.f;
           s += p0 + p1;
           __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+          pk[8 * k + j / 2] = *reinterpret_cast<uint32_t*>(&h2);
         }
-        if (!kWin) tok_sum[k] = s;
-        // columns k*16 .. k*16+15 are chunks 2*(k%4), 2*(k%4)+1 of N-block k/4
-        uint8_t* prow = (k < 4) ? prow0 : prow1;
-        const int c0 = 2 * (k & 3);
-        *reinterpret_cast<uint4*>(prow + ((c0 ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        *reinterpret_cast<uint4*>(prow + (((c0 + 1) ^ (r & 7)) << 4)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        tok_sum[k] = s;
       }
+      // P^T(n) may overwrite the buffer once PV(n-1) has read it (a timeout here is
+      // carried to the vote at the top of the next tile, so no warp leaves early)
+      if (n > 0) ok = tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty);
+      ok = __all_sync(0xffffffffu, ok);
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       tc::tc_fence_before();
       tc::fence_async_smem();
       __syncwarp();
@@ -347,99 +365,107 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Phase 1: each group
       // of four lanes adds its own four blocks plus the lane just below it; phase 2: lane 31
       // hands its block (i % 4 == 3) to the first selection block of the next warp or tile.
-      const int wq = warp - 4;
-      const int j0 = n * (kBlk / 4) + wq * 8;    // first selection block of this warp
+      const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
 #pragma unroll
-      for (int k = 0; k < kTok; ++k) {
-        const float v = tok_sum[k];
-        float g4 = v + __shfl_xor_sync(0xffffffffu, v, 1);
+      for (int k = 0; k < 4; ++k) {
+        const float vv = tok_sum[k];
+        float g4 = vv + __shfl_xor_sync(0xffffffffu, vv, 1);
         g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
-        const float prev = __shfl_up_sync(0xffffffffu, v, 1);
+        const float prev = __shfl_up_sync(0xffffffffu, vv, 1);
         const int j = j0 + (lane >> 2);
-        if ((lane & 3) == 0 && j < nb_tok[k]) sScore[k * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
+        if ((lane & 3) == 0 && j < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
       }
-      named_sync(1, 128);
+      named_sync(gbar, 128);
       if (lane == 31) {
 #pragma unroll
-        for (int k = 0; k < kTok; ++k)
-          if (j0 + 8 < nb_tok[k]) sScore[k * kMaxSel + j0 + 8] += tok_sum[k];
+        for (int k = 0; k < 4; ++k)
+          if (j0 + 8 < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + j0 + 8] += tok_sum[k];
       }
-      named_sync(1, 128);
+      named_sync(gbar, 128);
     }
-    named_sync(1, 128);
+    named_sync(3, kSoftWarps * 32);
 
-    // top-k: warp wq takes tokens wq and wq+4
-    const int wq = warp - 4;
-    for (int k = wq; k < kTok && ok && !kWin; k += 4) {
+    // top-k: warp w takes token w
+    if (!kWin && ok) {
+      const int k = warp;
       const int t = t0 + k;
-      if (t >= T) continue;
-      const float* score = sScore + k * kMaxSel;
-      const int nb = t / kSel + 1;
-      int32_t* dst = idx_out + (((size_t)b * Hkv + g) * T + t) * top_k;
-      if (nb <= top_k) {
-        for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
-        continue;
-      }
-      const int own = t / kSel;
-      uint32_t taken = 0;
-      int nforced = 0;
-      if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
-      if (force_local && !(force_first && own == 0)) {
-        if (lane == (own & 31)) taken |= 1u << (own >> 5);
-        ++nforced;
-      }
-      const int mmax = (nb + 31) >> 5;
-      for (int rr = nforced; rr < top_k; ++rr) {
-        float bs = -FLT_MAX;
-        int bj = 0x7fffffff;
-        for (int mm = 0; mm < mmax; ++mm) {
-          const int j = lane + 32 * mm;
-          if (j < nb && !((taken >> mm) & 1u)) {
-            const float sc = score[j];
-            if (sc > bs) { bs = sc; bj = j; }
+      if (t < T) {
+        const float* score = sScore + k * kMaxSel;
+        const int nb = t / kSel + 1;
+        int32_t* dst = idx_out + (((size_t)b * Hkv + g) * T + t) * top_k;
+        if (nb <= top_k) {
+          for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
+        } else {
+          const int own = t / kSel;
+          uint32_t taken = 0;
+          int nforced = 0;
+          if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
+          if (force_local && !(force_first && own == 0)) {
+            if (lane == (own & 31)) taken |= 1u << (own >> 5);
+            ++nforced;
           }
-        }
+          const int mmax = (nb + 31) >> 5;
+          for (int rr = nforced; rr < top_k; ++rr) {
+            float bs = -FLT_MAX;
+            int bj = 0x7fffffff;
+            for (int mm = 0; mm < mmax; ++mm) {
+              const int j = lane + 32 * mm;
+              if (j < nb && !((taken >> mm) & 1u)) {
+                const float sc = score[j];
+                if (sc > bs) { bs = sc; bj = j; }
+              }
+            }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-          const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-          if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; }
+            for (int off = 16; off > 0; off >>= 1) {
+              const float os = __shfl_xor_sync(0xffffffffu, bs, off);
+              const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
+              if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; }
+            }
+            if (bj != 0x7fffffff && lane == (bj & 31)) taken |= 1u << (bj >> 5);
+          }
+          int pos = 0;
+          for (int mm = 0; mm < mmax; ++mm) {
+            const bool sel = (taken >> mm) & 1u;
+            const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+            if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
+            pos += __popc(bal);
+          }
+          for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
         }
-        if (bj != 0x7fffffff && lane == (bj & 31)) taken |= 1u << (bj >> 5);
       }
-      int pos = 0;
-      for (int mm = 0; mm < mmax; ++mm) {
-        const bool sel = (taken >> mm) & 1u;
-        const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-        if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
-        pos += __popc(bal);
-      }
-      for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
     }
 
-    // epilogue: thread r owns value dim r of O^T; column c = (token c/16, head c%16)
+    // epilogue: lane r = value dim r of O^T; this group's 64 columns = tokens 4*gr .. 4*gr+3
+    float prevacc[kWin ? 64 : 1];
+    if (kWin) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int t = t0 + 4 * gr + c / 16;
+        const size_t row = ((size_t)b * T + min(t, T - 1)) * Hq + g * 16 + (c % 16);
+        prevacc[c] = (t < T && r < DV) ? acc[row * DV + r] : 0.f;
+      }
+    }
     if (ok && ntiles > 0) ok = tc::mbar_wait(o_full, 0, err, kErrOFull);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc::tc_fence_after();
-#pragma unroll 1
-      for (int c0 = 0; c0 < kRowsM; c0 += 16) {
-        float v[16];
-        if (ntiles > 0) {
-          tc::tmem_ld16(lane_addr + kColO + c0, v);
-          tc::tmem_wait_ld();
-        } else {
+      float v[64];
+      if (ntiles > 0) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = 0.f;
-        }
-        const int k = c0 / 16, t = t0 + k;
+        for (int c = 0; c < 4; ++c) tc::tmem_ld16(lane_addr + kColO + col0 + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+        tc::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) v[c] = 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const int t = t0 + 4 * gr + c / 16;
         if (t < T && r < DV) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const size_t row = ((size_t)b * T + t) * Hq + g * 16 + j;
-            if (kWin) out[row * DV + r] = __float2bfloat16_rn(acc[row * DV + r] + sGate[c0 + j] * v[j]);
-            else acc[row * DV + r] = sGate[c0 + j] * v[j];
-          }
+          const size_t row = ((size_t)b * T + t) * Hq + g * 16 + (c % 16);
+          const float gv = sGate[col0 + c] * v[c];
+          if (kWin) out[row * DV + r] = __float2bfloat16_rn(prevacc[c] + gv);
+          else acc[row * DV + r] = gv;
         }
       }
     }
@@ -447,7 +473,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, kTmemCols);
   }

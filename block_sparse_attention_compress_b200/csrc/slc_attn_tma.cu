@@ -17,22 +17,24 @@
 namespace nsa {
 
 namespace {
-constexpr int kConsumers = 4;
-constexpr int kThreads = (kConsumers + 1) * 32;
+constexpr int kConsumers = 4;                       // consumer warps per group
+constexpr int kGroups = 2;                          // independent pipelines per CTA
+constexpr int kThreads = kGroups * (kConsumers + 1) * 32;
 constexpr int kBlk = 64;
-constexpr int kSlots = 4;
+constexpr int kSlots = 2;                           // ring slots per group
 constexpr int kCtasPerSm = 1;
 constexpr uint32_t kBox = kBlk * 128;   // one 64-row x 64-column box: 8 KB
 
 template <int DK, int DV>
 struct Smem {
   static constexpr uint32_t kSlotBytes = (DK / 64 + DV / 64) * kBox;
-  static constexpr uint32_t kRing = 0;
-  // merge scratch: every warp leaves, for each of the other three warps, the 32-column
-  // slice that warp owns ([writer][owner slot][16 rows][DV/4]), plus its m and l per row
-  static constexpr uint32_t kMerge = kRing + kSlots * kSlotBytes;
-  static constexpr uint32_t kBar = kMerge + kConsumers * 3 * 16 * (DV / 4) * 4 + kConsumers * 16 * 2 * 4;
-  static constexpr uint32_t kBytes = kBar + 2 * kSlots * 8;
+  static constexpr uint32_t kRing = 0;                                       // [group][slot]
+  // merge scratch per group: every warp leaves, for each of the other three warps, the
+  // column slice that warp owns ([writer][owner slot][16 rows][DV/4]), plus its m, l per row
+  static constexpr uint32_t kScratch = kConsumers * 3 * 16 * (DV / 4) * 4 + kConsumers * 16 * 2 * 4;
+  static constexpr uint32_t kMerge = kRing + kGroups * kSlots * kSlotBytes;
+  static constexpr uint32_t kBar = kMerge + kGroups * kScratch;
+  static constexpr uint32_t kBytes = kBar + kGroups * 2 * kSlots * 8;
   static constexpr uint32_t kAlloc = kBytes + 1024;
   static_assert(kAlloc * kCtasPerSm <= 232448, "shared memory");
 };
@@ -65,20 +67,26 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   using SM = Smem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar);
-  uint64_t* empty = full + kSlots;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp >= kGroups * kConsumers;
+  const int grp = producer ? warp - kGroups * kConsumers : warp / kConsumers;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar) + grp * 2 * kSlots;
+  uint64_t* empty = full + kSlots;
+  uint8_t* ring = smem + SM::kRing + grp * kSlots * SM::kSlotBytes;
   if (tid == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      tc::mbar_init(full + s, 1);
-      tc::mbar_init(empty + s, kConsumers);
-    }
+    uint64_t* all = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+    for (int gg = 0; gg < kGroups; ++gg)
+      for (int s = 0; s < kSlots; ++s) {
+        tc::mbar_init(all + gg * 2 * kSlots + s, 1);
+        tc::mbar_init(all + gg * 2 * kSlots + kSlots + s, kConsumers);
+      }
     tc::fence_barrier_init();
   }
   __syncthreads();
   const long total = (long)Hkv * B * T;
+  const long it0 = (long)blockIdx.x * kGroups + grp, stride = (long)gridDim.x * kGroups;
 
-  if (warp == kConsumers) {
+  if (producer) {
     // ---------------------------------------------------------------- producer
     // (the whole warp runs the loop; lane 0 issues the copies)
     if (lane == 0) {
@@ -87,7 +95,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     long fill = 0;
     bool ok = true;
-    for (long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+    for (long it = it0; it < total && ok; it += stride) {
       const int g = (int)(it / ((long)B * T));
       const int bt = (int)(it % ((long)B * T));
       const int b = bt / T, t = bt % T;
@@ -101,7 +109,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (lane == 0) {
-          uint8_t* dst = smem + SM::kRing + slot * SM::kSlotBytes;
+          uint8_t* dst = ring + slot * SM::kSlotBytes;
           tc::mbar_expect_tx(full + slot, SM::kSlotBytes);
           for (int s = 0; s < DK / 64; ++s)
             tc::tma_load_3d(dst + s * kBox, &tm_k, full + slot, s * 64, g, b * T + jb * kBlk);
@@ -118,11 +126,11 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   } else {
     // ---------------------------------------------------------------- consumers
     const int gl = lane >> 2, cq = lane & 3;
-    float* sO = reinterpret_cast<float*>(smem + SM::kMerge);
-    float* sML = sO + kConsumers * 16 * DV;
+    const int cw = warp % kConsumers;          // consumer warp within the group
+    const int gbar = 1 + grp;                  // named barrier of this group
     long use = 0;
     bool ok = true;
-    for (long it = blockIdx.x; it < total && ok; it += gridDim.x) {
+    for (long it = it0; it < total && ok; it += stride) {
       const int g = (int)(it / ((long)B * T));
       const int bt = (int)(it % ((long)B * T));
       const int b = bt / T, t = bt % T;
@@ -152,14 +160,14 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         ok = tc::mbar_wait(full + slot, (uint32_t)((use / kSlots) & 1), err, 23);
         ok = __all_sync(0xffffffffu, ok);   // reconverge the warp before ldmatrix / mma
         if (!ok) break;
-        const uint8_t* kb = smem + SM::kRing + slot * SM::kSlotBytes;
+        const uint8_t* kb = ring + slot * SM::kSlotBytes;
         const uint8_t* vb = kb + (DK / 64) * kBox;
-        const int u0 = jb * kBlk + warp * 16;      // this warp's 16 keys
+        const int u0 = jb * kBlk + cw * 16;        // this warp's 16 keys
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
           uint32_t b0, b1, b2, b3;
-          const int row = warp * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int row = cw * 16 + (lane & 7) + ((lane >> 4) << 3);
           const int c = 2 * (ks & 3) + ((lane >> 3) & 1);
           ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (ks >> 2) * kBox + swz(row, c)));
           mma16816(s[0], qf[ks], b0, b1);
@@ -208,7 +216,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
         for (int np = 0; np < DV / 16; ++np) {
           uint32_t b0, b1, b2, b3;
-          const int row = warp * 16 + (lane & 15);
+          const int row = cw * 16 + (lane & 15);
           const int c = 2 * (np & 3) + (lane >> 4);
           ldsm_x4_t(b0, b1, b2, b3, smem_u32(vb + (np >> 2) * kBox + swz(row, c)));
           mma16816(o[2 * np], a, b0, b1);
@@ -218,12 +226,12 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane == 0) tc::mbar_arrive(empty + slot);
         ++use;
       }
-      ok = vote_all(1, kConsumers * 32, ok);
+      ok = vote_all(gbar, kConsumers * 32, ok);
       if (!ok) break;
       // merge the four warps' partial states: warp w owns value columns [w*DV/4, (w+1)*DV/4)
       {
         constexpr int kNt = DV / 8 / kConsumers;            // n-tiles (8 columns) per owned slice
-        float* sX = reinterpret_cast<float*>(smem + SM::kMerge);
+        float* sX = reinterpret_cast<float*>(smem + SM::kMerge + grp * SM::kScratch);
         float* sMl = sX + kConsumers * 3 * 16 * (DV / 4);
         auto xaddr = [&](int writer, int owner, int row, int col_in_slice) {
           const int slot = owner - (owner > writer);      // owner's position among the writer's three peers
@@ -232,16 +240,16 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
         for (int x = 0; x < DV / 8; ++x) {
           const int owner = x / kNt;
-          if (owner == warp) continue;
+          if (owner == cw) continue;
           const int cs = (x % kNt) * 8 + 2 * cq;
-          *reinterpret_cast<float2*>(xaddr(warp, owner, gl, cs)) = make_float2(o[x][0], o[x][1]);
-          *reinterpret_cast<float2*>(xaddr(warp, owner, gl + 8, cs)) = make_float2(o[x][2], o[x][3]);
+          *reinterpret_cast<float2*>(xaddr(cw, owner, gl, cs)) = make_float2(o[x][0], o[x][1]);
+          *reinterpret_cast<float2*>(xaddr(cw, owner, gl + 8, cs)) = make_float2(o[x][2], o[x][3]);
         }
         if (cq == 0) {
-          sMl[(warp * 16 + gl) * 2] = m0;
-          sMl[(warp * 16 + gl) * 2 + 1] = l0;
-          sMl[(warp * 16 + gl + 8) * 2] = m1;
-          sMl[(warp * 16 + gl + 8) * 2 + 1] = l1;
+          sMl[(cw * 16 + gl) * 2] = m0;
+          sMl[(cw * 16 + gl) * 2 + 1] = l0;
+          sMl[(cw * 16 + gl + 8) * 2] = m1;
+          sMl[(cw * 16 + gl + 8) * 2 + 1] = l1;
         }
         // the accumulator values this lane updates (prefetched before the barrier)
         const size_t row0 = ((size_t)b * T + t) * Hq + g * G;
@@ -251,10 +259,10 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
           for (int xx = 0; xx < kNt; ++xx) {
             const int r = gl + 8 * hh;
-            const int c = warp * (DV / 4) + xx * 8 + 2 * cq;
+            const int c = cw * (DV / 4) + xx * 8 + 2 * cq;
             prev[hh][xx] = r < G ? *reinterpret_cast<const float2*>(acc + (row0 + r) * DV + c) : make_float2(0.f, 0.f);
           }
-        named_sync(1, kConsumers * 32);
+        named_sync(gbar, kConsumers * 32);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const int r = gl + 8 * hh;
@@ -272,21 +280,21 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           const float scl = L > 0.f ? gs / L : 0.f;
           float fw = f[0];
 #pragma unroll
-          for (int w = 1; w < kConsumers; ++w) fw = w == warp ? f[w] : fw;
+          for (int w = 1; w < kConsumers; ++w) fw = w == cw ? f[w] : fw;
 #pragma unroll
           for (int x = 0; x < DV / 8; ++x) {
-            if (x / kNt != warp) continue;               // x stays a compile-time index into o
+            if (x / kNt != cw) continue;               // x stays a compile-time index into o
             const int xx = x % kNt;
             const int cs = xx * 8 + 2 * cq;
             float ox = fw * o[x][2 * hh], oy = fw * o[x][2 * hh + 1];
 #pragma unroll
             for (int w = 0; w < kConsumers; ++w) {
-              if (w == warp) continue;
-              const float2 pv = *reinterpret_cast<const float2*>(xaddr(w, warp, r, cs));
+              if (w == cw) continue;
+              const float2 pv = *reinterpret_cast<const float2*>(xaddr(w, cw, r, cs));
               ox += f[w] * pv.x;
               oy += f[w] * pv.y;
             }
-            const int c = warp * (DV / 4) + cs;
+            const int c = cw * (DV / 4) + cs;
             float2 pr = prev[hh][0];
 #pragma unroll
             for (int y = 1; y < kNt; ++y) pr = y == xx ? prev[hh][y] : pr;
@@ -294,7 +302,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           }
         }
       }
-      named_sync(1, kConsumers * 32);
+      named_sync(gbar, kConsumers * 32);
     }
   }
   __syncthreads();
@@ -322,7 +330,8 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long total = (long)a.Hkv * a.B * a.T;
-  const int grid = (int)(total < (long)sms * kCtasPerSm ? total : (long)sms * kCtasPerSm);
+  const long ctas = (total + kGroups - 1) / kGroups;
+  const int grid = (int)(ctas < (long)sms * kCtasPerSm ? ctas : (long)sms * kCtasPerSm);
   slc_attn_tma_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B,
       a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, a.err);

@@ -333,6 +333,8 @@ def run_decode_bench(args, dev, world):
     out = torch.empty((B, hq, dv), dtype=torch.bfloat16, device=dev)
     cfg = nsa.make_config(batch=B, seqlen=L, h_q=hq, h_kv=hkv, d_k=dk, d_v=dv, top_k=c["top_k"], window=c["window"],
                           w_cmp_k=d.w_k, w_cmp_v=d.w_v, sel_idx_out=idx)
+    ws = torch.empty(nsa.nsa_workspace_size(cfg, B), dtype=torch.uint8, device=dev)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     step = lambda: nsa.nsa_decode(d.q, d.k_cache, d.v_cache, kc, vc, d.seqlens, L, d.gates, cfg, out)
     for _ in range(max(3, args.warmup)):
@@ -340,14 +342,19 @@ def run_decode_bench(args, dev, world):
         step()
     torch.cuda.synchronize()
     barrier(world)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for a, b in evs:
-        flush.zero_()
-        a.record()
-        step()
-        b.record()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for es in evs:
+        for e in es:
+            e.record()
     torch.cuda.synchronize()
-    ms = [a.elapsed_time(b) for a, b in evs]
+    handles = [ctypes_array(es) for es in evs]
+    for i in range(args.steps):
+        flush.zero_()
+        cfg.stage_events, cfg.n_stage_events = handles[i][0], 2
+        step()
+    torch.cuda.synchronize()
+    ms = [es[0].elapsed_time(es[-1]) for es in evs]
+
     mean_ms = allreduce_max(statistics.mean(ms), world, dev)
     nbytes = decode_bytes(idx.cpu(), d.seqlens.cpu(), hq, dk, dv, c["window"])
     peaks, src = load_peaks()

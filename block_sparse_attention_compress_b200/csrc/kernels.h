@@ -61,6 +61,7 @@ struct DecodeArgs {
 // K6: one decode step per sequence, all branches in one launch.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
+
 struct MobaLayout {
   size_t kbar, idx, counts, offsets, chunks, fill, list, part_lse, part_o, total;
 };

@@ -128,7 +128,8 @@ const char* nsa_status_string(nsa_status s) {
 size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch) {
   if (check_cfg(cfg) != NSA_OK || decode_batch < 0) return 0;
   if (decode_batch == 0) return workspace_bytes(cfg);
-  return 0;   // nsa_decode keeps everything on chip
+  if (cfg->mode != NSA_MODE_NSA) return 0;
+  return kAlign;   // nsa_decode: the status word only
 }
 
 nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t T, int32_t H, int32_t d, int32_t d_out,
@@ -209,8 +210,11 @@ nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache, c
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
   a.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = check_workspace(cfg, kAlign);
+  if (st != NSA_OK) return st;
   StageMarks marks(cfg, 1);
-  cudaError_t e = marks.mark(s);
+  cudaError_t e = cudaMemsetAsync(cfg->workspace, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = marks.mark(s);
   if (e == cudaSuccess) e = nsa::launch_decode(a, s);
   if (e == cudaSuccess) e = marks.mark(s);
   return from_cuda(e);

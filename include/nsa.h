@@ -111,8 +111,10 @@ typedef struct {
   int32_t n_stage_events;
 } nsa_config;
 
-/* Bytes of workspace nsa_forward (decode_batch == 0) needs for `cfg`; 0 if cfg is invalid.
- * nsa_decode (decode_batch > 0) needs none: the result is 0 and its workspace fields are ignored. */
+/* Bytes of workspace nsa_forward (decode_batch == 0) or nsa_decode (decode_batch > 0) needs
+ * for `cfg`; 0 if cfg is invalid.  The first 4 bytes of either workspace hold a status word
+ * that the call zeroes and that a device-side wait which timed out sets to a nonzero code
+ * (read it after synchronising to detect NSA_ERR_TIMEOUT). */
 NSA_API size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch);
 
 /*
@@ -166,10 +168,11 @@ NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, cons
  *             Values outside that range are clamped into it on the device.
  *   max_seqlen an upper bound of seqlens (host), 1 <= max_seqlen <= cfg->seqlen <= 65536.
  *   gates     bf16 [B, H_q, 3];  out bf16 [B, H_q, d_v].
- * cfg->batch = B, cfg->seqlen = L_max; sel_idx_out (optional) is [B, H_kv, top_k].
- * One launch (stage_events: 1 kernel): per (sequence, KV head), compressed attention with
- * the group-summed block scores and top-k, then the selected blocks and the window,
- * then the gated sum -- the same arithmetic as the last row of nsa_forward.
+ * cfg->batch = B, cfg->seqlen = L_max; sel_idx_out (optional) is [B, H_kv, top_k];
+ * cfg->workspace: nsa_workspace_size(cfg, B) bytes (the status word).  One launch: per
+ * (sequence, KV head), compressed attention with the group-summed block scores and
+ * top-k, then the selected blocks and the window, then the gated sum -- the same
+ * arithmetic as the last row of nsa_forward.
  */
 NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache,
                       const void* kc_cache, const void* vc_cache, const int32_t* seqlens,

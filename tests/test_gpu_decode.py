@@ -29,9 +29,12 @@ def run_decode(d, seqlens, top_k, window, Lmax=None):
     out = torch.empty((B, hq, dv), dtype=torch.bfloat16, device=DEV)
     cfg = nsa.make_config(batch=B, seqlen=L, h_q=hq, h_kv=hkv, d_k=dk, d_v=dv, top_k=top_k, window=window,
                           w_cmp_k=d.w_k, w_cmp_v=d.w_v, sel_idx_out=idx)
+    ws = torch.empty(max(nsa.nsa_workspace_size(cfg, B), 4), dtype=torch.uint8, device=DEV)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
     sl = dev(seqlens.to(torch.int32))
     nsa.nsa_decode(dev(d.q), k, v, kc, vc, sl, int(seqlens.max()), dev(d.gates), cfg, out)
     torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "a device-side wait timed out"
     return out.cpu(), idx.cpu()
 
 

@@ -71,22 +71,8 @@ __device__ __forceinline__ float ex2(float x) {
 
 __device__ __forceinline__ int n_visible(int t, int nc) { return t < kL - 1 ? 0 : min(nc, (t - kL + 1) / kS + 1); }
 
-__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-
-// Barrier among the softmax warps that also ANDs `pred` across them, so that every warp
-// takes the same branch afterwards (no warp can be left waiting at a later barrier).
-__device__ __forceinline__ bool vote_all(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
+using tc::named_sync;
+using tc::vote_all;
 
 // kWin = false: compressed branch (keys = compressed blocks, scores + top-k, acc = g_cmp * o).
 // kWin = true:  sliding window (keys = tokens [t0-w+1, t0+7], each row masked to its own

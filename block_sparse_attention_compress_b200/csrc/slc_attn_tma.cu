@@ -2,14 +2,21 @@
 // ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5: the top-k blocks are expanded to
 // all their tokens; §10: the group's heads share every loaded block).
 //
-// Persistent CTAs walk the (KV group, batch, token) items, group-major so that the
-// CTAs running at the same time share one group's K/V in L2.  Warp 4 is a TMA
-// producer: for every chosen block of every item it copies the whole 64-token K and V
-// block (128-byte swizzle, 64-column boxes) into a 4-slot ring of 40 KB slots.  Warps
-// 0-3 each take 16 of the 64 keys of every block, with the group's G <= 16 heads as
-// the 16 rows of warp-level m16n8k16 MMAs and an online softmax; at the end of an
-// item their four states are merged and acc += g_slc * o_slc is written.  The ring
-// runs across item boundaries, so the loads of the next token overlap the merge.
+// Persistent CTAs (one per SM) walk the (KV group, batch, token) items, group-major
+// so that the CTAs running at the same time share one group's K/V in L2.  Each CTA
+// runs two independent pipelines on alternate items.  In a pipeline, one warp is the
+// TMA producer: for every chosen block of every item it copies the whole 64-token K
+// and V block (128-byte swizzle, 64-column boxes) into a 2-slot ring of 40 KB slots;
+// four consumer warps each take 16 of the 64 keys of every block, with the group's
+// G <= 16 heads as the 16 rows of warp-level m16n8k16 MMAs and an online softmax.  At
+// the end of an item the four states are merged in registers (each warp owns a
+// quarter of the value columns) and acc += g_slc * o_slc is written.  The ring runs
+// across item boundaries, so the loads of the next token overlap the merge.
+//
+// Slot release: the consumers read a slot with ldmatrix (generic proxy) and the
+// producer refills it with TMA (async proxy).  A proxy fence before each release
+// orders the reads before the refill; without it a refill was seen to overwrite the
+// last value columns a warp read from the slot (about one item in 10^5-10^6).
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -41,19 +48,8 @@ struct Smem {
 
 __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
-__device__ __forceinline__ bool vote_all(int id, int n, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
-__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+using tc::named_sync;
+using tc::vote_all;
 
 // byte offset of (row, 16-byte chunk c of a 64-column box) in a 128-byte-swizzled box
 __device__ __forceinline__ uint32_t swz(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
@@ -222,6 +218,9 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           mma16816(o[2 * np], a, b0, b1);
           mma16816(o[2 * np + 1], a, b2, b3);
         }
+        // the slot is refilled by TMA (async proxy): order this warp's ldmatrix reads
+        // (generic proxy) before the release that lets the producer overwrite it
+        tc::fence_async_smem();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(empty + slot);
         ++use;

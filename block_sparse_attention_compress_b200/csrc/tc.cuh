@@ -19,6 +19,33 @@
 namespace nsa {
 namespace tc {
 
+// ------------------------------------------------------------------ named barriers
+// Barriers among a subset of the CTA's warps (n threads, a multiple of 32).  These use
+// the non-.aligned barrier forms, which count each thread as it arrives: the warps
+// here reach them straight after per-lane polling loops and single-lane branches, and
+// the .aligned forms (bar.sync, bar.red) are undefined for a warp that is not
+// converged at the barrier -- in practice such a warp can be counted twice and let
+// the barrier open before every participating warp has arrived.
+__device__ __forceinline__ void named_sync(int id, int n) {
+  __syncwarp();
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// named_sync that also ANDs `pred` over the participating threads, so that every warp
+// takes the same branch afterwards (none is left waiting at a later barrier).
+__device__ __forceinline__ bool vote_all(int id, int n, bool pred) {
+  uint32_t r;
+  __syncwarp();
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(bar)), "r"(count));

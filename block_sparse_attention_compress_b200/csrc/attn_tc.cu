@@ -22,6 +22,7 @@
 // timeout the kernel records an error word, stops issuing work, and frees its TMEM.
 #include <cfloat>
 
+#include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
 
@@ -63,11 +64,6 @@ struct Smem {
   static_assert(kAlloc <= 232448, "shared memory");
 };
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
 __device__ __forceinline__ int n_visible(int t, int nc) { return t < kL - 1 ? 0 : min(nc, (t - kL + 1) / kS + 1); }
 

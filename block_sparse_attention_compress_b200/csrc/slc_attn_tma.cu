@@ -31,6 +31,7 @@ constexpr int kBlk = 64;
 constexpr int kSlots = 2;                           // ring slots per group
 constexpr int kCtasPerSm = 1;
 constexpr uint32_t kBox = kBlk * 128;   // one 64-row x 64-column box: 8 KB
+constexpr float kSlack = 8.f;            // log2 headroom of the lazily moved softmax reference
 
 template <int DK, int DV>
 struct Smem {
@@ -144,6 +145,22 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           qf[ks][3] = rv1 ? ld_u32(q1 + ks * 16 + 8 + 2 * cq) : 0u;
         }
       }
+      // warm L2 for what comes from DRAM later: the next item's queries (this pipeline's
+      // next token; its index row is read early by the producer) and the accumulator
+      // rows of this item, which the merge reads back
+      {
+        const long itn = it + stride;
+        if (itn < total) {
+          const int gn = (int)(itn / ((long)B * T));
+          const int btn = (int)(itn % ((long)B * T));
+          const char* qn = reinterpret_cast<const char*>(q + ((size_t)btn * Hq + gn * G) * DK);
+          constexpr int kLines = 16 * DK * 2 / 128;               // 16 heads of queries
+          for (int ln = cw * 32 + lane; ln < kLines; ln += kConsumers * 32)
+            if (ln < G * DK * 2 / 128) prefetch_l2(qn + ln * 128);
+        }
+        if (lane < G)
+          prefetch_l2(acc + (((size_t)b * T + t) * Hq + g * G + lane) * DV + cw * (DV / 4));
+      }
       float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
       float o[DV / 8][4];
 #pragma unroll
@@ -169,7 +186,10 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           mma16816(s[0], qf[ks], b0, b1);
           mma16816(s[1], qf[ks], b2, b3);
         }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        // scores in the log2 domain; the reference m of a row only moves when a score
+        // exceeds it by more than kSlack (so p <= 2^kSlack), which after the first block
+        // is rare: the common case needs no cross-lane reduction and no rescaling
+        float lmx0 = -INFINITY, lmx1 = -INFINITY;
 #pragma unroll
         for (int x = 0; x < 2; ++x)
 #pragma unroll
@@ -178,32 +198,31 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             const bool vis = u <= t;
             s[x][e] = vis ? s[x][e] * scale_log2 : -INFINITY;
             s[x][2 + e] = vis ? s[x][2 + e] * scale_log2 : -INFINITY;
-            mx0 = fmaxf(mx0, s[x][e]);
-            mx1 = fmaxf(mx1, s[x][2 + e]);
+            lmx0 = fmaxf(lmx0, s[x][e]);
+            lmx1 = fmaxf(lmx1, s[x][2 + e]);
           }
-        mx0 = warp_max4(mx0);
-        mx1 = warp_max4(mx1);
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        const float base0 = n0 == -INFINITY ? 0.f : n0, base1 = n1 == -INFINITY ? 0.f : n1;
-        const float c0 = exp2f(m0 - base0), c1 = exp2f(m1 - base1);
-        float sum0 = 0.f, sum1 = 0.f;
+        if (__any_sync(0xffffffffu, lmx0 > m0 + kSlack || lmx1 > m1 + kSlack)) {
+          const float n0 = fmaxf(m0, warp_max4(lmx0)), n1 = fmaxf(m1, warp_max4(lmx1));
+          const float c0 = n0 == -INFINITY ? 1.f : ex2(m0 - n0), c1 = n1 == -INFINITY ? 1.f : ex2(m1 - n1);
+          l0 *= c0;
+          l1 *= c1;
+#pragma unroll
+          for (int x = 0; x < DV / 8; ++x) {
+            o[x][0] *= c0; o[x][1] *= c0; o[x][2] *= c1; o[x][3] *= c1;
+          }
+          m0 = n0;
+          m1 = n1;
+        }
+        const float base0 = m0 == -INFINITY ? 0.f : m0, base1 = m1 == -INFINITY ? 0.f : m1;
 #pragma unroll
         for (int x = 0; x < 2; ++x)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            s[x][e] = exp2f(s[x][e] - base0);
-            s[x][2 + e] = exp2f(s[x][2 + e] - base1);
-            sum0 += s[x][e];
-            sum1 += s[x][2 + e];
+            s[x][e] = ex2(s[x][e] - base0);
+            s[x][2 + e] = ex2(s[x][2 + e] - base1);
+            l0 += s[x][e];                   // this lane's part of the row sums
+            l1 += s[x][2 + e];
           }
-        l0 = l0 * c0 + warp_sum4(sum0);
-        l1 = l1 * c1 + warp_sum4(sum1);
-        m0 = n0;
-        m1 = n1;
-#pragma unroll
-        for (int x = 0; x < DV / 8; ++x) {
-          o[x][0] *= c0; o[x][1] *= c0; o[x][2] *= c1; o[x][3] *= c1;
-        }
         uint32_t a[4];
         a[0] = pack_bf16(s[0][0], s[0][1]);
         a[1] = pack_bf16(s[0][2], s[0][3]);
@@ -225,6 +244,8 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane == 0) tc::mbar_arrive(empty + slot);
         ++use;
       }
+      l0 = warp_sum4(l0);
+      l1 = warp_sum4(l1);
       ok = vote_all(gbar, kConsumers * 32, ok);
       if (!ok) break;
       // merge the four warps' partial states: warp w owns value columns [w*DV/4, (w+1)*DV/4)

@@ -261,18 +261,31 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(s_empty + sb);
-        float cm = -INFINITY;
+        // masked, scaled scores; only a tile that straddles this row's range needs the
+        // per-element test.  Max and sum use eight independent chains each.
+        const int i0 = kv_lo + n * kBlk + col0;
+        if (i0 >= my_lo && i0 + 63 < my_hi) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const int i = kv_lo + n * kBlk + col0 + j;
-          v[j] = (i >= my_lo && i < my_hi) ? v[j] * scale_log2 : -INFINITY;
-          cm = fmaxf(cm, v[j]);
+          for (int j = 0; j < 64; ++j) v[j] *= scale_log2;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 64; ++j) v[j] = (i0 + j >= my_lo && i0 + j < my_hi) ? v[j] * scale_log2 : -INFINITY;
         }
+        float cmx[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(fmaxf(v[c], v[c + 8]), fmaxf(v[c + 16], v[c + 24]));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
+        const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                               fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
         const float mn = fmaxf(m, cm);
         if (mn != -INFINITY) {
-          float sum = 0.f;
+          float ps[8];
 #pragma unroll
-          for (int j = 0; j < 64; ++j) sum += ex2(v[j] - mn);
+          for (int c = 0; c < 8; ++c) ps[c] = ex2(v[c] - mn);
+#pragma unroll
+          for (int j = 8; j < 64; ++j) ps[j & 7] += ex2(v[j] - mn);
+          const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
           l = l * ex2(m - mn) + sum;
           m = mn;
         }

@@ -230,7 +230,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int gr = warp >> 2, q4 = warp & 3;
     const int r = 32 * q4 + lane;
     const int col0 = 64 * gr;
-    const int gbar = 1 + gr;                     // named barrier of this group (128 threads)
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
     bool ok = true;
     int use = 0;
@@ -313,10 +312,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       nb_tok[k] = in ? t / kSel + 1 : 0;
     }
     uint8_t* prow = sP + gr * kSlice + r * 128;   // row r of N-block gr of P^T
+    // Selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Each group of four
+    // lanes adds its own four blocks plus the lane just below it into the block's entry.
+    // Lane 31's block (i % 4 == 3) also belongs to the first selection block of the next
+    // warp (or of the next tile); that carry is added two tiles later, after waiting for
+    // the P^T phase that every softmax warp releases only after its own score writes, so
+    // no barrier is needed inside the loop.  Each entry receives at most two additions.
+    float carry_a[4] = {0.f, 0.f, 0.f, 0.f}, carry_b[4] = {0.f, 0.f, 0.f, 0.f};   // tiles n-1, n-2
+    auto add_carry = [&](const float (&c)[4], int tile) {
+      const int jt = tile * (kBlk / 4) + q4 * 8 + 8;
+      if (lane == 31) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          if (jt < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + jt] += c[k];
+      }
+    };
     for (int n = 0; n < ntiles; ++n, ++use) {
       const int sb = use & 1;
-      if (ok) ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
-      ok = vote_all(3, kSoftWarps * 32, ok);   // all eight warps leave together or not at all
+      // no barrier inside this loop: a warp that gives up leaves at once and the others
+      // give up at their next wait (they see the error word); all meet after the loop
+      ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc::tc_fence_after();
       const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
@@ -341,10 +357,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         tok_sum[k] = s;
       }
-      // P^T(n) may overwrite the buffer once PV(n-1) has read it (a timeout here is
-      // carried to the vote at the top of the next tile, so no warp leaves early)
+      if (!kWin) {
+        const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float vv = tok_sum[k];
+          float g4 = vv + __shfl_xor_sync(0xffffffffu, vv, 1);
+          g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
+          const float prev = __shfl_up_sync(0xffffffffu, vv, 1);
+          const int j = j0 + (lane >> 2);
+          if ((lane & 3) == 0 && j < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
+        }
+      }
+      // P^T(n) may overwrite the buffer once PV(n-1) has read it
       if (n > 0) ok = tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty);
+      if (!kWin && n > 0 && ok) {
+        // P^T(n-1) was released by every softmax warp after its score writes of tiles
+        // <= n-1; this warp has not released P^T(n) yet, so the phase is unambiguous
+        ok = tc::mbar_wait(p_full, (n - 1) & 1, err, kErrPFull);
+        if (n > 1) add_carry(carry_b, n - 2);
+      }
       ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        carry_b[k] = carry_a[k];
+        carry_a[k] = tok_sum[k];
+      }
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
@@ -356,27 +395,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::mbar_arrive(s_empty + sb);
         tc::mbar_arrive(p_full);
       }
-      if (kWin) continue;
-      // selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Phase 1: each group
-      // of four lanes adds its own four blocks plus the lane just below it; phase 2: lane 31
-      // hands its block (i % 4 == 3) to the first selection block of the next warp or tile.
-      const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float vv = tok_sum[k];
-        float g4 = vv + __shfl_xor_sync(0xffffffffu, vv, 1);
-        g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
-        const float prev = __shfl_up_sync(0xffffffffu, vv, 1);
-        const int j = j0 + (lane >> 2);
-        if ((lane & 3) == 0 && j < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
-      }
-      named_sync(gbar, 128);
-      if (lane == 31) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (j0 + 8 < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + j0 + 8] += tok_sum[k];
-      }
-      named_sync(gbar, 128);
+    }
+    ok = vote_all(3, kSoftWarps * 32, ok);
+    if (!kWin && ok) {    // the carries of the last two tiles
+      if (ntiles > 1) add_carry(carry_b, ntiles - 2);
+      if (ntiles > 0) add_carry(carry_a, ntiles - 1);
     }
     named_sync(3, kSoftWarps * 32);
 

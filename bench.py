@@ -204,6 +204,19 @@ def workload_config(c, name):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+# DRAM bytes (read + write) per (token, KV group) item of each forward stage, from one ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum) of the T=8192 workload (B=1,
+# 64 query heads, 4 KV groups: 32768 items).  These kernels' DRAM traffic is their q,
+# accumulator and output rows, so it grows in proportion to the items; K/V and the
+# compressed cache stay mostly in L2.  An entry goes back to None whenever its kernel
+# changes, until it is captured again.
+NCU_DRAM_BYTES_PER_ITEM = {
+    "cmp_select": (209.031424e6 + 222.252800e6) / 32768,
+    "slc_attn": (501.390080e6 + 230.337536e6) / 32768,
+    "swa_combine": (499.956736e6 + 118.288128e6) / 32768,
+}
+
+
 def run_ours(args, rank, world, local_rank):
     import block_sparse_attention_compress_b200 as nsa
     from block_sparse_attention_compress_b200.torch_ops import NSAForward
@@ -272,7 +285,10 @@ def run_ours(args, rank, world, local_rank):
         "tflops_computed": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12,
         "frac_of_bf16_peak": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / peaks["bf16_tflops"],
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                     "frac": ach / peak, "traffic": None,
+                     "frac": ach / peak,
+                     "traffic": (None if NCU_DRAM_BYTES_PER_ITEM.get(dom) is None
+                                 else NCU_DRAM_BYTES_PER_ITEM[dom] * B * T * hkv),
+                     "traffic_note": "DRAM bytes per launch, scaled by items from an ncu capture at T=8192",
                      "peak_source": f"{src} bf16_tflops_sustained (kernel timed inside the step)"},
         "stages_ms": {s: round(v, 4) for s, v in stage_mean.items()},
         "stage_tflops": {s: round(flops[s] / (stage_mean[s] * 1e-3) / 1e12, 1) for s in STAGES},

@@ -6,12 +6,15 @@
 // so that the CTAs running at the same time share one group's K/V in L2.  Each CTA
 // runs two independent pipelines on alternate items.  In a pipeline, one warp is the
 // TMA producer: for every chosen block of every item it copies the whole 64-token K
-// and V block (128-byte swizzle, 64-column boxes) into a 2-slot ring of 40 KB slots;
-// four consumer warps each take 16 of the 64 keys of every block, with the group's
-// G <= 16 heads as the 16 rows of warp-level m16n8k16 MMAs and an online softmax.  At
-// the end of an item the four states are merged in registers (each warp owns a
-// quarter of the value columns) and acc += g_slc * o_slc is written.  The ring runs
-// across item boundaries, so the loads of the next token overlap the merge.
+// and V block (128-byte swizzle, 64-column boxes) into a 2-slot ring of 40 KB slots.
+// Four consumer warps share each block: warp w computes the scores of keys 16w..16w+15
+// with the group's G <= 16 heads as the 16 rows of warp-level m16n8k16 MMAs, writes
+// its columns of the block's P[16 heads][64 keys] (bf16) to shared memory, and after
+// one group barrier multiplies the whole P by value columns w*DV/4 .. (w+1)*DV/4 - 1.
+// The softmax reference of a row is shared by the four warps and moves only when a
+// score exceeds it by 2^8 (decided in that same barrier), so the warps' row sums add
+// directly and the item ends without merging partial outputs.  The ring runs across
+// item boundaries, so the loads of the next token overlap the end of this one.
 //
 // Slot release: the consumers read a slot with ldmatrix (generic proxy) and the
 // producer refills it with TMA (async proxy).  A proxy fence before each release
@@ -37,11 +40,11 @@ template <int DK, int DV>
 struct Smem {
   static constexpr uint32_t kSlotBytes = (DK / 64 + DV / 64) * kBox;
   static constexpr uint32_t kRing = 0;                                       // [group][slot]
-  // merge scratch per group: every warp leaves, for each of the other three warps, the
-  // column slice that warp owns ([writer][owner slot][16 rows][DV/4]), plus its m, l per row
-  static constexpr uint32_t kScratch = kConsumers * 3 * 16 * (DV / 4) * 4 + kConsumers * 16 * 2 * 4;
-  static constexpr uint32_t kMerge = kRing + kGroups * kSlots * kSlotBytes;
-  static constexpr uint32_t kBar = kMerge + kGroups * kScratch;
+  static constexpr uint32_t kPBytes = 16 * 128;                              // P [16 heads][64 keys] bf16
+  static constexpr uint32_t kP = kRing + kGroups * kSlots * kSlotBytes;      // [group][2]
+  static constexpr uint32_t kRedBytes = 2 * kConsumers * 16 * 4 + 16;        // [group]: maxima, sums [4][16], flags [4]
+  static constexpr uint32_t kRed = kP + kGroups * 2 * kPBytes;
+  static constexpr uint32_t kBar = kRed + kGroups * kRedBytes;
   static constexpr uint32_t kBytes = kBar + kGroups * 2 * kSlots * 8;
   static constexpr uint32_t kAlloc = kBytes + 1024;
   static_assert(kAlloc * kCtasPerSm <= 232448, "shared memory");
@@ -122,9 +125,16 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         tc::mbar_wait(full + (f % kSlots), (uint32_t)((f / kSlots) & 1), err, 22);
   } else {
     // ---------------------------------------------------------------- consumers
+    // Warp cw computes the scores of keys 16cw..16cw+15 of every block and, from the whole
+    // block's P (shared through SMEM), the values of columns cw*DV/4 .. (cw+1)*DV/4 - 1.
+    constexpr int kNt = DV / 32;                 // 8-column n-tiles per warp
     const int gl = lane >> 2, cq = lane & 3;
-    const int cw = warp % kConsumers;          // consumer warp within the group
-    const int gbar = 1 + grp;                  // named barrier of this group
+    const int cw = warp % kConsumers;
+    const int gbar = 1 + grp;                    // named barrier of this group
+    uint8_t* sPg = smem + SM::kP + grp * 2 * SM::kPBytes;
+    float* sMx = reinterpret_cast<float*>(smem + SM::kRed + grp * SM::kRedBytes);   // [warp][row] block maxima
+    float* sL = sMx + kConsumers * 16;                                                // [warp][row] row sums
+    int* sFlag = reinterpret_cast<int*>(sL + kConsumers * 16);                      // [warp] no wait failed
     long use = 0;
     bool ok = true;
     for (long it = it0; it < total && ok; it += stride) {
@@ -147,7 +157,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       }
       // warm L2 for what comes from DRAM later: the next item's queries (this pipeline's
       // next token; its index row is read early by the producer) and the accumulator
-      // rows of this item, which the merge reads back
+      // rows of this item
       {
         const long itn = it + stride;
         if (itn < total) {
@@ -161,10 +171,12 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane < G)
           prefetch_l2(acc + (((size_t)b * T + t) * Hq + g * G + lane) * DV + cw * (DV / 4));
       }
+      // per row (gl, gl + 8): the softmax reference, shared by the four warps, and this
+      // warp's part of the row sums; it moves only when a score exceeds it by kSlack
       float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-      float o[DV / 8][4];
+      float o[kNt][4];
 #pragma unroll
-      for (int j = 0; j < DV / 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+      for (int x = 0; x < kNt; ++x) o[x][0] = o[x][1] = o[x][2] = o[x][3] = 0.f;
       for (int jj = 0; jj < top_k; ++jj) {
         const int j = __shfl_sync(0xffffffffu, mine, jj);
         if (j < 0) break;
@@ -172,70 +184,107 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const int slot = (int)(use % kSlots);
         ok = tc::mbar_wait(full + slot, (uint32_t)((use / kSlots) & 1), err, 23);
         ok = __all_sync(0xffffffffu, ok);   // reconverge the warp before ldmatrix / mma
-        if (!ok) break;
         const uint8_t* kb = ring + slot * SM::kSlotBytes;
         const uint8_t* vb = kb + (DK / 64) * kBox;
         const int u0 = jb * kBlk + cw * 16;        // this warp's 16 keys
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int ks = 0; ks < DK / 16; ++ks) {
-          uint32_t b0, b1, b2, b3;
-          const int row = cw * 16 + (lane & 7) + ((lane >> 4) << 3);
-          const int c = 2 * (ks & 3) + ((lane >> 3) & 1);
-          ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (ks >> 2) * kBox + swz(row, c)));
-          mma16816(s[0], qf[ks], b0, b1);
-          mma16816(s[1], qf[ks], b2, b3);
-        }
-        // scores in the log2 domain; the reference m of a row only moves when a score
-        // exceeds it by more than kSlack (so p <= 2^kSlack), which after the first block
-        // is rare: the common case needs no cross-lane reduction and no rescaling
         float lmx0 = -INFINITY, lmx1 = -INFINITY;
+        // this warp's 16 columns of the block's P[16 heads][64 keys] (bf16, 16-byte chunks
+        // XOR-swizzled by row), computed against the current reference
+        uint8_t* pbuf = sPg + (use & 1) * SM::kPBytes;
+        float ps0 = 0.f, ps1 = 0.f;
+        auto write_p = [&]() {
+          const float base0 = m0 == -INFINITY ? 0.f : m0, base1 = m1 == -INFINITY ? 0.f : m1;
+          ps0 = 0.f;
+          ps1 = 0.f;
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int u = u0 + x * 8 + 2 * cq + e;
-            const bool vis = u <= t;
-            s[x][e] = vis ? s[x][e] * scale_log2 : -INFINITY;
-            s[x][2 + e] = vis ? s[x][2 + e] * scale_log2 : -INFINITY;
-            lmx0 = fmaxf(lmx0, s[x][e]);
-            lmx1 = fmaxf(lmx1, s[x][2 + e]);
+          for (int x = 0; x < 2; ++x) {
+            const float p00 = ex2(s[x][0] - base0), p01 = ex2(s[x][1] - base0);
+            const float p10 = ex2(s[x][2] - base1), p11 = ex2(s[x][3] - base1);
+            ps0 += p00 + p01;
+            ps1 += p10 + p11;
+            const int ch = 2 * cw + x;
+            *reinterpret_cast<uint32_t*>(pbuf + gl * 128 + ((ch ^ (gl & 7)) << 4) + 4 * cq) = pack_bf16(p00, p01);
+            *reinterpret_cast<uint32_t*>(pbuf + (gl + 8) * 128 + ((ch ^ (gl & 7)) << 4) + 4 * cq) = pack_bf16(p10, p11);
           }
-        if (__any_sync(0xffffffffu, lmx0 > m0 + kSlack || lmx1 > m1 + kSlack)) {
-          const float n0 = fmaxf(m0, warp_max4(lmx0)), n1 = fmaxf(m1, warp_max4(lmx1));
+        };
+        if (ok) {
+#pragma unroll
+          for (int ks = 0; ks < DK / 16; ++ks) {
+            uint32_t b0, b1, b2, b3;
+            const int row = cw * 16 + (lane & 7) + ((lane >> 4) << 3);
+            const int c = 2 * (ks & 3) + ((lane >> 3) & 1);
+            ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (ks >> 2) * kBox + swz(row, c)));
+            mma16816(s[0], qf[ks], b0, b1);
+            mma16816(s[1], qf[ks], b2, b3);
+          }
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int u = u0 + x * 8 + 2 * cq + e;
+              const bool vis = u <= t;
+              s[x][e] = vis ? s[x][e] * scale_log2 : -INFINITY;
+              s[x][2 + e] = vis ? s[x][2 + e] * scale_log2 : -INFINITY;
+              lmx0 = fmaxf(lmx0, s[x][e]);
+              lmx1 = fmaxf(lmx1, s[x][2 + e]);
+            }
+          write_p();
+        }
+        // One decision for the group's four warps, which share P and the reference; the
+        // barrier also makes every warp's P columns visible.  A failed wait takes the
+        // exchange too, so that all four warps leave together (none is left at a barrier).
+        if (tc::vote_any(gbar, kConsumers * 32, !ok || lmx0 > m0 + kSlack || lmx1 > m1 + kSlack)) {
+          const float mx0 = warp_max4(lmx0), mx1 = warp_max4(lmx1);
+          if (cq == 0) {
+            sMx[cw * 16 + gl] = mx0;
+            sMx[cw * 16 + gl + 8] = mx1;
+          }
+          if (lane == 0) sFlag[cw] = ok;
+          named_sync(gbar, kConsumers * 32);
+          if (!(sFlag[0] && sFlag[1] && sFlag[2] && sFlag[3])) {
+            ok = false;
+            break;
+          }
+          float n0 = m0, n1 = m1;
+#pragma unroll
+          for (int w = 0; w < kConsumers; ++w) {
+            n0 = fmaxf(n0, sMx[w * 16 + gl]);
+            n1 = fmaxf(n1, sMx[w * 16 + gl + 8]);
+          }
           const float c0 = n0 == -INFINITY ? 1.f : ex2(m0 - n0), c1 = n1 == -INFINITY ? 1.f : ex2(m1 - n1);
           l0 *= c0;
           l1 *= c1;
 #pragma unroll
-          for (int x = 0; x < DV / 8; ++x) {
+          for (int x = 0; x < kNt; ++x) {
             o[x][0] *= c0; o[x][1] *= c0; o[x][2] *= c1; o[x][3] *= c1;
           }
           m0 = n0;
           m1 = n1;
+          write_p();
+          named_sync(gbar, kConsumers * 32);
         }
-        const float base0 = m0 == -INFINITY ? 0.f : m0, base1 = m1 == -INFINITY ? 0.f : m1;
+        l0 += ps0;
+        l1 += ps1;
+        // O[:, this warp's columns] += P . V over the block's 64 keys
 #pragma unroll
-        for (int x = 0; x < 2; ++x)
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            s[x][e] = ex2(s[x][e] - base0);
-            s[x][2 + e] = ex2(s[x][2 + e] - base1);
-            l0 += s[x][e];                   // this lane's part of the row sums
-            l1 += s[x][2 + e];
+        for (int ks = 0; ks < kBlk / 16; ++ks) {
+          uint32_t a[4];
+          {
+            const int row = lane & 15;
+            const int ch = 2 * ks + (lane >> 4);
+            ldsm_x4(a[0], a[1], a[2], a[3], smem_u32(pbuf + row * 128 + ((ch ^ (row & 7)) << 4)));
           }
-        uint32_t a[4];
-        a[0] = pack_bf16(s[0][0], s[0][1]);
-        a[1] = pack_bf16(s[0][2], s[0][3]);
-        a[2] = pack_bf16(s[1][0], s[1][1]);
-        a[3] = pack_bf16(s[1][2], s[1][3]);
 #pragma unroll
-        for (int np = 0; np < DV / 16; ++np) {
-          uint32_t b0, b1, b2, b3;
-          const int row = cw * 16 + (lane & 15);
-          const int c = 2 * (np & 3) + (lane >> 4);
-          ldsm_x4_t(b0, b1, b2, b3, smem_u32(vb + (np >> 2) * kBox + swz(row, c)));
-          mma16816(o[2 * np], a, b0, b1);
-          mma16816(o[2 * np + 1], a, b2, b3);
+          for (int np = 0; np < kNt / 2; ++np) {
+            const int pg = cw * (kNt / 2) + np;       // 16-column pair within the value row
+            uint32_t b0, b1, b2, b3;
+            const int row = ks * 16 + (lane & 15);
+            const int c = 2 * (pg & 3) + (lane >> 4);
+            ldsm_x4_t(b0, b1, b2, b3, smem_u32(vb + (pg >> 2) * kBox + swz(row, c)));
+            mma16816(o[2 * np], a, b0, b1);
+            mma16816(o[2 * np + 1], a, b2, b3);
+          }
         }
         // the slot is refilled by TMA (async proxy): order this warp's ldmatrix reads
         // (generic proxy) before the release that lets the producer overwrite it
@@ -244,85 +293,41 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane == 0) tc::mbar_arrive(empty + slot);
         ++use;
       }
+      // the row sums over the block keys of all four warps, and the output
       l0 = warp_sum4(l0);
       l1 = warp_sum4(l1);
+      if (cq == 0) {
+        sL[cw * 16 + gl] = l0;
+        sL[cw * 16 + gl + 8] = l1;
+      }
+      const size_t row0 = ((size_t)b * T + t) * Hq + g * G;
+      float2 prev[2][kNt];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int x = 0; x < kNt; ++x) {
+          const int r = gl + 8 * hh;
+          const int c = cw * (DV / 4) + x * 8 + 2 * cq;
+          prev[hh][x] = r < G ? *reinterpret_cast<const float2*>(acc + (row0 + r) * DV + c) : make_float2(0.f, 0.f);
+        }
       ok = vote_all(gbar, kConsumers * 32, ok);
       if (!ok) break;
-      // merge the four warps' partial states: warp w owns value columns [w*DV/4, (w+1)*DV/4)
-      {
-        constexpr int kNt = DV / 8 / kConsumers;            // n-tiles (8 columns) per owned slice
-        float* sX = reinterpret_cast<float*>(smem + SM::kMerge + grp * SM::kScratch);
-        float* sMl = sX + kConsumers * 3 * 16 * (DV / 4);
-        auto xaddr = [&](int writer, int owner, int row, int col_in_slice) {
-          const int slot = owner - (owner > writer);      // owner's position among the writer's three peers
-          return sX + (((writer * 3 + slot) * 16 + row) * (DV / 4) + col_in_slice);
-        };
 #pragma unroll
-        for (int x = 0; x < DV / 8; ++x) {
-          const int owner = x / kNt;
-          if (owner == cw) continue;
-          const int cs = (x % kNt) * 8 + 2 * cq;
-          *reinterpret_cast<float2*>(xaddr(cw, owner, gl, cs)) = make_float2(o[x][0], o[x][1]);
-          *reinterpret_cast<float2*>(xaddr(cw, owner, gl + 8, cs)) = make_float2(o[x][2], o[x][3]);
-        }
-        if (cq == 0) {
-          sMl[(cw * 16 + gl) * 2] = m0;
-          sMl[(cw * 16 + gl) * 2 + 1] = l0;
-          sMl[(cw * 16 + gl + 8) * 2] = m1;
-          sMl[(cw * 16 + gl + 8) * 2 + 1] = l1;
-        }
-        // the accumulator values this lane updates (prefetched before the barrier)
-        const size_t row0 = ((size_t)b * T + t) * Hq + g * G;
-        float2 prev[2][kNt];
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r = gl + 8 * hh;
+        if (r >= G) continue;
+        float L = 0.f;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
+        for (int w = 0; w < kConsumers; ++w) L += sL[w * 16 + r];
+        const float gs = __bfloat162float(gates[(row0 + r) * 3 + 1]);
+        const float scl = L > 0.f ? gs / L : 0.f;
 #pragma unroll
-          for (int xx = 0; xx < kNt; ++xx) {
-            const int r = gl + 8 * hh;
-            const int c = cw * (DV / 4) + xx * 8 + 2 * cq;
-            prev[hh][xx] = r < G ? *reinterpret_cast<const float2*>(acc + (row0 + r) * DV + c) : make_float2(0.f, 0.f);
-          }
-        named_sync(gbar, kConsumers * 32);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int r = gl + 8 * hh;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < kConsumers; ++w) M = fmaxf(M, sMl[(w * 16 + r) * 2]);
-          float f[kConsumers], L = 0.f;
-#pragma unroll
-          for (int w = 0; w < kConsumers; ++w) {
-            f[w] = M == -INFINITY ? 0.f : exp2f(sMl[(w * 16 + r) * 2] - M);
-            L += f[w] * sMl[(w * 16 + r) * 2 + 1];
-          }
-          if (r >= G) continue;
-          const float gs = __bfloat162float(gates[(row0 + r) * 3 + 1]);
-          const float scl = L > 0.f ? gs / L : 0.f;
-          float fw = f[0];
-#pragma unroll
-          for (int w = 1; w < kConsumers; ++w) fw = w == cw ? f[w] : fw;
-#pragma unroll
-          for (int x = 0; x < DV / 8; ++x) {
-            if (x / kNt != cw) continue;               // x stays a compile-time index into o
-            const int xx = x % kNt;
-            const int cs = xx * 8 + 2 * cq;
-            float ox = fw * o[x][2 * hh], oy = fw * o[x][2 * hh + 1];
-#pragma unroll
-            for (int w = 0; w < kConsumers; ++w) {
-              if (w == cw) continue;
-              const float2 pv = *reinterpret_cast<const float2*>(xaddr(w, cw, r, cs));
-              ox += f[w] * pv.x;
-              oy += f[w] * pv.y;
-            }
-            const int c = cw * (DV / 4) + cs;
-            float2 pr = prev[hh][0];
-#pragma unroll
-            for (int y = 1; y < kNt; ++y) pr = y == xx ? prev[hh][y] : pr;
-            *reinterpret_cast<float2*>(acc + (row0 + r) * DV + c) = make_float2(pr.x + scl * ox, pr.y + scl * oy);
-          }
+        for (int x = 0; x < kNt; ++x) {
+          const int c = cw * (DV / 4) + x * 8 + 2 * cq;
+          *reinterpret_cast<float2*>(acc + (row0 + r) * DV + c) =
+              make_float2(prev[hh][x].x + scl * o[x][2 * hh], prev[hh][x].y + scl * o[x][2 * hh + 1]);
         }
       }
-      named_sync(gbar, kConsumers * 32);
     }
   }
   __syncthreads();

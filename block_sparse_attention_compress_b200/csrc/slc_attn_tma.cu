@@ -27,9 +27,11 @@
 namespace nsa {
 
 namespace {
-constexpr int kConsumers = 4;                       // consumer warps per group
+// consumer warps per pipeline: each takes 64/n keys of a block and DV/n value columns.
+// (Eight, at a 96-register cap for 18 warps, spilled and ran 1.5x slower than four.)
+template <int DV> constexpr int consumers() { return 4; }
 constexpr int kGroups = 2;                          // independent pipelines per CTA
-constexpr int kThreads = kGroups * (kConsumers + 1) * 32;
+template <int DV> constexpr int threads() { return kGroups * (consumers<DV>() + 1) * 32; }
 constexpr int kBlk = 64;
 constexpr int kSlots = 2;                           // ring slots per group
 constexpr int kCtasPerSm = 1;
@@ -42,7 +44,8 @@ struct Smem {
   static constexpr uint32_t kRing = 0;                                       // [group][slot]
   static constexpr uint32_t kPBytes = 16 * 128;                              // P [16 heads][64 keys] bf16
   static constexpr uint32_t kP = kRing + kGroups * kSlots * kSlotBytes;      // [group][2]
-  static constexpr uint32_t kRedBytes = 2 * kConsumers * 16 * 4 + 16;        // [group]: maxima, sums [4][16], flags [4]
+  static constexpr int kConsumers = consumers<DV>();
+  static constexpr uint32_t kRedBytes = 2 * kConsumers * 16 * 4 + kConsumers * 4;   // [group]: maxima, sums [warp][16], flags
   static constexpr uint32_t kRed = kP + kGroups * 2 * kPBytes;
   static constexpr uint32_t kBar = kRed + kGroups * kRedBytes;
   static constexpr uint32_t kBytes = kBar + kGroups * 2 * kSlots * 8;
@@ -59,12 +62,14 @@ using tc::vote_all;
 __device__ __forceinline__ uint32_t swz(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__global__ void __launch_bounds__(threads<DV>(), kCtasPerSm)
 slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gates,
                     const int32_t* __restrict__ idx, float* __restrict__ acc, int B, int T, int Hq, int Hkv, int G,
                     int top_k, float scale_log2, int* __restrict__ err) {
   using SM = Smem<DK, DV>;
+  constexpr int kConsumers = SM::kConsumers;
+  constexpr int kKW = kBlk / kConsumers;            // keys per consumer warp: 16 or 8
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -127,7 +132,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     // ---------------------------------------------------------------- consumers
     // Warp cw computes the scores of keys 16cw..16cw+15 of every block and, from the whole
     // block's P (shared through SMEM), the values of columns cw*DV/4 .. (cw+1)*DV/4 - 1.
-    constexpr int kNt = DV / 32;                 // 8-column n-tiles per warp
+    constexpr int kNt = DV / 8 / kConsumers;     // 8-column n-tiles per warp
     const int gl = lane >> 2, cq = lane & 3;
     const int cw = warp % kConsumers;
     const int gbar = 1 + grp;                    // named barrier of this group
@@ -169,7 +174,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             if (ln < G * DK * 2 / 128) prefetch_l2(qn + ln * 128);
         }
         if (lane < G)
-          prefetch_l2(acc + (((size_t)b * T + t) * Hq + g * G + lane) * DV + cw * (DV / 4));
+          prefetch_l2(acc + (((size_t)b * T + t) * Hq + g * G + lane) * DV + cw * (DV / kConsumers));
       }
       // per row (gl, gl + 8): the softmax reference, shared by the four warps, and this
       // warp's part of the row sums; it moves only when a score exceeds it by kSlack
@@ -186,8 +191,10 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         ok = __all_sync(0xffffffffu, ok);   // reconverge the warp before ldmatrix / mma
         const uint8_t* kb = ring + slot * SM::kSlotBytes;
         const uint8_t* vb = kb + (DK / 64) * kBox;
-        const int u0 = jb * kBlk + cw * 16;        // this warp's 16 keys
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const int u0 = jb * kBlk + cw * kKW;       // this warp's keys
+        float s[kKW / 8][4];
+#pragma unroll
+        for (int x = 0; x < kKW / 8; ++x) s[x][0] = s[x][1] = s[x][2] = s[x][3] = 0.f;
         float lmx0 = -INFINITY, lmx1 = -INFINITY;
         // this warp's 16 columns of the block's P[16 heads][64 keys] (bf16, 16-byte chunks
         // XOR-swizzled by row), computed against the current reference
@@ -198,28 +205,45 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           ps0 = 0.f;
           ps1 = 0.f;
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
+          for (int x = 0; x < kKW / 8; ++x) {
             const float p00 = ex2(s[x][0] - base0), p01 = ex2(s[x][1] - base0);
             const float p10 = ex2(s[x][2] - base1), p11 = ex2(s[x][3] - base1);
             ps0 += p00 + p01;
             ps1 += p10 + p11;
-            const int ch = 2 * cw + x;
+            const int ch = cw * (kKW / 8) + x;
             *reinterpret_cast<uint32_t*>(pbuf + gl * 128 + ((ch ^ (gl & 7)) << 4) + 4 * cq) = pack_bf16(p00, p01);
             *reinterpret_cast<uint32_t*>(pbuf + (gl + 8) * 128 + ((ch ^ (gl & 7)) << 4) + 4 * cq) = pack_bf16(p10, p11);
           }
         };
         if (ok) {
+          if constexpr (kKW == 16) {
 #pragma unroll
-          for (int ks = 0; ks < DK / 16; ++ks) {
-            uint32_t b0, b1, b2, b3;
-            const int row = cw * 16 + (lane & 7) + ((lane >> 4) << 3);
-            const int c = 2 * (ks & 3) + ((lane >> 3) & 1);
-            ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (ks >> 2) * kBox + swz(row, c)));
-            mma16816(s[0], qf[ks], b0, b1);
-            mma16816(s[1], qf[ks], b2, b3);
+            for (int ks = 0; ks < DK / 16; ++ks) {
+              uint32_t b0, b1, b2, b3;
+              const int row = cw * 16 + (lane & 7) + ((lane >> 4) << 3);
+              const int c = 2 * (ks & 3) + ((lane >> 3) & 1);
+              ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (ks >> 2) * kBox + swz(row, c)));
+              mma16816(s[0], qf[ks], b0, b1);
+              mma16816(s[kKW / 8 - 1], qf[ks], b2, b3);
+            }
+          } else {
+            // 8 keys: one ldmatrix covers two 16-wide K steps; the even and odd steps
+            // accumulate separately (two dependency chains) and are added at the end
+            float s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int j = 0; j < DK / 32; ++j) {
+              uint32_t b0, b1, b2, b3;
+              const int row = cw * 8 + (lane & 7);
+              const int c = 4 * (j & 1) + (lane >> 3);
+              ldsm_x4(b0, b1, b2, b3, smem_u32(kb + (j >> 1) * kBox + swz(row, c)));
+              mma16816(s[0], qf[2 * j], b0, b1);
+              mma16816(s2, qf[2 * j + 1], b2, b3);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[0][e] += s2[e];
           }
 #pragma unroll
-          for (int x = 0; x < 2; ++x)
+          for (int x = 0; x < kKW / 8; ++x)
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
               const int u = u0 + x * 8 + 2 * cq + e;
@@ -242,7 +266,10 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           }
           if (lane == 0) sFlag[cw] = ok;
           named_sync(gbar, kConsumers * 32);
-          if (!(sFlag[0] && sFlag[1] && sFlag[2] && sFlag[3])) {
+          bool all_ok = true;
+#pragma unroll
+          for (int w = 0; w < kConsumers; ++w) all_ok = all_ok && sFlag[w];
+          if (!all_ok) {
             ok = false;
             break;
           }
@@ -307,7 +334,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 #pragma unroll
         for (int x = 0; x < kNt; ++x) {
           const int r = gl + 8 * hh;
-          const int c = cw * (DV / 4) + x * 8 + 2 * cq;
+          const int c = cw * (DV / kConsumers) + x * 8 + 2 * cq;
           prev[hh][x] = r < G ? *reinterpret_cast<const float2*>(acc + (row0 + r) * DV + c) : make_float2(0.f, 0.f);
         }
       ok = vote_all(gbar, kConsumers * 32, ok);
@@ -323,7 +350,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         const float scl = L > 0.f ? gs / L : 0.f;
 #pragma unroll
         for (int x = 0; x < kNt; ++x) {
-          const int c = cw * (DV / 4) + x * 8 + 2 * cq;
+          const int c = cw * (DV / kConsumers) + x * 8 + 2 * cq;
           *reinterpret_cast<float2*>(acc + (row0 + r) * DV + c) =
               make_float2(prev[hh][x].x + scl * o[x][2 * hh], prev[hh][x].y + scl * o[x][2 * hh + 1]);
         }
@@ -357,7 +384,7 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   const long total = (long)a.Hkv * a.B * a.T;
   const long ctas = (total + kGroups - 1) / kGroups;
   const int grid = (int)(ctas < (long)sms * kCtasPerSm ? ctas : (long)sms * kCtasPerSm);
-  slc_attn_tma_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
+  slc_attn_tma_kernel<DK, DV><<<grid, threads<DV>(), SM::kAlloc, st>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B,
       a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, a.err);
   return cudaGetLastError();

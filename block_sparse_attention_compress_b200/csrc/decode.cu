@@ -385,23 +385,36 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
         ++nforced;
       }
       const int mmax = (nb + 31) >> 5;
-      for (int r = nforced; r < top_k; ++r) {
-        float bs = -FLT_MAX;
-        int bj = 0x7fffffff;
-        for (int m = 0; m < mmax; ++m) {
-          const int j = lane + 32 * m;
-          if (j < nb && !((taken >> m) & 1u)) {
-            const float sc = sScore[j];
-            if (sc > bs) { bs = sc; bj = j; }
-          }
-        }
+      // this lane's candidates j = lane + 32*mm as order-preserving integer keys (the
+      // scores are sums of probabilities, >= 0); key 0 marks "no candidate"
+      uint32_t key[32];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float os = __shfl_xor_sync(0xffffffffu, bs, off);
-          const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-          if (os > bs || (os == bs && oj < bj)) { bs = os; bj = oj; }
+      for (int mm = 0; mm < 32; ++mm) {
+        const int j = lane + 32 * mm;
+        key[mm] = (mm < mmax && j < nb && !((taken >> mm) & 1u)) ? __float_as_uint(sScore[j]) + 1u : 0u;
+      }
+      uint32_t bk = 0;   // this lane's best key and its mm (the lowest mm among equal keys)
+      int bm = 0;
+      auto local_best = [&]() {
+        bk = 0;
+        bm = 0;
+#pragma unroll
+        for (int mm = 0; mm < 32; ++mm)
+          if (key[mm] > bk) { bk = key[mm]; bm = mm; }
+      };
+      local_best();
+      for (int rr = nforced; rr < top_k; ++rr) {
+        const uint32_t vmax = __reduce_max_sync(0xffffffffu, bk);
+        if (vmax == 0u) break;
+        const uint32_t jmin = __reduce_min_sync(0xffffffffu, bk == vmax ? (uint32_t)(lane + 32 * bm) : 0xffffffffu);
+        if (lane == (int)(jmin & 31u)) {
+          const int mw = (int)(jmin >> 5);
+          taken |= 1u << mw;
+#pragma unroll
+          for (int mm = 0; mm < 32; ++mm)
+            if (mm == mw) key[mm] = 0u;
+          local_best();
         }
-        if (bj != 0x7fffffff && lane == (bj & 31)) taken |= 1u << (bj >> 5);
       }
       int pos = 0;
       for (int m = 0; m < mmax; ++m) {

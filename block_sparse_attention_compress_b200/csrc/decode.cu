@@ -8,17 +8,19 @@
 //      shared-memory ring (16 blocks = 10 KB per stage): online softmax for o_cmp and,
 //      per head, the running sums of exp(s - m) per 64-token selection block
 //      (rescaled whenever that head's running max grows);
-//   M  the warps' states are merged: per-head log-sum-exp, the group-summed
-//      normalised block scores, top-k (forced blocks first, ties to the lower
-//      index), and o_cmp;
-//   B  the selected blocks (two per warp), then the window (one chunk per warp),
-//      each with its own softmax, merged the same way;
+//   M  the warps' states are merged: per-head log-sum-exp, each warp's weight and the
+//      group-summed normalised block scores; then warp 0 runs the top-k (forced blocks
+//      first, ties to the lower index) while warps 1..7 sum o_cmp and stream the
+//      window, which needs no selection, with their own softmax states;
+//   B  the selected blocks (two per warp), with one more softmax state per warp;
+//      each branch's states are merged by log-sum-exp weights;
 //   C  out = g_cmp*o_cmp + g_slc*o_slc + g_win*o_win, rounded to bf16.
 // Loads are 16-byte cp.async of whole K/V rows (coalesced, each row 384 + 256 bytes).
 #include <cfloat>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace nsa {
 
@@ -38,7 +40,7 @@ struct Smem {
   static constexpr size_t kPart = (size_t)kWarps * 16 * kJ * 4;                  // per-warp per-head block sums
   static constexpr size_t kPersist =
       ((size_t)(kWarps * 16 * 2 + kWarps * 16 + kMaxSel + 32 + 3 * 16 * DV) * 4 + 127) / 128 * 128;
-  static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (DV + 2) * 4;
+  static constexpr size_t kMergeBytes = (size_t)kWarps * 16 * (DV + 8) * 4 + (size_t)kWarps * 16 * 3 * 4;
   static constexpr size_t kPhaseB = kPersist + (kRing > kMergeBytes ? kRing : kMergeBytes);
   static constexpr size_t kTotal = (kRing + kPart) > kPhaseB ? (kRing + kPart) : kPhaseB;
   static_assert(kTotal <= 232448, "decode shared memory");
@@ -185,44 +187,84 @@ __device__ void attend_rows(const uint32_t (&qf)[DK / 16][4], State<DV>& st, Til
   __syncwarp();
 }
 
-// Merge the 8 warps' states into o (normalised) for rows < G; result in sOut [16][DV].
-// sScratch must hold kWarps*16*DV floats + kWarps*16*2 floats.
+// Shared-memory scratch of the cross-warp merges: per warp 16 rows of DV floats, each row
+// padded by 8 floats so that the float2 stores of a C fragment (8 rows x 4 column pairs per
+// half-warp) fall on 32 distinct banks.
 template <int DV>
-__device__ void merge_states(const State<DV>& st, float* sScratch, float* sOut, int G, int warp, int lane) {
+struct MergeBuf {
+  static constexpr int kStride = DV + 8;
+  static constexpr size_t kBytes = (size_t)kWarps * 16 * kStride * 4;
+  __device__ static float* row(float* base, int w, int r) { return base + (w * 16 + r) * kStride; }
+};
+
+// Store the warp's (scaled) accumulator rows into its slot of the merge scratch.
+template <int DV>
+__device__ __forceinline__ void store_o(float* sO, const State<DV>& st, float f0, float f1, int warp, int lane) {
   const int gl = lane >> 2, cq = lane & 3;
-  float* sO = sScratch;
-  float* sML = sScratch + kWarps * 16 * DV;
-  __syncthreads();   // every warp is done with its stage ring, which the scratch overlays
+  float* r0 = MergeBuf<DV>::row(sO, warp, gl) + 2 * cq;
+  float* r1 = MergeBuf<DV>::row(sO, warp, gl + 8) + 2 * cq;
 #pragma unroll
   for (int j = 0; j < DV / 8; ++j) {
-    sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq] = st.o[j][0];
-    sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq + 1] = st.o[j][1];
-    sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq] = st.o[j][2];
-    sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq + 1] = st.o[j][3];
+    *reinterpret_cast<float2*>(r0 + j * 8) = make_float2(st.o[j][0] * f0, st.o[j][1] * f0);
+    *reinterpret_cast<float2*>(r1 + j * 8) = make_float2(st.o[j][2] * f1, st.o[j][3] * f1);
   }
-  if (cq == 0) {
-    sML[(warp * 16 + gl) * 2] = st.m0;
-    sML[(warp * 16 + gl) * 2 + 1] = st.l0;
-    sML[(warp * 16 + gl + 8) * 2] = st.m1;
-    sML[(warp * 16 + gl + 8) * 2 + 1] = st.l1;
+}
+
+__device__ __forceinline__ void store_ml(float* sML, float m0, float l0, float m1, float l1, int warp, int lane) {
+  const int gl = lane >> 2;
+  if ((lane & 3) == 0) {
+    sML[(warp * 16 + gl) * 2] = m0;
+    sML[(warp * 16 + gl) * 2 + 1] = l0;
+    sML[(warp * 16 + gl + 8) * 2] = m1;
+    sML[(warp * 16 + gl + 8) * 2 + 1] = l1;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < G * DV; e += kThreads) {
+}
+
+// For row r (tid < 16): coef[w][r] = 2^(m_w - lse) with lse the log2-sum-exp over the warps'
+// (m, l); the normalised merged row is sum_w coef[w][r] * o_w.  Rows >= G or with no
+// visible key get coefficient 0.
+__device__ __forceinline__ void merge_coefs(const float* sML, float* sCoef, int G, int r) {
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sML[(w * 16 + r) * 2]);
+  float Ls = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) Ls += exp2f(sML[(w * 16 + r) * 2] - M) * sML[(w * 16 + r) * 2 + 1];
+  }
+  const float lse = (r < G && Ls > 0.f) ? M + __log2f(Ls) : INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) sCoef[w * 16 + r] = exp2f(sML[(w * 16 + r) * 2] - lse);
+}
+
+// dst[r][c] = sum_w coef[w][r] * sO[w][r][c] for r < G, over threads [t0, t0 + nthr).
+template <int DV>
+__device__ __forceinline__ void merge_sum(const float* sO, const float* sCoef, float* dst, int G, int t0, int nthr) {
+  for (int e = threadIdx.x - t0; e < G * DV; e += nthr) {
     const int r = e / DV, c = e % DV;
-    float M = -INFINITY;
+    float acc = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sML[(w * 16 + r) * 2]);
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float f = exp2f(sML[(w * 16 + r) * 2] - M);
-        L += f * sML[(w * 16 + r) * 2 + 1];
-        O += f * sO[(w * 16 + r) * DV + c];
-      }
-    }
-    sOut[r * DV + c] = L > 0.f ? O / L : 0.f;
+    for (int w = 0; w < kWarps; ++w)
+      acc += sCoef[w * 16 + r] * MergeBuf<DV>::row(const_cast<float*>(sO), w, r)[c];
+    dst[r * DV + c] = acc;
   }
+}
+
+// Merge the 8 warps' states into normalised rows (r < G) of sOut [16][DV].  The scratch
+// (MergeBuf bytes, then 16 x kWarps coefficients and 16 x kWarps x 2 (m, l)) overlays the
+// stage rings, so the call starts with a barrier.
+template <int DV>
+__device__ void merge_states(const State<DV>& st, uint8_t* scratch, float* sOut, int G, int warp, int lane) {
+  float* sO = reinterpret_cast<float*>(scratch);
+  float* sCoef = reinterpret_cast<float*>(scratch + MergeBuf<DV>::kBytes);
+  float* sML = sCoef + kWarps * 16;
+  __syncthreads();   // every warp is done with its stage ring
+  store_o<DV>(sO, st, 1.f, 1.f, warp, lane);
+  store_ml(sML, st.m0, st.l0, st.m1, st.l1, warp, lane);
+  __syncthreads();
+  if (threadIdx.x < 16) merge_coefs(sML, sCoef, G, threadIdx.x);
+  __syncthreads();
+  merge_sum<DV>(sO, sCoef, sOut, G, 0, kThreads);
   __syncthreads();
 }
 
@@ -330,7 +372,7 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
 
   // ---------------- M: merge, scores, top-k, o_cmp ----------------
   // Small persistent buffers sit at the bottom (over the dead phase-A rings); above them one
-  // union region serves the cross-warp merges and, in phase B, the stage rings.
+  // union region serves the cross-warp merges and, later, the stage rings.
   float* sML = reinterpret_cast<float*>(smem);                         // [8][16][2] m, l
   float* sCoef = sML + kWarps * 16 * 2;                                // [8][16]
   float* sScore = sCoef + kWarps * 16;                                 // [kMaxSel]
@@ -338,25 +380,12 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
   float* sOcmp = reinterpret_cast<float*>(sIdx + 32);                  // [16][DV]
   float* sOslc = sOcmp + 16 * DV;                                      // [16][DV]
   float* sOwin = sOslc + 16 * DV;                                      // [16][DV]
-  uint8_t* uni = smem + SM::kPersist;                                  // merge scratch / phase-B rings
+  uint8_t* uni = smem + SM::kPersist;                                  // merge scratch / stage rings
   float* sMerge = reinterpret_cast<float*>(uni);
-  if (cq == 0) {
-    sML[(warp * 16 + gl) * 2] = st.m0;
-    sML[(warp * 16 + gl) * 2 + 1] = st.l0;
-    sML[(warp * 16 + gl + 8) * 2] = st.m1;
-    sML[(warp * 16 + gl + 8) * 2 + 1] = st.l1;
-  }
+  store_o<DV>(sMerge, st, 1.f, 1.f, warp, lane);
+  store_ml(sML, st.m0, st.l0, st.m1, st.l1, warp, lane);
   __syncthreads();
-  if (tid < 16) {   // per-head log-sum-exp (log2 units) and each warp's coefficient
-    const int r = tid;
-    float M = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, sML[(w * 16 + r) * 2]);
-    float Ls = 0.f;
-    if (M != -INFINITY)
-      for (int w = 0; w < kWarps; ++w) Ls += exp2f(sML[(w * 16 + r) * 2] - M) * sML[(w * 16 + r) * 2 + 1];
-    const float lse = (r < G && Ls > 0.f) ? M + __log2f(Ls) : INFINITY;
-    for (int w = 0; w < kWarps; ++w) sCoef[w * 16 + r] = exp2f(sML[(w * 16 + r) * 2] - lse);
-  }
+  if (tid < 16) merge_coefs(sML, sCoef, G, tid);   // per-head log-sum-exp -> each warp's weight
   __syncthreads();
   const int nb = t / kSel + 1;
   {
@@ -371,12 +400,17 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
       sScore[J] = sc;
     }
   }
-  __syncthreads();
-  if (warp == 0) {   // top-k over the nb eligible blocks
+  __syncthreads();   // the block sums are dead from here on
+  const int own = t / kSel;
+  Tile<DK, DV> rb0{reinterpret_cast<__nv_bfloat16*>(uni + (size_t)warp * 2 * SM::kStage), nullptr};
+  rb0.v = rb0.k + kRows * DK;
+  Tile<DK, DV> rb1{reinterpret_cast<__nv_bfloat16*>(uni + (size_t)warp * 2 * SM::kStage + SM::kStage), nullptr};
+  rb1.v = rb1.k + kRows * DK;
+  st.init();
+  if (warp == 0) {   // top-k over the nb eligible blocks, while the other warps stream the window
     if (nb <= top_k) {
       for (int j = lane; j < top_k; j += 32) sIdx[j] = j < nb ? j : -1;
     } else {
-      const int own = t / kSel;
       uint32_t taken = 0;
       int nforced = 0;
       if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
@@ -425,39 +459,28 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
       }
       for (int j = pos + lane; j < top_k; j += 32) sIdx[j] = -1;
     }
+    __syncwarp();
+    if (idx_out)
+      for (int j = lane; j < top_k; j += 32) idx_out[((size_t)b * Hkv + g) * top_k + j] = sIdx[j];
+  } else {
+    // o_cmp = sum over warps of weight x o, then the window, split over warps 1..7 in
+    // 16-row tiles (its rings overlay the merge scratch, hence the barrier in between)
+    merge_sum<DV>(sMerge, sCoef, sOcmp, G, 32, kThreads - 32);
+    tc::named_sync(1, kThreads - 32);
+    const int lo = max(0, t - window + 1);
+    const int nwin = t - lo + 1;
+    const int per = ((nwin + kRows - 1) / kRows + kWarps - 2) / (kWarps - 1) * kRows;
+    const int r0 = min(nwin, (warp - 1) * per);
+    const int n = min(nwin, r0 + per) - r0;
+    auto rowk = [&](int r) { return kcache + (((size_t)b * Lmax + lo + r0 + r) * Hkv + g) * DK; };
+    auto rowv = [&](int r) { return vcache + (((size_t)b * Lmax + lo + r0 + r) * Hkv + g) * DV; };
+    attend_rows<DK, DV>(qf, st, rb0, rb1, n, rowk, rowv, [](int) { return true; }, scale_log2, lane);
   }
-  __syncthreads();
-  if (idx_out)
-    for (int j = tid; j < top_k; j += kThreads) idx_out[((size_t)b * Hkv + g) * top_k + j] = sIdx[j];
-  // o_cmp: each warp's o scaled by its coefficient, summed over warps
-  {
-    float* sO = sMerge;
-#pragma unroll
-    for (int j = 0; j < DV / 8; ++j) {
-      const float f0 = sCoef[warp * 16 + gl], f1 = sCoef[warp * 16 + gl + 8];
-      sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq] = st.o[j][0] * f0;
-      sO[(warp * 16 + gl) * DV + j * 8 + 2 * cq + 1] = st.o[j][1] * f0;
-      sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq] = st.o[j][2] * f1;
-      sO[(warp * 16 + gl + 8) * DV + j * 8 + 2 * cq + 1] = st.o[j][3] * f1;
-    }
-    __syncthreads();
-    for (int e = tid; e < 16 * DV; e += kThreads) {
-      float acc = 0.f;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) acc += sO[w * 16 * DV + e];
-      sOcmp[e] = acc;
-    }
-    __syncthreads();
-  }
+  merge_states<DV>(st, uni, sOwin, G, warp, lane);   // warp 0's state is empty
 
-  // ---------------- B: selected blocks, then the window ----------------
-  Tile<DK, DV> rb0{reinterpret_cast<__nv_bfloat16*>(uni + (size_t)warp * 2 * SM::kStage), nullptr};
-  rb0.v = rb0.k + kRows * DK;
-  Tile<DK, DV> rb1{reinterpret_cast<__nv_bfloat16*>(uni + (size_t)warp * 2 * SM::kStage + SM::kStage), nullptr};
-  rb1.v = rb1.k + kRows * DK;
-  const int own = t / kSel;
+  // ---------------- B: the selected blocks ----------------
   {
-    // warp w takes the chosen blocks at positions 2w and 2w+1 (and more when top_k > 16)
+    // warp w takes the chosen blocks at positions w and w + 8 (and more when top_k > 16)
     st.init();
     for (int p = warp; p < top_k; p += kWarps) {
       const int j = sIdx[p];
@@ -469,19 +492,7 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
       auto rowv = [&](int r) { return vcache + (((size_t)b * Lmax + u0 + r) * Hkv + g) * DV; };
       attend_rows<DK, DV>(qf, st, rb0, rb1, n, rowk, rowv, [](int) { return true; }, scale_log2, lane);
     }
-    merge_states<DV>(st, sMerge, sOslc, G, warp, lane);
-  }
-  {
-    st.init();
-    const int lo = max(0, t - window + 1);
-    const int nwin = t - lo + 1;
-    const int chunk = (nwin + kWarps - 1) / kWarps;
-    const int r0 = min(nwin, warp * chunk);
-    const int n = min(nwin, r0 + chunk) - r0;
-    auto rowk = [&](int r) { return kcache + (((size_t)b * Lmax + lo + r0 + r) * Hkv + g) * DK; };
-    auto rowv = [&](int r) { return vcache + (((size_t)b * Lmax + lo + r0 + r) * Hkv + g) * DV; };
-    attend_rows<DK, DV>(qf, st, rb0, rb1, n, rowk, rowv, [](int) { return true; }, scale_log2, lane);
-    merge_states<DV>(st, sMerge, sOwin, G, warp, lane);
+    merge_states<DV>(st, uni, sOslc, G, warp, lane);
   }
 
   // ---------------- C: gated combine ----------------

@@ -76,6 +76,11 @@ def test_decode_tiny_heads():
     check(d, torch.tensor([1024, 600], dtype=torch.int32), 4, 128)
 
 
+def test_decode_head_dim_128():
+    d = synth.decode_inputs(3, 2600, 32, 2, 128, 128, seed=24)
+    check(d, torch.tensor([2600, 65, 1999], dtype=torch.int32), 16, 256)
+
+
 def test_decode_matches_last_prefill_row_on_gpu():
     """The decode step at position L-1 and the prefill's last row are the same arithmetic."""
     L = 1500

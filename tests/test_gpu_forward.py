@@ -74,6 +74,19 @@ def test_ragged_multi_group_full():
     check_against_oracle(x, 16, 200)
 
 
+def test_head_dim_128_full():
+    """d_k = d_v = 128 with 16 heads per group: the tensor-core instances of the compressed,
+    selected and window kernels at that head size; two groups, a ragged T."""
+    x = synth.nsa_inputs(1, 1333, 32, 2, 128, 128, seed=31)
+    check_against_oracle(x, 16, 300)
+
+
+def test_head_dim_128_small_group():
+    """d_k = d_v = 128 with 8 heads per group (padded rows in every kernel)."""
+    x = synth.nsa_inputs(1, 777, 16, 2, 128, 128, seed=32)
+    check_against_oracle(x, 8, 200)
+
+
 @pytest.mark.parametrize("T", [1, 7, 31, 32, 33, 47, 48, 64, 65])
 def test_short_sequences(T):
     """No compressed block (T < 32), exactly one, and the first few selection blocks."""

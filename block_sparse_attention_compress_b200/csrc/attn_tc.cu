@@ -1,11 +1,12 @@
-// K2 and K4 on the 5th-generation tensor cores.  K2: compressed attention + group-summed block
-// scores + top-k ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5, §8; "一文比较 Kimi 和
-// Deepseek 的两篇稀疏注意力机制论文", "Deepseek 的论文核心点": the selection scores come
-// from the compressed attention and the group's heads add them before one top-k).
+// K2 on the 5th-generation tensor cores: compressed attention + group-summed block scores +
+// top-k ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5, §8; "一文比较 Kimi 和 Deepseek
+// 的两篇稀疏注意力机制论文", "Deepseek 的论文核心点": the selection scores come from the
+// compressed attention and the group's heads add them before one top-k).
 //
-// One CTA = one KV group g and 8 consecutive tokens; its 128 query rows (token-major,
-// 16 heads per token) are one tcgen05 M=128 tile held in shared memory.  The group's
-// compressed keys/values stream through shared memory by TMA in tiles of 128 blocks.
+// Persistent: one CTA per SM walks a static list of items, item = one KV group g and 8
+// consecutive tokens (longest rows first).  An item's 128 query rows (token-major, 16 heads
+// per token) are one tcgen05 M=128 tile held in shared memory.  The group's compressed
+// keys/values stream through shared memory by TMA in tiles of 128 blocks.
 //   pass A   S = Q Kc^T into TMEM (rows = (token, head)); each softmax thread owns a
 //            row and keeps its running max and sum -> log-sum-exp per row.
 //   pass B   S^T = Kc Q^T into TMEM (rows = compressed blocks, columns = (token, head)):
@@ -16,10 +17,15 @@
 //            (rows = value dims), already normalised, so no rescaling is ever needed.
 //   top-k    per token over the selection-block scores in shared memory.
 //   epilogue acc[t, h, :] = g_cmp * o_cmp, read from O^T (each thread one value dim).
-// Warp roles: 8 TMA producer, 9 MMA issuer (and TMEM owner), 0-7 softmax / epilogue in
-// two groups of four (warp w owns TMEM lanes 32*(w%4)..+31; group w/4 takes one half of
-// every tile's 128 columns: in the second pass that half is exactly four tokens).  Every wait is bounded (see tc.cuh); on a
-// timeout the kernel records an error word, stops issuing work, and frees its TMEM.
+// Warp roles: 8 TMA producer, 9 MMA issuer (and TMEM owner), 10-11 top-k, 0-7 softmax /
+// epilogue in two groups of four (warp w owns TMEM lanes 32*(w%4)..+31; group w/4 takes one
+// half of every tile's 128 columns: in the second pass that half is exactly four tokens).
+// Items overlap: while the softmax warps finish an item (last tiles, epilogue), the TMA and
+// MMA warps already load and multiply the next item's first tiles, and the top-k warps
+// select the finished item's blocks while the softmax warps run the next item's pass A.
+// Every wait is bounded (see tc.cuh); on a timeout the kernel records an error word, stops
+// issuing work, and frees its TMEM.
+#include <algorithm>
 #include <cfloat>
 
 #include "common.cuh"
@@ -30,8 +36,8 @@ namespace nsa {
 
 namespace {
 constexpr int kSoftWarps = 8;                 // two groups of four softmax warps
-constexpr int kTmaWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9, kTopkWarp0 = 10, kTopkWarps = 2;
+constexpr int kThreads = 384;
 constexpr int kTok = 8;            // tokens per CTA
 constexpr int kRowsM = 128;        // query rows per CTA (8 tokens x 16 heads)
 constexpr int kBlk = 128;          // compressed blocks per tile
@@ -43,7 +49,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 
 enum Err { kErrQ = 1, kErrKcFull, kErrKcEmpty, kErrVcFull, kErrVcEmpty, kErrSFull, kErrSEmpty, kErrPFull,
-           kErrPEmpty, kErrOFull };
+           kErrPEmpty, kErrOFull, kErrQEmpty, kErrScFull, kErrScEmpty, kErrOEmpty };
 
 template <int DK, int DV>
 struct Smem {
@@ -54,10 +60,10 @@ struct Smem {
   static constexpr uint32_t kP = kVc + 2 * kVSlices * kSlice;               // P^T: 2 x 16 KB (N = 128 rows)
   static constexpr uint32_t kScore = kP + 2 * kSlice;                       // [8][1024] fp32
   static constexpr uint32_t kLse = kScore + kTok * kMaxSel * 4;             // [128] fp32
-  static constexpr uint32_t kGate = kLse + kRowsM * 4;                      // [128] fp32
+  static constexpr uint32_t kGate = kLse + kRowsM * 4;                      // [2][128] fp32, by item parity
   static constexpr uint32_t kML = kP;                                       // [2][128][2] fp32, while P^T is unused
-  static constexpr uint32_t kBar = kGate + kRowsM * 4;                      // mbarriers
-  static constexpr int kNumBars = 1 + 2 * kKcSlots + 2 * 2 + 2 * 2 + 2 + 1;
+  static constexpr uint32_t kBar = kGate + 2 * kRowsM * 4;                  // mbarriers
+  static constexpr int kNumBars = 1 + 2 * kKcSlots + 2 * 2 + 2 * 2 + 2 + 1 + 4;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;                         // room to align the base to 1 KB
@@ -70,16 +76,91 @@ __device__ __forceinline__ int n_visible(int t, int nc) { return t < kL - 1 ? 0 
 using tc::named_sync;
 using tc::vote_all;
 
-// kWin = false: compressed branch (keys = compressed blocks, scores + top-k, acc = g_cmp * o).
-// kWin = true:  sliding window (keys = tokens [t0-w+1, t0+7], each row masked to its own
-//               window, out = bf16(acc + g_win * o)).
-template <int DK, int DV, bool kWin>
+// Top-k of one token over score[0, nb) (ties to the lower block index; blocks 0 and the
+// token's own block first when forced), written in increasing block order to dst[0, top_k)
+// with -1 padding.  Also zeroes score[0, nb) for the next item.  One warp.
+__device__ __forceinline__ void topk_token(float* score, int t, int top_k, int force_first, int force_local,
+                                           int32_t* dst, int lane) {
+  const int nb = t / kSel + 1;
+  if (nb <= top_k) {
+    for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
+    for (int j = lane; j < nb; j += 32) score[j] = 0.f;
+    return;
+  }
+  const int own = t / kSel;
+  uint32_t taken = 0;
+  int nforced = 0;
+  if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
+  if (force_local && !(force_first && own == 0)) {
+    if (lane == (own & 31)) taken |= 1u << (own >> 5);
+    ++nforced;
+  }
+  const int mmax = (nb + 31) >> 5;
+  // this lane's candidates j = lane + 32*mm as order-preserving integer keys: the scores
+  // are sums of probabilities (>= 0), so their bit patterns order like the values; key 0
+  // marks "no candidate"
+  uint32_t key[32];
+#pragma unroll
+  for (int mm = 0; mm < 32; ++mm) {
+    const int j = lane + 32 * mm;
+    const bool in = mm < mmax && j < nb;
+    key[mm] = (in && !((taken >> mm) & 1u)) ? __float_as_uint(score[j]) + 1u : 0u;
+    if (in) score[j] = 0.f;
+  }
+  // this lane's best key and its mm (the lowest mm among equal keys), by a pairwise tree
+  uint32_t bk = 0;
+  int bm = 0;
+  auto local_best = [&]() {
+    uint32_t k16[16];
+    int m16[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const bool c = key[2 * i + 1] > key[2 * i];
+      k16[i] = c ? key[2 * i + 1] : key[2 * i];
+      m16[i] = c ? 2 * i + 1 : 2 * i;
+    }
+#pragma unroll
+    for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) {
+        const bool c = k16[2 * i + 1] > k16[2 * i];
+        k16[i] = c ? k16[2 * i + 1] : k16[2 * i];
+        m16[i] = c ? m16[2 * i + 1] : m16[2 * i];
+      }
+    bk = k16[0];
+    bm = m16[0];
+  };
+  local_best();
+  for (int rr = nforced; rr < top_k; ++rr) {
+    const uint32_t vmax = __reduce_max_sync(0xffffffffu, bk);
+    if (vmax == 0u) break;
+    // the lowest block index among the lanes holding the maximum
+    const uint32_t jmin = __reduce_min_sync(0xffffffffu, bk == vmax ? (uint32_t)(lane + 32 * bm) : 0xffffffffu);
+    if (lane == (int)(jmin & 31u)) {
+      const int mw = (int)(jmin >> 5);
+      taken |= 1u << mw;
+#pragma unroll
+      for (int mm = 0; mm < 32; ++mm)
+        if (mm == mw) key[mm] = 0u;
+      local_best();
+    }
+  }
+  int pos = 0;
+  for (int mm = 0; mm < mmax; ++mm) {
+    const bool sel = (taken >> mm) & 1u;
+    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+    if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
+    pos += __popc(bal);
+  }
+  for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
+}
+
+template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                const __grid_constant__ CUtensorMap tm_vc, const __nv_bfloat16* __restrict__ gates,
-               float* __restrict__ acc, int32_t* __restrict__ idx_out, __nv_bfloat16* __restrict__ out, int T, int Hq,
-               int Hkv, int nc, int top_k, int force_first, int force_local, int window, float scale_log2,
-               int* __restrict__ err) {
+               float* __restrict__ acc, int32_t* __restrict__ idx_out, int B, int T, int Hq, int Hkv, int nc,
+               int top_k, int force_first, int force_local, float scale_log2, int* __restrict__ err) {
   using SM = Smem<DK, DV>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -102,17 +183,26 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* p_full = s_empty + 2;
   uint64_t* p_empty = p_full + 1;
   uint64_t* o_full = p_empty + 1;
+  uint64_t* q_empty = o_full + 1;    // the MMAs that read an item's Q have completed
+  uint64_t* sc_full = q_empty + 1;   // an item's block scores are complete
+  uint64_t* sc_empty = sc_full + 1;  // the top-k warps have read (and zeroed) them
+  uint64_t* o_empty = sc_empty + 1;  // the softmax warps have read an item's O^T
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tok_tiles = (T + kTok - 1) / kTok;
-  const int t0 = (n_tok_tiles - 1 - (int)blockIdx.x) * kTok;   // longest rows first
-  const int g = blockIdx.y, b = blockIdx.z;
-  const int t_last = min(t0 + kTok - 1, T - 1);
-  // keys: compressed blocks 0.. (kWin = false) or tokens kv_lo.. (kWin = true)
-  const int kv_lo = kWin ? max(0, t0 - window + 1) : 0;
-  const int ntiles = kWin ? (t_last - kv_lo + kBlk) / kBlk : (n_visible(t_last, nc) + kBlk - 1) / kBlk;
-  const int kv_rows = kWin ? T : nc;   // rows per batch in the key/value tensor maps
+  const int n_items = n_tok_tiles * Hkv * B;
+  // item -> (token tile, group, batch); the longest rows come first
+  struct Item { int t0, g, b, ntiles; };
+  auto item_of = [&](int it) {
+    Item x;
+    x.g = it % Hkv;
+    x.b = (it / Hkv) % B;
+    x.t0 = (n_tok_tiles - 1 - it / (Hkv * B)) * kTok;
+    const int t_last = min(x.t0 + kTok - 1, T - 1);
+    x.ntiles = (n_visible(t_last, nc) + kBlk - 1) / kBlk;
+    return x;
+  };
 
   if (tid == 0) {
     tc::mbar_init(bar_q, 1);
@@ -126,6 +216,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc::mbar_init(p_full, kSoftWarps);
     tc::mbar_init(p_empty, 1);
     tc::mbar_init(o_full, 1);
+    tc::mbar_init(q_empty, 1);
+    tc::mbar_init(sc_full, 1);
+    tc::mbar_init(sc_empty, kTopkWarps);
+    tc::mbar_init(o_empty, kSoftWarps);
     tc::fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -143,27 +237,37 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::prefetch_tmap(&tm_q);
       tc::prefetch_tmap(&tm_kc);
       tc::prefetch_tmap(&tm_vc);
-      tc::mbar_expect_tx(bar_q, SM::kQSlices * kSlice);
-      for (int s = 0; s < SM::kQSlices; ++s) tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, g * 16, b * T + t0);
-      int fill = 0;   // Kc slice fills so far
+      int fill = 0;   // Kc slice fills so far (all items)
+      int vcnt = 0;   // Vc tile fills so far
       bool ok = true;
-      for (int pass = 0; pass < 2 && ok; ++pass) {
-        for (int n = 0; n < ntiles && ok; ++n) {
-          const int row = b * kv_rows + kv_lo + n * kBlk;
-          for (int s = 0; s < SM::kQSlices && ok; ++s, ++fill) {
-            const int slot = fill % kKcSlots;
-            ok = tc::mbar_wait(kc_empty + slot, ((fill / kKcSlots) & 1) ^ 1, err, kErrKcEmpty);
-            if (!ok) break;
-            tc::mbar_expect_tx(kc_full + slot, kSlice);
-            tc::tma_load_3d(sKc + slot * kSlice, &tm_kc, kc_full + slot, s * 64, g, row);
-          }
-          if (pass == 1 && ok) {
-            const int vb = n & 1;
-            ok = tc::mbar_wait(vc_empty + vb, ((n >> 1) & 1) ^ 1, err, kErrVcEmpty);
-            if (!ok) break;
-            tc::mbar_expect_tx(vc_full + vb, SM::kVSlices * kSlice);
-            for (int s = 0; s < SM::kVSlices; ++s)
-              tc::tma_load_3d(sVc + (vb * SM::kVSlices + s) * kSlice, &tm_vc, vc_full + vb, s * 64, g, row);
+      int k = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+        const Item x = item_of(it);
+        // Q of this item once the previous item's S MMAs are done with the buffer
+        if (k > 0) ok = tc::mbar_wait(q_empty, (k - 1) & 1, err, kErrQEmpty);
+        if (!ok) break;
+        tc::mbar_expect_tx(bar_q, SM::kQSlices * kSlice);
+        for (int s = 0; s < SM::kQSlices; ++s)
+          tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, x.g * 16, x.b * T + x.t0);
+        for (int pass = 0; pass < 2 && ok; ++pass) {
+          for (int n = 0; n < x.ntiles && ok; ++n) {
+            const int row = x.b * nc + n * kBlk;
+            for (int s = 0; s < SM::kQSlices && ok; ++s, ++fill) {
+              const int slot = fill % kKcSlots;
+              ok = tc::mbar_wait(kc_empty + slot, ((fill / kKcSlots) & 1) ^ 1, err, kErrKcEmpty);
+              if (!ok) break;
+              tc::mbar_expect_tx(kc_full + slot, kSlice);
+              tc::tma_load_3d(sKc + slot * kSlice, &tm_kc, kc_full + slot, s * 64, x.g, row);
+            }
+            if (pass == 1 && ok) {
+              const int vb = vcnt & 1;
+              ok = tc::mbar_wait(vc_empty + vb, ((vcnt >> 1) & 1) ^ 1, err, kErrVcEmpty);
+              if (!ok) break;
+              tc::mbar_expect_tx(vc_full + vb, SM::kVSlices * kSlice);
+              for (int s = 0; s < SM::kVSlices; ++s)
+                tc::tma_load_3d(sVc + (vb * SM::kVSlices + s) * kSlice, &tm_vc, vc_full + vb, s * 64, x.g, row);
+              ++vcnt;
+            }
           }
         }
       }
@@ -172,56 +276,91 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int f = fill - 1 - i;
         tc::mbar_wait(kc_full + (f % kKcSlots), (f / kKcSlots) & 1, err, kErrKcFull);
       }
-      for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
+      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
+      if (k > 0) tc::mbar_wait(bar_q, (k - 1) & 1, err, kErrQ);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (tc::elect_one()) {
       const uint32_t idA = tc::idesc_bf16(128, 128, 0, 0);     // S  = Q  Kc^T   (both K-major)
       const uint32_t idPV = tc::idesc_bf16(128, 128, 1, 1);    // O^T = Vc^T P^T (both MN-major)
-      bool ok = tc::mbar_wait(bar_q, 0, err, kErrQ);
-      tc::tc_fence_after();
-      int use = 0;    // S buffer uses over both passes
+      int use = 0;    // S buffer uses (all items, both passes)
       int fill = 0;   // Kc slices consumed
-      auto issue_s = [&](int pass) -> bool {
-        const int sb = use & 1;
-        if (!tc::mbar_wait(s_empty + sb, ((use >> 1) & 1) ^ 1, err, kErrSEmpty)) return false;
+      int pc = 0;     // pass-B tiles (P^T phases, Vc tiles) so far
+      bool ok = true;
+      int k = 0;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+        const Item x = item_of(it);
+        ok = tc::mbar_wait(bar_q, k & 1, err, kErrQ);
+        if (!ok) break;
         tc::tc_fence_after();
-        const uint32_t d = tmem + (sb ? kColS1 : kColS0);
-        for (int s = 0; s < SM::kQSlices; ++s, ++fill) {
-          const int slot = fill % kKcSlots;
-          if (!tc::mbar_wait(kc_full + slot, (fill / kKcSlots) & 1, err, kErrKcFull)) return false;
+        auto issue_s = [&](int pass) -> bool {
+          const int sb = use & 1;
+          if (!tc::mbar_wait(s_empty + sb, ((use >> 1) & 1) ^ 1, err, kErrSEmpty)) return false;
           tc::tc_fence_after();
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t dq = tc::sdesc(sQ + s * kSlice + ks * 32, 16, 1024);
-            const uint64_t dk = tc::sdesc(sKc + slot * kSlice + ks * 32, 16, 1024);
-            if (pass == 0) tc::mma_ss(d, dq, dk, idA, (s | ks) != 0);
-            else tc::mma_ss(d, dk, dq, idA, (s | ks) != 0);
+          const uint32_t d = tmem + (sb ? kColS1 : kColS0);
+          for (int s = 0; s < SM::kQSlices; ++s, ++fill) {
+            const int slot = fill % kKcSlots;
+            if (!tc::mbar_wait(kc_full + slot, (fill / kKcSlots) & 1, err, kErrKcFull)) return false;
+            tc::tc_fence_after();
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t dq = tc::sdesc(sQ + s * kSlice + ks * 32, 16, 1024);
+              const uint64_t dk = tc::sdesc(sKc + slot * kSlice + ks * 32, 16, 1024);
+              if (pass == 0) tc::mma_ss(d, dq, dk, idA, (s | ks) != 0);
+              else tc::mma_ss(d, dk, dq, idA, (s | ks) != 0);
+            }
+            tc::mma_commit(kc_empty + slot);
           }
-          tc::mma_commit(kc_empty + slot);
+          tc::mma_commit(s_full + sb);
+          ++use;
+          return true;
+        };
+        for (int n = 0; n < x.ntiles && ok; ++n) ok = issue_s(0);
+        if (ok && x.ntiles > 0) ok = issue_s(1);
+        if (ok && x.ntiles <= 1) tc::mma_commit(q_empty);
+        // O^T is overwritten (and o_full committed) only after the previous item's epilogue read it
+        if (ok && k > 0) ok = tc::mbar_wait(o_empty, (k - 1) & 1, err, kErrOEmpty);
+        for (int n = 0; n < x.ntiles && ok; ++n, ++pc) {
+          if (n + 1 < x.ntiles) {
+            ok = issue_s(1);
+            if (ok && n + 2 == x.ntiles) tc::mma_commit(q_empty);   // the item's last S reads Q
+          }
+          if (!ok) break;
+          ok = tc::mbar_wait(p_full, pc & 1, err, kErrPFull) &&
+               tc::mbar_wait(vc_full + (pc & 1), (pc >> 1) & 1, err, kErrVcFull);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint8_t* vb = sVc + (pc & 1) * SM::kVSlices * kSlice;
+          for (int ks = 0; ks < kBlk / 16; ++ks) {
+            const uint64_t da = tc::sdesc(vb + ks * 16 * 128, kSlice, 1024);
+            const uint64_t db = tc::sdesc(sP + ks * 16 * 128, kSlice, 1024);
+            tc::mma_ss(tmem + kColO, da, db, idPV, (n | ks) != 0);
+          }
+          tc::mma_commit(p_empty);
+          tc::mma_commit(vc_empty + (pc & 1));
         }
-        tc::mma_commit(s_full + sb);
-        ++use;
-        return true;
-      };
-      for (int n = 0; n < ntiles && ok; ++n) ok = issue_s(0);
-      if (ok && ntiles > 0) ok = issue_s(1);
-      for (int n = 0; n < ntiles && ok; ++n) {
-        if (n + 1 < ntiles) ok = issue_s(1);
-        if (!ok) break;
-        ok = tc::mbar_wait(p_full, n & 1, err, kErrPFull) && tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
-        if (!ok) break;
-        tc::tc_fence_after();
-        const uint8_t* vb = sVc + (n & 1) * SM::kVSlices * kSlice;
-        for (int ks = 0; ks < kBlk / 16; ++ks) {
-          const uint64_t da = tc::sdesc(vb + ks * 16 * 128, kSlice, 1024);
-          const uint64_t db = tc::sdesc(sP + ks * 16 * 128, kSlice, 1024);
-          tc::mma_ss(tmem + kColO, da, db, idPV, (n | ks) != 0);
-        }
-        tc::mma_commit(p_empty);
-        tc::mma_commit(vc_empty + (n & 1));
+        if (ok) tc::mma_commit(o_full);
       }
-      if (ok && ntiles > 0) tc::mma_commit(o_full);
+    }
+  } else if (warp >= kTopkWarp0) {
+    // ------------------------------------------------------------ top-k
+    // warp kTopkWarp0 + i takes tokens 4i .. 4i+3 of each item
+    const int w = warp - kTopkWarp0;
+    bool ok = true;
+    int k = 0;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      const Item x = item_of(it);
+      ok = tc::mbar_wait(sc_full, k & 1, err, kErrScFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      for (int kk = 4 * w; kk < 4 * w + 4; ++kk) {
+        const int t = x.t0 + kk;
+        if (t < T)
+          topk_token(sScore + kk * kMaxSel, t, top_k, force_first, force_local,
+                     idx_out + (((size_t)x.b * Hkv + x.g) * T + t) * top_k, lane);
+      }
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(sc_empty);
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
@@ -232,24 +371,114 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const int col0 = 64 * gr;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
     bool ok = true;
-    int use = 0;
-    if (gr == 0) {   // gates of the 128 rows
-      const int t = t0 + r / 16, h = g * 16 + (r % 16);
-      sGate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3 + (kWin ? 2 : 0)]) : 0.f;
-    }
-    if (!kWin)
-      for (int i = gr * 128 + r; i < kTok * kMaxSel; i += 256) sScore[i] = 0.f;
+    int use = 0;   // S buffer uses
+    int pc = 0;    // pass-B tiles
+    for (int i = gr * 128 + r; i < kTok * kMaxSel; i += 256) sScore[i] = 0.f;
+    int k = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+      const Item x = item_of(it);
+      const int t0 = x.t0, g = x.g, b = x.b, ntiles = x.ntiles;
+      float* gate = sGate + (k & 1) * kRowsM;
+      if (gr == 0) {   // gates of the 128 rows (double-buffered: group 1 may still be in the previous epilogue)
+        const int t = t0 + r / 16, h = g * 16 + (r % 16);
+        gate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3]) : 0.f;
+      }
 
-    // pass A: this thread's row r = (token r/16, head r%16), its half of every tile's columns
-    {
-      const int my_t = t0 + r / 16;
-      const int my_lo = kWin ? max(0, my_t - window + 1) : 0;
-      const int my_hi = my_t < T ? (kWin ? my_t + 1 : n_visible(my_t, nc)) : 0;
-      float m = -INFINITY, l = 0.f;
-      for (int n = 0; n < ntiles && ok; ++n, ++use) {
+      // pass A: this thread's row r = (token r/16, head r%16), its half of every tile's columns
+      {
+        const int my_t = t0 + r / 16;
+        const int my_hi = my_t < T ? n_visible(my_t, nc) : 0;
+        float m = -INFINITY, l = 0.f;
+        for (int n = 0; n < ntiles && ok; ++n, ++use) {
+          const int sb = use & 1;
+          ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
+          ok = __all_sync(0xffffffffu, ok);      // reconverge before the warp-wide TMEM loads
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
+          float v[64];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+          tc::tmem_wait_ld();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(s_empty + sb);
+          // masked, scaled scores; only a tile that straddles this row's range needs the
+          // per-element test.  Max and sum use eight independent chains each.
+          const int i0 = n * kBlk + col0;
+          if (i0 + 63 < my_hi) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] *= scale_log2;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = i0 + j < my_hi ? v[j] * scale_log2 : -INFINITY;
+          }
+          float cmx[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(fmaxf(v[c], v[c + 8]), fmaxf(v[c + 16], v[c + 24]));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
+          const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                                 fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+          const float mn = fmaxf(m, cm);
+          if (mn != -INFINITY) {
+            float ps[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) ps[c] = ex2(v[c] - mn);
+#pragma unroll
+            for (int j = 8; j < 64; ++j) ps[j & 7] += ex2(v[j] - mn);
+            const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+            l = l * ex2(m - mn) + sum;
+            m = mn;
+          }
+        }
+        sML[(gr * 128 + r) * 2] = m;
+        sML[(gr * 128 + r) * 2 + 1] = l;
+      }
+      ok = vote_all(3, kSoftWarps * 32, ok);
+      if (!ok) break;
+      if (gr == 0) {
+        const float m0 = sML[r * 2], l0 = sML[r * 2 + 1], m1 = sML[(128 + r) * 2], l1 = sML[(128 + r) * 2 + 1];
+        const float M = fmaxf(m0, m1);
+        const float L = M == -INFINITY ? 0.f : l0 * ex2(m0 - M) + l1 * ex2(m1 - M);
+        sLse[r] = (t0 + r / 16 < T && L > 0.f) ? M + __log2f(L) : INFINITY;
+      }
+      // the previous item's scores must have been taken (and zeroed) by the top-k warps
+      if (k > 0) ok = tc::mbar_wait(sc_empty, (k - 1) & 1, err, kErrScEmpty);
+      ok = vote_all(3, kSoftWarps * 32, ok);
+      if (!ok) break;
+
+      // pass B: this thread's key r of every tile; columns = tokens 4*gr .. 4*gr+3, 16 heads each
+      int hi_tok[4], nb_tok[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int t = t0 + 4 * gr + kk;
+        const bool in = t < T;
+        hi_tok[kk] = in ? n_visible(t, nc) : 0;
+        nb_tok[kk] = in ? t / kSel + 1 : 0;
+      }
+      uint8_t* prow = sP + gr * kSlice + r * 128;   // row r of N-block gr of P^T
+      // Selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Each group of four
+      // lanes adds its own four blocks plus the lane just below it into the block's entry.
+      // Lane 31's block (i % 4 == 3) also belongs to the first selection block of the next
+      // warp (or of the next tile); that carry is added two tiles later, after waiting for
+      // the P^T phase that every softmax warp releases only after its own score writes, so
+      // no barrier is needed inside the loop.  Each entry receives at most two additions.
+      float carry_a[4] = {0.f, 0.f, 0.f, 0.f}, carry_b[4] = {0.f, 0.f, 0.f, 0.f};   // tiles n-1, n-2
+      auto add_carry = [&](const float (&c)[4], int tile) {
+        const int jt = tile * (kBlk / 4) + q4 * 8 + 8;
+        if (lane == 31) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            if (jt < nb_tok[kk]) sScore[(4 * gr + kk) * kMaxSel + jt] += c[kk];
+        }
+      };
+      for (int n = 0; n < ntiles; ++n, ++use, ++pc) {
         const int sb = use & 1;
+        // no barrier inside this loop: a warp that gives up leaves at once and the others
+        // give up at their next wait (they see the error word); all meet after the loop
         ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
-        ok = __all_sync(0xffffffffu, ok);      // reconverge before the warp-wide TMEM loads
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc::tc_fence_after();
         const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
@@ -257,248 +486,96 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
         tc::tmem_wait_ld();
+        const int i = n * kBlk + r;        // this thread's compressed block
+        float tok_sum[4];
+        uint32_t pk[32];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const bool vis = i < hi_tok[kk];
+          float s = 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const float p0 = vis ? ex2(v[16 * kk + j] * scale_log2 - sLse[col0 + 16 * kk + j]) : 0.f;
+            const float p1 = vis ? ex2(v[16 * kk + j + 1] * scale_log2 - sLse[col0 + 16 * kk + j + 1]) : 0.f;
+            s += p0 + p1;
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            pk[8 * kk + j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          tok_sum[kk] = s;
+        }
+        {
+          const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const float vv = tok_sum[kk];
+            float g4 = vv + __shfl_xor_sync(0xffffffffu, vv, 1);
+            g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
+            const float prev = __shfl_up_sync(0xffffffffu, vv, 1);
+            const int j = j0 + (lane >> 2);
+            if ((lane & 3) == 0 && j < nb_tok[kk]) sScore[(4 * gr + kk) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
+          }
+        }
+        // P^T(pc) may overwrite the buffer once PV(pc-1) has read it
+        if (pc > 0) ok = tc::mbar_wait(p_empty, (pc - 1) & 1, err, kErrPEmpty);
+        if (n > 0 && ok) {
+          // P^T(pc-1) was released by every softmax warp after its score writes of tiles
+          // <= n-1; this warp has not released P^T(pc) yet, so the phase is unambiguous
+          ok = tc::mbar_wait(p_full, (pc - 1) & 1, err, kErrPFull);
+          if (n > 1) add_carry(carry_b, n - 2);
+        }
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          carry_b[kk] = carry_a[kk];
+          carry_a[kk] = tok_sum[kk];
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         tc::tc_fence_before();
+        tc::fence_async_smem();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(s_empty + sb);
-        // masked, scaled scores; only a tile that straddles this row's range needs the
-        // per-element test.  Max and sum use eight independent chains each.
-        const int i0 = kv_lo + n * kBlk + col0;
-        if (i0 >= my_lo && i0 + 63 < my_hi) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] *= scale_log2;
-        } else {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = (i0 + j >= my_lo && i0 + j < my_hi) ? v[j] * scale_log2 : -INFINITY;
-        }
-        float cmx[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(fmaxf(v[c], v[c + 8]), fmaxf(v[c + 16], v[c + 24]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
-        const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
-                               fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
-        const float mn = fmaxf(m, cm);
-        if (mn != -INFINITY) {
-          float ps[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) ps[c] = ex2(v[c] - mn);
-#pragma unroll
-          for (int j = 8; j < 64; ++j) ps[j & 7] += ex2(v[j] - mn);
-          const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-          l = l * ex2(m - mn) + sum;
-          m = mn;
+        if (lane == 0) {
+          tc::mbar_arrive(s_empty + sb);
+          tc::mbar_arrive(p_full);
         }
       }
-      sML[(gr * 128 + r) * 2] = m;
-      sML[(gr * 128 + r) * 2 + 1] = l;
-    }
-    ok = vote_all(3, kSoftWarps * 32, ok);
-    if (gr == 0) {
-      const float m0 = sML[r * 2], l0 = sML[r * 2 + 1], m1 = sML[(128 + r) * 2], l1 = sML[(128 + r) * 2 + 1];
-      const float M = fmaxf(m0, m1);
-      const float L = M == -INFINITY ? 0.f : l0 * ex2(m0 - M) + l1 * ex2(m1 - M);
-      sLse[r] = (t0 + r / 16 < T && L > 0.f) ? M + __log2f(L) : INFINITY;
-    }
-    named_sync(3, kSoftWarps * 32);
-
-    // pass B: this thread's key r of every tile; columns = tokens 4*gr .. 4*gr+3, 16 heads each
-    int lo_tok[4], hi_tok[4], nb_tok[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int t = t0 + 4 * gr + k;
-      const bool in = t < T;
-      lo_tok[k] = kWin ? max(0, t - window + 1) : 0;
-      hi_tok[k] = in ? (kWin ? t + 1 : n_visible(t, nc)) : 0;
-      nb_tok[k] = in ? t / kSel + 1 : 0;
-    }
-    uint8_t* prow = sP + gr * kSlice + r * 128;   // row r of N-block gr of P^T
-    // Selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Each group of four
-    // lanes adds its own four blocks plus the lane just below it into the block's entry.
-    // Lane 31's block (i % 4 == 3) also belongs to the first selection block of the next
-    // warp (or of the next tile); that carry is added two tiles later, after waiting for
-    // the P^T phase that every softmax warp releases only after its own score writes, so
-    // no barrier is needed inside the loop.  Each entry receives at most two additions.
-    float carry_a[4] = {0.f, 0.f, 0.f, 0.f}, carry_b[4] = {0.f, 0.f, 0.f, 0.f};   // tiles n-1, n-2
-    auto add_carry = [&](const float (&c)[4], int tile) {
-      const int jt = tile * (kBlk / 4) + q4 * 8 + 8;
-      if (lane == 31) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          if (jt < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + jt] += c[k];
-      }
-    };
-    for (int n = 0; n < ntiles; ++n, ++use) {
-      const int sb = use & 1;
-      // no barrier inside this loop: a warp that gives up leaves at once and the others
-      // give up at their next wait (they see the error word); all meet after the loop
-      ok = tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = vote_all(3, kSoftWarps * 32, ok);
       if (!ok) break;
-      tc::tc_fence_after();
-      const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
-      float v[64];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
-      tc::tmem_wait_ld();
-      const int i = kv_lo + n * kBlk + r;        // this thread's key (compressed block or token)
-      float tok_sum[4];
-      uint32_t pk[32];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const bool vis = i >= lo_tok[k] && i < hi_tok[k];
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < 16; j += 2) {
-          const float p0 = vis ? ex2(v[16 * k + j] * scale_log2 - sLse[col0 + 16 * k + j]) : 0.f;
-          const float p1 = vis ? ex2(v[16 * k + j + 1] * scale_log2 - sLse[col0 + 16 * k + j + 1]) : 0.f;
-          s += p0 + p1;
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-          pk[8 * k + j / 2] = *reinterpret_cast<uint32_t*>(&h2);
-        }
-        tok_sum[k] = s;
-      }
-      if (!kWin) {
-        const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float vv = tok_sum[k];
-          float g4 = vv + __shfl_xor_sync(0xffffffffu, vv, 1);
-          g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
-          const float prev = __shfl_up_sync(0xffffffffu, vv, 1);
-          const int j = j0 + (lane >> 2);
-          if ((lane & 3) == 0 && j < nb_tok[k]) sScore[(4 * gr + k) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
-        }
-      }
-      // P^T(n) may overwrite the buffer once PV(n-1) has read it
-      if (n > 0) ok = tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty);
-      if (!kWin && n > 0 && ok) {
-        // P^T(n-1) was released by every softmax warp after its score writes of tiles
-        // <= n-1; this warp has not released P^T(n) yet, so the phase is unambiguous
-        ok = tc::mbar_wait(p_full, (n - 1) & 1, err, kErrPFull);
-        if (n > 1) add_carry(carry_b, n - 2);
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        carry_b[k] = carry_a[k];
-        carry_a[k] = tok_sum[k];
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      tc::tc_fence_before();
-      tc::fence_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tc::mbar_arrive(s_empty + sb);
-        tc::mbar_arrive(p_full);
-      }
-    }
-    ok = vote_all(3, kSoftWarps * 32, ok);
-    if (!kWin && ok) {    // the carries of the last two tiles
+      // the carries of the last two tiles, then hand the scores to the top-k warps
       if (ntiles > 1) add_carry(carry_b, ntiles - 2);
       if (ntiles > 0) add_carry(carry_a, ntiles - 1);
-    }
-    named_sync(3, kSoftWarps * 32);
+      named_sync(3, kSoftWarps * 32);
+      if (tid == 0) tc::mbar_arrive(sc_full);
 
-    // top-k: warp w takes token w
-    if (!kWin && ok) {
-      const int k = warp;
-      const int t = t0 + k;
-      if (t < T) {
-        const float* score = sScore + k * kMaxSel;
-        const int nb = t / kSel + 1;
-        int32_t* dst = idx_out + (((size_t)b * Hkv + g) * T + t) * top_k;
-        if (nb <= top_k) {
-          for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
+      // epilogue: lane r = value dim r of O^T; this group's 64 columns = tokens 4*gr .. 4*gr+3.
+      // A failed wait here only skips the stores: the next item's vote ends the loop for all.
+      ok = tc::mbar_wait(o_full, k & 1, err, kErrOFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc::tc_fence_after();
+        float v[64];
+        if (ntiles > 0) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tc::tmem_ld16(lane_addr + kColO + col0 + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+          tc::tmem_wait_ld();
         } else {
-          const int own = t / kSel;
-          uint32_t taken = 0;
-          int nforced = 0;
-          if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
-          if (force_local && !(force_first && own == 0)) {
-            if (lane == (own & 31)) taken |= 1u << (own >> 5);
-            ++nforced;
-          }
-          const int mmax = (nb + 31) >> 5;
-          // this lane's candidates j = lane + 32*mm as order-preserving integer keys: the
-          // scores are sums of probabilities (>= 0), so their bit patterns order like the
-          // values; key 0 marks "no candidate"
-          uint32_t key[32];
 #pragma unroll
-          for (int mm = 0; mm < 32; ++mm) {
-            const int j = lane + 32 * mm;
-            key[mm] = (mm < mmax && j < nb && !((taken >> mm) & 1u)) ? __float_as_uint(score[j]) + 1u : 0u;
-          }
-          uint32_t bk = 0;   // this lane's best key and its mm (the lowest mm among equal keys)
-          int bm = 0;
-          auto local_best = [&]() {
-            bk = 0;
-            bm = 0;
-#pragma unroll
-            for (int mm = 0; mm < 32; ++mm)
-              if (key[mm] > bk) { bk = key[mm]; bm = mm; }
-          };
-          local_best();
-          for (int rr = nforced; rr < top_k; ++rr) {
-            const uint32_t vmax = __reduce_max_sync(0xffffffffu, bk);
-            if (vmax == 0u) break;
-            // the lowest block index among the lanes holding the maximum
-            const uint32_t jmin = __reduce_min_sync(0xffffffffu, bk == vmax ? (uint32_t)(lane + 32 * bm) : 0xffffffffu);
-            if (lane == (int)(jmin & 31u)) {
-              const int mw = (int)(jmin >> 5);
-              taken |= 1u << mw;
-#pragma unroll
-              for (int mm = 0; mm < 32; ++mm)
-                if (mm == mw) key[mm] = 0u;
-              local_best();
-            }
-          }
-          int pos = 0;
-          for (int mm = 0; mm < mmax; ++mm) {
-            const bool sel = (taken >> mm) & 1u;
-            const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-            if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
-            pos += __popc(bal);
-          }
-          for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
+          for (int c = 0; c < 64; ++c) v[c] = 0.f;
         }
-      }
-    }
-
-    // epilogue: lane r = value dim r of O^T; this group's 64 columns = tokens 4*gr .. 4*gr+3
-    float prevacc[kWin ? 64 : 1];
-    if (kWin) {
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(o_empty);
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int t = t0 + 4 * gr + c / 16;
-        const size_t row = ((size_t)b * T + min(t, T - 1)) * Hq + g * 16 + (c % 16);
-        prevacc[c] = (t < T && r < DV) ? acc[row * DV + r] : 0.f;
-      }
-    }
-    if (ok && ntiles > 0) ok = tc::mbar_wait(o_full, 0, err, kErrOFull);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      tc::tc_fence_after();
-      float v[64];
-      if (ntiles > 0) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tc::tmem_ld16(lane_addr + kColO + col0 + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
-        tc::tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) v[c] = 0.f;
-      }
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const int t = t0 + 4 * gr + c / 16;
-        if (t < T && r < DV) {
-          const size_t row = ((size_t)b * T + t) * Hq + g * 16 + (c % 16);
-          const float gv = sGate[col0 + c] * v[c];
-          if (kWin) out[row * DV + r] = __float2bfloat16_rn(prevacc[c] + gv);
-          else acc[row * DV + r] = gv;
+        for (int c = 0; c < 64; ++c) {
+          const int t = t0 + 4 * gr + c / 16;
+          if (t < T && r < DV) {
+            const size_t row = ((size_t)b * T + t) * Hq + g * 16 + (c % 16);
+            acc[row * DV + r] = gate[col0 + c] * v[c];
+          }
         }
       }
     }
@@ -512,40 +589,44 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
 }
 
-template <int DK, int DV, bool kWin>
+template <int DK, int DV>
 cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   using SM = Smem<DK, DV>;
   static bool attr = false;
+  static int sms = 0;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV, kWin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::kAlloc);
     if (e != cudaSuccess) return e;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
     attr = true;
   }
-  const int rows = kWin ? a.T : a.nc;
-  const void* kp = kWin ? a.k : a.kc;
-  const void* vp = kWin ? a.v : a.vc;
   CUtensorMap mq, mk, mv;
   const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
   const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
   const uint32_t bq[3] = {64, 16, kTok};
-  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * rows};
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
   const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
-  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * rows};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
   const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
   const uint32_t bkv[3] = {64, 1, kBlk};
   if (!make_tmap_bf16(&mq, a.q, 3, dq, sq, bq)) return cudaErrorInvalidValue;
-  if (rows > 0) {
-    if (!make_tmap_bf16(&mk, kp, 3, dk3, sk3, bkv) || !make_tmap_bf16(&mv, vp, 3, dv3, sv3, bkv))
+  if (a.nc > 0) {
+    if (!make_tmap_bf16(&mk, a.kc, 3, dk3, sk3, bkv) || !make_tmap_bf16(&mv, a.vc, 3, dv3, sv3, bkv))
       return cudaErrorInvalidValue;
   } else {
-    mk = mq;   // never dereferenced: no tile is loaded when there is no key
+    mk = mq;   // never dereferenced: no tile is loaded when there is no compressed block
     mv = mq;
   }
-  dim3 grid((a.T + kTok - 1) / kTok, a.Hkv, a.B);
-  attn_tc_kernel<DK, DV, kWin><<<grid, kThreads, SM::kAlloc, st>>>(
-      mq, mk, mv, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, static_cast<__nv_bfloat16*>(a.out), a.T,
-      a.Hq, a.Hkv, a.nc, a.top_k, a.force_first, a.force_local, a.window, a.scale_log2, a.err);
+  const long long n_items = (long long)((a.T + kTok - 1) / kTok) * a.Hkv * a.B;
+  if (n_items == 0) return cudaSuccess;
+  const int grid = (int)std::min<long long>(n_items, sms);
+  attn_tc_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
+      mq, mk, mv, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, a.B, a.T, a.Hq, a.Hkv, a.nc, a.top_k,
+      a.force_first, a.force_local, a.scale_log2, a.err);
   return cudaGetLastError();
 }
 }  // namespace
@@ -555,15 +636,8 @@ bool cmp_select_tc_supported(const FwdArgs& a) {
 }
 
 cudaError_t launch_cmp_select_tc(const FwdArgs& a, cudaStream_t st) {
-  if (a.dk == 192) return launch_tc<192, 128, false>(a, st);
-  return launch_tc<128, 128, false>(a, st);
-}
-
-bool swa_tc_supported(const FwdArgs& a) { return cmp_select_tc_supported(a); }
-
-cudaError_t launch_swa_tc(const FwdArgs& a, cudaStream_t st) {
-  if (a.dk == 192) return launch_tc<192, 128, true>(a, st);
-  return launch_tc<128, 128, true>(a, st);
+  if (a.dk == 192) return launch_tc<192, 128>(a, st);
+  return launch_tc<128, 128>(a, st);
 }
 
 }  // namespace nsa

@@ -40,8 +40,6 @@ bool slc_attn_tma_supported(const FwdArgs& a);
 cudaError_t launch_slc_attn_tma(const FwdArgs& a, cudaStream_t st);
 // K4 + K5: sliding window and gated combine (out = bf16(acc + g_win * o_win)).
 cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st);
-bool swa_tc_supported(const FwdArgs& a);
-cudaError_t launch_swa_tc(const FwdArgs& a, cudaStream_t st);
 // K4 + K5 in one pass on tcgen05 (G == 16, d_v == 128, d_k in {128, 192}).
 bool window_tc_supported(const FwdArgs& a);
 cudaError_t launch_window_tc(const FwdArgs& a, cudaStream_t st);

@@ -213,7 +213,6 @@ cudaError_t launch(const FwdArgs& a, cudaStream_t st) {
 
 cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st) {
   if (window_tc_supported(a)) return launch_window_tc(a, st);
-  if (swa_tc_supported(a)) return launch_swa_tc(a, st);
   if (a.dk == 64 && a.dv == 64) return launch<64, 64>(a, st);
   if (a.dk == 128 && a.dv == 128) return launch<128, 128>(a, st);
   if (a.dk == 192 && a.dv == 128) return launch<192, 128>(a, st);

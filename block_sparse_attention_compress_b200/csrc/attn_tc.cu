@@ -76,84 +76,96 @@ __device__ __forceinline__ int n_visible(int t, int nc) { return t < kL - 1 ? 0 
 using tc::named_sync;
 using tc::vote_all;
 
-// Top-k of one token over score[0, nb) (ties to the lower block index; blocks 0 and the
-// token's own block first when forced), written in increasing block order to dst[0, top_k)
-// with -1 padding.  Also zeroes score[0, nb) for the next item.  One warp.
-__device__ __forceinline__ void topk_token(float* score, int t, int top_k, int force_first, int force_local,
-                                           int32_t* dst, int lane) {
-  const int nb = t / kSel + 1;
-  if (nb <= top_k) {
-    for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
-    for (int j = lane; j < nb; j += 32) score[j] = 0.f;
-    return;
-  }
-  const int own = t / kSel;
-  uint32_t taken = 0;
-  int nforced = 0;
-  if (force_first) { if (lane == 0) taken |= 1u; ++nforced; }
-  if (force_local && !(force_first && own == 0)) {
-    if (lane == (own & 31)) taken |= 1u << (own >> 5);
-    ++nforced;
-  }
-  const int mmax = (nb + 31) >> 5;
-  // this lane's candidates j = lane + 32*mm as order-preserving integer keys: the scores
-  // are sums of probabilities (>= 0), so their bit patterns order like the values; key 0
-  // marks "no candidate"
-  uint32_t key[32];
+// Top-k of NT tokens (one warp).  Phase 1 copies each token's scores score[k][0, nb_k) into
+// registers as order-preserving integer keys (the scores are sums of probabilities, >= 0,
+// so their bit patterns order like the values; key 0 marks "no candidate") and zeroes the
+// entries for the next item, so the caller can release the score buffer right after it.
+// Phase 2 selects per token: forced blocks 0 and the token's own block first, then the
+// largest scores, ties to the lower block index; written in increasing block order to
+// dst[k][0, top_k) with -1 padding.
+template <int NT>
+struct TopkWarp {
+  uint32_t key[NT][32];
+  uint32_t taken[NT];
+
+  __device__ __forceinline__ void load(float* score, int stride, const int (&nb)[NT], const int (&own)[NT],
+                                       int force_first, int force_local, int lane) {
 #pragma unroll
-  for (int mm = 0; mm < 32; ++mm) {
-    const int j = lane + 32 * mm;
-    const bool in = mm < mmax && j < nb;
-    key[mm] = (in && !((taken >> mm) & 1u)) ? __float_as_uint(score[j]) + 1u : 0u;
-    if (in) score[j] = 0.f;
-  }
-  // this lane's best key and its mm (the lowest mm among equal keys), by a pairwise tree
-  uint32_t bk = 0;
-  int bm = 0;
-  auto local_best = [&]() {
-    uint32_t k16[16];
-    int m16[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const bool c = key[2 * i + 1] > key[2 * i];
-      k16[i] = c ? key[2 * i + 1] : key[2 * i];
-      m16[i] = c ? 2 * i + 1 : 2 * i;
-    }
-#pragma unroll
-    for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-      for (int i = 0; i < w; ++i) {
-        const bool c = k16[2 * i + 1] > k16[2 * i];
-        k16[i] = c ? k16[2 * i + 1] : k16[2 * i];
-        m16[i] = c ? m16[2 * i + 1] : m16[2 * i];
+    for (int k = 0; k < NT; ++k) {
+      taken[k] = 0;
+      if (nb[k] > 0) {
+        if (force_first && lane == 0) taken[k] |= 1u;
+        if (force_local && lane == (own[k] & 31)) taken[k] |= 1u << (own[k] >> 5);
       }
-    bk = k16[0];
-    bm = m16[0];
-  };
-  local_best();
-  for (int rr = nforced; rr < top_k; ++rr) {
-    const uint32_t vmax = __reduce_max_sync(0xffffffffu, bk);
-    if (vmax == 0u) break;
-    // the lowest block index among the lanes holding the maximum
-    const uint32_t jmin = __reduce_min_sync(0xffffffffu, bk == vmax ? (uint32_t)(lane + 32 * bm) : 0xffffffffu);
-    if (lane == (int)(jmin & 31u)) {
-      const int mw = (int)(jmin >> 5);
-      taken |= 1u << mw;
 #pragma unroll
-      for (int mm = 0; mm < 32; ++mm)
-        if (mm == mw) key[mm] = 0u;
-      local_best();
+      for (int mm = 0; mm < 32; ++mm) {
+        const int j = lane + 32 * mm;
+        const bool in = j < nb[k];
+        key[k][mm] = (in && !((taken[k] >> mm) & 1u)) ? __float_as_uint(score[k * stride + j]) + 1u : 0u;
+        if (in) score[k * stride + j] = 0.f;
+      }
     }
   }
-  int pos = 0;
-  for (int mm = 0; mm < mmax; ++mm) {
-    const bool sel = (taken >> mm) & 1u;
-    const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-    if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
-    pos += __popc(bal);
+
+  template <int K>
+  __device__ __forceinline__ void select(int nb, int own, int top_k, int force_first, int force_local,
+                                         int32_t* dst, int lane) {
+    if (nb <= 0) return;
+    if (nb <= top_k) {
+      for (int j = lane; j < top_k; j += 32) dst[j] = j < nb ? j : -1;
+      return;
+    }
+    int nforced = force_first ? 1 : 0;
+    if (force_local && !(force_first && own == 0)) ++nforced;
+    // this lane's best key and its mm (the lowest mm among equal keys), by a pairwise tree
+    uint32_t bk = 0;
+    int bm = 0;
+    auto local_best = [&]() {
+      uint32_t k16[16];
+      int m16[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const bool c = key[K][2 * i + 1] > key[K][2 * i];
+        k16[i] = c ? key[K][2 * i + 1] : key[K][2 * i];
+        m16[i] = c ? 2 * i + 1 : 2 * i;
+      }
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+          const bool c = k16[2 * i + 1] > k16[2 * i];
+          k16[i] = c ? k16[2 * i + 1] : k16[2 * i];
+          m16[i] = c ? m16[2 * i + 1] : m16[2 * i];
+        }
+      bk = k16[0];
+      bm = m16[0];
+    };
+    local_best();
+    for (int rr = nforced; rr < top_k; ++rr) {
+      const uint32_t vmax = __reduce_max_sync(0xffffffffu, bk);
+      if (vmax == 0u) break;
+      // the lowest block index among the lanes holding the maximum
+      const uint32_t jmin = __reduce_min_sync(0xffffffffu, bk == vmax ? (uint32_t)(lane + 32 * bm) : 0xffffffffu);
+      if (lane == (int)(jmin & 31u)) {
+        const int mw = (int)(jmin >> 5);
+        taken[K] |= 1u << mw;
+#pragma unroll
+        for (int mm = 0; mm < 32; ++mm)
+          if (mm == mw) key[K][mm] = 0u;
+        local_best();
+      }
+    }
+    const int mmax = (nb + 31) >> 5;
+    int pos = 0;
+    for (int mm = 0; mm < mmax; ++mm) {
+      const bool sel = (taken[K] >> mm) & 1u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+      if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
+      pos += __popc(bal);
+    }
+    for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
   }
-  for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
-}
+};
 
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -344,23 +356,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp >= kTopkWarp0) {
     // ------------------------------------------------------------ top-k
-    // warp kTopkWarp0 + i takes tokens 4i .. 4i+3 of each item
+    // warp kTopkWarp0 + i takes tokens 4i .. 4i+3 of each item: it copies their scores out
+    // (zeroing them), releases the buffer, then selects from registers
     const int w = warp - kTopkWarp0;
     bool ok = true;
     int k = 0;
+    TopkWarp<4> tk;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
       const Item x = item_of(it);
       ok = tc::mbar_wait(sc_full, k & 1, err, kErrScFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      for (int kk = 4 * w; kk < 4 * w + 4; ++kk) {
-        const int t = x.t0 + kk;
-        if (t < T)
-          topk_token(sScore + kk * kMaxSel, t, top_k, force_first, force_local,
-                     idx_out + (((size_t)x.b * Hkv + x.g) * T + t) * top_k, lane);
+      int nb[4], own[4];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int t = x.t0 + 4 * w + kk;
+        nb[kk] = t < T ? t / kSel + 1 : 0;
+        own[kk] = t / kSel;
       }
+      tk.load(sScore + 4 * w * kMaxSel, kMaxSel, nb, own, force_first, force_local, lane);
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(sc_empty);
+      int32_t* dst = idx_out + (((size_t)x.b * Hkv + x.g) * T + x.t0 + 4 * w) * top_k;
+      tk.template select<0>(nb[0], own[0], top_k, force_first, force_local, dst, lane);
+      tk.template select<1>(nb[1], own[1], top_k, force_first, force_local, dst + top_k, lane);
+      tk.template select<2>(nb[2], own[2], top_k, force_first, force_local, dst + 2 * top_k, lane);
+      tk.template select<3>(nb[3], own[3], top_k, force_first, force_local, dst + 3 * top_k, lane);
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue

@@ -160,9 +160,10 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           qf[ks][3] = rv1 ? ld_u32(q1 + ks * 16 + 8 + 2 * cq) : 0u;
         }
       }
-      // warm L2 for what comes from DRAM later: the next item's queries (this pipeline's
-      // next token; its index row is read early by the producer) and the accumulator
-      // rows of this item
+      // warm L2 for what comes from DRAM later: the next item's queries and block list
+      // (this pipeline's next token; the producer reads the list about two blocks ahead
+      // of the consumers, too late to hide a DRAM access), and this item's accumulator
+      // rows and gates
       {
         const long itn = it + stride;
         if (itn < total) {
@@ -172,9 +173,17 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           constexpr int kLines = 16 * DK * 2 / 128;               // 16 heads of queries
           for (int ln = cw * 32 + lane; ln < kLines; ln += kConsumers * 32)
             if (ln < G * DK * 2 / 128) prefetch_l2(qn + ln * 128);
+          if (cw == 0 && lane == 0) {
+            const int bn = btn / T, tn = btn % T;
+            prefetch_l2(idx + (((size_t)bn * Hkv + gn) * T + tn) * top_k);
+          }
         }
         if (lane < G)
           prefetch_l2(acc + (((size_t)b * T + t) * Hq + g * G + lane) * DV + cw * (DV / kConsumers));
+        if (cw == 1 && lane < 2) {   // the G x 3 gates of this item's rows (at most two lines)
+          const char* gp = reinterpret_cast<const char*>(gates + ((size_t)b * T + t) * Hq * 3 + g * G * 3);
+          prefetch_l2(lane == 0 ? gp : gp + G * 3 * 2 - 1);
+        }
       }
       // per row (gl, gl + 8): the softmax reference, shared by the four warps, and this
       // warp's part of the row sums; it moves only when a score exceeds it by kSlack

@@ -117,28 +117,46 @@ struct TopkWarp {
     }
     int nforced = force_first ? 1 : 0;
     if (force_local && !(force_first && own == 0)) ++nforced;
+    const int mmax = (nb + 31) >> 5;   // candidate slots in use per lane
+    if (mmax <= 4) rounds<K, 4>(nforced, top_k, lane);
+    else if (mmax <= 8) rounds<K, 8>(nforced, top_k, lane);
+    else if (mmax <= 16) rounds<K, 16>(nforced, top_k, lane);
+    else rounds<K, 32>(nforced, top_k, lane);
+    int pos = 0;
+    for (int mm = 0; mm < mmax; ++mm) {
+      const bool sel = (taken[K] >> mm) & 1u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+      if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
+      pos += __popc(bal);
+    }
+    for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
+  }
+
+  // The selection rounds over the first M slots of each lane (slots >= M hold no candidate).
+  template <int K, int M>
+  __device__ __forceinline__ void rounds(int nforced, int top_k, int lane) {
     // this lane's best key and its mm (the lowest mm among equal keys), by a pairwise tree
     uint32_t bk = 0;
     int bm = 0;
     auto local_best = [&]() {
-      uint32_t k16[16];
-      int m16[16];
+      uint32_t kt[M / 2];
+      int mt[M / 2];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < M / 2; ++i) {
         const bool c = key[K][2 * i + 1] > key[K][2 * i];
-        k16[i] = c ? key[K][2 * i + 1] : key[K][2 * i];
-        m16[i] = c ? 2 * i + 1 : 2 * i;
+        kt[i] = c ? key[K][2 * i + 1] : key[K][2 * i];
+        mt[i] = c ? 2 * i + 1 : 2 * i;
       }
 #pragma unroll
-      for (int w = 8; w >= 1; w >>= 1)
+      for (int w = M / 4; w >= 1; w >>= 1)
 #pragma unroll
         for (int i = 0; i < w; ++i) {
-          const bool c = k16[2 * i + 1] > k16[2 * i];
-          k16[i] = c ? k16[2 * i + 1] : k16[2 * i];
-          m16[i] = c ? m16[2 * i + 1] : m16[2 * i];
+          const bool c = kt[2 * i + 1] > kt[2 * i];
+          kt[i] = c ? kt[2 * i + 1] : kt[2 * i];
+          mt[i] = c ? mt[2 * i + 1] : mt[2 * i];
         }
-      bk = k16[0];
-      bm = m16[0];
+      bk = kt[0];
+      bm = mt[0];
     };
     local_best();
     for (int rr = nforced; rr < top_k; ++rr) {
@@ -150,20 +168,11 @@ struct TopkWarp {
         const int mw = (int)(jmin >> 5);
         taken[K] |= 1u << mw;
 #pragma unroll
-        for (int mm = 0; mm < 32; ++mm)
+        for (int mm = 0; mm < M; ++mm)
           if (mm == mw) key[K][mm] = 0u;
         local_best();
       }
     }
-    const int mmax = (nb + 31) >> 5;
-    int pos = 0;
-    for (int mm = 0; mm < mmax; ++mm) {
-      const bool sel = (taken[K] >> mm) & 1u;
-      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
-      if (sel) dst[pos + __popc(bal & ((1u << lane) - 1u))] = lane + 32 * mm;
-      pos += __popc(bal);
-    }
-    for (int j = pos + lane; j < top_k; j += 32) dst[j] = -1;
   }
 };
 

@@ -17,9 +17,9 @@
 //            (rows = value dims), already normalised, so no rescaling is ever needed.
 //   top-k    per token over the selection-block scores in shared memory.
 //   epilogue acc[t, h, :] = g_cmp * o_cmp, read from O^T (each thread one value dim).
-// Warp roles: 8 TMA producer, 9 MMA issuer (and TMEM owner), 10-11 top-k, 0-7 softmax /
-// epilogue in two groups of four (warp w owns TMEM lanes 32*(w%4)..+31; group w/4 takes one
-// half of every tile's 128 columns: in the second pass that half is exactly four tokens).
+// Warp roles: 16 TMA producer, 17 MMA issuer (and TMEM owner), 18-19 top-k, 0-15 softmax /
+// epilogue in four groups of four (warp w owns TMEM lanes 32*(w%4)..+31; group w/4 takes 32
+// of every tile's 128 columns: in the second pass that is exactly two tokens).
 // Items overlap: while the softmax warps finish an item (last tiles, epilogue), the TMA and
 // MMA warps already load and multiply the next item's first tiles, and the top-k warps
 // select the finished item's blocks while the softmax warps run the next item's pass A.
@@ -35,9 +35,12 @@
 namespace nsa {
 
 namespace {
-constexpr int kSoftWarps = 8;                 // two groups of four softmax warps
-constexpr int kTmaWarp = 8, kMmaWarp = 9, kTopkWarp0 = 10, kTopkWarps = 2;
-constexpr int kThreads = 384;
+constexpr int kSoftGroups = 4;                  // softmax warp groups, 32 tile columns each
+constexpr int kSoftWarps = 4 * kSoftGroups;     // four warps per group (one per TMEM lane quarter)
+constexpr int kCols = 128 / kSoftGroups;        // tile columns per softmax thread
+constexpr int kTokG = kCols / 16;               // tokens per group in the second pass
+constexpr int kTmaWarp = kSoftWarps, kMmaWarp = kSoftWarps + 1, kTopkWarp0 = kSoftWarps + 2, kTopkWarps = 2;
+constexpr int kThreads = 32 * (kSoftWarps + 4);
 constexpr int kTok = 8;            // tokens per CTA
 constexpr int kRowsM = 128;        // query rows per CTA (8 tokens x 16 heads)
 constexpr int kBlk = 128;          // compressed blocks per tile
@@ -61,7 +64,7 @@ struct Smem {
   static constexpr uint32_t kScore = kP + 2 * kSlice;                       // [8][1024] fp32
   static constexpr uint32_t kLse = kScore + kTok * kMaxSel * 4;             // [128] fp32
   static constexpr uint32_t kGate = kLse + kRowsM * 4;                      // [2][128] fp32, by item parity
-  static constexpr uint32_t kML = kP;                                       // [2][128][2] fp32, while P^T is unused
+  static constexpr uint32_t kML = kP;                                       // [groups][128][2] fp32, while P^T is unused
   static constexpr uint32_t kBar = kGate + 2 * kRowsM * 4;                  // mbarriers
   static constexpr int kNumBars = 1 + 2 * kKcSlots + 2 * 2 + 2 * 2 + 2 + 1 + 4;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
@@ -365,56 +368,62 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp >= kTopkWarp0) {
     // ------------------------------------------------------------ top-k
-    // warp kTopkWarp0 + i takes tokens 4i .. 4i+3 of each item: it copies their scores out
-    // (zeroing them), releases the buffer, then selects from registers
+    // warp kTopkWarp0 + i takes tokens 4i .. 4i+3 of each item, two at a time: it copies
+    // their scores out (zeroing them), selects from registers, and releases the score
+    // buffer after the last pair has been copied
     const int w = warp - kTopkWarp0;
     bool ok = true;
     int k = 0;
-    TopkWarp<4> tk;
+    TopkWarp<2> tk;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
       const Item x = item_of(it);
       ok = tc::mbar_wait(sc_full, k & 1, err, kErrScFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
-      int nb[4], own[4];
+#pragma unroll 1
+      for (int pr = 0; pr < 2; ++pr) {
+        const int t0p = x.t0 + 4 * w + 2 * pr;
+        int nb[2], own[2];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int t = x.t0 + 4 * w + kk;
-        nb[kk] = t < T ? t / kSel + 1 : 0;
-        own[kk] = t / kSel;
+        for (int kk = 0; kk < 2; ++kk) {
+          const int t = t0p + kk;
+          nb[kk] = t < T ? t / kSel + 1 : 0;
+          own[kk] = t / kSel;
+        }
+        tk.load(sScore + (4 * w + 2 * pr) * kMaxSel, kMaxSel, nb, own, force_first, force_local, lane);
+        if (pr == 1) {
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(sc_empty);
+        }
+        int32_t* dst = idx_out + (((size_t)x.b * Hkv + x.g) * T + t0p) * top_k;
+        tk.template select<0>(nb[0], own[0], top_k, force_first, force_local, dst, lane);
+        tk.template select<1>(nb[1], own[1], top_k, force_first, force_local, dst + top_k, lane);
       }
-      tk.load(sScore + 4 * w * kMaxSel, kMaxSel, nb, own, force_first, force_local, lane);
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(sc_empty);
-      int32_t* dst = idx_out + (((size_t)x.b * Hkv + x.g) * T + x.t0 + 4 * w) * top_k;
-      tk.template select<0>(nb[0], own[0], top_k, force_first, force_local, dst, lane);
-      tk.template select<1>(nb[1], own[1], top_k, force_first, force_local, dst + top_k, lane);
-      tk.template select<2>(nb[2], own[2], top_k, force_first, force_local, dst + 2 * top_k, lane);
-      tk.template select<3>(nb[3], own[3], top_k, force_first, force_local, dst + 3 * top_k, lane);
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    // Two groups of four warps; group gr takes columns [64*gr, 64*gr+64) of every tile.
+    // Four groups of four warps; group gr takes columns [32*gr, 32*gr+32) of every tile.
     // Warp quarter q = warp % 4 owns TMEM lanes 32q..32q+31; r is this thread's lane.
     const int gr = warp >> 2, q4 = warp & 3;
     const int r = 32 * q4 + lane;
-    const int col0 = 64 * gr;
+    const int col0 = kCols * gr;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
+    constexpr int kNT = kSoftWarps * 32;   // softmax threads
     bool ok = true;
     int use = 0;   // S buffer uses
     int pc = 0;    // pass-B tiles
-    for (int i = gr * 128 + r; i < kTok * kMaxSel; i += 256) sScore[i] = 0.f;
+    for (int i = tid; i < kTok * kMaxSel; i += kNT) sScore[i] = 0.f;
     int k = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
       const Item x = item_of(it);
       const int t0 = x.t0, g = x.g, b = x.b, ntiles = x.ntiles;
       float* gate = sGate + (k & 1) * kRowsM;
-      if (gr == 0) {   // gates of the 128 rows (double-buffered: group 1 may still be in the previous epilogue)
+      if (gr == 0) {   // gates of the 128 rows (double-buffered: other groups may still be in the previous epilogue)
         const int t = t0 + r / 16, h = g * 16 + (r % 16);
         gate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3]) : 0.f;
       }
 
-      // pass A: this thread's row r = (token r/16, head r%16), its half of every tile's columns
+      // pass A: this thread's row r = (token r/16, head r%16), its 32 columns of every tile
       {
         const int my_t = t0 + r / 16;
         const int my_hi = my_t < T ? n_visible(my_t, nc) : 0;
@@ -426,9 +435,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (!ok) break;
           tc::tc_fence_after();
           const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
-          float v[64];
+          float v[kCols];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+          for (int c = 0; c < kCols / 16; ++c)
+            tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
           tc::tmem_wait_ld();
           tc::tc_fence_before();
           __syncwarp();
@@ -436,18 +446,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // masked, scaled scores; only a tile that straddles this row's range needs the
           // per-element test.  Max and sum use eight independent chains each.
           const int i0 = n * kBlk + col0;
-          if (i0 + 63 < my_hi) {
+          if (i0 + kCols - 1 < my_hi) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] *= scale_log2;
+            for (int j = 0; j < kCols; ++j) v[j] *= scale_log2;
           } else {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = i0 + j < my_hi ? v[j] * scale_log2 : -INFINITY;
+            for (int j = 0; j < kCols; ++j) v[j] = i0 + j < my_hi ? v[j] * scale_log2 : -INFINITY;
           }
           float cmx[8];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(fmaxf(v[c], v[c + 8]), fmaxf(v[c + 16], v[c + 24]));
+          for (int c = 0; c < 8; ++c) cmx[c] = v[c];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
+          for (int j = 8; j < kCols; ++j) cmx[j & 7] = fmaxf(cmx[j & 7], v[j]);
           const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
                                  fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
           const float mn = fmaxf(m, cm);
@@ -456,7 +466,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < 8; ++c) ps[c] = ex2(v[c] - mn);
 #pragma unroll
-            for (int j = 8; j < 64; ++j) ps[j & 7] += ex2(v[j] - mn);
+            for (int j = 8; j < kCols; ++j) ps[j & 7] += ex2(v[j] - mn);
             const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             l = l * ex2(m - mn) + sum;
             m = mn;
@@ -465,42 +475,51 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         sML[(gr * 128 + r) * 2] = m;
         sML[(gr * 128 + r) * 2 + 1] = l;
       }
-      ok = vote_all(3, kSoftWarps * 32, ok);
+      ok = vote_all(3, kNT, ok);
       if (!ok) break;
       if (gr == 0) {
-        const float m0 = sML[r * 2], l0 = sML[r * 2 + 1], m1 = sML[(128 + r) * 2], l1 = sML[(128 + r) * 2 + 1];
-        const float M = fmaxf(m0, m1);
-        const float L = M == -INFINITY ? 0.f : l0 * ex2(m0 - M) + l1 * ex2(m1 - M);
+        float M = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kSoftGroups; ++q) M = fmaxf(M, sML[(q * 128 + r) * 2]);
+        float L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int q = 0; q < kSoftGroups; ++q) L += sML[(q * 128 + r) * 2 + 1] * ex2(sML[(q * 128 + r) * 2] - M);
+        }
         sLse[r] = (t0 + r / 16 < T && L > 0.f) ? M + __log2f(L) : INFINITY;
       }
       // the previous item's scores must have been taken (and zeroed) by the top-k warps
       if (k > 0) ok = tc::mbar_wait(sc_empty, (k - 1) & 1, err, kErrScEmpty);
-      ok = vote_all(3, kSoftWarps * 32, ok);
+      ok = vote_all(3, kNT, ok);
       if (!ok) break;
 
-      // pass B: this thread's key r of every tile; columns = tokens 4*gr .. 4*gr+3, 16 heads each
-      int hi_tok[4], nb_tok[4];
+      // pass B: this thread's key r of every tile; columns = tokens kTokG*gr .., 16 heads each
+      int hi_tok[kTokG], nb_tok[kTokG];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int t = t0 + 4 * gr + kk;
+      for (int kk = 0; kk < kTokG; ++kk) {
+        const int t = t0 + kTokG * gr + kk;
         const bool in = t < T;
         hi_tok[kk] = in ? n_visible(t, nc) : 0;
         nb_tok[kk] = in ? t / kSel + 1 : 0;
       }
-      uint8_t* prow = sP + gr * kSlice + r * 128;   // row r of N-block gr of P^T
+      // row r of P^T; this group's columns are 16-byte chunks (col0 % 64)/8 .. of N-block col0/64
+      uint8_t* prow = sP + (col0 / 64) * kSlice + r * 128;
+      const int ch0 = (col0 % 64) / 8;
       // Selection-block scores: block j = i/4 collects i = 4j-1 .. 4j+3.  Each group of four
       // lanes adds its own four blocks plus the lane just below it into the block's entry.
       // Lane 31's block (i % 4 == 3) also belongs to the first selection block of the next
       // warp (or of the next tile); that carry is added two tiles later, after waiting for
       // the P^T phase that every softmax warp releases only after its own score writes, so
       // no barrier is needed inside the loop.  Each entry receives at most two additions.
-      float carry_a[4] = {0.f, 0.f, 0.f, 0.f}, carry_b[4] = {0.f, 0.f, 0.f, 0.f};   // tiles n-1, n-2
-      auto add_carry = [&](const float (&c)[4], int tile) {
+      float carry_a[kTokG], carry_b[kTokG];   // tiles n-1, n-2
+#pragma unroll
+      for (int kk = 0; kk < kTokG; ++kk) carry_a[kk] = carry_b[kk] = 0.f;
+      auto add_carry = [&](const float (&c)[kTokG], int tile) {
         const int jt = tile * (kBlk / 4) + q4 * 8 + 8;
         if (lane == 31) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            if (jt < nb_tok[kk]) sScore[(4 * gr + kk) * kMaxSel + jt] += c[kk];
+          for (int kk = 0; kk < kTokG; ++kk)
+            if (jt < nb_tok[kk]) sScore[(kTokG * gr + kk) * kMaxSel + jt] += c[kk];
         }
       };
       for (int n = 0; n < ntiles; ++n, ++use, ++pc) {
@@ -512,37 +531,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         if (!ok) break;
         tc::tc_fence_after();
         const uint32_t base = lane_addr + (sb ? kColS1 : kColS0) + col0;
-        float v[64];
+        float v[kCols];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+        for (int c = 0; c < kCols / 16; ++c)
+          tc::tmem_ld16(base + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
         tc::tmem_wait_ld();
         const int i = n * kBlk + r;        // this thread's compressed block
-        float tok_sum[4];
-        uint32_t pk[32];
+        float tok_sum[kTokG];
+        uint32_t pk[kCols / 2];
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < kTokG; ++kk) {
           const bool vis = i < hi_tok[kk];
-          float s = 0.f;
+          float sacc = 0.f;
 #pragma unroll
           for (int j = 0; j < 16; j += 2) {
             const float p0 = vis ? ex2(v[16 * kk + j] * scale_log2 - sLse[col0 + 16 * kk + j]) : 0.f;
             const float p1 = vis ? ex2(v[16 * kk + j + 1] * scale_log2 - sLse[col0 + 16 * kk + j + 1]) : 0.f;
-            s += p0 + p1;
+            sacc += p0 + p1;
             __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             pk[8 * kk + j / 2] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          tok_sum[kk] = s;
+          tok_sum[kk] = sacc;
         }
         {
           const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < kTokG; ++kk) {
             const float vv = tok_sum[kk];
             float g4 = vv + __shfl_xor_sync(0xffffffffu, vv, 1);
             g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
             const float prev = __shfl_up_sync(0xffffffffu, vv, 1);
             const int j = j0 + (lane >> 2);
-            if ((lane & 3) == 0 && j < nb_tok[kk]) sScore[(4 * gr + kk) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
+            if ((lane & 3) == 0 && j < nb_tok[kk]) sScore[(kTokG * gr + kk) * kMaxSel + j] += g4 + (lane > 0 ? prev : 0.f);
           }
         }
         // P^T(pc) may overwrite the buffer once PV(pc-1) has read it
@@ -556,13 +576,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        for (int kk = 0; kk < kTokG; ++kk) {
           carry_b[kk] = carry_a[kk];
           carry_a[kk] = tok_sum[kk];
         }
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) =
+        for (int c = 0; c < kCols / 8; ++c)
+          *reinterpret_cast<uint4*>(prow + (((ch0 + c) ^ (r & 7)) << 4)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         tc::tc_fence_before();
         tc::fence_async_smem();
@@ -572,36 +592,36 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc::mbar_arrive(p_full);
         }
       }
-      ok = vote_all(3, kSoftWarps * 32, ok);
+      ok = vote_all(3, kNT, ok);
       if (!ok) break;
       // the carries of the last two tiles, then hand the scores to the top-k warps
       if (ntiles > 1) add_carry(carry_b, ntiles - 2);
       if (ntiles > 0) add_carry(carry_a, ntiles - 1);
-      named_sync(3, kSoftWarps * 32);
+      named_sync(3, kNT);
       if (tid == 0) tc::mbar_arrive(sc_full);
 
-      // epilogue: lane r = value dim r of O^T; this group's 64 columns = tokens 4*gr .. 4*gr+3.
+      // epilogue: lane r = value dim r of O^T; this group's 32 columns = tokens kTokG*gr ..
       // A failed wait here only skips the stores: the next item's vote ends the loop for all.
       ok = tc::mbar_wait(o_full, k & 1, err, kErrOFull);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc::tc_fence_after();
-        float v[64];
+        float v[kCols];
         if (ntiles > 0) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < kCols / 16; ++c)
             tc::tmem_ld16(lane_addr + kColO + col0 + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
           tc::tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) v[c] = 0.f;
+          for (int c = 0; c < kCols; ++c) v[c] = 0.f;
         }
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(o_empty);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int t = t0 + 4 * gr + c / 16;
+        for (int c = 0; c < kCols; ++c) {
+          const int t = t0 + kTokG * gr + c / 16;
           if (t < T && r < DV) {
             const size_t row = ((size_t)b * T + t) * Hq + g * 16 + (c % 16);
             acc[row * DV + r] = gate[col0 + c] * v[c];

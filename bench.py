@@ -211,9 +211,9 @@ def workload_config(c, name):
 # compressed cache stay mostly in L2.  An entry goes back to None whenever its kernel
 # changes, until it is captured again.
 NCU_DRAM_BYTES_PER_ITEM = {
-    "cmp_select": (209.339136e6 + 221.811200e6) / 32768,
-    "slc_attn": (501.146112e6 + 229.680896e6) / 32768,
-    "swa_combine": (499.481088e6 + 117.558272e6) / 32768,
+    "cmp_select": (205.900800e6 + 217.100032e6) / 32768,
+    "slc_attn": (501.110528e6 + 232.153088e6) / 32768,
+    "swa_combine": (499.490048e6 + 117.897984e6) / 32768,
 }
 
 

@@ -18,7 +18,7 @@ NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUD
 NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
 
 EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_forward", "nsa_decode", "nsa_forward_noalloc",
-            "nsa_status_string")
+            "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
 
 
 class NsaConfig(ctypes.Structure):
@@ -68,6 +68,10 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_decode.restype = ctypes.c_int
     lib.nsa_forward_noalloc.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
     lib.nsa_forward_noalloc.restype = ctypes.c_int
+    lib.nsa_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
+    lib.nsa_device_status.restype = ctypes.c_int
+    lib.nsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
+    lib.nsa_selftest_wait_timeout.restype = ctypes.c_int
     lib.nsa_status_string.argtypes = [ctypes.c_int]
     lib.nsa_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -141,6 +145,21 @@ def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, max_seqlen: int
                                    _ptr(seqlens), int(max_seqlen), _ptr(gates), ctypes.byref(cfg), _ptr(out),
                                    _stream(stream, q))
     return _check(st, "nsa_decode") if check else st
+
+
+def nsa_device_status(workspace, stream=None) -> tuple[int, int]:
+    """(status, word) of the workspace's status word after synchronising the stream:
+    NSA_OK with word 0, or NSA_ERR_TIMEOUT with the code of the wait that gave up."""
+    word = ctypes.c_int32(0)
+    st = load_library().nsa_device_status(_ptr(workspace), ctypes.byref(word), _stream(stream, workspace))
+    return st, int(word.value)
+
+
+def nsa_selftest_wait_timeout(workspace, limit_us: int, stream=None, check: bool = True) -> int:
+    """Launch the timeout self-test: one bounded wait that nothing releases (see include/nsa.h)."""
+    st = load_library().nsa_selftest_wait_timeout(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                  int(limit_us), _stream(stream, workspace))
+    return _check(st, "nsa_selftest_wait_timeout") if check else st
 
 
 def nsa_forward_noalloc(q, k, v, gates, cfg: NsaConfig, out, stream=None, check: bool = True) -> int:

@@ -62,6 +62,10 @@ struct DecodeArgs {
 // K6: one decode step per sequence, all branches in one launch.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
+// Self-test of the bounded-wait path: one wait on an mbarrier that nothing arrives at,
+// which gives up after limit_ns and records `code` in *err.
+cudaError_t launch_wait_timeout(int* err, uint64_t limit_ns, int code, cudaStream_t st);
+
 
 struct MobaLayout {
   size_t kbar, idx, counts, offsets, chunks, fill, list, part_lse, part_o, total;

@@ -125,6 +125,26 @@ const char* nsa_status_string(nsa_status s) {
   return "NSA_ERR_UNKNOWN";
 }
 
+nsa_status nsa_device_status(const void* workspace, int32_t* code_out, void* stream) {
+  if (!workspace) return NSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return NSA_ERR_CUDA;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return NSA_ERR_CUDA;
+  if (code_out) *code_out = word;
+  return word == 0 ? NSA_OK : NSA_ERR_TIMEOUT;
+}
+
+nsa_status nsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us, void* stream) {
+  if (!workspace || workspace_bytes < sizeof(int32_t) || (reinterpret_cast<uintptr_t>(workspace) % 4) ||
+      limit_us < 1 || limit_us > 1000000)
+    return NSA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* err = static_cast<int*>(workspace);
+  if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
+  return nsa::launch_wait_timeout(err, (uint64_t)limit_us * 1000ull, 99, s) == cudaSuccess ? NSA_OK : NSA_ERR_CUDA;
+}
+
 size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch) {
   if (check_cfg(cfg) != NSA_OK || decode_batch < 0) return 0;
   if (decode_batch == 0) return workspace_bytes(cfg);

@@ -92,18 +92,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Waits for the phase with the given parity to complete.  Gives up after one second,
-// or as soon as another thread has given up, records `code` in *err and returns
-// false: callers then stop issuing work and leave.
+// Waits for the phase with the given parity to complete.  Gives up after `limit_ns`
+// nanoseconds (one second by default), or as soon as another thread has given up, records
+// `code` in *err and returns false: callers then stop issuing work and leave.
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int code,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63) == 0) {
       if (*(volatile int*)err) return false;   // another role already gave up
-      if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      if (globaltimer_ns() - t0 > limit_ns) break;
     }
   }
   atomicCAS(err, 0, code);

@@ -45,7 +45,7 @@ typedef enum {
   NSA_ERR_UNSUPPORTED = 2,  /* a legal config these kernels do not implement */
   NSA_ERR_WORKSPACE = 3,    /* workspace missing, misaligned or smaller than nsa_workspace_size() */
   NSA_ERR_CUDA = 4,         /* a kernel launch failed (cudaGetLastError) */
-  NSA_ERR_TIMEOUT = 5       /* reserved for bounded device-side waits (none in this version) */
+  NSA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see nsa_device_status) */
 } nsa_status;
 
 typedef enum {
@@ -206,6 +206,31 @@ NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_
  */
 NSA_API nsa_status nsa_forward_noalloc(const void* q, const void* k, const void* v, const void* gates,
                                        const nsa_config* cfg, void* out, void* stream);
+
+/*
+ * nsa_device_status -- the outcome of the device-side work of earlier calls that used
+ * `workspace` (the pointer passed as cfg->workspace; nsa_decode and nsa_forward zero its
+ * first 4 bytes, the status word, when they start).  The tensor-core kernels bound every
+ * wait on an mbarrier (one second); a wait that gives up writes a nonzero code to the word,
+ * and the kernel stops issuing work and returns instead of hanging.
+ * Synchronises `stream` (a cudaStream_t, NULL = the default stream), reads the word and
+ * returns NSA_OK if it is 0, NSA_ERR_TIMEOUT otherwise (code_out, if not NULL, receives the
+ * word: which wait gave up).  NSA_ERR_INVALID_ARG for a null workspace, NSA_ERR_CUDA if the
+ * synchronisation or the copy fails.
+ */
+NSA_API nsa_status nsa_device_status(const void* workspace, int32_t* code_out, void* stream);
+
+/*
+ * nsa_selftest_wait_timeout -- test hook for the timeout path above; no part of the method.
+ * Zeroes the status word of `workspace` (device memory, at least 4 bytes, 4-byte aligned),
+ * then launches one thread that waits, with a limit of limit_us microseconds (1 .. 1000000),
+ * on an mbarrier that nothing arrives at.  The wait gives up, writes code 99 to the status
+ * word and the kernel returns; nsa_device_status then reports NSA_ERR_TIMEOUT.  Nothing else
+ * is touched and the context stays usable.  NSA_ERR_INVALID_ARG for a null, misaligned or
+ * too small workspace or a limit out of range; NSA_ERR_CUDA if the launch fails.
+ */
+NSA_API nsa_status nsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us,
+                                             void* stream);
 
 /* Human-readable name of a status code (static storage). */
 NSA_API const char* nsa_status_string(nsa_status s);

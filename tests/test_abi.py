@@ -137,3 +137,15 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(nsa, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         nsa.load_library()
+
+
+def test_status_and_selftest_reject_bad_arguments(lib):
+    """Argument checks that return before any CUDA call (safe without a GPU)."""
+    word = ctypes.c_int32(7)
+    assert lib.nsa_device_status(None, ctypes.byref(word), None) == nsa.NSA_ERR_INVALID_ARG
+    assert lib.nsa_selftest_wait_timeout(None, 256, 1000, None) == nsa.NSA_ERR_INVALID_ARG
+    fake = 0x10000   # never dereferenced: every call below fails its checks first
+    assert lib.nsa_selftest_wait_timeout(fake, 2, 1000, None) == nsa.NSA_ERR_INVALID_ARG          # too small
+    assert lib.nsa_selftest_wait_timeout(fake + 2, 256, 1000, None) == nsa.NSA_ERR_INVALID_ARG    # misaligned
+    assert lib.nsa_selftest_wait_timeout(fake, 256, 0, None) == nsa.NSA_ERR_INVALID_ARG           # no limit
+    assert lib.nsa_selftest_wait_timeout(fake, 256, 1000001, None) == nsa.NSA_ERR_INVALID_ARG     # above 1 s

@@ -4,6 +4,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace nsa {
@@ -68,7 +69,7 @@ cudaError_t launch_wait_timeout(int* err, uint64_t limit_ns, int code, cudaStrea
 
 
 struct MobaLayout {
-  size_t kbar, idx, counts, offsets, chunks, fill, list, part_lse, part_o, total;
+  size_t err, kbar, idx, counts, offsets, chunks, fill, list, part_lse, part_o, total;
 };
 // Workspace carve-up of MoBA mode (each region 256-byte aligned).
 MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k);
@@ -84,10 +85,18 @@ struct MobaArgs {
   float scale_log2;
   cudaError_t (*mark)(void*, cudaStream_t);   // optional stage marker (measurement events)
   void* mark_ctx;
+  int* err;             // status word (the workspace's first 4 bytes), zeroed by launch_moba
 };
 
 // MoBA mode: block means, selection, per-block query lists, past-block attention,
 // own-block attention + merge.
 cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st);
+// Past-block attention on tcgen05 (chunks of moba_past_tc_chunk() queries; block size a
+// multiple of 128).  max_chunks bounds the chunk count written to chunks[E] on the device.
+bool moba_past_tc_supported(const MobaArgs& a);
+int moba_past_tc_chunk();
+cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const int32_t* offsets,
+                                const int32_t* chunks, const int32_t* list, __nv_bfloat16* part_o, float* part_lse,
+                                int nblk, int E, size_t max_chunks, cudaStream_t st);
 
 }  // namespace nsa

@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
 // Exclusive scans over all (b, h, j): list offsets and 64-query chunk starts (one CTA).
 __global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets, int32_t* __restrict__ chunks,
-                                                         int32_t* __restrict__ fill, int E) {
+                                                         int32_t* __restrict__ fill, int E, int cq) {
   __shared__ int32_t s0[1024], s1[1024];
   __shared__ int32_t carry0, carry1;
   if (threadIdx.x == 0) { carry0 = 0; carry1 = 0; }
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restri
     const int e = base + threadIdx.x;
     const int c = e < E ? counts[e] : 0;
     s0[threadIdx.x] = c;
-    s1[threadIdx.x] = (c + kQ - 1) / kQ;
+    s1[threadIdx.x] = (c + cq - 1) / cq;
     __syncthreads();
     for (int off = 1; off < 1024; off <<= 1) {   // Hillis-Steele inclusive scan
       const int a0 = threadIdx.x >= off ? s0[threadIdx.x - off] : 0;
@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restri
     }
     if (e < E) {
       offsets[e] = carry0 + s0[threadIdx.x] - c;
-      chunks[e] = carry1 + s1[threadIdx.x] - (c + kQ - 1) / kQ;
+      chunks[e] = carry1 + s1[threadIdx.x] - (c + cq - 1) / cq;
       fill[e] = 0;
     }
     __syncthreads();
@@ -489,6 +489,7 @@ MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k) {
   const size_t nblk = (T + bsz - 1) / bsz;
   const size_t E = (size_t)B * H * nblk;
   size_t off = 0;
+  L.err = off; off = up(off + 4);   // status word of the bounded device waits
   L.kbar = off; off = up(off + (size_t)B * nblk * H * D * 4);
   L.idx = off; off = up(off + (size_t)B * H * T * (top_k + 1) * 4);
   L.counts = off; off = up(off + E * 4);
@@ -527,6 +528,7 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q);
   const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(a.k);
   const __nv_bfloat16* v = static_cast<const __nv_bfloat16*>(a.v);
+  const bool tc = moba_past_tc_supported(a);
   cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)E * 4, st);
   if (e != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
@@ -537,7 +539,8 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
                                                                               nblk, a.top_k);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, E);
+  const int cq = tc ? moba_past_tc_chunk() : kQ;   // queries per past-attention chunk
+  moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, E, cq);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   moba_scatter_kernel<<<dim3((a.T + 255) / 256, a.B * a.H), 256, 0, st>>>(idx, offsets, fill, list, a.T, a.H, nblk,
                                                                          a.top_k, a.bsz);
@@ -546,7 +549,13 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (a.top_k > 0) {
+  if (a.top_k > 0 && tc) {
+    // every list holds at most B*H*T*top_k entries in all: the chunk count is bounded by
+    // that over the chunk size plus one partial chunk per list
+    const size_t max_chunks = ((size_t)a.B * a.H * a.T * a.top_k + cq - 1) / cq + (size_t)E;
+    e = launch_moba_past_tc(a, counts, offsets, chunks, list, part_o, part_lse, nblk, E, max_chunks, st);
+    if (e != cudaSuccess) return e;
+  } else if (a.top_k > 0) {
     moba_past_kernel<<<sms * 3, kThreads, kAttnSmem, st>>>(q, k, v, counts, offsets, chunks, list, part_o, part_lse,
                                                            a.T, a.H, nblk, a.bsz, a.top_k, E, a.scale_log2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -106,6 +106,8 @@ nsa_status moba_forward(const void* q, const void* k, const void* v, const nsa_c
   a.scale_log2 = scale * 1.4426950408889634f;
   a.mark = mark_trampoline;
   a.mark_ctx = &marks;
+  a.err = static_cast<int*>(cfg->workspace);   // the status word leads the workspace
+  if (cudaMemsetAsync(a.err, 0, sizeof(int), s) != cudaSuccess) return NSA_ERR_CUDA;
   return from_cuda(nsa::launch_moba(a, s));
 }
 

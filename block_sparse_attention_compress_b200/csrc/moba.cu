@@ -5,10 +5,12 @@
 // top 3; the queries that chose one KV block are gathered so the block is read once).
 //
 // Five launches on the caller's stream:
-//   M1 block means      kbar[b, j, h, :] = mean of the keys of block j (fp32);
-//   M2 select           per 64-token tile and head: score_j = q . kbar_j for the past blocks
-//                       (kbar split into two bf16 halves so the tensor-core dot product keeps
-//                       fp32 accuracy), running top-k per row, idx = [past ascending.., own];
+//   M1 block means      kbar[b, j, h, :] = mean of the keys of block j, accumulated in fp32 and
+//                       stored as two bf16 halves (hi = bf16(mean), lo = bf16(mean - hi)) so
+//                       that the tensor-core dot product keeps about 16 mantissa bits;
+//   M2 select           per 64-token tile and head: score_j = q . hi_j + q . lo_j for the past
+//                       blocks (tiles of 64 blocks double buffered by cp.async), running top-k
+//                       per row, idx = [past ascending.., own];
 //                       counts the queries that chose each (b, h, j);
 //   M3 lists            one CTA: exclusive scans of the counts (list offsets, 64-query chunks);
 //                       then every choice is scattered into its (b, h, j) list as t*8 + slot;
@@ -114,13 +116,19 @@ __device__ __forceinline__ void online(float (&s)[8][4], float& m0, float& m1, f
 }
 
 // ------------------------------------------------------------------ M1
-__global__ void __launch_bounds__(D) moba_mean_kernel(const __nv_bfloat16* __restrict__ k, float* __restrict__ kbar,
-                                                      int T, int H, int bsz, int nblk) {
+// kbar: [2][B][nblk][H][D] bf16, the hi halves then the lo halves.
+__global__ void __launch_bounds__(D) moba_mean_kernel(const __nv_bfloat16* __restrict__ k,
+                                                      __nv_bfloat16* __restrict__ kbar, int B, int T, int H, int bsz,
+                                                      int nblk) {
   const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z, c = threadIdx.x;
   const int u0 = j * bsz, u1 = min(T, u0 + bsz);
   float acc = 0.f;
   for (int u = u0; u < u1; ++u) acc += __bfloat162float(k[(((size_t)b * T + u) * H + h) * D + c]);
-  kbar[(((size_t)b * nblk + j) * H + h) * D + c] = acc / (float)(u1 - u0);
+  const float mean = acc / (float)(u1 - u0);
+  const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+  const size_t o = (((size_t)b * nblk + j) * H + h) * D + c;
+  kbar[o] = hi;
+  kbar[(size_t)B * nblk * H * D + o] = __float2bfloat16_rn(mean - __bfloat162float(hi));
 }
 
 // ------------------------------------------------------------------ M2
@@ -147,14 +155,16 @@ struct TopK {
 };
 
 __global__ void __launch_bounds__(kThreads) moba_select_kernel(
-    const __nv_bfloat16* __restrict__ q, const float* __restrict__ kbar, int32_t* __restrict__ idx,
-    int32_t* __restrict__ counts, int T, int H, int bsz, int nblk, int top_k) {
-  __shared__ __align__(128) __nv_bfloat16 sHi[kKT * D];
-  __shared__ __align__(128) __nv_bfloat16 sLo[kKT * D];
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kbar, int32_t* __restrict__ idx,
+    int32_t* __restrict__ counts, int B, int T, int H, int bsz, int nblk, int top_k) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __nv_bfloat16* sHi = reinterpret_cast<__nv_bfloat16*>(smem);          // [2][kKT][D]
+  __nv_bfloat16* sLo = sHi + 2 * kKT * D;                               // [2][kKT][D]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
   const int t0 = blockIdx.x * kQ, h = blockIdx.y, b = blockIdx.z;
   const int J = t0 / bsz;                      // own block, the same for the whole tile (bsz % 64 == 0)
   const int ta = t0 + warp * 16 + gl, tb = ta + 8;
+  const size_t lo_off = (size_t)B * nblk * H * D;
   uint32_t qf[D / 16][4];
   load_q_frag(qf, q + (((size_t)b * T + min(ta, T - 1)) * H + h) * D, q + (((size_t)b * T + min(tb, T - 1)) * H + h) * D,
               ta < T, tb < T, cq);
@@ -163,37 +173,27 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
   k1.init();
   const int kk = min(top_k, J);
   if (J > top_k && top_k > 0) {
-    for (int j0 = 0; j0 < J; j0 += kKT) {
-      __syncthreads();
-      for (int e = tid; e < kKT * (D / 8); e += kThreads) {   // fp32 means -> bf16 hi + bf16 lo
+    auto load = [&](int j0, int buf) {   // blocks j0 .. j0+63 (zeros past J)
+      for (int e = tid; e < kKT * (D / 8); e += kThreads) {
         const int r = e / (D / 8), ch = e % (D / 8);
         const int j = j0 + r;
-        float x[8];
-        if (j < J) {
-          const float4* src = reinterpret_cast<const float4*>(kbar + (((size_t)b * nblk + j) * H + h) * D + ch * 8);
-          const float4 a = src[0], c = src[1];
-          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = c.x; x[5] = c.y; x[6] = c.z; x[7] = c.w;
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = 0.f;
-        }
-        uint32_t hi[4], lo[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-          const float2 hf = __bfloat1622float2(h2);
-          hi[i] = *reinterpret_cast<const uint32_t*>(&h2);
-          lo[i] = pack_bf16(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
-        }
-        *reinterpret_cast<uint4*>(sHi + SwzTile<D>::offset(r, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(sLo + SwzTile<D>::offset(r, ch)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        const size_t src = (((size_t)b * nblk + min(j, J - 1)) * H + h) * D + ch * 8;
+        cp_async16(sHi + buf * kKT * D + SwzTile<D>::offset(r, ch), kbar + src, j < J);
+        cp_async16(sLo + buf * kKT * D + SwzTile<D>::offset(r, ch), kbar + lo_off + src, j < J);
       }
+    };
+    load(0, 0);
+    cp_async_commit();
+    for (int j0 = 0, it = 0; j0 < J; j0 += kKT, ++it) {
+      if (j0 + kKT < J) load(j0 + kKT, (it + 1) & 1);
+      cp_async_commit();
+      cp_async_wait<1>();
       __syncthreads();
       float s[8][4];
 #pragma unroll
       for (int i = 0; i < 8; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
-      qk64(qf, sHi, s, lane);
-      qk64(qf, sLo, s, lane);
+      qk64(qf, sHi + (it & 1) * kKT * D, s, lane);
+      qk64(qf, sLo + (it & 1) * kKT * D, s, lane);
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -204,7 +204,9 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
             k1.offer(s[nt][2 + e], j, kk);
           }
         }
+      __syncthreads();   // this buffer is refilled two tiles later
     }
+    cp_async_wait<0>();
   }
   // merge the quad's four lists: kk rounds of a quad-wide argmax
   int sel0[kMaxK + 1], sel1[kMaxK + 1];
@@ -480,6 +482,7 @@ __global__ void __launch_bounds__(kThreads) moba_own_kernel(
 }
 
 constexpr size_t kAttnSmem = 4ull * kKT * D * 2;   // K and V, double buffered: 64 KB
+constexpr size_t kSelectSmem = 4ull * kKT * D * 2; // hi and lo block means, double buffered: 64 KB
 
 }  // namespace
 
@@ -490,7 +493,7 @@ MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k) {
   const size_t E = (size_t)B * H * nblk;
   size_t off = 0;
   L.err = off; off = up(off + 4);   // status word of the bounded device waits
-  L.kbar = off; off = up(off + (size_t)B * nblk * H * D * 4);
+  L.kbar = off; off = up(off + (size_t)B * nblk * H * D * 4);   // hi and lo bf16 halves
   L.idx = off; off = up(off + (size_t)B * H * T * (top_k + 1) * 4);
   L.counts = off; off = up(off + E * 4);
   L.offsets = off; off = up(off + (E + 1) * 4);
@@ -509,6 +512,8 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(moba_past_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moba_own_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moba_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelectSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -516,7 +521,7 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   const int E = a.B * a.H * nblk;
   const MobaLayout L = moba_layout(a.B, a.T, a.H, a.bsz, a.top_k);
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-  float* kbar = reinterpret_cast<float*>(ws + L.kbar);
+  __nv_bfloat16* kbar = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar);
   int32_t* idx = a.idx ? a.idx : reinterpret_cast<int32_t*>(ws + L.idx);
   int32_t* counts = reinterpret_cast<int32_t*>(ws + L.counts);
   int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
@@ -532,11 +537,11 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)E * 4, st);
   if (e != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  moba_mean_kernel<<<dim3(nblk, a.H, a.B), D, 0, st>>>(k, kbar, a.T, a.H, a.bsz, nblk);
+  moba_mean_kernel<<<dim3(nblk, a.H, a.B), D, 0, st>>>(k, kbar, a.B, a.T, a.H, a.bsz, nblk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  moba_select_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, 0, st>>>(q, kbar, idx, counts, a.T, a.H, a.bsz,
-                                                                              nblk, a.top_k);
+  moba_select_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kSelectSmem, st>>>(
+      q, kbar, idx, counts, a.B, a.T, a.H, a.bsz, nblk, a.top_k);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
   const int cq = tc ? moba_past_tc_chunk() : kQ;   // queries per past-attention chunk

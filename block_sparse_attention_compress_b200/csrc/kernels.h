@@ -69,7 +69,7 @@ cudaError_t launch_wait_timeout(int* err, uint64_t limit_ns, int code, cudaStrea
 
 
 struct MobaLayout {
-  size_t err, kbar, idx, counts, offsets, chunks, fill, list, part_lse, part_o, total;
+  size_t err, kbar, idx, counts, offsets, chunks, fill, chunk_list, list, part_lse, part_o, total;
 };
 // Workspace carve-up of MoBA mode (each region 256-byte aligned).
 MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k);
@@ -96,7 +96,8 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st);
 bool moba_past_tc_supported(const MobaArgs& a);
 int moba_past_tc_chunk();
 cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const int32_t* offsets,
-                                const int32_t* chunks, const int32_t* list, __nv_bfloat16* part_o, float* part_lse,
-                                int nblk, int E, size_t max_chunks, cudaStream_t st);
+                                const int32_t* chunks, const int32_t* chunk_list, const int32_t* list,
+                                __nv_bfloat16* part_o, float* part_lse, int nblk, int E, size_t max_chunks,
+                                cudaStream_t st);
 
 }  // namespace nsa

@@ -256,7 +256,8 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
 // Exclusive scans over all (b, h, j): list offsets and 64-query chunk starts (one CTA).
 __global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restrict__ counts,
                                                          int32_t* __restrict__ offsets, int32_t* __restrict__ chunks,
-                                                         int32_t* __restrict__ fill, int E, int cq) {
+                                                         int32_t* __restrict__ fill, int32_t* __restrict__ chunk_list,
+                                                         int E, int cq) {
   __shared__ int32_t s0[1024], s1[1024];
   __shared__ int32_t carry0, carry1;
   if (threadIdx.x == 0) { carry0 = 0; carry1 = 0; }
@@ -285,6 +286,10 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restri
     __syncthreads();
   }
   if (threadIdx.x == 0) { offsets[E] = carry0; chunks[E] = carry1; }
+  __syncthreads();
+  // the list of every chunk, so that a chunk finds its list with one load
+  for (int e = threadIdx.x; e < E; e += 1024)
+    for (int c = chunks[e]; c < chunks[e + 1]; ++c) chunk_list[c] = e;
 }
 
 __global__ void moba_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ offsets,
@@ -499,6 +504,8 @@ MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k) {
   L.offsets = off; off = up(off + (E + 1) * 4);
   L.chunks = off; off = up(off + (E + 1) * 4);
   L.fill = off; off = up(off + E * 4);
+  // chunk -> list, for the smallest chunk size used (64 queries)
+  L.chunk_list = off; off = up(off + ((size_t)B * H * T * top_k / kQ + E + 1) * 4);
   L.list = off; off = up(off + (size_t)B * H * T * top_k * 4);
   L.part_lse = off; off = up(off + (size_t)B * T * H * top_k * 4);
   L.part_o = off; off = up(off + (size_t)B * T * H * top_k * D * 2);
@@ -527,6 +534,7 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
   int32_t* chunks = reinterpret_cast<int32_t*>(ws + L.chunks);
   int32_t* fill = reinterpret_cast<int32_t*>(ws + L.fill);
+  int32_t* chunk_list = reinterpret_cast<int32_t*>(ws + L.chunk_list);
   int32_t* list = reinterpret_cast<int32_t*>(ws + L.list);
   float* part_lse = reinterpret_cast<float*>(ws + L.part_lse);
   __nv_bfloat16* part_o = reinterpret_cast<__nv_bfloat16*>(ws + L.part_o);
@@ -545,7 +553,7 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
   const int cq = tc ? moba_past_tc_chunk() : kQ;   // queries per past-attention chunk
-  moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, E, cq);
+  moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, chunk_list, E, cq);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   moba_scatter_kernel<<<dim3((a.T + 255) / 256, a.B * a.H), 256, 0, st>>>(idx, offsets, fill, list, a.T, a.H, nblk,
                                                                          a.top_k, a.bsz);
@@ -558,7 +566,7 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
     // every list holds at most B*H*T*top_k entries in all: the chunk count is bounded by
     // that over the chunk size plus one partial chunk per list
     const size_t max_chunks = ((size_t)a.B * a.H * a.T * a.top_k + cq - 1) / cq + (size_t)E;
-    e = launch_moba_past_tc(a, counts, offsets, chunks, list, part_o, part_lse, nblk, E, max_chunks, st);
+    e = launch_moba_past_tc(a, counts, offsets, chunks, chunk_list, list, part_o, part_lse, nblk, E, max_chunks, st);
     if (e != cudaSuccess) return e;
   } else if (a.top_k > 0) {
     moba_past_kernel<<<sms * 3, kThreads, kAttnSmem, st>>>(q, k, v, counts, offsets, chunks, list, part_o, part_lse,

@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ counts,
                     const int32_t* __restrict__ offsets, const int32_t* __restrict__ chunks,
-                    const int32_t* __restrict__ list, __nv_bfloat16* __restrict__ part_o,
+                    const int32_t* __restrict__ chunk_list, const int32_t* __restrict__ list,
+                    __nv_bfloat16* __restrict__ part_o,
                     float* __restrict__ part_lse, int T, int H, int nblk, int bsz, int top_k, int E, float scale_log2,
                     int* __restrict__ err) {
   using SM = Smem;
@@ -88,13 +89,7 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // (b, h, j) whose chunk range holds c: the last e with chunks[e] <= c
-  int lo = 0, hi = E - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (chunks[mid] <= c) lo = mid; else hi = mid - 1;
-  }
-  const int e = lo;
+  const int e = chunk_list[c];   // the (b, h, j) list this chunk belongs to
   const int bh = e / nblk, j = e % nblk, b = bh / H, h = bh % H;
   const int first = (c - chunks[e]) * kRowsM;
   const int nq = min(kRowsM, counts[e] - first);
@@ -356,8 +351,9 @@ bool moba_past_tc_supported(const MobaArgs& a) {
 int moba_past_tc_chunk() { return kRowsM; }
 
 cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const int32_t* offsets,
-                                const int32_t* chunks, const int32_t* list, __nv_bfloat16* part_o, float* part_lse,
-                                int nblk, int E, size_t max_chunks, cudaStream_t st) {
+                                const int32_t* chunks, const int32_t* chunk_list, const int32_t* list,
+                                __nv_bfloat16* part_o, float* part_lse, int nblk, int E, size_t max_chunks,
+                                cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
@@ -373,7 +369,8 @@ cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const 
   if (!make_tmap_bf16(&mk, a.k, 3, d3, s3, box) || !make_tmap_bf16(&mv, a.v, 3, d3, s3, box))
     return cudaErrorInvalidValue;
   moba_past_tc_kernel<<<(unsigned)max_chunks, kThreads, Smem::kAlloc, st>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(a.q), counts, offsets, chunks, list, part_o, part_lse, a.T, a.H, nblk,
+      mk, mv, static_cast<const __nv_bfloat16*>(a.q), counts, offsets, chunks, chunk_list, list, part_o, part_lse, a.T,
+      a.H, nblk,
       a.bsz, a.top_k, E, a.scale_log2, a.err);
   return cudaGetLastError();
 }

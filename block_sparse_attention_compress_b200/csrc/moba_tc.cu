@@ -3,19 +3,23 @@
 // §16-§17: the queries that chose one KV block are gathered, so that the block is read once
 // for all of them and the attention over it is a dense product).
 //
-// One CTA = one chunk of up to 128 gathered queries of one (batch, head, past block j) list
-// (one TMEM lane per query) against the block's keys in 128-key tiles:
+// Persistent: one CTA per SM walks the chunks, a chunk = up to 128 gathered queries of one
+// (batch, head, past block j) list (one TMEM lane per query), against the block's keys in
+// 128-key tiles:
 //   S = Q K^T        (M = 128 queries, N = 128 keys; two TMEM buffers)
 //   O += P V         (M = 128, N = 128; P in SMEM as the K-major A operand)
 // Every key of a past block precedes every query that chose it, so nothing is masked.
-// Warp roles as in the window kernel: a TMA producer (K slices into a 3-slot ring, V tiles
-// double buffered), a single-thread MMA issuer that puts S(n+1) ahead of the P.V of tile n,
+// Warp roles as in the window kernel: a producer warp (it gathers each chunk's query rows
+// with cp.async once the previous chunk's S MMAs are done with them, and streams K slices
+// into a 3-slot ring and V tiles double buffered by TMA; both run across chunk boundaries),
+// a single-thread MMA issuer that puts S(n+1) ahead of the P.V of tile n,
 // and 8 softmax warps: warps w and w+4 share TMEM lanes 32(w%4).. (the same queries) and
 // take the key halves [0, 64) and [64, 128) of every tile.  A row's softmax reference moves
 // only when a score exceeds it by more than 2^8; the two threads of a row agree on it through
 // one barrier of the warp pair per tile, and rescale their halves of O in TMEM when it moves.
-// The softmax warps gather the chunk's query rows with cp.async.  Epilogue per query of the
-// chunk: part_o = bf16(O / l) and part_lse = m + log2(l), merged later with the own block.
+// Epilogue per query of the chunk: part_o = bf16(O / l) and part_lse = m + log2(l), merged
+// later with the own block.
+#include <algorithm>
 #include <cfloat>
 
 #include "common.cuh"
@@ -38,7 +42,7 @@ constexpr uint32_t kColS = 0, kColO = 256;        // S buffer b at 128b; O at 25
 constexpr float kSlack = 8.f;
 
 enum Err { kErrQ = 61, kErrKFull, kErrKEmpty, kErrVFull, kErrVEmpty, kErrSFull, kErrSEmpty, kErrPFull, kErrPEmpty,
-           kErrOFull };
+           kErrOFull, kErrQEmpty, kErrOEmpty };
 
 struct Smem {
   static constexpr uint32_t kQ = 0;                                         // 2 x 64-column slices
@@ -46,9 +50,8 @@ struct Smem {
   static constexpr uint32_t kV = kK + kKSlots * kSlice;                     // 2 tiles x 2 slices
   static constexpr uint32_t kP = kV + 2 * 2 * kSlice;                       // P: [2 key halves][128 rows][128 B]
   static constexpr uint32_t kPair = kP + 2 * kSlice;                        // [2][128] fp32 + [2][128] flags
-  static constexpr uint32_t kEnt = kPair + 2 * kRowsM * 4 + 2 * kRowsM * 4; // [128] list entries of the chunk
-  static constexpr uint32_t kBar = kEnt + kRowsM * 4;
-  static constexpr int kNumBars = 1 + 2 * kKSlots + 2 * 2 + 2 * 2 + 2 + 1;
+  static constexpr uint32_t kBar = kPair + 2 * kRowsM * 4 + 2 * kRowsM * 4;
+  static constexpr int kNumBars = 1 + 2 * kKSlots + 2 * 2 + 2 * 2 + 2 + 1 + 2;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;
@@ -60,12 +63,11 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                     const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ counts,
                     const int32_t* __restrict__ offsets, const int32_t* __restrict__ chunks,
                     const int32_t* __restrict__ chunk_list, const int32_t* __restrict__ list,
-                    __nv_bfloat16* __restrict__ part_o,
-                    float* __restrict__ part_lse, int T, int H, int nblk, int bsz, int top_k, int E, float scale_log2,
-                    int* __restrict__ err) {
+                    __nv_bfloat16* __restrict__ part_o, float* __restrict__ part_lse, int T, int H, int nblk, int bsz,
+                    int top_k, int E, float scale_log2, int* __restrict__ err) {
   using SM = Smem;
-  const int c = blockIdx.x;
-  if (c >= chunks[E]) return;   // the grid is an upper bound of the chunk count
+  const int total = chunks[E];
+  if ((int)blockIdx.x >= total) return;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + SM::kQ;
@@ -74,7 +76,6 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   uint8_t* sP = smem + SM::kP;
   float* sPairMax = reinterpret_cast<float*>(smem + SM::kPair);            // [half][row]
   int* sPairFlag = reinterpret_cast<int*>(sPairMax + 2 * kRowsM);           // [half][row]
-  int32_t* sEnt = reinterpret_cast<int32_t*>(smem + SM::kEnt);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* bar_q = bars;
   uint64_t* k_full = bars + 1;
@@ -86,14 +87,24 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   uint64_t* p_full = s_empty + 2;
   uint64_t* p_empty = p_full + 1;
   uint64_t* o_full = p_empty + 1;
+  uint64_t* q_empty = o_full + 1;   // the S MMAs of a chunk have read its queries
+  uint64_t* o_empty = q_empty + 1;  // the softmax warps have read a chunk's O
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int e = chunk_list[c];   // the (b, h, j) list this chunk belongs to
-  const int bh = e / nblk, j = e % nblk, b = bh / H, h = bh % H;
-  const int first = (c - chunks[e]) * kRowsM;
-  const int nq = min(kRowsM, counts[e] - first);
   const int ntiles = bsz / kBlk;
+  struct Chunk { int e, b, h, j, first, nq; };
+  auto chunk_of = [&](int c) {
+    Chunk x;
+    x.e = chunk_list[c];   // the (b, h, j) list this chunk belongs to
+    const int bh = x.e / nblk;
+    x.j = x.e % nblk;
+    x.b = bh / H;
+    x.h = bh % H;
+    x.first = (c - chunks[x.e]) * kRowsM;
+    x.nq = min(kRowsM, counts[x.e] - x.first);
+    return x;
+  };
 
   if (tid == 0) {
     tc::mbar_init(bar_q, 1);
@@ -110,6 +121,8 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tc::mbar_init(p_full, kSoftWarps);
     tc::mbar_init(p_empty, 1);
     tc::mbar_init(o_full, 1);
+    tc::mbar_init(q_empty, 1);
+    tc::mbar_init(o_empty, kSoftWarps);
     tc::fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -122,45 +135,71 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kTmaWarp) {
-    // ------------------------------------------------------------ TMA producer
-    if (tc::elect_one()) {
+    // ------------------------------------------------------------ producer
+    // Per chunk: gather its query rows (each lane four rows, cp.async into the K-major,
+    // 128-byte-swizzled operand; zeros past the chunk's end) once the previous chunk's S
+    // MMAs are done with the buffer, then stream the block's K/V tiles (lane 0, TMA).
+    if (lane == 0) {
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
-      int fill = 0;
-      bool ok = true;
+    }
+    int fill = 0, vcnt = 0, k = 0;
+    bool ok = true;
+    for (int c = blockIdx.x; c < total && ok; c += gridDim.x, ++k) {
+      const Chunk x = chunk_of(c);
+      if (k > 0) ok = __all_sync(0xffffffffu, tc::mbar_wait(q_empty, (k - 1) & 1, err, kErrQEmpty));
+      if (!ok) break;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane + 32 * i;
+        const int ent = r < x.nq ? list[offsets[x.e] + x.first + r] : -1;
+        const __nv_bfloat16* src = q + (((size_t)x.b * T + (ent >= 0 ? (ent >> 3) : 0)) * H + x.h) * D;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch)
+          cp_async16(sQ + (ch >> 3) * kSlice + r * 128 + (((ch & 7) ^ (r & 7)) << 4), src + 8 * ch, ent >= 0);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      tc::fence_async_smem();   // the MMAs read these rows through the async proxy
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(bar_q);
       for (int n = 0; n < ntiles && ok; ++n) {
-        const int row = b * T + j * bsz + n * kBlk;
+        const int row = x.b * T + x.j * bsz + n * kBlk;
         for (int s = 0; s < 2 && ok; ++s, ++fill) {
           const int slot = fill % kKSlots;
-          ok = tc::mbar_wait(k_empty + slot, ((fill / kKSlots) & 1) ^ 1, err, kErrKEmpty);
-          if (!ok) break;
-          tc::mbar_expect_tx(k_full + slot, kSlice);
-          tc::tma_load_3d(sK + slot * kSlice, &tm_k, k_full + slot, s * 64, h, row);
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(k_empty + slot, ((fill / kKSlots) & 1) ^ 1, err, kErrKEmpty));
+          if (ok && lane == 0) {
+            tc::mbar_expect_tx(k_full + slot, kSlice);
+            tc::tma_load_3d(sK + slot * kSlice, &tm_k, k_full + slot, s * 64, x.h, row);
+          }
         }
         if (!ok) break;
-        const int vb = n & 1;
-        ok = tc::mbar_wait(v_empty + vb, ((n >> 1) & 1) ^ 1, err, kErrVEmpty);
-        if (!ok) break;
-        tc::mbar_expect_tx(v_full + vb, 2 * kSlice);
-        for (int s = 0; s < 2; ++s) tc::tma_load_3d(sV + (vb * 2 + s) * kSlice, &tm_v, v_full + vb, s * 64, h, row);
+        const int vb = vcnt & 1;
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(v_empty + vb, ((vcnt >> 1) & 1) ^ 1, err, kErrVEmpty));
+        if (ok && lane == 0) {
+          tc::mbar_expect_tx(v_full + vb, 2 * kSlice);
+          for (int s = 0; s < 2; ++s) tc::tma_load_3d(sV + (vb * 2 + s) * kSlice, &tm_v, v_full + vb, s * 64, x.h, row);
+        }
+        ++vcnt;
       }
-      for (int i = 0; i < kKSlots && i < fill; ++i) {   // let the copies in flight land (bounded)
+    }
+    if (lane == 0) {   // let the copies in flight land (bounded)
+      for (int i = 0; i < kKSlots && i < fill; ++i) {
         const int f = fill - 1 - i;
         tc::mbar_wait(k_full + (f % kKSlots), (f / kKSlots) & 1, err, kErrKFull);
       }
-      for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull);
+      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (tc::elect_one()) {
       const uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);      // S = Q K^T  (both K-major)
       const uint32_t idPV = tc::idesc_bf16(128, D, 0, 1);       // O = P V    (P K-major, V MN-major)
-      bool ok = tc::mbar_wait(bar_q, 0, err, kErrQ);
-      tc::tc_fence_after();
-      int fill = 0;
-      auto issue_s = [&](int n) -> bool {
-        const int sb = n & 1;
-        if (!tc::mbar_wait(s_empty + sb, ((n >> 1) & 1) ^ 1, err, kErrSEmpty)) return false;
+      int fill = 0, use = 0, pc = 0, k = 0;
+      bool ok = true;
+      auto issue_s = [&]() -> bool {
+        const int sb = use & 1;
+        if (!tc::mbar_wait(s_empty + sb, ((use >> 1) & 1) ^ 1, err, kErrSEmpty)) return false;
         tc::tc_fence_after();
         for (int s = 0; s < 2; ++s, ++fill) {
           const int slot = fill % kKSlots;
@@ -174,164 +213,171 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           tc::mma_commit(k_empty + slot);
         }
         tc::mma_commit(s_full + sb);
+        ++use;
         return true;
       };
       auto issue_pv = [&](int n) -> bool {
-        if (!tc::mbar_wait(p_full, n & 1, err, kErrPFull) ||
-            !tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull))
+        if (!tc::mbar_wait(p_full, pc & 1, err, kErrPFull) ||
+            !tc::mbar_wait(v_full + (pc & 1), (pc >> 1) & 1, err, kErrVFull))
           return false;
         tc::tc_fence_after();
-        const uint8_t* vb = sV + (n & 1) * 2 * kSlice;
+        const uint8_t* vb = sV + (pc & 1) * 2 * kSlice;
         for (int ks = 0; ks < kBlk / 16; ++ks) {
           const uint64_t da = tc::sdesc(sP + (ks >> 2) * kSlice + (ks & 3) * 32, 16, 1024);
           const uint64_t db = tc::sdesc(vb + ks * 16 * 128, kSlice, 1024);
           tc::mma_ss(tmem + kColO, da, db, idPV, (n | ks) != 0);
         }
         tc::mma_commit(p_empty);
-        tc::mma_commit(v_empty + (n & 1));
+        tc::mma_commit(v_empty + (pc & 1));
+        ++pc;
         return true;
       };
-      if (ok && ntiles > 0) ok = issue_s(0);
-      for (int n = 0; n < ntiles && ok; ++n) {
-        if (n + 1 < ntiles) ok = issue_s(n + 1);
-        if (ok) ok = issue_pv(n);
+      for (int c = blockIdx.x; c < total && ok; c += gridDim.x, ++k) {
+        ok = tc::mbar_wait(bar_q, k & 1, err, kErrQ);
+        if (!ok) break;
+        tc::tc_fence_after();
+        ok = issue_s();
+        if (ok && ntiles == 1) tc::mma_commit(q_empty);
+        // O is overwritten (and o_full committed) only after the previous chunk's epilogue read it
+        if (ok && k > 0) ok = tc::mbar_wait(o_empty, (k - 1) & 1, err, kErrOEmpty);
+        for (int n = 0; n < ntiles && ok; ++n) {
+          if (n + 1 < ntiles) {
+            ok = issue_s();
+            if (ok && n + 2 == ntiles) tc::mma_commit(q_empty);   // the chunk's last S reads Q
+          }
+          if (ok) ok = issue_pv(n);
+        }
+        if (ok) tc::mma_commit(o_full);
       }
-      if (ok && ntiles > 0) tc::mma_commit(o_full);
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    // gather the chunk's queries: thread i copies row i/2, 64-column slice i%2 (zeros for
-    // the rows past the chunk's end), into the K-major, 128-byte-swizzled Q operand
-    {
-      const int qr = tid >> 1, qs = tid & 1;
-      const int ent = qr < nq ? list[offsets[e] + first + qr] : -1;
-      if (qs == 0) sEnt[qr] = ent;
-      const __nv_bfloat16* src = q + (((size_t)b * T + (ent >= 0 ? (ent >> 3) : 0)) * H + h) * D + 64 * qs;
-      uint8_t* dst = sQ + qs * kSlice + qr * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) cp_async16(dst + ((ch ^ (qr & 7)) << 4), src + 8 * ch, ent >= 0);
-      cp_async_commit();
-      cp_async_wait<0>();
-      tc::fence_async_smem();   // the MMAs read these rows through the async proxy
-      tc::named_sync(5, 32 * kSoftWarps);
-      if (tid == 0) tc::mbar_arrive(bar_q);
-    }
     const int gr = warp >> 2, q4 = warp & 3;       // key half, TMEM lane quadrant
     const int r = 32 * q4 + lane;                  // this thread's query row
     const int pbar = 1 + q4;                       // barrier of the warp pair sharing these rows
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int n = 0; n < ntiles; ++n) {
-      const int sb = n & 1;
-      ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_full + sb, (n >> 1) & 1, err, kErrSFull));
-      float v[64];
-      if (ok) {
-        tc::tc_fence_after();
+    int use = 0, pc = 0, k = 0;
+    for (int c = blockIdx.x; c < total; c += gridDim.x, ++k) {
+      const Chunk x = chunk_of(c);
+      // this row's list entry, read now for the epilogue (it is in L2: the producer read it)
+      const int ent = r < x.nq ? list[offsets[x.e] + x.first + r] : -1;
+      float m = -INFINITY, l = 0.f;
+      for (int n = 0; n < ntiles; ++n, ++use, ++pc) {
+        const int sb = use & 1;
+        ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull));
+        float v[64];
+        if (ok) {
+          tc::tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          tc::tmem_ld16(lane_addr + kColS + 128 * sb + 64 * gr + 16 * cc, *reinterpret_cast<float(*)[16]>(v + 16 * cc));
-        tc::tmem_wait_ld();
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(s_empty + sb);
-      }
-#pragma unroll
-      for (int jj = 0; jj < 64; ++jj) v[jj] *= scale_log2;
-      float cmx[8];
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) cmx[cc] = fmaxf(fmaxf(v[cc], v[cc + 8]), fmaxf(v[cc + 16], v[cc + 24]));
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        cmx[cc] = fmaxf(cmx[cc], fmaxf(fmaxf(v[cc + 32], v[cc + 40]), fmaxf(v[cc + 48], v[cc + 56])));
-      const float lmax = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
-                               fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
-      // the two threads of a row agree on its reference; a failed wait also takes the
-      // exchange, so that both warps of the pair leave together
-      if (tc::vote_any(pbar, 64, !ok || lmax > m + kSlack)) {
-        sPairMax[gr * kRowsM + r] = lmax;
-        sPairFlag[gr * kRowsM + r] = ok;
-        tc::named_sync(pbar, 64);
-        const bool pair_ok = __all_sync(0xffffffffu, sPairFlag[r] && sPairFlag[kRowsM + r]);
-        if (!pair_ok) {
-          ok = false;
-          break;
+          for (int cc = 0; cc < 4; ++cc)
+            tc::tmem_ld16(lane_addr + kColS + 128 * sb + 64 * gr + 16 * cc, *reinterpret_cast<float(*)[16]>(v + 16 * cc));
+          tc::tmem_wait_ld();
+          tc::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(s_empty + sb);
         }
-        const float mn = fmaxf(m, fmaxf(sPairMax[r], sPairMax[kRowsM + r]));
-        const float cf = mn == -INFINITY ? 1.f : ex2(m - mn);
-        l *= cf;
-        if (__any_sync(0xffffffffu, cf != 1.f) && n > 0) {
-          // rescale this thread's half of the row's O once the previous P.V has finished
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty));
-          if (ok) {
-            tc::tc_fence_after();
 #pragma unroll
-            for (int qq = 0; qq < D / 2 / 16; ++qq) {
-              float o[16];
-              const uint32_t addr = lane_addr + kColO + (D / 2) * gr + 16 * qq;
-              tc::tmem_ld16(addr, o);
-              tc::tmem_wait_ld();
+        for (int jj = 0; jj < 64; ++jj) v[jj] *= scale_log2;
+        float cmx[8];
 #pragma unroll
-              for (int i = 0; i < 16; ++i) o[i] *= cf;
-              tc::tmem_st16(addr, o);
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
+        for (int cc = 0; cc < 8; ++cc) cmx[cc] = fmaxf(fmaxf(v[cc], v[cc + 8]), fmaxf(v[cc + 16], v[cc + 24]));
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          cmx[cc] = fmaxf(cmx[cc], fmaxf(fmaxf(v[cc + 32], v[cc + 40]), fmaxf(v[cc + 48], v[cc + 56])));
+        const float lmax = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                                 fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+        // the two threads of a row agree on its reference; a failed wait also takes the
+        // exchange, so that both warps of the pair leave together
+        if (tc::vote_any(pbar, 64, !ok || lmax > m + kSlack)) {
+          sPairMax[gr * kRowsM + r] = lmax;
+          sPairFlag[gr * kRowsM + r] = ok;
+          tc::named_sync(pbar, 64);
+          const bool pair_ok = __all_sync(0xffffffffu, sPairFlag[r] && sPairFlag[kRowsM + r]);
+          if (!pair_ok) {
+            ok = false;
+            break;
           }
+          const float mn = fmaxf(m, fmaxf(sPairMax[r], sPairMax[kRowsM + r]));
+          const float cf = mn == -INFINITY ? 1.f : ex2(m - mn);
+          l *= cf;
+          if (__any_sync(0xffffffffu, cf != 1.f) && n > 0) {
+            // rescale this thread's half of the row's O once the previous P.V has finished
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(p_empty, (pc - 1) & 1, err, kErrPEmpty));
+            if (ok) {
+              tc::tc_fence_after();
+#pragma unroll
+              for (int qq = 0; qq < D / 2 / 16; ++qq) {
+                float o[16];
+                const uint32_t addr = lane_addr + kColO + (D / 2) * gr + 16 * qq;
+                tc::tmem_ld16(addr, o);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] *= cf;
+                tc::tmem_st16(addr, o);
+              }
+              tc::tmem_wait_st();
+              tc::tc_fence_before();
+            }
+          }
+          m = mn;
+          tc::named_sync(pbar, 64);   // both halves have read the exchange before it is reused
         }
-        m = mn;
-        tc::named_sync(pbar, 64);   // both halves have read the exchange before it is reused
+        const float base = m == -INFINITY ? 0.f : m;
+        uint32_t pk[32];
+        float ps[8];
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) ps[cc] = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 64; jj += 2) {
+          const float p0 = ex2(v[jj] - base), p1 = ex2(v[jj + 1] - base);
+          ps[(jj >> 1) & 7] += p0 + p1;
+          pk[jj / 2] = pack_bf16(p0, p1);
+        }
+        l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        // P(pc) overwrites the buffer once P.V(pc-1) has read it
+        if (pc > 0) ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(p_empty, (pc - 1) & 1, err, kErrPEmpty));
+        uint8_t* prow = sP + gr * kSlice + r * 128;     // row r, keys of this half: K-major, 128-byte swizzle
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)
+          *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+        tc::fence_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(p_full);
       }
-      const float base = m == -INFINITY ? 0.f : m;
-      uint32_t pk[32];
-      float ps[8];
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc) ps[cc] = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < 64; jj += 2) {
-        const float p0 = ex2(v[jj] - base), p1 = ex2(v[jj + 1] - base);
-        ps[(jj >> 1) & 7] += p0 + p1;
-        pk[jj / 2] = pack_bf16(p0, p1);
-      }
-      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      // P(n) overwrites the buffer once P.V(n-1) has read it
-      if (n > 0) ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty));
-      uint8_t* prow = sP + gr * kSlice + r * 128;     // row r, keys of this half: K-major, 128-byte swizzle
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      tc::fence_async_smem();
-      __syncwarp();
-      if (lane == 0) tc::mbar_arrive(p_full);
-    }
-    // epilogue: the row sum over both halves, then part_o = bf16(O / l), part_lse = m + log2(l)
-    sPairMax[gr * kRowsM + r] = l;
-    sPairFlag[gr * kRowsM + r] = ok;
-    tc::named_sync(pbar, 64);
-    const bool pair_ok = sPairFlag[r] && sPairFlag[kRowsM + r];
-    const float L = sPairMax[r] + sPairMax[kRowsM + r];
-    ok = __all_sync(0xffffffffu, pair_ok && (ntiles == 0 || tc::mbar_wait(o_full, 0, err, kErrOFull)));
-    if (ok) {
+      // epilogue: the row sum over both halves, then part_o = bf16(O / l), part_lse = m + log2(l)
+      sPairMax[gr * kRowsM + r] = l;
+      sPairFlag[gr * kRowsM + r] = ok;
+      tc::named_sync(pbar, 64);
+      const bool pair_ok = sPairFlag[r] && sPairFlag[kRowsM + r];
+      const float L = sPairMax[r] + sPairMax[kRowsM + r];
+      tc::named_sync(pbar, 64);   // both halves have read the sums before the next chunk reuses them
+      ok = tc::vote_all(5, 32 * kSoftWarps, pair_ok && tc::mbar_wait(o_full, k & 1, err, kErrOFull));
+      if (!ok) break;
       tc::tc_fence_after();
-      const int ent = sEnt[r];
       const float inv = L > 0.f ? 1.f / L : 0.f;
-      const size_t base = ent >= 0 ? (((size_t)b * T + (ent >> 3)) * H + h) * top_k + (ent & 7) : 0;
+      const size_t base = ent >= 0 ? (((size_t)x.b * T + (ent >> 3)) * H + x.h) * top_k + (ent & 7) : 0;
       __nv_bfloat16* orow = part_o + base * D + (D / 2) * gr;
+      float o[D / 2];
 #pragma unroll
-      for (int qq = 0; qq < D / 2 / 16; ++qq) {
-        float o[16];
-        tc::tmem_ld16(lane_addr + kColO + (D / 2) * gr + 16 * qq, o);
-        tc::tmem_wait_ld();
-        if (ent >= 0) {
+      for (int qq = 0; qq < D / 2 / 16; ++qq)
+        tc::tmem_ld16(lane_addr + kColO + (D / 2) * gr + 16 * qq, *reinterpret_cast<float(*)[16]>(o + 16 * qq));
+      tc::tmem_wait_ld();
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(o_empty);
+      if (ent >= 0) {
+#pragma unroll
+        for (int qq = 0; qq < D / 2 / 16; ++qq) {
           uint32_t w[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
+          for (int i = 0; i < 8; ++i) w[i] = pack_bf16(o[16 * qq + 2 * i] * inv, o[16 * qq + 2 * i + 1] * inv);
           *reinterpret_cast<uint4*>(orow + 16 * qq) = make_uint4(w[0], w[1], w[2], w[3]);
           *reinterpret_cast<uint4*>(orow + 16 * qq + 8) = make_uint4(w[4], w[5], w[6], w[7]);
         }
+        if (gr == 0) part_lse[base] = m + __log2f(L);
       }
-      if (ent >= 0 && gr == 0) part_lse[base] = m + __log2f(L);
     }
   }
 
@@ -368,7 +414,15 @@ cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const 
   const uint32_t box[3] = {64, 1, (uint32_t)kBlk};
   if (!make_tmap_bf16(&mk, a.k, 3, d3, s3, box) || !make_tmap_bf16(&mv, a.v, 3, d3, s3, box))
     return cudaErrorInvalidValue;
-  moba_past_tc_kernel<<<(unsigned)max_chunks, kThreads, Smem::kAlloc, st>>>(
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const unsigned grid = (unsigned)std::min<size_t>(max_chunks, (size_t)sms);
+  moba_past_tc_kernel<<<grid, kThreads, Smem::kAlloc, st>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), counts, offsets, chunks, chunk_list, list, part_o, part_lse, a.T,
       a.H, nblk,
       a.bsz, a.top_k, E, a.scale_log2, a.err);

@@ -372,6 +372,20 @@ def run_decode_bench(args, dev, world):
     ms = [es[0].elapsed_time(es[-1]) for es in evs]
 
     mean_ms = allreduce_max(statistics.mean(ms), world, dev)
+    # the compressed-cache update a decode step makes when its new token completes a block:
+    # at L = 65536 every sequence is at a block boundary, one new Kc and Vc row each
+    app_ms = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        nsa.nsa_compress_append(d.k_cache, d.w_k, d.seqlens, kc)
+        nsa.nsa_compress_append(d.v_cache, d.w_v, d.seqlens, vc)
+        e1.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            app_ms.append(e0.elapsed_time(e1))
+    app_us = allreduce_max(statistics.mean(app_ms), world, dev) * 1e3
     nbytes = decode_bytes(idx.cpu(), d.seqlens.cpu(), hq, dk, dv, c["window"])
     peaks, src = load_peaks()
     gbs = nbytes / (mean_ms * 1e-3) / 1e9
@@ -380,7 +394,10 @@ def run_decode_bench(args, dev, world):
             "us_per_step": mean_ms * 1e3, "tokens_per_s": world * B / (mean_ms * 1e-3),
             "bytes_per_step": nbytes, "achieved_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
             "frac": gbs / peaks["hbm_gbs"], "frac_of_8tbs": gbs / 8000.0, "bound": "hbm",
-            "peak_source": f"{src} hbm_gbs", "gpu_launches": args.steps,
+            "peak_source": f"{src} hbm_gbs", "gpu_launches": args.steps * 3,
+            "compress_append_us": app_us,
+            "compress_append_note": "nsa_compress_append for K and V (one new compressed row per sequence and "
+                                    "head, 32 x 4 heads), the update a step makes every 16 tokens",
             "l2": "256 MB flush before every timed step (outside the events)"}
 
 

@@ -17,8 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libnsa.so")
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
 NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
 
-EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_forward", "nsa_decode", "nsa_forward_noalloc",
-            "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
+EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_decode",
+            "nsa_forward_noalloc", "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
 
 
 class NsaConfig(ctypes.Structure):
@@ -62,6 +62,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_workspace_size.restype = sz
     lib.nsa_compress.argtypes = [vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.nsa_compress.restype = ctypes.c_int
+    lib.nsa_compress_append.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
+    lib.nsa_compress_append.restype = ctypes.c_int
     lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
     lib.nsa_forward.restype = ctypes.c_int
     lib.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, cfgp, vp, vp]
@@ -131,6 +133,15 @@ def nsa_compress(x, w, out, l: int = 32, s: int = 16, stream=None, check: bool =
     st = load_library().nsa_compress(_ptr(x), _ptr(w), B, T, H, d, w.shape[1], l, s, _ptr(out),
                                      _stream(stream, x))
     return _check(st, "nsa_compress") if check else st
+
+
+def nsa_compress_append(x_cache, w, seqlens, out_cache, l: int = 32, s: int = 16, stream=None,
+                        check: bool = True) -> int:
+    """Write the compressed block that each sequence's newest token completes (see include/nsa.h)."""
+    B, Lmax, H, d = x_cache.shape
+    st = load_library().nsa_compress_append(_ptr(x_cache), _ptr(w), _ptr(seqlens), B, Lmax, H, d, w.shape[1], l, s,
+                                            _ptr(out_cache), out_cache.shape[1], _stream(stream, x_cache))
+    return _check(st, "nsa_compress_append") if check else st
 
 
 def nsa_forward(q, k, v, gates, cfg: NsaConfig, out, stream=None, check: bool = True) -> int:

@@ -6,6 +6,10 @@
 // As a GEMM: M = N_c windows per (b, h), N = d_out, K = l*d.  The A operand is
 // never materialised: window i, k-chunk (r, c0) is read straight from x
 // (each 64-wide k-chunk lies inside one token because d % 64 == 0).
+// Append mode (decode with a growing cache): the CTA's rows are the sequences b instead of
+// the windows, each at the one window its newest token completes (or none).  A row's
+// arithmetic (k chunks in order, the same MMA fragments) does not depend on which rows share
+// its CTA, so every block equals bitwise the one the full compression computes.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -14,17 +18,34 @@ namespace nsa {
 namespace {
 constexpr int kBM = 64, kBN = 64, kBK = 64, kThreads = 128;
 
-template <int D, int DOUT>
+// STAGES-deep cp.async ring of (A, W) k-chunks: 2 when the grid is large enough to hide the
+// loads' latency; more for the append launch, whose few CTAs each run one long k chain.
+template <int D, int DOUT, int STAGES>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
-                int l, int s, int nc, __nv_bfloat16* __restrict__ out) {
-  __shared__ __align__(128) __nv_bfloat16 sA[2][kBM * kBK];
-  __shared__ __align__(128) __nv_bfloat16 sB[2][kBK * kBN];
+                int l, int s, int nc, __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ seqlens,
+                int B) {
+  extern __shared__ __align__(128) uint8_t csmem[];
+  auto sA = reinterpret_cast<__nv_bfloat16(*)[kBM * kBK]>(csmem);                          // [STAGES]
+  auto sB = reinterpret_cast<__nv_bfloat16(*)[kBK * kBN]>(csmem + STAGES * kBM * kBK * 2);  // [STAGES]
+  __shared__ int sWin[kBM];   // append mode: the window of each row's sequence, or -1
   using Swz = SwzTile<kBK>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
-  const int bh = blockIdx.z, b = bh / H, h = bh % H;
+  const bool app = seqlens != nullptr;
+  const int bh = blockIdx.z, b = app ? 0 : bh / H, h = app ? bh : bh % H;
   const int nk = l * D / kBK;
+  if (app) {
+    if (tid < kBM) {
+      const int bb = i0 + tid;
+      const int L = bb < B ? min(seqlens[bb], T) : 0;
+      sWin[tid] = (L >= l && (L - l) % s == 0 && (L - l) / s < nc) ? (L - l) / s : -1;
+    }
+    __syncthreads();
+  }
+  // the source row of CTA row `row`: (sequence, window) in append mode, else (b, i0 + row)
+  auto row_seq = [&](int row) { return app ? i0 + row : b; };
+  auto row_win = [&](int row) { return app ? sWin[row] : (i0 + row < nc ? i0 + row : -1); };
 
   auto load = [&](int kc, int buf) {
     const int kk0 = kc * kBK;
@@ -32,10 +53,10 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
 #pragma unroll
     for (int e = tid; e < kBM * (kBK / 8); e += kThreads) {
       const int row = e >> 3, ch = e & 7;
-      const int i = i0 + row;
-      const bool ok = i < nc;
+      const int i = row_win(row);
+      const bool ok = i >= 0;
       const __nv_bfloat16* src =
-          x + (((size_t)b * T + (ok ? (size_t)s * i + r : 0)) * H + h) * D + c0 + ch * 8;
+          x + (((size_t)(ok ? row_seq(row) : 0) * T + (ok ? (size_t)s * i + r : 0)) * H + h) * D + c0 + ch * 8;
       cp_async16(&sA[buf][Swz::offset(row, ch)], src, ok);
     }
 #pragma unroll
@@ -50,14 +71,17 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
 #pragma unroll
   for (int j = 0; j < kBN / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
 
-  load(0, 0);
-  cp_async_commit();
-  for (int kc = 0; kc < nk; ++kc) {
-    if (kc + 1 < nk) load(kc + 1, (kc + 1) & 1);
+#pragma unroll
+  for (int st = 0; st + 1 < STAGES; ++st) {
+    if (st < nk) load(st, st);
     cp_async_commit();
-    cp_async_wait<1>();
+  }
+  for (int kc = 0; kc < nk; ++kc) {
+    if (kc + STAGES - 1 < nk) load(kc + STAGES - 1, (kc + STAGES - 1) % STAGES);
+    cp_async_commit();
+    cp_async_wait<STAGES - 1>();
     __syncthreads();
-    const int buf = kc & 1;
+    const int buf = kc % STAGES;
 #pragma unroll
     for (int ks = 0; ks < kBK / 16; ++ks) {
       uint32_t a[4];
@@ -83,9 +107,10 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   const int gl = lane >> 2, cq = lane & 3;
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
-    const int i = i0 + warp * 16 + gl + half * 8;
-    if (i >= nc) continue;
-    __nv_bfloat16* dst = out + (((size_t)b * nc + i) * H + h) * DOUT + n0;
+    const int row = warp * 16 + gl + half * 8;
+    const int i = row_win(row);
+    if (i < 0) continue;
+    __nv_bfloat16* dst = out + (((size_t)row_seq(row) * nc + i) * H + h) * DOUT + n0;
 #pragma unroll
     for (int j = 0; j < kBN / 8; ++j) {
       const uint32_t v = pack_bf16(acc[j][2 * half], acc[j][2 * half + 1]);
@@ -94,16 +119,47 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   }
 }
 
+constexpr size_t smem_bytes(int stages) { return (size_t)stages * (kBM * kBK + kBK * kBN) * 2; }
+
 template <int D>
 cudaError_t launch(const void* x, const void* w, int B, int T, int H, int l, int s, int nc, void* out,
                    cudaStream_t st) {
   dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
-  compress_kernel<D, D><<<grid, kThreads, 0, st>>>(static_cast<const __nv_bfloat16*>(x),
+  compress_kernel<D, D, 2><<<grid, kThreads, smem_bytes(2), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w), T, H, l, s, nc,
-                                                   static_cast<__nv_bfloat16*>(out));
+                                                   static_cast<__nv_bfloat16*>(out), nullptr, B);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H, int l,
+                          int s, int ncmax, void* out, cudaStream_t st) {
+  constexpr int kStages = 8;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(compress_kernel<D, D, kStages>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((B + kBM - 1) / kBM, D / kBN, H);
+  compress_kernel<D, D, kStages><<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                   static_cast<const __nv_bfloat16*>(w), Lmax, H, l, s, ncmax,
+                                                   static_cast<__nv_bfloat16*>(out), seqlens, B);
   return cudaGetLastError();
 }
 }  // namespace
+
+cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,
+                                   int d, int l, int s, int ncmax, void* out, cudaStream_t st) {
+  if (B == 0 || H == 0 || ncmax == 0) return cudaSuccess;
+  switch (d) {
+    case 64: return launch_append<64>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
+    case 128: return launch_append<128>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
+    case 192: return launch_append<192>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
                             cudaStream_t st) {

@@ -12,6 +12,10 @@ namespace nsa {
 // K1: phi for every (b, h): out [B, N_c, H, d] bf16 (l = 32, s = 16 validated).
 cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
                             cudaStream_t st);
+// K1 for a growing cache: for each sequence b whose newest token (L = seqlens[b], clamped
+// to Lmax) completes window i = (L - l)/s < ncmax, out[b, i, h, :] for every head.
+cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,
+                                   int d, int l, int s, int ncmax, void* out, cudaStream_t st);
 
 struct FwdArgs {
   const void* q;      // [B, T, Hq, dk] bf16

@@ -163,6 +163,19 @@ nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t T, int3
   return from_cuda(nsa::launch_compress(x, w, B, T, H, d, l, s, out, static_cast<cudaStream_t>(stream)));
 }
 
+nsa_status nsa_compress_append(const void* x_cache, const void* w, const int32_t* seqlens, int32_t B, int32_t Lmax,
+                               int32_t H, int32_t d, int32_t d_out, int32_t l, int32_t s, void* out_cache,
+                               int32_t ncmax, void* stream) {
+  if (!x_cache || !w || !seqlens || !out_cache || B < 1 || Lmax < 1 || H < 1 || d < 1 || d_out < 1 || l < 1 ||
+      s < 1 || ncmax < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(x_cache) || !aligned16(w) || !aligned16(out_cache) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return NSA_ERR_INVALID_ARG;
+  if (l != 32 || s != 16 || d_out != d || (d != 64 && d != 128 && d != 192)) return NSA_ERR_UNSUPPORTED;
+  return from_cuda(nsa::launch_compress_append(x_cache, w, seqlens, B, Lmax, H, d, l, s, ncmax, out_cache,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* gates, const nsa_config* cfg,
                        void* out, void* stream) {
   nsa_status st = check_cfg(cfg);

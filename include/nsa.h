@@ -180,6 +180,25 @@ NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_
                       void* out, void* stream);
 
 /*
+ * nsa_compress_append -- keeps a compressed cache current while decoding ([NOTES] §5: each
+ * block of l tokens, taken every s tokens, is one compressed key/value; with a growing cache a
+ * new block is complete every s tokens).
+ *   x_cache  bf16 [B, Lmax, H, d]          keys (or values) of the cache
+ *   w        bf16 [l*d, d_out]             phi weights, as for nsa_compress
+ *   seqlens  int32 [B] device              L per sequence: tokens 0 .. L-1 are in the cache
+ *   out_cache bf16 [B, ncmax, H, d_out]    the compressed cache
+ * For every sequence b with L = min(seqlens[b], Lmax) >= l, (L - l) % s == 0 and
+ * i = (L - l)/s < ncmax: out_cache[b, i, h, :] = vec(x_cache[b, s*i : s*i+l, h, :]) @ w for
+ * every head h, the block that token L-1 completes.  No other row is written.  Each block is
+ * bitwise equal to the same row of nsa_compress over the whole cache.  Call it after
+ * appending token L-1 (for example before each nsa_decode); it is a no-op for the sequences
+ * not at a block boundary.  Status codes as for nsa_compress (seqlens must be 4-byte aligned).
+ */
+NSA_API nsa_status nsa_compress_append(const void* x_cache, const void* w, const int32_t* seqlens, int32_t B,
+                                       int32_t Lmax, int32_t H, int32_t d, int32_t d_out, int32_t l, int32_t s,
+                                       void* out_cache, int32_t ncmax, void* stream);
+
+/*
  * nsa_forward_noalloc -- nsa_forward for callers that cannot allocate device memory.
  * The pages have no counterpart: this is a library convenience, not part of the method.
  *

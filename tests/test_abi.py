@@ -149,3 +149,20 @@ def test_status_and_selftest_reject_bad_arguments(lib):
     assert lib.nsa_selftest_wait_timeout(fake + 2, 256, 1000, None) == nsa.NSA_ERR_INVALID_ARG    # misaligned
     assert lib.nsa_selftest_wait_timeout(fake, 256, 0, None) == nsa.NSA_ERR_INVALID_ARG           # no limit
     assert lib.nsa_selftest_wait_timeout(fake, 256, 1000001, None) == nsa.NSA_ERR_INVALID_ARG     # above 1 s
+
+
+def test_compress_append_rejects_bad_arguments(lib):
+    f = 0x10000   # never dereferenced: every call below fails its checks first
+    ok_args = dict(x=f, w=f, sl=f, B=2, L=64, H=1, d=64, dout=64, l=32, s=16, out=f, nc=3)
+
+    def call(**kw):
+        a = dict(ok_args, **kw)
+        return lib.nsa_compress_append(a["x"], a["w"], a["sl"], a["B"], a["L"], a["H"], a["d"], a["dout"], a["l"],
+                                       a["s"], a["out"], a["nc"], None)
+    assert call(x=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(sl=None) == nsa.NSA_ERR_INVALID_ARG
+    assert call(sl=f + 2) == nsa.NSA_ERR_INVALID_ARG      # seqlens misaligned
+    assert call(out=f + 8) == nsa.NSA_ERR_INVALID_ARG     # cache misaligned
+    assert call(nc=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(l=64) == nsa.NSA_ERR_UNSUPPORTED
+    assert call(d=96, dout=96) == nsa.NSA_ERR_UNSUPPORTED

@@ -98,6 +98,9 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st);
 // Past-block attention on tcgen05 (chunks of moba_past_tc_chunk() queries; block size a
 // multiple of 128).  max_chunks bounds the chunk count written to chunks[E] on the device.
 bool moba_past_tc_supported(const MobaArgs& a);
+// Own block + merge on tcgen05 (same support condition).
+cudaError_t launch_moba_own_tc(const MobaArgs& a, const int32_t* idx, const __nv_bfloat16* part_o,
+                               const float* part_lse, cudaStream_t st);
 int moba_past_tc_chunk();
 cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const int32_t* offsets,
                                 const int32_t* chunks, const int32_t* chunk_list, const int32_t* list,

@@ -574,9 +574,14 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  moba_own_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kAttnSmem, st>>>(
-      q, k, v, idx, part_o, part_lse, static_cast<__nv_bfloat16*>(a.out), a.T, a.H, a.bsz, a.top_k, a.scale_log2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (tc) {
+    e = launch_moba_own_tc(a, idx, part_o, part_lse, st);
+    if (e != cudaSuccess) return e;
+  } else {
+    moba_own_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kAttnSmem, st>>>(
+        q, k, v, idx, part_o, part_lse, static_cast<__nv_bfloat16*>(a.out), a.T, a.H, a.bsz, a.top_k, a.scale_log2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   if (a.mark) e = a.mark(a.mark_ctx, st);
   return e;
 }

@@ -40,6 +40,7 @@ constexpr uint32_t kSlice = kBlk * 128;           // 128 rows x 64 columns: 16 K
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256;        // S buffer b at 128b; O at 256
 constexpr float kSlack = 8.f;
+constexpr int kMaxPast = 8;                       // past-block slots per query (top_k <= 8)
 
 enum Err { kErrQ = 61, kErrKFull, kErrKEmpty, kErrVFull, kErrVEmpty, kErrSFull, kErrSEmpty, kErrPFull, kErrPEmpty,
            kErrOFull, kErrQEmpty, kErrOEmpty };
@@ -389,6 +390,348 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
 }
 }  // namespace
+
+namespace {
+// Own block + merge on tcgen05 ("逐篇讲解…" §16: every query also attends, causally, to the
+// block it sits in).  One CTA = 128 consecutive queries of one head (TMEM lane = query),
+// keys from the own block's start to the CTA's last query in 128-key tiles, masked to u <= t;
+// the same TMA / MMA / softmax roles and lazy reference as the past-block kernel.  Epilogue:
+// the own-block state (O unnormalised against the reference m, row sum l) merged with the
+// query's past-block partials by their log-sum-exps; out in bf16.
+__global__ void __launch_bounds__(kThreads, 1)
+moba_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,
+                   const __nv_bfloat16* __restrict__ part_o, const float* __restrict__ part_lse,
+                   __nv_bfloat16* __restrict__ out, int T, int H, int bsz, int top_k, float scale_log2,
+                   int* __restrict__ err) {
+  using SM = Smem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + SM::kQ;
+  uint8_t* sK = smem + SM::kK;
+  uint8_t* sV = smem + SM::kV;
+  uint8_t* sP = smem + SM::kP;
+  float* sPairMax = reinterpret_cast<float*>(smem + SM::kPair);            // [half][row]
+  int* sPairFlag = reinterpret_cast<int*>(sPairMax + 2 * kRowsM);           // [half][row]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+  uint64_t* bar_q = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + kKSlots;
+  uint64_t* v_full = k_empty + kKSlots;
+  uint64_t* v_empty = v_full + 2;
+  uint64_t* s_full = v_empty + 2;
+  uint64_t* s_empty = s_full + 2;
+  uint64_t* p_full = s_empty + 2;
+  uint64_t* p_empty = p_full + 1;
+  uint64_t* o_full = p_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int t0 = blockIdx.x * kRowsM, h = blockIdx.y, b = blockIdx.z;
+  const int J = t0 / bsz, u0 = J * bsz;            // the own block (bsz % 128 == 0)
+  const int t_last = min(T - 1, t0 + kRowsM - 1);
+  const int ntiles = (t_last - u0) / kBlk + 1;
+
+  if (tid == 0) {
+    tc::mbar_init(bar_q, 1);
+    for (int i = 0; i < kKSlots; ++i) {
+      tc::mbar_init(k_full + i, 1);
+      tc::mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(v_full + i, 1);
+      tc::mbar_init(v_empty + i, 1);
+      tc::mbar_init(s_full + i, 1);
+      tc::mbar_init(s_empty + i, kSoftWarps);
+    }
+    tc::mbar_init(p_full, kSoftWarps);
+    tc::mbar_init(p_empty, 1);
+    tc::mbar_init(o_full, 1);
+    tc::fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&tm_q);
+      tc::prefetch_tmap(&tm_k);
+      tc::prefetch_tmap(&tm_v);
+      tc::mbar_expect_tx(bar_q, 2 * kSlice);
+      for (int s = 0; s < 2; ++s) tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, h, b * T + t0);
+      int fill = 0;
+      bool ok = true;
+      for (int n = 0; n < ntiles && ok; ++n) {
+        const int row = b * T + u0 + n * kBlk;
+        for (int s = 0; s < 2 && ok; ++s, ++fill) {
+          const int slot = fill % kKSlots;
+          ok = tc::mbar_wait(k_empty + slot, ((fill / kKSlots) & 1) ^ 1, err, kErrKEmpty);
+          if (!ok) break;
+          tc::mbar_expect_tx(k_full + slot, kSlice);
+          tc::tma_load_3d(sK + slot * kSlice, &tm_k, k_full + slot, s * 64, h, row);
+        }
+        if (!ok) break;
+        const int vb = n & 1;
+        ok = tc::mbar_wait(v_empty + vb, ((n >> 1) & 1) ^ 1, err, kErrVEmpty);
+        if (!ok) break;
+        tc::mbar_expect_tx(v_full + vb, 2 * kSlice);
+        for (int s = 0; s < 2; ++s) tc::tma_load_3d(sV + (vb * 2 + s) * kSlice, &tm_v, v_full + vb, s * 64, h, row);
+      }
+      for (int i = 0; i < kKSlots && i < fill; ++i) {   // let the copies in flight land (bounded)
+        const int f = fill - 1 - i;
+        tc::mbar_wait(k_full + (f % kKSlots), (f / kKSlots) & 1, err, kErrKFull);
+      }
+      for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (tc::elect_one()) {
+      const uint32_t idS = tc::idesc_bf16(128, 128, 0, 0);
+      const uint32_t idPV = tc::idesc_bf16(128, D, 0, 1);
+      bool ok = tc::mbar_wait(bar_q, 0, err, kErrQ);
+      tc::tc_fence_after();
+      int fill = 0;
+      auto issue_s = [&](int n) -> bool {
+        const int sb = n & 1;
+        if (!tc::mbar_wait(s_empty + sb, ((n >> 1) & 1) ^ 1, err, kErrSEmpty)) return false;
+        tc::tc_fence_after();
+        for (int s = 0; s < 2; ++s, ++fill) {
+          const int slot = fill % kKSlots;
+          if (!tc::mbar_wait(k_full + slot, (fill / kKSlots) & 1, err, kErrKFull)) return false;
+          tc::tc_fence_after();
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t dq = tc::sdesc(sQ + s * kSlice + ks * 32, 16, 1024);
+            const uint64_t dk = tc::sdesc(sK + slot * kSlice + ks * 32, 16, 1024);
+            tc::mma_ss(tmem + kColS + 128 * sb, dq, dk, idS, (s | ks) != 0);
+          }
+          tc::mma_commit(k_empty + slot);
+        }
+        tc::mma_commit(s_full + sb);
+        return true;
+      };
+      auto issue_pv = [&](int n) -> bool {
+        if (!tc::mbar_wait(p_full, n & 1, err, kErrPFull) ||
+            !tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull))
+          return false;
+        tc::tc_fence_after();
+        const uint8_t* vb = sV + (n & 1) * 2 * kSlice;
+        for (int ks = 0; ks < kBlk / 16; ++ks) {
+          const uint64_t da = tc::sdesc(sP + (ks >> 2) * kSlice + (ks & 3) * 32, 16, 1024);
+          const uint64_t db = tc::sdesc(vb + ks * 16 * 128, kSlice, 1024);
+          tc::mma_ss(tmem + kColO, da, db, idPV, (n | ks) != 0);
+        }
+        tc::mma_commit(p_empty);
+        tc::mma_commit(v_empty + (n & 1));
+        return true;
+      };
+      if (ok && ntiles > 0) ok = issue_s(0);
+      for (int n = 0; n < ntiles && ok; ++n) {
+        if (n + 1 < ntiles) ok = issue_s(n + 1);
+        if (ok) ok = issue_pv(n);
+      }
+      if (ok && ntiles > 0) tc::mma_commit(o_full);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int gr = warp >> 2, q4 = warp & 3;       // key half, TMEM lane quadrant
+    const int r = 32 * q4 + lane;                  // this thread's query: token t0 + r
+    const int pbar = 1 + q4;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
+    const int t = t0 + r;
+    const bool row_ok = t < T;
+    const int my_hi = row_ok ? t : -1;             // keys [u0, my_hi]
+    // the past-block partials this query merges in: their slots and log-sum-exps, read now
+    const int32_t* irow = idx + (((size_t)b * H + h) * T + (row_ok ? t : 0)) * (top_k + 1);
+    float plse[kMaxPast];
+    int np = 0;
+#pragma unroll
+    for (int sl = 0; sl < kMaxPast; ++sl) {
+      const int jj = (row_ok && sl < top_k) ? irow[sl] : -1;
+      const bool in = jj >= 0 && jj < J && sl == np;
+      plse[sl] = in ? part_lse[(((size_t)b * T + t) * H + h) * top_k + sl] : -INFINITY;
+      np += in ? 1 : 0;
+    }
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int n = 0; n < ntiles; ++n) {
+      const int sb = n & 1;
+      ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_full + sb, (n >> 1) & 1, err, kErrSFull));
+      float v[64];
+      if (ok) {
+        tc::tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tc::tmem_ld16(lane_addr + kColS + 128 * sb + 64 * gr + 16 * cc, *reinterpret_cast<float(*)[16]>(v + 16 * cc));
+        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(s_empty + sb);
+      }
+      const int i0 = u0 + n * kBlk + 64 * gr;     // first key of this thread's half
+      if (i0 + 63 <= my_hi) {
+#pragma unroll
+        for (int jj = 0; jj < 64; ++jj) v[jj] *= scale_log2;
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 64; ++jj) v[jj] = i0 + jj <= my_hi ? v[jj] * scale_log2 : -INFINITY;
+      }
+      float cmx[8];
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) cmx[cc] = fmaxf(fmaxf(v[cc], v[cc + 8]), fmaxf(v[cc + 16], v[cc + 24]));
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        cmx[cc] = fmaxf(cmx[cc], fmaxf(fmaxf(v[cc + 32], v[cc + 40]), fmaxf(v[cc + 48], v[cc + 56])));
+      const float lmax = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                               fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+      if (tc::vote_any(pbar, 64, !ok || lmax > m + kSlack)) {
+        sPairMax[gr * kRowsM + r] = lmax;
+        sPairFlag[gr * kRowsM + r] = ok;
+        tc::named_sync(pbar, 64);
+        const bool pair_ok = __all_sync(0xffffffffu, sPairFlag[r] && sPairFlag[kRowsM + r]);
+        if (!pair_ok) {
+          ok = false;
+          break;
+        }
+        const float mn = fmaxf(m, fmaxf(sPairMax[r], sPairMax[kRowsM + r]));
+        const float cf = mn == -INFINITY ? 1.f : ex2(m - mn);
+        l *= cf;
+        if (__any_sync(0xffffffffu, cf != 1.f) && n > 0) {
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty));
+          if (ok) {
+            tc::tc_fence_after();
+#pragma unroll
+            for (int qq = 0; qq < D / 2 / 16; ++qq) {
+              float o[16];
+              const uint32_t addr = lane_addr + kColO + (D / 2) * gr + 16 * qq;
+              tc::tmem_ld16(addr, o);
+              tc::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) o[i] *= cf;
+              tc::tmem_st16(addr, o);
+            }
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+          }
+        }
+        m = mn;
+        tc::named_sync(pbar, 64);
+      }
+      const float base = m == -INFINITY ? 0.f : m;
+      uint32_t pk[32];
+      float ps[8];
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) ps[cc] = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < 64; jj += 2) {
+        const float p0 = ex2(v[jj] - base), p1 = ex2(v[jj + 1] - base);
+        ps[(jj >> 1) & 7] += p0 + p1;
+        pk[jj / 2] = pack_bf16(p0, p1);
+      }
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      if (n > 0) ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(p_empty, (n - 1) & 1, err, kErrPEmpty));
+      uint8_t* prow = sP + gr * kSlice + r * 128;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+      tc::fence_async_smem();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(p_full);
+    }
+    // epilogue: the own block's (m, L, O) merged with the past partials
+    sPairMax[gr * kRowsM + r] = l;
+    sPairFlag[gr * kRowsM + r] = ok;
+    tc::named_sync(pbar, 64);
+    const bool pair_ok = sPairFlag[r] && sPairFlag[kRowsM + r];
+    const float L = sPairMax[r] + sPairMax[kRowsM + r];
+    ok = __all_sync(0xffffffffu, pair_ok && (ntiles == 0 || tc::mbar_wait(o_full, 0, err, kErrOFull)));
+    if (ok) {
+      tc::tc_fence_after();
+      float M = m + __log2f(L);                      // the own block's log-sum-exp (L >= 1: key t is visible)
+#pragma unroll
+      for (int sl = 0; sl < kMaxPast; ++sl) M = fmaxf(M, plse[sl]);
+      const float w_own = ex2(m - M);               // multiplies the unnormalised O (row sum L)
+      float wsum = L * w_own;
+      float ws[kMaxPast];
+#pragma unroll
+      for (int sl = 0; sl < kMaxPast; ++sl) {
+        ws[sl] = sl < np ? ex2(plse[sl] - M) : 0.f;
+        wsum += ws[sl];
+      }
+      const float inv = row_ok && wsum > 0.f ? 1.f / wsum : 0.f;
+      const size_t qrow = ((size_t)b * T + (row_ok ? t : 0)) * H + h;
+      const __nv_bfloat16* po = part_o + qrow * top_k * D + (D / 2) * gr;
+      __nv_bfloat16* orow = out + qrow * D + (D / 2) * gr;
+#pragma unroll
+      for (int qq = 0; qq < D / 2 / 16; ++qq) {
+        float o[16];
+        tc::tmem_ld16(lane_addr + kColO + (D / 2) * gr + 16 * qq, o);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) o[i] *= w_own;
+#pragma unroll
+        for (int sl = 0; sl < kMaxPast; ++sl) {
+          if (sl < np) {
+            const uint4* src = reinterpret_cast<const uint4*>(po + sl * D + 16 * qq);
+            const uint4 a0 = src[0], a1 = src[1];
+            const uint32_t wv[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv[i]));
+              o[2 * i] += ws[sl] * f.x;
+              o[2 * i + 1] += ws[sl] * f.y;
+            }
+          }
+        }
+        if (row_ok) {
+          uint32_t w[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = pack_bf16(o[2 * i] * inv, o[2 * i + 1] * inv);
+          *reinterpret_cast<uint4*>(orow + 16 * qq) = make_uint4(w[0], w[1], w[2], w[3]);
+          *reinterpret_cast<uint4*>(orow + 16 * qq + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+      }
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+}  // namespace
+
+cudaError_t launch_moba_own_tc(const MobaArgs& a, const int32_t* idx, const __nv_bfloat16* part_o,
+                               const float* part_lse, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(moba_own_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Smem::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap mq, mk, mv;
+  const uint64_t d3[3] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)a.B * a.T};
+  const uint64_t s3[2] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2};
+  const uint32_t box[3] = {64, 1, (uint32_t)kBlk};
+  if (!make_tmap_bf16(&mq, a.q, 3, d3, s3, box) || !make_tmap_bf16(&mk, a.k, 3, d3, s3, box) ||
+      !make_tmap_bf16(&mv, a.v, 3, d3, s3, box))
+    return cudaErrorInvalidValue;
+  dim3 grid((a.T + kRowsM - 1) / kRowsM, a.H, a.B);
+  moba_own_tc_kernel<<<grid, kThreads, Smem::kAlloc, st>>>(mq, mk, mv, idx, part_o, part_lse,
+                                                            static_cast<__nv_bfloat16*>(a.out), a.T, a.H, a.bsz,
+                                                            a.top_k, a.scale_log2, a.err);
+  return cudaGetLastError();
+}
 
 bool moba_past_tc_supported(const MobaArgs& a) {
   return a.err != nullptr && a.bsz % kBlk == 0 && a.top_k > 0 && a.top_k <= 8;

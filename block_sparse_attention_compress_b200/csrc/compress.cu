@@ -20,7 +20,7 @@ constexpr int kBM = 64, kBN = 64, kBK = 64, kThreads = 128;
 
 // STAGES-deep cp.async ring of (A, W) k-chunks: 2 when the grid is large enough to hide the
 // loads' latency; more for the append launch, whose few CTAs each run one long k chain.
-template <int D, int DOUT, int STAGES>
+template <int D, int DOUT, int STAGES, bool APPEND>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
                 int l, int s, int nc, __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ seqlens,
@@ -28,14 +28,14 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   extern __shared__ __align__(128) uint8_t csmem[];
   auto sA = reinterpret_cast<__nv_bfloat16(*)[kBM * kBK]>(csmem);                          // [STAGES]
   auto sB = reinterpret_cast<__nv_bfloat16(*)[kBK * kBN]>(csmem + STAGES * kBM * kBK * 2);  // [STAGES]
-  __shared__ int sWin[kBM];   // append mode: the window of each row's sequence, or -1
+  __shared__ int sWin[APPEND ? kBM : 1];   // append mode: the window of each row's sequence, or -1
   using Swz = SwzTile<kBK>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int i0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
-  const bool app = seqlens != nullptr;
+  constexpr bool app = APPEND;
   const int bh = blockIdx.z, b = app ? 0 : bh / H, h = app ? bh : bh % H;
   const int nk = l * D / kBK;
-  if (app) {
+  if constexpr (APPEND) {
     if (tid < kBM) {
       const int bb = i0 + tid;
       const int L = bb < B ? min(seqlens[bb], T) : 0;
@@ -125,7 +125,7 @@ template <int D>
 cudaError_t launch(const void* x, const void* w, int B, int T, int H, int l, int s, int nc, void* out,
                    cudaStream_t st) {
   dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
-  compress_kernel<D, D, 2><<<grid, kThreads, smem_bytes(2), st>>>(static_cast<const __nv_bfloat16*>(x),
+  compress_kernel<D, D, 2, false><<<grid, kThreads, smem_bytes(2), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w), T, H, l, s, nc,
                                                    static_cast<__nv_bfloat16*>(out), nullptr, B);
   return cudaGetLastError();
@@ -137,13 +137,13 @@ cudaError_t launch_append(const void* x, const void* w, const int32_t* seqlens, 
   constexpr int kStages = 8;
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(compress_kernel<D, D, kStages>,
+    const cudaError_t e = cudaFuncSetAttribute(compress_kernel<D, D, kStages, true>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
     if (e != cudaSuccess) return e;
     attr = true;
   }
   dim3 grid((B + kBM - 1) / kBM, D / kBN, H);
-  compress_kernel<D, D, kStages><<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
+  compress_kernel<D, D, kStages, true><<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w), Lmax, H, l, s, ncmax,
                                                    static_cast<__nv_bfloat16*>(out), seqlens, B);
   return cudaGetLastError();

@@ -211,9 +211,9 @@ def workload_config(c, name):
 # compressed cache stay mostly in L2.  An entry goes back to None whenever its kernel
 # changes, until it is captured again.
 NCU_DRAM_BYTES_PER_ITEM = {
-    "cmp_select": (205.900800e6 + 217.100032e6) / 32768,
-    "slc_attn": (501.110528e6 + 232.153088e6) / 32768,
-    "swa_combine": (499.490048e6 + 117.897984e6) / 32768,
+    "cmp_select": (205.901056e6 + 216.682752e6) / 32768,
+    "slc_attn": (501.055744e6 + 230.477568e6) / 32768,
+    "swa_combine": (499.454208e6 + 117.621248e6) / 32768,
 }
 
 

@@ -132,31 +132,58 @@ __global__ void __launch_bounds__(D) moba_mean_kernel(const __nv_bfloat16* __res
 }
 
 // ------------------------------------------------------------------ M2
-// Keeps the k best (score desc, index asc) of the values offered to it.
+// Keeps the KK best (score desc, index asc) of the values offered to it, sorted best-first,
+// entirely in registers: every slot index is a compile-time constant.  The KK-th best is kept
+// apart as (tv, tj), so most offers cost one comparison.
+template <int KK>
 struct TopK {
-  float v[kMaxK];
-  int j[kMaxK];
-  __device__ void init() {
+  static constexpr int N = KK > 0 ? KK : 1;
+  float v[N];
+  int j[N];
+  float tv;
+  int tj;
+  __device__ __forceinline__ void init() {
 #pragma unroll
-    for (int i = 0; i < kMaxK; ++i) { v[i] = -FLT_MAX; j[i] = 0x7fffffff; }
+    for (int i = 0; i < N; ++i) { v[i] = -FLT_MAX; j[i] = 0x7fffffff; }
+    tv = -FLT_MAX;
+    tj = 0x7fffffff;
   }
-  __device__ static bool better(float a, int ja, float b, int jb) { return a > b || (a == b && ja < jb); }
-  __device__ void offer(float val, int idx, int k) {   // list sorted best-first in [0, k), 1 <= k <= kMaxK
-    if (!better(val, idx, v[k - 1], j[k - 1])) return;
-    int p = k - 1;
-    while (p > 0 && better(val, idx, v[p - 1], j[p - 1])) {
-      v[p] = v[p - 1];
-      j[p] = j[p - 1];
-      --p;
+  __device__ __forceinline__ static bool better(float a, int ja, float b, int jb) {
+    return a > b || (a == b && ja < jb);
+  }
+  __device__ __forceinline__ void offer(float val, int idx) {
+    if (!better(val, idx, tv, tj)) return;
+    float cv = val;
+    int cj = idx;
+#pragma unroll
+    for (int i = 0; i < N; ++i) {   // insertion by swapping down the sorted slots
+      if (better(cv, cj, v[i], j[i])) {
+        const float xv = v[i];
+        const int xj = j[i];
+        v[i] = cv;
+        j[i] = cj;
+        cv = xv;
+        cj = xj;
+      }
     }
-    v[p] = val;
-    j[p] = idx;
+    tv = v[N - 1];
+    tj = j[N - 1];
+  }
+  __device__ __forceinline__ void pop() {   // drop the best slot
+#pragma unroll
+    for (int i = 0; i + 1 < N; ++i) { v[i] = v[i + 1]; j[i] = j[i + 1]; }
+    v[N - 1] = -FLT_MAX;
+    j[N - 1] = 0x7fffffff;
   }
 };
 
+// One instantiation per top_k (0 .. kMaxK), so that the per-thread candidate lists and the
+// merged selections live in registers.
+template <int KK>
 __global__ void __launch_bounds__(kThreads) moba_select_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kbar, int32_t* __restrict__ idx,
-    int32_t* __restrict__ counts, int B, int T, int H, int bsz, int nblk, int top_k) {
+    int32_t* __restrict__ counts, int B, int T, int H, int bsz, int nblk) {
+  constexpr int N = TopK<KK>::N;
   extern __shared__ __align__(128) uint8_t smem[];
   __nv_bfloat16* sHi = reinterpret_cast<__nv_bfloat16*>(smem);          // [2][kKT][D]
   __nv_bfloat16* sLo = sHi + 2 * kKT * D;                               // [2][kKT][D]
@@ -165,14 +192,14 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
   const int J = t0 / bsz;                      // own block, the same for the whole tile (bsz % 64 == 0)
   const int ta = t0 + warp * 16 + gl, tb = ta + 8;
   const size_t lo_off = (size_t)B * nblk * H * D;
-  uint32_t qf[D / 16][4];
-  load_q_frag(qf, q + (((size_t)b * T + min(ta, T - 1)) * H + h) * D, q + (((size_t)b * T + min(tb, T - 1)) * H + h) * D,
-              ta < T, tb < T, cq);
-  TopK k0, k1;
+  const bool choose = KK > 0 && J > KK;        // else every past block is taken
+  TopK<KK> k0, k1;
   k0.init();
   k1.init();
-  const int kk = min(top_k, J);
-  if (J > top_k && top_k > 0) {
+  if (choose) {
+    uint32_t qf[D / 16][4];
+    load_q_frag(qf, q + (((size_t)b * T + min(ta, T - 1)) * H + h) * D,
+                q + (((size_t)b * T + min(tb, T - 1)) * H + h) * D, ta < T, tb < T, cq);
     auto load = [&](int j0, int buf) {   // blocks j0 .. j0+63 (zeros past J)
       for (int e = tid; e < kKT * (D / 8); e += kThreads) {
         const int r = e / (D / 8), ch = e % (D / 8);
@@ -200,54 +227,63 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
         for (int e = 0; e < 2; ++e) {
           const int j = j0 + nt * 8 + 2 * cq + e;
           if (j < J) {
-            k0.offer(s[nt][e], j, kk);
-            k1.offer(s[nt][2 + e], j, kk);
+            k0.offer(s[nt][e], j);
+            k1.offer(s[nt][2 + e], j);
           }
         }
       __syncthreads();   // this buffer is refilled two tiles later
     }
     cp_async_wait<0>();
   }
-  // merge the quad's four lists: kk rounds of a quad-wide argmax
-  int sel0[kMaxK + 1], sel1[kMaxK + 1];
-  if (J <= top_k) {
-    for (int i = 0; i < kk; ++i) sel0[i] = sel1[i] = i;
-  } else if (kk > 0) {
-    int p0 = 0, p1 = 0;
-    for (int r = 0; r < kk; ++r) {
-      float bv0 = p0 < kk ? k0.v[p0] : -FLT_MAX, bv1 = p1 < kk ? k1.v[p1] : -FLT_MAX;
-      int bj0 = p0 < kk ? k0.j[p0] : 0x7fffffff, bj1 = p1 < kk ? k1.j[p1] : 0x7fffffff;
+  // merge the quad's four lists: KK rounds of a quad-wide argmax over the lists' heads
+  int sel0[N], sel1[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) sel0[i] = sel1[i] = i;
+  if (choose) {
+#pragma unroll
+    for (int r = 0; r < N; ++r) {
+      float bv0 = k0.v[0], bv1 = k1.v[0];
+      int bj0 = k0.j[0], bj1 = k1.j[0];
 #pragma unroll
       for (int off = 1; off < 4; off <<= 1) {
         const float ov0 = __shfl_xor_sync(0xffffffffu, bv0, off), ov1 = __shfl_xor_sync(0xffffffffu, bv1, off);
         const int oj0 = __shfl_xor_sync(0xffffffffu, bj0, off), oj1 = __shfl_xor_sync(0xffffffffu, bj1, off);
-        if (TopK::better(ov0, oj0, bv0, bj0)) { bv0 = ov0; bj0 = oj0; }
-        if (TopK::better(ov1, oj1, bv1, bj1)) { bv1 = ov1; bj1 = oj1; }
+        if (TopK<KK>::better(ov0, oj0, bv0, bj0)) { bv0 = ov0; bj0 = oj0; }
+        if (TopK<KK>::better(ov1, oj1, bv1, bj1)) { bv1 = ov1; bj1 = oj1; }
       }
       sel0[r] = bj0;
       sel1[r] = bj1;
-      if (p0 < kk && k0.j[p0] == bj0) ++p0;   // indices are unique across the quad's lanes
-      if (p1 < kk && k1.j[p1] == bj1) ++p1;
+      if (k0.j[0] == bj0) k0.pop();   // indices are unique across the quad's lanes
+      if (k1.j[0] == bj1) k1.pop();
     }
+    // ascending block order: odd-even transposition sort over the N slots
+#pragma unroll
+    for (int pass = 0; pass < N; ++pass)
+#pragma unroll
+      for (int i = pass & 1; i + 1 < N; i += 2) {
+        if (sel0[i] > sel0[i + 1]) { const int x = sel0[i]; sel0[i] = sel0[i + 1]; sel0[i + 1] = x; }
+        if (sel1[i] > sel1[i + 1]) { const int x = sel1[i]; sel1[i] = sel1[i + 1]; sel1[i + 1] = x; }
+      }
   }
-  // ascending order (kk <= 7)
-  for (int a = 1; a < kk; ++a)
-    for (int c = a; c > 0 && sel0[c - 1] > sel0[c]; --c) { const int x = sel0[c]; sel0[c] = sel0[c - 1]; sel0[c - 1] = x; }
-  for (int a = 1; a < kk; ++a)
-    for (int c = a; c > 0 && sel1[c - 1] > sel1[c]; --c) { const int x = sel1[c]; sel1[c] = sel1[c - 1]; sel1[c - 1] = x; }
   if (cq == 0) {
+    const int kk = min(KK, J);
+    int32_t* cnt = counts + ((size_t)b * H + h) * nblk;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int t = half ? tb : ta;
       if (t >= T) continue;
-      const int* sel = half ? sel1 : sel0;
-      int32_t* dst = idx + (((size_t)b * H + h) * T + t) * (top_k + 1);
-      for (int i = 0; i < kk; ++i) {
-        dst[i] = sel[i];
-        atomicAdd(&counts[((size_t)b * H + h) * nblk + sel[i]], 1);
+      int32_t* dst = idx + (((size_t)b * H + h) * T + t) * (KK + 1);
+#pragma unroll
+      for (int i = 0; i < KK; ++i) {
+        if (i < kk) {
+          const int sj = half ? sel1[i] : sel0[i];
+          dst[i] = sj;
+          atomicAdd(cnt + sj, 1);
+        } else {
+          dst[i + 1] = -1;
+        }
       }
       dst[kk] = J;
-      for (int i = kk + 1; i <= top_k; ++i) dst[i] = -1;
     }
   }
 }
@@ -513,14 +549,27 @@ MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k) {
   return L;
 }
 
+template <int KK>
+static cudaError_t launch_select(const MobaArgs& a, const __nv_bfloat16* q, const __nv_bfloat16* kbar, int32_t* idx,
+                                 int32_t* counts, int nblk, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(moba_select_kernel<KK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelectSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  moba_select_kernel<KK><<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kSelectSmem, st>>>(q, kbar, idx, counts, a.B,
+                                                                                            a.T, a.H, a.bsz, nblk);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(moba_past_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moba_own_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(moba_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelectSmem);
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -548,9 +597,18 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   moba_mean_kernel<<<dim3(nblk, a.H, a.B), D, 0, st>>>(k, kbar, a.B, a.T, a.H, a.bsz, nblk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  moba_select_kernel<<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kSelectSmem, st>>>(
-      q, kbar, idx, counts, a.B, a.T, a.H, a.bsz, nblk, a.top_k);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  switch (a.top_k) {
+    case 0: e = launch_select<0>(a, q, kbar, idx, counts, nblk, st); break;
+    case 1: e = launch_select<1>(a, q, kbar, idx, counts, nblk, st); break;
+    case 2: e = launch_select<2>(a, q, kbar, idx, counts, nblk, st); break;
+    case 3: e = launch_select<3>(a, q, kbar, idx, counts, nblk, st); break;
+    case 4: e = launch_select<4>(a, q, kbar, idx, counts, nblk, st); break;
+    case 5: e = launch_select<5>(a, q, kbar, idx, counts, nblk, st); break;
+    case 6: e = launch_select<6>(a, q, kbar, idx, counts, nblk, st); break;
+    case 7: e = launch_select<7>(a, q, kbar, idx, counts, nblk, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
   const int cq = tc ? moba_past_tc_chunk() : kQ;   // queries per past-attention chunk
   moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, chunk_list, E, cq);

@@ -71,6 +71,7 @@ struct Smem {
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;                         // room to align the base to 1 KB
   static_assert(kAlloc <= 232448, "shared memory");
+  static_assert(kLse % 16 == 0, "the log-sum-exp row is read as float4");
 };
 
 
@@ -443,15 +444,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(s_empty + sb);
-          // masked, scaled scores; only a tile that straddles this row's range needs the
-          // per-element test.  Max and sum use eight independent chains each.
+          // masked scores; only a tile that straddles this row's range needs the per-element
+          // test.  The maximum is taken on the raw scores (the scale is positive, and rounding
+          // x * scale is monotone, so it equals the maximum of the scaled ones) and the scale
+          // is applied inside the exponent's FMA.  Max and sum use eight independent chains each.
           const int i0 = n * kBlk + col0;
-          if (i0 + kCols - 1 < my_hi) {
+          if (i0 + kCols - 1 >= my_hi) {
 #pragma unroll
-            for (int j = 0; j < kCols; ++j) v[j] *= scale_log2;
-          } else {
-#pragma unroll
-            for (int j = 0; j < kCols; ++j) v[j] = i0 + j < my_hi ? v[j] * scale_log2 : -INFINITY;
+            for (int j = 0; j < kCols; ++j) v[j] = i0 + j < my_hi ? v[j] : -INFINITY;
           }
           float cmx[8];
 #pragma unroll
@@ -459,14 +459,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int j = 8; j < kCols; ++j) cmx[j & 7] = fmaxf(cmx[j & 7], v[j]);
           const float cm = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
-                                 fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+                                 fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7]))) * scale_log2;
           const float mn = fmaxf(m, cm);
           if (mn != -INFINITY) {
             float ps[8];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) ps[c] = ex2(v[c] - mn);
+            for (int c = 0; c < 8; ++c) ps[c] = ex2(fmaf(v[c], scale_log2, -mn));
 #pragma unroll
-            for (int j = 8; j < kCols; ++j) ps[j & 7] += ex2(v[j] - mn);
+            for (int j = 8; j < kCols; ++j) ps[j & 7] += ex2(fmaf(v[j], scale_log2, -mn));
             const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
             l = l * ex2(m - mn) + sum;
             m = mn;
@@ -544,12 +544,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const bool vis = i < hi_tok[kk];
           float sacc = 0.f;
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const float p0 = vis ? ex2(v[16 * kk + j] * scale_log2 - sLse[col0 + 16 * kk + j]) : 0.f;
-            const float p1 = vis ? ex2(v[16 * kk + j + 1] * scale_log2 - sLse[col0 + 16 * kk + j + 1]) : 0.f;
-            sacc += p0 + p1;
+          for (int j = 0; j < 16; j += 4) {
+            // the log-sum-exp of four columns in one broadcast load
+            const float4 ls = *reinterpret_cast<const float4*>(sLse + col0 + 16 * kk + j);
+            const float p0 = vis ? ex2(fmaf(v[16 * kk + j], scale_log2, -ls.x)) : 0.f;
+            const float p1 = vis ? ex2(fmaf(v[16 * kk + j + 1], scale_log2, -ls.y)) : 0.f;
+            const float p2 = vis ? ex2(fmaf(v[16 * kk + j + 2], scale_log2, -ls.z)) : 0.f;
+            const float p3 = vis ? ex2(fmaf(v[16 * kk + j + 3], scale_log2, -ls.w)) : 0.f;
+            sacc += (p0 + p1) + (p2 + p3);
             __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
             pk[8 * kk + j / 2] = *reinterpret_cast<uint32_t*>(&h2);
+            h2 = __floats2bfloat162_rn(p2, p3);
+            pk[8 * kk + j / 2 + 1] = *reinterpret_cast<uint32_t*>(&h2);
           }
           tok_sum[kk] = sacc;
         }

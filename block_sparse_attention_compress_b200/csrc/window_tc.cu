@@ -234,12 +234,11 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0) tc::mbar_arrive(s_empty + sb);
       }
       const int i0 = kv_lo + n * kBlk + 64 * gr;     // first key of this thread's half
-      if (i0 >= my_lo && i0 + 63 <= my_hi) {
+      // masked raw scores: the scale (positive) is applied to the maximum and inside the
+      // exponent's FMA (rounding x * scale is monotone, so the maxima agree)
+      if (!(i0 >= my_lo && i0 + 63 <= my_hi)) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] *= scale_log2;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 64; ++j) v[j] = (i0 + j >= my_lo && i0 + j <= my_hi) ? v[j] * scale_log2 : -INFINITY;
+        for (int j = 0; j < 64; ++j) v[j] = (i0 + j >= my_lo && i0 + j <= my_hi) ? v[j] : -INFINITY;
       }
       float cmx[8];
 #pragma unroll
@@ -247,7 +246,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
       for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
       const float lmax = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
-                               fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7])));
+                               fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7]))) * scale_log2;
       // the two threads of a row agree on its reference; a failed wait also takes the
       // exchange, so that both warps of the pair leave together
       if (tc::vote_any(pbar, 64, !ok || lmax > m + kSlack)) {
@@ -291,7 +290,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int c = 0; c < 8; ++c) ps[c] = 0.f;
 #pragma unroll
       for (int j = 0; j < 64; j += 2) {
-        const float p0 = ex2(v[j] - base), p1 = ex2(v[j + 1] - base);
+        const float p0 = ex2(fmaf(v[j], scale_log2, -base)), p1 = ex2(fmaf(v[j + 1], scale_log2, -base));
         ps[(j >> 1) & 7] += p0 + p1;
         pk[j / 2] = pack_bf16(p0, p1);
       }

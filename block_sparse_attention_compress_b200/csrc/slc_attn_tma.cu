@@ -16,6 +16,10 @@
 // directly and the item ends without merging partial outputs.  The ring runs across
 // item boundaries, so the loads of the next token overlap the end of this one.
 //
+// The producer also brings each item's queries (the group's 16 head rows, 128-byte
+// swizzled boxes) into a 2-slot buffer by TMA; the consumer warps take their MMA operand
+// fragments from there with ldmatrix, once per item.
+//
 // Slot release: the consumers read a slot with ldmatrix (generic proxy) and the
 // producer refills it with TMA (async proxy).  A proxy fence before each release
 // orders the reads before the refill; without it a refill was seen to overwrite the
@@ -42,18 +46,20 @@ template <int DK, int DV>
 struct Smem {
   static constexpr uint32_t kSlotBytes = (DK / 64 + DV / 64) * kBox;
   static constexpr uint32_t kRing = 0;                                       // [group][slot]
+  static constexpr uint32_t kQBytes = (DK / 64) * 16 * 128;                 // queries: 16 rows, DK/64 boxes
+  static constexpr uint32_t kQ = kRing + kGroups * kSlots * kSlotBytes;      // [group][2]
   static constexpr uint32_t kPBytes = 16 * 128;                              // P [16 heads][64 keys] bf16
-  static constexpr uint32_t kP = kRing + kGroups * kSlots * kSlotBytes;      // [group][2]
+  static constexpr uint32_t kP = kQ + kGroups * 2 * kQBytes;                 // [group][2]
   static constexpr int kConsumers = consumers<DV>();
   static constexpr uint32_t kRedBytes = 2 * kConsumers * 16 * 4 + kConsumers * 4;   // [group]: maxima, sums [warp][16], flags
   static constexpr uint32_t kRed = kP + kGroups * 2 * kPBytes;
   static constexpr uint32_t kBar = kRed + kGroups * kRedBytes;
-  static constexpr uint32_t kBytes = kBar + kGroups * 2 * kSlots * 8;
+  static constexpr int kBarsPerGroup = 2 * kSlots + 4;                       // full, empty, q_full, q_empty
+  static constexpr uint32_t kBytes = kBar + kGroups * kBarsPerGroup * 8;
   static constexpr uint32_t kAlloc = kBytes + 1024;
   static_assert(kAlloc * kCtasPerSm <= 232448, "shared memory");
+  static_assert(kQ % 1024 == 0 && kQBytes % 1024 == 0, "swizzled query boxes need 1 KB alignment");
 };
-
-__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
 using tc::named_sync;
 using tc::vote_all;
@@ -64,9 +70,9 @@ __device__ __forceinline__ uint32_t swz(int row, int c) { return row * 128 + ((c
 template <int DK, int DV>
 __global__ void __launch_bounds__(threads<DV>(), kCtasPerSm)
 slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gates,
+                    const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gates,
                     const int32_t* __restrict__ idx, float* __restrict__ acc, int B, int T, int Hq, int Hkv, int G,
-                    int top_k, float scale_log2, int* __restrict__ err) {
+                    int top_k, float scale_log2, int q_rows, int* __restrict__ err) {
   using SM = Smem<DK, DV>;
   constexpr int kConsumers = SM::kConsumers;
   constexpr int kKW = kBlk / kConsumers;            // keys per consumer warp: 16 or 8
@@ -75,16 +81,25 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool producer = warp >= kGroups * kConsumers;
   const int grp = producer ? warp - kGroups * kConsumers : warp / kConsumers;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar) + grp * 2 * kSlots;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::kBar) + grp * SM::kBarsPerGroup;
   uint64_t* empty = full + kSlots;
+  uint64_t* q_full = empty + kSlots;   // [2]
+  uint64_t* q_empty = q_full + 2;      // [2]
   uint8_t* ring = smem + SM::kRing + grp * kSlots * SM::kSlotBytes;
+  uint8_t* qbuf = smem + SM::kQ + grp * 2 * SM::kQBytes;
   if (tid == 0) {
     uint64_t* all = reinterpret_cast<uint64_t*>(smem + SM::kBar);
-    for (int gg = 0; gg < kGroups; ++gg)
+    for (int gg = 0; gg < kGroups; ++gg) {
+      uint64_t* b0 = all + gg * SM::kBarsPerGroup;
       for (int s = 0; s < kSlots; ++s) {
-        tc::mbar_init(all + gg * 2 * kSlots + s, 1);
-        tc::mbar_init(all + gg * 2 * kSlots + kSlots + s, kConsumers);
+        tc::mbar_init(b0 + s, 1);
+        tc::mbar_init(b0 + kSlots + s, kConsumers);
       }
+      for (int s = 0; s < 2; ++s) {
+        tc::mbar_init(b0 + 2 * kSlots + s, 1);
+        tc::mbar_init(b0 + 2 * kSlots + 2 + s, kConsumers);
+      }
+    }
     tc::fence_barrier_init();
   }
   __syncthreads();
@@ -97,13 +112,29 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     if (lane == 0) {
       tc::prefetch_tmap(&tm_k);
       tc::prefetch_tmap(&tm_v);
+      tc::prefetch_tmap(&tm_q);
     }
-    long fill = 0;
+    long fill = 0, qfill = 0;
     bool ok = true;
-    for (long it = it0; it < total && ok; it += stride) {
+    for (long it = it0; it < total && ok; it += stride, ++qfill) {
       const int g = (int)(it / ((long)B * T));
       const int bt = (int)(it % ((long)B * T));
       const int b = bt / T, t = bt % T;
+      // this item's queries: rows g*G .. g*G+q_rows-1 of token (b, t) (q_rows = min(16, Hq);
+      // rows past the group are masked by the consumers, rows past the last head are
+      // zero-filled by TMA)
+      {
+        const int qs = (int)(qfill & 1);
+        ok = tc::mbar_wait(q_empty + qs, (uint32_t)(((qfill >> 1) & 1) ^ 1), err, 24);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0) {
+          tc::mbar_expect_tx(q_full + qs, (uint32_t)((DK / 64) * q_rows * 128));
+          for (int s = 0; s < DK / 64; ++s)
+            tc::tma_load_3d(qbuf + qs * SM::kQBytes + s * 16 * 128, &tm_q, q_full + qs, s * 64, g * G, b * T + t);
+        }
+        __syncwarp();
+      }
       const int mine = lane < top_k ? idx[(((size_t)b * Hkv + g) * T + t) * top_k + lane] : -1;
       for (int jj = 0; jj < top_k && ok; ++jj) {
         const int j = __shfl_sync(0xffffffffu, mine, jj);
@@ -125,9 +156,12 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         ++fill;
       }
     }
-    if (lane == 0)
-      for (long f = fill - 1; f >= 0 && f >= fill - kSlots; --f)   // let copies in flight land
+    if (lane == 0) {   // let copies in flight land
+      for (long f = fill - 1; f >= 0 && f >= fill - kSlots; --f)
         tc::mbar_wait(full + (f % kSlots), (uint32_t)((f / kSlots) & 1), err, 22);
+      for (long f = qfill - 1; f >= 0 && f >= qfill - 2; --f)   // qfill = query copies issued
+        tc::mbar_wait(q_full + (f & 1), (uint32_t)((f >> 1) & 1), err, 25);
+    }
   } else {
     // ---------------------------------------------------------------- consumers
     // Warp cw computes the scores of keys 16cw..16cw+15 of every block and, from the whole
@@ -140,25 +174,35 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     float* sMx = reinterpret_cast<float*>(smem + SM::kRed + grp * SM::kRedBytes);   // [warp][row] block maxima
     float* sL = sMx + kConsumers * 16;                                                // [warp][row] row sums
     int* sFlag = reinterpret_cast<int*>(sL + kConsumers * 16);                      // [warp] no wait failed
-    long use = 0;
+    long use = 0, quse = 0;
     bool ok = true;
-    for (long it = it0; it < total && ok; it += stride) {
+    for (long it = it0; it < total && ok; it += stride, ++quse) {
       const int g = (int)(it / ((long)B * T));
       const int bt = (int)(it % ((long)B * T));
       const int b = bt / T, t = bt % T;
       const int mine = lane < top_k ? idx[(((size_t)b * Hkv + g) * T + t) * top_k + lane] : -1;
       const bool rv0 = gl < G, rv1 = gl + 8 < G;
+      // the item's query fragments (A operand of the q.k MMAs), from the swizzled boxes;
+      // rows past the group are zeroed.  A failed wait is carried in ok into the block
+      // loop's exchange, so that the group's warps leave together.
       uint32_t qf[DK / 16][4];
       {
-        const __nv_bfloat16* q0 = q + (((size_t)b * T + t) * Hq + g * G + gl) * DK;
-        const __nv_bfloat16* q1 = q0 + 8 * DK;
+        const int qs = (int)(quse & 1);
+        ok = tc::mbar_wait(q_full + qs, (uint32_t)((quse >> 1) & 1), err, 26);
+        ok = __all_sync(0xffffffffu, ok);
+        const uint8_t* qb = qbuf + qs * SM::kQBytes;
+        const int row = lane & 15;
 #pragma unroll
         for (int ks = 0; ks < DK / 16; ++ks) {
-          qf[ks][0] = rv0 ? ld_u32(q0 + ks * 16 + 2 * cq) : 0u;
-          qf[ks][1] = rv1 ? ld_u32(q1 + ks * 16 + 2 * cq) : 0u;
-          qf[ks][2] = rv0 ? ld_u32(q0 + ks * 16 + 8 + 2 * cq) : 0u;
-          qf[ks][3] = rv1 ? ld_u32(q1 + ks * 16 + 8 + 2 * cq) : 0u;
+          const int c = 2 * (ks & 3) + (lane >> 4);
+          if (ok) ldsm_x4(qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], smem_u32(qb + (ks >> 2) * 16 * 128 + swz(row, c)));
+          else qf[ks][0] = qf[ks][1] = qf[ks][2] = qf[ks][3] = 0u;
+          if (!rv0) qf[ks][0] = qf[ks][2] = 0u;
+          if (!rv1) qf[ks][1] = qf[ks][3] = 0u;
         }
+        tc::fence_async_smem();   // the buffer is refilled by TMA after the release
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(q_empty + qs);
       }
       // warm L2 for what comes from DRAM later: the next item's queries and block list
       // (this pipeline's next token; the producer reads the list about two blocks ahead
@@ -196,7 +240,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (j < 0) break;
         const int jb = min(j, t / kBlk);
         const int slot = (int)(use % kSlots);
-        ok = tc::mbar_wait(full + slot, (uint32_t)((use / kSlots) & 1), err, 23);
+        ok = ok && tc::mbar_wait(full + slot, (uint32_t)((use / kSlots) & 1), err, 23);
         ok = __all_sync(0xffffffffu, ok);   // reconverge the warp before ldmatrix / mma
         const uint8_t* kb = ring + slot * SM::kSlotBytes;
         const uint8_t* vb = kb + (DK / 64) * kBox;
@@ -385,7 +429,13 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
   const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
   const uint32_t box[3] = {64, 1, kBlk};
-  if (!make_tmap_bf16(&mk, a.k, 3, dk3, sk3, box) || !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, box))
+  CUtensorMap mq;
+  const uint64_t dq3[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
+  const uint64_t sq3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
+  const int q_rows = a.Hq < 16 ? a.Hq : 16;   // a box is never taller than the tensor
+  const uint32_t qbox[3] = {64, (uint32_t)q_rows, 1};
+  if (!make_tmap_bf16(&mk, a.k, 3, dk3, sk3, box) || !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, box) ||
+      !make_tmap_bf16(&mq, a.q, 3, dq3, sq3, qbox))
     return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -394,8 +444,8 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   const long ctas = (total + kGroups - 1) / kGroups;
   const int grid = (int)(ctas < (long)sms * kCtasPerSm ? ctas : (long)sms * kCtasPerSm);
   slc_attn_tma_kernel<DK, DV><<<grid, threads<DV>(), SM::kAlloc, st>>>(
-      mk, mv, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B,
-      a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, a.err);
+      mk, mv, mq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B,
+      a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, q_rows, a.err);
   return cudaGetLastError();
 }
 }  // namespace

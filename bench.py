@@ -216,7 +216,7 @@ def workload_config(c, name):
 NCU_DRAM_BYTES_PER_ITEM = {
     "cmp_select": (205.893888e6 + 217.393408e6) / 32768,
     "slc_attn": (501.284608e6 + 229.739008e6) / 32768,
-    "swa_combine": (499.571200e6 + 117.488896e6) / 32768,
+    "swa_combine": None,   # changed since its capture
 }
 
 

@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libnsa.so")
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
 NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
 
-EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_decode",
+EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_forward_varlen",
+            "nsa_decode",
             "nsa_forward_noalloc", "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
 
 
@@ -65,6 +66,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_compress_append.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     lib.nsa_compress_append.restype = ctypes.c_int
     lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
+    lib.nsa_forward_varlen.restype = ctypes.c_int
+    lib.nsa_forward_varlen.argtypes = [vp, vp, vp, vp, vp, i32, cfgp, vp, vp]
     lib.nsa_forward.restype = ctypes.c_int
     lib.nsa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp, cfgp, vp, vp]
     lib.nsa_decode.restype = ctypes.c_int
@@ -148,6 +151,14 @@ def nsa_forward(q, k, v, gates, cfg: NsaConfig, out, stream=None, check: bool = 
     st = load_library().nsa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), ctypes.byref(cfg), _ptr(out),
                                     _stream(stream, q))
     return _check(st, "nsa_forward") if check else st
+
+
+def nsa_forward_varlen(q, k, v, gates, cu_seqlens, cfg: NsaConfig, out, stream=None, check: bool = True) -> int:
+    """Packed variable-length batch: q [total, H_q, d_k] etc., cu_seqlens int32 [B + 1] on the
+    device (see include/nsa.h); total = q.shape[0]."""
+    st = load_library().nsa_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(cu_seqlens),
+                                           int(q.shape[0]), ctypes.byref(cfg), _ptr(out), _stream(stream, q))
+    return _check(st, "nsa_forward_varlen") if check else st
 
 
 def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, max_seqlen: int, gates, cfg: NsaConfig, out,

@@ -180,13 +180,17 @@ struct TopkWarp {
   }
 };
 
-template <int DK, int DV>
+// VARLEN: a packed batch of sequences of different lengths (cu); its own instantiation, so
+// that the equal-length one keeps its plain row arithmetic.
+template <int DK, int DV, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                const __grid_constant__ CUtensorMap tm_vc, const __nv_bfloat16* __restrict__ gates,
                float* __restrict__ acc, int32_t* __restrict__ idx_out, int B, int T, int Hq, int Hkv, int nc,
-               int top_k, int force_first, int force_local, float scale_log2, int* __restrict__ err) {
+               int top_k, int force_first, int force_local, float scale_log2, const int32_t* __restrict__ cu_in,
+               int* __restrict__ err) {
   using SM = Smem<DK, DV>;
+  const int32_t* cu = VARLEN ? cu_in : nullptr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + SM::kQ;
@@ -217,16 +221,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tok_tiles = (T + kTok - 1) / kTok;
   const int n_items = n_tok_tiles * Hkv * B;
-  // item -> (token tile, group, batch); the longest rows come first
-  struct Item { int t0, g, b, ntiles; };
+  // item -> (token tile, group, batch); the longest rows come first.  In a variable-length
+  // batch, tiles past a sequence's end are no items: every role skips them alike.
+  struct Item { int t0, g, b, ntiles, base, len; };
   auto item_of = [&](int it) {
     Item x;
     x.g = it % Hkv;
     x.b = (it / Hkv) % B;
     x.t0 = (n_tok_tiles - 1 - it / (Hkv * B)) * kTok;
-    const int t_last = min(x.t0 + kTok - 1, T - 1);
+    x.base = seq_base(cu, x.b, T);   // first row of the sequence in q, gates and acc
+    x.len = seq_len(cu, x.b, T);
+    const int t_last = min(x.t0 + kTok - 1, x.len - 1);
     x.ntiles = (n_visible(t_last, nc) + kBlk - 1) / kBlk;
     return x;
+  };
+  auto next_item = [&](int it) {   // the first item >= it of this CTA's stride that has tokens
+    if (cu)
+      while (it < n_items && (n_tok_tiles - 1 - it / (Hkv * B)) * kTok >= seq_len(cu, (it / Hkv) % B, T))
+        it += gridDim.x;
+    return it;
   };
 
   if (tid == 0) {
@@ -266,14 +279,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int vcnt = 0;   // Vc tile fills so far
       bool ok = true;
       int k = 0;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      for (int it = next_item(blockIdx.x); it < n_items && ok; it = next_item(it + gridDim.x), ++k) {
         const Item x = item_of(it);
         // Q of this item once the previous item's S MMAs are done with the buffer
         if (k > 0) ok = tc::mbar_wait(q_empty, (k - 1) & 1, err, kErrQEmpty);
         if (!ok) break;
         tc::mbar_expect_tx(bar_q, SM::kQSlices * kSlice);
         for (int s = 0; s < SM::kQSlices; ++s)
-          tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, x.g * 16, x.b * T + x.t0);
+          tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, x.g * 16, x.base + x.t0);
         for (int pass = 0; pass < 2 && ok; ++pass) {
           for (int n = 0; n < x.ntiles && ok; ++n) {
             const int row = x.b * nc + n * kBlk;
@@ -314,7 +327,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int pc = 0;     // pass-B tiles (P^T phases, Vc tiles) so far
       bool ok = true;
       int k = 0;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      for (int it = next_item(blockIdx.x); it < n_items && ok; it = next_item(it + gridDim.x), ++k) {
         const Item x = item_of(it);
         ok = tc::mbar_wait(bar_q, k & 1, err, kErrQ);
         if (!ok) break;
@@ -376,7 +389,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     bool ok = true;
     int k = 0;
     TopkWarp<2> tk;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+    for (int it = next_item(blockIdx.x); it < n_items && ok; it = next_item(it + gridDim.x), ++k) {
       const Item x = item_of(it);
       ok = tc::mbar_wait(sc_full, k & 1, err, kErrScFull);
       ok = __all_sync(0xffffffffu, ok);
@@ -388,7 +401,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk) {
           const int t = t0p + kk;
-          nb[kk] = t < T ? t / kSel + 1 : 0;
+          nb[kk] = t < x.len ? t / kSel + 1 : 0;
           own[kk] = t / kSel;
         }
         tk.load(sScore + (4 * w + 2 * pr) * kMaxSel, kMaxSel, nb, own, force_first, force_local, lane);
@@ -415,19 +428,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int pc = 0;    // pass-B tiles
     for (int i = tid; i < kTok * kMaxSel; i += kNT) sScore[i] = 0.f;
     int k = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+    for (int it = next_item(blockIdx.x); it < n_items; it = next_item(it + gridDim.x), ++k) {
       const Item x = item_of(it);
-      const int t0 = x.t0, g = x.g, b = x.b, ntiles = x.ntiles;
+      const int t0 = x.t0, g = x.g, ntiles = x.ntiles, len = x.len;
+      const size_t base = x.base;
       float* gate = sGate + (k & 1) * kRowsM;
       if (gr == 0) {   // gates of the 128 rows (double-buffered: other groups may still be in the previous epilogue)
         const int t = t0 + r / 16, h = g * 16 + (r % 16);
-        gate[r] = t < T ? __bfloat162float(gates[(((size_t)b * T + t) * Hq + h) * 3]) : 0.f;
+        gate[r] = t < len ? __bfloat162float(gates[((base + t) * Hq + h) * 3]) : 0.f;
       }
 
       // pass A: this thread's row r = (token r/16, head r%16), its 32 columns of every tile
       {
         const int my_t = t0 + r / 16;
-        const int my_hi = my_t < T ? n_visible(my_t, nc) : 0;
+        const int my_hi = my_t < len ? n_visible(my_t, nc) : 0;
         float m = -INFINITY, l = 0.f;
         for (int n = 0; n < ntiles && ok; ++n, ++use) {
           const int sb = use & 1;
@@ -486,7 +500,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int q = 0; q < kSoftGroups; ++q) L += sML[(q * 128 + r) * 2 + 1] * ex2(sML[(q * 128 + r) * 2] - M);
         }
-        sLse[r] = (t0 + r / 16 < T && L > 0.f) ? M + __log2f(L) : INFINITY;
+        sLse[r] = (t0 + r / 16 < len && L > 0.f) ? M + __log2f(L) : INFINITY;
       }
       // the previous item's scores must have been taken (and zeroed) by the top-k warps
       if (k > 0) ok = tc::mbar_wait(sc_empty, (k - 1) & 1, err, kErrScEmpty);
@@ -498,7 +512,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
       for (int kk = 0; kk < kTokG; ++kk) {
         const int t = t0 + kTokG * gr + kk;
-        const bool in = t < T;
+        const bool in = t < len;
         hi_tok[kk] = in ? n_visible(t, nc) : 0;
         nb_tok[kk] = in ? t / kSel + 1 : 0;
       }
@@ -628,8 +642,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
         for (int c = 0; c < kCols; ++c) {
           const int t = t0 + kTokG * gr + c / 16;
-          if (t < T && r < DV) {
-            const size_t row = ((size_t)b * T + t) * Hq + g * 16 + (c % 16);
+          if (t < len && r < DV) {
+            const size_t row = (base + t) * Hq + g * 16 + (c % 16);
             acc[row * DV + r] = gate[col0 + c] * v[c];
           }
         }
@@ -651,8 +665,11 @@ cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   static bool attr = false;
   static int sms = 0;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)SM::kAlloc);
     if (e != cudaSuccess) return e;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -661,7 +678,7 @@ cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
     attr = true;
   }
   CUtensorMap mq, mk, mv;
-  const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
+  const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.total};
   const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
   const uint32_t bq[3] = {64, 16, kTok};
   const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.nc};
@@ -680,9 +697,10 @@ cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   const long long n_items = (long long)((a.T + kTok - 1) / kTok) * a.Hkv * a.B;
   if (n_items == 0) return cudaSuccess;
   const int grid = (int)std::min<long long>(n_items, sms);
-  attn_tc_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
+  auto kernel = a.cu ? attn_tc_kernel<DK, DV, true> : attn_tc_kernel<DK, DV, false>;
+  kernel<<<grid, kThreads, SM::kAlloc, st>>>(
       mq, mk, mv, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, a.B, a.T, a.Hq, a.Hkv, a.nc, a.top_k,
-      a.force_first, a.force_local, a.scale_log2, a.err);
+      a.force_first, a.force_local, a.scale_log2, a.cu, a.err);
   return cudaGetLastError();
 }
 }  // namespace

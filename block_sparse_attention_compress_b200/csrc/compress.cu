@@ -10,6 +10,10 @@
 // the windows, each at the one window its newest token completes (or none).  A row's
 // arithmetic (k chunks in order, the same MMA fragments) does not depend on which rows share
 // its CTA, so every block equals bitwise the one the full compression computes.
+// Variable-length batch (cu != nullptr): sequence b's tokens are rows cu[b] .. cu[b+1] of x
+// and its n_cmp(cu[b+1] - cu[b]) blocks go to out[b, 0 .. ); its rows from there up to nc are
+// zeroed, so that a reader of whole 128-row tiles (masked past the sequence) only ever
+// multiplies finite values by its zero weights.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,7 +28,7 @@ template <int D, int DOUT, int STAGES, bool APPEND>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
                 int l, int s, int nc, __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ seqlens,
-                int B) {
+                int B, const int32_t* __restrict__ cu) {
   extern __shared__ __align__(128) uint8_t csmem[];
   auto sA = reinterpret_cast<__nv_bfloat16(*)[kBM * kBK]>(csmem);                          // [STAGES]
   auto sB = reinterpret_cast<__nv_bfloat16(*)[kBK * kBN]>(csmem + STAGES * kBM * kBK * 2);  // [STAGES]
@@ -35,6 +39,20 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   constexpr bool app = APPEND;
   const int bh = blockIdx.z, b = app ? 0 : bh / H, h = app ? bh : bh % H;
   const int nk = l * D / kBK;
+  // full mode: the first token row of sequence b and its number of blocks
+  int base = 0, nc_b = nc;
+  if constexpr (!APPEND) {
+    base = seq_base(cu, b, T);
+    const int L = seq_len(cu, b, T);
+    nc_b = L < l ? 0 : min(nc, (L - l) / s + 1);
+    if (i0 >= nc_b) {   // the whole CTA: no block of this sequence, zero its rows
+      for (int e = tid; e < kBM * (kBN / 8); e += kThreads) {
+        const int i = i0 + e / (kBN / 8), c = (e % (kBN / 8)) * 8;
+        if (i < nc) *reinterpret_cast<uint4*>(out + (((size_t)b * nc + i) * H + h) * DOUT + n0 + c) = make_uint4(0, 0, 0, 0);
+      }
+      return;
+    }
+  }
   if constexpr (APPEND) {
     if (tid < kBM) {
       const int bb = i0 + tid;
@@ -45,7 +63,10 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   }
   // the source row of CTA row `row`: (sequence, window) in append mode, else (b, i0 + row)
   auto row_seq = [&](int row) { return app ? i0 + row : b; };
-  auto row_win = [&](int row) { return app ? sWin[row] : (i0 + row < nc ? i0 + row : -1); };
+  auto row_win = [&](int row) { return app ? sWin[row] : (i0 + row < nc_b ? i0 + row : -1); };
+  auto src_row = [&](int row, int i, int r) -> size_t {   // token row of x
+    return app ? (size_t)row_seq(row) * T + (size_t)s * i + r : (size_t)base + (size_t)s * i + r;
+  };
 
   auto load = [&](int kc, int buf) {
     const int kk0 = kc * kBK;
@@ -55,8 +76,7 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
       const int row = e >> 3, ch = e & 7;
       const int i = row_win(row);
       const bool ok = i >= 0;
-      const __nv_bfloat16* src =
-          x + (((size_t)(ok ? row_seq(row) : 0) * T + (ok ? (size_t)s * i + r : 0)) * H + h) * D + c0 + ch * 8;
+      const __nv_bfloat16* src = x + ((ok ? src_row(row, i, r) : 0) * H + h) * D + c0 + ch * 8;
       cp_async16(&sA[buf][Swz::offset(row, ch)], src, ok);
     }
 #pragma unroll
@@ -109,7 +129,14 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   for (int half = 0; half < 2; ++half) {
     const int row = warp * 16 + gl + half * 8;
     const int i = row_win(row);
-    if (i < 0) continue;
+    if (i < 0) {
+      if (!APPEND && i0 + row < nc) {   // past this sequence's blocks: zeros
+        __nv_bfloat16* dst = out + (((size_t)b * nc + i0 + row) * H + h) * DOUT + n0;
+#pragma unroll
+        for (int j = 0; j < kBN / 8; ++j) *reinterpret_cast<uint32_t*>(dst + j * 8 + 2 * cq) = 0u;
+      }
+      continue;
+    }
     __nv_bfloat16* dst = out + (((size_t)row_seq(row) * nc + i) * H + h) * DOUT + n0;
 #pragma unroll
     for (int j = 0; j < kBN / 8; ++j) {
@@ -123,11 +150,11 @@ constexpr size_t smem_bytes(int stages) { return (size_t)stages * (kBM * kBK + k
 
 template <int D>
 cudaError_t launch(const void* x, const void* w, int B, int T, int H, int l, int s, int nc, void* out,
-                   cudaStream_t st) {
+                   cudaStream_t st, const int32_t* cu) {
   dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
   compress_kernel<D, D, 2, false><<<grid, kThreads, smem_bytes(2), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w), T, H, l, s, nc,
-                                                   static_cast<__nv_bfloat16*>(out), nullptr, B);
+                                                   static_cast<__nv_bfloat16*>(out), nullptr, B, cu);
   return cudaGetLastError();
 }
 
@@ -145,7 +172,7 @@ cudaError_t launch_append(const void* x, const void* w, const int32_t* seqlens, 
   dim3 grid((B + kBM - 1) / kBM, D / kBN, H);
   compress_kernel<D, D, kStages, true><<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w), Lmax, H, l, s, ncmax,
-                                                   static_cast<__nv_bfloat16*>(out), seqlens, B);
+                                                   static_cast<__nv_bfloat16*>(out), seqlens, B, nullptr);
   return cudaGetLastError();
 }
 }  // namespace
@@ -162,13 +189,13 @@ cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* 
 }
 
 cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
-                            cudaStream_t st) {
+                            cudaStream_t st, const int32_t* cu) {
   const int nc = T < l ? 0 : (T - l) / s + 1;
   if (nc == 0 || B == 0 || H == 0) return cudaSuccess;
   switch (d) {
-    case 64: return launch<64>(x, w, B, T, H, l, s, nc, out, st);
-    case 128: return launch<128>(x, w, B, T, H, l, s, nc, out, st);
-    case 192: return launch<192>(x, w, B, T, H, l, s, nc, out, st);
+    case 64: return launch<64>(x, w, B, T, H, l, s, nc, out, st, cu);
+    case 128: return launch<128>(x, w, B, T, H, l, s, nc, out, st, cu);
+    case 192: return launch<192>(x, w, B, T, H, l, s, nc, out, st, cu);
     default: return cudaErrorInvalidValue;
   }
 }

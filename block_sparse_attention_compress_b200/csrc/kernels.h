@@ -11,7 +11,8 @@ namespace nsa {
 
 // K1: phi for every (b, h): out [B, N_c, H, d] bf16 (l = 32, s = 16 validated).
 cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
-                            cudaStream_t st);
+                            cudaStream_t st,
+                            const int32_t* cu = nullptr);
 // K1 for a growing cache: for each sequence b whose newest token (L = seqlens[b], clamped
 // to Lmax) completes window i = (L - l)/s < ncmax, out[b, i, h, :] for every head.
 cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,
@@ -31,7 +32,18 @@ struct FwdArgs {
   int top_k, window, force_first, force_local;
   float scale_log2;   // softmax scale * log2(e)
   int* err;           // device word, zeroed before the launches; nonzero = a bounded wait timed out
+  // Variable-length batch: cu[b] .. cu[b+1] are sequence b's rows of q, k, v, gates, acc and out
+  // (device, [B + 1], cu[0] = 0, lengths <= T); nullptr = B sequences of T tokens each.  Kc/Vc
+  // and idx keep their per-sequence layouts with T as the (maximum) length.
+  const int32_t* cu = nullptr;
+  int total = 0;      // token rows (cu[B], or B * T)
 };
+
+// First row and length of sequence b in a (possibly variable-length) batch.
+__device__ __forceinline__ int seq_base(const int32_t* cu, int b, int T) { return cu ? __ldg(cu + b) : b * T; }
+__device__ __forceinline__ int seq_len(const int32_t* cu, int b, int T) {
+  return cu ? __ldg(cu + b + 1) - __ldg(cu + b) : T;
+}
 
 // K2: compressed attention (writes acc = g_cmp * o_cmp) + group-summed block
 // scores + top-k (writes idx).

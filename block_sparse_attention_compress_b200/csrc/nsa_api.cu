@@ -111,6 +111,58 @@ nsa_status moba_forward(const void* q, const void* k, const void* v, const nsa_c
   return from_cuda(nsa::launch_moba(a, s));
 }
 
+// The launch sequence of an NSA forward: phi of K and V, compressed branch with the block
+// scores and top-k, selected branch, window branch with the gated combine.  cu == nullptr is a
+// batch of equal lengths (cfg->seqlen each); otherwise sequence b is rows cu[b] .. cu[b+1].
+nsa_status nsa_forward_impl(const void* q, const void* k, const void* v, const void* gates, const nsa_config* cfg,
+                            void* out, cudaStream_t s, const int32_t* cu, int total) {
+  const FwdLayout L = forward_layout(cfg);
+  auto ws = static_cast<uint8_t*>(cfg->workspace);
+  nsa::FwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.gates = gates; a.out = out;
+  a.B = cfg->batch; a.T = cfg->seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
+  a.dk = cfg->d_k; a.dv = cfg->d_v; a.nc = n_cmp(cfg->seqlen, cfg->cmp_block, cfg->cmp_stride);
+  a.top_k = cfg->top_k; a.window = cfg->window;
+  a.force_first = cfg->force_first; a.force_local = cfg->force_local;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  void* kc = cfg->kc_out ? cfg->kc_out : ws + L.kc;
+  void* vc = cfg->vc_out ? cfg->vc_out : ws + L.vc;
+  a.kc = kc; a.vc = vc;
+  a.idx = cfg->sel_idx_out ? cfg->sel_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
+  a.acc = reinterpret_cast<float*>(ws + L.acc);
+  a.err = reinterpret_cast<int*>(ws + L.err);
+  a.cu = cu;
+  a.total = total;
+
+  StageMarks marks(cfg, 5);
+  cudaError_t e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess)
+    e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, kc, s, cu);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess)
+    e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, cfg->cmp_block, cfg->cmp_stride, vc, s, cu);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_cmp_select(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_slc_attn(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_swa_combine(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  return from_cuda(e);
+}
+
+// A variable-length batch runs on the tensor-core kernels only (their shapes).
+bool varlen_supported(const nsa_config* c) {
+  nsa::FwdArgs a{};
+  a.B = c->batch; a.T = c->seqlen; a.Hq = c->h_q; a.Hkv = c->h_kv; a.G = c->h_q / c->h_kv;
+  a.dk = c->d_k; a.dv = c->d_v; a.window = c->window; a.top_k = c->top_k;
+  int dummy = 0;
+  a.err = &dummy;   // the kernels' status word exists on this path
+  return nsa::cmp_select_tc_supported(a) && nsa::slc_attn_tma_supported(a) && nsa::window_tc_supported(a);
+}
+
 }  // namespace
 
 extern "C" {
@@ -187,41 +239,24 @@ nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* 
   st = check_workspace(cfg, workspace_bytes(cfg));
   if (st != NSA_OK) return st;
   if (cfg->mode == NSA_MODE_MOBA) return moba_forward(q, k, v, cfg, out, static_cast<cudaStream_t>(stream));
-  const FwdLayout L = forward_layout(cfg);
+  return nsa_forward_impl(q, k, v, gates, cfg, out, static_cast<cudaStream_t>(stream), nullptr,
+                          cfg->batch * cfg->seqlen);
+}
 
-  auto ws = static_cast<uint8_t*>(cfg->workspace);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  nsa::FwdArgs a{};
-  a.q = q; a.k = k; a.v = v; a.gates = gates; a.out = out;
-  a.B = cfg->batch; a.T = cfg->seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
-  a.dk = cfg->d_k; a.dv = cfg->d_v; a.nc = n_cmp(cfg->seqlen, cfg->cmp_block, cfg->cmp_stride);
-  a.top_k = cfg->top_k; a.window = cfg->window;
-  a.force_first = cfg->force_first; a.force_local = cfg->force_local;
-  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
-  a.scale_log2 = scale * 1.4426950408889634f;
-  void* kc = cfg->kc_out ? cfg->kc_out : ws + L.kc;
-  void* vc = cfg->vc_out ? cfg->vc_out : ws + L.vc;
-  a.kc = kc; a.vc = vc;
-  a.idx = cfg->sel_idx_out ? cfg->sel_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
-  a.acc = reinterpret_cast<float*>(ws + L.acc);
-  a.err = reinterpret_cast<int*>(ws + L.err);
-
-  StageMarks marks(cfg, 5);
-  cudaError_t e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess)
-    e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, kc, s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess)
-    e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, cfg->cmp_block, cfg->cmp_stride, vc, s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess) e = nsa::launch_cmp_select(a, s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess) e = nsa::launch_slc_attn(a, s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess) e = nsa::launch_swa_combine(a, s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  return from_cuda(e);
+nsa_status nsa_forward_varlen(const void* q, const void* k, const void* v, const void* gates,
+                              const int32_t* cu_seqlens, int32_t total_tokens, const nsa_config* cfg, void* out,
+                              void* stream) {
+  nsa_status st = check_cfg(cfg);
+  if (st != NSA_OK) return st;
+  if (cfg->mode != NSA_MODE_NSA) return NSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !gates || !cu_seqlens || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(gates) & 1u) || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+    return NSA_ERR_INVALID_ARG;
+  if (total_tokens < 1 || (int64_t)total_tokens > (int64_t)cfg->batch * cfg->seqlen) return NSA_ERR_INVALID_ARG;
+  if (!varlen_supported(cfg)) return NSA_ERR_UNSUPPORTED;
+  st = check_workspace(cfg, workspace_bytes(cfg));
+  if (st != NSA_OK) return st;
+  return nsa_forward_impl(q, k, v, gates, cfg, out, static_cast<cudaStream_t>(stream), cu_seqlens, total_tokens);
 }
 
 nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* kc_cache,

@@ -67,13 +67,17 @@ using tc::vote_all;
 // byte offset of (row, 16-byte chunk c of a 64-column box) in a 128-byte-swizzled box
 __device__ __forceinline__ uint32_t swz(int row, int c) { return row * 128 + ((c ^ (row & 7)) << 4); }
 
-template <int DK, int DV>
+// VARLEN: a packed batch of sequences of different lengths (cu); its own instantiation, so
+// that the equal-length one keeps its plain row arithmetic.
+template <int DK, int DV, bool VARLEN>
 __global__ void __launch_bounds__(threads<DV>(), kCtasPerSm)
 slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ gates,
                     const int32_t* __restrict__ idx, float* __restrict__ acc, int B, int T, int Hq, int Hkv, int G,
-                    int top_k, float scale_log2, int q_rows, int* __restrict__ err) {
+                    int top_k, float scale_log2, int q_rows, const int32_t* __restrict__ cu_in,
+                    int* __restrict__ err) {
   using SM = Smem<DK, DV>;
+  const int32_t* cu = cu_in;
   constexpr int kConsumers = SM::kConsumers;
   constexpr int kKW = kBlk / kConsumers;            // keys per consumer warp: 16 or 8
   extern __shared__ uint8_t smem_raw[];
@@ -104,7 +108,21 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
   }
   __syncthreads();
   const long total = (long)Hkv * B * T;
-  const long it0 = (long)blockIdx.x * kGroups + grp, stride = (long)gridDim.x * kGroups;
+  const long stride = (long)gridDim.x * kGroups;
+  // item it = (group, batch, token); in a variable-length batch the tokens past a
+  // sequence's end are no items, and producer and consumers skip them alike
+  auto next_item = [&](long it) {
+    if constexpr (VARLEN)
+      while (it < total && (int)(it % T) >= seq_len(cu, (int)((it / T) % B), T)) it += stride;
+    return it;
+  };
+  const long it0 = next_item((long)blockIdx.x * kGroups + grp);
+  // the row of token t of sequence b in q, k, v, gates and acc (recomputed where it is used, so
+  // that nothing extra stays live across the block loop)
+  auto row_of = [&](int b, int t) -> size_t {
+    if constexpr (VARLEN) return (size_t)seq_base(cu, b, T) + t;
+    else return (size_t)b * T + t;
+  };
 
   if (producer) {
     // ---------------------------------------------------------------- producer
@@ -116,10 +134,11 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     long fill = 0, qfill = 0;
     bool ok = true;
-    for (long it = it0; it < total && ok; it += stride, ++qfill) {
+    for (long it = it0; it < total && ok; it = next_item(it + stride), ++qfill) {
       const int g = (int)(it / ((long)B * T));
       const int bt = (int)(it % ((long)B * T));
       const int b = bt / T, t = bt % T;
+      const int base = (int)row_of(b, 0);   // first row of the sequence in q, k and v
       // this item's queries: rows g*G .. g*G+q_rows-1 of token (b, t) (q_rows = min(16, Hq);
       // rows past the group are masked by the consumers, rows past the last head are
       // zero-filled by TMA)
@@ -131,7 +150,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane == 0) {
           tc::mbar_expect_tx(q_full + qs, (uint32_t)((DK / 64) * q_rows * 128));
           for (int s = 0; s < DK / 64; ++s)
-            tc::tma_load_3d(qbuf + qs * SM::kQBytes + s * 16 * 128, &tm_q, q_full + qs, s * 64, g * G, b * T + t);
+            tc::tma_load_3d(qbuf + qs * SM::kQBytes + s * 16 * 128, &tm_q, q_full + qs, s * 64, g * G, base + t);
         }
         __syncwarp();
       }
@@ -148,9 +167,9 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           uint8_t* dst = ring + slot * SM::kSlotBytes;
           tc::mbar_expect_tx(full + slot, SM::kSlotBytes);
           for (int s = 0; s < DK / 64; ++s)
-            tc::tma_load_3d(dst + s * kBox, &tm_k, full + slot, s * 64, g, b * T + jb * kBlk);
+            tc::tma_load_3d(dst + s * kBox, &tm_k, full + slot, s * 64, g, base + jb * kBlk);
           for (int s = 0; s < DV / 64; ++s)
-            tc::tma_load_3d(dst + (DK / 64 + s) * kBox, &tm_v, full + slot, s * 64, g, b * T + jb * kBlk);
+            tc::tma_load_3d(dst + (DK / 64 + s) * kBox, &tm_v, full + slot, s * 64, g, base + jb * kBlk);
         }
         __syncwarp();
         ++fill;
@@ -176,7 +195,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     int* sFlag = reinterpret_cast<int*>(sL + kConsumers * 16);                      // [warp] no wait failed
     long use = 0, quse = 0;
     bool ok = true;
-    for (long it = it0; it < total && ok; it += stride, ++quse) {
+    for (long it = it0; it < total && ok; it = next_item(it + stride), ++quse) {
       const int g = (int)(it / ((long)B * T));
       const int bt = (int)(it % ((long)B * T));
       const int b = bt / T, t = bt % T;
@@ -209,11 +228,11 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
       // of the consumers, too late to hide a DRAM access), and this item's accumulator
       // rows and gates
       {
-        const long itn = it + stride;
+        const long itn = next_item(it + stride);
         if (itn < total) {
           const int gn = (int)(itn / ((long)B * T));
           const int btn = (int)(itn % ((long)B * T));
-          const char* qn = reinterpret_cast<const char*>(q + ((size_t)btn * Hq + gn * G) * DK);
+          const char* qn = reinterpret_cast<const char*>(q + (row_of(btn / T, btn % T) * Hq + gn * G) * DK);
           constexpr int kLines = 16 * DK * 2 / 128;               // 16 heads of queries
           for (int ln = cw * 32 + lane; ln < kLines; ln += kConsumers * 32)
             if (ln < G * DK * 2 / 128) prefetch_l2(qn + ln * 128);
@@ -223,9 +242,9 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
           }
         }
         if (lane < G)
-          prefetch_l2(acc + (((size_t)b * T + t) * Hq + g * G + lane) * DV + cw * (DV / kConsumers));
+          prefetch_l2(acc + (row_of(b, t) * Hq + g * G + lane) * DV + cw * (DV / kConsumers));
         if (cw == 1 && lane < 2) {   // the G x 3 gates of this item's rows (at most two lines)
-          const char* gp = reinterpret_cast<const char*>(gates + ((size_t)b * T + t) * Hq * 3 + g * G * 3);
+          const char* gp = reinterpret_cast<const char*>(gates + row_of(b, t) * Hq * 3 + g * G * 3);
           prefetch_l2(lane == 0 ? gp : gp + G * 3 * 2 - 1);
         }
       }
@@ -380,7 +399,7 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         sL[cw * 16 + gl] = l0;
         sL[cw * 16 + gl + 8] = l1;
       }
-      const size_t row0 = ((size_t)b * T + t) * Hq + g * G;
+      const size_t row0 = row_of(b, t) * Hq + g * G;
       float2 prev[2][kNt];
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
@@ -419,18 +438,21 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
-        cudaFuncSetAttribute(slc_attn_tma_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+        cudaFuncSetAttribute(slc_attn_tma_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(slc_attn_tma_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)SM::kAlloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   CUtensorMap mk, mv;
-  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.total};
   const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
-  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.total};
   const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
   const uint32_t box[3] = {64, 1, kBlk};
   CUtensorMap mq;
-  const uint64_t dq3[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
+  const uint64_t dq3[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.total};
   const uint64_t sq3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
   const int q_rows = a.Hq < 16 ? a.Hq : 16;   // a box is never taller than the tensor
   const uint32_t qbox[3] = {64, (uint32_t)q_rows, 1};
@@ -443,9 +465,10 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   const long total = (long)a.Hkv * a.B * a.T;
   const long ctas = (total + kGroups - 1) / kGroups;
   const int grid = (int)(ctas < (long)sms * kCtasPerSm ? ctas : (long)sms * kCtasPerSm);
-  slc_attn_tma_kernel<DK, DV><<<grid, threads<DV>(), SM::kAlloc, st>>>(
+  auto kernel = a.cu ? slc_attn_tma_kernel<DK, DV, true> : slc_attn_tma_kernel<DK, DV, false>;
+  kernel<<<grid, threads<DV>(), SM::kAlloc, st>>>(
       mk, mv, mq, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B,
-      a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, q_rows, a.err);
+      a.T, a.Hq, a.Hkv, a.G, a.top_k, a.scale_log2, q_rows, a.cu, a.err);
   return cudaGetLastError();
 }
 }  // namespace

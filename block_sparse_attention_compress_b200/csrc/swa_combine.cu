@@ -213,6 +213,7 @@ cudaError_t launch(const FwdArgs& a, cudaStream_t st) {
 
 cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st) {
   if (window_tc_supported(a)) return launch_window_tc(a, st);
+  if (a.cu) return cudaErrorInvalidValue;   // variable-length batches run on the tensor-core kernels only
   if (a.dk == 64 && a.dv == 64) return launch<64, 64>(a, st);
   if (a.dk == 128 && a.dv == 128) return launch<128, 128>(a, st);
   if (a.dk == 192 && a.dv == 128) return launch<192, 128>(a, st);

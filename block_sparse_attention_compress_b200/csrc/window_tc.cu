@@ -61,13 +61,16 @@ struct Smem {
   static_assert(kAlloc <= 232448, "shared memory");
 };
 
-template <int DK, int DV>
+// VARLEN: a packed batch of sequences of different lengths (cu); its own instantiation, so
+// that the equal-length one keeps its plain row arithmetic.
+template <int DK, int DV, bool VARLEN>
 __global__ void __launch_bounds__(kThreads, 1)
 window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16* __restrict__ gates,
                  const float* __restrict__ acc, __nv_bfloat16* __restrict__ out, int B, int T, int Hq, int Hkv,
-                 int window, float scale_log2, int* __restrict__ err) {
+                 int window, float scale_log2, const int32_t* __restrict__ cu_in, int* __restrict__ err) {
   using SM = Smem<DK, DV>;
+  const int32_t* cu = VARLEN ? cu_in : nullptr;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + SM::kQ;
@@ -96,17 +99,26 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int n_tok_tiles = (T + kTok - 1) / kTok;
   const int n_items = n_tok_tiles * Hkv * B;
   // item -> (token tile, group, batch), the latest tokens first (all items but the first
-  // few have the same number of key tiles)
-  struct Item { int t0, g, b, kv_lo, ntiles; };
+  // few have the same number of key tiles).  In a variable-length batch, tiles past a
+  // sequence's end are no items: every role skips them alike.
+  struct Item { int t0, g, b, kv_lo, ntiles, base, len; };
   auto item_of = [&](int it) {
     Item x;
     x.g = it % Hkv;
     x.b = (it / Hkv) % B;
     x.t0 = (n_tok_tiles - 1 - it / (Hkv * B)) * kTok;
-    const int t_last = min(x.t0 + kTok - 1, T - 1);
+    x.base = seq_base(cu, x.b, T);   // first row of the sequence in q, k, v, gates, acc, out
+    x.len = seq_len(cu, x.b, T);
+    const int t_last = min(x.t0 + kTok - 1, x.len - 1);
     x.kv_lo = max(0, x.t0 - window + 1);
     x.ntiles = (t_last - x.kv_lo + kBlk) / kBlk;   // >= 1
     return x;
+  };
+  auto next_item = [&](int it) {   // the first item >= it of this CTA's stride that has tokens
+    if (cu)
+      while (it < n_items && (n_tok_tiles - 1 - it / (Hkv * B)) * kTok >= seq_len(cu, (it / Hkv) % B, T))
+        it += gridDim.x;
+    return it;
   };
 
   if (tid == 0) {
@@ -147,15 +159,15 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc::prefetch_tmap(&tm_v);
       int fill = 0, vcnt = 0, k = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      for (int it = next_item(blockIdx.x); it < n_items && ok; it = next_item(it + gridDim.x), ++k) {
         const Item x = item_of(it);
         if (k > 0) ok = tc::mbar_wait(q_empty, (k - 1) & 1, err, kErrQEmpty);
         if (!ok) break;
         tc::mbar_expect_tx(bar_q, SM::kQSlices * kSlice);
         for (int s = 0; s < SM::kQSlices; ++s)
-          tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, x.g * 16, x.b * T + x.t0);
+          tc::tma_load_3d(sQ + s * kSlice, &tm_q, bar_q, s * 64, x.g * 16, x.base + x.t0);
         for (int n = 0; n < x.ntiles && ok; ++n) {
-          const int row = x.b * T + x.kv_lo + n * kBlk;
+          const int row = x.base + x.kv_lo + n * kBlk;
           for (int s = 0; s < SM::kQSlices && ok; ++s, ++fill) {
             const int slot = fill % kKSlots;
             ok = tc::mbar_wait(k_empty + slot, ((fill / kKSlots) & 1) ^ 1, err, kErrKEmpty);
@@ -223,7 +235,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         ++pc;
         return true;
       };
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++k) {
+      for (int it = next_item(blockIdx.x); it < n_items && ok; it = next_item(it + gridDim.x), ++k) {
         const Item x = item_of(it);
         const int ob = k & 1;
         const uint32_t o_col = kColO + 128 * ob;
@@ -252,14 +264,14 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
     bool ok = true;
     int use = 0, pc = 0, k = 0;
-    for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++k) {
+    for (int it = next_item(blockIdx.x); it < n_items; it = next_item(it + gridDim.x), ++k) {
       const Item x = item_of(it);
       const int ob = k & 1;
       const uint32_t o_col = kColO + 128 * ob;
       const int my_t = x.t0 + r / 16;
-      const bool row_ok = my_t < T;
+      const bool row_ok = my_t < x.len;
       const int my_lo = max(0, my_t - window + 1), my_hi = row_ok ? my_t : -1;   // keys [my_lo, my_hi]
-      const size_t grow = ((size_t)x.b * T + min(my_t, T - 1)) * Hq + x.g * 16 + (r % 16);
+      const size_t grow = ((size_t)x.base + min(my_t, x.len - 1)) * Hq + x.g * 16 + (r % 16);
       float* gate = sGate + ob * kRowsM;
       if (gr == 0) gate[r] = row_ok ? __bfloat162float(gates[grow * 3 + 2]) : 0.f;
       // the epilogue reads this thread's half of the accumulator row (256 B): start it now
@@ -413,17 +425,20 @@ cudaError_t launch_w(const FwdArgs& a, cudaStream_t st) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
-        cudaFuncSetAttribute(window_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+        cudaFuncSetAttribute(window_tc_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(window_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)SM::kAlloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   CUtensorMap mq, mk, mv;
-  const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.B * a.T};
+  const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.total};
   const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
   const uint32_t bq[3] = {64, 16, kTok};
-  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.total};
   const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
-  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.B * a.T};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.total};
   const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
   const uint32_t bkv[3] = {64, 1, (uint32_t)kBlk};
   if (!make_tmap_bf16(&mq, a.q, 3, dq, sq, bq) || !make_tmap_bf16(&mk, a.k, 3, dk3, sk3, bkv) ||
@@ -438,9 +453,10 @@ cudaError_t launch_w(const FwdArgs& a, cudaStream_t st) {
   }
   const long items = (long)((a.T + kTok - 1) / kTok) * a.Hkv * a.B;
   const int grid = (int)(items < sms ? items : sms);
-  window_tc_kernel<DK, DV><<<grid, kThreads, SM::kAlloc, st>>>(
+  auto kernel = a.cu ? window_tc_kernel<DK, DV, true> : window_tc_kernel<DK, DV, false>;
+  kernel<<<grid, kThreads, SM::kAlloc, st>>>(
       mq, mk, mv, static_cast<const __nv_bfloat16*>(a.gates), a.acc, static_cast<__nv_bfloat16*>(a.out), a.B, a.T,
-      a.Hq, a.Hkv, a.window, a.scale_log2, a.err);
+      a.Hq, a.Hkv, a.window, a.scale_log2, a.cu, a.err);
   return cudaGetLastError();
 }
 }  // namespace

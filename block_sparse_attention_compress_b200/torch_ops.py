@@ -6,7 +6,7 @@ from __future__ import annotations
 import torch
 
 from . import (NSA_MODE_MOBA, NSA_MODE_NSA, make_config, nsa_compress, nsa_decode, nsa_forward,
-               nsa_workspace_size)
+               nsa_forward_varlen, nsa_workspace_size)
 
 
 def n_cmp(T: int, l: int = 32, s: int = 16) -> int:
@@ -45,6 +45,20 @@ class NSAForward:
         if out is None:
             out = torch.empty((B, T, h_q, d_v), dtype=torch.bfloat16, device=q.device)
         nsa_forward(q, k, v, gates, self.cfg, out)
+        return out
+
+
+class NSAForwardVarlen(NSAForward):
+    """Prefill forward of a packed batch of sequences of different lengths (at most T
+    tokens each): q [total, h_q, d_k], k/v [total, h_kv, d], gates [total, h_q, 3], and
+    cu_seqlens int32 [B + 1] on the device.  idx, kc and vc keep the per-sequence layouts of
+    NSAForward (B sequences of up to T tokens)."""
+
+    def __call__(self, q, k, v, gates, cu_seqlens, out=None):
+        B, T, h_q, h_kv, d_k, d_v = self.shape
+        if out is None:
+            out = torch.empty((q.shape[0], h_q, d_v), dtype=torch.bfloat16, device=q.device)
+        nsa_forward_varlen(q, k, v, gates, cu_seqlens, self.cfg, out)
         return out
 
 

@@ -157,6 +157,29 @@ NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, cons
                        const nsa_config* cfg, void* out, void* stream);
 
 /*
+ * nsa_forward_varlen -- prefill forward of a batch of sequences of different lengths, packed
+ * one after another ([NOTES] §5-§8: every sequence is attended on its own, exactly as
+ * nsa_forward computes it for that sequence alone).  NSA mode only.
+ *   cu_seqlens   int32 [B + 1] device: sequence b is rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *                of q, k, v, gates and out; cu_seqlens[0] = 0, non-decreasing, every length
+ *                <= cfg->seqlen (empty sequences allowed), cu_seqlens[B] = total_tokens.  The
+ *                contents are not checked: values outside these rules give undefined results.
+ *   total_tokens the packed row count (host), 1 <= total_tokens <= B * cfg->seqlen.
+ *   q bf16 [total, H_q, d_k];  k [total, H_kv, d_k];  v [total, H_kv, d_v];
+ *   gates bf16 [total, H_q, 3];  out bf16 [total, H_q, d_v].
+ * cfg->batch = B and cfg->seqlen = the largest length (or any bound of it).  Per-sequence
+ * outputs keep the layouts of nsa_forward with T = cfg->seqlen: kc_out/vc_out
+ * [B, N_c(T), H_kv, d] (rows past N_c(length) zero), sel_idx_out [B, H_kv, T, top_k]
+ * (rows past the length unwritten).  Workspace: nsa_workspace_size(cfg, 0) bytes.
+ * Runs on the tensor-core kernels, which need G = 16, d_v = 128, d_k in {128, 192} and
+ * cfg->seqlen <= 65536; other shapes return NSA_ERR_UNSUPPORTED.  Other status codes as for
+ * nsa_forward.
+ */
+NSA_API nsa_status nsa_forward_varlen(const void* q, const void* k, const void* v, const void* gates,
+                                      const int32_t* cu_seqlens, int32_t total_tokens, const nsa_config* cfg,
+                                      void* out, void* stream);
+
+/*
  * nsa_decode -- one decode step per sequence ([NOTES] §13: decoding is bound by
  * the KV bytes read per step).  NSA mode only.
  *   q         bf16 [B, H_q, d_k]        the new token's queries

@@ -166,3 +166,27 @@ def test_compress_append_rejects_bad_arguments(lib):
     assert call(nc=0) == nsa.NSA_ERR_INVALID_ARG
     assert call(l=64) == nsa.NSA_ERR_UNSUPPORTED
     assert call(d=96, dout=96) == nsa.NSA_ERR_UNSUPPORTED
+
+
+def test_forward_varlen_rejects_bad_arguments(lib):
+    """Checks that return before any CUDA call (safe without a GPU): pointers, the packed row
+    count, the mode, and the shapes the tensor-core kernels do not take."""
+    f = 0x10000   # never dereferenced: every call below fails its checks first
+
+    def call(c, cu=f, total=100, q=f, gates=f):
+        return lib.nsa_forward_varlen(q, f, f, gates, cu, total, ctypes.byref(c), f, None)
+
+    c = _cfg(h_q=16, h_kv=1, d_k=192, d_v=128, batch=2, seqlen=64, workspace=0x100000, workspace_bytes=1 << 30)
+    assert call(c, cu=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(c, cu=f + 2) == nsa.NSA_ERR_INVALID_ARG            # misaligned offsets
+    assert call(c, gates=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(c, q=f + 8) == nsa.NSA_ERR_INVALID_ARG             # misaligned q
+    assert call(c, total=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(c, total=129) == nsa.NSA_ERR_INVALID_ARG           # more rows than batch x seqlen
+    small = _cfg(h_q=4, h_kv=1, d_k=64, d_v=64, batch=2, seqlen=64, workspace=0x100000, workspace_bytes=1 << 30)
+    assert call(small, total=64) == nsa.NSA_ERR_UNSUPPORTED        # the warp-MMA shapes
+    moba = _cfg(mode=nsa.NSA_MODE_MOBA, h_q=2, h_kv=2, d_k=128, d_v=128, sel_block=64, top_k=3, w_cmp_k=0,
+                w_cmp_v=0, batch=1, seqlen=128)
+    assert call(moba, total=64) == nsa.NSA_ERR_UNSUPPORTED
+    c.workspace_bytes = 16
+    assert call(c, total=64) == nsa.NSA_ERR_WORKSPACE

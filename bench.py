@@ -309,6 +309,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         result["moba"] = run_moba_bench(args, dev, world)
         result["gpu_launches"] += result["moba"]["gpu_launches"]
+    if not args.no_varlen:
+        torch.cuda.empty_cache()
+        result["varlen"] = run_varlen_bench(args, dev, world)
+        result["gpu_launches"] += result["varlen"]["gpu_launches"]
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         r, info = oracle_rate(cpu_workload(), args.ref_sample, seed=7, threads=os.cpu_count() or 1)
         result["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
@@ -447,6 +451,54 @@ def run_moba_bench(args, dev, world):
             "gpu_launches": 6 * args.steps}
 
 
+def run_varlen_bench(args, dev, world):
+    """NSA forward of a packed batch of 8 sequences of different lengths, 65536 tokens in all
+    (nsa_forward_varlen; stage times from the library's events)."""
+    from block_sparse_attention_compress_b200.torch_ops import NSAForwardVarlen
+    c = synth.WORKLOADS["nsa_varlen"]
+    lengths = list(c["lengths"])
+    hq, hkv, dk, dv = c["h_q"], c["h_kv"], c["d_k"], c["d_v"]
+    x, cu = synth.nsa_varlen_inputs(lengths, hq, hkv, dk, dv, seed=0, device=dev)
+    total = int(sum(lengths))
+    f = NSAForwardVarlen(len(lengths), max(lengths), hq, hkv, dk, dv, x.w_k, x.w_v, top_k=c["top_k"],
+                         window=c["window"], device=dev)
+    out = torch.empty((total, hq, dv), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nstage = len(STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    for es in evs:
+        for e in es:
+            e.record()
+    torch.cuda.synchronize()
+    handles = [ctypes_array(es) for es in evs]
+    for _ in range(args.warmup):
+        flush.zero_()
+        f.cfg.stage_events, f.cfg.n_stage_events = None, 0
+        f(x.q, x.k, x.v, x.gates, cu, out)
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        f.cfg.stage_events, f.cfg.n_stage_events = handles[i][0], nstage
+        f(x.q, x.k, x.v, x.gates, cu, out)
+    torch.cuda.synchronize()
+    assert f.device_status() == 0, "a device-side wait timed out"
+    step_ms = statistics.mean(es[0].elapsed_time(es[-1]) for es in evs)
+    stages = {n: statistics.mean(es[j].elapsed_time(es[j + 1]) for es in evs) for j, n in enumerate(STAGES)}
+    ms = allreduce_max(step_ms, world, dev)
+    flops = 0.0
+    for L in lengths:
+        flops += sum(nsa_flops(L, hq, hkv, dk, dv, c["top_k"], c["window"], 1).values())
+    peaks, _ = load_peaks()
+    return {"workload": f"nsa_varlen: 8 packed sequences of lengths {lengths} ({total} tokens), h_q={hq} "
+                        f"h_kv={hkv} d_k={dk} d_v={dv} top_k={c['top_k']} window={c['window']}",
+            "ms_per_step": ms, "tokens_per_s": world * total / (ms * 1e-3),
+            "tflops_computed": flops / (ms * 1e-3) / 1e12,
+            "frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "stages_ms": {n: round(v, 4) for n, v in stages.items()},
+            "gpu_launches": len(STAGES) * args.steps}
+
+
 def run_e2e(args, f, x, out, dev, world):
     """Same step through the public API with inputs in pinned host memory: H2D copies of
     q, k, v, gates, the forward, and the D2H copy of the output, all inside the timed region."""
@@ -511,6 +563,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-moba", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

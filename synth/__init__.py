@@ -115,6 +115,21 @@ def decode_inputs(B: int, L: int, h_q: int, h_kv: int, d_k: int, d_v: int,
     return DecodeInputs(q, k, v, w_k, w_v, gates, seqlens)
 
 
+def nsa_varlen_inputs(lengths, h_q: int, h_kv: int, d_k: int, d_v: int, cmp_block: int = 32, seed: int = 0,
+                      device="cpu"):
+    """A packed variable-length batch: sequence i is its own draw of nsa_inputs(1, L_i, ...)
+    with seed + i (the compression weights are sequence 0's), concatenated along the tokens.
+    Returns (NSAInputs with [total, ...] tensors and [l*d, d] weights, cu_seqlens int32 [B+1])."""
+    xs = [nsa_inputs(1, max(int(L), 1), h_q, h_kv, d_k, d_v, cmp_block, seed + i, device)
+          for i, L in enumerate(lengths)]
+    cat = lambda name: torch.cat([getattr(x, name)[0, :int(L)] for x, L in zip(xs, lengths)])
+    cu = [0]
+    for L in lengths:
+        cu.append(cu[-1] + int(L))
+    packed = NSAInputs(cat("q"), cat("k"), cat("v"), xs[0].w_k, xs[0].w_v, cat("gates"))
+    return packed, torch.tensor(cu, dtype=torch.int32, device=device)
+
+
 def moba_inputs(B: int, T: int, h: int, d: int, seed: int = 0, device="cpu") -> MobaInputs:
     g = _gen(seed, device)
     q = _randn(g, (B, T, h, d), device).to(torch.bfloat16)
@@ -137,4 +152,7 @@ WORKLOADS = {
     "nsa_64k": dict(B=1, T=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512),
     "nsa_decode": dict(B=32, L=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512),
     "moba_128k": dict(B=1, T=131072, h=32, d=128, block=512, top_k=3),
+    # a packed batch of 8 sequences of different lengths, 65536 tokens in all
+    "nsa_varlen": dict(lengths=(16384, 12288, 9000, 8192, 7000, 5000, 4096, 3576), h_q=64, h_kv=4, d_k=192,
+                       d_v=128, top_k=16, window=512),
 }

@@ -24,16 +24,8 @@ def _lib():
 
 
 def packed_inputs(lengths, hq, hkv, dk, dv, seed):
-    """One seeded draw per sequence (its own NSA inputs), packed along the token axis; the
-    compression weights are the first sequence's."""
-    xs = [synth.nsa_inputs(1, max(L, 1), hq, hkv, dk, dv, seed=seed + i) for i, L in enumerate(lengths)]
-    cut = lambda t, L: t[0, :L]
-    q = torch.cat([cut(x.q, L) for x, L in zip(xs, lengths)])
-    k = torch.cat([cut(x.k, L) for x, L in zip(xs, lengths)])
-    v = torch.cat([cut(x.v, L) for x, L in zip(xs, lengths)])
-    gates = torch.cat([cut(x.gates, L) for x, L in zip(xs, lengths)])
-    cu = torch.tensor([0] + list(torch.tensor(lengths).cumsum(0).tolist()), dtype=torch.int32)
-    return q, k, v, gates, xs[0].w_k, xs[0].w_v, cu
+    x, cu = synth.nsa_varlen_inputs(lengths, hq, hkv, dk, dv, seed=seed)
+    return x.q, x.k, x.v, x.gates, x.w_k, x.w_v, cu
 
 
 def run_varlen(lengths, hq, hkv, dk, dv, top_k, window, seed):

@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libnsa.so")
 
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
 NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
+NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
 EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_forward_varlen",
             "nsa_decode",
@@ -37,6 +38,7 @@ class NsaConfig(ctypes.Structure):
         ("kc_out", ctypes.c_void_p), ("vc_out", ctypes.c_void_p),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("n_stage_events", ctypes.c_int32),
+        ("score_map", ctypes.c_int32),
     ]
 
 

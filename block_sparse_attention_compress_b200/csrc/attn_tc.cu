@@ -187,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                const __grid_constant__ CUtensorMap tm_vc, const __nv_bfloat16* __restrict__ gates,
                float* __restrict__ acc, int32_t* __restrict__ idx_out, int B, int T, int Hq, int Hkv, int nc,
-               int top_k, int force_first, int force_local, float scale_log2, const int32_t* __restrict__ cu_in,
-               int* __restrict__ err) {
+               int top_k, int force_first, int force_local, float scale_log2, float w_straddle,
+               const int32_t* __restrict__ cu_in, int* __restrict__ err) {
   using SM = Smem<DK, DV>;
   const int32_t* cu = VARLEN ? cu_in : nullptr;
   extern __shared__ uint8_t smem_raw[];
@@ -571,7 +571,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             h2 = __floats2bfloat162_rn(p2, p3);
             pk[8 * kk + j / 2 + 1] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          tok_sum[kk] = sacc;
+          // block i = this thread's r straddles two selection blocks when i % 4 == 3
+          tok_sum[kk] = (lane & 3) == 3 ? sacc * w_straddle : sacc;
         }
         {
           const int j0 = n * (kBlk / 4) + q4 * 8;    // first selection block of this warp
@@ -700,7 +701,7 @@ cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   auto kernel = a.cu ? attn_tc_kernel<DK, DV, true> : attn_tc_kernel<DK, DV, false>;
   kernel<<<grid, kThreads, SM::kAlloc, st>>>(
       mq, mk, mv, static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, a.B, a.T, a.Hq, a.Hkv, a.nc, a.top_k,
-      a.force_first, a.force_local, a.scale_log2, a.cu, a.err);
+      a.force_first, a.force_local, a.scale_log2, a.w_straddle, a.cu, a.err);
   return cudaGetLastError();
 }
 }  // namespace

@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 cmp_select_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
                   const __nv_bfloat16* __restrict__ vc, const __nv_bfloat16* __restrict__ gates,
                   float* __restrict__ acc, int32_t* __restrict__ idx_out, int T, int Hq, int Hkv, int G, int nc,
-                  int top_k, int force_first, int force_local, float scale_log2) {
+                  int top_k, int force_first, int force_local, float scale_log2, float w_straddle) {
   using SM = Smem<DK, DV>;
   using SwzK = SwzTile<DK>;
   using SwzV = SwzTile<DV>;
@@ -235,9 +235,9 @@ cmp_select_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
         c0 += __shfl_xor_sync(0xffffffffu, c0, off);
         c1 += __shfl_xor_sync(0xffffffffu, c1, off);
       }
-      if (lane < 4) {
+      if (lane < 4) {   // block 2*lane + 1 (mod 4) straddles two selection blocks when lane is odd
         cs[j * 8 + 2 * lane] = c0;
-        cs[j * 8 + 2 * lane + 1] = c1;
+        cs[j * 8 + 2 * lane + 1] = (lane & 1) ? c1 * w_straddle : c1;
       }
     }
     __syncwarp();
@@ -331,7 +331,7 @@ cudaError_t launch(const FwdArgs& a, cudaStream_t st) {
   cmp_select_kernel<DK, DV><<<grid, kThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.kc),
       static_cast<const __nv_bfloat16*>(a.vc), static_cast<const __nv_bfloat16*>(a.gates), a.acc, a.idx, a.T,
-      a.Hq, a.Hkv, a.G, a.nc, a.top_k, a.force_first, a.force_local, a.scale_log2);
+      a.Hq, a.Hkv, a.G, a.nc, a.top_k, a.force_first, a.force_local, a.scale_log2, a.w_straddle);
   return cudaGetLastError();
 }
 }  // namespace

@@ -275,7 +275,7 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
               const __nv_bfloat16* __restrict__ vccache, const int32_t* __restrict__ seqlens,
               const __nv_bfloat16* __restrict__ gates, __nv_bfloat16* __restrict__ out, int32_t* __restrict__ idx_out,
               int Lmax, int Ncmax, int max_seqlen, int Hq, int Hkv, int G, int top_k, int window, int force_first,
-              int force_local, float scale_log2) {
+              int force_local, float scale_log2, float w_straddle) {
   using SM = Smem<DK, DV>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -346,7 +346,9 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int jb = 4 * it + 2 * nt + (cq >> 1);
-        float a0 = s[nt][0] + s[nt][1], a1 = s[nt][2] + s[nt][3];
+        // local index 2*cq + 1 (mod 4) straddles two selection blocks when cq is odd
+        const float w1 = (cq & 1) ? w_straddle : 1.f;
+        float a0 = s[nt][0] + w1 * s[nt][1], a1 = s[nt][2] + w1 * s[nt][3];
         a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
         a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
         if ((cq & 1) == 0) {
@@ -359,8 +361,8 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
       for (int nt = 0; nt < 2; ++nt) {
         const int jb = 4 * it + 2 * nt + (cq >> 1) + 1;
         if (cq & 1) {
-          if (rv0) part[gl * kJ + jb] += s[nt][1];
-          if (rv1) part[(gl + 8) * kJ + jb] += s[nt][3];
+          if (rv0) part[gl * kJ + jb] += w_straddle * s[nt][1];
+          if (rv1) part[(gl + 8) * kJ + jb] += w_straddle * s[nt][3];
         }
       }
       pv_tile<DV>(s, cur.v, st.o, lane);
@@ -521,7 +523,7 @@ cudaError_t launch(const DecodeArgs& a, cudaStream_t st) {
       static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.kc),
       static_cast<const __nv_bfloat16*>(a.vc), a.seqlens, static_cast<const __nv_bfloat16*>(a.gates),
       static_cast<__nv_bfloat16*>(a.out), a.idx, a.Lmax, a.Ncmax, a.max_seqlen, a.Hq, a.Hkv, a.G, a.top_k, a.window,
-      a.force_first, a.force_local, a.scale_log2);
+      a.force_first, a.force_local, a.scale_log2, a.w_straddle);
   return cudaGetLastError();
 }
 }  // namespace

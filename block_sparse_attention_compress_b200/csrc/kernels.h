@@ -32,6 +32,10 @@ struct FwdArgs {
   int top_k, window, force_first, force_local;
   float scale_log2;   // softmax scale * log2(e)
   int* err;           // device word, zeroed before the launches; nonzero = a bounded wait timed out
+  // Weight of the compressed blocks that straddle two selection blocks (i % 4 == 3 for l = 32,
+  // s = 16, b = 64) in each of the two: 1 (touch), 0 (contained) or 0.5 (overlap).  The others
+  // lie inside one selection block and count fully there.
+  float w_straddle = 1.f;
   // Variable-length batch: cu[b] .. cu[b+1] are sequence b's rows of q, k, v, gates, acc and out
   // (device, [B + 1], cu[0] = 0, lengths <= T); nullptr = B sequences of T tokens each.  Kc/Vc
   // and idx keep their per-sequence layouts with T as the (maximum) length.
@@ -74,6 +78,7 @@ struct DecodeArgs {
   int B, Lmax, Ncmax, max_seqlen, Hq, Hkv, G, dk, dv;
   int top_k, window, force_first, force_local;
   float scale_log2;
+  float w_straddle = 1.f;   // as in FwdArgs
 };
 
 // K6: one decode step per sequence, all branches in one launch.

@@ -32,6 +32,7 @@ nsa_status check_cfg(const nsa_config* c) {
   if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return NSA_ERR_INVALID_ARG;
   if (c->mode == NSA_MODE_NSA) {
     if (c->cmp_block < 1 || c->cmp_stride < 1 || c->window < 1) return NSA_ERR_INVALID_ARG;
+    if (c->score_map < NSA_MAP_TOUCH || c->score_map > NSA_MAP_OVERLAP) return NSA_ERR_INVALID_ARG;
     if ((c->force_first != 0 && c->force_first != 1) || (c->force_local != 0 && c->force_local != 1))
       return NSA_ERR_INVALID_ARG;
     if (c->top_k < 1 || c->top_k < c->force_first + c->force_local) return NSA_ERR_INVALID_ARG;
@@ -78,6 +79,11 @@ nsa_status check_workspace(const nsa_config* c, size_t need) {
   if (!c->workspace || (reinterpret_cast<uintptr_t>(c->workspace) % kAlign)) return NSA_ERR_WORKSPACE;
   if (c->workspace_bytes < need) return NSA_ERR_WORKSPACE;
   return NSA_OK;
+}
+
+// Weight, in each of its two selection blocks, of a compressed block that straddles them.
+float straddle_weight(const nsa_config* c) {
+  return c->score_map == NSA_MAP_CONTAINED ? 0.f : c->score_map == NSA_MAP_OVERLAP ? 0.5f : 1.f;
 }
 
 nsa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? NSA_OK : NSA_ERR_CUDA; }
@@ -134,6 +140,7 @@ nsa_status nsa_forward_impl(const void* q, const void* k, const void* v, const v
   a.err = reinterpret_cast<int*>(ws + L.err);
   a.cu = cu;
   a.total = total;
+  a.w_straddle = straddle_weight(cfg);
 
   StageMarks marks(cfg, 5);
   cudaError_t e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
@@ -279,6 +286,7 @@ nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache, c
   a.force_first = cfg->force_first; a.force_local = cfg->force_local;
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.w_straddle = straddle_weight(cfg);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   st = check_workspace(cfg, kAlign);
   if (st != NSA_OK) return st;

@@ -17,7 +17,8 @@ class NSAForward:
     """Prefill forward with a reusable workspace (one allocation per shape)."""
 
     def __init__(self, B, T, h_q, h_kv, d_k, d_v, w_k, w_v, *, top_k=16, window=512, sel_block=64,
-                 force_first=1, force_local=1, softmax_scale=0.0, keep_idx=True, keep_kc=True, device="cuda"):
+                 force_first=1, force_local=1, softmax_scale=0.0, keep_idx=True, keep_kc=True, device="cuda",
+                 score_map=0):
         self.shape = (B, T, h_q, h_kv, d_k, d_v)
         nc = n_cmp(T)
         self.idx = torch.empty((B, h_kv, T, top_k), dtype=torch.int32, device=device) if keep_idx else None
@@ -27,7 +28,7 @@ class NSAForward:
         self.cfg = make_config(mode=NSA_MODE_NSA, batch=B, seqlen=T, h_q=h_q, h_kv=h_kv, d_k=d_k, d_v=d_v,
                                top_k=top_k, window=window, sel_block=sel_block, force_first=force_first,
                                force_local=force_local, softmax_scale=softmax_scale, w_cmp_k=w_k, w_cmp_v=w_v,
-                               sel_idx_out=self.idx, kc_out=self.kc, vc_out=self.vc)
+                               sel_idx_out=self.idx, kc_out=self.kc, vc_out=self.vc, score_map=score_map)
         nbytes = nsa_workspace_size(self.cfg)
         if nbytes == 0:
             raise ValueError("nsa_workspace_size rejected the configuration")

@@ -53,6 +53,17 @@ typedef enum {
   NSA_MODE_MOBA = 1   /* MoBA: mean-pooled block keys, per-head top-k plus the own block */
 } nsa_mode;
 
+/* How the probabilities of the compressed blocks (span [s*i, s*i+l)) add up into the score of
+ * a selection block (span [b*j, b*j+b)) when the two block sizes differ.  The method's
+ * description says only that the selection scores come from the compressed attention
+ * ([BLOG] "Deepseek 的论文核心点"); it fixes no mapping for l = 32, s = 16, b = 64. */
+typedef enum {
+  NSA_MAP_TOUCH = 0,      /* every compressed block adds its whole probability to each
+                             selection block its span meets (the default) */
+  NSA_MAP_CONTAINED = 1,  /* only the compressed blocks that lie inside a selection block count */
+  NSA_MAP_OVERLAP = 2     /* each adds its probability times the fraction of its span inside */
+} nsa_score_map;
+
 /*
  * Problem description.  Fields marked (NSA) are ignored in MoBA mode.
  *
@@ -93,6 +104,7 @@ typedef enum {
  *                 combine) and 5 in MoBA mode (block means, selection, query lists,
  *                 past-block attention, own block + merge); nsa_decode has 1.
  *                 NULL or too few: nothing is recorded.
+ *   score_map     (NSA) nsa_score_map; 0 (NSA_MAP_TOUCH) when left zero.
  */
 typedef struct {
   int32_t mode;
@@ -109,6 +121,7 @@ typedef struct {
   size_t workspace_bytes;
   void* const* stage_events;
   int32_t n_stage_events;
+  int32_t score_map;
 } nsa_config;
 
 /* Bytes of workspace nsa_forward (decode_batch == 0) or nsa_decode (decode_batch > 0) needs

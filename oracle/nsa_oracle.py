@@ -27,7 +27,10 @@ listed as R1..R14 in the docstring of the function that applies it:
   R3  the score of 64-token selection block j is the sum of the probabilities
       of every visible compressed block whose span [s*i, s*i+l) intersects
       [b*j, b*j+b) ("parity unpinned": the pages fix no mapping when the
-      block sizes differ).
+      block sizes differ).  The two other readings are kept as options:
+      "contained" (only the compressed blocks that lie inside one selection
+      block count) and "overlap" (each counts with the fraction of its span
+      inside the selection block).
   R4  the group sums post-softmax probabilities (each head normalised over
       its own visible compressed blocks).
   R5  block 0 and the query's own block are always selected and count toward
@@ -132,28 +135,44 @@ def attend(Q: torch.Tensor, Kx: torch.Tensor, Vx: torch.Tensor, scale: float):
 # a2-a5 for one query token and one GQA group
 # --------------------------------------------------------------------------
 
-def selection_scores(p_cmp: torch.Tensor, t: int, l: int, s: int, b: int) -> torch.Tensor:
+SCORE_MAPS = ("touch", "contained", "overlap")   # the library's NSA_MAP_* order
+
+
+def selection_scores(p_cmp: torch.Tensor, t: int, l: int, s: int, b: int,
+                     mapping: str = "touch") -> torch.Tensor:
     """a3, block importance for the selection branch.
 
     [BLOG] "Deepseek 的论文核心点": the selection scores come straight from the
     compressed attention.  [NOTES] §8: the heads of one GQA group add their
     block-selection scores before one shared top-k.  R3/R4: every visible
     compressed block i adds its probability (summed over the group's heads)
-    to each selection block j whose span [b*j, b*j+b) meets [s*i, s*i+l).
+    to each selection block j whose span [b*j, b*j+b) meets [s*i, s*i+l),
+    with weight 1 ("touch"); 1 if the span lies inside block j alone, else 0
+    ("contained"); or the fraction of the span inside block j ("overlap").
 
     p_cmp: [G, n_vis] -> scores [t//b + 1]."""
+    if mapping not in SCORE_MAPS:
+        raise ValueError(mapping)
     nb = t // b + 1
     score = torch.zeros(nb, dtype=F64)
     if p_cmp.shape[1] == 0:
         return score
     per_block = p_cmp.sum(dim=0)                       # group sum
     i = torch.arange(per_block.shape[0])
-    first = (s * i) // b                                # first selection block touched
-    last = (s * i + l - 1) // b                         # last selection block touched
+    start, end = s * i, s * i + l                       # span [start, end)
+    first = start // b                                  # first selection block touched
+    last = (end - 1) // b                               # last selection block touched
     for off in range(int((last - first).max()) + 1):
         j = first + off
         hit = j <= last
-        score.index_add_(0, j[hit], per_block[hit])
+        if mapping == "touch":
+            w = torch.ones_like(per_block)
+        elif mapping == "contained":
+            w = (first == last).to(F64)
+        else:
+            inside = torch.minimum(end, b * (j + 1)) - torch.maximum(start, b * j)
+            w = inside.to(F64) / l
+        score.index_add_(0, j[hit], (w * per_block)[hit])
     return score
 
 
@@ -191,7 +210,7 @@ def window_tokens(t: int, w: int) -> torch.Tensor:
 
 
 def nsa_token(Qg, K, V, Kc, Vc, gates_g, t, *, l, s, b, k, w, scale,
-              force_first=True, force_local=True, idx=None):
+              force_first=True, force_local=True, idx=None, score_map="touch"):
     """All three branches of one query token for one GQA group.
 
     Qg: [G, d_k] the group's query rows; K, V: [>=t+1, d] this KV head's
@@ -201,7 +220,7 @@ def nsa_token(Qg, K, V, Kc, Vc, gates_g, t, *, l, s, b, k, w, scale,
     Returns dict(out, o_cmp, o_slc, o_win, idx, score)."""
     n_vis = num_visible_cmp_blocks(t, l, s, Kc.shape[0])
     o_cmp, p_cmp = attend(Qg, Kc[:n_vis], Vc[:n_vis], scale)          # a2
-    score = selection_scores(p_cmp, t, l, s, b)                      # a3
+    score = selection_scores(p_cmp, t, l, s, b, score_map)           # a3
     if idx is None:
         idx = select_blocks(score, t, b, k, force_first, force_local)
     sel = block_tokens(idx, t, b)
@@ -219,7 +238,7 @@ def nsa_token(Qg, K, V, Kc, Vc, gates_g, t, *, l, s, b, k, w, scale,
 def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
                 sel_block=64, top_k=16, window=512, force_first=True,
                 force_local=True, scale=None, tokens=None, round_kc=True,
-                keep_branches=False):
+                keep_branches=False, score_map="touch"):
     """NSA prefill forward over the query positions ``tokens`` (all by default).
 
     q [B,T,H_q,d_k], k [B,T,H_kv,d_k], v [B,T,H_kv,d_v], gates [B,T,H_q,3],
@@ -251,7 +270,8 @@ def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
             for n_i, t in enumerate(toks):
                 r = nsa_token(q[bi, t, hs], k[bi, :, g], v[bi, :, g], kc[bi, :, g], vc[bi, :, g],
                               gates[bi, t, hs], t, l=l, s=s, b=b, k=top_k, w=window,
-                              scale=scale, force_first=force_first, force_local=force_local)
+                              scale=scale, force_first=force_first, force_local=force_local,
+                              score_map=score_map)
                 out[bi, n_i, hs] = r["out"]
                 idx[bi, g, n_i] = torch.tensor(r["idx"])
                 scores[bi][g][n_i] = r["score"]
@@ -270,7 +290,7 @@ def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
 
 def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, gates, *,
                cmp_block=32, cmp_stride=16, sel_block=64, top_k=16, window=512,
-               force_first=True, force_local=True, scale=None, batch=None):
+               force_first=True, force_local=True, scale=None, batch=None, score_map="touch"):
     """One decode step.  [NOTES] §13: decoding reads the KV cache once per
     step; R11: sequence b's cache holds seqlens[b] tokens including the new
     one, whose position is t = seqlens[b] - 1.  The compressed caches are
@@ -301,7 +321,7 @@ def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, gates, *,
             r = nsa_token(q[bi, hs], _f64(k_cache[bi, :L, g]), _f64(v_cache[bi, :L, g]),
                           _f64(kc_cache[bi, :nc, g]), _f64(vc_cache[bi, :nc, g]),
                           gates[bi, hs], t, l=l, s=s, b=b, k=top_k, w=window, scale=scale,
-                          force_first=force_first, force_local=force_local)
+                          force_first=force_first, force_local=force_local, score_map=score_map)
             out[n_i, hs] = r["out"]
             idx[n_i, g] = torch.tensor(r["idx"])
             row.append(r["score"])

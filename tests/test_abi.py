@@ -49,6 +49,7 @@ def test_config_layout_matches_header():
       F(mode) F(batch) F(seqlen) F(h_q) F(h_kv) F(d_k) F(d_v) F(cmp_block) F(cmp_stride) F(sel_block)
       F(top_k) F(window) F(force_first) F(force_local) F(softmax_scale) F(w_cmp_k) F(w_cmp_v)
       F(sel_idx_out) F(kc_out) F(vc_out) F(workspace) F(workspace_bytes) F(stage_events) F(n_stage_events)
+      F(score_map)
       return 0;
     }
     """
@@ -190,3 +191,9 @@ def test_forward_varlen_rejects_bad_arguments(lib):
     assert call(moba, total=64) == nsa.NSA_ERR_UNSUPPORTED
     c.workspace_bytes = 16
     assert call(c, total=64) == nsa.NSA_ERR_WORKSPACE
+
+
+def test_unknown_score_map_is_rejected(lib):
+    c = _cfg(score_map=3)
+    assert nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0x40000, c, 0x50000, check=False) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_workspace_size(_cfg(score_map=-1)) == 0

@@ -19,7 +19,7 @@ def _lib():
     build.build()
 
 
-def run_decode(d, seqlens, top_k, window, Lmax=None):
+def run_decode(d, seqlens, top_k, window, Lmax=None, score_map=0):
     B, L, hkv, dk = d.k_cache.shape
     hq, dv = d.q.shape[1], d.v_cache.shape[3]
     dev = lambda t: t.to(DEV)
@@ -28,7 +28,7 @@ def run_decode(d, seqlens, top_k, window, Lmax=None):
     idx = torch.full((B, hkv, top_k), -7, dtype=torch.int32, device=DEV)
     out = torch.empty((B, hq, dv), dtype=torch.bfloat16, device=DEV)
     cfg = nsa.make_config(batch=B, seqlen=L, h_q=hq, h_kv=hkv, d_k=dk, d_v=dv, top_k=top_k, window=window,
-                          w_cmp_k=d.w_k, w_cmp_v=d.w_v, sel_idx_out=idx)
+                          w_cmp_k=d.w_k, w_cmp_v=d.w_v, sel_idx_out=idx, score_map=score_map)
     ws = torch.empty(max(nsa.nsa_workspace_size(cfg, B), 4), dtype=torch.uint8, device=DEV)
     cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
     sl = dev(seqlens.to(torch.int32))
@@ -38,14 +38,14 @@ def run_decode(d, seqlens, top_k, window, Lmax=None):
     return out.cpu(), idx.cpu()
 
 
-def check(d, seqlens, top_k, window, batch=None):
-    out, idx = run_decode(d, seqlens, top_k, window)
+def check(d, seqlens, top_k, window, batch=None, score_map=0):
+    out, idx = run_decode(d, seqlens, top_k, window, score_map=score_map)
     bs = list(range(d.q.shape[0])) if batch is None else batch
     sub = lambda t: t[bs]
     kc = oracle.compress_cache(sub(d.k_cache), d.w_k, 32, 16)
     vc = oracle.compress_cache(sub(d.v_cache), d.w_v, 32, 16)
     ref = oracle.nsa_decode(sub(d.q), sub(d.k_cache), sub(d.v_cache), kc, vc, seqlens[bs], sub(d.gates),
-                            top_k=top_k, window=window)
+                            top_k=top_k, window=window, score_map=oracle.SCORE_MAPS[score_map])
     toks = [int(seqlens[b]) - 1 for b in bs]
     gi = idx[bs]
     hq, hkv = d.q.shape[1], d.k_cache.shape[2]
@@ -119,3 +119,10 @@ def test_decode_workload_sampled():
             if sw:
                 mask[i, g * G:(g + 1) * G] = False
     assert_close(out[bs], ref["out"], mask=mask.unsqueeze(-1).expand(-1, -1, out.shape[-1]), what="decode 64K")
+
+
+@pytest.mark.parametrize("score_map", [1, 2])
+def test_decode_score_maps(score_map):
+    """The contained and overlap readings of the compressed-to-selection mapping in decode."""
+    d = synth.decode_inputs(4, 2100, 64, 4, 192, 128, seed=63)
+    check(d, torch.tensor([2100, 1500, 95, 1025], dtype=torch.int32), 16, 512, score_map=score_map)

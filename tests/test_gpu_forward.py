@@ -29,13 +29,14 @@ def run_gpu(x, top_k, window, gates=None, **kw):
     return out.cpu(), f.idx.cpu(), f.kc.cpu(), f.vc.cpu()
 
 
-def check_against_oracle(x, top_k, window, tokens=None, gates=None, min_exact=0.97):
+def check_against_oracle(x, top_k, window, tokens=None, gates=None, min_exact=0.97, score_map=0):
     B, T, hq, dk = x.q.shape
     hkv = x.k.shape[2]
     G = hq // hkv
     g = x.gates if gates is None else gates
-    out, idx, kc, vc = run_gpu(x, top_k, window, gates=g)
-    ref = oracle.nsa_forward(x.q, x.k, x.v, g, x.w_k, x.w_v, top_k=top_k, window=window, tokens=tokens)
+    out, idx, kc, vc = run_gpu(x, top_k, window, gates=g, score_map=score_map)
+    ref = oracle.nsa_forward(x.q, x.k, x.v, g, x.w_k, x.w_v, top_k=top_k, window=window, tokens=tokens,
+                             score_map=oracle.SCORE_MAPS[score_map])
     toks = ref["tokens"]
     assert_phi_close(kc, x.k, x.w_k, "kc")
     assert_phi_close(vc, x.v, x.w_v, "vc")
@@ -182,3 +183,19 @@ def test_prefill_64k_sampled():
     c = synth.WORKLOADS["nsa_64k"]
     x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=0)
     check_against_oracle(x, c["top_k"], c["window"], tokens=sampled_tokens(c["T"], 90, 2))
+
+
+@pytest.mark.parametrize("score_map", [1, 2])
+def test_score_maps_tensor_core_path(score_map):
+    """The other readings of the compressed-to-selection mapping (contained, overlap) on the
+    tensor-core compressed kernel: ragged T, two groups of 16 heads."""
+    x = synth.nsa_inputs(1, 1001, 32, 2, 192, 128, seed=61)
+    check_against_oracle(x, 16, 256, score_map=score_map)
+
+
+@pytest.mark.parametrize("score_map", [1, 2])
+def test_score_maps_warp_mma_path(score_map):
+    """The same on the warp-MMA compressed kernel (4 heads per group, d = 64)."""
+    c = synth.WORKLOADS["nsa_tiny"]
+    x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=62)
+    check_against_oracle(x, c["top_k"], c["window"], score_map=score_map)

@@ -60,12 +60,12 @@ def test_visibility_off_by_one_is_caught(monkeypatch):
 
 def test_single_head_scores_are_caught(monkeypatch):
     real = O.selection_scores
-    monkeypatch.setattr(O, "selection_scores", lambda p, t, l, s, b: real(p[:1], t, l, s, b))
+    monkeypatch.setattr(O, "selection_scores", lambda p, t, l, s, b, mapping="touch": real(p[:1], t, l, s, b, mapping))
     assert _caught(pins.test_nsa_handworked_closed_forms)
 
 
 def test_contained_only_mapping_is_caught(monkeypatch):
-    def bad(p, t, l, s, b):
+    def bad(p, t, l, s, b, mapping="touch"):
         nb = t // b + 1
         score = torch.zeros(nb, dtype=O.F64)
         ph = p.sum(0)

@@ -379,3 +379,42 @@ def test_moba_selection_is_best_subset_per_head_and_keeps_own_block():
             rows.append(sel)
         per_head_differs |= rows[0] != rows[1]
     assert per_head_differs
+
+
+# ---------------------------------------------------------------- score mappings (R3 and its alternatives)
+
+@pytest.mark.parametrize("mapping,inside,straddle", [
+    ("touch", [0, 1, 0], [1, 1, 0]),
+    ("contained", [0, 1, 0], [0, 0, 0]),
+    ("overlap", [0, 1, 0], [0.5, 0.5, 0]),
+])
+def test_score_maps_on_single_blocks(mapping, inside, straddle):
+    """l = 32, s = 16, b = 64: compressed block 4 spans [64, 96), inside selection block 1;
+    block 3 spans [48, 80), half in block 0 and half in block 1."""
+    t = 150   # 9 visible compressed blocks, selection blocks 0..2
+    p = torch.zeros(1, 9, dtype=torch.float64)
+    p[0, 4] = 1.0
+    assert oracle.selection_scores(p, t, 32, 16, 64, mapping).tolist() == inside
+    p.zero_()
+    p[0, 3] = 1.0
+    assert oracle.selection_scores(p, t, 32, 16, 64, mapping).tolist() == straddle
+
+
+def test_score_maps_order_and_overlap_keeps_the_mass():
+    """Overlap splits each probability exactly (the scores add up to the total); contained <=
+    overlap <= touch block by block; touch counts every straddling block twice."""
+    g = torch.Generator().manual_seed(5)
+    t = 1000
+    n = oracle.num_visible_cmp_blocks(t, 32, 16, 10**6)
+    p = torch.rand(4, n, generator=g, dtype=torch.float64)
+    p /= p.sum(dim=1, keepdim=True)
+    sc = {m: oracle.selection_scores(p, t, 32, 16, 64, m) for m in oracle.SCORE_MAPS}
+    assert torch.allclose(sc["overlap"].sum(), p.sum())
+    assert (sc["contained"] <= sc["overlap"] + 1e-15).all() and (sc["overlap"] <= sc["touch"] + 1e-15).all()
+    straddling = p.sum(dim=0)[3::4].sum()
+    assert torch.allclose(sc["touch"].sum() - sc["contained"].sum(), 2 * straddling)
+
+
+def test_unknown_score_map_is_rejected():
+    with pytest.raises(ValueError):
+        oracle.selection_scores(torch.ones(1, 4, dtype=torch.float64), 100, 32, 16, 64, "nearest")

@@ -39,6 +39,9 @@ class NsaConfig(ctypes.Structure):
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("stage_events", ctypes.POINTER(ctypes.c_void_p)), ("n_stage_events", ctypes.c_int32),
         ("score_map", ctypes.c_int32),
+        ("phi_mlp", ctypes.c_int32),
+        ("w_cmp_k2", ctypes.c_void_p), ("w_cmp_v2", ctypes.c_void_p),
+        ("b_cmp_k", ctypes.c_void_p), ("b_cmp_v", ctypes.c_void_p),
     ]
 
 
@@ -112,7 +115,8 @@ def make_config(**fields) -> NsaConfig:
                     force_first=1, force_local=1, softmax_scale=0.0)
     defaults.update(fields)
     for name, val in defaults.items():
-        if name in ("w_cmp_k", "w_cmp_v", "sel_idx_out", "kc_out", "vc_out", "workspace"):
+        if name in ("w_cmp_k", "w_cmp_v", "sel_idx_out", "kc_out", "vc_out", "workspace", "w_cmp_k2", "w_cmp_v2",
+                    "b_cmp_k", "b_cmp_v"):
             val = _ptr(val)
         setattr(cfg, name, val)
     return cfg

@@ -10,6 +10,9 @@
 // the windows, each at the one window its newest token completes (or none).  A row's
 // arithmetic (k chunks in order, the same MMA fragments) does not depend on which rows share
 // its CTA, so every block equals bitwise the one the full compression computes.
+// MLP mode (phi as a two-layer MLP): the first layer is this GEMM with the epilogue
+// GELU(acc + bias) (MLP1), stored in bf16; the second layer is this GEMM again over the hidden
+// rows with a "block" of one row (l = s = 1).
 // Variable-length batch (cu != nullptr): sequence b's tokens are rows cu[b] .. cu[b+1] of x
 // and its n_cmp(cu[b+1] - cu[b]) blocks go to out[b, 0 .. ); its rows from there up to nc are
 // zeroed, so that a reader of whole 128-row tiles (masked past the sequence) only ever
@@ -24,11 +27,13 @@ constexpr int kBM = 64, kBN = 64, kBK = 64, kThreads = 128;
 
 // STAGES-deep cp.async ring of (A, W) k-chunks: 2 when the grid is large enough to hide the
 // loads' latency; more for the append launch, whose few CTAs each run one long k chain.
-template <int D, int DOUT, int STAGES, bool APPEND>
+__device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
+
+template <int D, int DOUT, int STAGES, bool APPEND, bool MLP1 = false>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
                 int l, int s, int nc, __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ seqlens,
-                int B, const int32_t* __restrict__ cu) {
+                int B, const int32_t* __restrict__ cu, const __nv_bfloat16* __restrict__ bias = nullptr) {
   extern __shared__ __align__(128) uint8_t csmem[];
   auto sA = reinterpret_cast<__nv_bfloat16(*)[kBM * kBK]>(csmem);                          // [STAGES]
   auto sB = reinterpret_cast<__nv_bfloat16(*)[kBK * kBN]>(csmem + STAGES * kBM * kBK * 2);  // [STAGES]
@@ -140,8 +145,13 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
     __nv_bfloat16* dst = out + (((size_t)row_seq(row) * nc + i) * H + h) * DOUT + n0;
 #pragma unroll
     for (int j = 0; j < kBN / 8; ++j) {
-      const uint32_t v = pack_bf16(acc[j][2 * half], acc[j][2 * half + 1]);
-      *reinterpret_cast<uint32_t*>(dst + j * 8 + 2 * cq) = v;
+      float v0 = acc[j][2 * half], v1 = acc[j][2 * half + 1];
+      if constexpr (MLP1) {
+        const int col = n0 + j * 8 + 2 * cq;
+        v0 = gelu(v0 + __bfloat162float(bias[col]));
+        v1 = gelu(v1 + __bfloat162float(bias[col + 1]));
+      }
+      *reinterpret_cast<uint32_t*>(dst + j * 8 + 2 * cq) = pack_bf16(v0, v1);
     }
   }
 }
@@ -175,7 +185,34 @@ cudaError_t launch_append(const void* x, const void* w, const int32_t* seqlens, 
                                                    static_cast<__nv_bfloat16*>(out), seqlens, B, nullptr);
   return cudaGetLastError();
 }
+template <int D>
+cudaError_t launch_mlp(const void* x, const void* w1, const void* b1, const void* w2, int B, int T, int H, int l,
+                       int s, int nc, void* hidden, void* out, cudaStream_t st, const int32_t* cu) {
+  dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
+  compress_kernel<D, D, 2, false, true><<<grid, kThreads, smem_bytes(2), st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w1), T, H, l, s, nc,
+      static_cast<__nv_bfloat16*>(hidden), nullptr, B, cu, static_cast<const __nv_bfloat16*>(b1));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // second layer: every hidden row is a "block" of one row
+  compress_kernel<D, D, 2, false, false><<<grid, kThreads, smem_bytes(2), st>>>(
+      static_cast<const __nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(w2), nc, H, 1, 1, nc,
+      static_cast<__nv_bfloat16*>(out), nullptr, B, nullptr);
+  return cudaGetLastError();
+}
 }  // namespace
+
+cudaError_t launch_compress_mlp(const void* x, const void* w1, const void* b1, const void* w2, int B, int T, int H,
+                                int d, int l, int s, void* hidden, void* out, cudaStream_t st, const int32_t* cu) {
+  const int nc = T < l ? 0 : (T - l) / s + 1;
+  if (nc == 0 || B == 0 || H == 0) return cudaSuccess;
+  switch (d) {
+    case 64: return launch_mlp<64>(x, w1, b1, w2, B, T, H, l, s, nc, hidden, out, st, cu);
+    case 128: return launch_mlp<128>(x, w1, b1, w2, B, T, H, l, s, nc, hidden, out, st, cu);
+    case 192: return launch_mlp<192>(x, w1, b1, w2, B, T, H, l, s, nc, hidden, out, st, cu);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,
                                    int d, int l, int s, int ncmax, void* out, cudaStream_t st) {

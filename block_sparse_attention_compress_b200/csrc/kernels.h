@@ -13,6 +13,11 @@ namespace nsa {
 cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,
                             cudaStream_t st,
                             const int32_t* cu = nullptr);
+// K1 with phi as a two-layer MLP: hidden = bf16(GELU(vec(block) @ w1 + b1)) [B, nc, H, d],
+// out = bf16(hidden @ w2) [B, nc, H, d] (hidden width d; w1 [l*d, d], b1 [d], w2 [d, d]).
+cudaError_t launch_compress_mlp(const void* x, const void* w1, const void* b1, const void* w2, int B, int T, int H,
+                                int d, int l, int s, void* hidden, void* out, cudaStream_t st,
+                                const int32_t* cu = nullptr);
 // K1 for a growing cache: for each sequence b whose newest token (L = seqlens[b], clamped
 // to Lmax) completes window i = (L - l)/s < ncmax, out[b, i, h, :] for every head.
 cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,

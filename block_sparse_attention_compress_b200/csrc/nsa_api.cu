@@ -33,6 +33,11 @@ nsa_status check_cfg(const nsa_config* c) {
   if (c->mode == NSA_MODE_NSA) {
     if (c->cmp_block < 1 || c->cmp_stride < 1 || c->window < 1) return NSA_ERR_INVALID_ARG;
     if (c->score_map < NSA_MAP_TOUCH || c->score_map > NSA_MAP_OVERLAP) return NSA_ERR_INVALID_ARG;
+    if (c->phi_mlp != 0 && c->phi_mlp != 1) return NSA_ERR_INVALID_ARG;
+    if (c->phi_mlp &&
+        (!c->w_cmp_k2 || !c->w_cmp_v2 || !c->b_cmp_k || !c->b_cmp_v || !aligned16(c->w_cmp_k2) ||
+         !aligned16(c->w_cmp_v2) || !aligned16(c->b_cmp_k) || !aligned16(c->b_cmp_v)))
+      return NSA_ERR_INVALID_ARG;
     if ((c->force_first != 0 && c->force_first != 1) || (c->force_local != 0 && c->force_local != 1))
       return NSA_ERR_INVALID_ARG;
     if (c->top_k < 1 || c->top_k < c->force_first + c->force_local) return NSA_ERR_INVALID_ARG;
@@ -53,7 +58,7 @@ nsa_status check_cfg(const nsa_config* c) {
 }
 
 struct FwdLayout {
-  size_t err, kc, vc, idx, acc, total;
+  size_t err, kc, vc, idx, acc, hk, hv, total;   // hk, hv: the MLP's hidden rows (phi_mlp only)
 };
 
 FwdLayout forward_layout(const nsa_config* c) {
@@ -65,6 +70,10 @@ FwdLayout forward_layout(const nsa_config* c) {
   L.vc = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
   L.idx = off; off = align_up(off + B * c->h_kv * T * c->top_k * 4);
   L.acc = off; off = align_up(off + B * T * c->h_q * c->d_v * 4);
+  if (c->phi_mlp) {
+    L.hk = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
+    L.hv = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
+  }
   L.total = off;
   return L;
 }
@@ -145,11 +154,16 @@ nsa_status nsa_forward_impl(const void* q, const void* k, const void* v, const v
   StageMarks marks(cfg, 5);
   cudaError_t e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
   if (e == cudaSuccess) e = marks.mark(s);
+  const int l = cfg->cmp_block, st = cfg->cmp_stride;
   if (e == cudaSuccess)
-    e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, kc, s, cu);
+    e = cfg->phi_mlp ? nsa::launch_compress_mlp(k, cfg->w_cmp_k, cfg->b_cmp_k, cfg->w_cmp_k2, a.B, a.T, a.Hkv, a.dk, l,
+                                                st, ws + L.hk, kc, s, cu)
+                     : nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, l, st, kc, s, cu);
   if (e == cudaSuccess) e = marks.mark(s);
   if (e == cudaSuccess)
-    e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, cfg->cmp_block, cfg->cmp_stride, vc, s, cu);
+    e = cfg->phi_mlp ? nsa::launch_compress_mlp(v, cfg->w_cmp_v, cfg->b_cmp_v, cfg->w_cmp_v2, a.B, a.T, a.Hkv, a.dv, l,
+                                                st, ws + L.hv, vc, s, cu)
+                     : nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, l, st, vc, s, cu);
   if (e == cudaSuccess) e = marks.mark(s);
   if (e == cudaSuccess) e = nsa::launch_cmp_select(a, s);
   if (e == cudaSuccess) e = marks.mark(s);

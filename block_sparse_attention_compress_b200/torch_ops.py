@@ -18,7 +18,9 @@ class NSAForward:
 
     def __init__(self, B, T, h_q, h_kv, d_k, d_v, w_k, w_v, *, top_k=16, window=512, sel_block=64,
                  force_first=1, force_local=1, softmax_scale=0.0, keep_idx=True, keep_kc=True, device="cuda",
-                 score_map=0):
+                 score_map=0, mlp=None):
+        """mlp: dict(b_k, w_k2, b_v, w_v2) of device tensors makes phi the two-layer MLP (w_k and
+        w_v are then its first layers); None keeps the linear phi."""
         self.shape = (B, T, h_q, h_kv, d_k, d_v)
         nc = n_cmp(T)
         self.idx = torch.empty((B, h_kv, T, top_k), dtype=torch.int32, device=device) if keep_idx else None
@@ -29,6 +31,11 @@ class NSAForward:
                                top_k=top_k, window=window, sel_block=sel_block, force_first=force_first,
                                force_local=force_local, softmax_scale=softmax_scale, w_cmp_k=w_k, w_cmp_v=w_v,
                                sel_idx_out=self.idx, kc_out=self.kc, vc_out=self.vc, score_map=score_map)
+        if mlp is not None:
+            self.mlp = mlp   # keep the weights alive as long as the config points at them
+            for name, val in (("phi_mlp", 1), ("w_cmp_k2", mlp["w_k2"].data_ptr()), ("w_cmp_v2", mlp["w_v2"].data_ptr()),
+                              ("b_cmp_k", mlp["b_k"].data_ptr()), ("b_cmp_v", mlp["b_v"].data_ptr())):
+                setattr(self.cfg, name, val)
         nbytes = nsa_workspace_size(self.cfg)
         if nbytes == 0:
             raise ValueError("nsa_workspace_size rejected the configuration")

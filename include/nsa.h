@@ -105,6 +105,19 @@ typedef enum {
  *                 past-block attention, own block + merge); nsa_decode has 1.
  *                 NULL or too few: nothing is recorded.
  *   score_map     (NSA) nsa_score_map; 0 (NSA_MAP_TOUCH) when left zero.
+ *   phi_mlp       (NSA) 0: phi is the linear map above.  1: phi is a two-layer MLP of hidden
+ *                 width d ([BLOG] "Deepseek 的论文核心点": the blocks are compressed with an
+ *                 MLP): for keys
+ *                   hidden = bf16(GELU(vec(K[s*i : s*i+l]) @ w_cmp_k + b_cmp_k)),
+ *                   compressed key i = bf16(hidden @ w_cmp_k2),
+ *                 GELU(x) = x * (1 + erf(x / sqrt(2))) / 2; values alike with the _v weights.
+ *                 w_cmp_k is then the first layer [l*d_k, d_k], b_cmp_k its bias bf16 [d_k],
+ *                 w_cmp_k2 the second layer bf16 [d_k, d_k] (values: d_v).  An intra-block
+ *                 position embedding pe [l, d] added to every block before the first layer is
+ *                 exactly the bias b = vec(pe) @ w_cmp_k.  Only nsa_forward and
+ *                 nsa_forward_varlen take phi_mlp = 1 (nsa_compress, nsa_compress_append and
+ *                 nsa_decode work on the linear phi or on caches the caller compressed).
+ *   w_cmp_k2, w_cmp_v2, b_cmp_k, b_cmp_v   (NSA, phi_mlp = 1) as above, 16-byte aligned.
  */
 typedef struct {
   int32_t mode;
@@ -122,6 +135,11 @@ typedef struct {
   void* const* stage_events;
   int32_t n_stage_events;
   int32_t score_map;
+  int32_t phi_mlp;
+  const void* w_cmp_k2;
+  const void* w_cmp_v2;
+  const void* b_cmp_k;
+  const void* b_cmp_v;
 } nsa_config;
 
 /* Bytes of workspace nsa_forward (decode_batch == 0) or nsa_decode (decode_batch > 0) needs

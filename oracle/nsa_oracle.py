@@ -46,6 +46,10 @@ listed as R1..R14 in the docstring of the function that applies it:
       the mean of the block's keys; top-k past blocks plus the own block.
   R14 compressed K/V are stored as bf16 tensors (like every K/V tensor of the
       method); ``round_kc=True`` rounds phi's output accordingly.
+  R15 phi as an MLP (an option; [BLOG] "Deepseek 的论文核心点" says the blocks are
+      compressed by an MLP): two layers of hidden width d with GELU between,
+      a bias on the first layer, hidden values stored in bf16.  An intra-block
+      position embedding added before the first layer is that bias.
 """
 from __future__ import annotations
 
@@ -101,15 +105,39 @@ def phi_compress(X: torch.Tensor, W: torch.Tensor, l: int, s: int) -> torch.Tens
     return blocks @ W
 
 
+def gelu(x: torch.Tensor) -> torch.Tensor:
+    """GELU with the exact normal CDF: x * (1 + erf(x / sqrt(2))) / 2."""
+    return 0.5 * x * (1.0 + torch.erf(x / math.sqrt(2.0)))
+
+
+def phi_mlp(X: torch.Tensor, W1: torch.Tensor, b1: torch.Tensor, W2: torch.Tensor, l: int, s: int,
+            round_hidden: bool = True) -> torch.Tensor:
+    """R15: phi as a two-layer MLP of one sequence and KV head.
+
+    Row i is GELU(vec(X[s*i : s*i+l]) @ W1 + b1) @ W2, the hidden values rounded
+    to bf16 where the library stores them (``round_hidden``).
+
+    X: [T, d]; W1: [l*d, h]; b1: [h]; W2: [h, d_out] -> [N_c, d_out] (fp64)."""
+    hidden = gelu(phi_compress(X, W1, l, s) + _f64(b1))
+    if round_hidden:
+        hidden = round_bf16(hidden)
+    return hidden @ _f64(W2)
+
+
 def compress_cache(K: torch.Tensor, W: torch.Tensor, l: int, s: int,
-                   round_kc: bool = True) -> torch.Tensor:
-    """phi over every (batch, KV head): K [B, T, H, d] -> [B, N_c, H, d_out]."""
+                   round_kc: bool = True, mlp=None) -> torch.Tensor:
+    """phi over every (batch, KV head): K [B, T, H, d] -> [B, N_c, H, d_out].
+    ``mlp`` = (b1, W2) makes phi the two-layer MLP of R15 with W as its first layer."""
     B, T, H, _ = K.shape
     n = num_cmp_blocks(T, l, s)
-    out = torch.zeros((B, n, H, W.shape[1]), dtype=F64)
+    d_out = W.shape[1] if mlp is None else mlp[1].shape[1]
+    out = torch.zeros((B, n, H, d_out), dtype=F64)
     for b in range(B):
         for h in range(H):
-            out[b, :, h] = phi_compress(K[b, :, h], W, l, s)
+            if mlp is None:
+                out[b, :, h] = phi_compress(K[b, :, h], W, l, s)
+            else:
+                out[b, :, h] = phi_mlp(K[b, :, h], W, mlp[0], mlp[1], l, s, round_hidden=round_kc)
     return round_bf16(out) if round_kc else out
 
 
@@ -238,12 +266,15 @@ def nsa_token(Qg, K, V, Kc, Vc, gates_g, t, *, l, s, b, k, w, scale,
 def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
                 sel_block=64, top_k=16, window=512, force_first=True,
                 force_local=True, scale=None, tokens=None, round_kc=True,
-                keep_branches=False, score_map="touch"):
+                keep_branches=False, score_map="touch", mlp=None):
     """NSA prefill forward over the query positions ``tokens`` (all by default).
 
     q [B,T,H_q,d_k], k [B,T,H_kv,d_k], v [B,T,H_kv,d_v], gates [B,T,H_q,3],
     w_k [l*d_k,d_k], w_v [l*d_v,d_v].  Query head h belongs to group
     h // (H_q // H_kv) ([EN], GQA paragraph; [NOTES] §7).
+
+    ``mlp`` = dict(b_k, w_k2, b_v, w_v2) makes phi the two-layer MLP of R15
+    (w_k, w_v are then its first layers); ``score_map`` picks the R3 reading.
 
     Returns a dict with fp64 ``out`` [B, n_tok, H_q, d_v], int ``idx``
     [B, H_kv, n_tok, top_k], ``score`` (list per (b, g, token) of the block
@@ -256,8 +287,8 @@ def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
     l, s, b = cmp_block, cmp_stride, sel_block
     scale = 1.0 / math.sqrt(dk) if scale is None else scale                 # R10
     toks = list(range(T)) if tokens is None else [int(t) for t in tokens]
-    kc = compress_cache(k, w_k, l, s, round_kc)
-    vc = compress_cache(v, w_v, l, s, round_kc)
+    kc = compress_cache(k, w_k, l, s, round_kc, None if mlp is None else (mlp["b_k"], mlp["w_k2"]))
+    vc = compress_cache(v, w_v, l, s, round_kc, None if mlp is None else (mlp["b_v"], mlp["w_v2"]))
     n = len(toks)
     out = torch.zeros((B, n, Hq, dv), dtype=F64)
     idx = torch.full((B, Hkv, n, top_k), -1, dtype=torch.long)

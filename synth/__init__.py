@@ -115,6 +115,16 @@ def decode_inputs(B: int, L: int, h_q: int, h_kv: int, d_k: int, d_v: int,
     return DecodeInputs(q, k, v, w_k, w_v, gates, seqlens)
 
 
+def phi_mlp_weights(l: int, d: int, seed: int = 0, device="cpu"):
+    """Weights of phi as a two-layer MLP of hidden width d: w1 ~ N(0, 1/(l*d)) [l*d, d],
+    b1 ~ N(0, 0.1^2) [d], w2 ~ N(0, 1/d) [d, d]; drawn in that order in fp32, rounded to bf16."""
+    g = _gen(seed, device)
+    w1 = _randn(g, (l * d, d), device, 1.0 / math.sqrt(l * d)).to(torch.bfloat16)
+    b1 = _randn(g, (d,), device, 0.1).to(torch.bfloat16)
+    w2 = _randn(g, (d, d), device, 1.0 / math.sqrt(d)).to(torch.bfloat16)
+    return w1, b1, w2
+
+
 def nsa_varlen_inputs(lengths, h_q: int, h_kv: int, d_k: int, d_v: int, cmp_block: int = 32, seed: int = 0,
                       device="cpu"):
     """A packed variable-length batch: sequence i is its own draw of nsa_inputs(1, L_i, ...)

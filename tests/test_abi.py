@@ -49,7 +49,7 @@ def test_config_layout_matches_header():
       F(mode) F(batch) F(seqlen) F(h_q) F(h_kv) F(d_k) F(d_v) F(cmp_block) F(cmp_stride) F(sel_block)
       F(top_k) F(window) F(force_first) F(force_local) F(softmax_scale) F(w_cmp_k) F(w_cmp_v)
       F(sel_idx_out) F(kc_out) F(vc_out) F(workspace) F(workspace_bytes) F(stage_events) F(n_stage_events)
-      F(score_map)
+      F(score_map) F(phi_mlp) F(w_cmp_k2) F(w_cmp_v2) F(b_cmp_k) F(b_cmp_v)
       return 0;
     }
     """
@@ -197,3 +197,16 @@ def test_unknown_score_map_is_rejected(lib):
     c = _cfg(score_map=3)
     assert nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0x40000, c, 0x50000, check=False) == nsa.NSA_ERR_INVALID_ARG
     assert nsa.nsa_workspace_size(_cfg(score_map=-1)) == 0
+
+
+def test_phi_mlp_needs_its_weights(lib):
+    base = dict(workspace=0x100000, workspace_bytes=1 << 30)
+    assert nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0x40000, _cfg(phi_mlp=1, **base), 0x50000,
+                           check=False) == nsa.NSA_ERR_INVALID_ARG
+    misaligned = _cfg(phi_mlp=1, w_cmp_k2=0x3000, w_cmp_v2=0x4000, b_cmp_k=0x5008, b_cmp_v=0x6000, **base)
+    assert nsa.nsa_forward(0x10000, 0x20000, 0x30000, 0x40000, misaligned, 0x50000,
+                           check=False) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_workspace_size(_cfg(phi_mlp=2)) == 0
+    lin = nsa.nsa_workspace_size(_cfg())
+    mlp = nsa.nsa_workspace_size(_cfg(phi_mlp=1, w_cmp_k2=0x3000, w_cmp_v2=0x4000, b_cmp_k=0x5000, b_cmp_v=0x6000))
+    assert mlp > lin   # the hidden rows

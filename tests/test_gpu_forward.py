@@ -199,3 +199,36 @@ def test_score_maps_warp_mma_path(score_map):
     c = synth.WORKLOADS["nsa_tiny"]
     x = synth.nsa_inputs(c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"], seed=62)
     check_against_oracle(x, c["top_k"], c["window"], score_map=score_map)
+
+
+def _mlp_weights(dk, dv, seed):
+    w_k, b_k, w_k2 = synth.phi_mlp_weights(32, dk, seed=seed)
+    w_v, b_v, w_v2 = synth.phi_mlp_weights(32, dv, seed=seed + 1)
+    return (w_k, w_v), dict(b_k=b_k, w_k2=w_k2, b_v=b_v, w_v2=w_v2)
+
+
+@pytest.mark.parametrize("shape", [(1, 1001, 32, 2, 192, 128), (1, 1024, 4, 1, 64, 64)])
+def test_phi_mlp_forward(shape):
+    """phi as a two-layer MLP (GELU, hidden width d): the compressed keys/values against the
+    oracle's MLP, then the whole forward (tensor-core and warp-MMA compressed kernels)."""
+    B, T, hq, hkv, dk, dv = shape
+    x = synth.nsa_inputs(B, T, hq, hkv, dk, dv, seed=64)
+    (w_k, w_v), mlp = _mlp_weights(dk, dv, seed=65)
+    top_k, window = (16, 256) if hq // hkv == 16 else (4, 128)
+    dev = [t.to(DEV) for t in (x.q, x.k, x.v, x.gates, w_k, w_v)]
+    f = NSAForward(B, T, hq, hkv, dk, dv, dev[4], dev[5], top_k=top_k, window=window,
+                   mlp={n: t.to(DEV) for n, t in mlp.items()})
+    out = f(*dev[:4])
+    torch.cuda.synchronize()
+    assert f.device_status() == 0
+    kc_ref = oracle.compress_cache(x.k, w_k, 32, 16, True, (mlp["b_k"], mlp["w_k2"]))
+    vc_ref = oracle.compress_cache(x.v, w_v, 32, 16, True, (mlp["b_v"], mlp["w_v2"]))
+    assert_close(f.kc.cpu(), kc_ref, max_abs=3e-2, mean_abs=2e-3, what="mlp kc")
+    assert_close(f.vc.cpu(), vc_ref, max_abs=3e-2, mean_abs=2e-3, what="mlp vc")
+    ref = oracle.nsa_forward(x.q, x.k, x.v, x.gates, w_k, w_v, top_k=top_k, window=window, mlp=mlp)
+    toks = ref["tokens"]
+    gi = f.idx.cpu()[:, :, toks]
+    exact, swapped = idx_agreement(gi, ref["idx"], ref["score"], tokens=toks)
+    assert exact >= 0.97 * gi.numel() / gi.shape[-1]
+    mask = token_mask((B, len(toks), hq), swapped, hq // hkv)
+    assert_close(out.cpu()[:, toks], ref["out"], mask=mask.unsqueeze(-1).expand(-1, -1, -1, dv), what="mlp out")

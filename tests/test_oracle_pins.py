@@ -418,3 +418,46 @@ def test_score_maps_order_and_overlap_keeps_the_mass():
 def test_unknown_score_map_is_rejected():
     with pytest.raises(ValueError):
         oracle.selection_scores(torch.ones(1, 4, dtype=torch.float64), 100, 32, 16, 64, "nearest")
+
+
+# ---------------------------------------------------------------- phi as a two-layer MLP (R15)
+
+def test_gelu_matches_the_library_routine():
+    x = torch.linspace(-8, 8, 1001, dtype=torch.float64)
+    assert torch.allclose(oracle.gelu(x), torch.nn.functional.gelu(x), atol=1e-14, rtol=0)
+
+
+def test_phi_mlp_matches_bruteforce_and_position_term_is_the_bias():
+    """Block by block with explicit loops, and an intra-block position embedding added to the
+    keys equals the bias vec(pe) @ W1 (the identity the library relies on)."""
+    g = torch.Generator().manual_seed(7)
+    T, d, l, s, h = 70, 8, 32, 16, 8
+    X = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(l * d, h, generator=g, dtype=torch.float64) / 16
+    W2 = torch.randn(h, d, generator=g, dtype=torch.float64) / 3
+    pe = torch.randn(l, d, generator=g, dtype=torch.float64)
+    b1 = pe.reshape(-1) @ W1
+    got = oracle.phi_mlp(X, W1, b1, W2, l, s, round_hidden=False)
+    n = (T - l) // s + 1
+    assert got.shape == (n, d)
+    for i in range(n):
+        z = torch.zeros(h, dtype=torch.float64)
+        for r in range(l):
+            for c in range(d):
+                z += (X[s * i + r, c] + pe[r, c]) * W1[r * d + c]
+        hid = 0.5 * z * (1 + torch.erf(z / math.sqrt(2)))
+        assert torch.allclose(got[i], hid @ W2, atol=1e-12, rtol=0)
+
+
+def test_phi_mlp_reduces_to_the_linear_phi_in_the_linear_regime():
+    """With a large bias the GELU is the identity up to exp(-b^2/2): the MLP becomes the linear
+    phi with W1 @ W2 plus the constant (b1 @ W2)."""
+    g = torch.Generator().manual_seed(8)
+    T, d, l, s = 64, 4, 32, 16
+    X = torch.randn(T, d, generator=g, dtype=torch.float64)
+    W1 = torch.randn(l * d, d, generator=g, dtype=torch.float64) / 100
+    W2 = torch.randn(d, d, generator=g, dtype=torch.float64)
+    b1 = torch.full((d,), 20.0, dtype=torch.float64)
+    got = oracle.phi_mlp(X, W1, b1, W2, l, s, round_hidden=False)
+    want = oracle.phi_compress(X, W1 @ W2, l, s) + b1 @ W2
+    assert torch.allclose(got, want, atol=1e-9, rtol=0)

@@ -313,6 +313,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         result["varlen"] = run_varlen_bench(args, dev, world)
         result["gpu_launches"] += result["varlen"]["gpu_launches"]
+    if not args.no_phi_mlp:
+        torch.cuda.empty_cache()
+        result["phi_mlp"] = run_phi_mlp_bench(args, dev, world)
+        result["gpu_launches"] += result["phi_mlp"]["gpu_launches"]
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         r, info = oracle_rate(cpu_workload(), args.ref_sample, seed=7, threads=os.cpu_count() or 1)
         result["cpu_baseline"] = {"value": r, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
@@ -499,6 +503,50 @@ def run_varlen_bench(args, dev, world):
             "gpu_launches": len(STAGES) * args.steps}
 
 
+def run_phi_mlp_bench(args, dev, world):
+    """The 64K forward with phi as the two-layer MLP (hidden width d): its two phi stages and
+    the step time (stage times from the library's events)."""
+    from block_sparse_attention_compress_b200.torch_ops import NSAForward
+    c = synth.WORKLOADS["nsa_64k"]
+    B, T, hq, hkv, dk, dv = c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"]
+    x = synth.nsa_inputs(B, T, hq, hkv, dk, dv, seed=0, device=dev)
+    w_k, b_k, w_k2 = synth.phi_mlp_weights(32, dk, seed=1, device=dev)
+    w_v, b_v, w_v2 = synth.phi_mlp_weights(32, dv, seed=2, device=dev)
+    f = NSAForward(B, T, hq, hkv, dk, dv, w_k, w_v, top_k=c["top_k"], window=c["window"], device=dev,
+                   mlp=dict(b_k=b_k, w_k2=w_k2, b_v=b_v, w_v2=w_v2))
+    out = torch.empty((B, T, hq, dv), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    nstage = len(STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nstage)] for _ in range(args.steps)]
+    for es in evs:
+        for e in es:
+            e.record()
+    torch.cuda.synchronize()
+    handles = [ctypes_array(es) for es in evs]
+    for _ in range(args.warmup):
+        flush.zero_()
+        f.cfg.stage_events, f.cfg.n_stage_events = None, 0
+        f(x.q, x.k, x.v, x.gates, out)
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        f.cfg.stage_events, f.cfg.n_stage_events = handles[i][0], nstage
+        f(x.q, x.k, x.v, x.gates, out)
+    torch.cuda.synchronize()
+    assert f.device_status() == 0, "a device-side wait timed out"
+    step_ms = allreduce_max(statistics.mean(es[0].elapsed_time(es[-1]) for es in evs), world, dev)
+    stages = {n: statistics.mean(es[j].elapsed_time(es[j + 1]) for es in evs) for j, n in enumerate(STAGES)}
+    nc = (T - 32) // 16 + 1
+    flops = 2.0 * B * nc * hkv * (32 * dk * dk + dk * dk + 32 * dv * dv + dv * dv)
+    phi_ms = stages["phi_k"] + stages["phi_v"]
+    return {"workload": "nsa_64k with phi as a two-layer MLP (GELU, hidden width d)",
+            "ms_per_step": step_ms, "phi_ms": round(phi_ms, 4),
+            "phi_tflops": flops / (phi_ms * 1e-3) / 1e12,
+            "stages_ms": {n: round(v, 4) for n, v in stages.items()},
+            "gpu_launches": (len(STAGES) + 2) * args.steps}
+
+
 def run_e2e(args, f, x, out, dev, world):
     """Same step through the public API with inputs in pinned host memory: H2D copies of
     q, k, v, gates, the forward, and the D2H copy of the output, all inside the timed region."""
@@ -564,6 +612,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-moba", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-phi-mlp", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -214,9 +214,9 @@ def workload_config(c, name):
 # compressed cache stay mostly in L2.  An entry goes back to None whenever its kernel
 # changes, until it is captured again.
 NCU_DRAM_BYTES_PER_ITEM = {
-    "cmp_select": (205.893888e6 + 217.393408e6) / 32768,
-    "slc_attn": (501.284608e6 + 229.739008e6) / 32768,
-    "swa_combine": None,   # changed since its capture
+    "cmp_select": (205.892864e6 + 216.708352e6) / 32768,
+    "slc_attn": (501.060352e6 + 229.711616e6) / 32768,
+    "swa_combine": (494.174976e6 + 118.646784e6) / 32768,
 }
 
 

@@ -15,11 +15,11 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnsa.so")
 
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
-NSA_MODE_NSA, NSA_MODE_MOBA = 0, 1
+NSA_MODE_NSA, NSA_MODE_MOBA, NSA_MODE_DSA = 0, 1, 2
 NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
 EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_forward_varlen",
-            "nsa_decode",
+            "nsa_dsa_forward", "nsa_decode",
             "nsa_forward_noalloc", "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
 
 
@@ -71,6 +71,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_compress_append.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     lib.nsa_compress_append.restype = ctypes.c_int
     lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
+    lib.nsa_dsa_forward.restype = ctypes.c_int
+    lib.nsa_dsa_forward.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, cfgp, vp, vp, vp]
     lib.nsa_forward_varlen.restype = ctypes.c_int
     lib.nsa_forward_varlen.argtypes = [vp, vp, vp, vp, vp, i32, cfgp, vp, vp]
     lib.nsa_forward.restype = ctypes.c_int
@@ -165,6 +167,15 @@ def nsa_forward_varlen(q, k, v, gates, cu_seqlens, cfg: NsaConfig, out, stream=N
     st = load_library().nsa_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(cu_seqlens),
                                            int(q.shape[0]), ctypes.byref(cfg), _ptr(out), _stream(stream, q))
     return _check(st, "nsa_forward_varlen") if check else st
+
+
+def nsa_dsa_forward(q, k, v, q_idx, k_idx, w_idx, cfg: NsaConfig, out, sel_out=None, stream=None,
+                    check: bool = True) -> int:
+    """DSA forward (cfg.mode = NSA_MODE_DSA): indexer heads and dim from q_idx's shape."""
+    st = load_library().nsa_dsa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(k_idx), _ptr(w_idx),
+                                        int(q_idx.shape[-2]), int(q_idx.shape[-1]), ctypes.byref(cfg), _ptr(out),
+                                        _ptr(sel_out), _stream(stream, q))
+    return _check(st, "nsa_dsa_forward") if check else st
 
 
 def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, max_seqlen: int, gates, cfg: NsaConfig, out,

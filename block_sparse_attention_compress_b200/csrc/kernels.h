@@ -86,6 +86,24 @@ struct DecodeArgs {
   float w_straddle = 1.f;   // as in FwdArgs
 };
 
+// DSA: token-wise sparse attention behind a lightning indexer.
+struct DsaArgs {
+  const void* q;      // [B, T, Hq, dk]
+  const void* k;      // [B, T, Hkv, dk]
+  const void* v;      // [B, T, Hkv, dv]
+  const void* qi;     // [B, T, hi, di] indexer queries
+  const void* ki;     // [B, T, di] indexer keys
+  const void* wi;     // [B, T, hi] indexer head weights
+  void* out;          // [B, T, Hq, dv]
+  int32_t* sel;       // [B, T, top_k] chosen tokens, ascending, -1 padded
+  float* scores;      // [B, T, T] indexer scores (entries s <= t)
+  int B, T, Hq, Hkv, G, dk, dv, hi, di, top_k;
+  float scale_log2;
+};
+cudaError_t launch_dsa_indexer(const DsaArgs& a, cudaStream_t st);
+cudaError_t launch_dsa_topk(const DsaArgs& a, cudaStream_t st);
+cudaError_t launch_dsa_attn(const DsaArgs& a, cudaStream_t st);
+
 // K6: one decode step per sequence, all branches in one launch.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 

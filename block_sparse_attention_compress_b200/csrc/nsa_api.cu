@@ -10,7 +10,9 @@
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr int kMaxTokensNsa = 65536;   // 1024 selection blocks per token (top-k kept in shared memory)
+constexpr int kMaxTokensNsa = 65536;
+constexpr int kMaxTokensDsa = 32768;   // the [T, T] fp32 score matrix: 4 GB per sequence at this length
+constexpr int kMaxDsaTopk = 8192;   // 1024 selection blocks per token (top-k kept in shared memory)
 constexpr int kMaxTokensMoba = 1 << 20;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -24,7 +26,7 @@ bool dims_supported(int dk, int dv) {
 // Shape checks common to every entry point.  Returns NSA_OK or the error to report.
 nsa_status check_cfg(const nsa_config* c) {
   if (!c) return NSA_ERR_INVALID_ARG;
-  if (c->mode != NSA_MODE_NSA && c->mode != NSA_MODE_MOBA) return NSA_ERR_INVALID_ARG;
+  if (c->mode != NSA_MODE_NSA && c->mode != NSA_MODE_MOBA && c->mode != NSA_MODE_DSA) return NSA_ERR_INVALID_ARG;
   if (c->batch < 1 || c->seqlen < 1 || c->h_q < 1 || c->h_kv < 1 || c->d_k < 1 || c->d_v < 1)
     return NSA_ERR_INVALID_ARG;
   if (c->h_q % c->h_kv) return NSA_ERR_INVALID_ARG;
@@ -47,6 +49,11 @@ nsa_status check_cfg(const nsa_config* c) {
     if (c->cmp_block != 32 || c->cmp_stride != 16 || c->sel_block != 64) return NSA_ERR_UNSUPPORTED;
     if (c->h_q / c->h_kv > 16 || !dims_supported(c->d_k, c->d_v) || c->top_k > 32) return NSA_ERR_UNSUPPORTED;
     if (c->seqlen > kMaxTokensNsa) return NSA_ERR_UNSUPPORTED;
+  } else if (c->mode == NSA_MODE_DSA) {
+    if (c->top_k < 1) return NSA_ERR_INVALID_ARG;
+    if (c->h_q / c->h_kv > 16 || !dims_supported(c->d_k, c->d_v) || c->top_k > kMaxDsaTopk ||
+        c->seqlen > kMaxTokensDsa)
+      return NSA_ERR_UNSUPPORTED;
   } else {
     if (c->h_q != c->h_kv || c->d_k != c->d_v) return NSA_ERR_INVALID_ARG;
     if (c->d_k != 128 || c->sel_block % 64 || c->top_k > 7 || c->seqlen > kMaxTokensMoba) return NSA_ERR_UNSUPPORTED;
@@ -78,8 +85,25 @@ FwdLayout forward_layout(const nsa_config* c) {
   return L;
 }
 
+// DSA workspace: status word, the [B, T, T] fp32 scores, the [B, T, top_k] chosen tokens.
+struct DsaLayout {
+  size_t err, scores, sel, total;
+};
+
+DsaLayout dsa_layout(const nsa_config* c) {
+  const size_t B = c->batch, T = c->seqlen;
+  DsaLayout L{};
+  size_t off = 0;
+  L.err = off; off = align_up(off + 4);
+  L.scores = off; off = align_up(off + B * T * T * 4);
+  L.sel = off; off = align_up(off + B * T * (size_t)c->top_k * 4);
+  L.total = off;
+  return L;
+}
+
 size_t workspace_bytes(const nsa_config* c) {
   if (c->mode == NSA_MODE_MOBA) return nsa::moba_layout(c->batch, c->seqlen, c->h_q, c->sel_block, c->top_k).total;
+  if (c->mode == NSA_MODE_DSA) return dsa_layout(c).total;
   return forward_layout(c).total;
 }
 
@@ -278,6 +302,43 @@ nsa_status nsa_forward_varlen(const void* q, const void* k, const void* v, const
   st = check_workspace(cfg, workspace_bytes(cfg));
   if (st != NSA_OK) return st;
   return nsa_forward_impl(q, k, v, gates, cfg, out, static_cast<cudaStream_t>(stream), cu_seqlens, total_tokens);
+}
+
+nsa_status nsa_dsa_forward(const void* q, const void* k, const void* v, const void* q_idx, const void* k_idx,
+                           const void* w_idx, int32_t idx_heads, int32_t idx_dim, const nsa_config* cfg, void* out,
+                           int32_t* sel_out, void* stream) {
+  nsa_status st = check_cfg(cfg);
+  if (st != NSA_OK) return st;
+  if (cfg->mode != NSA_MODE_DSA) return NSA_ERR_INVALID_ARG;
+  if (!q || !k || !v || !q_idx || !k_idx || !w_idx || !out) return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) || !aligned16(k_idx) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(w_idx) & 1u) || (sel_out && (reinterpret_cast<uintptr_t>(sel_out) & 3u)))
+    return NSA_ERR_INVALID_ARG;
+  if (idx_heads < 1 || idx_dim < 1) return NSA_ERR_INVALID_ARG;
+  if (idx_heads > 64 || (idx_dim != 64 && idx_dim != 128)) return NSA_ERR_UNSUPPORTED;
+  st = check_workspace(cfg, workspace_bytes(cfg));
+  if (st != NSA_OK) return st;
+  const DsaLayout L = dsa_layout(cfg);
+  auto ws = static_cast<uint8_t*>(cfg->workspace);
+  nsa::DsaArgs a{};
+  a.q = q; a.k = k; a.v = v; a.qi = q_idx; a.ki = k_idx; a.wi = w_idx; a.out = out;
+  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel);
+  a.scores = reinterpret_cast<float*>(ws + L.scores);
+  a.B = cfg->batch; a.T = cfg->seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
+  a.dk = cfg->d_k; a.dv = cfg->d_v; a.hi = idx_heads; a.di = idx_dim; a.top_k = cfg->top_k;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  StageMarks marks(cfg, 3);
+  cudaError_t e = cudaMemsetAsync(ws + L.err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_dsa_indexer(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_dsa_topk(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  if (e == cudaSuccess) e = nsa::launch_dsa_attn(a, s);
+  if (e == cudaSuccess) e = marks.mark(s);
+  return from_cuda(e);
 }
 
 nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_cache, const void* kc_cache,

@@ -50,7 +50,8 @@ typedef enum {
 
 typedef enum {
   NSA_MODE_NSA = 0,   /* compressed + selected + sliding-window branches, gated sum */
-  NSA_MODE_MOBA = 1   /* MoBA: mean-pooled block keys, per-head top-k plus the own block */
+  NSA_MODE_MOBA = 1,  /* MoBA: mean-pooled block keys, per-head top-k plus the own block */
+  NSA_MODE_DSA = 2    /* DSA: lightning-indexer scores, token-wise top-k (nsa_dsa_forward only) */
 } nsa_mode;
 
 /* How the probabilities of the compressed blocks (span [s*i, s*i+l)) add up into the score of
@@ -209,6 +210,29 @@ NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, cons
 NSA_API nsa_status nsa_forward_varlen(const void* q, const void* k, const void* v, const void* gates,
                                       const int32_t* cu_seqlens, int32_t total_tokens, const nsa_config* cfg,
                                       void* out, void* stream);
+
+/*
+ * nsa_dsa_forward -- token-wise sparse attention behind a lightning indexer (DSA; 10100.com,
+ * "机器之心PRO · 会员通讯 Week 45", "Which Attention is All You Need?", section "Linear v.s.
+ * Sparse", point 6: a light indexer scores every earlier token, the k best are kept, and full
+ * attention runs over them).  cfg->mode = NSA_MODE_DSA; used fields: batch, seqlen, h_q, h_kv,
+ * d_k, d_v, top_k (1 .. 8192), softmax_scale, workspace.
+ *   q bf16 [B, T, H_q, d_k];  k [B, T, H_kv, d_k];  v [B, T, H_kv, d_v]
+ *   q_idx bf16 [B, T, idx_heads, idx_dim]   indexer queries (idx_heads 1 .. 64)
+ *   k_idx bf16 [B, T, idx_dim]              indexer keys, one per token (idx_dim 64 or 128)
+ *   w_idx bf16 [B, T, idx_heads]            indexer head weights
+ *   out   bf16 [B, T, H_q, d_v]
+ *   sel_out int32 [B, T, top_k] (optional): the chosen tokens, ascending, -1 padded.
+ * For every token t: score[s] = sum_j w_idx[t, j] * ReLU(q_idx[t, j] . k_idx[s]) for s <= t
+ * (fp32); the top_k keys by score (ties to the lower index; all of them when t + 1 <= top_k);
+ * per query head, softmax attention over the chosen tokens (its GQA group's K/V).
+ * Workspace: nsa_workspace_size(cfg, 0) bytes (it holds the [B, T, T] fp32 score matrix).
+ * Shapes: G = h_q / h_kv <= 16, (d_k, d_v) as nsa_forward, T <= 32768.  Status codes as for
+ * nsa_forward.
+ */
+NSA_API nsa_status nsa_dsa_forward(const void* q, const void* k, const void* v, const void* q_idx,
+                                   const void* k_idx, const void* w_idx, int32_t idx_heads, int32_t idx_dim,
+                                   const nsa_config* cfg, void* out, int32_t* sel_out, void* stream);
 
 /*
  * nsa_decode -- one decode step per sequence ([NOTES] §13: decoding is bound by

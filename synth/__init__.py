@@ -115,6 +115,31 @@ def decode_inputs(B: int, L: int, h_q: int, h_kv: int, d_k: int, d_v: int,
     return DecodeInputs(q, k, v, w_k, w_v, gates, seqlens)
 
 
+@dataclasses.dataclass
+class DsaInputs:
+    q: torch.Tensor          # [B, T, H_q, d_k] bf16
+    k: torch.Tensor          # [B, T, H_kv, d_k] bf16
+    v: torch.Tensor          # [B, T, H_kv, d_v] bf16
+    q_idx: torch.Tensor      # [B, T, H_I, d_I] bf16
+    k_idx: torch.Tensor      # [B, T, d_I] bf16
+    w_idx: torch.Tensor      # [B, T, H_I] bf16
+
+
+def dsa_inputs(B: int, T: int, h_q: int, h_kv: int, d_k: int, d_v: int, h_i: int, d_i: int, seed: int = 0,
+               device="cpu") -> DsaInputs:
+    """q, k (with the 64-token key offsets), v as for NSA, then the indexer tensors: q_idx ~ N(0, 1),
+    k_idx ~ N(0, 1) plus its own per-64-token offset ~ N(0, 0.5^2), w_idx ~ N(0, 1/h_i); drawn in
+    that order in fp32 and rounded to bf16."""
+    g = _gen(seed, device)
+    q = _randn(g, (B, T, h_q, d_k), device).to(torch.bfloat16)
+    k = _keys(g, B, T, h_kv, d_k, device)
+    v = _randn(g, (B, T, h_kv, d_v), device).to(torch.bfloat16)
+    q_idx = _randn(g, (B, T, h_i, d_i), device).to(torch.bfloat16)
+    k_idx = _keys(g, B, T, 1, d_i, device)[:, :, 0].contiguous()
+    w_idx = _randn(g, (B, T, h_i), device, 1.0 / math.sqrt(h_i)).to(torch.bfloat16)
+    return DsaInputs(q, k, v, q_idx, k_idx, w_idx)
+
+
 def phi_mlp_weights(l: int, d: int, seed: int = 0, device="cpu"):
     """Weights of phi as a two-layer MLP of hidden width d: w1 ~ N(0, 1/(l*d)) [l*d, d],
     b1 ~ N(0, 0.1^2) [d], w2 ~ N(0, 1/d) [d, d]; drawn in that order in fp32, rounded to bf16."""

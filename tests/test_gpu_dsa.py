@@ -1,0 +1,76 @@
+"""GPU parity of the DSA forward (nsa_dsa_forward: lightning indexer, token-wise top-k,
+attention over the chosen tokens) against the fp64 oracle on the same seeded inputs."""
+import pytest
+import torch
+
+import block_sparse_attention_compress_b200 as nsa
+import oracle
+import synth
+from block_sparse_attention_compress_b200 import build
+from tests.helpers import assert_close
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+NEAR_TIE = 1e-4   # relative: a chosen token may differ from the oracle's only within this of the k-th score
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build.build()
+
+
+def run_gpu(x, top_k):
+    B, T, hq, dk = x.q.shape
+    hkv, dv = x.k.shape[2], x.v.shape[3]
+    dev = [t.to(DEV) for t in (x.q, x.k, x.v, x.q_idx, x.k_idx, x.w_idx)]
+    cfg = nsa.make_config(mode=nsa.NSA_MODE_DSA, batch=B, seqlen=T, h_q=hq, h_kv=hkv, d_k=dk, d_v=dv, top_k=top_k)
+    ws = torch.empty(nsa.nsa_workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    out = torch.empty((B, T, hq, dv), dtype=torch.bfloat16, device=DEV)
+    sel = torch.full((B, T, top_k), -7, dtype=torch.int32, device=DEV)
+    nsa.nsa_dsa_forward(*dev, cfg, out, sel_out=sel)
+    torch.cuda.synchronize()
+    return out.cpu(), sel.cpu()
+
+
+def check(x, top_k, tokens, min_exact=0.97):
+    out, sel = run_gpu(x, top_k)
+    ref = oracle.dsa_forward(x.q, x.k, x.v, x.q_idx, x.k_idx, x.w_idx, top_k=top_k, tokens=tokens)
+    B = x.q.shape[0]
+    keep = torch.ones(B, len(tokens), dtype=torch.bool)
+    exact = 0
+    for b in range(B):
+        for n, t in enumerate(tokens):
+            a = sel[b, t].tolist()
+            o = ref["idx"][b, n].tolist()
+            m = min(t + 1, top_k)
+            assert a[:m] == sorted(a[:m]) and all(0 <= j <= t for j in a[:m]) and a[m:] == [-1] * (top_k - m), (b, t)
+            assert len(set(a[:m])) == m, (b, t)
+            if a == o:
+                exact += 1
+                continue
+            sc = ref["score"][b][n]
+            kth = sorted(sc.tolist(), reverse=True)[m - 1]
+            eps = NEAR_TIE * max(1.0, abs(kth))
+            for j in set(a[:m]) - set(o[:m]):
+                assert sc[j] >= kth - eps, (b, t, j, float(sc[j]), kth)
+            keep[b, n] = False
+    assert exact >= min_exact * B * len(tokens), exact
+    mask = keep[:, :, None, None].expand(-1, -1, x.q.shape[2], x.v.shape[3])
+    assert_close(out[:, tokens], ref["out"], mask=mask, what="dsa out")
+
+
+def test_dsa_group_of_16():
+    x = synth.dsa_inputs(1, 700, 32, 2, 192, 128, 4, 64, seed=71)
+    check(x, 64, tokens=[0, 1, 5, 63, 64, 65, 200, 411, 699])
+
+
+def test_dsa_small_heads_and_batch():
+    x = synth.dsa_inputs(2, 333, 4, 1, 64, 64, 2, 128, seed=72)
+    check(x, 16, tokens=list(range(0, 333, 7)))
+
+
+def test_dsa_every_token_chosen_is_full_causal_attention():
+    """top_k >= T: the indexer no longer matters; the output is full causal attention."""
+    x = synth.dsa_inputs(1, 130, 16, 1, 128, 128, 3, 64, seed=73)
+    check(x, 256, tokens=list(range(130)), min_exact=1.0)

@@ -313,6 +313,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         result["varlen"] = run_varlen_bench(args, dev, world)
         result["gpu_launches"] += result["varlen"]["gpu_launches"]
+    if not args.no_dsa:
+        torch.cuda.empty_cache()
+        result["dsa"] = run_dsa_bench(args, dev, world)
+        result["gpu_launches"] += result["dsa"]["gpu_launches"]
     if not args.no_phi_mlp:
         torch.cuda.empty_cache()
         result["phi_mlp"] = run_phi_mlp_bench(args, dev, world)
@@ -547,6 +551,59 @@ def run_phi_mlp_bench(args, dev, world):
             "gpu_launches": (len(STAGES) + 2) * args.steps}
 
 
+def dsa_flops(T, h_q, d_k, d_v, h_i, d_i, top_k, B=1):
+    """Indexer: 2 * h_i * d_i per (query, key <= query) pair; attention: 2 * (d_k + d_v) per
+    (query head, chosen token)."""
+    pairs = T * (T + 1) // 2
+    chosen = sum(min(t + 1, top_k) for t in range(T))
+    return {"indexer": 2.0 * B * pairs * h_i * d_i, "attention": 2.0 * B * chosen * h_q * (d_k + d_v)}
+
+
+def run_dsa_bench(args, dev, world):
+    """DSA forward (lightning indexer, token-wise top-k, attention over the chosen tokens)."""
+    import block_sparse_attention_compress_b200 as nsa
+    c = synth.WORKLOADS["dsa_8k"]
+    B, T, hq, hkv, dk, dv, hi, di, K = (c[n] for n in ("B", "T", "h_q", "h_kv", "d_k", "d_v", "h_i", "d_i", "top_k"))
+    x = synth.dsa_inputs(B, T, hq, hkv, dk, dv, hi, di, seed=0, device=dev)
+    cfg = nsa.make_config(mode=nsa.NSA_MODE_DSA, batch=B, seqlen=T, h_q=hq, h_kv=hkv, d_k=dk, d_v=dv, top_k=K)
+    ws = torch.empty(nsa.nsa_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    cfg.workspace, cfg.workspace_bytes = ws.data_ptr(), ws.numel()
+    out = torch.empty((B, T, hq, dv), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    names = ["indexer", "topk", "attention"]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
+    for es in evs:
+        for e in es:
+            e.record()
+    torch.cuda.synchronize()
+    handles = [ctypes_array(es) for es in evs]
+    args_in = (x.q, x.k, x.v, x.q_idx, x.k_idx, x.w_idx)
+    for _ in range(args.warmup):
+        flush.zero_()
+        cfg.stage_events, cfg.n_stage_events = None, 0
+        nsa.nsa_dsa_forward(*args_in, cfg, out)
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        cfg.stage_events, cfg.n_stage_events = handles[i][0], len(names) + 1
+        nsa.nsa_dsa_forward(*args_in, cfg, out)
+    torch.cuda.synchronize()
+    step_ms = allreduce_max(statistics.mean(es[0].elapsed_time(es[-1]) for es in evs), world, dev)
+    stages = {n: statistics.mean(es[j].elapsed_time(es[j + 1]) for es in evs) for j, n in enumerate(names)}
+    fl = dsa_flops(T, hq, dk, dv, hi, di, K, B)
+    peaks, _ = load_peaks()
+    return {"workload": f"dsa_8k: B={B} T={T} h_q={hq} h_kv={hkv} d_k={dk} d_v={dv}, indexer {hi} heads x {di}, "
+                        f"top_k={K}",
+            "ms_per_step": step_ms, "tokens_per_s": world * B * T / (step_ms * 1e-3),
+            "tflops_computed": sum(fl.values()) / (step_ms * 1e-3) / 1e12,
+            "frac_of_bf16_peak": sum(fl.values()) / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "stages_ms": {n: round(v, 4) for n, v in stages.items()},
+            "stage_tflops": {"indexer": round(fl["indexer"] / (stages["indexer"] * 1e-3) / 1e12, 1),
+                             "attention": round(fl["attention"] / (stages["attention"] * 1e-3) / 1e12, 1)},
+            "gpu_launches": len(names) * args.steps}
+
+
 def run_e2e(args, f, x, out, dev, world):
     """Same step through the public API with inputs in pinned host memory: H2D copies of
     q, k, v, gates, the forward, and the D2H copy of the output, all inside the timed region."""
@@ -613,6 +670,7 @@ def main():
     ap.add_argument("--no-moba", action="store_true")
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-phi-mlp", action="store_true")
+    ap.add_argument("--no-dsa", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

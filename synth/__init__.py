@@ -187,6 +187,8 @@ WORKLOADS = {
     "nsa_64k": dict(B=1, T=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512),
     "nsa_decode": dict(B=32, L=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512),
     "moba_128k": dict(B=1, T=131072, h=32, d=128, block=512, top_k=3),
+    # DSA (token-wise sparse attention): 4 indexer heads of 64 dims, 2048 tokens per query
+    "dsa_8k": dict(B=1, T=8192, h_q=64, h_kv=4, d_k=192, d_v=128, h_i=4, d_i=64, top_k=2048),
     # a packed batch of 8 sequences of different lengths, 65536 tokens in all
     "nsa_varlen": dict(lengths=(16384, 12288, 9000, 8192, 7000, 5000, 4096, 3576), h_q=64, h_kv=4, d_k=192,
                        d_v=128, top_k=16, window=512),

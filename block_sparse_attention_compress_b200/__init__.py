@@ -19,7 +19,7 @@ NSA_MODE_NSA, NSA_MODE_MOBA, NSA_MODE_DSA = 0, 1, 2
 NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
 EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_forward_varlen",
-            "nsa_dsa_forward", "nsa_decode",
+            "nsa_dsa_forward", "nsa_backward", "nsa_decode",
             "nsa_forward_noalloc", "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
 
 
@@ -71,6 +71,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_compress_append.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     lib.nsa_compress_append.restype = ctypes.c_int
     lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
+    lib.nsa_backward.restype = ctypes.c_int
+    lib.nsa_backward.argtypes = [vp, vp, vp, vp, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, vp]
     lib.nsa_dsa_forward.restype = ctypes.c_int
     lib.nsa_dsa_forward.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, cfgp, vp, vp, vp]
     lib.nsa_forward_varlen.restype = ctypes.c_int
@@ -167,6 +169,15 @@ def nsa_forward_varlen(q, k, v, gates, cu_seqlens, cfg: NsaConfig, out, stream=N
     st = load_library().nsa_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(cu_seqlens),
                                            int(q.shape[0]), ctypes.byref(cfg), _ptr(out), _stream(stream, q))
     return _check(st, "nsa_forward_varlen") if check else st
+
+
+def nsa_backward(q, k, v, gates, sel_idx, dout, cfg: NsaConfig, dq, dk, dv, dgates, dw_k, dw_v, stream=None,
+                 check: bool = True) -> int:
+    """Gradients of the NSA forward (see include/nsa.h); every gradient buffer is fp32 and written."""
+    st = load_library().nsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(sel_idx), _ptr(dout),
+                                     ctypes.byref(cfg), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgates), _ptr(dw_k),
+                                     _ptr(dw_v), _stream(stream, q))
+    return _check(st, "nsa_backward") if check else st
 
 
 def nsa_dsa_forward(q, k, v, q_idx, k_idx, w_idx, cfg: NsaConfig, out, sel_out=None, stream=None,

@@ -1,0 +1,395 @@
+// Backward of the NSA forward: gradients of q, k, v, the gates and the phi weights from the
+// gradient of the output ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §13: NSA is trained
+// natively, forward and backward; the chosen blocks are a discrete choice with no gradient).
+//
+// bwd_attn_kernel, one CTA per (batch, token t, KV group), 8 warps, the group's G <= 16 heads as
+// the 16 rows of m16n8k16 MMAs.  For each branch (compressed, selected, window), with its gate
+// g and output o (all per head):
+//   pass 1  o and the log-sum-exp of the branch, recomputed (online softmax over its rows);
+//           dgate = dout . o and D = g * (dout . o);
+//   pass 2  per 16-row tile: P = exp(S - lse), dP = g * (dout V^T), dS = P * (dP - D);
+//           dQ += dS K (registers); dK_rows += dS^T Q and dV_rows += (g P)^T dout, added to
+//           the fp32 gradient buffers of the rows (K/V rows, or Kc/Vc rows) with atomics.
+//   dq = scale * dQ, summed over the warps in shared memory.
+// phi's backward (per KV head, keys and values alike):
+//   bwd_phi_dx_kernel  dX[u] += sum over the compressed blocks i covering token u of
+//                      W[(u - s*i)*d : (u - s*i + 1)*d, :] . dXc[i];
+//   bwd_phi_dw_kernel  dW[r*d + c, j] = sum over (b, h, i) of X[b, s*i + r, h, c] * dXc[b, i, h, j].
+// A first version: pass 2 loads each tile and waits for it, and the row gradients are atomics.
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "rows_attn.cuh"
+
+namespace nsa {
+
+namespace {
+constexpr int kL = 32, kS = 16, kSel = 64;
+
+template <int DK, int DV>
+struct BwdSmem {
+  static constexpr size_t kStage = (size_t)kRows * (DK + DV) * 2;            // one tile (K then V)
+  static constexpr size_t kRings = (size_t)kWarps * kStage;                  // one stage per warp
+  static constexpr size_t kMerge = MergeBuf<DV>::kBytes + (size_t)kWarps * 16 * 3 * 4;
+  static constexpr size_t kU = kRings > kMerge ? kRings : kMerge;            // rings / merge scratch
+  static constexpr size_t kQ = kU;                                           // Q bf16 [16][DK]
+  static constexpr size_t kDO = kQ + 16 * DK * 2;                            // dout bf16 [16][DV]
+  static constexpr size_t kX = kDO + 16 * DV * 2;                            // per warp [16][16] bf16
+  static constexpr size_t kO = kX + (size_t)kWarps * 16 * 16 * 2;            // o of the branch [16][DV] fp32
+  static constexpr size_t kDQ = kO + 16 * DV * 4;                            // dq [16][DK] fp32
+  static constexpr size_t kRow = kDQ + 16 * DK * 4;                          // lse, D, gate [16] each
+  static constexpr size_t kTotal = kRow + 3 * 16 * 4;
+  static_assert(kTotal <= 232448, "backward shared memory");
+};
+
+// A = X^T for X [16 rows][16 cols] bf16 (row stride 16): the m16k16 fragment of the transpose.
+__device__ __forceinline__ void load_at(const __nv_bfloat16* X, uint32_t (&a)[4], int lane) {
+  const int mi = lane >> 3, ri = lane & 7;
+  const int row = (mi >> 1) * 8 + ri, col = (mi & 1) * 8;
+  ldsm_x4_t(a[0], a[1], a[2], a[3], smem_u32(X + row * 16 + col));
+}
+
+// out[16][N] += A (16 x 16) . B, B = [16 rows][N] bf16 in the SwzTile<N> layout.
+template <int N>
+__device__ __forceinline__ void mma_ab(const uint32_t (&a)[4], const __nv_bfloat16* B, float (&out)[N / 8][4],
+                                       int lane) {
+#pragma unroll
+  for (int np = 0; np < N / 16; ++np) {
+    uint32_t b0, b1, b2, b3;
+    const int row = lane & 15;
+    const int ch = 2 * np + (lane >> 4);
+    ldsm_x4_t(b0, b1, b2, b3, smem_u32(B + SwzTile<N>::offset(row, ch)));
+    mma16816(out[2 * np], a, b0, b1);
+    mma16816(out[2 * np + 1], a, b2, b3);
+  }
+}
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ kc,
+                const __nv_bfloat16* __restrict__ vc, const __nv_bfloat16* __restrict__ gates,
+                const __nv_bfloat16* __restrict__ dout, const int32_t* __restrict__ idx, float* __restrict__ dq,
+                float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dkc, float* __restrict__ dvc,
+                float* __restrict__ dgates, int T, int Hq, int Hkv, int G, int nc, int top_k, int window,
+                float scale_log2) {
+  using SM = BwdSmem<DK, DV>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + SM::kQ);
+  __nv_bfloat16* sDO = reinterpret_cast<__nv_bfloat16*>(smem + SM::kDO);
+  __nv_bfloat16* sX = reinterpret_cast<__nv_bfloat16*>(smem + SM::kX) + warp * 256;
+  float* sO = reinterpret_cast<float*>(smem + SM::kO);
+  float* sDQ = reinterpret_cast<float*>(smem + SM::kDQ);
+  float* sLse = reinterpret_cast<float*>(smem + SM::kRow);
+  float* sD = sLse + 16;
+  float* sG = sD + 16;
+  const size_t row0 = ((size_t)b * T + t) * Hq + g * G;   // the group's first head row of this token
+  for (int e = tid; e < 16 * (DK / 8); e += kThreads) {
+    const int r = e / (DK / 8), ch = e % (DK / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < G) val = *reinterpret_cast<const uint4*>(q + (row0 + r) * DK + ch * 8);
+    *reinterpret_cast<uint4*>(sQ + SwzTile<DK>::offset(r, ch)) = val;
+  }
+  for (int e = tid; e < 16 * (DV / 8); e += kThreads) {
+    const int r = e / (DV / 8), ch = e % (DV / 8);
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (r < G) val = *reinterpret_cast<const uint4*>(dout + (row0 + r) * DV + ch * 8);
+    *reinterpret_cast<uint4*>(sDO + SwzTile<DV>::offset(r, ch)) = val;
+  }
+  for (int e = tid; e < 16 * DK; e += kThreads) sDQ[e] = 0.f;
+  __syncthreads();
+  uint32_t qf[DK / 16][4], df[DV / 16][4];
+#pragma unroll
+  for (int ks = 0; ks < DK / 16; ++ks) {
+    const int row = lane & 15, ch = 2 * ks + (lane >> 4);
+    ldsm_x4(qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], smem_u32(sQ + SwzTile<DK>::offset(row, ch)));
+  }
+#pragma unroll
+  for (int ks = 0; ks < DV / 16; ++ks) {
+    const int row = lane & 15, ch = 2 * ks + (lane >> 4);
+    ldsm_x4(df[ks][0], df[ks][1], df[ks][2], df[ks][3], smem_u32(sDO + SwzTile<DV>::offset(row, ch)));
+  }
+  float dqa[DK / 8][4];
+#pragma unroll
+  for (int j = 0; j < DK / 8; ++j) dqa[j][0] = dqa[j][1] = dqa[j][2] = dqa[j][3] = 0.f;
+  Tile<DK, DV> tile{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)warp * SM::kStage), nullptr};
+  tile.v = tile.k + kRows * DK;
+  const int32_t* myidx = idx + (((size_t)b * Hkv + g) * T + t) * top_k;
+  const int own = t / kSel;
+
+  for (int br = 0; br < 3; ++br) {   // 0 compressed, 1 selected, 2 window
+    // the branch's rows: global row of row r, or -1 when it is masked
+    int n = 0, lo = 0;
+    if (br == 0) n = t < kL - 1 ? 0 : min(nc, (t - kL + 1) / kS + 1);
+    else if (br == 1) n = top_k * kSel;
+    else { lo = max(0, t - window + 1); n = t - lo + 1; }
+    auto row_of = [&](int r) -> int {
+      if (br == 0) return r;
+      if (br == 2) return lo + r;
+      const int j = myidx[r / kSel];
+      if (j < 0) return -1;
+      const int u = min(j, own) * kSel + r % kSel;
+      return u <= t ? u : -1;
+    };
+    auto src_k = [&](int r) {
+      const int u = max(row_of(r), 0);
+      return br == 0 ? kc + (((size_t)b * nc + u) * Hkv + g) * DK : k + (((size_t)b * T + u) * Hkv + g) * DK;
+    };
+    auto src_v = [&](int r) {
+      const int u = max(row_of(r), 0);
+      return br == 0 ? vc + (((size_t)b * nc + u) * Hkv + g) * DV : v + (((size_t)b * T + u) * Hkv + g) * DV;
+    };
+    const int ntiles = (n + kRows - 1) / kRows;
+    auto load_tile = [&](int it) {
+      load_rows<DK, DV>(tile, it * kRows, n, src_k, src_v, lane);
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncwarp();
+    };
+    auto scores = [&](int it, float (&s)[2][4]) {   // masked S of the tile, log2 units
+      qk_tile<DK>(qf, tile.k, s, scale_log2, lane);
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int r = it * kRows + j * 8 + 2 * cq + e;
+          if (r >= n || row_of(r) < 0) { s[j][e] = -INFINITY; s[j][2 + e] = -INFINITY; }
+        }
+    };
+    // ---- pass 1: o and log-sum-exp of the branch
+    State<DV> st;
+    st.init();
+    for (int it = warp; it < ntiles; it += kWarps) {
+      load_tile(it);
+      float s[2][4];
+      scores(it, s);
+      float c0, c1;
+      softmax_update<DV>(st, s, c0, c1);
+      pv_tile<DV>(s, tile.v, st.o, lane);
+      __syncwarp();
+    }
+    {
+      float* mO = reinterpret_cast<float*>(smem);
+      float* mCoef = reinterpret_cast<float*>(smem + MergeBuf<DV>::kBytes);
+      float* mML = mCoef + kWarps * 16;
+      __syncthreads();
+      store_o<DV>(mO, st, 1.f, 1.f, warp, lane);
+      store_ml(mML, st.m0, st.l0, st.m1, st.l1, warp, lane);
+      __syncthreads();
+      if (tid < 16) {   // per head: lse (log2 units) and each warp's weight
+        float M = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) M = fmaxf(M, mML[(w * 16 + tid) * 2]);
+        float L = 0.f;
+        if (M != -INFINITY)
+          for (int w = 0; w < kWarps; ++w) L += exp2f(mML[(w * 16 + tid) * 2] - M) * mML[(w * 16 + tid) * 2 + 1];
+        const float lse = (tid < G && L > 0.f) ? M + __log2f(L) : INFINITY;
+        sLse[tid] = lse;
+        for (int w = 0; w < kWarps; ++w) mCoef[w * 16 + tid] = exp2f(mML[(w * 16 + tid) * 2] - lse);
+      }
+      __syncthreads();
+      merge_sum<DV>(mO, mCoef, sO, G, 0, kThreads);
+      __syncthreads();
+      if (tid < 16) {   // dgate = dout . o, D = g * dgate
+        float dg = 0.f;
+        if (tid < G)
+          for (int c = 0; c < DV; ++c) dg += __bfloat162float(dout[(row0 + tid) * DV + c]) * sO[tid * DV + c];
+        const float gb = tid < G ? __bfloat162float(gates[(row0 + tid) * 3 + br]) : 0.f;
+        sD[tid] = gb * dg;
+        sG[tid] = gb;
+        if (tid < G) dgates[(row0 + tid) * 3 + br] = dg;
+      }
+      __syncthreads();
+    }
+    const float g0 = sG[gl], g1 = sG[gl + 8];
+    const float lse0 = sLse[gl], lse1 = sLse[gl + 8], D0 = sD[gl], D1 = sD[gl + 8];
+    __syncthreads();   // the merge scratch becomes the tiles again
+    // ---- pass 2: dS and the gradients
+    for (int it = warp; it < ntiles; it += kWarps) {
+      load_tile(it);
+      float s[2][4], dp[2][4];
+      scores(it, s);
+      qk_tile<DV>(df, tile.v, dp, 1.f, lane);   // dout V^T
+      float p[2][4], ds[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        p[j][0] = exp2f(s[j][0] - lse0); p[j][1] = exp2f(s[j][1] - lse0);
+        p[j][2] = exp2f(s[j][2] - lse1); p[j][3] = exp2f(s[j][3] - lse1);
+        ds[j][0] = p[j][0] * (g0 * dp[j][0] - D0); ds[j][1] = p[j][1] * (g0 * dp[j][1] - D0);
+        ds[j][2] = p[j][2] * (g1 * dp[j][2] - D1); ds[j][3] = p[j][3] * (g1 * dp[j][3] - D1);
+      }
+      pv_tile<DK>(ds, tile.k, dqa, lane);   // dQ += dS K
+      // dK rows += dS^T Q, then dV rows += (g P)^T dout, through the per-warp [16 heads][16 rows] tile
+#pragma unroll
+      for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int c = j * 8 + 2 * cq;
+          const float x00 = pass ? g0 * p[j][0] : ds[j][0], x01 = pass ? g0 * p[j][1] : ds[j][1];
+          const float x10 = pass ? g1 * p[j][2] : ds[j][2], x11 = pass ? g1 * p[j][3] : ds[j][3];
+          *reinterpret_cast<uint32_t*>(sX + gl * 16 + c) = pack_bf16(x00, x01);
+          *reinterpret_cast<uint32_t*>(sX + (gl + 8) * 16 + c) = pack_bf16(x10, x11);
+        }
+        __syncwarp();
+        uint32_t a[4];
+        load_at(sX, a, lane);
+        __syncwarp();
+        if (pass == 0) {
+          float acc[DK / 8][4];
+#pragma unroll
+          for (int x = 0; x < DK / 8; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
+          mma_ab<DK>(a, sQ, acc, lane);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = it * kRows + gl + 8 * hh;
+            const int u = r < n ? row_of(r) : -1;
+            if (u < 0) continue;
+            float* dst = br == 0 ? dkc + (((size_t)b * nc + u) * Hkv + g) * DK : dk + (((size_t)b * T + u) * Hkv + g) * DK;
+            const float sc = scale_log2 * 0.69314718055994531f;   // the softmax scale
+#pragma unroll
+            for (int x = 0; x < DK / 8; ++x) {
+              atomicAdd(dst + x * 8 + 2 * cq, sc * acc[x][2 * hh]);
+              atomicAdd(dst + x * 8 + 2 * cq + 1, sc * acc[x][2 * hh + 1]);
+            }
+          }
+        } else {
+          float acc[DV / 8][4];
+#pragma unroll
+          for (int x = 0; x < DV / 8; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
+          mma_ab<DV>(a, sDO, acc, lane);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int r = it * kRows + gl + 8 * hh;
+            const int u = r < n ? row_of(r) : -1;
+            if (u < 0) continue;
+            float* dst = br == 0 ? dvc + (((size_t)b * nc + u) * Hkv + g) * DV : dv + (((size_t)b * T + u) * Hkv + g) * DV;
+#pragma unroll
+            for (int x = 0; x < DV / 8; ++x) {
+              atomicAdd(dst + x * 8 + 2 * cq, acc[x][2 * hh]);
+              atomicAdd(dst + x * 8 + 2 * cq + 1, acc[x][2 * hh + 1]);
+            }
+          }
+        }
+      }
+      __syncwarp();
+    }
+    __syncthreads();   // before the next branch reuses the tiles and the merge scratch
+  }
+  // dq = scale * sum over the warps of dS K
+#pragma unroll
+  for (int x = 0; x < DK / 8; ++x) {
+    atomicAdd(sDQ + gl * DK + x * 8 + 2 * cq, dqa[x][0]);
+    atomicAdd(sDQ + gl * DK + x * 8 + 2 * cq + 1, dqa[x][1]);
+    atomicAdd(sDQ + (gl + 8) * DK + x * 8 + 2 * cq, dqa[x][2]);
+    atomicAdd(sDQ + (gl + 8) * DK + x * 8 + 2 * cq + 1, dqa[x][3]);
+  }
+  __syncthreads();
+  const float sc = scale_log2 * 0.69314718055994531f;
+  for (int e = tid; e < G * DK; e += kThreads) dq[row0 * DK + e] = sc * sDQ[e];
+}
+
+// dX[b, u, h, c] += sum over i with s*i <= u < s*i + l of sum_j W[(u - s*i)*D + c, j] dXc[b, i, h, j].
+// One warp per (b, u, h); lane c-loop.
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_phi_dx_kernel(const __nv_bfloat16* __restrict__ w, const float* __restrict__ dxc, float* __restrict__ dx, int B,
+                  int T, int H, int nc) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (gw >= B * T * H) return;
+  const int h = gw % H, u = (gw / H) % T, b = gw / (H * T);
+  float acc[D / 32];
+#pragma unroll
+  for (int x = 0; x < D / 32; ++x) acc[x] = 0.f;
+  for (int i = max(0, (u - kL) / kS); i <= u / kS && i < nc; ++i) {
+    const int r = u - kS * i;
+    if (r < 0 || r >= kL) continue;
+    const float* g = dxc + (((size_t)b * nc + i) * H + h) * D;
+    for (int j = 0; j < D; ++j) {
+      const float gj = g[j];
+#pragma unroll
+      for (int x = 0; x < D / 32; ++x)
+        acc[x] += __bfloat162float(w[((size_t)r * D + x * 32 + lane) * D + j]) * gj;
+    }
+  }
+  float* dst = dx + (((size_t)b * T + u) * H + h) * D;
+#pragma unroll
+  for (int x = 0; x < D / 32; ++x) dst[x * 32 + lane] += acc[x];
+}
+
+// dW[r*D + c, j] = sum over (b, h, i) of X[b, s*i + r, h, c] * dXc[b, i, h, j]: one thread per
+// output element, a loop over every compressed block.
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_phi_dw_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dxc, float* __restrict__ dw, int B,
+                  int T, int H, int nc) {
+  const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (size_t)kL * D * D) return;
+  const int j = (int)(e % D), rc = (int)(e / D), r = rc / D, c = rc % D;
+  float acc = 0.f;
+  for (int b = 0; b < B; ++b)
+    for (int i = 0; i < nc; ++i)
+      for (int h = 0; h < H; ++h)
+        acc += __bfloat162float(x[(((size_t)b * T + kS * i + r) * H + h) * D + c]) *
+               dxc[(((size_t)b * nc + i) * H + h) * D + j];
+  dw[e] = acc;
+}
+
+template <int DK, int DV>
+cudaError_t launch_attn(const BwdArgs& a, cudaStream_t st) {
+  using SM = BwdSmem<DK, DV>;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(bwd_attn_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  bwd_attn_kernel<DK, DV><<<dim3(a.T, a.Hkv, a.B), kThreads, SM::kTotal, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.kc),
+      static_cast<const __nv_bfloat16*>(a.vc), static_cast<const __nv_bfloat16*>(a.gates),
+      static_cast<const __nv_bfloat16*>(a.dout), a.idx, a.dq, a.gk, a.gv, a.gkc, a.gvc, a.dgates, a.T, a.Hq, a.Hkv,
+      a.G, a.nc, a.top_k, a.window, a.scale_log2);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_phi(const void* x, const void* w, const float* dxc, float* dx, float* dw, int B, int T, int H,
+                       int nc, cudaStream_t st) {
+  if (nc == 0) return cudaSuccess;
+  const long warps = (long)B * T * H;
+  bwd_phi_dx_kernel<D><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(w), dxc, dx, B, T, H, nc);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t n = (size_t)kL * D * D;
+  bwd_phi_dw_kernel<D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), dxc, dw, B,
+                                                                    T, H, nc);
+  return cudaGetLastError();
+}
+
+cudaError_t phi_dispatch(int d, const void* x, const void* w, const float* dxc, float* dx, float* dw, int B, int T,
+                         int H, int nc, cudaStream_t st) {
+  switch (d) {
+    case 64: return launch_phi<64>(x, w, dxc, dx, dw, B, T, H, nc, st);
+    case 128: return launch_phi<128>(x, w, dxc, dx, dw, B, T, H, nc, st);
+    case 192: return launch_phi<192>(x, w, dxc, dx, dw, B, T, H, nc, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+}  // namespace
+
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t st) {
+  cudaError_t e = cudaErrorInvalidValue;
+  if (a.dk == 192 && a.dv == 128) e = launch_attn<192, 128>(a, st);
+  else if (a.dk == 128 && a.dv == 128) e = launch_attn<128, 128>(a, st);
+  else if (a.dk == 64 && a.dv == 64) e = launch_attn<64, 64>(a, st);
+  if (e != cudaSuccess) return e;
+  e = phi_dispatch(a.dk, a.k, a.w_k, a.gkc, a.gk, a.dw_k, a.B, a.T, a.Hkv, a.nc, st);
+  if (e != cudaSuccess) return e;
+  return phi_dispatch(a.dv, a.v, a.w_v, a.gvc, a.gv, a.dw_v, a.B, a.T, a.Hkv, a.nc, st);
+}
+
+}  // namespace nsa

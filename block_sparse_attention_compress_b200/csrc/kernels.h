@@ -104,6 +104,32 @@ cudaError_t launch_dsa_indexer(const DsaArgs& a, cudaStream_t st);
 cudaError_t launch_dsa_topk(const DsaArgs& a, cudaStream_t st);
 cudaError_t launch_dsa_attn(const DsaArgs& a, cudaStream_t st);
 
+// Backward of the NSA forward (linear phi, equal lengths).  Gradients in fp32; gk, gv, gkc, gvc
+// must be zero on entry (the attention kernel adds into them).
+struct BwdArgs {
+  const void* q;      // [B, T, Hq, dk]
+  const void* k;      // [B, T, Hkv, dk]
+  const void* v;      // [B, T, Hkv, dv]
+  const void* kc;     // [B, nc, Hkv, dk] phi(k), as the forward computed it
+  const void* vc;     // [B, nc, Hkv, dv]
+  const void* w_k;    // [l*dk, dk]
+  const void* w_v;    // [l*dv, dv]
+  const void* gates;  // [B, T, Hq, 3]
+  const void* dout;   // [B, T, Hq, dv]
+  const int32_t* idx; // [B, Hkv, T, top_k] the forward's chosen blocks
+  float* dq;          // [B, T, Hq, dk]
+  float* gk;          // [B, T, Hkv, dk]
+  float* gv;          // [B, T, Hkv, dv]
+  float* gkc;         // [B, nc, Hkv, dk] scratch
+  float* gvc;         // [B, nc, Hkv, dv] scratch
+  float* dgates;      // [B, T, Hq, 3]
+  float* dw_k;        // [l*dk, dk]
+  float* dw_v;        // [l*dv, dv]
+  int B, T, Hq, Hkv, G, dk, dv, nc, top_k, window;
+  float scale_log2;
+};
+cudaError_t launch_backward(const BwdArgs& a, cudaStream_t st);
+
 // K6: one decode step per sequence, all branches in one launch.
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 

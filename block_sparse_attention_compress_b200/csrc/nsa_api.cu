@@ -304,6 +304,55 @@ nsa_status nsa_forward_varlen(const void* q, const void* k, const void* v, const
   return nsa_forward_impl(q, k, v, gates, cfg, out, static_cast<cudaStream_t>(stream), cu_seqlens, total_tokens);
 }
 
+nsa_status nsa_backward(const void* q, const void* k, const void* v, const void* gates, const int32_t* sel_idx,
+                        const void* dout, const nsa_config* cfg, float* dq, float* dk, float* dv, float* dgates,
+                        float* dw_k, float* dw_v, void* stream) {
+  nsa_status st = check_cfg(cfg);
+  if (st != NSA_OK) return st;
+  if (cfg->mode != NSA_MODE_NSA || cfg->phi_mlp) return NSA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !gates || !sel_idx || !dout || !dq || !dk || !dv || !dgates || !dw_k || !dw_v)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
+      !aligned16(dv) || (reinterpret_cast<uintptr_t>(gates) & 1u) || (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dgates) & 3u) || (reinterpret_cast<uintptr_t>(dw_k) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dw_v) & 3u))
+    return NSA_ERR_INVALID_ARG;
+  st = check_workspace(cfg, workspace_bytes(cfg));
+  if (st != NSA_OK) return st;
+  const FwdLayout L = forward_layout(cfg);
+  auto ws = static_cast<uint8_t*>(cfg->workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  nsa::BwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.gates = gates; a.dout = dout; a.idx = sel_idx;
+  a.w_k = cfg->w_cmp_k; a.w_v = cfg->w_cmp_v;
+  a.B = cfg->batch; a.T = cfg->seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
+  a.dk = cfg->d_k; a.dv = cfg->d_v; a.nc = n_cmp(cfg->seqlen, cfg->cmp_block, cfg->cmp_stride);
+  a.top_k = cfg->top_k; a.window = cfg->window;
+  const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.kc = ws + L.kc; a.vc = ws + L.vc;
+  a.dq = dq; a.gk = dk; a.gv = dv; a.dgates = dgates; a.dw_k = dw_k; a.dw_v = dw_v;
+  // the Kc/Vc gradients use the forward's accumulator region (it is larger)
+  const size_t nkc = (size_t)a.B * a.nc * a.Hkv;
+  a.gkc = reinterpret_cast<float*>(ws + L.acc);
+  a.gvc = a.gkc + nkc * a.dk;
+  const size_t nk = (size_t)a.B * a.T * a.Hkv;
+  cudaError_t e = cudaMemsetAsync(ws + L.err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nk * a.dk * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, nk * a.dv * 4, s);
+  if (e == cudaSuccess && nkc) e = cudaMemsetAsync(a.gkc, 0, nkc * (a.dk + a.dv) * 4, s);
+  if (e == cudaSuccess && a.nc == 0) {   // no compressed block: phi's weights get no gradient
+    e = cudaMemsetAsync(dw_k, 0, (size_t)cfg->cmp_block * a.dk * a.dk * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw_v, 0, (size_t)cfg->cmp_block * a.dv * a.dv * 4, s);
+  }
+  if (e == cudaSuccess)
+    e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, ws + L.kc, s);
+  if (e == cudaSuccess)
+    e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, cfg->cmp_block, cfg->cmp_stride, ws + L.vc, s);
+  if (e == cudaSuccess) e = nsa::launch_backward(a, s);
+  return from_cuda(e);
+}
+
 nsa_status nsa_dsa_forward(const void* q, const void* k, const void* v, const void* q_idx, const void* k_idx,
                            const void* w_idx, int32_t idx_heads, int32_t idx_dim, const nsa_config* cfg, void* out,
                            int32_t* sel_out, void* stream) {

@@ -212,6 +212,23 @@ NSA_API nsa_status nsa_forward_varlen(const void* q, const void* k, const void* 
                                       void* out, void* stream);
 
 /*
+ * nsa_backward -- gradients of the NSA forward ([NOTES] §13: NSA is trained natively, forward
+ * and backward).  NSA mode, linear phi (phi_mlp = 0), batch of equal lengths.
+ *   q, k, v, gates  the forward's inputs (as for nsa_forward);
+ *   sel_idx   int32 [B, H_kv, T, top_k]: the blocks the forward chose (its sel_idx_out).  The
+ *             choice is discrete: no gradient flows through the scores and the top-k;
+ *   dout      bf16 [B, T, H_q, d_v]: the gradient of the output;
+ *   dq fp32 [B, T, H_q, d_k];  dk fp32 [B, T, H_kv, d_k];  dv fp32 [B, T, H_kv, d_v];
+ *   dgates fp32 [B, T, H_q, 3];  dw_k fp32 [l*d_k, d_k];  dw_v fp32 [l*d_v, d_v]
+ *             (all written; dk and dv include the paths through phi).
+ * Workspace: nsa_workspace_size(cfg, 0) bytes, as for nsa_forward.  Status codes as for
+ * nsa_forward.
+ */
+NSA_API nsa_status nsa_backward(const void* q, const void* k, const void* v, const void* gates,
+                                const int32_t* sel_idx, const void* dout, const nsa_config* cfg, float* dq,
+                                float* dk, float* dv, float* dgates, float* dw_k, float* dw_v, void* stream);
+
+/*
  * nsa_dsa_forward -- token-wise sparse attention behind a lightning indexer (DSA; 10100.com,
  * "机器之心PRO · 会员通讯 Week 45", "Which Attention is All You Need?", section "Linear v.s.
  * Sparse", point 6: a light indexer scores every earlier token, the k best are kept, and full

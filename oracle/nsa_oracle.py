@@ -61,6 +61,9 @@ F64 = torch.float64
 
 
 def _f64(x: torch.Tensor) -> torch.Tensor:
+    """fp64 on the CPU; an fp64 CPU tensor that requires grad is kept as is (autograd)."""
+    if x.requires_grad and x.dtype == F64 and x.device.type == "cpu":
+        return x
     return x.detach().to("cpu", F64)
 
 
@@ -266,7 +269,7 @@ def nsa_token(Qg, K, V, Kc, Vc, gates_g, t, *, l, s, b, k, w, scale,
 def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
                 sel_block=64, top_k=16, window=512, force_first=True,
                 force_local=True, scale=None, tokens=None, round_kc=True,
-                keep_branches=False, score_map="touch", mlp=None):
+                keep_branches=False, score_map="touch", mlp=None, forced_idx=None):
     """NSA prefill forward over the query positions ``tokens`` (all by default).
 
     q [B,T,H_q,d_k], k [B,T,H_kv,d_k], v [B,T,H_kv,d_v], gates [B,T,H_q,3],
@@ -274,7 +277,10 @@ def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
     h // (H_q // H_kv) ([EN], GQA paragraph; [NOTES] §7).
 
     ``mlp`` = dict(b_k, w_k2, b_v, w_v2) makes phi the two-layer MLP of R15
-    (w_k, w_v are then its first layers); ``score_map`` picks the R3 reading.
+    (w_k, w_v are then its first layers); ``score_map`` picks the R3 reading;
+    ``forced_idx`` [B, H_kv, n_tok, top_k] imposes the chosen blocks (forced-index mode).
+    The function is differentiable (torch autograd) in q, k, v, gates, w_k, w_v
+    given fp64 leaf tensors; the block choice is discrete.
 
     Returns a dict with fp64 ``out`` [B, n_tok, H_q, d_v], int ``idx``
     [B, H_kv, n_tok, top_k], ``score`` (list per (b, g, token) of the block
@@ -302,7 +308,8 @@ def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
                 r = nsa_token(q[bi, t, hs], k[bi, :, g], v[bi, :, g], kc[bi, :, g], vc[bi, :, g],
                               gates[bi, t, hs], t, l=l, s=s, b=b, k=top_k, w=window,
                               scale=scale, force_first=force_first, force_local=force_local,
-                              score_map=score_map)
+                              score_map=score_map,
+                              idx=None if forced_idx is None else [int(j) for j in forced_idx[bi, g, n_i]])
                 out[bi, n_i, hs] = r["out"]
                 idx[bi, g, n_i] = torch.tensor(r["idx"])
                 scores[bi][g][n_i] = r["score"]

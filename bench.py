@@ -313,6 +313,10 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.empty_cache()
         result["varlen"] = run_varlen_bench(args, dev, world)
         result["gpu_launches"] += result["varlen"]["gpu_launches"]
+    if not args.no_backward:
+        torch.cuda.empty_cache()
+        result["backward"] = run_backward_bench(args, dev, world)
+        result["gpu_launches"] += result["backward"]["gpu_launches"]
     if not args.no_dsa:
         torch.cuda.empty_cache()
         result["dsa"] = run_dsa_bench(args, dev, world)
@@ -604,6 +608,51 @@ def run_dsa_bench(args, dev, world):
             "gpu_launches": len(names) * args.steps}
 
 
+def run_backward_bench(args, dev, world):
+    """NSA backward (nsa_backward) of the 8K workload: gradients of q, k, v, gates and phi's weights
+    for the blocks a forward chose; at most 3 timed steps (it is a first, atomics-based version)."""
+    import block_sparse_attention_compress_b200 as nsa
+    from block_sparse_attention_compress_b200.torch_ops import NSAForward
+    c = synth.WORKLOADS["nsa_8k"]
+    B, T, hq, hkv, dk, dv = c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"]
+    x = synth.nsa_inputs(B, T, hq, hkv, dk, dv, seed=0, device=dev)
+    f = NSAForward(B, T, hq, hkv, dk, dv, x.w_k, x.w_v, top_k=c["top_k"], window=c["window"], device=dev)
+    f(x.q, x.k, x.v, x.gates)
+    dout = torch.randn(B, T, hq, dv, device=dev).to(torch.bfloat16)
+    g = dict(dq=torch.empty(B, T, hq, dk, device=dev), dk=torch.empty(B, T, hkv, dk, device=dev),
+             dv=torch.empty(B, T, hkv, dv, device=dev), dgates=torch.empty(B, T, hq, 3, device=dev),
+             dw_k=torch.empty(32 * dk, dk, device=dev), dw_v=torch.empty(32 * dv, dv, device=dev))
+
+    def step():
+        nsa.nsa_backward(x.q, x.k, x.v, x.gates, f.idx, dout, f.cfg, g["dq"], g["dk"], g["dv"], g["dgates"],
+                         g["dw_k"], g["dw_v"])
+
+    steps = max(1, min(args.steps, 3))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = allreduce_max(statistics.mean(times), world, dev)
+    fw = nsa_flops(T, hq, hkv, dk, dv, c["top_k"], c["window"], B)
+    pairs = sum(fw[s] / (2.0 * (dk + dv)) for s in ("cmp_select", "slc_attn", "swa_combine"))
+    flops = 2.0 * pairs * (4 * dk + 3 * dv)   # recompute (S, P.V) + dP + dQ + dK + dV
+    return {"workload": f"nsa_8k backward: B={B} T={T} h_q={hq} h_kv={hkv} d_k={dk} d_v={dv} top_k={c['top_k']} "
+                        f"window={c['window']} (dq, dk, dv, dgates, dw_k, dw_v)",
+            "ms_per_step": ms, "steps": steps, "tokens_per_s": world * B * T / (ms * 1e-3),
+            "tflops_computed": flops / (ms * 1e-3) / 1e12, "gpu_launches": 5 * steps}
+
+
 def run_e2e(args, f, x, out, dev, world):
     """Same step through the public API with inputs in pinned host memory: H2D copies of
     q, k, v, gates, the forward, and the D2H copy of the output, all inside the timed region."""
@@ -671,6 +720,7 @@ def main():
     ap.add_argument("--no-varlen", action="store_true")
     ap.add_argument("--no-phi-mlp", action="store_true")
     ap.add_argument("--no-dsa", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

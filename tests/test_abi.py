@@ -210,3 +210,26 @@ def test_phi_mlp_needs_its_weights(lib):
     lin = nsa.nsa_workspace_size(_cfg())
     mlp = nsa.nsa_workspace_size(_cfg(phi_mlp=1, w_cmp_k2=0x3000, w_cmp_v2=0x4000, b_cmp_k=0x5000, b_cmp_v=0x6000))
     assert mlp > lin   # the hidden rows
+
+
+def test_backward_rejects_bad_arguments(lib):
+    f = 0x10000   # never dereferenced: every call below fails its checks first
+    base = dict(workspace=0x100000, workspace_bytes=1 << 30)
+
+    def call(c, **kw):
+        a = dict(q=f, k=f, v=f, gates=f, sel=f, dout=f, dq=f, dk=f, dv=f, dg=f, dwk=f, dwv=f)
+        a.update(kw)
+        return lib.nsa_backward(a["q"], a["k"], a["v"], a["gates"], a["sel"], a["dout"], ctypes.byref(c), a["dq"],
+                                a["dk"], a["dv"], a["dg"], a["dwk"], a["dwv"], None)
+
+    c = _cfg(**base)
+    assert call(c, sel=0) == nsa.NSA_ERR_INVALID_ARG
+    assert call(c, dout=f + 8) == nsa.NSA_ERR_INVALID_ARG
+    assert call(c, dg=f + 2) == nsa.NSA_ERR_INVALID_ARG
+    mlp = _cfg(phi_mlp=1, w_cmp_k2=0x3000, w_cmp_v2=0x4000, b_cmp_k=0x5000, b_cmp_v=0x6000, **base)
+    assert call(mlp) == nsa.NSA_ERR_UNSUPPORTED
+    moba = _cfg(mode=nsa.NSA_MODE_MOBA, h_q=2, h_kv=2, d_k=128, d_v=128, sel_block=64, top_k=3, w_cmp_k=0,
+                w_cmp_v=0, **base)
+    assert call(moba) == nsa.NSA_ERR_UNSUPPORTED
+    c.workspace_bytes = 16
+    assert call(c) == nsa.NSA_ERR_WORKSPACE

@@ -461,3 +461,36 @@ def test_phi_mlp_reduces_to_the_linear_phi_in_the_linear_regime():
     got = oracle.phi_mlp(X, W1, b1, W2, l, s, round_hidden=False)
     want = oracle.phi_compress(X, W1 @ W2, l, s) + b1 @ W2
     assert torch.allclose(got, want, atol=1e-9, rtol=0)
+
+
+# ---------------------------------------------------------------- gradients (the backward's reference)
+
+def test_oracle_gradients_match_finite_differences():
+    """torch autograd through the fp64 oracle (forced block choice) against central differences
+    of the same function, at a few coordinates of every input: pins that the oracle forward is
+    differentiable end to end (phi, the three branches, the gates)."""
+    x = synth.nsa_inputs(1, 70, 4, 1, 64, 64, seed=9)
+    base = {n: getattr(x, n).double() for n in ("q", "k", "v", "gates", "w_k", "w_v")}
+    first = oracle.nsa_forward(*[base[n] for n in ("q", "k", "v", "gates", "w_k", "w_v")], top_k=3, window=20,
+                               round_kc=False)
+    forced = first["idx"]
+    g = torch.Generator().manual_seed(10)
+    dout = torch.randn(first["out"].shape, generator=g, dtype=torch.float64)
+
+    def loss(inp):
+        r = oracle.nsa_forward(*[inp[n] for n in ("q", "k", "v", "gates", "w_k", "w_v")], top_k=3, window=20,
+                               round_kc=False, forced_idx=forced)
+        return (r["out"] * dout).sum()
+
+    leaves = {n: t.clone().requires_grad_() for n, t in base.items()}
+    loss(leaves).backward()
+    for name, t in base.items():
+        flat = t.reshape(-1)
+        for pos in torch.randint(0, flat.numel(), (3,), generator=g).tolist():
+            h = 1e-6 * max(1.0, abs(float(flat[pos])))
+            up, dn = t.clone(), t.clone()
+            up.reshape(-1)[pos] += h
+            dn.reshape(-1)[pos] -= h
+            fd = (loss({**base, name: up}) - loss({**base, name: dn})) / (2 * h)
+            ad = leaves[name].grad.reshape(-1)[pos]
+            assert abs(float(fd - ad)) <= 1e-5 * max(1.0, abs(float(ad))), (name, pos, float(fd), float(ad))

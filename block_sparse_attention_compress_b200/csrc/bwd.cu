@@ -291,7 +291,8 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 }
 
 // dX[b, u, h, c] += sum over i with s*i <= u < s*i + l of sum_j W[(u - s*i)*D + c, j] dXc[b, i, h, j].
-// One warp per (b, u, h); lane c-loop.
+// One warp per (b, u, h): the lanes split j (each holds D/32 values of dXc[i]) and read the W
+// rows contiguously; each output c is a warp sum.
 template <int D>
 __global__ void __launch_bounds__(256)
 bwd_phi_dx_kernel(const __nv_bfloat16* __restrict__ w, const float* __restrict__ dxc, float* __restrict__ dx, int B,
@@ -299,23 +300,24 @@ bwd_phi_dx_kernel(const __nv_bfloat16* __restrict__ w, const float* __restrict__
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (gw >= B * T * H) return;
   const int h = gw % H, u = (gw / H) % T, b = gw / (H * T);
-  float acc[D / 32];
-#pragma unroll
-  for (int x = 0; x < D / 32; ++x) acc[x] = 0.f;
+  float* dst = dx + (((size_t)b * T + u) * H + h) * D;
   for (int i = max(0, (u - kL) / kS); i <= u / kS && i < nc; ++i) {
     const int r = u - kS * i;
     if (r < 0 || r >= kL) continue;
-    const float* g = dxc + (((size_t)b * nc + i) * H + h) * D;
-    for (int j = 0; j < D; ++j) {
-      const float gj = g[j];
+    const float* gi = dxc + (((size_t)b * nc + i) * H + h) * D;
+    float gj[D / 32];
 #pragma unroll
-      for (int x = 0; x < D / 32; ++x)
-        acc[x] += __bfloat162float(w[((size_t)r * D + x * 32 + lane) * D + j]) * gj;
+    for (int x = 0; x < D / 32; ++x) gj[x] = gi[x * 32 + lane];
+    for (int c = 0; c < D; ++c) {
+      const __nv_bfloat16* wr = w + ((size_t)r * D + c) * D;
+      float part = 0.f;
+#pragma unroll
+      for (int x = 0; x < D / 32; ++x) part += __bfloat162float(wr[x * 32 + lane]) * gj[x];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      if (lane == (c & 31)) dst[c] += part;   // spread the stores over the lanes
     }
   }
-  float* dst = dx + (((size_t)b * T + u) * H + h) * D;
-#pragma unroll
-  for (int x = 0; x < D / 32; ++x) dst[x * 32 + lane] += acc[x];
 }
 
 // dW[r*D + c, j] = sum over (b, h, i) of X[b, s*i + r, h, c] * dXc[b, i, h, j]: one thread per

@@ -15,7 +15,8 @@
 //   bwd_phi_dx_kernel  dX[u] += sum over the compressed blocks i covering token u of
 //                      W[(u - s*i)*d : (u - s*i + 1)*d, :] . dXc[i];
 //   bwd_phi_dw_kernel  dW[r*d + c, j] = sum over (b, h, i) of X[b, s*i + r, h, c] * dXc[b, i, h, j].
-// A first version: pass 2 loads each tile and waits for it, and the row gradients are atomics.
+// A first version: pass 2 loads each tile and waits for it, and the row gradients are float4
+// atomics (one per lane and 8 columns of a row).
 #include <cfloat>
 
 #include "common.cuh"
@@ -62,6 +63,25 @@ __device__ __forceinline__ void mma_ab(const uint32_t (&a)[4], const __nv_bfloat
     ldsm_x4_t(b0, b1, b2, b3, smem_u32(B + SwzTile<N>::offset(row, ch)));
     mma16816(out[2 * np], a, b0, b1);
     mma16816(out[2 * np + 1], a, b2, b3);
+  }
+}
+
+// Adds a 16-row x (8 NX)-column MMA accumulator to the row gradients, scaled by sc, with one
+// float4 atomic per lane and 8 columns: lanes cq and cq ^ 1 swap half their pairs, so that the
+// even lane holds columns 4 (cq / 2) .. + 3 of row gl and the odd lane the same columns of row
+// gl + 8.  dst is the lane's row (row gl for an even cq, gl + 8 for an odd one), or null when
+// that row is masked; every lane takes part in the shuffles.
+template <int NX>
+__device__ __forceinline__ void red_rows(const float (&acc)[NX][4], float* dst, float sc, int cq) {
+  const bool odd = cq & 1;
+  const int col = 4 * (cq >> 1);
+#pragma unroll
+  for (int x = 0; x < NX; ++x) {
+    const float s0 = odd ? acc[x][0] : acc[x][2], s1 = odd ? acc[x][1] : acc[x][3];
+    const float r0 = __shfl_xor_sync(0xffffffffu, s0, 1), r1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+    const float4 val = odd ? make_float4(sc * r0, sc * r1, sc * acc[x][2], sc * acc[x][3])
+                           : make_float4(sc * acc[x][0], sc * acc[x][1], sc * r0, sc * r1);
+    if (dst) atomicAdd(reinterpret_cast<float4*>(dst + x * 8 + col), val);
   }
 }
 
@@ -241,36 +261,23 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 #pragma unroll
           for (int x = 0; x < DK / 8; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
           mma_ab<DK>(a, sQ, acc, lane);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int r = it * kRows + gl + 8 * hh;
-            const int u = r < n ? row_of(r) : -1;
-            if (u < 0) continue;
-            float* dst = br == 0 ? dkc + (((size_t)b * nc + u) * Hkv + g) * DK : dk + (((size_t)b * T + u) * Hkv + g) * DK;
-            const float sc = scale_log2 * 0.69314718055994531f;   // the softmax scale
-#pragma unroll
-            for (int x = 0; x < DK / 8; ++x) {
-              atomicAdd(dst + x * 8 + 2 * cq, sc * acc[x][2 * hh]);
-              atomicAdd(dst + x * 8 + 2 * cq + 1, sc * acc[x][2 * hh + 1]);
-            }
-          }
+          const int r = it * kRows + gl + 8 * (cq & 1);   // this lane's row of the float4 adds
+          const int u = r < n ? row_of(r) : -1;
+          float* dst = u < 0 ? nullptr
+                             : br == 0 ? dkc + (((size_t)b * nc + u) * Hkv + g) * DK
+                                       : dk + (((size_t)b * T + u) * Hkv + g) * DK;
+          red_rows<DK / 8>(acc, dst, scale_log2 * 0.69314718055994531f, cq);   // times the softmax scale
         } else {
           float acc[DV / 8][4];
 #pragma unroll
           for (int x = 0; x < DV / 8; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
           mma_ab<DV>(a, sDO, acc, lane);
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int r = it * kRows + gl + 8 * hh;
-            const int u = r < n ? row_of(r) : -1;
-            if (u < 0) continue;
-            float* dst = br == 0 ? dvc + (((size_t)b * nc + u) * Hkv + g) * DV : dv + (((size_t)b * T + u) * Hkv + g) * DV;
-#pragma unroll
-            for (int x = 0; x < DV / 8; ++x) {
-              atomicAdd(dst + x * 8 + 2 * cq, acc[x][2 * hh]);
-              atomicAdd(dst + x * 8 + 2 * cq + 1, acc[x][2 * hh + 1]);
-            }
-          }
+          const int r = it * kRows + gl + 8 * (cq & 1);
+          const int u = r < n ? row_of(r) : -1;
+          float* dst = u < 0 ? nullptr
+                             : br == 0 ? dvc + (((size_t)b * nc + u) * Hkv + g) * DV
+                                       : dv + (((size_t)b * T + u) * Hkv + g) * DV;
+          red_rows<DV / 8>(acc, dst, 1.f, cq);
         }
       }
       __syncwarp();

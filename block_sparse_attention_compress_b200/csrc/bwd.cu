@@ -15,8 +15,9 @@
 //   bwd_phi_dx_kernel  dX[u] += sum over the compressed blocks i covering token u of
 //                      W[(u - s*i)*d : (u - s*i + 1)*d, :] . dXc[i];
 //   bwd_phi_dw_kernel  dW[r*d + c, j] = sum over (b, h, i) of X[b, s*i + r, h, c] * dXc[b, i, h, j].
-// A first version: pass 2 loads each tile and waits for it, and the row gradients are float4
-// atomics (one per lane and 8 columns of a row).
+// Each warp streams its tiles through two shared-memory stages (the next tile is requested
+// before the current one is waited for); the row gradients are float4 atomics (one per lane
+// and 8 columns of a row).
 #include <cfloat>
 
 #include "common.cuh"
@@ -31,7 +32,7 @@ constexpr int kL = 32, kS = 16, kSel = 64;
 template <int DK, int DV>
 struct BwdSmem {
   static constexpr size_t kStage = (size_t)kRows * (DK + DV) * 2;            // one tile (K then V)
-  static constexpr size_t kRings = (size_t)kWarps * kStage;                  // one stage per warp
+  static constexpr size_t kRings = (size_t)kWarps * 2 * kStage;              // two stages per warp
   static constexpr size_t kMerge = MergeBuf<DV>::kBytes + (size_t)kWarps * 16 * 3 * 4;
   static constexpr size_t kU = kRings > kMerge ? kRings : kMerge;            // rings / merge scratch
   static constexpr size_t kQ = kU;                                           // Q bf16 [16][DK]
@@ -40,7 +41,8 @@ struct BwdSmem {
   static constexpr size_t kO = kX + (size_t)kWarps * 16 * 16 * 2;            // o of the branch [16][DV] fp32
   static constexpr size_t kDQ = kO + 16 * DV * 4;                            // dq [16][DK] fp32
   static constexpr size_t kRow = kDQ + 16 * DK * 4;                          // lse, D, gate [16] each
-  static constexpr size_t kTotal = kRow + 3 * 16 * 4;
+  static constexpr size_t kIdx = kRow + 3 * 16 * 4;                          // the chosen blocks [<= 32]
+  static constexpr size_t kTotal = kIdx + 32 * 4;
   static_assert(kTotal <= 232448, "backward shared memory");
 };
 
@@ -106,6 +108,8 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   float* sLse = reinterpret_cast<float*>(smem + SM::kRow);
   float* sD = sLse + 16;
   float* sG = sD + 16;
+  int* sIdx = reinterpret_cast<int*>(smem + SM::kIdx);
+  static_assert(kThreads == 256, "the dgate sums take 16 threads per head row");
   const size_t row0 = ((size_t)b * T + t) * Hq + g * G;   // the group's first head row of this token
   for (int e = tid; e < 16 * (DK / 8); e += kThreads) {
     const int r = e / (DK / 8), ch = e % (DK / 8);
@@ -120,6 +124,8 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     *reinterpret_cast<uint4*>(sDO + SwzTile<DV>::offset(r, ch)) = val;
   }
   for (int e = tid; e < 16 * DK; e += kThreads) sDQ[e] = 0.f;
+  const int32_t* myidx = idx + (((size_t)b * Hkv + g) * T + t) * top_k;
+  for (int e = tid; e < top_k; e += kThreads) sIdx[e] = myidx[e];
   __syncthreads();
   uint32_t qf[DK / 16][4], df[DV / 16][4];
 #pragma unroll
@@ -135,9 +141,10 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   float dqa[DK / 8][4];
 #pragma unroll
   for (int j = 0; j < DK / 8; ++j) dqa[j][0] = dqa[j][1] = dqa[j][2] = dqa[j][3] = 0.f;
-  Tile<DK, DV> tile{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)warp * SM::kStage), nullptr};
-  tile.v = tile.k + kRows * DK;
-  const int32_t* myidx = idx + (((size_t)b * Hkv + g) * T + t) * top_k;
+  Tile<DK, DV> t0{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)warp * 2 * SM::kStage), nullptr};
+  t0.v = t0.k + kRows * DK;
+  Tile<DK, DV> t1{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)(warp * 2 + 1) * SM::kStage), nullptr};
+  t1.v = t1.k + kRows * DK;
   const int own = t / kSel;
 
   for (int br = 0; br < 3; ++br) {   // 0 compressed, 1 selected, 2 window
@@ -149,48 +156,65 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     auto row_of = [&](int r) -> int {
       if (br == 0) return r;
       if (br == 2) return lo + r;
-      const int j = myidx[r / kSel];
+      const int j = sIdx[r / kSel];
       if (j < 0) return -1;
       const int u = min(j, own) * kSel + r % kSel;
       return u <= t ? u : -1;
     };
-    auto src_k = [&](int r) {
-      const int u = max(row_of(r), 0);
-      return br == 0 ? kc + (((size_t)b * nc + u) * Hkv + g) * DK : k + (((size_t)b * T + u) * Hkv + g) * DK;
-    };
-    auto src_v = [&](int r) {
-      const int u = max(row_of(r), 0);
-      return br == 0 ? vc + (((size_t)b * nc + u) * Hkv + g) * DV : v + (((size_t)b * T + u) * Hkv + g) * DV;
-    };
+    const __nv_bfloat16* kb = br == 0 ? kc + ((size_t)b * nc * Hkv + g) * DK : k + ((size_t)b * T * Hkv + g) * DK;
+    const __nv_bfloat16* vb = br == 0 ? vc + ((size_t)b * nc * Hkv + g) * DV : v + ((size_t)b * T * Hkv + g) * DV;
     const int ntiles = (n + kRows - 1) / kRows;
-    auto load_tile = [&](int it) {
-      load_rows<DK, DV>(tile, it * kRows, n, src_k, src_v, lane);
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncwarp();
+    // Lane l loads row l & 15 of a tile (chunks of parity l >> 4) and holds that row's global
+    // index, -1 when the row is masked or past n; the masks of the other rows come from it by
+    // shuffles.  Each warp takes tiles warp, warp + 8, ... through its two stages: the next
+    // one is requested before the current one is waited for.
+    auto tile_row = [&](int it) {
+      const int r = it * kRows + (lane & 15);
+      return r < n ? row_of(r) : -1;
     };
-    auto scores = [&](int it, float (&s)[2][4]) {   // masked S of the tile, log2 units
-      qk_tile<DK>(qf, tile.k, s, scale_log2, lane);
+    auto issue = [&](int it, int slot, int u) {
+      if (it < ntiles) {
+        const Tile<DK, DV> dst = slot ? t1 : t0;
+        const int rr = lane & 15, half = lane >> 4;
+        const __nv_bfloat16* sk = kb + (size_t)max(u, 0) * Hkv * DK;
+        const __nv_bfloat16* sv = vb + (size_t)max(u, 0) * Hkv * DV;
+#pragma unroll
+        for (int c = 0; c < DK / 16; ++c)
+          cp_async16(dst.k + SwzTile<DK>::offset(rr, 2 * c + half), sk + (2 * c + half) * 8, u >= 0);
+#pragma unroll
+        for (int c = 0; c < DV / 16; ++c)
+          cp_async16(dst.v + SwzTile<DV>::offset(rr, 2 * c + half), sv + (2 * c + half) * 8, u >= 0);
+      }
+      cp_async_commit();
+    };
+    auto scores = [&](const __nv_bfloat16* tk, int u, float (&s)[2][4]) {   // masked S of the tile, log2 units
+      qk_tile<DK>(qf, tk, s, scale_log2, lane);
 #pragma unroll
       for (int j = 0; j < 2; ++j)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int r = it * kRows + j * 8 + 2 * cq + e;
-          if (r >= n || row_of(r) < 0) { s[j][e] = -INFINITY; s[j][2 + e] = -INFINITY; }
-        }
+        for (int e = 0; e < 2; ++e)
+          if (__shfl_sync(0xffffffffu, u, j * 8 + 2 * cq + e) < 0) { s[j][e] = -INFINITY; s[j][2 + e] = -INFINITY; }
     };
     // ---- pass 1: o and log-sum-exp of the branch
     State<DV> st;
     st.init();
-    for (int it = warp; it < ntiles; it += kWarps) {
-      load_tile(it);
+    int u_cur = tile_row(warp);
+    issue(warp, 0, u_cur);
+    for (int it = warp, slot = 0; it < ntiles; it += kWarps, slot ^= 1) {
+      const int u_nxt = tile_row(it + kWarps);
+      issue(it + kWarps, slot ^ 1, u_nxt);
+      cp_async_wait<1>();
+      __syncwarp();
+      const Tile<DK, DV> cur = slot ? t1 : t0;
       float s[2][4];
-      scores(it, s);
+      scores(cur.k, u_cur, s);
       float c0, c1;
       softmax_update<DV>(st, s, c0, c1);
-      pv_tile<DV>(s, tile.v, st.o, lane);
+      pv_tile<DV>(s, cur.v, st.o, lane);
       __syncwarp();
+      u_cur = u_nxt;
     }
+    cp_async_wait<0>();
     {
       float* mO = reinterpret_cast<float*>(smem);
       float* mCoef = reinterpret_cast<float*>(smem + MergeBuf<DV>::kBytes);
@@ -212,14 +236,24 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
       __syncthreads();
       merge_sum<DV>(mO, mCoef, sO, G, 0, kThreads);
       __syncthreads();
-      if (tid < 16) {   // dgate = dout . o, D = g * dgate
+      {   // dgate = dout . o and D = g * dgate: 16 threads per head row, 8 columns at a time
+        const int r = tid >> 4, part = tid & 15;
         float dg = 0.f;
-        if (tid < G)
-          for (int c = 0; c < DV; ++c) dg += __bfloat162float(dout[(row0 + tid) * DV + c]) * sO[tid * DV + c];
-        const float gb = tid < G ? __bfloat162float(gates[(row0 + tid) * 3 + br]) : 0.f;
-        sD[tid] = gb * dg;
-        sG[tid] = gb;
-        if (tid < G) dgates[(row0 + tid) * 3 + br] = dg;
+        if (r < G)
+          for (int ch = part; ch < DV / 8; ch += 16) {
+            const __nv_bfloat16* d8 = sDO + SwzTile<DV>::offset(r, ch);
+            const float* o8 = sO + r * DV + ch * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dg += __bfloat162float(d8[i]) * o8[i];
+          }
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) dg += __shfl_xor_sync(0xffffffffu, dg, off);
+        if (part == 0) {
+          const float gb = r < G ? __bfloat162float(gates[(row0 + r) * 3 + br]) : 0.f;
+          sD[r] = gb * dg;
+          sG[r] = gb;
+          if (r < G) dgates[(row0 + r) * 3 + br] = dg;
+        }
       }
       __syncthreads();
     }
@@ -227,11 +261,19 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
     const float lse0 = sLse[gl], lse1 = sLse[gl + 8], D0 = sD[gl], D1 = sD[gl + 8];
     __syncthreads();   // the merge scratch becomes the tiles again
     // ---- pass 2: dS and the gradients
-    for (int it = warp; it < ntiles; it += kWarps) {
-      load_tile(it);
+    u_cur = tile_row(warp);
+    issue(warp, 0, u_cur);
+    for (int it = warp, slot = 0; it < ntiles; it += kWarps, slot ^= 1) {
+      const int u_nxt = tile_row(it + kWarps);
+      issue(it + kWarps, slot ^ 1, u_nxt);
+      cp_async_wait<1>();
+      __syncwarp();
+      const Tile<DK, DV> cur = slot ? t1 : t0;
+      // this lane's row of the float4 gradient adds: gl for an even cq, gl + 8 for an odd one
+      const int u_add = __shfl_sync(0xffffffffu, u_cur, gl + 8 * (cq & 1));
       float s[2][4], dp[2][4];
-      scores(it, s);
-      qk_tile<DV>(df, tile.v, dp, 1.f, lane);   // dout V^T
+      scores(cur.k, u_cur, s);
+      qk_tile<DV>(df, cur.v, dp, 1.f, lane);   // dout V^T
       float p[2][4], ds[2][4];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -240,7 +282,7 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         ds[j][0] = p[j][0] * (g0 * dp[j][0] - D0); ds[j][1] = p[j][1] * (g0 * dp[j][1] - D0);
         ds[j][2] = p[j][2] * (g1 * dp[j][2] - D1); ds[j][3] = p[j][3] * (g1 * dp[j][3] - D1);
       }
-      pv_tile<DK>(ds, tile.k, dqa, lane);   // dQ += dS K
+      pv_tile<DK>(ds, cur.k, dqa, lane);   // dQ += dS K
       // dK rows += dS^T Q, then dV rows += (g P)^T dout, through the per-warp [16 heads][16 rows] tile
 #pragma unroll
       for (int pass = 0; pass < 2; ++pass) {
@@ -261,8 +303,7 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 #pragma unroll
           for (int x = 0; x < DK / 8; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
           mma_ab<DK>(a, sQ, acc, lane);
-          const int r = it * kRows + gl + 8 * (cq & 1);   // this lane's row of the float4 adds
-          const int u = r < n ? row_of(r) : -1;
+          const int u = u_add;
           float* dst = u < 0 ? nullptr
                              : br == 0 ? dkc + (((size_t)b * nc + u) * Hkv + g) * DK
                                        : dk + (((size_t)b * T + u) * Hkv + g) * DK;
@@ -272,8 +313,7 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 #pragma unroll
           for (int x = 0; x < DV / 8; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
           mma_ab<DV>(a, sDO, acc, lane);
-          const int r = it * kRows + gl + 8 * (cq & 1);
-          const int u = r < n ? row_of(r) : -1;
+          const int u = u_add;
           float* dst = u < 0 ? nullptr
                              : br == 0 ? dvc + (((size_t)b * nc + u) * Hkv + g) * DV
                                        : dv + (((size_t)b * T + u) * Hkv + g) * DV;
@@ -281,7 +321,9 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
         }
       }
       __syncwarp();
+      u_cur = u_nxt;
     }
+    cp_async_wait<0>();
     __syncthreads();   // before the next branch reuses the tiles and the merge scratch
   }
   // dq = scale * sum over the warps of dS K

@@ -27,6 +27,7 @@ def rel_err(got, ref):
 @pytest.mark.parametrize("shape,top_k,window", [
     ((1, 200, 16, 1, 192, 128), 4, 96),     # one group of 16 heads, ragged blocks
     ((2, 150, 8, 2, 64, 64), 3, 40),        # two groups of 4 heads, batch 2
+    ((1, 520, 16, 1, 192, 128), 8, 300),    # several 16-row tiles per warp in the selected and window branches
 ])
 def test_backward_matches_autograd(shape, top_k, window):
     B, T, hq, hkv, dk, dv = shape

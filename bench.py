@@ -610,7 +610,7 @@ def run_dsa_bench(args, dev, world):
 
 def run_backward_bench(args, dev, world):
     """NSA backward (nsa_backward) of the 8K workload: gradients of q, k, v, gates and phi's weights
-    for the blocks a forward chose; at most 3 timed steps (it is a first, atomics-based version)."""
+    for the blocks a forward chose; at most 3 timed steps (about 42 ms each)."""
     import block_sparse_attention_compress_b200 as nsa
     from block_sparse_attention_compress_b200.torch_ops import NSAForward
     c = synth.WORKLOADS["nsa_8k"]

@@ -177,6 +177,61 @@ struct DsaSmem {
   static_assert(kTotal <= 232448, "dsa shared memory");
 };
 
+// One warp's online softmax over the chosen tokens rows[0, cnt) (each kept inside [0, t]), through
+// its two-stage ring.  Lane l loads row l & 15 of a tile (the 16-byte chunks of parity l >> 4)
+// and holds that row's token, -1 past cnt; the masks of the other rows come from it by shuffles.
+// A tile's tokens are read two tiles ahead, so their loads overlap the math.
+template <int DK, int DV>
+__device__ void attend_tokens(const uint32_t (&qf)[DK / 16][4], State<DV>& st, Tile<DK, DV> ring0, Tile<DK, DV> ring1,
+                              int cnt, const int32_t* rows, int t, const __nv_bfloat16* kb, const __nv_bfloat16* vb,
+                              size_t kstride, size_t vstride, float scale_log2, int lane) {
+  const int ntiles = (cnt + kRows - 1) / kRows;
+  if (ntiles == 0) return;
+  const int rr = lane & 15, half = lane >> 4, cq = lane & 3;
+  auto token = [&](int it) {
+    const int r = it * kRows + rr;
+    return r < cnt ? min(max(rows[r], 0), t) : -1;
+  };
+  auto issue = [&](int it, int u) {
+    if (it < ntiles) {
+      const Tile<DK, DV> dst = (it & 1) ? ring1 : ring0;
+      const __nv_bfloat16* sk = kb + (size_t)max(u, 0) * kstride;
+      const __nv_bfloat16* sv = vb + (size_t)max(u, 0) * vstride;
+#pragma unroll
+      for (int c = 0; c < DK / 16; ++c)
+        cp_async16(dst.k + SwzTile<DK>::offset(rr, 2 * c + half), sk + (2 * c + half) * 8, u >= 0);
+#pragma unroll
+      for (int c = 0; c < DV / 16; ++c)
+        cp_async16(dst.v + SwzTile<DV>::offset(rr, 2 * c + half), sv + (2 * c + half) * 8, u >= 0);
+    }
+    cp_async_commit();
+  };
+  int u_cur = token(0), u_nxt = token(1);
+  issue(0, u_cur);
+  for (int it = 0; it < ntiles; ++it) {
+    const int u_nn = token(it + 2);
+    issue(it + 1, u_nxt);
+    cp_async_wait<1>();
+    __syncwarp();
+    const Tile<DK, DV> cur = (it & 1) ? ring1 : ring0;
+    float s[2][4];
+    qk_tile<DK>(qf, cur.k, s, scale_log2, lane);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (__shfl_sync(0xffffffffu, u_cur, j * 8 + 2 * cq + e) < 0) { s[j][e] = -INFINITY; s[j][2 + e] = -INFINITY; }
+    float c0, c1;
+    softmax_update<DV>(st, s, c0, c1);
+    pv_tile<DV>(s, cur.v, st.o, lane);
+    __syncwarp();
+    u_cur = u_nxt;
+    u_nxt = u_nn;
+  }
+  cp_async_wait<0>();
+  __syncwarp();
+}
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kThreads, 1)
 dsa_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -207,12 +262,10 @@ dsa_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   ring0.v = ring0.k + kRows * DK;
   Tile<DK, DV> ring1{reinterpret_cast<__nv_bfloat16*>(smem + (size_t)warp * 2 * SM::kStage + SM::kStage), nullptr};
   ring1.v = ring1.k + kRows * DK;
-  auto tok = [&](int r) { return min(max(my[r0 + r], 0), t); };   // a chosen token, kept inside [0, t]
-  auto rowk = [&](int r) { return k + (((size_t)b * T + tok(r)) * Hkv + g) * DK; };
-  auto rowv = [&](int r) { return v + (((size_t)b * T + tok(r)) * Hkv + g) * DV; };
   State<DV> st;
   st.init();
-  attend_rows<DK, DV>(qf, st, ring0, ring1, cnt, rowk, rowv, [](int) { return true; }, scale_log2, lane);
+  attend_tokens<DK, DV>(qf, st, ring0, ring1, cnt, my + r0, t, k + ((size_t)b * T * Hkv + g) * DK,
+                        v + ((size_t)b * T * Hkv + g) * DV, (size_t)Hkv * DK, (size_t)Hkv * DV, scale_log2, lane);
   float* sOut = reinterpret_cast<float*>(smem + SM::kOut);
   merge_states<DV>(st, smem, sOut, G, warp, lane);
   for (int e = tid; e < G * DV; e += kThreads) {

@@ -34,17 +34,24 @@ struct Tile {
 };
 
 // Issue the copies of rows [r0, r0+16) of a K/V source into a stage; rows >= n are zero-filled.
+// Eight lanes cover one 128-byte line of a row, so each copy instruction moves four whole lines
+// (rows lane / 8 + 4m); each lane looks its four rows up once and steps through their lines.
 template <int DK, int DV, class RowK, class RowV>
 __device__ __forceinline__ void load_rows(Tile<DK, DV> st, int r0, int n, RowK rowk, RowV rowv, int lane) {
-  for (int e = lane; e < kRows * (DK / 8); e += 32) {
-    const int r = e / (DK / 8), ch = e % (DK / 8);
+  static_assert(DK % 64 == 0 && DV % 64 == 0, "rows are whole 128-byte lines");
+  const int rq = lane >> 3, cl = lane & 7;
+#pragma unroll
+  for (int m = 0; m < kRows / 4; ++m) {
+    const int r = rq + 4 * m;
     const bool ok = r0 + r < n;
-    cp_async16(st.k + SwzTile<DK>::offset(r, ch), rowk(ok ? r0 + r : 0) + ch * 8, ok);
-  }
-  for (int e = lane; e < kRows * (DV / 8); e += 32) {
-    const int r = e / (DV / 8), ch = e % (DV / 8);
-    const bool ok = r0 + r < n;
-    cp_async16(st.v + SwzTile<DV>::offset(r, ch), rowv(ok ? r0 + r : 0) + ch * 8, ok);
+    const __nv_bfloat16* pk = rowk(ok ? r0 + r : 0);
+    const __nv_bfloat16* pv = rowv(ok ? r0 + r : 0);
+#pragma unroll
+    for (int x = 0; x < DK / 64; ++x)
+      cp_async16(st.k + SwzTile<DK>::offset(r, cl + 8 * x), pk + (cl + 8 * x) * 8, ok);
+#pragma unroll
+    for (int x = 0; x < DV / 64; ++x)
+      cp_async16(st.v + SwzTile<DV>::offset(r, cl + 8 * x), pv + (cl + 8 * x) * 8, ok);
   }
 }
 

@@ -221,7 +221,9 @@ NSA_API nsa_status nsa_forward_varlen(const void* q, const void* k, const void* 
  *   dq fp32 [B, T, H_q, d_k];  dk fp32 [B, T, H_kv, d_k];  dv fp32 [B, T, H_kv, d_v];
  *   dgates fp32 [B, T, H_q, 3];  dw_k fp32 [l*d_k, d_k];  dw_v fp32 [l*d_v, d_v]
  *             (all written; dk and dv include the paths through phi).
- * Workspace: nsa_workspace_size(cfg, 0) bytes, as for nsa_forward.  Status codes as for
+ * dq, dk, dv, dw_k and dw_v are fp32 sums taken in no fixed order (atomics across tokens, and
+ * across a CTA's warps for dq), so their last bits can differ from run to run; dgates is
+ * reproducible.  Workspace: nsa_workspace_size(cfg, 0) bytes, as for nsa_forward.  Status codes as for
  * nsa_forward.
  */
 NSA_API nsa_status nsa_backward(const void* q, const void* k, const void* v, const void* gates,

@@ -20,7 +20,8 @@ NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
 EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_forward_varlen",
             "nsa_dsa_forward", "nsa_backward", "nsa_decode",
-            "nsa_forward_noalloc", "nsa_device_status", "nsa_selftest_wait_timeout", "nsa_status_string")
+            "nsa_forward_noalloc", "nsa_device_status", "nsa_device_status_noalloc", "nsa_selftest_wait_timeout",
+            "nsa_status_string")
 
 
 class NsaConfig(ctypes.Structure):
@@ -84,6 +85,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_forward_noalloc.restype = ctypes.c_int
     lib.nsa_device_status.argtypes = [vp, ctypes.POINTER(i32), vp]
     lib.nsa_device_status.restype = ctypes.c_int
+    lib.nsa_device_status_noalloc.argtypes = [ctypes.POINTER(i32), vp]
+    lib.nsa_device_status_noalloc.restype = ctypes.c_int
     lib.nsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
     lib.nsa_selftest_wait_timeout.restype = ctypes.c_int
     lib.nsa_status_string.argtypes = [ctypes.c_int]
@@ -217,3 +220,13 @@ def nsa_forward_noalloc(q, k, v, gates, cfg: NsaConfig, out, stream=None, check:
     st = load_library().nsa_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), ctypes.byref(cfg), _ptr(out),
                                             _stream(stream, q))
     return _check(st, "nsa_forward_noalloc") if check else st
+
+
+def nsa_device_status_noalloc(stream=None) -> tuple[int, int]:
+    """(status, word) of the status word of the library's built-in scratch array (the one
+    nsa_forward_noalloc uses on the current device), after synchronising the stream."""
+    import torch
+    word = ctypes.c_int32(0)
+    s = _stream(stream) if stream is not None else torch.cuda.current_stream().cuda_stream
+    st = load_library().nsa_device_status_noalloc(ctypes.byref(word), s)
+    return st, int(word.value)

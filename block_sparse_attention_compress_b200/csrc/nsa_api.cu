@@ -277,6 +277,7 @@ nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* 
                        void* out, void* stream) {
   nsa_status st = check_cfg(cfg);
   if (st != NSA_OK) return st;
+  if (cfg->mode == NSA_MODE_DSA) return NSA_ERR_INVALID_ARG;   // DSA runs through nsa_dsa_forward only
   if (!q || !k || !v || !out || !aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return NSA_ERR_INVALID_ARG;
   if (cfg->mode == NSA_MODE_NSA && (!gates || (reinterpret_cast<uintptr_t>(gates) & 1u)))

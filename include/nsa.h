@@ -184,6 +184,8 @@ NSA_API nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t
  * MoBA mode, per token t and head h ([BLOG] "Kimi 的论文核心点"; [NOTES] §16-§17):
  *   the top_k complete past blocks j < t/b by q.mean(K_j) plus the own block t/b,
  *   one softmax over their tokens u <= t.
+ * cfg->mode = NSA_MODE_DSA is rejected with NSA_ERR_INVALID_ARG before anything runs
+ * (DSA has its own entry point, nsa_dsa_forward).
  */
 NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* gates,
                        const nsa_config* cfg, void* out, void* stream);
@@ -318,7 +320,11 @@ NSA_API nsa_status nsa_compress_append(const void* x_cache, const void* w, const
  *     each call writes every scratch byte it later reads.  Calls whose execution
  *     overlaps on the GPU (different streams, or different host threads) race on the
  *     array: serialise them.
- * Arguments, layouts and the other status codes are those of nsa_forward.
+ *   - A device-side timeout inside a call (see nsa_device_status) is written to the
+ *     array's status word; nsa_device_status_noalloc reads it.
+ * Arguments, layouts and the other status codes are those of nsa_forward (NSA and MoBA
+ * modes; NSA_MODE_DSA gets NSA_ERR_INVALID_ARG).  If the address lookup fails the call
+ * returns NSA_ERR_CUDA and the next call on that device tries the lookup again.
  */
 NSA_API nsa_status nsa_forward_noalloc(const void* q, const void* k, const void* v, const void* gates,
                                        const nsa_config* cfg, void* out, void* stream);
@@ -335,6 +341,16 @@ NSA_API nsa_status nsa_forward_noalloc(const void* q, const void* k, const void*
  * synchronisation or the copy fails.
  */
 NSA_API nsa_status nsa_device_status(const void* workspace, int32_t* code_out, void* stream);
+
+/*
+ * nsa_device_status_noalloc -- nsa_device_status for the scratch array built into the
+ * library, the one nsa_forward_noalloc uses on the current device (the pages have no
+ * counterpart).  Synchronises `stream`, reads the array's status word (the outcome of the
+ * latest nsa_forward_noalloc on this device) and returns NSA_OK or NSA_ERR_TIMEOUT, with
+ * the word in code_out if not NULL.  NSA_ERR_CUDA if the address lookup, the
+ * synchronisation or the copy fails.  Allocates nothing.
+ */
+NSA_API nsa_status nsa_device_status_noalloc(int32_t* code_out, void* stream);
 
 /*
  * nsa_selftest_wait_timeout -- test hook for the timeout path above; no part of the method.

@@ -53,11 +53,14 @@ def attend(qh: torch.Tensor, K: torch.Tensor, V: torch.Tensor, scale: float) -> 
     return p @ V
 
 
-def dsa_forward(q, k, v, q_i, k_i, w_i, *, top_k=2048, scale=None, tokens=None):
+def dsa_forward(q, k, v, q_i, k_i, w_i, *, top_k=2048, scale=None, tokens=None, forced_idx=None):
     """DSA forward over the query positions ``tokens`` (all by default).
 
     q [B,T,H_q,d_k], k [B,T,H_kv,d_k], v [B,T,H_kv,d_v]; q_i [B,T,H_I,d_I],
-    k_i [B,T,d_I], w_i [B,T,H_I].  Returns dict(out [B, n, H_q, d_v] fp64,
+    k_i [B,T,d_I], w_i [B,T,H_I].  ``forced_idx`` [B, n, top_k] (-1 padded)
+    imposes the chosen tokens (forced-index mode: the attention over a choice
+    that differs from the oracle's only at a near tie).
+    Returns dict(out [B, n, H_q, d_v] fp64,
     idx [B, n, top_k] (-1 padded), score: list per (b, token) of the indexer
     scores, for the near-tie rule)."""
     q, k, v = q.to(F64), k.to(F64), v.to(F64)
@@ -72,7 +75,10 @@ def dsa_forward(q, k, v, q_i, k_i, w_i, *, top_k=2048, scale=None, tokens=None):
     for b in range(B):
         for n, t in enumerate(toks):
             sc = indexer_scores(q_i[b, t], k_i[b], w_i[b, t], t)
-            sel = select_tokens(sc, top_k)
+            if forced_idx is None:
+                sel = select_tokens(sc, top_k)
+            else:
+                sel = [int(j) for j in forced_idx[b, n] if j >= 0]
             scores[b][n] = sc
             idx[b, n, : len(sel)] = torch.tensor(sel)
             rows = torch.tensor(sel)

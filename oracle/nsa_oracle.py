@@ -395,13 +395,16 @@ def moba_select(qt: torch.Tensor, kbar: torch.Tensor, t: int, block: int, top_k:
     return chosen + [-1] * (top_k + 1 - len(chosen))
 
 
-def moba_forward(q, k, v, *, block=512, top_k=3, scale=None, tokens=None, heads=None):
+def moba_forward(q, k, v, *, block=512, top_k=3, scale=None, tokens=None, heads=None, forced_idx=None):
     """MoBA forward: per head, softmax attention over the tokens (<= t) of
     the chosen past blocks and of the own block (causal inside it).
     [BLOG] "Kimi 的论文核心点": selecting every block gives full attention,
     selecting none leaves only the own block.
 
-    q, k, v: [B, T, H, d].  Returns dict(out [B, n_tok, H, d], idx
+    q, k, v: [B, T, H, d].  ``forced_idx`` [B, H, n_tok, top_k+1] imposes the
+    chosen blocks (forced-index mode, as in ``nsa_forward``: where two block
+    choices are equally correct up to a near tie, the output is checked for
+    the choice actually made).  Returns dict(out [B, n_tok, H, d], idx
     [B, H, n_tok, top_k+1], score list for the near-tie rule)."""
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, T, H, d = q.shape
@@ -416,7 +419,10 @@ def moba_forward(q, k, v, *, block=512, top_k=3, scale=None, tokens=None, heads=
         for h in hl:
             kbar = moba_block_keys(k[bi, :, h], block)
             for n_i, t in enumerate(toks):
-                sel = moba_select(q[bi, t, h], kbar, t, block, top_k)
+                if forced_idx is None:
+                    sel = moba_select(q[bi, t, h], kbar, t, block, top_k)
+                else:
+                    sel = [int(j) for j in forced_idx[bi, h, n_i]]
                 toks_u = block_tokens(sel, t, block)
                 o, _ = attend(q[bi, t, h:h + 1], k[bi, toks_u, h], v[bi, toks_u, h], scale)
                 out[bi, n_i, h] = o[0]

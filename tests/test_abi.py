@@ -233,3 +233,14 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(moba) == nsa.NSA_ERR_UNSUPPORTED
     c.workspace_bytes = 16
     assert call(c) == nsa.NSA_ERR_WORKSPACE
+
+
+def test_forward_rejects_dsa_mode(lib):
+    """DSA has its own entry point; nsa_forward and nsa_forward_noalloc refuse its mode
+    before anything runs (real host tensors, never dereferenced)."""
+    import torch
+    t = [torch.zeros(4096, dtype=torch.uint8) for _ in range(6)]
+    c = _cfg(mode=nsa.NSA_MODE_DSA, h_q=16, h_kv=1, d_k=192, d_v=128, top_k=16, cmp_stride=0,
+             workspace=t[5].data_ptr(), workspace_bytes=1 << 30)
+    assert nsa.nsa_forward(t[0], t[1], t[2], t[3], c, t[4], check=False) == nsa.NSA_ERR_INVALID_ARG
+    assert nsa.nsa_forward_noalloc(t[0], t[1], t[2], t[3], c, t[4], check=False) == nsa.NSA_ERR_INVALID_ARG

@@ -12,7 +12,8 @@ from block_sparse_attention_compress_b200.torch_ops import NSAForward
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-REL = 2e-2   # relative L2 error per gradient (bf16 operands, fp32 accumulation)
+MAX_REL = 2e-2    # per gradient tensor: max |err| <= MAX_REL * max |ref|  (bf16 operands, fp32 accumulation)
+MEAN_REL = 2e-3   #                      mean |err| <= MEAN_REL * max |ref|
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -20,8 +21,45 @@ def _lib():
     build.build()
 
 
-def rel_err(got, ref):
-    return float((got.double() - ref).norm() / ref.norm().clamp_min(1e-30))
+def assert_grad_close(name, got, ref):
+    """Element by element: every entry within MAX_REL of the tensor's largest reference entry,
+    and the mean error within MEAN_REL of it."""
+    ref = ref.detach().double()
+    err = (got.detach().cpu().double() - ref).abs()
+    scale = float(ref.abs().max())
+    assert scale > 0, name
+    mx, mn = float(err.max()), float(err.mean())
+    print(f"{name}: max {mx / scale:.2e} mean {mn / scale:.2e} of max|ref| {scale:.3e}")
+    assert mx <= MAX_REL * scale and mn <= MEAN_REL * scale, \
+        f"{name}: max {mx:.3e} mean {mn:.3e} against max|ref| {scale:.3e}"
+
+
+def run_and_compare(x, dout, top_k, window, tokens=None):
+    """GPU forward (for the chosen blocks) and backward through the C ABI; the oracle's fp64
+    autograd through its forward at ``tokens`` (all if None; dout must be zero elsewhere) in
+    forced-index mode on the GPU's choice; every gradient compared element by element."""
+    B, T, hq, dk = x.q.shape
+    hkv, dv = x.k.shape[2], x.v.shape[3]
+    dev = [t.to(DEV) for t in (x.q, x.k, x.v, x.gates, x.w_k, x.w_v, dout)]
+    f = NSAForward(B, T, hq, hkv, dk, dv, dev[4], dev[5], top_k=top_k, window=window)
+    f(*dev[:4])
+    grads = dict(dq=torch.empty(B, T, hq, dk), dk=torch.empty(B, T, hkv, dk), dv=torch.empty(B, T, hkv, dv),
+                 dgates=torch.empty(B, T, hq, 3), dw_k=torch.empty(32 * dk, dk), dw_v=torch.empty(32 * dv, dv))
+    gd = {n: t.to(DEV) for n, t in grads.items()}
+    nsa.nsa_backward(dev[0], dev[1], dev[2], dev[3], f.idx, dev[6], f.cfg, gd["dq"], gd["dk"], gd["dv"], gd["dgates"],
+                     gd["dw_k"], gd["dw_v"])
+    torch.cuda.synchronize()
+    assert f.device_status() == 0
+    idx = f.idx.cpu()
+    toks = list(range(T)) if tokens is None else list(tokens)
+    leaves = {n: t.double().requires_grad_() for n, t in
+              (("q", x.q), ("k", x.k), ("v", x.v), ("gates", x.gates), ("w_k", x.w_k), ("w_v", x.w_v))}
+    ref = oracle.nsa_forward(leaves["q"], leaves["k"], leaves["v"], leaves["gates"], leaves["w_k"], leaves["w_v"],
+                             top_k=top_k, window=window, tokens=toks, forced_idx=idx[:, :, toks])
+    (ref["out"] * dout[:, toks].double()).sum().backward()
+    pairs = dict(dq="q", dk="k", dv="v", dgates="gates", dw_k="w_k", dw_v="w_v")
+    for name, leaf in pairs.items():
+        assert_grad_close(name, gd[name], leaves[leaf].grad)
 
 
 @pytest.mark.parametrize("shape,top_k,window", [
@@ -34,22 +72,19 @@ def test_backward_matches_autograd(shape, top_k, window):
     x = synth.nsa_inputs(B, T, hq, hkv, dk, dv, seed=81)
     g = torch.Generator().manual_seed(82)
     dout = torch.randn(B, T, hq, dv, generator=g).to(torch.bfloat16)
-    dev = [t.to(DEV) for t in (x.q, x.k, x.v, x.gates, x.w_k, x.w_v, dout)]
-    f = NSAForward(B, T, hq, hkv, dk, dv, dev[4], dev[5], top_k=top_k, window=window)
-    f(*dev[:4])
-    grads = dict(dq=torch.empty(B, T, hq, dk), dk=torch.empty(B, T, hkv, dk), dv=torch.empty(B, T, hkv, dv),
-                 dgates=torch.empty(B, T, hq, 3), dw_k=torch.empty(32 * dk, dk), dw_v=torch.empty(32 * dv, dv))
-    gd = {n: t.to(DEV) for n, t in grads.items()}
-    nsa.nsa_backward(dev[0], dev[1], dev[2], dev[3], f.idx, dev[6], f.cfg, gd["dq"], gd["dk"], gd["dv"], gd["dgates"],
-                     gd["dw_k"], gd["dw_v"])
-    torch.cuda.synchronize()
-    idx = f.idx.cpu()
-    leaves = {n: t.double().requires_grad_() for n, t in
-              (("q", x.q), ("k", x.k), ("v", x.v), ("gates", x.gates), ("w_k", x.w_k), ("w_v", x.w_v))}
-    ref = oracle.nsa_forward(leaves["q"], leaves["k"], leaves["v"], leaves["gates"], leaves["w_k"], leaves["w_v"],
-                             top_k=top_k, window=window, forced_idx=idx)
-    (ref["out"] * dout.double()).sum().backward()
-    pairs = dict(dq="q", dk="k", dv="v", dgates="gates", dw_k="w_k", dw_v="w_v")
-    for name, leaf in pairs.items():
-        err = rel_err(gd[name].cpu(), leaves[leaf].grad)
-        assert err <= REL, f"{name}: relative error {err:.2e}"
+    run_and_compare(x, dout, top_k, window)
+
+
+def test_backward_8k_workload_sampled_rows():
+    """The 8K workload the benchmark times (64 query heads in 4 groups, d_k 192, d_v 128,
+    top-16, window 512) with dout nonzero on sampled rows only: every gradient then depends on
+    those rows alone, so the oracle's autograd over the sampled tokens gives all of dq, dk, dv,
+    dgates, dW_k and dW_v, each compared element by element."""
+    c = synth.WORKLOADS["nsa_8k"]
+    B, T, hq, hkv, dk, dv = c["B"], c["T"], c["h_q"], c["h_kv"], c["d_k"], c["d_v"]
+    x = synth.nsa_inputs(B, T, hq, hkv, dk, dv, seed=0)
+    g = torch.Generator().manual_seed(83)
+    toks = sorted(set([0, 31, 64, 511, 512, 4096, T - 1] + torch.randint(0, T, (17,), generator=g).tolist()))
+    dout = torch.zeros(B, T, hq, dv)
+    dout[:, toks] = torch.randn(B, len(toks), hq, dv, generator=g)
+    run_and_compare(x, dout.to(torch.bfloat16), c["top_k"], c["window"], tokens=toks)

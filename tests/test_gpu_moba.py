@@ -7,7 +7,7 @@ import block_sparse_attention_compress_b200 as nsa
 import oracle
 import synth
 from block_sparse_attention_compress_b200 import build
-from tests.helpers import NEAR_TIE, assert_close
+from tests.helpers import NEAR_TIE, assert_close, check_swap
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -32,42 +32,49 @@ def run_moba(x, block, top_k):
     return out.cpu(), idx.cpu()
 
 
-def compare(out, idx, ref, heads, top_k, min_exact=0.98):
-    """Choices bit-exact except near ties (then each swapped-in block scores within
-    NEAR_TIE of the oracle's k-th); outputs compared on rows with identical choices."""
+def compare(out, idx, ref, heads, rerun, min_exact=0.98):
+    """Choices bit-exact except legal near-tie swaps (check_swap: the own block kept last, each
+    added past block within NEAR_TIE of the oracle's lowest pick, each dropped one within
+    NEAR_TIE of the GPU's lowest pick); every output row compared, the swapped (token, head)
+    rows against the oracle in forced-index mode on the GPU's choice (``rerun(tokens, forced)``
+    with forced [B, H, n, top_k+1] returns the oracle's output [B, n, H, d])."""
     B, n, H, d = ref["out"].shape
     toks = ref["tokens"]
-    mask = torch.zeros(B, n, H, dtype=torch.bool)
     exact = total = 0
+    swapped = set()
     for b in range(B):
-        for h in heads:
+        for hi, h in enumerate(heads):
             for i, t in enumerate(toks):
                 g = idx[b, h, t].tolist()
                 o = ref["idx"][b, h, i].tolist()
                 total += 1
                 if g == o:
                     exact += 1
-                    mask[b, i, h] = True
                     continue
-                own = t // (ref.get("block") or 1)
                 sg, so = [j for j in g if j >= 0], [j for j in o if j >= 0]
-                assert len(sg) == len(so) and sg[-1] == so[-1], (b, h, t, g, o)
-                sc = ref["score"][(b, h, i)]
-                thr = min(float(sc[j]) for j in so[:-1])
-                for j in set(sg[:-1]) - set(so[:-1]):
-                    assert float(sc[j]) >= thr - NEAR_TIE, (b, h, t, j, float(sc[j]), thr)
+                own = t // ref["block"]
+                assert sg[-1] == own and so[-1] == own, (b, h, t, g, o)
+                assert sg[:-1] == sorted(sg[:-1]) and all(0 <= j < own for j in sg[:-1]), (b, h, t, g)
+                check_swap(sg[:-1], so[:-1], ref["score"][(b, h, i)], (), NEAR_TIE, (b, h, t))
+                swapped.add((b, hi, i))
     assert exact >= min_exact * total, (exact, total)
-    m = mask.unsqueeze(-1).expand(-1, -1, -1, d)
-    return assert_close(out[:, toks], ref["out"], mask=m, what="moba out")
+    ref_out = ref["out"].clone()
+    pos = sorted(set(i for (_, _, i) in swapped))
+    if pos:
+        forced = idx[:, :, [toks[i] for i in pos]].long()
+        ref_out[:, pos] = rerun([toks[i] for i in pos], forced)
+    return assert_close(out[:, toks][:, :, list(heads)], ref_out, what="moba out")
 
 
 @pytest.mark.parametrize("T,H,block,top_k", [(2048, 4, 256, 3), (1000, 2, 64, 2), (640, 2, 64, 5)])
 def test_moba_full(T, H, block, top_k):
     x = synth.moba_inputs(1, T, H, 128, seed=31)
     out, idx = run_moba(x, block, top_k)
-    ref = oracle.moba_forward(x.q, x.k, x.v, block=block, top_k=top_k)
+    run = lambda toks, forced=None: oracle.moba_forward(x.q, x.k, x.v, block=block, top_k=top_k, tokens=toks,
+                                                        forced_idx=forced)
+    ref = run(None)
     ref["block"] = block
-    compare(out, idx, ref, range(H), top_k)
+    compare(out, idx, ref, range(H), lambda toks, forced: run(toks, forced)["out"])
 
 
 def test_moba_no_past_block_is_block_local_attention():
@@ -100,24 +107,13 @@ def test_moba_workload_sampled():
     g = torch.Generator().manual_seed(5)
     toks = sorted(set([0, 511, 512, 1535, 1536, c["T"] - 1] + torch.randint(0, c["T"], (40,), generator=g).tolist()))
     heads = [0, 7, 19, 31]
-    ref = oracle.moba_forward(x.q, x.k, x.v, block=c["block"], top_k=c["top_k"], tokens=toks, heads=heads)
+
+    def run(toks_, forced=None):
+        # the oracle on the checked heads only (q/k/v sliced to them; forced choices come sliced)
+        sub = lambda a: a[:, :, heads]
+        return oracle.moba_forward(sub(x.q), sub(x.k), sub(x.v), block=c["block"], top_k=c["top_k"], tokens=toks_,
+                                   forced_idx=forced)
+    ref = run(toks)
     ref["block"] = c["block"]
-    B, n = 1, len(toks)
-    # compare only the checked heads
-    sub_out = out[:, toks][:, :, heads]
-    sub_ref = dict(ref, out=ref["out"][:, :, heads])
-    mask = torch.zeros(B, n, len(heads), dtype=torch.bool)
-    for hi, h in enumerate(heads):
-        for i, t in enumerate(toks):
-            g_ = idx[0, h, t].tolist()
-            o_ = ref["idx"][0, h, i].tolist()
-            if g_ == o_:
-                mask[0, i, hi] = True
-            else:
-                sc = ref["score"][(0, h, i)]
-                so = [j for j in o_ if j >= 0][:-1]
-                thr = min(float(sc[j]) for j in so)
-                for j in set(j for j in g_ if j >= 0) - set(o_):
-                    assert float(sc[j]) >= thr - NEAR_TIE
-    assert mask.float().mean() > 0.95
-    assert_close(sub_out, sub_ref["out"], mask=mask.unsqueeze(-1).expand(-1, -1, -1, c["d"]), what="moba 128K")
+    sub_idx = idx[:, heads]
+    compare(out[:, :, heads], sub_idx, ref, range(len(heads)), lambda t_, f_: run(t_, f_)["out"], min_exact=0.95)

@@ -215,9 +215,14 @@ def workload_config(c, name):
 # changes, until it is captured again.
 NCU_DRAM_BYTES_PER_ITEM = {
     "cmp_select": (205.892864e6 + 216.708352e6) / 32768,
-    "slc_attn": (501.060352e6 + 229.711616e6) / 32768,
+    "slc_attn": None,
     "swa_combine": (494.174976e6 + 118.646784e6) / 32768,
 }
+
+# The selected branch gathers whole 64-token K/V blocks from L2 into shared memory; its
+# ceiling is the L2 -> SM gather rate, measured at 67 B per clock per SM by a probe of the
+# same access pattern (TMA gathers of random 64-row blocks while K/V fit in L2).
+GATHER_B_PER_CLK_SM = 67.0
 
 
 def run_ours(args, rank, world, local_rank):
@@ -294,6 +299,7 @@ def run_ours(args, rank, world, local_rank):
                      "traffic_note": "DRAM bytes per launch, scaled by items from an ncu capture at T=8192",
                      "peak_source": f"{src} bf16_tflops (burst: the kernel is timed by CUDA events inside a "
                                     f"step of tens of milliseconds)"},
+        "gather": slc_gather(T, hq, hkv, dk, dv, c["top_k"], stage_mean["slc_attn"], B),
         "stages_ms": {s: round(v, 4) for s, v in stage_mean.items()},
         "stage_tflops": {s: round(flops[s] / (stage_mean[s] * 1e-3) / 1e12, 1) for s in STAGES},
         "gpu_launches": len(STAGES) * args.steps,
@@ -334,6 +340,21 @@ def run_ours(args, rank, world, local_rank):
                                   **info}
     if rank == 0:
         print(json.dumps(result), flush=True)
+
+
+def slc_gather(T, h_q, h_kv, d_k, d_v, top_k, ms, B=1, sms=148):
+    """The selected branch against the resource that bounds it: the K/V bytes it moves from L2
+    into shared memory (every token u <= t of the chosen blocks, once per (token, group):
+    (d_k + d_v) * 2 bytes each), per launch, against the L2 -> SM gather ceiling (the probe's
+    bytes per clock per SM x SMs x the sampled SM clock is taken as 1.95 GHz)."""
+    t = torch.arange(T, dtype=torch.float64)
+    nb = torch.div(t, BSEL, rounding_mode="floor") + 1
+    toks = torch.where(nb <= top_k, t + 1, 64.0 * (top_k - 1) + torch.remainder(t, BSEL) + 1)
+    nbytes = float(toks.sum()) * B * h_kv * (d_k + d_v) * 2
+    ach = nbytes / (ms * 1e-3) / 1e12
+    peak = GATHER_B_PER_CLK_SM * sms * 1.95e9 / 1e12
+    return {"bound": "l2_gather", "bytes_per_launch": nbytes, "achieved": ach, "peak": peak, "unit": "TB/s",
+            "frac": ach / peak, "peak_source": f"probe: {GATHER_B_PER_CLK_SM} B/clk per SM x {sms} SMs x 1.95 GHz"}
 
 
 def decode_bytes(idx, seqlens, h_q, d_k, d_v, window):

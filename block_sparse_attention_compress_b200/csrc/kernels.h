@@ -46,6 +46,10 @@ struct FwdArgs {
   // and idx keep their per-sequence layouts with T as the (maximum) length.
   const int32_t* cu = nullptr;
   int total = 0;      // token rows (cu[B], or B * T)
+  // (token, group) items of the selected branch to recompute exactly (see slc_attn_tc.cu): a
+  // count zeroed before the launches, and the item indices ([B * Hkv * T] capacity).
+  int* redo_count = nullptr;
+  int* redo_list = nullptr;
 };
 
 // First row and length of sequence b in a (possibly variable-length) batch.
@@ -63,6 +67,9 @@ cudaError_t launch_cmp_select_tc(const FwdArgs& a, cudaStream_t st);
 // K3: selected-block attention (acc += g_slc * o_slc).
 cudaError_t launch_slc_attn(const FwdArgs& a, cudaStream_t st);
 bool slc_attn_tma_supported(const FwdArgs& a);
+// K3 on tcgen05 + TMA (G == 16, d_v == 128, d_k in {128, 192}, top_k <= 32).
+bool slc_attn_tc_supported(const FwdArgs& a);
+cudaError_t launch_slc_attn_tc(const FwdArgs& a, cudaStream_t st);
 cudaError_t launch_slc_attn_tma(const FwdArgs& a, cudaStream_t st);
 // K4 + K5: sliding window and gated combine (out = bf16(acc + g_win * o_win)).
 cudaError_t launch_swa_combine(const FwdArgs& a, cudaStream_t st);

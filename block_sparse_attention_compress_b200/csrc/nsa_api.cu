@@ -65,18 +65,19 @@ nsa_status check_cfg(const nsa_config* c) {
 }
 
 struct FwdLayout {
-  size_t err, kc, vc, idx, acc, hk, hv, total;   // hk, hv: the MLP's hidden rows (phi_mlp only)
+  size_t err, kc, vc, idx, acc, redo, hk, hv, total;   // hk, hv: the MLP's hidden rows (phi_mlp only)
 };
 
 FwdLayout forward_layout(const nsa_config* c) {
   const size_t B = c->batch, T = c->seqlen, nc = n_cmp(c->seqlen, c->cmp_block, c->cmp_stride);
   FwdLayout L{};
   size_t off = 0;
-  L.err = off; off = align_up(off + 4);
+  L.err = off; off = align_up(off + 8);   // the status word, then the selected branch's redo count
   L.kc = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
   L.vc = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
   L.idx = off; off = align_up(off + B * c->h_kv * T * c->top_k * 4);
   L.acc = off; off = align_up(off + B * T * c->h_q * c->d_v * 4);
+  L.redo = off; off = align_up(off + B * c->h_kv * T * 4);   // the selected branch's redo list
   if (c->phi_mlp) {
     L.hk = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
     L.hv = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
@@ -171,12 +172,14 @@ nsa_status nsa_forward_impl(const void* q, const void* k, const void* v, const v
   a.idx = cfg->sel_idx_out ? cfg->sel_idx_out : reinterpret_cast<int32_t*>(ws + L.idx);
   a.acc = reinterpret_cast<float*>(ws + L.acc);
   a.err = reinterpret_cast<int*>(ws + L.err);
+  a.redo_count = a.err + 1;
+  a.redo_list = reinterpret_cast<int*>(ws + L.redo);
   a.cu = cu;
   a.total = total;
   a.w_straddle = straddle_weight(cfg);
 
   StageMarks marks(cfg, 5);
-  cudaError_t e = cudaMemsetAsync(a.err, 0, sizeof(int), s);
+  cudaError_t e = cudaMemsetAsync(a.err, 0, 2 * sizeof(int), s);   // the status word and the redo count
   if (e == cudaSuccess) e = marks.mark(s);
   const int l = cfg->cmp_block, st = cfg->cmp_stride;
   if (e == cudaSuccess)

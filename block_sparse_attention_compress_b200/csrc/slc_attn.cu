@@ -219,6 +219,7 @@ cudaError_t launch(const FwdArgs& a, cudaStream_t st) {
 }  // namespace
 
 cudaError_t launch_slc_attn(const FwdArgs& a, cudaStream_t st) {
+  if (slc_attn_tc_supported(a)) return launch_slc_attn_tc(a, st);
   if (slc_attn_tma_supported(a)) return launch_slc_attn_tma(a, st);
   if (a.cu) return cudaErrorInvalidValue;   // variable-length batches run on the tensor-core kernels only
   if (a.dk == 64 && a.dv == 64) return launch<64, 64>(a, st);

@@ -1,0 +1,788 @@
+// K3 on the fifth-generation tensor cores: selected-block attention
+// ("逐篇讲解DeepSeek、Kimi、MiniMax注意力机制新论文" §5: the top-k blocks are expanded to all
+// their tokens and attended; §10: the group's heads share every loaded block, so the
+// matrix products take the heads as one dimension).
+//
+// An item is one (token, KV group): the group's 16 query heads over the tokens of the
+// blocks the group chose for that token.  The chosen blocks are taken two at a time: a
+// pair is 128 keys, the M dimension of the tcgen05 MMAs, and the 16 heads are N:
+//   S^T = K_pair Q^T      (A = 128 key rows, K-major; B = the 16 query rows, K-major)
+//   O^T += V_pair^T P^T   (A = V^T, MN-major as TMA lays V down; B = P^T, K-major)
+// Both accumulate in TMEM (S^T: lane = key, column = head; O^T: lane = value column,
+// column = head), so no thread holds an accumulator.
+//
+// Two costs of the tensor-core path shape the design (measured on this GPU):
+//   - an MMA that accumulates into the accumulator of the MMA just before it waits for that
+//     one (about 170 cycles), while independent N = 16 MMAs take 45-60: so S^T is spread
+//     over four partial accumulators (K step k of each 64-column slab into partial k) and
+//     O^T over eight (16-key step k into partial k), and the readers add the partials;
+//   - a tcgen05.commit drains the MMA pipe: so each pair has two, one after its S (S^T
+//     ready; its K slot free) and one after its P.V (P^T buffer and V slot free), plus
+//     one per item (O^T complete).
+//
+// Persistent: one CTA per SM walks the items group-major (the CTAs running together share
+// one group's K/V in L2).  Warp roles:
+//   warp 8     TMA producer of keys: the item's block list (into shared memory), its 16
+//              query rows (3-slot item ring), each pair's K (2-slot ring of 48 KB pairs).
+//   warp 10    TMA producer of values: each pair's V (2-slot ring of 32 KB pairs).  The
+//              rings run across items.
+//   warp 9     MMA issuer (one thread): S of pair n, then the P.V of pair n - 1, so the
+//              softmax of a pair overlaps the next pair's S.  Alternate items accumulate
+//              into two O buffers, so an item's pairs overlap the previous item's epilogue.
+//   warps 0-7  softmax: warp w takes TMEM lane quadrant w % 4 (32 keys of each pair) and
+//              heads 8(w / 4) .. 8(w / 4) + 7.  p = 2^(s*scale - m) with a reference m per
+//              (quadrant, head) set from the quadrant's first valid scores of the item and
+//              never moved: the keys of quadrant q reach O^T only through partials 2q and
+//              2q + 1, so the epilogue brings the quadrants to a common reference and no
+//              warp waits for another.  P^T (bf16) goes to shared memory; each thread keeps
+//              its keys' partial row sums, added up once per item.
+//   warps 8-11 epilogue, one quadrant of value columns each: acc += g_slc * O / l.
+//
+// A later score can exceed its fixed reference without bound, so p is not bounded by 1.
+// fp32 and bf16 carry such values exactly up to 2^127; an item whose row sum in any
+// quadrant passes 2^64 (or is not finite) is not written but listed, and a second kernel
+// recomputes the listed items with an exact two-pass softmax on the CUDA cores.  Scores that
+// far apart do not occur in attention over trained or random keys; the path keeps the result
+// right when they do.
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace nsa {
+
+namespace {
+constexpr int kSoftWarps = 8;                      // warps 0-7
+constexpr int kEpiWarp0 = 8;                       // warps 8-11
+constexpr int kTmaWarp = 12, kMmaWarp = 13, kTmaVWarp = 14;
+constexpr int kThreads = 480;
+constexpr int kHH = 8;                             // heads per softmax warp
+constexpr int kBlk = 64;
+constexpr int kG = 16;                             // heads per group: the MMA N
+constexpr int kKSlots = 2, kVSlots = 2;            // pair slots (also the P^T buffers: pair n uses n % 2)
+static_assert(kKSlots == 2 && kVSlots == 2, "the MMA thread takes slots and phases from the pair counter's low bits");
+constexpr int kItemSlots = 3;
+constexpr uint32_t kBox = kBlk * 128;              // 64 rows x 64 bf16 (128-byte swizzle): 8 KB
+constexpr uint32_t kSlab = 2 * kBox;               // the pair's 128 rows x 64 columns: 16 KB
+constexpr int kSChains = 4, kOChains = 8;          // partial accumulators of S^T and O^T
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;                      // S buffer b, partial c: 64b + 16c
+constexpr uint32_t kColO = 2 * kSChains * kG;      // O buffer b, partial c: 128 + 128b + 16c
+constexpr float kRowSumLimit = 18446744073709551616.f;   // 2^64: above it the item is recomputed
+constexpr int kMetaInts = 36;                      // per item slot: 32 block ids, the count
+
+enum Err { kErrQEmpty = 61, kErrQFull, kErrKEmpty, kErrKFull, kErrVEmpty, kErrVFull, kErrSEmpty, kErrSFull,
+           kErrPEmpty, kErrPFull, kErrOEmpty, kErrOFull, kErrLEmpty, kErrLFull };
+
+template <int DK, int DV>
+struct Smem {
+  static constexpr int kKS = DK / 64, kVS = DV / 64;
+  static constexpr uint32_t kKBytes = kKS * kSlab, kVBytes = kVS * kSlab;   // a pair's K or V slabs
+  static constexpr uint32_t kK = 0;                                    // [K slot]
+  static constexpr uint32_t kV = kK + kKSlots * kKBytes;               // [V slot]
+  static constexpr uint32_t kQBytes = kKS * kG * 128;                  // 16 rows x DK: kKS boxes of 2 KB
+  static constexpr uint32_t kQ = kV + kVSlots * kVBytes;               // [item slot]
+  static constexpr uint32_t kPBytes = 2 * kG * 128;                    // P^T: [key half][16 heads][128 B]
+  static constexpr uint32_t kP = kQ + kItemSlots * kQBytes;            // [2]
+  static constexpr uint32_t kMeta = kP + 2 * kPBytes;                  // [item slot][kMetaInts]
+  static constexpr uint32_t kLsum = kMeta + kItemSlots * kMetaInts * 4;   // [2][quadrant][16] row sums
+  static constexpr uint32_t kRef = kLsum + 2 * 4 * kG * 4;                 // [quadrant][16] first-pair maxima
+  static constexpr uint32_t kBar = (kRef + 4 * kG * 4 + 7) & ~7u;
+  static constexpr int kNumBars = 2 * kItemSlots + 2 * kKSlots + 2 * kVSlots + 2 + 2 * 2 + 2 * 2;
+  static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
+  static constexpr uint32_t kBytes = kTmemSlot + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;
+  static_assert(kAlloc <= 232448, "shared memory");
+  static_assert(kQ % 1024 == 0 && kQBytes % 1024 == 0 && kP % 1024 == 0, "swizzled tiles need 1 KB alignment");
+};
+
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// the sum of the n partial accumulators (16 columns each, consecutive) of this thread's lane
+template <int N>
+__device__ __forceinline__ void tmem_sum_partials(uint32_t addr, float (&x)[kG]) {
+  float y[kG];
+  tc::tmem_ld16(addr, x);
+  tc::tmem_ld16(addr + kG, y);
+  tc::tmem_wait_ld();
+#pragma unroll
+  for (int h = 0; h < kG; ++h) x[h] += y[h];
+#pragma unroll
+  for (int c = 2; c < N; ++c) {
+    tc::tmem_ld16(addr + c * kG, y);
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int h = 0; h < kG; ++h) x[h] += y[h];
+  }
+}
+
+template <int DK, int DV, bool VARLEN>
+__global__ void __launch_bounds__(kThreads, 1)
+slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ gates,
+                   const int32_t* __restrict__ idx, float* __restrict__ acc, int B, int T, int Hq, int Hkv,
+                   int top_k, float scale_log2, const int32_t* __restrict__ cu_in, int* __restrict__ redo_count,
+                   int* __restrict__ redo_list, int* __restrict__ err) {
+  using SM = Smem<DK, DV>;
+  static_assert(DV == 128, "the value columns are the 128 TMEM lanes of O^T");
+  const int32_t* cu = VARLEN ? cu_in : nullptr;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem + SM::kK;
+  uint8_t* sV = smem + SM::kV;
+  uint8_t* sQ = smem + SM::kQ;
+  uint8_t* sP = smem + SM::kP;
+  int* sMeta = reinterpret_cast<int*>(smem + SM::kMeta);
+  float* sLsum = reinterpret_cast<float*>(smem + SM::kLsum);               // [2][quadrant][16]
+  float* sRef = reinterpret_cast<float*>(smem + SM::kRef);                 // [quadrant][16]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
+  // Pair n (counted over the CTA's whole walk) uses K slot, V slot, S buffer and P^T buffer n % 2.
+  uint64_t* q_full = bars;                       // [item slot] block list written and queries landed
+  uint64_t* q_empty = q_full + kItemSlots;       // [item slot] the softmax warps are done with the item
+  uint64_t* k_full = q_empty + kItemSlots;       // [K slot]
+  uint64_t* s_done = k_full + kKSlots;           // [K slot] S of the pair is done: S^T ready, K slot free
+  uint64_t* v_full = s_done + kKSlots;           // [V slot]
+  uint64_t* pv_done = v_full + kVSlots;          // [V slot] P.V of the pair is done: V slot and P^T free
+  uint64_t* p_full = pv_done + kVSlots;          // [2] P^T of the pair is in buffer n % 2 (its S^T is read)
+  uint64_t* o_full = p_full + 2;                 // [2] an item's O^T is complete
+  uint64_t* o_empty = o_full + 2;                // [2] the epilogue has read it
+  uint64_t* l_full = o_empty + 2;                // [2] an item's row sums are in shared memory
+  uint64_t* l_empty = l_full + 2;                // [2] the epilogue has read them
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int i = 0; i < kItemSlots; ++i) {
+      tc::mbar_init(q_full + i, 1);
+      tc::mbar_init(q_empty + i, kSoftWarps);
+    }
+    for (int i = 0; i < kKSlots; ++i) {
+      tc::mbar_init(k_full + i, 1);
+      tc::mbar_init(s_done + i, 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
+      tc::mbar_init(v_full + i, 1);
+      tc::mbar_init(pv_done + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(p_full + i, kSoftWarps);
+      tc::mbar_init(o_full + i, 1);
+      tc::mbar_init(o_empty + i, 4);
+      tc::mbar_init(l_full + i, kSoftWarps);
+      tc::mbar_init(l_empty + i, 4);
+    }
+    tc::fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tc::tmem_alloc(tmem_slot, kTmemCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // item it = (group, batch, token), group-major; in a variable-length batch the tokens
+  // past a sequence's end are no items, and every role skips them alike
+  const long total = (long)Hkv * B * T;
+  const long stride = gridDim.x;
+  auto next_item = [&](long it) {
+    if constexpr (VARLEN)
+      while (it < total && (int)(it % T) >= seq_len(cu, (int)((it / T) % B), T)) it += stride;
+    return it;
+  };
+  auto row_of = [&](int b, int t) -> size_t {   // row of token t of sequence b in q, k, v, gates, acc
+    if constexpr (VARLEN) return (size_t)seq_base(cu, b, T) + t;
+    else return (size_t)b * T + t;
+  };
+
+  if (warp == kTmaWarp || warp == kTmaVWarp) {
+    // ------------------------------------------------------------ TMA producers (the whole
+    // warp loops; lane 0 issues the copies).  Warp kTmaWarp: block lists, queries and keys;
+    // warp kTmaVWarp: values.
+    const bool keys = warp == kTmaWarp;
+    if (lane == 0) {
+      tc::prefetch_tmap(keys ? &tm_k : &tm_v);
+      if (keys) tc::prefetch_tmap(&tm_q);
+    }
+    const int nslots = keys ? kKSlots : kVSlots;
+    const int nslab = keys ? SM::kKS : SM::kVS;
+    const uint32_t slot_bytes = keys ? SM::kKBytes : SM::kVBytes;
+    uint8_t* const ring = keys ? sK : sV;
+    uint64_t* const full = keys ? k_full : v_full;
+    uint64_t* const done = keys ? s_done : pv_done;   // the pair that used the slot before is done with it
+    const CUtensorMap* const map = keys ? &tm_k : &tm_v;
+    long k = 0, f = 0;
+    bool ok = true;
+    for (long it = next_item(blockIdx.x); it < total && ok; it = next_item(it + stride), ++k) {
+      const int g = (int)(it / ((long)B * T));
+      const int bt = (int)(it % ((long)B * T));
+      const int b = bt / T, t = bt % T;
+      const int base = (int)row_of(b, 0);
+      int j = lane < top_k ? idx[(((size_t)b * Hkv + g) * T + t) * top_k + lane] : -1;
+      j = j >= 0 ? min(j, t / kBlk) : -1;
+      const int nblk = __popc(__ballot_sync(0xffffffffu, j >= 0));   // the list is -1 padded at its end
+      if (keys) {
+        const int qs = (int)(k % kItemSlots);
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(q_empty + qs, (uint32_t)(((k / kItemSlots) & 1) ^ 1), err,
+                                                   kErrQEmpty));
+        if (!ok) break;
+        int* meta = sMeta + qs * kMetaInts;
+        if (lane < nblk) meta[lane] = j;
+        if (lane == 0) meta[32] = nblk;
+        __threadfence_block();
+        __syncwarp();
+        if (lane == 0) {
+          tc::mbar_expect_tx(q_full + qs, SM::kQBytes);   // also publishes the block list
+          for (int s = 0; s < SM::kKS; ++s)
+            tc::tma_load_3d(sQ + qs * SM::kQBytes + s * kG * 128, &tm_q, q_full + qs, s * 64, g * kG, base + t);
+        }
+      }
+      const int npairs = (nblk + 1) / 2;
+      for (int p = 0; p < npairs && ok; ++p, ++f) {
+        const int j0 = __shfl_sync(0xffffffffu, j, 2 * p);
+        const int j1r = __shfl_sync(0xffffffffu, j, (2 * p + 1) & 31);
+        const int j1 = 2 * p + 1 < nblk ? j1r : j0;   // an odd count repeats the block (masked out)
+        const int slot = (int)(f % nslots);
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(done + slot, (uint32_t)(((f / nslots) & 1) ^ 1), err,
+                                                   keys ? kErrKEmpty : kErrVEmpty));
+        if (!ok) break;
+        if (lane == 0) {
+          uint8_t* dst = ring + slot * slot_bytes;
+          tc::mbar_expect_tx(full + slot, slot_bytes);
+          for (int s = 0; s < nslab; ++s) {
+            tc::tma_load_3d(dst + s * kSlab, map, full + slot, s * 64, g, base + j0 * kBlk);
+            tc::tma_load_3d(dst + s * kSlab + kBox, map, full + slot, s * 64, g, base + j1 * kBlk);
+          }
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) {   // let the copies in flight land (bounded)
+      for (long x = f - 1; x >= 0 && x >= f - nslots; --x)
+        tc::mbar_wait(full + (x % nslots), (uint32_t)((x / nslots) & 1), err, keys ? kErrKFull : kErrVFull);
+      if (keys)
+        for (long x = k - 1; x >= 0 && x >= k - kItemSlots; --x)
+          tc::mbar_wait(q_full + (x % kItemSlots), (uint32_t)((x / kItemSlots) & 1), err, kErrQFull);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    // The pairs of all items form one stream.  Once P^T of pair n is ready the thread issues
+    // the P.V of pair n, then the S of pair n + 2, while the softmax of pair n + 1 runs (S
+    // buffer n % 2 is free again once P^T of pair n is written).  The two products stay in
+    // blocks of their own: alternating MMAs of the K-major S with those of the MN-major V^T
+    // slowed both down.  An item without pairs takes a place in the stream too, so that its
+    // (empty) O is committed in order.
+    if (tc::elect_one()) {
+      const uint32_t idS = tc::idesc_bf16(128, kG, 0, 0);    // S^T = K Q^T: both K-major
+      const uint32_t idPV = tc::idesc_bf16(128, kG, 1, 0);   // O^T = V^T P^T: V^T MN-major, P^T K-major
+      const uint64_t dp0 = tc::sdesc(sP, 16, 1024);
+      // A stream entry: pair f (or an item without pairs) of the item with counter k (k's low
+      // bit picks its O buffer) in item slot qs.  Everything the issuing thread computes per
+      // entry is 32-bit adds, compares and bit operations: this one thread issues every MMA.
+      struct Entry { uint32_t f, k; int qs; bool first, last, pair; };
+      long it_c = next_item(blockIdx.x);
+      uint32_t k_c = 0, f_c = 0, qph = 0;   // qph: the phase bit of item slot qs_c
+      int qs_c = 0, p_c = 0, np_c = -1;
+      bool ok = true;
+      auto next_entry = [&](Entry& e) -> bool {   // false: the walk is over (or a wait failed)
+        if (it_c >= total) return false;
+        if (np_c < 0) {
+          ok = tc::mbar_wait(q_full + qs_c, qph, err, kErrQFull);
+          if (!ok) return false;
+          np_c = (sMeta[qs_c * kMetaInts + 32] + 1) >> 1;
+          p_c = 0;
+        }
+        e.k = k_c;
+        e.qs = qs_c;
+        e.pair = np_c != 0;
+        e.f = f_c;
+        e.first = p_c == 0;
+        e.last = p_c == np_c - 1;
+        if (e.pair) {
+          ++f_c;
+          ++p_c;
+        }
+        if (!e.pair || p_c == np_c) {   // the item is done: move to the next
+          it_c = next_item(it_c + stride);
+          ++k_c;
+          np_c = -1;
+          if (++qs_c == kItemSlots) {
+            qs_c = 0;
+            qph ^= 1u;
+          }
+        }
+        return true;
+      };
+      // S MMA number i of a pair (12 for d_k = 192): K step (i % 4) of slab (i / 4) into partial i % 4
+      auto s_mma = [&](const Entry& y, int i, uint64_t dk0, uint64_t dq0) {
+        const int sl = i >> 2, kk = i & 3;
+        tc::mma_ss(tmem + kColS + kSChains * kG * (uint32_t)(y.f & 1) + kG * kk,
+                   dk0 + (uint64_t)((sl * kSlab + kk * 32) / 16), dq0 + (uint64_t)((sl * kG * 128 + kk * 32) / 16), idS,
+                   sl != 0);
+      };
+      // the K slot of pair y (its S buffer is free: P^T of the pair two back is written,
+      // which the softmax warps do after reading that pair's S^T)
+      auto wait_s = [&](const Entry& y) -> bool {
+        return tc::mbar_wait(k_full + (y.f & 1), (y.f >> 1) & 1u, err, kErrKFull);
+      };
+      Entry q0{}, q1{};   // the stream entries whose S is issued and P.V not yet (two registers, no array)
+      int nq = 0;
+      // prologue: the S of the first two pairs
+      while (ok && nq < 2) {
+        Entry e;
+        if (!next_entry(e)) break;
+        if (e.pair) {
+          if (!(ok = wait_s(e))) break;
+          tc::tc_fence_after();
+          const uint64_t dk0 = tc::sdesc(sK + (e.f & 1) * SM::kKBytes, 16, 1024);
+          const uint64_t dq0 = tc::sdesc(sQ + e.qs * SM::kQBytes, 16, 1024);
+#pragma unroll 4
+          for (int i = 0; i < 4 * SM::kKS; ++i) s_mma(e, i, dk0, dq0);
+          tc::mma_commit(s_done + (e.f & 1));
+        }
+        if (nq == 0) q0 = e;
+        else q1 = e;
+        ++nq;
+      }
+      while (ok && nq > 0) {
+        const Entry x = q0;
+        Entry y;
+        const bool have_y = next_entry(y);
+        if (!ok) break;
+        const bool s_next = have_y && y.pair;
+        if (s_next && !(ok = wait_s(y))) break;
+        const int ob = (int)(x.k & 1);
+        if (x.pair) {
+          const int vs = (int)(x.f & 1);
+          ok = (!x.first || tc::mbar_wait(o_empty + ob, ((x.k >> 1) & 1u) ^ 1u, err, kErrOEmpty)) &&
+               tc::mbar_wait(v_full + vs, (x.f >> 1) & 1u, err, kErrVFull) &&
+               tc::mbar_wait(p_full + vs, (x.f >> 1) & 1u, err, kErrPFull);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint64_t dv0 = tc::sdesc(sV + vs * SM::kVBytes, kSlab, 1024);
+          const uint64_t dp = dp0 + (uint64_t)((x.f & 1) * SM::kPBytes / 16);
+          const uint32_t d_o = tmem + kColO + kOChains * kG * ob;
+          const uint32_t accum = x.first ? 0u : 1u;
+          uint64_t dk0 = 0, dq0 = 0;
+          if (s_next) {
+            dk0 = tc::sdesc(sK + (y.f & 1) * SM::kKBytes, 16, 1024);
+            dq0 = tc::sdesc(sQ + y.qs * SM::kQBytes, 16, 1024);
+          }
+#pragma unroll
+          for (int ks = 0; ks < 2 * kBlk / 16; ++ks)   // 16-key step ks into partial ks
+            tc::mma_ss(d_o + kG * ks, dv0 + (uint64_t)(ks * 16 * 128 / 16),
+                       dp + (uint64_t)(((ks >> 2) * (kG * 128) + (ks & 3) * 32) / 16), idPV, accum);
+          tc::mma_commit(pv_done + vs);
+          if (x.last) tc::mma_commit(o_full + ob);
+          if (s_next) {
+#pragma unroll 4
+            for (int i = 0; i < 4 * SM::kKS; ++i) s_mma(y, i, dk0, dq0);
+            tc::mma_commit(s_done + (y.f & 1));
+          }
+        } else {   // an item without pairs: its empty O, in order
+          if (!(ok = tc::mbar_wait(o_empty + ob, ((x.k >> 1) & 1u) ^ 1u, err, kErrOEmpty))) break;
+          if (s_next) {
+            tc::tc_fence_after();
+            const uint64_t dk0 = tc::sdesc(sK + (y.f & 1) * SM::kKBytes, 16, 1024);
+            const uint64_t dq0 = tc::sdesc(sQ + y.qs * SM::kQBytes, 16, 1024);
+#pragma unroll 4
+            for (int i = 0; i < 4 * SM::kKS; ++i) s_mma(y, i, dk0, dq0);
+            tc::mma_commit(s_done + (y.f & 1));
+          }
+          tc::mma_commit(o_full + ob);
+        }
+        q0 = q1;
+        if (have_y) q1 = y;
+        else --nq;
+      }
+    }
+  } else if (warp < kSoftWarps) {
+    // ------------------------------------------------------------ softmax
+    const int qd = warp & 3;                           // TMEM lane quadrant: keys 32qd .. 32qd + 31
+    const int h0 = kHH * (warp >> 2);                  // this warp's heads h0 .. h0 + 7
+    const int r = 32 * qd + lane;                      // this thread's key of the pair
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * qd) << 16) + h0;
+    // this thread's column of P^T (K-major, 128-byte swizzle): key half, 16-byte chunk, element
+    uint8_t* const pcol = sP + (r >> 6) * (kG * 128) + 2 * (r & 7);
+    const int pchunk = (r & 63) >> 3;
+    const int bar_g = 1 + (warp >> 2);               // named barrier of the four warps of this head half
+    long k = 0, f = 0;
+    bool ok = true;
+    for (long it = next_item(blockIdx.x); it < total; it = next_item(it + stride), ++k) {
+      const int t = (int)((it % ((long)B * T)) % T);
+      const int qs = (int)(k % kItemSlots);
+      // one decision for the four warps, which meet at a barrier in the item's first pair;
+      // after a failed wait they leave together
+      ok = tc::vote_all(bar_g, 4 * 32,
+                        ok && tc::mbar_wait(q_full + qs, (uint32_t)((k / kItemSlots) & 1), err, kErrQFull));
+      if (!ok) break;
+      const int* meta = sMeta + qs * kMetaInts;
+      const int nblk = meta[32];
+      const int npairs = (nblk + 1) / 2;
+      float m[kHH], lp[kHH];                           // reference (log2 units) and partial row sums
+#pragma unroll
+      for (int h = 0; h < kHH; ++h) {
+        m[h] = -INFINITY;
+        lp[h] = 0.f;
+      }
+      for (int p = 0; p < npairs; ++p, ++f) {
+        const int sb = (int)(f & 1);
+        ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_done + (f % kKSlots), (uint32_t)((f / kKSlots) & 1),
+                                                         err, kErrSFull));
+        float x[kHH], y[kHH];
+#pragma unroll
+        for (int h = 0; h < kHH; ++h) x[h] = 0.f;
+        tc::tc_fence_after();
+        if (ok) {
+          const uint32_t sa = lane_addr + kColS + kSChains * kG * sb;
+          tc::tmem_ld8(sa, x);
+          tc::tmem_ld8(sa + kG, y);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) x[h] += y[h];
+#pragma unroll
+          for (int c = 2; c < kSChains; ++c) {
+            tc::tmem_ld8(sa + c * kG, y);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) x[h] += y[h];
+          }
+        }
+        tc::tc_fence_before();   // the S^T reads are ordered before the P^T arrival below
+        const int jj = 2 * p + (r >> 6);
+        const int j = jj < nblk ? meta[jj] : -1;
+        const bool valid = j >= 0 && j * kBlk + (r & 63) <= t;
+        // the reference: per head, the largest valid score of the item's first pair over the
+        // four quadrants (the first key of the first pair is always valid)
+        if (p == 0) {
+          float wm[kHH];
+#pragma unroll
+          for (int h = 0; h < kHH; ++h) wm[h] = warp_max_f32(valid ? x[h] : -INFINITY);
+          if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < kHH; ++h) sRef[qd * kG + h0 + h] = wm[h];
+          }
+          const bool all_ok = tc::vote_all(bar_g, 4 * 32, ok);
+#pragma unroll
+          for (int h = 0; h < kHH; ++h)
+            m[h] = fmaxf(fmaxf(sRef[h0 + h], sRef[kG + h0 + h]), fmaxf(sRef[2 * kG + h0 + h], sRef[3 * kG + h0 + h])) *
+                   scale_log2;
+          tc::named_sync(bar_g, 4 * 32);   // read before the next item rewrites it
+          ok = all_ok;
+          if (!ok) break;                  // all four warps together
+        }
+        // after a failed wait a warp runs out the item's pairs doing nothing; the four warps
+        // leave together at the next item's vote
+        if (!ok) continue;
+        uint32_t pk[kHH / 2];
+#pragma unroll
+        for (int h = 0; h < kHH; h += 2) {
+          const float p0 = valid ? ex2(fmaf(x[h], scale_log2, -m[h])) : 0.f;
+          const float p1 = valid ? ex2(fmaf(x[h + 1], scale_log2, -m[h + 1])) : 0.f;
+          lp[h] += p0;
+          lp[h + 1] += p1;
+          pk[h / 2] = pack_bf16(p0, p1);
+        }
+        // P^T goes to buffer f % 2 once the P.V of the pair two back has read it
+        if (f >= 2)
+          ok = __all_sync(0xffffffffu, tc::mbar_wait(pv_done + (f & 1), (uint32_t)(((f >> 1) & 1) ^ 1), err,
+                                                     kErrPEmpty));
+        if (!ok) continue;
+        uint8_t* const pc = pcol + (f & 1) * SM::kPBytes;
+#pragma unroll
+        for (int h = 0; h < kHH; ++h)
+          *reinterpret_cast<uint16_t*>(pc + (h0 + h) * 128 + ((pchunk ^ (h & 7)) << 4)) =
+              (uint16_t)(pk[h / 2] >> (16 * (h & 1)));
+        tc::fence_async_smem();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(p_full + (f & 1));
+      }
+      if (!ok) continue;   // the next item's vote ends the walk
+      // the item's row sums of this quadrant: reduce the 8 partial sums over the warp's 32
+      // keys (each step halves the heads a lane keeps); lane 4i holds head h0 + i
+      float a4[4], a2[2], a1;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bool hi = lane & 16;
+        const float send = hi ? lp[i] : lp[i + 4];
+        a4[i] = (hi ? lp[i + 4] : lp[i]) + __shfl_xor_sync(0xffffffffu, send, 16);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const bool hi = lane & 8;
+        const float send = hi ? a4[i] : a4[i + 2];
+        a2[i] = (hi ? a4[i + 2] : a4[i]) + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+      {
+        const bool hi = lane & 4;
+        const float send = hi ? a2[0] : a2[1];
+        a1 = (hi ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+      a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, 1);       // head h0 + ((lane >> 2) & 7)
+      const int ob = (int)(k & 1);
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(l_empty + ob, (uint32_t)(((k >> 1) & 1) ^ 1), err, kErrLEmpty));
+      if (!ok) continue;
+      if ((lane & 3) == 0) sLsum[(ob * 4 + qd) * kG + h0 + (lane >> 2)] = a1;
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(l_full + ob);
+        tc::mbar_arrive(q_empty + qs);                 // done with the item's block list and queries
+      }
+    }
+  } else if (warp < kEpiWarp0 + 4) {
+    // ------------------------------------------------------------ epilogue: acc += g_slc O / l
+    const int qd = warp & 3;
+    const int d = 32 * qd + lane;                      // this thread's value column
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * qd) << 16);
+    long k = 0;
+    bool ok = true;
+    for (long it = next_item(blockIdx.x); it < total && ok; it = next_item(it + stride), ++k) {
+      const int g = (int)(it / ((long)B * T));
+      const int bt = (int)(it % ((long)B * T));
+      const size_t row0 = row_of(bt / T, bt % T) * Hq + (size_t)g * kG;   // (token, head 0 of the group)
+      // start the accumulator rows (this warp's 128-byte column segment of each head row) and
+      // the gates on their way to L2; they are read after the item's O is complete
+      if (lane < kG) prefetch_l2(acc + (row0 + lane) * DV + 32 * qd);
+      if (lane == kG) prefetch_l2(gates + row0 * 3);
+      const int ob = (int)(k & 1);
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(l_full + ob, (uint32_t)((k >> 1) & 1), err, kErrLFull));
+      if (!ok) break;
+      // the row sums of the four quadrants (all taken against the same reference)
+      const float* ls = sLsum + ob * 4 * kG;
+      float L[kG];
+      bool bad = false;
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        const float l0 = ls[h], l1 = ls[kG + h], l2 = ls[2 * kG + h], l3 = ls[3 * kG + h];
+        bad = bad || !(l0 <= kRowSumLimit && l1 <= kRowSumLimit && l2 <= kRowSumLimit && l3 <= kRowSumLimit);
+        L[h] = (l0 + l1) + (l2 + l3);
+      }
+      float o[kG];
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(o_full + ob, (uint32_t)((k >> 1) & 1), err, kErrOFull));
+      if (!ok) break;
+      tc::tc_fence_after();
+      tmem_sum_partials<kOChains>(lane_addr + kColO + kOChains * kG * ob, o);
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        tc::mbar_arrive(o_empty + ob);
+        tc::mbar_arrive(l_empty + ob);
+      }
+      if (bad) {   // a row sum out of range: the item is recomputed exactly by the redo kernel
+        if (qd == 0 && lane == 0) redo_list[atomicAdd(redo_count, 1)] = (int)it;
+        continue;
+      }
+      float a[kG];
+#pragma unroll
+      for (int h = 0; h < kG; ++h) {
+        a[h] = acc[(row0 + h) * DV + d];
+        L[h] = L[h] > 0.f ? __bfloat162float(gates[(row0 + h) * 3 + 1]) / L[h] : 0.f;
+      }
+#pragma unroll
+      for (int h = 0; h < kG; ++h)
+        if (L[h] != 0.f) acc[(row0 + h) * DV + d] = a[h] + L[h] * o[h];
+    }
+  }
+
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// The exact path for the items the tensor-core kernel listed (a row sum out of range):
+// one CTA per listed item, fp32 on the CUDA cores, a two-pass softmax per head (the
+// largest score first, then the probabilities), acc += g_slc * o_slc.  Shared memory:
+// the item's queries, its key rows' positions and the [keys][16] scores.
+constexpr int kRedoThreads = 256;
+constexpr int kRedoMaxKeys = 32 * kBlk;
+
+template <int DK>
+struct RedoSmem {
+  static constexpr uint32_t kScores = 0;                                  // [key][16] float
+  static constexpr uint32_t kQ = kScores + kRedoMaxKeys * kG * 4;         // [16][DK] float
+  static constexpr uint32_t kKeys = kQ + kG * DK * 4;                     // [key] token positions
+  static constexpr uint32_t kRed = kKeys + kRedoMaxKeys * 4;              // [16][16] float
+  static constexpr uint32_t kBytes = kRed + 2 * kG * kG * 4 + 16;
+};
+
+template <int DK, int DV, bool VARLEN>
+__global__ void __launch_bounds__(kRedoThreads)
+slc_redo_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ gates,
+                const int32_t* __restrict__ idx, float* __restrict__ acc, int B, int T, int Hq, int Hkv, int top_k,
+                float scale_log2, const int32_t* __restrict__ cu_in, const int* __restrict__ redo_count,
+                const int* __restrict__ redo_list) {
+  using RS = RedoSmem<DK>;
+  const int32_t* cu = VARLEN ? cu_in : nullptr;
+  extern __shared__ __align__(16) uint8_t rsm[];
+  float* sS = reinterpret_cast<float*>(rsm + RS::kScores);
+  float* sQ = reinterpret_cast<float*>(rsm + RS::kQ);
+  int* sU = reinterpret_cast<int*>(rsm + RS::kKeys);
+  float* sRed = reinterpret_cast<float*>(rsm + RS::kRed);   // [16 slices][16 heads], then [16] maxima, [16] sums
+  int* sN = reinterpret_cast<int*>(sRed + 2 * kG * kG);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = *redo_count;
+  for (int i = blockIdx.x; i < n; i += gridDim.x) {
+    const long it = redo_list[i];
+    const int g = (int)(it / ((long)B * T));
+    const int bt = (int)(it % ((long)B * T));
+    const int b = bt / T, t = bt % T;
+    const size_t base = VARLEN ? (size_t)seq_base(cu, b, T) : (size_t)b * T;
+    const size_t qrow = ((base + t) * Hq + (size_t)g * kG);
+    __syncthreads();   // the previous item is done with shared memory
+    for (int x = tid; x < kG * DK; x += kRedoThreads) sQ[x] = __bfloat162float(q[qrow * DK + x]);
+    if (tid == 0) {   // the key positions: the chosen blocks' tokens u <= t
+      int nk = 0;
+      for (int jj = 0; jj < top_k; ++jj) {
+        const int j = idx[(((size_t)b * Hkv + g) * T + t) * top_k + jj];
+        if (j < 0) break;
+        const int jb = min(j, t / kBlk);
+        for (int u = jb * kBlk; u < jb * kBlk + kBlk && u <= t; ++u) sU[nk++] = u;
+      }
+      *sN = nk;
+    }
+    __syncthreads();
+    const int nk = *sN;
+    // scores, scaled to log2 units: warp per key, lane = (head, half of the dot product)
+    {
+      const int h = lane & 15, half = lane >> 4;
+      for (int e = warp; e < nk; e += kRedoThreads / 32) {
+        const __nv_bfloat16* kr = k + ((base + sU[e]) * Hkv + g) * DK;
+        float a = 0.f;
+        for (int c = half * (DK / 2); c < (half + 1) * (DK / 2); ++c) a += sQ[h * DK + c] * __bfloat162float(kr[c]);
+        a += __shfl_xor_sync(0xffffffffu, a, 16);
+        if (half == 0) sS[e * kG + h] = a * scale_log2;
+      }
+    }
+    __syncthreads();
+    // per head: the largest score, then p = 2^(s - max) in place and the row sum
+    {
+      const int h = tid & 15, sl = tid >> 4;   // 16 slices of the keys
+      float mx = -INFINITY;
+      for (int e = sl; e < nk; e += 16) mx = fmaxf(mx, sS[e * kG + h]);
+      sRed[sl * kG + h] = mx;
+      __syncthreads();
+      if (tid < kG) {
+        float m2 = -INFINITY;
+        for (int x = 0; x < 16; ++x) m2 = fmaxf(m2, sRed[x * kG + tid]);
+        sRed[kG * kG + tid] = m2;
+      }
+      __syncthreads();
+      const float m2 = sRed[kG * kG + h];
+      float l = 0.f;
+      for (int e = sl; e < nk; e += 16) {
+        const float pr = exp2f(sS[e * kG + h] - m2);
+        sS[e * kG + h] = pr;
+        l += pr;
+      }
+      __syncthreads();
+      sRed[sl * kG + h] = l;
+      __syncthreads();
+      if (tid < kG) {
+        float l2 = 0.f;
+        for (int x = 0; x < 16; ++x) l2 += sRed[x * kG + tid];
+        sRed[kG * kG + kG + tid] = l2;
+      }
+      __syncthreads();
+    }
+    // o_slc: thread = (head, 8 value columns)
+    {
+      const int h = tid >> 4, d0 = (tid & 15) * (DV / 16);
+      float o[DV / 16];
+#pragma unroll
+      for (int x = 0; x < DV / 16; ++x) o[x] = 0.f;
+      for (int e = 0; e < nk; ++e) {
+        const float pr = sS[e * kG + h];
+        const __nv_bfloat16* vr = v + ((base + sU[e]) * Hkv + g) * DV + d0;
+#pragma unroll
+        for (int x = 0; x < DV / 16; ++x) o[x] += pr * __bfloat162float(vr[x]);
+      }
+      const float L = sRed[kG * kG + kG + h];
+      const float gs = __bfloat162float(gates[(qrow + h) * 3 + 1]);
+      const float scl = L > 0.f ? gs / L : 0.f;
+      float* ar = acc + (qrow + h) * DV + d0;
+#pragma unroll
+      for (int x = 0; x < DV / 16; ++x) ar[x] += scl * o[x];
+    }
+  }
+}
+
+template <int DK, int DV>
+cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
+  using SM = Smem<DK, DV>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(slc_attn_tc_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(slc_attn_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)SM::kAlloc);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(slc_redo_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)RedoSmem<DK>::kBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(slc_redo_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)RedoSmem<DK>::kBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  CUtensorMap mk, mv, mq;
+  const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.total};
+  const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
+  const uint64_t dv3[3] = {(uint64_t)DV, (uint64_t)a.Hkv, (uint64_t)a.total};
+  const uint64_t sv3[2] = {(uint64_t)DV * 2, (uint64_t)a.Hkv * DV * 2};
+  const uint32_t box[3] = {64, 1, kBlk};
+  const uint64_t dq3[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.total};
+  const uint64_t sq3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
+  const uint32_t qbox[3] = {64, (uint32_t)kG, 1};
+  if (!make_tmap_bf16(&mk, a.k, 3, dk3, sk3, box) || !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, box) ||
+      !make_tmap_bf16(&mq, a.q, 3, dq3, sq3, qbox))
+    return cudaErrorInvalidValue;
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  const long items = (long)a.Hkv * a.B * a.T;
+  const int grid = (int)(items < sms ? items : sms);
+  auto kernel = a.cu ? slc_attn_tc_kernel<DK, DV, true> : slc_attn_tc_kernel<DK, DV, false>;
+  kernel<<<grid, kThreads, SM::kAlloc, st>>>(mk, mv, mq, static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc,
+                                             a.B, a.T, a.Hq, a.Hkv, a.top_k, a.scale_log2, a.cu, a.redo_count,
+                                             a.redo_list, a.err);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // the listed items (normally none: the CTAs read a zero count and return)
+  auto redo = a.cu ? slc_redo_kernel<DK, DV, true> : slc_redo_kernel<DK, DV, false>;
+  redo<<<grid, kRedoThreads, RedoSmem<DK>::kBytes, st>>>(
+      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+      static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.gates), a.idx, a.acc, a.B, a.T,
+      a.Hq, a.Hkv, a.top_k, a.scale_log2, a.cu, a.redo_count, a.redo_list);
+  return cudaGetLastError();
+}
+}  // namespace
+
+bool slc_attn_tc_supported(const FwdArgs& a) {
+  return a.err != nullptr && a.redo_count != nullptr && a.redo_list != nullptr && a.G == 16 && a.dv == 128 &&
+         (a.dk == 128 || a.dk == 192) && a.top_k <= 32;
+}
+
+cudaError_t launch_slc_attn_tc(const FwdArgs& a, cudaStream_t st) {
+  if (a.dk == 192 && a.dv == 128) return launch_tc<192, 128>(a, st);
+  if (a.dk == 128 && a.dv == 128) return launch_tc<128, 128>(a, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace nsa

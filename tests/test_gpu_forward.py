@@ -238,3 +238,24 @@ def test_phi_mlp_forward(shape):
     ref_out = with_forced_rows(ref["out"], swapped,
                                lambda pos: run_oracle([toks[i] for i in pos], gi[:, :, pos])["out"])
     assert_close(out.cpu()[:, toks], ref_out, what="mlp out")
+
+
+def test_far_apart_scores_take_the_exact_path():
+    """The tensor-core selected branch fixes its softmax reference at each item's first scores;
+    a key whose score lies far above them (here one key row of block 5 made 60 times the
+    all-ones vector, so that the heads with a positive q.1 score it some 80 log2 units higher)
+    makes the row sum pass the limit, and the item is recomputed exactly.  Every block is
+    selected, and the output still matches the oracle on every token."""
+    T = 700
+    x = synth.nsa_inputs(1, T, 16, 1, 192, 128, seed=18)
+    x.k[0, 5 * 64 + 7, 0] = 60.0
+    gates = synth.one_hot_gates(1, T, 16, 1)
+    dev = [t.to(DEV) for t in (x.q, x.k, x.v, gates, x.w_k, x.w_v)]
+    f = NSAForward(1, T, 16, 1, 192, 128, dev[4], dev[5], top_k=16, window=64)
+    out = f(*dev[:4]).cpu()
+    torch.cuda.synchronize()
+    assert f.device_status() == 0
+    redone = int(f.workspace[4:8].view(torch.int32).item())   # the redo count follows the status word
+    assert redone > 0, "no item took the exact path"
+    ref = oracle.nsa_forward(x.q, x.k, x.v, gates, x.w_k, x.w_v, top_k=16, window=64)
+    assert_close(out, ref["out"], what="far-apart scores")

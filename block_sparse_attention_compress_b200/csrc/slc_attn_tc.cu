@@ -11,14 +11,16 @@
 // Both accumulate in TMEM (S^T: lane = key, column = head; O^T: lane = value column,
 // column = head), so no thread holds an accumulator.
 //
-// Two costs of the tensor-core path shape the design (measured on this GPU):
+// The costs that shape the design (measured on this GPU):
 //   - an MMA that accumulates into the accumulator of the MMA just before it waits for that
 //     one (about 170 cycles), while independent N = 16 MMAs take 45-60: so S^T is spread
 //     over four partial accumulators (K step k of each 64-column slab into partial k) and
 //     O^T over eight (16-key step k into partial k), and the readers add the partials;
-//   - a tcgen05.commit drains the MMA pipe: so each pair has two, one after its S (S^T
-//     ready; its K slot free) and one after its P.V (P^T buffer and V slot free), plus
-//     one per item (O^T complete).
+//   - one thread issues every MMA, so its own work per pair (waits, commits, bookkeeping)
+//     adds to the pair's time: it waits once and commits once per pair.  Step n of the
+//     stream of pairs is the P.V of pair n and the S of pair n + 2; its "ready" barrier
+//     collects the keys of pair n + 2, the values of pair n and P^T of pair n, its "done"
+//     commit frees their slots and makes S^T of pair n + 2 readable.
 //
 // Persistent: one CTA per SM walks the items group-major (the CTAs running together share
 // one group's K/V in L2).  Warp roles:
@@ -61,7 +63,7 @@ constexpr int kHH = 8;                             // heads per softmax warp
 constexpr int kBlk = 64;
 constexpr int kG = 16;                             // heads per group: the MMA N
 constexpr int kKSlots = 2, kVSlots = 2;            // pair slots (also the P^T buffers: pair n uses n % 2)
-static_assert(kKSlots == 2 && kVSlots == 2, "the MMA thread takes slots and phases from the pair counter's low bits");
+static_assert(kKSlots == 2 && kVSlots == 2, "slots and phases come from the pair counter's low bits");
 constexpr int kItemSlots = 3;
 constexpr uint32_t kBox = kBlk * 128;              // 64 rows x 64 bf16 (128-byte swizzle): 8 KB
 constexpr uint32_t kSlab = 2 * kBox;               // the pair's 128 rows x 64 columns: 16 KB
@@ -72,8 +74,8 @@ constexpr uint32_t kColO = 2 * kSChains * kG;      // O buffer b, partial c: 128
 constexpr float kRowSumLimit = 18446744073709551616.f;   // 2^64: above it the item is recomputed
 constexpr int kMetaInts = 36;                      // per item slot: 32 block ids, the count
 
-enum Err { kErrQEmpty = 61, kErrQFull, kErrKEmpty, kErrKFull, kErrVEmpty, kErrVFull, kErrSEmpty, kErrSFull,
-           kErrPEmpty, kErrPFull, kErrOEmpty, kErrOFull, kErrLEmpty, kErrLFull };
+enum Err { kErrQEmpty = 61, kErrQFull, kErrKSlot, kErrProK, kErrVSlot, kErrReady, kErrSDone, kErrOEmpty, kErrOFull,
+           kErrLEmpty, kErrLFull };
 
 template <int DK, int DV>
 struct Smem {
@@ -89,7 +91,7 @@ struct Smem {
   static constexpr uint32_t kLsum = kMeta + kItemSlots * kMetaInts * 4;   // [2][quadrant][16] row sums
   static constexpr uint32_t kRef = kLsum + 2 * 4 * kG * 4;                 // [quadrant][16] first-pair maxima
   static constexpr uint32_t kBar = (kRef + 4 * kG * 4 + 7) & ~7u;
-  static constexpr int kNumBars = 2 * kItemSlots + 2 * kKSlots + 2 * kVSlots + 2 + 2 * 2 + 2 * 2;
+  static constexpr int kNumBars = 2 * kItemSlots + 2 + 2 + 2 + 2 + 2 * 2 + 2 * 2;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;
@@ -142,14 +144,14 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   float* sRef = reinterpret_cast<float*>(smem + SM::kRef);                 // [quadrant][16]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   // Pair n (counted over the CTA's whole walk) uses K slot, V slot, S buffer and P^T buffer n % 2.
+  // Step n = the P.V of pair n and the S of pair n + 2 (the S of pairs 0 and 1 come before).
   uint64_t* q_full = bars;                       // [item slot] block list written and queries landed
   uint64_t* q_empty = q_full + kItemSlots;       // [item slot] the softmax warps are done with the item
-  uint64_t* k_full = q_empty + kItemSlots;       // [K slot]
-  uint64_t* s_done = k_full + kKSlots;           // [K slot] S of the pair is done: S^T ready, K slot free
-  uint64_t* v_full = s_done + kKSlots;           // [V slot]
-  uint64_t* pv_done = v_full + kVSlots;          // [V slot] P.V of the pair is done: V slot and P^T free
-  uint64_t* p_full = pv_done + kVSlots;          // [2] P^T of the pair is in buffer n % 2 (its S^T is read)
-  uint64_t* o_full = p_full + 2;                 // [2] an item's O^T is complete
+  uint64_t* pro_k = q_empty + kItemSlots;        // [2] the keys of pair 0 / 1 landed
+  uint64_t* pro_done = pro_k + 2;                // [2] the S of pair 0 / 1 is done
+  uint64_t* ready = pro_done + 2;                // [n % 2] step n: K of pair n + 2, V of pair n, P^T of pair n
+  uint64_t* done = ready + 2;                    // [n % 2] step n is done: S^T of pair n + 2 ready, slots free
+  uint64_t* o_full = done + 2;                   // [2] an item's O^T is complete
   uint64_t* o_empty = o_full + 2;                // [2] the epilogue has read it
   uint64_t* l_full = o_empty + 2;                // [2] an item's row sums are in shared memory
   uint64_t* l_empty = l_full + 2;                // [2] the epilogue has read them
@@ -161,16 +163,11 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       tc::mbar_init(q_full + i, 1);
       tc::mbar_init(q_empty + i, kSoftWarps);
     }
-    for (int i = 0; i < kKSlots; ++i) {
-      tc::mbar_init(k_full + i, 1);
-      tc::mbar_init(s_done + i, 1);
-    }
-    for (int i = 0; i < kVSlots; ++i) {
-      tc::mbar_init(v_full + i, 1);
-      tc::mbar_init(pv_done + i, 1);
-    }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(p_full + i, kSoftWarps);
+      tc::mbar_init(pro_k + i, 1);
+      tc::mbar_init(pro_done + i, 1);
+      tc::mbar_init(ready + i, 2 + kSoftWarps);   // the two producers, the softmax warps
+      tc::mbar_init(done + i, 1);
       tc::mbar_init(o_full + i, 1);
       tc::mbar_init(o_empty + i, 4);
       tc::mbar_init(l_full + i, kSoftWarps);
@@ -204,20 +201,32 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
   if (warp == kTmaWarp || warp == kTmaVWarp) {
     // ------------------------------------------------------------ TMA producers (the whole
     // warp loops; lane 0 issues the copies).  Warp kTmaWarp: block lists, queries and keys;
-    // warp kTmaVWarp: values.
+    // warp kTmaVWarp: values.  An item has at least one pair: with no block chosen (never
+    // the case for a token's own list) the pair's keys are all masked.
     const bool keys = warp == kTmaWarp;
     if (lane == 0) {
       tc::prefetch_tmap(keys ? &tm_k : &tm_v);
       if (keys) tc::prefetch_tmap(&tm_q);
     }
-    const int nslots = keys ? kKSlots : kVSlots;
     const int nslab = keys ? SM::kKS : SM::kVS;
-    const uint32_t slot_bytes = keys ? SM::kKBytes : SM::kVBytes;
+    const uint32_t slot_bytes = nslab * kSlab;
     uint8_t* const ring = keys ? sK : sV;
-    uint64_t* const full = keys ? k_full : v_full;
-    uint64_t* const done = keys ? s_done : pv_done;   // the pair that used the slot before is done with it
     const CUtensorMap* const map = keys ? &tm_k : &tm_v;
-    long k = 0, f = 0;
+    // pair f's slot (f % 2) is free once the pair two back is done with it: its S for keys
+    // (step f - 4, or the prologue for f < 4), its P.V for values (step f - 2)
+    auto wait_slot = [&](uint32_t f) -> bool {
+      if (keys) {
+        if (f < 2) return true;
+        if (f < 4) return tc::mbar_wait(pro_done + (f & 1), 0u, err, kErrKSlot);
+        return tc::mbar_wait(done + (f & 1), (f >> 1) & 1u, err, kErrKSlot);
+      }
+      return tc::mbar_wait(done + (f & 1), ((f >> 1) & 1u) ^ 1u, err, kErrVSlot);
+    };
+    // where pair f's copies arrive: the keys of pairs 0 and 1 on their own barriers, the
+    // others on step f - 2 (keys) or step f (values)
+    auto arrive_bar = [&](uint32_t f) -> uint64_t* { return keys && f < 2 ? pro_k + f : ready + (f & 1); };
+    long k = 0;
+    uint32_t f = 0;
     bool ok = true;
     for (long it = next_item(blockIdx.x); it < total && ok; it = next_item(it + stride), ++k) {
       const int g = (int)(it / ((long)B * T));
@@ -243,72 +252,70 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tc::tma_load_3d(sQ + qs * SM::kQBytes + s * kG * 128, &tm_q, q_full + qs, s * 64, g * kG, base + t);
         }
       }
-      const int npairs = (nblk + 1) / 2;
+      const int npairs = max(1, (nblk + 1) / 2);
       for (int p = 0; p < npairs && ok; ++p, ++f) {
-        const int j0 = __shfl_sync(0xffffffffu, j, 2 * p);
-        const int j1r = __shfl_sync(0xffffffffu, j, (2 * p + 1) & 31);
-        const int j1 = 2 * p + 1 < nblk ? j1r : j0;   // an odd count repeats the block (masked out)
-        const int slot = (int)(f % nslots);
-        ok = __all_sync(0xffffffffu, tc::mbar_wait(done + slot, (uint32_t)(((f / nslots) & 1) ^ 1), err,
-                                                   keys ? kErrKEmpty : kErrVEmpty));
+        const int jr0 = __shfl_sync(0xffffffffu, j, (2 * p) & 31);
+        const int jr1 = __shfl_sync(0xffffffffu, j, (2 * p + 1) & 31);
+        const int j0 = 2 * p < nblk ? jr0 : t / kBlk;   // (masked: nothing was chosen)
+        const int j1 = 2 * p + 1 < nblk ? jr1 : j0;     // an odd count repeats the block (masked out)
+        ok = __all_sync(0xffffffffu, wait_slot(f));
         if (!ok) break;
         if (lane == 0) {
-          uint8_t* dst = ring + slot * slot_bytes;
-          tc::mbar_expect_tx(full + slot, slot_bytes);
+          uint8_t* dst = ring + (f & 1) * slot_bytes;
+          uint64_t* bar = arrive_bar(f);
+          tc::mbar_expect_tx(bar, slot_bytes);
           for (int s = 0; s < nslab; ++s) {
-            tc::tma_load_3d(dst + s * kSlab, map, full + slot, s * 64, g, base + j0 * kBlk);
-            tc::tma_load_3d(dst + s * kSlab + kBox, map, full + slot, s * 64, g, base + j1 * kBlk);
+            tc::tma_load_3d(dst + s * kSlab, map, bar, s * 64, g, base + j0 * kBlk);
+            tc::tma_load_3d(dst + s * kSlab + kBox, map, bar, s * 64, g, base + j1 * kBlk);
           }
         }
         __syncwarp();
       }
     }
-    if (lane == 0) {   // let the copies in flight land (bounded)
-      for (long x = f - 1; x >= 0 && x >= f - nslots; --x)
-        tc::mbar_wait(full + (x % nslots), (uint32_t)((x / nslots) & 1), err, keys ? kErrKFull : kErrVFull);
-      if (keys)
-        for (long x = k - 1; x >= 0 && x >= k - kItemSlots; --x)
-          tc::mbar_wait(q_full + (x % kItemSlots), (uint32_t)((x / kItemSlots) & 1), err, kErrQFull);
+    if (ok && keys) {
+      // steps F - 2 and F - 1 (F = this CTA's pairs) have no pair two ahead: their key
+      // arrivals carry no bytes, made once their phase is the current one
+      for (uint32_t ff = max(f, 2u); ff < f + 2 && ok; ++ff) {
+        ok = __all_sync(0xffffffffu, wait_slot(ff));
+        if (ok && lane == 0) tc::mbar_arrive(ready + (ff & 1));
+        __syncwarp();
+      }
     }
+    // No drain here: every copy lands on a barrier the MMA thread waits for (the queries and
+    // keys of every pair, the values of every step) before the CTA's final barrier.  (A wait
+    // on a step barrier from here could also see its phase bit already turned twice.)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    // The pairs of all items form one stream.  Once P^T of pair n is ready the thread issues
-    // the P.V of pair n, then the S of pair n + 2, while the softmax of pair n + 1 runs (S
-    // buffer n % 2 is free again once P^T of pair n is written).  The two products stay in
-    // blocks of their own: alternating MMAs of the K-major S with those of the MN-major V^T
-    // slowed both down.  An item without pairs takes a place in the stream too, so that its
-    // (empty) O is committed in order.
+    // Prologue: the S of pairs 0 and 1.  Step n: once its barrier is complete (keys of pair
+    // n + 2, values and P^T of pair n), the P.V of pair n, then the S of pair n + 2, one
+    // commit.  The two products stay in blocks of their own: alternating MMAs of the K-major
+    // S with those of the MN-major V^T slowed both down.
     if (tc::elect_one()) {
       const uint32_t idS = tc::idesc_bf16(128, kG, 0, 0);    // S^T = K Q^T: both K-major
       const uint32_t idPV = tc::idesc_bf16(128, kG, 1, 0);   // O^T = V^T P^T: V^T MN-major, P^T K-major
       const uint64_t dp0 = tc::sdesc(sP, 16, 1024);
-      // A stream entry: pair f (or an item without pairs) of the item with counter k (k's low
-      // bit picks its O buffer) in item slot qs.  Everything the issuing thread computes per
-      // entry is 32-bit adds, compares and bit operations: this one thread issues every MMA.
-      struct Entry { uint32_t f, k; int qs; bool first, last, pair; };
+      // A pair of the stream: its counter f, its item's counter k (the low bit picks the O
+      // buffer) and item slot.  Everything this thread computes per pair is 32-bit adds,
+      // compares and bit operations.
+      struct Pair { uint32_t f, k; int qs; bool first, last; };
       long it_c = next_item(blockIdx.x);
       uint32_t k_c = 0, f_c = 0, qph = 0;   // qph: the phase bit of item slot qs_c
       int qs_c = 0, p_c = 0, np_c = -1;
       bool ok = true;
-      auto next_entry = [&](Entry& e) -> bool {   // false: the walk is over (or a wait failed)
+      auto next_pair = [&](Pair& e) -> bool {   // false: the walk is over (or a wait failed)
         if (it_c >= total) return false;
         if (np_c < 0) {
           ok = tc::mbar_wait(q_full + qs_c, qph, err, kErrQFull);
           if (!ok) return false;
-          np_c = (sMeta[qs_c * kMetaInts + 32] + 1) >> 1;
+          np_c = max(1, (sMeta[qs_c * kMetaInts + 32] + 1) >> 1);
           p_c = 0;
         }
+        e.f = f_c++;
         e.k = k_c;
         e.qs = qs_c;
-        e.pair = np_c != 0;
-        e.f = f_c;
         e.first = p_c == 0;
         e.last = p_c == np_c - 1;
-        if (e.pair) {
-          ++f_c;
-          ++p_c;
-        }
-        if (!e.pair || p_c == np_c) {   // the item is done: move to the next
+        if (++p_c == np_c) {   // the item is done: move to the next
           it_c = next_item(it_c + stride);
           ++k_c;
           np_c = -1;
@@ -319,84 +326,54 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         return true;
       };
-      // S MMA number i of a pair (12 for d_k = 192): K step (i % 4) of slab (i / 4) into partial i % 4
-      auto s_mma = [&](const Entry& y, int i, uint64_t dk0, uint64_t dq0) {
-        const int sl = i >> 2, kk = i & 3;
-        tc::mma_ss(tmem + kColS + kSChains * kG * (uint32_t)(y.f & 1) + kG * kk,
-                   dk0 + (uint64_t)((sl * kSlab + kk * 32) / 16), dq0 + (uint64_t)((sl * kG * 128 + kk * 32) / 16), idS,
-                   sl != 0);
-      };
-      // the K slot of pair y (its S buffer is free: P^T of the pair two back is written,
-      // which the softmax warps do after reading that pair's S^T)
-      auto wait_s = [&](const Entry& y) -> bool {
-        return tc::mbar_wait(k_full + (y.f & 1), (y.f >> 1) & 1u, err, kErrKFull);
-      };
-      Entry q0{}, q1{};   // the stream entries whose S is issued and P.V not yet (two registers, no array)
-      int nq = 0;
-      // prologue: the S of the first two pairs
-      while (ok && nq < 2) {
-        Entry e;
-        if (!next_entry(e)) break;
-        if (e.pair) {
-          if (!(ok = wait_s(e))) break;
-          tc::tc_fence_after();
-          const uint64_t dk0 = tc::sdesc(sK + (e.f & 1) * SM::kKBytes, 16, 1024);
-          const uint64_t dq0 = tc::sdesc(sQ + e.qs * SM::kQBytes, 16, 1024);
-#pragma unroll 4
-          for (int i = 0; i < 4 * SM::kKS; ++i) s_mma(e, i, dk0, dq0);
-          tc::mma_commit(s_done + (e.f & 1));
+      // the S MMAs of pair y (K step kk of slab sl into partial kk)
+      auto issue_s = [&](const Pair& y) {
+        const uint64_t dk0 = tc::sdesc(sK + (y.f & 1) * SM::kKS * kSlab, 16, 1024);
+        const uint64_t dq0 = tc::sdesc(sQ + y.qs * SM::kQBytes, 16, 1024);
+        const uint32_t d_s = tmem + kColS + kSChains * kG * (y.f & 1);
+#pragma unroll 1
+        for (int sl = 0; sl < SM::kKS; ++sl) {
+          const uint64_t dk = dk0 + (uint64_t)(sl * kSlab / 16), dq = dq0 + (uint64_t)(sl * kG * 128 / 16);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc::mma_ss(d_s + kG * kk, dk + (uint64_t)(kk * 2), dq + (uint64_t)(kk * 2), idS, sl != 0);
         }
+      };
+      Pair q0{}, q1{};   // pairs whose S is issued and whose P.V is not (in registers, no array)
+      int nq = 0;
+      for (; nq < 2 && ok; ++nq) {
+        Pair e;
+        if (!next_pair(e)) break;
+        if (!(ok = tc::mbar_wait(pro_k + nq, 0u, err, kErrProK))) break;
+        tc::tc_fence_after();
+        issue_s(e);
+        tc::mma_commit(pro_done + nq);
         if (nq == 0) q0 = e;
         else q1 = e;
-        ++nq;
       }
       while (ok && nq > 0) {
-        const Entry x = q0;
-        Entry y;
-        const bool have_y = next_entry(y);
+        const Pair x = q0;
+        Pair y;
+        const bool have_y = next_pair(y);
         if (!ok) break;
-        const bool s_next = have_y && y.pair;
-        if (s_next && !(ok = wait_s(y))) break;
         const int ob = (int)(x.k & 1);
-        if (x.pair) {
-          const int vs = (int)(x.f & 1);
-          ok = (!x.first || tc::mbar_wait(o_empty + ob, ((x.k >> 1) & 1u) ^ 1u, err, kErrOEmpty)) &&
-               tc::mbar_wait(v_full + vs, (x.f >> 1) & 1u, err, kErrVFull) &&
-               tc::mbar_wait(p_full + vs, (x.f >> 1) & 1u, err, kErrPFull);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint64_t dv0 = tc::sdesc(sV + vs * SM::kVBytes, kSlab, 1024);
+        ok = (!x.first || tc::mbar_wait(o_empty + ob, ((x.k >> 1) & 1u) ^ 1u, err, kErrOEmpty)) &&
+             tc::mbar_wait(ready + (x.f & 1), (x.f >> 1) & 1u, err, kErrReady);
+        if (!ok) break;
+        tc::tc_fence_after();
+        {
+          const uint64_t dv0 = tc::sdesc(sV + (x.f & 1) * SM::kVBytes, kSlab, 1024);
           const uint64_t dp = dp0 + (uint64_t)((x.f & 1) * SM::kPBytes / 16);
           const uint32_t d_o = tmem + kColO + kOChains * kG * ob;
           const uint32_t accum = x.first ? 0u : 1u;
-          uint64_t dk0 = 0, dq0 = 0;
-          if (s_next) {
-            dk0 = tc::sdesc(sK + (y.f & 1) * SM::kKBytes, 16, 1024);
-            dq0 = tc::sdesc(sQ + y.qs * SM::kQBytes, 16, 1024);
-          }
 #pragma unroll
           for (int ks = 0; ks < 2 * kBlk / 16; ++ks)   // 16-key step ks into partial ks
             tc::mma_ss(d_o + kG * ks, dv0 + (uint64_t)(ks * 16 * 128 / 16),
                        dp + (uint64_t)(((ks >> 2) * (kG * 128) + (ks & 3) * 32) / 16), idPV, accum);
-          tc::mma_commit(pv_done + vs);
-          if (x.last) tc::mma_commit(o_full + ob);
-          if (s_next) {
-#pragma unroll 4
-            for (int i = 0; i < 4 * SM::kKS; ++i) s_mma(y, i, dk0, dq0);
-            tc::mma_commit(s_done + (y.f & 1));
-          }
-        } else {   // an item without pairs: its empty O, in order
-          if (!(ok = tc::mbar_wait(o_empty + ob, ((x.k >> 1) & 1u) ^ 1u, err, kErrOEmpty))) break;
-          if (s_next) {
-            tc::tc_fence_after();
-            const uint64_t dk0 = tc::sdesc(sK + (y.f & 1) * SM::kKBytes, 16, 1024);
-            const uint64_t dq0 = tc::sdesc(sQ + y.qs * SM::kQBytes, 16, 1024);
-#pragma unroll 4
-            for (int i = 0; i < 4 * SM::kKS; ++i) s_mma(y, i, dk0, dq0);
-            tc::mma_commit(s_done + (y.f & 1));
-          }
-          tc::mma_commit(o_full + ob);
         }
+        if (have_y) issue_s(y);
+        tc::mma_commit(done + (x.f & 1));
+        if (x.last) tc::mma_commit(o_full + ob);
         q0 = q1;
         if (have_y) q1 = y;
         else --nq;
@@ -424,7 +401,7 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       if (!ok) break;
       const int* meta = sMeta + qs * kMetaInts;
       const int nblk = meta[32];
-      const int npairs = (nblk + 1) / 2;
+      const int npairs = max(1, (nblk + 1) / 2);
       float m[kHH], lp[kHH];                           // reference (log2 units) and partial row sums
 #pragma unroll
       for (int h = 0; h < kHH; ++h) {
@@ -433,8 +410,10 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
       }
       for (int p = 0; p < npairs; ++p, ++f) {
         const int sb = (int)(f & 1);
-        ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_done + (f % kKSlots), (uint32_t)((f / kKSlots) & 1),
-                                                         err, kErrSFull));
+        // S^T of pair f is ready and P^T buffer f % 2 free: the prologue (pairs 0, 1) or step f - 2
+        ok = __all_sync(0xffffffffu, ok && (f < 2 ? tc::mbar_wait(pro_done + f, 0u, err, kErrSDone)
+                                                  : tc::mbar_wait(done + (f & 1), (uint32_t)(((f >> 1) & 1) ^ 1),
+                                                                  err, kErrSDone)));
         float x[kHH], y[kHH];
 #pragma unroll
         for (int h = 0; h < kHH; ++h) x[h] = 0.f;
@@ -489,11 +468,6 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
           lp[h + 1] += p1;
           pk[h / 2] = pack_bf16(p0, p1);
         }
-        // P^T goes to buffer f % 2 once the P.V of the pair two back has read it
-        if (f >= 2)
-          ok = __all_sync(0xffffffffu, tc::mbar_wait(pv_done + (f & 1), (uint32_t)(((f >> 1) & 1) ^ 1), err,
-                                                     kErrPEmpty));
-        if (!ok) continue;
         uint8_t* const pc = pcol + (f & 1) * SM::kPBytes;
 #pragma unroll
         for (int h = 0; h < kHH; ++h)
@@ -501,7 +475,7 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
               (uint16_t)(pk[h / 2] >> (16 * (h & 1)));
         tc::fence_async_smem();
         __syncwarp();
-        if (lane == 0) tc::mbar_arrive(p_full + (f & 1));
+        if (lane == 0) tc::mbar_arrive(ready + (f & 1));
       }
       if (!ok) continue;   // the next item's vote ends the walk
       // the item's row sums of this quadrant: reduce the 8 partial sums over the warp's 32

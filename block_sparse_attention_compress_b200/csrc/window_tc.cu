@@ -12,9 +12,10 @@
 // buffer, K slices into a 3-slot ring, V tiles double buffered; the rings run across items),
 // a single-thread MMA issuer that puts S(n+1) ahead of the P.V of tile n and accumulates
 // alternate items into two O buffers in TMEM (so an item's tiles overlap the previous
-// item's epilogue),
-// and 8 softmax warps: warp w and warp w+4 share TMEM lanes 32(w%4).. (the same rows)
-// and take the tile's key columns [0, 64) and [64, 128).
+// item's epilogue), 8 softmax warps: warp w and warp w+4 share TMEM lanes 32(w%4).. (the
+// same rows) and take the tile's key columns [0, 64) and [64, 128); and 4 epilogue warps
+// (one per TMEM lane quadrant) that write an item's rows while the softmax warps run the
+// next item's tiles.
 //
 // Softmax in one pass: a row's reference m moves only when a score exceeds it by more
 // than 2^8 (so p <= 2^8).  The two threads of a row agree on it through one barrier of
@@ -30,8 +31,8 @@ namespace nsa {
 
 namespace {
 constexpr int kSoftWarps = 8;
-constexpr int kTmaWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9, kEpiWarp0 = 10;   // epilogue: warps 10-13
+constexpr int kThreads = 448;
 constexpr int kTok = 8;
 constexpr int kRowsM = 128;
 constexpr int kBlk = 128;                         // keys per tile
@@ -42,7 +43,7 @@ constexpr uint32_t kColS = 0, kColO = 256;        // S buffer b at 128b; O buffe
 constexpr float kSlack = 8.f;
 
 enum Err { kErrQ = 41, kErrKFull, kErrKEmpty, kErrVFull, kErrVEmpty, kErrSFull, kErrSEmpty, kErrPFull, kErrPEmpty,
-           kErrOFull, kErrOEmpty, kErrQEmpty };
+           kErrOFull, kErrOEmpty, kErrQEmpty, kErrLFull, kErrLEmpty };
 
 template <int DK, int DV>
 struct Smem {
@@ -52,9 +53,9 @@ struct Smem {
   static constexpr uint32_t kV = kK + kKSlots * kSlice;                     // 2 tiles x kVSlices slices
   static constexpr uint32_t kP = kV + 2 * kVSlices * kSlice;                // P: [2 key halves][128 rows][128 B]
   static constexpr uint32_t kPair = kP + 2 * kSlice;                        // [2][128] fp32 + [2][128] flags
-  static constexpr uint32_t kGate = kPair + 2 * kRowsM * 4 + 2 * kRowsM * 4;
-  static constexpr uint32_t kBar = kGate + 2 * kRowsM * 4;                  // gates: [item parity][128]
-  static constexpr int kNumBars = 1 + 2 * kKSlots + 2 * 2 + 2 * 2 + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kL = kPair + 2 * kRowsM * 4 + 2 * kRowsM * 4;   // row sums: [item parity][128]
+  static constexpr uint32_t kBar = kL + 2 * kRowsM * 4;
+  static constexpr int kNumBars = 1 + 2 * kKSlots + 2 * 2 + 2 * 2 + 2 + 2 + 2 + 1 + 2 + 2;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;
@@ -79,7 +80,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint8_t* sP = smem + SM::kP;
   float* sPairMax = reinterpret_cast<float*>(smem + SM::kPair);            // [half][row]
   int* sPairFlag = reinterpret_cast<int*>(sPairMax + 2 * kRowsM);           // [half][row]
-  float* sGate = reinterpret_cast<float*>(smem + SM::kGate);                // [item parity][row]
+  float* sL = reinterpret_cast<float*>(smem + SM::kL);                      // [item parity][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SM::kBar);
   uint64_t* bar_q = bars;
   uint64_t* k_full = bars + 1;
@@ -91,8 +92,10 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   uint64_t* p_full = s_empty + 2;
   uint64_t* p_empty = p_full + 1;
   uint64_t* o_full = p_empty + 1;    // [2] an item's O (buffer k & 1) is complete
-  uint64_t* o_empty = o_full + 2;    // [2] the softmax warps have read it
+  uint64_t* o_empty = o_full + 2;    // [2] the epilogue warps have read it
   uint64_t* q_empty = o_empty + 2;   // the S MMAs of an item have read its Q
+  uint64_t* l_full = q_empty + 1;    // [2] an item's row sums are in sL
+  uint64_t* l_empty = l_full + 2;    // [2] the epilogue warps have read them
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + SM::kTmemSlot);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -133,7 +136,9 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       tc::mbar_init(s_full + i, 1);
       tc::mbar_init(s_empty + i, kSoftWarps);
       tc::mbar_init(o_full + i, 1);
-      tc::mbar_init(o_empty + i, kSoftWarps);
+      tc::mbar_init(o_empty + i, 4);
+      tc::mbar_init(l_full + i, 4);   // the four warps of the first key half
+      tc::mbar_init(l_empty + i, 4);
     }
     tc::mbar_init(p_full, kSoftWarps);
     tc::mbar_init(p_empty, 1);
@@ -256,8 +261,8 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (ok) tc::mma_commit(o_full + ob);
       }
     }
-  } else {
-    // ------------------------------------------------------------ softmax / epilogue
+  } else if (warp < kSoftWarps) {
+    // ------------------------------------------------------------ softmax
     const int gr = warp >> 2, q4 = warp & 3;       // key half, TMEM lane quadrant
     const int r = 32 * q4 + lane;                  // this thread's row: token r / 16, head r % 16
     const int pbar = 1 + q4;                       // barrier of the warp pair sharing these rows
@@ -271,43 +276,37 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const int my_t = x.t0 + r / 16;
       const bool row_ok = my_t < x.len;
       const int my_lo = max(0, my_t - window + 1), my_hi = row_ok ? my_t : -1;   // keys [my_lo, my_hi]
-      const size_t grow = ((size_t)x.base + min(my_t, x.len - 1)) * Hq + x.g * 16 + (r % 16);
-      float* gate = sGate + ob * kRowsM;
-      if (gr == 0) gate[r] = row_ok ? __bfloat162float(gates[grow * 3 + 2]) : 0.f;
-      // the epilogue reads this thread's half of the accumulator row (256 B): start it now
-      if (row_ok) {
-        prefetch_l2(acc + grow * DV + (DV / 2) * gr);
-        prefetch_l2(acc + grow * DV + (DV / 2) * gr + 32);
-      }
       float m = -INFINITY, l = 0.f;
       for (int n = 0; n < x.ntiles; ++n, ++use, ++pc) {
         const int sb = use & 1;
         ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_full + sb, (use >> 1) & 1, err, kErrSFull));
+        const uint32_t s_addr = lane_addr + kColS + 128 * sb + 64 * gr;
+        const int i0 = x.kv_lo + n * kBlk + 64 * gr;     // first key of this thread's half
+        const bool full = i0 >= my_lo && i0 + 63 <= my_hi;
+        // the masked raw scores (the scale, positive, is applied to the maximum and inside the
+        // exponent's FMA: rounding x * scale is monotone, so the maxima agree)
         float v[64];
+        float lmax = -INFINITY;
         if (ok) {
           tc::tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tc::tmem_ld16(lane_addr + kColS + 128 * sb + 64 * gr + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
+          for (int c = 0; c < 4; ++c) tc::tmem_ld16(s_addr + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
           tc::tmem_wait_ld();
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(s_empty + sb);
+          if (!full) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = (i0 + j >= my_lo && i0 + j <= my_hi) ? v[j] : -INFINITY;
+          }
+          float cmx[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(fmaxf(v[c], v[c + 8]), fmaxf(v[c + 16], v[c + 24]));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
+          lmax = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
+                       fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7]))) * scale_log2;
         }
-        const int i0 = x.kv_lo + n * kBlk + 64 * gr;     // first key of this thread's half
-        // masked raw scores: the scale (positive) is applied to the maximum and inside the
-        // exponent's FMA (rounding x * scale is monotone, so the maxima agree)
-        if (!(i0 >= my_lo && i0 + 63 <= my_hi)) {
-#pragma unroll
-          for (int j = 0; j < 64; ++j) v[j] = (i0 + j >= my_lo && i0 + j <= my_hi) ? v[j] : -INFINITY;
-        }
-        float cmx[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(fmaxf(v[c], v[c + 8]), fmaxf(v[c + 16], v[c + 24]));
-#pragma unroll
-        for (int c = 0; c < 8; ++c) cmx[c] = fmaxf(cmx[c], fmaxf(fmaxf(v[c + 32], v[c + 40]), fmaxf(v[c + 48], v[c + 56])));
-        const float lmax = fmaxf(fmaxf(fmaxf(cmx[0], cmx[1]), fmaxf(cmx[2], cmx[3])),
-                                 fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7]))) * scale_log2;
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0 && ok) tc::mbar_arrive(s_empty + sb);
         // the two threads of a row agree on its reference; a failed wait also takes the
         // exchange, so that both warps of the pair leave together
         if (tc::vote_any(pbar, 64, !ok || lmax > m + kSlack)) {
@@ -367,42 +366,83 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(p_full);
       }
-      // epilogue: the row sum over both halves, then out = bf16(acc + g_win * O / l)
+      // the row sum over both halves, for the epilogue warps
       sPairMax[gr * kRowsM + r] = l;
       sPairFlag[gr * kRowsM + r] = ok;
       tc::named_sync(pbar, 64);
       const bool pair_ok = sPairFlag[r] && sPairFlag[kRowsM + r];
       const float L = sPairMax[r] + sPairMax[kRowsM + r];
-      // all eight warps: the gates are written, and both halves of every row have read the
-      // exchange before the next item's first tile reuses it
+      // all eight warps: both halves of every row have read the exchange before the next
+      // item's first tile reuses it
       ok = tc::vote_all(5, 256, ok && pair_ok);
       if (!ok) break;
-      // the accumulator half-row, loaded before waiting for the last P.V
-      const float* arow = acc + grow * DV + (DV / 2) * gr;
+      if (gr == 0) {
+        ok = __all_sync(0xffffffffu, tc::mbar_wait(l_empty + ob, ((k >> 1) & 1) ^ 1, err, kErrLEmpty));
+        sL[ob * kRowsM + r] = L;
+        __threadfence_block();
+        __syncwarp();
+        if (lane == 0 && ok) tc::mbar_arrive(l_full + ob);
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------ epilogue: out = bf16(acc + g_win * O / l)
+    const int q4 = warp & 3;
+    const int r = 32 * q4 + lane;                  // this thread's row: token r / 16, head r % 16
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * q4) << 16);
+    bool ok = true;
+    int k = 0;
+    for (int it = next_item(blockIdx.x); it < n_items && ok; it = next_item(it + gridDim.x), ++k) {
+      const Item x = item_of(it);
+      const int ob = k & 1;
+      const uint32_t o_col = kColO + 128 * ob;
+      const int my_t = x.t0 + r / 16;
+      const bool row_ok = my_t < x.len;
+      const size_t grow = ((size_t)x.base + min(my_t, x.len - 1)) * Hq + x.g * 16 + (r % 16);
+      const float gw = row_ok ? __bfloat162float(gates[grow * 3 + 2]) : 0.f;
+      const float* arow = acc + grow * DV;
+      __nv_bfloat16* orow = out + grow * DV;
+      // the accumulator row: its first half loaded (and the second asked of L2) while the
+      // softmax warps still run the item's tiles
       float4 a4[DV / 2 / 4];
 #pragma unroll
       for (int i = 0; i < DV / 2 / 4; ++i)
         a4[i] = row_ok ? *reinterpret_cast<const float4*>(arow + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      if (row_ok) {
+        prefetch_l2(arow + DV / 2);
+        prefetch_l2(arow + DV / 2 + 32);
+      }
+      ok = __all_sync(0xffffffffu, tc::mbar_wait(l_full + ob, (k >> 1) & 1, err, kErrLFull));
+      if (!ok) break;
+      const float L = sL[ob * kRowsM + r];
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(l_empty + ob);
+      const float scl = L > 0.f ? gw / L : 0.f;
       ok = __all_sync(0xffffffffu, tc::mbar_wait(o_full + ob, (k >> 1) & 1, err, kErrOFull));
       if (!ok) break;
       tc::tc_fence_after();
-      const float scl = L > 0.f ? gate[r] / L : 0.f;
-      __nv_bfloat16* orow = out + grow * DV + (DV / 2) * gr;
 #pragma unroll
-      for (int q = 0; q < DV / 2 / 16; ++q) {
-        float o[16];
-        tc::tmem_ld16(lane_addr + o_col + (DV / 2) * gr + 16 * q, o);
-        tc::tmem_wait_ld();
-        if (row_ok) {
-          uint32_t w[8];
+      for (int half = 0; half < 2; ++half) {
+        if (half == 1) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            const float4 av = a4[(16 * q + i) / 4];
-            w[i / 2] = pack_bf16(av.x + scl * o[i], av.y + scl * o[i + 1]);
-            w[i / 2 + 1] = pack_bf16(av.z + scl * o[i + 2], av.w + scl * o[i + 3]);
+          for (int i = 0; i < DV / 2 / 4; ++i)
+            a4[i] = row_ok ? *reinterpret_cast<const float4*>(arow + DV / 2 + 4 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < DV / 2 / 16; ++q) {
+          float o[16];
+          tc::tmem_ld16(lane_addr + o_col + (DV / 2) * half + 16 * q, o);
+          tc::tmem_wait_ld();
+          if (row_ok) {
+            uint32_t w[8];
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              const float4 av = a4[(16 * q + i) / 4];
+              w[i / 2] = pack_bf16(av.x + scl * o[i], av.y + scl * o[i + 1]);
+              w[i / 2 + 1] = pack_bf16(av.z + scl * o[i + 2], av.w + scl * o[i + 3]);
+            }
+            *reinterpret_cast<uint4*>(orow + (DV / 2) * half + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(orow + (DV / 2) * half + 16 * q + 8) = make_uint4(w[4], w[5], w[6], w[7]);
           }
-          *reinterpret_cast<uint4*>(orow + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
-          *reinterpret_cast<uint4*>(orow + 16 * q + 8) = make_uint4(w[4], w[5], w[6], w[7]);
         }
       }
       tc::tc_fence_before();   // this thread's reads of O buffer ob are done

@@ -18,7 +18,8 @@ NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUD
 NSA_MODE_NSA, NSA_MODE_MOBA, NSA_MODE_DSA = 0, 1, 2
 NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
-EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_forward", "nsa_forward_varlen",
+EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_compress_mlp",
+            "nsa_compress_append_mlp", "nsa_forward", "nsa_forward_varlen",
             "nsa_dsa_forward", "nsa_backward", "nsa_decode",
             "nsa_forward_noalloc", "nsa_device_status", "nsa_device_status_noalloc", "nsa_selftest_wait_timeout",
             "nsa_status_string")
@@ -71,6 +72,10 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_compress.restype = ctypes.c_int
     lib.nsa_compress_append.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp, i32, vp]
     lib.nsa_compress_append.restype = ctypes.c_int
+    lib.nsa_compress_mlp.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, vp]
+    lib.nsa_compress_mlp.restype = ctypes.c_int
+    lib.nsa_compress_append_mlp.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, i32, vp]
+    lib.nsa_compress_append_mlp.restype = ctypes.c_int
     lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
     lib.nsa_backward.restype = ctypes.c_int
     lib.nsa_backward.argtypes = [vp, vp, vp, vp, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, vp]
@@ -158,6 +163,24 @@ def nsa_compress_append(x_cache, w, seqlens, out_cache, l: int = 32, s: int = 16
     st = load_library().nsa_compress_append(_ptr(x_cache), _ptr(w), _ptr(seqlens), B, Lmax, H, d, w.shape[1], l, s,
                                             _ptr(out_cache), out_cache.shape[1], _stream(stream, x_cache))
     return _check(st, "nsa_compress_append") if check else st
+
+
+def nsa_compress_mlp(x, w1, b1, w2, hidden, out, l: int = 32, s: int = 16, stream=None, check: bool = True) -> int:
+    """phi as the two-layer MLP over [B, T, H, d]; hidden and out [B, N_c, H, d] (see include/nsa.h)."""
+    B, T, H, d = x.shape
+    st = load_library().nsa_compress_mlp(_ptr(x), _ptr(w1), _ptr(b1), _ptr(w2), B, T, H, d, l, s, _ptr(hidden),
+                                         _ptr(out), _stream(stream, x))
+    return _check(st, "nsa_compress_mlp") if check else st
+
+
+def nsa_compress_append_mlp(x_cache, w1, b1, w2, seqlens, hidden, out_cache, l: int = 32, s: int = 16, stream=None,
+                            check: bool = True) -> int:
+    """nsa_compress_append with phi as the two-layer MLP; hidden is scratch [B, H, d] (see include/nsa.h)."""
+    B, Lmax, H, d = x_cache.shape
+    st = load_library().nsa_compress_append_mlp(_ptr(x_cache), _ptr(w1), _ptr(b1), _ptr(w2), _ptr(seqlens), B, Lmax,
+                                                H, d, l, s, _ptr(hidden), _ptr(out_cache), out_cache.shape[1],
+                                                _stream(stream, x_cache))
+    return _check(st, "nsa_compress_append_mlp") if check else st
 
 
 def nsa_forward(q, k, v, gates, cfg: NsaConfig, out, stream=None, check: bool = True) -> int:

@@ -12,7 +12,10 @@
 // its CTA, so every block equals bitwise the one the full compression computes.
 // MLP mode (phi as a two-layer MLP): the first layer is this GEMM with the epilogue
 // GELU(acc + bias) (MLP1), stored in bf16; the second layer is this GEMM again over the hidden
-// rows with a "block" of one row (l = s = 1).
+// rows with a "block" of one row (l = s = 1).  Appending with the MLP: the first layer writes
+// each due sequence's hidden row to a small buffer [B, H, d] (HID_OUT), and the second layer
+// reads that row as a one-token block (HID_IN) and writes the cache row of the window; both
+// follow the same per-row arithmetic as the full compression.
 // Variable-length batch (cu != nullptr): sequence b's tokens are rows cu[b] .. cu[b+1] of x
 // and its n_cmp(cu[b+1] - cu[b]) blocks go to out[b, 0 .. ); its rows from there up to nc are
 // zeroed, so that a reader of whole 128-row tiles (masked past the sequence) only ever
@@ -29,7 +32,7 @@ constexpr int kBM = 64, kBN = 64, kBK = 64, kThreads = 128;
 // loads' latency; more for the append launch, whose few CTAs each run one long k chain.
 __device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
 
-template <int D, int DOUT, int STAGES, bool APPEND, bool MLP1 = false>
+template <int D, int DOUT, int STAGES, bool APPEND, bool MLP1 = false, bool HID_OUT = false, bool HID_IN = false>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
                 int l, int s, int nc, __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ seqlens,
@@ -43,7 +46,8 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   const int i0 = blockIdx.x * kBM, n0 = blockIdx.y * kBN;
   constexpr bool app = APPEND;
   const int bh = blockIdx.z, b = app ? 0 : bh / H, h = app ? bh : bh % H;
-  const int nk = l * D / kBK;
+  static_assert(APPEND || (!HID_OUT && !HID_IN), "the hidden row buffer is an append-mode layout");
+  const int nk = (HID_IN ? 1 : l) * D / kBK;
   // full mode: the first token row of sequence b and its number of blocks
   int base = 0, nc_b = nc;
   if constexpr (!APPEND) {
@@ -70,6 +74,7 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
   auto row_seq = [&](int row) { return app ? i0 + row : b; };
   auto row_win = [&](int row) { return app ? sWin[row] : (i0 + row < nc_b ? i0 + row : -1); };
   auto src_row = [&](int row, int i, int r) -> size_t {   // token row of x
+    if constexpr (HID_IN) return (size_t)row_seq(row);   // the hidden row [B, H, d] of the sequence
     return app ? (size_t)row_seq(row) * T + (size_t)s * i + r : (size_t)base + (size_t)s * i + r;
   };
 
@@ -142,7 +147,7 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
       }
       continue;
     }
-    __nv_bfloat16* dst = out + (((size_t)row_seq(row) * nc + i) * H + h) * DOUT + n0;
+    __nv_bfloat16* dst = out + (((size_t)row_seq(row) * (HID_OUT ? 1 : nc) + (HID_OUT ? 0 : i)) * H + h) * DOUT + n0;
 #pragma unroll
     for (int j = 0; j < kBN / 8; ++j) {
       float v0 = acc[j][2 * half], v1 = acc[j][2 * half + 1];
@@ -186,6 +191,34 @@ cudaError_t launch_append(const void* x, const void* w, const int32_t* seqlens, 
   return cudaGetLastError();
 }
 template <int D>
+cudaError_t launch_append_mlp(const void* x, const void* w1, const void* b1, const void* w2, const int32_t* seqlens,
+                              int B, int Lmax, int H, int l, int s, int ncmax, void* hidden, void* out,
+                              cudaStream_t st) {
+  constexpr int kStages = 8;
+  auto k1 = compress_kernel<D, D, kStages, true, true, true, false>;
+  auto k2 = compress_kernel<D, D, kStages, true, false, false, true>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  dim3 grid((B + kBM - 1) / kBM, D / kBN, H);
+  k1<<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
+                                                   static_cast<const __nv_bfloat16*>(w1), Lmax, H, l, s, ncmax,
+                                                   static_cast<__nv_bfloat16*>(hidden), seqlens, B, nullptr,
+                                                   static_cast<const __nv_bfloat16*>(b1));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k2<<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(hidden),
+                                                   static_cast<const __nv_bfloat16*>(w2), Lmax, H, l, s, ncmax,
+                                                   static_cast<__nv_bfloat16*>(out), seqlens, B, nullptr, nullptr);
+  return cudaGetLastError();
+}
+
+template <int D>
 cudaError_t launch_mlp(const void* x, const void* w1, const void* b1, const void* w2, int B, int T, int H, int l,
                        int s, int nc, void* hidden, void* out, cudaStream_t st, const int32_t* cu) {
   dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
@@ -221,6 +254,18 @@ cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* 
     case 64: return launch_append<64>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
     case 128: return launch_append<128>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
     case 192: return launch_append<192>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_compress_append_mlp(const void* x, const void* w1, const void* b1, const void* w2,
+                                       const int32_t* seqlens, int B, int Lmax, int H, int d, int l, int s,
+                                       int ncmax, void* hidden, void* out, cudaStream_t st) {
+  if (B == 0 || H == 0 || ncmax == 0) return cudaSuccess;
+  switch (d) {
+    case 64: return launch_append_mlp<64>(x, w1, b1, w2, seqlens, B, Lmax, H, l, s, ncmax, hidden, out, st);
+    case 128: return launch_append_mlp<128>(x, w1, b1, w2, seqlens, B, Lmax, H, l, s, ncmax, hidden, out, st);
+    case 192: return launch_append_mlp<192>(x, w1, b1, w2, seqlens, B, Lmax, H, l, s, ncmax, hidden, out, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -22,6 +22,10 @@ cudaError_t launch_compress_mlp(const void* x, const void* w1, const void* b1, c
 // to Lmax) completes window i = (L - l)/s < ncmax, out[b, i, h, :] for every head.
 cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,
                                    int d, int l, int s, int ncmax, void* out, cudaStream_t st);
+// The same with phi as the two-layer MLP; hidden is scratch bf16 [B, H, d] for the due rows.
+cudaError_t launch_compress_append_mlp(const void* x, const void* w1, const void* b1, const void* w2,
+                                       const int32_t* seqlens, int B, int Lmax, int H, int d, int l, int s,
+                                       int ncmax, void* hidden, void* out, cudaStream_t st);
 
 struct FwdArgs {
   const void* q;      // [B, T, Hq, dk] bf16

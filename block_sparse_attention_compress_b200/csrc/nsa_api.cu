@@ -276,6 +276,31 @@ nsa_status nsa_compress_append(const void* x_cache, const void* w, const int32_t
                                                static_cast<cudaStream_t>(stream)));
 }
 
+nsa_status nsa_compress_mlp(const void* x, const void* w1, const void* b1, const void* w2, int32_t B, int32_t T,
+                            int32_t H, int32_t d, int32_t l, int32_t s, void* hidden, void* out, void* stream) {
+  if (!x || !w1 || !b1 || !w2 || !hidden || !out || B < 1 || T < 1 || H < 1 || d < 1 || l < 1 || s < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w1) || !aligned16(b1) || !aligned16(w2) || !aligned16(hidden) || !aligned16(out))
+    return NSA_ERR_INVALID_ARG;
+  if (l != 32 || s != 16 || (d != 64 && d != 128 && d != 192)) return NSA_ERR_UNSUPPORTED;
+  return from_cuda(nsa::launch_compress_mlp(x, w1, b1, w2, B, T, H, d, l, s, hidden, out,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+nsa_status nsa_compress_append_mlp(const void* x_cache, const void* w1, const void* b1, const void* w2,
+                                   const int32_t* seqlens, int32_t B, int32_t Lmax, int32_t H, int32_t d, int32_t l,
+                                   int32_t s, void* hidden, void* out_cache, int32_t ncmax, void* stream) {
+  if (!x_cache || !w1 || !b1 || !w2 || !seqlens || !hidden || !out_cache || B < 1 || Lmax < 1 || H < 1 || d < 1 ||
+      l < 1 || s < 1 || ncmax < 1)
+    return NSA_ERR_INVALID_ARG;
+  if (!aligned16(x_cache) || !aligned16(w1) || !aligned16(b1) || !aligned16(w2) || !aligned16(hidden) ||
+      !aligned16(out_cache) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return NSA_ERR_INVALID_ARG;
+  if (l != 32 || s != 16 || (d != 64 && d != 128 && d != 192)) return NSA_ERR_UNSUPPORTED;
+  return from_cuda(nsa::launch_compress_append_mlp(x_cache, w1, b1, w2, seqlens, B, Lmax, H, d, l, s, ncmax, hidden,
+                                                   out_cache, static_cast<cudaStream_t>(stream)));
+}
+
 nsa_status nsa_forward(const void* q, const void* k, const void* v, const void* gates, const nsa_config* cfg,
                        void* out, void* stream) {
   nsa_status st = check_cfg(cfg);

@@ -115,9 +115,10 @@ typedef enum {
  *                 w_cmp_k is then the first layer [l*d_k, d_k], b_cmp_k its bias bf16 [d_k],
  *                 w_cmp_k2 the second layer bf16 [d_k, d_k] (values: d_v).  An intra-block
  *                 position embedding pe [l, d] added to every block before the first layer is
- *                 exactly the bias b = vec(pe) @ w_cmp_k.  Only nsa_forward and
- *                 nsa_forward_varlen take phi_mlp = 1 (nsa_compress, nsa_compress_append and
- *                 nsa_decode work on the linear phi or on caches the caller compressed).
+ *                 exactly the bias b = vec(pe) @ w_cmp_k.  nsa_forward and
+ *                 nsa_forward_varlen take phi_mlp = 1; nsa_compress_mlp and
+ *                 nsa_compress_append_mlp compute the same map for a decode cache, which
+ *                 nsa_decode reads like any other compressed cache.
  *   w_cmp_k2, w_cmp_v2, b_cmp_k, b_cmp_v   (NSA, phi_mlp = 1) as above, 16-byte aligned.
  */
 typedef struct {
@@ -160,6 +161,25 @@ NSA_API size_t nsa_workspace_size(const nsa_config* cfg, int decode_batch);
  */
 NSA_API nsa_status nsa_compress(const void* x, const void* w, int32_t B, int32_t T, int32_t H, int32_t d,
                         int32_t d_out, int32_t l, int32_t s, void* out, void* stream);
+
+/*
+ * nsa_compress_mlp -- phi as a two-layer MLP of hidden width d ([BLOG] "Deepseek 的论文核心点":
+ * the blocks are compressed with an MLP; the form is the one nsa_forward takes with
+ * phi_mlp = 1).
+ *   x       bf16 [B, T, H, d]       keys or values
+ *   w1      bf16 [l*d, d]           first layer;  b1 bf16 [d] its bias
+ *   w2      bf16 [d, d]             second layer
+ *   hidden  bf16 [B, N_c, H, d]     caller-owned scratch, overwritten
+ *   out     bf16 [B, N_c, H, d]     row i = bf16(bf16(GELU(vec(x[s*i : s*i+l]) @ w1 + b1)) @ w2),
+ *                                   GELU(x) = x (1 + erf(x / sqrt 2)) / 2, each product
+ *                                   accumulated in fp32; equal bitwise to the compressed keys
+ *                                   (values) nsa_forward writes to kc_out (vc_out).
+ * All pointers 16-byte aligned device memory.  Implemented: d in {64,128,192},
+ * (l, s) = (32, 16).  Status codes as for nsa_compress.
+ */
+NSA_API nsa_status nsa_compress_mlp(const void* x, const void* w1, const void* b1, const void* w2, int32_t B,
+                                    int32_t T, int32_t H, int32_t d, int32_t l, int32_t s, void* hidden, void* out,
+                                    void* stream);
 
 /*
  * nsa_forward -- prefill forward.
@@ -296,6 +316,21 @@ NSA_API nsa_status nsa_decode(const void* q, const void* k_cache, const void* v_
 NSA_API nsa_status nsa_compress_append(const void* x_cache, const void* w, const int32_t* seqlens, int32_t B,
                                        int32_t Lmax, int32_t H, int32_t d, int32_t d_out, int32_t l, int32_t s,
                                        void* out_cache, int32_t ncmax, void* stream);
+
+/*
+ * nsa_compress_append_mlp -- nsa_compress_append with phi as the two-layer MLP of
+ * nsa_compress_mlp (same w1, b1, w2), so that a cache compressed by nsa_forward with
+ * phi_mlp = 1 stays current while decoding.
+ *   hidden   bf16 [B, H, d]   caller-owned scratch, overwritten for the sequences at a
+ *                             block boundary
+ * Writes out_cache[b, i, h, :] for the same (b, i) as nsa_compress_append, each bitwise
+ * equal to row i of nsa_compress_mlp over the whole cache; no other row of out_cache.
+ * Status codes as for nsa_compress_mlp (seqlens must be 4-byte aligned).
+ */
+NSA_API nsa_status nsa_compress_append_mlp(const void* x_cache, const void* w1, const void* b1, const void* w2,
+                                           const int32_t* seqlens, int32_t B, int32_t Lmax, int32_t H, int32_t d,
+                                           int32_t l, int32_t s, void* hidden, void* out_cache, int32_t ncmax,
+                                           void* stream);
 
 /*
  * nsa_forward_noalloc -- nsa_forward for callers that cannot allocate device memory.

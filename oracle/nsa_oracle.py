@@ -328,7 +328,8 @@ def nsa_forward(q, k, v, gates, w_k, w_v, *, cmp_block=32, cmp_stride=16,
 
 def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, gates, *,
                cmp_block=32, cmp_stride=16, sel_block=64, top_k=16, window=512,
-               force_first=True, force_local=True, scale=None, batch=None, score_map="touch"):
+               force_first=True, force_local=True, scale=None, batch=None, score_map="touch",
+               forced_idx=None):
     """One decode step.  [NOTES] §13: decoding reads the KV cache once per
     step; R11: sequence b's cache holds seqlens[b] tokens including the new
     one, whose position is t = seqlens[b] - 1.  The compressed caches are
@@ -336,7 +337,8 @@ def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, gates, *,
     length-seqlens[b] sequence).
 
     q [B,H_q,d_k], caches [B,L,H_kv,d], kc/vc [B,N_c,H_kv,d], gates [B,H_q,3].
-    ``batch`` restricts the work to some sequences.
+    ``batch`` restricts the work to some sequences.  ``forced_idx`` [nb, H_kv, top_k] (one
+    row per sequence worked on) imposes the chosen blocks (forced-index mode).
     Returns dict(out [nb, H_q, d_v], idx [nb, H_kv, top_k], score)."""
     q, gates = _f64(q), _f64(gates)
     B, Hq, dk = q.shape
@@ -359,7 +361,8 @@ def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, gates, *,
             r = nsa_token(q[bi, hs], _f64(k_cache[bi, :L, g]), _f64(v_cache[bi, :L, g]),
                           _f64(kc_cache[bi, :nc, g]), _f64(vc_cache[bi, :nc, g]),
                           gates[bi, hs], t, l=l, s=s, b=b, k=top_k, w=window, scale=scale,
-                          force_first=force_first, force_local=force_local, score_map=score_map)
+                          force_first=force_first, force_local=force_local, score_map=score_map,
+                          idx=None if forced_idx is None else [int(j) for j in forced_idx[n_i, g]])
             out[n_i, hs] = r["out"]
             idx[n_i, g] = torch.tensor(r["idx"])
             row.append(r["score"])

@@ -135,6 +135,24 @@ def test_compress_rejects_bad_arguments(lib):
     assert L.nsa_compress(0x1000, 0x2000, 0, 64, 1, 64, 64, 32, 16, 0x3000, None) == nsa.NSA_ERR_INVALID_ARG
 
 
+def test_compress_mlp_rejects_bad_arguments(lib):
+    """Argument checks of the MLP phi entry points, all before any CUDA call."""
+    L = lib
+    a, b, c, d, h, o = 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000
+    assert L.nsa_compress_mlp(a, b, 0, d, 1, 64, 1, 64, 32, 16, h, o, None) == nsa.NSA_ERR_INVALID_ARG  # no bias
+    assert L.nsa_compress_mlp(a, b, c, d, 1, 64, 1, 64, 32, 16, 0, o, None) == nsa.NSA_ERR_INVALID_ARG  # no hidden
+    assert L.nsa_compress_mlp(a, b, c + 8, d, 1, 64, 1, 64, 32, 16, h, o, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_mlp(a, b, c, d, 1, 64, 1, 96, 32, 16, h, o, None) == nsa.NSA_ERR_UNSUPPORTED
+    assert L.nsa_compress_mlp(a, b, c, d, 1, 64, 1, 64, 16, 8, h, o, None) == nsa.NSA_ERR_UNSUPPORTED
+    sl = 0x7000
+    assert L.nsa_compress_append_mlp(a, b, c, d, sl, 2, 64, 1, 64, 32, 16, 0, o, 3, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_append_mlp(a, b, c, d, sl + 2, 2, 64, 1, 64, 32, 16, h, o, 3, None) == \
+        nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_append_mlp(a, b, c, d, sl, 2, 64, 1, 64, 32, 16, h, o, 0, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_compress_append_mlp(a, b, c, d, sl, 2, 64, 1, 192, 16, 16, h, o, 3, None) == \
+        nsa.NSA_ERR_UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(nsa, "_lib", None)
     monkeypatch.setattr(nsa, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -39,28 +39,38 @@ def run_decode(d, seqlens, top_k, window, Lmax=None, score_map=0):
 
 
 def check(d, seqlens, top_k, window, batch=None, score_map=0):
+    """Every sequence's output against the oracle: where the GPU's block choice for a group
+    differs from the oracle's by a legal near-tie swap, the oracle reruns that sequence on the
+    GPU's blocks (forced-index mode) and that group's rows are compared with the rerun."""
     out, idx = run_decode(d, seqlens, top_k, window, score_map=score_map)
     bs = list(range(d.q.shape[0])) if batch is None else batch
     sub = lambda t: t[bs]
     kc = oracle.compress_cache(sub(d.k_cache), d.w_k, 32, 16)
     vc = oracle.compress_cache(sub(d.v_cache), d.w_v, 32, 16)
-    ref = oracle.nsa_decode(sub(d.q), sub(d.k_cache), sub(d.v_cache), kc, vc, seqlens[bs], sub(d.gates),
-                            top_k=top_k, window=window, score_map=oracle.SCORE_MAPS[score_map])
+    run = lambda rows, forced=None: oracle.nsa_decode(
+        sub(d.q), sub(d.k_cache), sub(d.v_cache), kc, vc, seqlens[bs], sub(d.gates), top_k=top_k, window=window,
+        score_map=oracle.SCORE_MAPS[score_map], batch=rows, forced_idx=forced)
+    ref = run(None)
     toks = [int(seqlens[b]) - 1 for b in bs]
     gi = idx[bs]
     hq, hkv = d.q.shape[1], d.k_cache.shape[2]
     G = hq // hkv
-    mask = torch.ones(len(bs), hq, dtype=torch.bool)
     n_exact = 0
-    for i, b in enumerate(bs):
+    ref_out = ref["out"].clone()
+    for i in range(len(bs)):
+        swapped_groups = []
         for g in range(hkv):
             e, sw = idx_agreement(gi[i:i + 1, g:g + 1].unsqueeze(2), ref["idx"][i:i + 1, g:g + 1].unsqueeze(2),
                                   [[[ref["score"][i][g]]]], tokens=[toks[i]])
             n_exact += e
             if sw:
-                mask[i, g * G:(g + 1) * G] = False
+                swapped_groups.append(g)
+        if swapped_groups:
+            forced = run([i], gi[i:i + 1])["out"][0]
+            for g in swapped_groups:
+                ref_out[i, g * G:(g + 1) * G] = forced[g * G:(g + 1) * G]
     assert n_exact >= 0.9 * len(bs) * hkv
-    assert_close(out[bs], ref["out"], mask=mask.unsqueeze(-1).expand(-1, -1, out.shape[-1]), what="decode out")
+    assert_close(out[bs], ref_out, what="decode out")
     return n_exact
 
 
@@ -108,17 +118,24 @@ def test_decode_workload_sampled():
     sub = lambda t: t[bs]
     kc = oracle.compress_cache(sub(host.k_cache), host.w_k, 32, 16)
     vc = oracle.compress_cache(sub(host.v_cache), host.w_v, 32, 16)
-    ref = oracle.nsa_decode(sub(host.q), sub(host.k_cache), sub(host.v_cache), kc, vc, host.seqlens[bs],
-                            sub(host.gates), top_k=c["top_k"], window=c["window"])
+    run = lambda rows, forced=None: oracle.nsa_decode(
+        sub(host.q), sub(host.k_cache), sub(host.v_cache), kc, vc, host.seqlens[bs], sub(host.gates),
+        top_k=c["top_k"], window=c["window"], batch=rows, forced_idx=forced)
+    ref = run(None)
     G = c["h_q"] // c["h_kv"]
-    mask = torch.ones(len(bs), c["h_q"], dtype=torch.bool)
+    ref_out = ref["out"].clone()
     for i, b in enumerate(bs):
+        swapped_groups = []
         for g in range(c["h_kv"]):
             _, sw = idx_agreement(idx[b:b + 1, g:g + 1].unsqueeze(2), ref["idx"][i:i + 1, g:g + 1].unsqueeze(2),
                                   [[[ref["score"][i][g]]]], tokens=[c["L"] - 1])
             if sw:
-                mask[i, g * G:(g + 1) * G] = False
-    assert_close(out[bs], ref["out"], mask=mask.unsqueeze(-1).expand(-1, -1, out.shape[-1]), what="decode 64K")
+                swapped_groups.append(g)
+        if swapped_groups:   # the oracle on the GPU's blocks for this sequence
+            forced = run([i], idx[b:b + 1])["out"][0]
+            for g in swapped_groups:
+                ref_out[i, g * G:(g + 1) * G] = forced[g * G:(g + 1) * G]
+    assert_close(out[bs], ref_out, what="decode 64K")
 
 
 @pytest.mark.parametrize("score_map", [1, 2])

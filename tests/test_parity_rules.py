@@ -92,3 +92,20 @@ def test_dsa_forced_index_mode_with_own_choice_reproduces_the_oracle():
     again = oracle.dsa_forward(x.q, x.k, x.v, x.q_idx, x.k_idx, x.w_idx, top_k=16, tokens=toks,
                                forced_idx=ref["idx"])
     assert torch.equal(ref["out"], again["out"])
+
+
+def test_decode_forced_index_mode_with_own_choice_reproduces_the_oracle():
+    d = synth.decode_inputs(2, 400, 8, 2, 64, 64, seed=93)
+    sl = torch.tensor([400, 257], dtype=torch.int32)
+    kc = oracle.compress_cache(d.k_cache, d.w_k, 32, 16)
+    vc = oracle.compress_cache(d.v_cache, d.w_v, 32, 16)
+    run = lambda forced=None, batch=None: oracle.nsa_decode(d.q, d.k_cache, d.v_cache, kc, vc, sl, d.gates,
+                                                            top_k=3, window=50, batch=batch, forced_idx=forced)
+    ref = run()
+    assert torch.equal(run(ref["idx"])["out"], ref["out"])
+    assert torch.equal(run(ref["idx"][1:], batch=[1])["out"], ref["out"][1:])
+    other = ref["idx"].clone()
+    other[0, 1] = torch.tensor([0, 1, 6])                 # another valid choice for sequence 0, group 1
+    moved = run(other)["out"]
+    assert torch.equal(moved[1], ref["out"][1]) and torch.equal(moved[0, :4], ref["out"][0, :4])
+    assert not torch.allclose(moved[0, 4:], ref["out"][0, 4:])

@@ -461,7 +461,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           // masked scores; only a tile that straddles this row's range needs the per-element
           // test.  The maximum is taken on the raw scores (the scale is positive, and rounding
           // x * scale is monotone, so it equals the maximum of the scaled ones) and the scale
-          // is applied inside the exponent's FMA.  Max and sum use eight independent chains each.
+          // is applied inside the exponent's FMA.  Max and sum use eight independent chains each
+          // (the sums as four packed pairs).
           const int i0 = n * kBlk + col0;
           if (i0 + kCols - 1 >= my_hi) {
 #pragma unroll
@@ -476,13 +477,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                  fmaxf(fmaxf(cmx[4], cmx[5]), fmaxf(cmx[6], cmx[7]))) * scale_log2;
           const float mn = fmaxf(m, cm);
           if (mn != -INFINITY) {
-            float ps[8];
+            // two columns per packed fma and add; four packed sums (eight chains)
+            const uint64_t sc2 = f2_pack(scale_log2, scale_log2), nm2 = f2_pack(-mn, -mn);
+            uint64_t ps[4];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) ps[c] = ex2(fmaf(v[c], scale_log2, -mn));
-#pragma unroll
-            for (int j = 8; j < kCols; ++j) ps[j & 7] += ex2(fmaf(v[j], scale_log2, -mn));
-            const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-            l = l * ex2(m - mn) + sum;
+            for (int c = 0; c < kCols / 2; ++c) {
+              const float2 a = f2_unpack(f2_fma(f2_pack(v[2 * c], v[2 * c + 1]), sc2, nm2));
+              const uint64_t p2 = f2_pack(ex2(a.x), ex2(a.y));
+              ps[c & 3] = c < 4 ? p2 : f2_add(ps[c & 3], p2);
+            }
+            const float2 t = f2_unpack(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])));
+            l = l * ex2(m - mn) + (t.x + t.y);
             m = mn;
           }
         }
@@ -500,7 +505,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
           for (int q = 0; q < kSoftGroups; ++q) L += sML[(q * 128 + r) * 2 + 1] * ex2(sML[(q * 128 + r) * 2] - M);
         }
-        sLse[r] = (t0 + r / 16 < len && L > 0.f) ? M + __log2f(L) : INFINITY;
+        sLse[r] = (t0 + r / 16 < len && L > 0.f) ? -(M + __log2f(L)) : -INFINITY;   // stored negated
       }
       // the previous item's scores must have been taken (and zeroed) by the top-k warps
       if (k > 0) ok = tc::mbar_wait(sc_empty, (k - 1) & 1, err, kErrScEmpty);
@@ -555,21 +560,28 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         uint32_t pk[kCols / 2];
 #pragma unroll
         for (int kk = 0; kk < kTokG; ++kk) {
-          const bool vis = i < hi_tok[kk];
           float sacc = 0.f;
+          if (i < hi_tok[kk]) {
+            // two columns per packed fma: x * scale - lse (the negated log-sum-exp of four
+            // columns in one broadcast load), then the exponents and a packed running sum
+            const uint64_t sc2 = f2_pack(scale_log2, scale_log2);
+            uint64_t acc2 = f2_pack(0.f, 0.f);
 #pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            // the log-sum-exp of four columns in one broadcast load
-            const float4 ls = *reinterpret_cast<const float4*>(sLse + col0 + 16 * kk + j);
-            const float p0 = vis ? ex2(fmaf(v[16 * kk + j], scale_log2, -ls.x)) : 0.f;
-            const float p1 = vis ? ex2(fmaf(v[16 * kk + j + 1], scale_log2, -ls.y)) : 0.f;
-            const float p2 = vis ? ex2(fmaf(v[16 * kk + j + 2], scale_log2, -ls.z)) : 0.f;
-            const float p3 = vis ? ex2(fmaf(v[16 * kk + j + 3], scale_log2, -ls.w)) : 0.f;
-            sacc += (p0 + p1) + (p2 + p3);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            pk[8 * kk + j / 2] = *reinterpret_cast<uint32_t*>(&h2);
-            h2 = __floats2bfloat162_rn(p2, p3);
-            pk[8 * kk + j / 2 + 1] = *reinterpret_cast<uint32_t*>(&h2);
+            for (int j = 0; j < 16; j += 4) {
+              const float4 nl = *reinterpret_cast<const float4*>(sLse + col0 + 16 * kk + j);
+              const float2 a01 = f2_unpack(f2_fma(f2_pack(v[16 * kk + j], v[16 * kk + j + 1]), sc2, f2_pack(nl.x, nl.y)));
+              const float2 a23 =
+                  f2_unpack(f2_fma(f2_pack(v[16 * kk + j + 2], v[16 * kk + j + 3]), sc2, f2_pack(nl.z, nl.w)));
+              const float p0 = ex2(a01.x), p1 = ex2(a01.y), p2 = ex2(a23.x), p3 = ex2(a23.y);
+              acc2 = f2_add(acc2, f2_add(f2_pack(p0, p1), f2_pack(p2, p3)));
+              pk[8 * kk + j / 2] = pack_bf16(p0, p1);
+              pk[8 * kk + j / 2 + 1] = pack_bf16(p2, p3);
+            }
+            const float2 a = f2_unpack(acc2);
+            sacc = a.x + a.y;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pk[8 * kk + j] = 0u;
           }
           // block i = this thread's r straddles two selection blocks when i % 4 == 3
           tok_sum[kk] = (lane & 3) == 3 ? sacc * w_straddle : sacc;

@@ -2,12 +2,16 @@
 // Week 45", "Which Attention is All You Need?", section "Linear v.s. Sparse", point 6: a light
 // indexer scores every earlier token, the top-k tokens are kept, and full attention runs over them).
 //
-//   D1 indexer   score[t, s] = sum_j w[t, j] * ReLU(q_I[t, j] . k_I[s]) for s <= t, fp32, by warp
-//                MMAs over 64 x 64 (query, key) tiles, one indexer head at a time.
-//   D2 top-k     per query token: radix select of the k-th largest score (order-preserving
-//                integer keys, four 8-bit passes), then one pass in index order that keeps the
-//                larger scores and, among the equal ones, the lowest indices -- the list comes
-//                out ascending.
+//   D1+D2 select  per 16 query tokens (one CTA, longest rows first), with no score matrix in
+//                memory: the indexer score tiles score[t, s] = sum_j w[t, j] * ReLU(q_I[t, j] . k_I[s]),
+//                s <= t (fp32, warp MMAs over 16 x 32 (query, key) tiles, one indexer head at a time)
+//                are computed, and recomputed, as the selection needs them.  Four passes of an
+//                8-bit radix select over order-preserving integer keys find each token's k-th
+//                largest score (a 256-bin histogram per token in shared memory), a fifth pass
+//                counts the keys above it and equal to it per quarter of the key range, and a
+//                sixth writes the chosen tokens: those above, then the lowest-index ones equal to
+//                it -- the list comes out ascending.  Every pass computes a tile with the same
+//                instructions in the same order, so the scores agree bit for bit between passes.
 //   D4 attention one CTA per (token, KV group): the 8 warps stream the chosen tokens' K/V rows
 //                (gathered with cp.async) with an online softmax over the group's heads, then
 //                merge their states.
@@ -20,151 +24,277 @@
 namespace nsa {
 
 namespace {
-constexpr int kIdxTile = 64;   // queries and keys per indexer tile
-constexpr int kIdxThreads = 128;
-
-template <int DI>
-__global__ void __launch_bounds__(kIdxThreads)
-dsa_indexer_kernel(const __nv_bfloat16* __restrict__ qi, const __nv_bfloat16* __restrict__ ki,
-                   const __nv_bfloat16* __restrict__ wi, float* __restrict__ scores, int T, int HI) {
-  const int tq = blockIdx.x, ts = blockIdx.y, b = blockIdx.z;
-  if (ts > tq) return;   // keys after every query of the tile
-  __shared__ __align__(128) __nv_bfloat16 sQ[kIdxTile * DI];
-  __shared__ __align__(128) __nv_bfloat16 sK[kIdxTile * DI];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
-  const int t0 = tq * kIdxTile, s0 = ts * kIdxTile;
-  for (int e = tid; e < kIdxTile * (DI / 8); e += kIdxThreads) {
-    const int r = e / (DI / 8), ch = e % (DI / 8);
-    const bool ok = s0 + r < T;
-    cp_async16(sK + SwzTile<DI>::offset(r, ch), ki + ((size_t)b * T + (ok ? s0 + r : 0)) * DI + ch * 8, ok);
-  }
-  const int ta = t0 + warp * 16 + gl, tb = ta + 8;   // this thread's two query rows
-  float acc[kIdxTile / 8][4];
-#pragma unroll
-  for (int j = 0; j < kIdxTile / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  for (int h = 0; h < HI; ++h) {
-    __syncthreads();   // the previous head's query tile is no longer read
-    for (int e = tid; e < kIdxTile * (DI / 8); e += kIdxThreads) {
-      const int r = e / (DI / 8), ch = e % (DI / 8);
-      const bool ok = t0 + r < T;
-      cp_async16(sQ + SwzTile<DI>::offset(r, ch), qi + (((size_t)b * T + (ok ? t0 + r : 0)) * HI + h) * DI + ch * 8, ok);
-    }
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    uint32_t qf[DI / 16][4];
-#pragma unroll
-    for (int ks = 0; ks < DI / 16; ++ks) {
-      const int row = warp * 16 + (lane & 15);
-      const int ch = 2 * ks + (lane >> 4);
-      ldsm_x4(qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], smem_u32(sQ + SwzTile<DI>::offset(row, ch)));
-    }
-    const float wa = ta < T ? __bfloat162float(wi[((size_t)b * T + ta) * HI + h]) : 0.f;
-    const float wb = tb < T ? __bfloat162float(wi[((size_t)b * T + tb) * HI + h]) : 0.f;
-#pragma unroll
-    for (int kt = 0; kt < kIdxTile / 16; ++kt) {
-      float s[2][4];
-      qk_tile<DI>(qf, sK + kt * 16 * DI, s, 1.f, lane);
-#pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        acc[2 * kt + x][0] += wa * fmaxf(s[x][0], 0.f);
-        acc[2 * kt + x][1] += wa * fmaxf(s[x][1], 0.f);
-        acc[2 * kt + x][2] += wb * fmaxf(s[x][2], 0.f);
-        acc[2 * kt + x][3] += wb * fmaxf(s[x][3], 0.f);
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < kIdxTile / 8; ++j)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int s = s0 + j * 8 + 2 * cq + e;
-      if (s < T && ta < T && s <= ta) scores[((size_t)b * T + ta) * T + s] = acc[j][e];
-      if (s < T && tb < T && s <= tb) scores[((size_t)b * T + tb) * T + s] = acc[j][2 + e];
-    }
-}
-
 // Order-preserving map of a float to an unsigned integer (larger float, larger key).
 __device__ __forceinline__ uint32_t ordered_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-constexpr int kTopkThreads = 256;
+constexpr int kSelRows = 16;                    // query tokens per CTA (one MMA M)
+constexpr int kSelWarps = 4;                    // each takes a contiguous quarter of the key tiles
+constexpr int kSelThreads = 32 * kSelWarps;
+constexpr int kSelKeys = 32;                    // keys per tile
+constexpr int kBins = 256;
+constexpr int kQResident = 32768;               // bytes of indexer queries kept in shared memory
 
-// Block-wide exclusive prefix count of `flag` over the CTA's threads (in thread order) and
-// the total; `sw` is shared scratch of kTopkThreads / 32 ints.
-__device__ __forceinline__ int block_scan(bool flag, int* sw, int& total) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t bal = __ballot_sync(0xffffffffu, flag);
-  if (lane == 0) sw[warp] = __popc(bal);
+template <int DI>
+struct SelSmem {
+  static constexpr size_t kKTile = (size_t)kSelKeys * DI * 2;
+  static constexpr size_t kK = 0;                                          // [warp][2] key tiles
+  static constexpr size_t kQ = kK + (size_t)kSelWarps * 2 * kKTile;        // [HI][16][DI] when resident
+  static constexpr size_t kW = kQ + kQResident;                            // [HI][16] fp32 head weights
+  static constexpr size_t kHist = kW + (size_t)64 * kSelRows * 4;          // [16][256]
+  static constexpr size_t kState = kHist + (size_t)kSelRows * kBins * 4;   // prefix, mask, remaining [16]
+  static constexpr size_t kCnt = kState + 3 * kSelRows * 4;                // [warp][16] (above, equal)
+  static constexpr size_t kTotal = kCnt + (size_t)kSelWarps * kSelRows * 2 * 4;
+  static_assert(kTotal <= 232448, "dsa select shared memory");
+};
+
+template <int DI>
+__global__ void __launch_bounds__(kSelThreads)
+dsa_select_kernel(const __nv_bfloat16* __restrict__ qi, const __nv_bfloat16* __restrict__ ki,
+                  const __nv_bfloat16* __restrict__ wi, int32_t* __restrict__ sel, int T, int HI, int K) {
+  using SM = SelSmem<DI>;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int nq = (T + kSelRows - 1) / kSelRows;
+  const int t0 = (nq - 1 - (int)blockIdx.x) * kSelRows, b = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + SM::kHist);
+  uint32_t* s_prefix = reinterpret_cast<uint32_t*>(smem + SM::kState);
+  uint32_t* s_mask = s_prefix + kSelRows;
+  int* s_rem = reinterpret_cast<int*>(s_mask + kSelRows);
+  int* s_cnt = reinterpret_cast<int*>(smem + SM::kCnt);
+  float* sW = reinterpret_cast<float*>(smem + SM::kW);
+
+  // tokens t0 .. t0+15; a token with t + 1 <= K takes every earlier token, the others select
+  const int t_last = min(t0 + kSelRows - 1, T - 1);
+  bool any_select = false;
+  for (int r = 0; r < kSelRows; ++r) {
+    const int t = t0 + r;
+    if (t < T && t + 1 > K) any_select = true;
+  }
+  if (t0 + 1 <= K) {
+    for (int e = tid; e < kSelRows * K; e += kSelThreads) {
+      const int r = e / K, i = e % K, t = t0 + r;
+      if (t < T && t + 1 <= K) sel[((size_t)b * T + t) * K + i] = i <= t ? i : -1;
+    }
+  }
+  if (!any_select) return;
+
+  const bool resident = (size_t)HI * kSelRows * DI * 2 <= (size_t)kQResident && HI <= 64;
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + SM::kQ);
+  if (resident) {
+    for (int e = tid; e < HI * kSelRows * (DI / 8); e += kSelThreads) {
+      const int h = e / (kSelRows * (DI / 8)), r = (e / (DI / 8)) % kSelRows, ch = e % (DI / 8);
+      const bool ok = t0 + r < T;
+      cp_async16(sQ + h * kSelRows * DI + SwzTile<DI>::offset(r, ch),
+                 qi + (((size_t)b * T + (ok ? t0 + r : 0)) * HI + h) * DI + ch * 8, ok);
+    }
+    cp_async_commit();
+  }
+  for (int e = tid; e < HI * kSelRows; e += kSelThreads) {
+    const int h = e / kSelRows, r = e % kSelRows;
+    sW[e] = t0 + r < T ? __bfloat162float(wi[((size_t)b * T + t0 + r) * HI + h]) : 0.f;
+  }
+  if (tid < kSelRows) {
+    s_prefix[tid] = 0u;
+    s_mask[tid] = 0u;
+    s_rem[tid] = K;
+  }
+  cp_async_wait<0>();
   __syncthreads();
-  int before = 0;
-  total = 0;
-#pragma unroll
-  for (int w = 0; w < kTopkThreads / 32; ++w) {
-    const int c = sw[w];
-    before += w < warp ? c : 0;
-    total += c;
-  }
-  __syncthreads();   // sw is reused by the next scan
-  return before + __popc(bal & ((1u << lane) - 1u));
-}
 
-__global__ void __launch_bounds__(kTopkThreads)
-dsa_topk_kernel(const float* __restrict__ scores, int32_t* __restrict__ sel, int T, int K) {
-  const int t = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
-  const int n = t + 1;
-  int32_t* dst = sel + ((size_t)b * T + t) * K;
-  if (n <= K) {
-    for (int i = tid; i < K; i += kTopkThreads) dst[i] = i < n ? i : -1;
-    return;
-  }
-  const float* row = scores + ((size_t)b * T + t) * T;
-  __shared__ int hist[256];
-  __shared__ int s_digit, s_remaining;
-  __shared__ int sw[kTopkThreads / 32];
-  uint32_t prefix = 0, mask = 0;
-  int remaining = K;   // how many of the keys matching prefix/mask are still to be taken
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < 256; i += kTopkThreads) hist[i] = 0;
-    __syncthreads();
-    for (int s = tid; s < n; s += kTopkThreads) {
-      const uint32_t u = ordered_key(row[s]);
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (tid == 0) {   // the digit of the remaining-th largest key among the matching ones
-      int cum = 0, d = 255;
-      for (; d > 0; --d) {
-        if (cum + hist[d] >= remaining) break;
-        cum += hist[d];
+  // this thread's two tokens (rows gl and gl + 8 of the MMA tile) and whether they select
+  const int ta = t0 + gl, tb = ta + 8;
+  const bool sa = ta < T && ta + 1 > K, sb = tb < T && tb + 1 > K;
+  // this warp's key tiles: a contiguous quarter of 0 .. ntk-1
+  const int ntk = t_last / kSelKeys + 1;
+  const int kt_begin = warp * ntk / kSelWarps, kt_end = (warp + 1) * ntk / kSelWarps;
+  __nv_bfloat16* sK0 = reinterpret_cast<__nv_bfloat16*>(smem + SM::kK + (size_t)warp * 2 * SM::kKTile);
+  __nv_bfloat16* sK1 = sK0 + kSelKeys * DI;
+
+  auto load_keys = [&](int kt, __nv_bfloat16* dst) {
+    if (kt < kt_end) {
+      const int s0 = kt * kSelKeys;
+#pragma unroll
+      for (int e = lane; e < kSelKeys * (DI / 8); e += 32) {
+        const int r = e / (DI / 8), ch = e % (DI / 8);
+        const bool ok = s0 + r < T;
+        cp_async16(dst + SwzTile<DI>::offset(r, ch), ki + ((size_t)b * T + (ok ? s0 + r : 0)) * DI + ch * 8, ok);
       }
-      s_digit = d;
-      s_remaining = remaining - cum;
+    }
+    cp_async_commit();
+  };
+  // The score tile of key tile kt (keys kt*32 ..): acc[j][e] is token ta's score of key
+  // kt*32 + 8j + 2cq + e, acc[j][2 + e] token tb's.  The same instructions in every pass.
+  auto tile_scores = [&](const __nv_bfloat16* sKt, float (&acc)[kSelKeys / 8][4]) {
+#pragma unroll
+    for (int j = 0; j < kSelKeys / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    for (int h = 0; h < HI; ++h) {
+      uint32_t qf[DI / 16][4];
+      if (resident) {
+#pragma unroll
+        for (int ks = 0; ks < DI / 16; ++ks)
+          ldsm_x4(qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3],
+                  smem_u32(sQ + h * kSelRows * DI + SwzTile<DI>::offset(lane & 15, 2 * ks + (lane >> 4))));
+      } else {
+        const __nv_bfloat16* q0 = qi + (((size_t)b * T + min(ta, T - 1)) * HI + h) * DI;
+        const __nv_bfloat16* q1 = qi + (((size_t)b * T + min(tb, T - 1)) * HI + h) * DI;
+#pragma unroll
+        for (int ks = 0; ks < DI / 16; ++ks) {
+          qf[ks][0] = ld_u32(q0 + ks * 16 + 2 * cq);
+          qf[ks][1] = ld_u32(q1 + ks * 16 + 2 * cq);
+          qf[ks][2] = ld_u32(q0 + ks * 16 + 8 + 2 * cq);
+          qf[ks][3] = ld_u32(q1 + ks * 16 + 8 + 2 * cq);
+        }
+      }
+      const float wa = sW[h * kSelRows + gl], wb = sW[h * kSelRows + gl + 8];
+#pragma unroll
+      for (int kt = 0; kt < kSelKeys / 16; ++kt) {
+        float s[2][4];
+        qk_tile<DI>(qf, sKt + kt * 16 * DI, s, 1.f, lane);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          acc[2 * kt + x][0] += wa * fmaxf(s[x][0], 0.f);
+          acc[2 * kt + x][1] += wa * fmaxf(s[x][1], 0.f);
+          acc[2 * kt + x][2] += wb * fmaxf(s[x][2], 0.f);
+          acc[2 * kt + x][3] += wb * fmaxf(s[x][3], 0.f);
+        }
+      }
+    }
+  };
+  // one sweep of this warp's key tiles; visit(kt, acc) sees every tile in ascending order
+  auto sweep = [&](auto&& visit) {
+    load_keys(kt_begin, sK0);
+    for (int kt = kt_begin; kt < kt_end; ++kt) {
+      const int i = kt - kt_begin;
+      load_keys(kt + 1, (i & 1) ? sK0 : sK1);
+      cp_async_wait<1>();
+      __syncwarp();
+      float acc[kSelKeys / 8][4];
+      tile_scores((i & 1) ? sK1 : sK0, acc);
+      visit(kt, acc);
+      __syncwarp();   // the buffer is refilled by the next iteration's load
+    }
+    cp_async_wait<0>();
+  };
+
+  // radix passes: the digit of the remaining-th largest key among those matching the prefix
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int e = tid; e < kSelRows * kBins; e += kSelThreads) hist[e] = 0u;
+    __syncthreads();
+    const uint32_t pa = s_prefix[gl], ma = s_mask[gl], pb = s_prefix[gl + 8], mb = s_mask[gl + 8];
+    sweep([&](int kt, const float (&acc)[kSelKeys / 8][4]) {
+#pragma unroll
+      for (int j = 0; j < kSelKeys / 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int s = kt * kSelKeys + j * 8 + 2 * cq + e;
+          const uint32_t ua = ordered_key(acc[j][e]), ub = ordered_key(acc[j][2 + e]);
+          if (sa && s <= ta && (ua & ma) == pa) atomicAdd(&hist[gl * kBins + ((ua >> shift) & 255u)], 1u);
+          if (sb && s <= tb && (ub & mb) == pb) atomicAdd(&hist[(gl + 8) * kBins + ((ub >> shift) & 255u)], 1u);
+        }
+    });
+    __syncthreads();
+    if (tid < kSelRows) {
+      const int t = t0 + tid;
+      if (t < T && t + 1 > K) {
+        const int remaining = s_rem[tid];
+        int cum = 0, d = 255;
+        for (; d > 0; --d) {
+          const int c = (int)hist[tid * kBins + d];
+          if (cum + c >= remaining) break;
+          cum += c;
+        }
+        s_prefix[tid] |= (uint32_t)d << shift;
+        s_mask[tid] |= 255u << shift;
+        s_rem[tid] = remaining - cum;
+      }
     }
     __syncthreads();
-    prefix |= (uint32_t)s_digit << shift;
-    mask |= 255u << shift;
-    remaining = s_remaining;
-    __syncthreads();   // s_digit / s_remaining are rewritten in the next pass
   }
-  // keys above the threshold, plus the `remaining` lowest-index keys equal to it
-  const uint32_t thr = prefix;
-  int eq_before = 0, out_before = 0;
-  for (int base = 0; base < n; base += kTopkThreads) {
-    const int s = base + tid;
-    const uint32_t u = s < n ? ordered_key(row[s]) : 0u;
-    const bool gt = s < n && u > thr, eq = s < n && u == thr;
+
+  // count pass: per warp and token, the keys above the threshold and equal to it
+  const uint32_t thr_a = s_prefix[gl], thr_b = s_prefix[gl + 8];
+  const int rem_a = s_rem[gl], rem_b = s_rem[gl + 8];
+  {
+    int ga = 0, ea = 0, gb = 0, eb = 0;
+    sweep([&](int kt, const float (&acc)[kSelKeys / 8][4]) {
+#pragma unroll
+      for (int j = 0; j < kSelKeys / 8; ++j)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int s = kt * kSelKeys + j * 8 + 2 * cq + e;
+          const uint32_t ua = ordered_key(acc[j][e]), ub = ordered_key(acc[j][2 + e]);
+          const bool va = sa && s <= ta, vb = sb && s <= tb;
+          ga += va && ua > thr_a;
+          ea += va && ua == thr_a;
+          gb += vb && ub > thr_b;
+          eb += vb && ub == thr_b;
+        }
+    });
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      ga += __shfl_xor_sync(0xffffffffu, ga, o);
+      ea += __shfl_xor_sync(0xffffffffu, ea, o);
+      gb += __shfl_xor_sync(0xffffffffu, gb, o);
+      eb += __shfl_xor_sync(0xffffffffu, eb, o);
+    }
+    if (cq == 0) {
+      s_cnt[(warp * kSelRows + gl) * 2] = ga;
+      s_cnt[(warp * kSelRows + gl) * 2 + 1] = ea;
+      s_cnt[(warp * kSelRows + gl + 8) * 2] = gb;
+      s_cnt[(warp * kSelRows + gl + 8) * 2 + 1] = eb;
+    }
+  }
+  __syncthreads();
+
+  // emit pass: this warp's first output slot and equal-key rank for each of its two tokens
+  int out_a = 0, eqs_a = 0, out_b = 0, eqs_b = 0;
+  for (int w = 0; w < warp; ++w) {
+    const int g_a = s_cnt[(w * kSelRows + gl) * 2], e_a = s_cnt[(w * kSelRows + gl) * 2 + 1];
+    const int g_b = s_cnt[(w * kSelRows + gl + 8) * 2], e_b = s_cnt[(w * kSelRows + gl + 8) * 2 + 1];
+    out_a += g_a + min(e_a, max(0, rem_a - eqs_a));
+    out_b += g_b + min(e_b, max(0, rem_b - eqs_b));
+    eqs_a += e_a;
+    eqs_b += e_b;
+  }
+  int32_t* dst_a = sel + ((size_t)b * T + min(ta, T - 1)) * K;
+  int32_t* dst_b = sel + ((size_t)b * T + min(tb, T - 1)) * K;
+  // the quad's exclusive prefix of x in key order (lane cq holds keys 2cq, 2cq+1 of a chunk)
+  auto quad_scan = [&](int x, int& total) {
+    int inc = x;
+    const int p1 = __shfl_up_sync(0xffffffffu, inc, 1, 4);
+    if (cq >= 1) inc += p1;
+    const int p2 = __shfl_up_sync(0xffffffffu, inc, 2, 4);
+    if (cq >= 2) inc += p2;
+    total = __shfl_sync(0xffffffffu, inc, 3, 4);
+    return inc - x;
+  };
+  auto emit = [&](int s0, float v0, float v1, bool sel_row, int t, uint32_t thr, int rem, int& out, int& eqs,
+                  int32_t* dst) {
+    const uint32_t u0 = ordered_key(v0), u1 = ordered_key(v1);
+    const bool ok0 = sel_row && s0 <= t, ok1 = sel_row && s0 + 1 <= t;
+    const bool e0 = ok0 && u0 == thr, e1 = ok1 && u1 == thr;
     int eq_total;
-    const int eq_rank = eq_before + block_scan(eq, sw, eq_total);
-    const bool take = gt || (eq && eq_rank < remaining);
+    const int r0 = eqs + quad_scan((int)e0 + (int)e1, eq_total);
+    const bool k0 = (ok0 && u0 > thr) || (e0 && r0 < rem);
+    const bool k1 = (ok1 && u1 > thr) || (e1 && r0 + (int)e0 < rem);
     int take_total;
-    const int pos = out_before + block_scan(take, sw, take_total);
-    if (take && pos < K) dst[pos] = s;
-    eq_before += eq_total;
-    out_before += take_total;
-  }
+    const int p0 = out + quad_scan((int)k0 + (int)k1, take_total);
+    if (k0 && p0 < K) dst[p0] = s0;
+    if (k1 && p0 + (int)k0 < K) dst[p0 + (int)k0] = s0 + 1;
+    out += take_total;
+    eqs += eq_total;
+  };
+  sweep([&](int kt, const float (&acc)[kSelKeys / 8][4]) {
+#pragma unroll
+    for (int j = 0; j < kSelKeys / 8; ++j) {
+      const int s0 = kt * kSelKeys + j * 8 + 2 * cq;
+      emit(s0, acc[j][0], acc[j][1], sa, ta, thr_a, rem_a, out_a, eqs_a, dst_a);
+      emit(s0, acc[j][2], acc[j][3], sb, tb, thr_b, rem_b, out_b, eqs_b, dst_b);
+    }
+  });
 }
 
 template <int DK, int DV>
@@ -290,23 +420,30 @@ cudaError_t launch_attn(const DsaArgs& a, cudaStream_t st) {
       a.top_k, a.scale_log2);
   return cudaGetLastError();
 }
-}  // namespace
 
-cudaError_t launch_dsa_indexer(const DsaArgs& a, cudaStream_t st) {
-  const int nt = (a.T + kIdxTile - 1) / kIdxTile;
-  dim3 grid(nt, nt, a.B);
-  const auto* qi = static_cast<const __nv_bfloat16*>(a.qi);
-  const auto* ki = static_cast<const __nv_bfloat16*>(a.ki);
-  const auto* wi = static_cast<const __nv_bfloat16*>(a.wi);
-  if (a.di == 64) dsa_indexer_kernel<64><<<grid, kIdxThreads, 0, st>>>(qi, ki, wi, a.scores, a.T, a.hi);
-  else if (a.di == 128) dsa_indexer_kernel<128><<<grid, kIdxThreads, 0, st>>>(qi, ki, wi, a.scores, a.T, a.hi);
-  else return cudaErrorInvalidValue;
+template <int DI>
+cudaError_t launch_select(const DsaArgs& a, cudaStream_t st) {
+  using SM = SelSmem<DI>;
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(dsa_select_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int nq = (a.T + kSelRows - 1) / kSelRows;
+  dsa_select_kernel<DI><<<dim3(nq, a.B), kSelThreads, SM::kTotal, st>>>(
+      static_cast<const __nv_bfloat16*>(a.qi), static_cast<const __nv_bfloat16*>(a.ki),
+      static_cast<const __nv_bfloat16*>(a.wi), a.sel, a.T, a.hi, a.top_k);
   return cudaGetLastError();
 }
+}  // namespace
 
-cudaError_t launch_dsa_topk(const DsaArgs& a, cudaStream_t st) {
-  dsa_topk_kernel<<<dim3(a.T, a.B), kTopkThreads, 0, st>>>(a.scores, a.sel, a.T, a.top_k);
-  return cudaGetLastError();
+cudaError_t launch_dsa_select(const DsaArgs& a, cudaStream_t st) {
+  if (a.hi < 1 || a.hi > 64) return cudaErrorInvalidValue;
+  if (a.di == 64) return launch_select<64>(a, st);
+  if (a.di == 128) return launch_select<128>(a, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_dsa_attn(const DsaArgs& a, cudaStream_t st) {

@@ -107,12 +107,11 @@ struct DsaArgs {
   const void* wi;     // [B, T, hi] indexer head weights
   void* out;          // [B, T, Hq, dv]
   int32_t* sel;       // [B, T, top_k] chosen tokens, ascending, -1 padded
-  float* scores;      // [B, T, T] indexer scores (entries s <= t)
   int B, T, Hq, Hkv, G, dk, dv, hi, di, top_k;
   float scale_log2;
 };
-cudaError_t launch_dsa_indexer(const DsaArgs& a, cudaStream_t st);
-cudaError_t launch_dsa_topk(const DsaArgs& a, cudaStream_t st);
+// D1 + D2: indexer scores and the token-wise top-k, streamed (no score matrix in memory).
+cudaError_t launch_dsa_select(const DsaArgs& a, cudaStream_t st);
 cudaError_t launch_dsa_attn(const DsaArgs& a, cudaStream_t st);
 
 // Backward of the NSA forward (linear phi, equal lengths).  Gradients in fp32; gk, gv, gkc, gvc

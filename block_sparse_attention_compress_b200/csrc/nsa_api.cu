@@ -11,7 +11,7 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int kMaxTokensNsa = 65536;
-constexpr int kMaxTokensDsa = 32768;   // the [T, T] fp32 score matrix: 4 GB per sequence at this length
+constexpr int kMaxTokensDsa = 131072;  // the indexer's work grows as T^2 (six sweeps of the earlier keys)
 constexpr int kMaxDsaTopk = 8192;   // 1024 selection blocks per token (top-k kept in shared memory)
 constexpr int kMaxTokensMoba = 1 << 20;
 
@@ -86,9 +86,9 @@ FwdLayout forward_layout(const nsa_config* c) {
   return L;
 }
 
-// DSA workspace: status word, the [B, T, T] fp32 scores, the [B, T, top_k] chosen tokens.
+// DSA workspace: status word, the [B, T, top_k] chosen tokens.
 struct DsaLayout {
-  size_t err, scores, sel, total;
+  size_t err, sel, total;
 };
 
 DsaLayout dsa_layout(const nsa_config* c) {
@@ -96,7 +96,6 @@ DsaLayout dsa_layout(const nsa_config* c) {
   DsaLayout L{};
   size_t off = 0;
   L.err = off; off = align_up(off + 4);
-  L.scores = off; off = align_up(off + B * T * T * 4);
   L.sel = off; off = align_up(off + B * T * (size_t)c->top_k * 4);
   L.total = off;
   return L;
@@ -401,18 +400,15 @@ nsa_status nsa_dsa_forward(const void* q, const void* k, const void* v, const vo
   nsa::DsaArgs a{};
   a.q = q; a.k = k; a.v = v; a.qi = q_idx; a.ki = k_idx; a.wi = w_idx; a.out = out;
   a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel);
-  a.scores = reinterpret_cast<float*>(ws + L.scores);
   a.B = cfg->batch; a.T = cfg->seqlen; a.Hq = cfg->h_q; a.Hkv = cfg->h_kv; a.G = cfg->h_q / cfg->h_kv;
   a.dk = cfg->d_k; a.dv = cfg->d_v; a.hi = idx_heads; a.di = idx_dim; a.top_k = cfg->top_k;
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
   a.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  StageMarks marks(cfg, 3);
+  StageMarks marks(cfg, 2);
   cudaError_t e = cudaMemsetAsync(ws + L.err, 0, sizeof(int), s);
   if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess) e = nsa::launch_dsa_indexer(a, s);
-  if (e == cudaSuccess) e = marks.mark(s);
-  if (e == cudaSuccess) e = nsa::launch_dsa_topk(a, s);
+  if (e == cudaSuccess) e = nsa::launch_dsa_select(a, s);
   if (e == cudaSuccess) e = marks.mark(s);
   if (e == cudaSuccess) e = nsa::launch_dsa_attn(a, s);
   if (e == cudaSuccess) e = marks.mark(s);

@@ -267,9 +267,10 @@ NSA_API nsa_status nsa_backward(const void* q, const void* k, const void* v, con
  * For every token t: score[s] = sum_j w_idx[t, j] * ReLU(q_idx[t, j] . k_idx[s]) for s <= t
  * (fp32); the top_k keys by score (ties to the lower index; all of them when t + 1 <= top_k);
  * per query head, softmax attention over the chosen tokens (its GQA group's K/V).
- * Workspace: nsa_workspace_size(cfg, 0) bytes (it holds the [B, T, T] fp32 score matrix).
- * Shapes: G = h_q / h_kv <= 16, (d_k, d_v) as nsa_forward, T <= 32768.  Status codes as for
- * nsa_forward.
+ * Workspace: nsa_workspace_size(cfg, 0) bytes: a status word and the [B, T, top_k] chosen
+ * tokens (no score matrix is kept: the scores are recomputed as the selection needs them).
+ * Shapes: G = h_q / h_kv <= 16, (d_k, d_v) as nsa_forward, T <= 131072.  Status codes as for
+ * nsa_forward.  stage_events: 2 stages (indexer + top-k, attention).
  */
 NSA_API nsa_status nsa_dsa_forward(const void* q, const void* k, const void* v, const void* q_idx,
                                    const void* k_idx, const void* w_idx, int32_t idx_heads, int32_t idx_dim,

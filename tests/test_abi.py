@@ -255,6 +255,16 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(c) == nsa.NSA_ERR_WORKSPACE
 
 
+def test_dsa_workspace_holds_only_the_chosen_tokens(lib):
+    """DSA keeps no score matrix: the status word and the [B, T, top_k] chosen tokens."""
+    up = lambda n: (n + 255) // 256 * 256
+    for B, T, K in [(1, 8192, 2048), (2, 32768, 2048), (1, 131072, 512)]:
+        c = nsa.make_config(mode=nsa.NSA_MODE_DSA, batch=B, seqlen=T, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=K)
+        assert nsa.nsa_workspace_size(c) == 256 + up(B * T * K * 4), (B, T, K)
+    c = nsa.make_config(mode=nsa.NSA_MODE_DSA, batch=1, seqlen=131073, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=64)
+    assert nsa.nsa_workspace_size(c) == 0   # past the supported length
+
+
 def test_forward_rejects_dsa_mode(lib):
     """DSA has its own entry point; nsa_forward and nsa_forward_noalloc refuse its mode
     before anything runs (real host tensors, never dereferenced)."""

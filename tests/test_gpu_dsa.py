@@ -1,5 +1,7 @@
 """GPU parity of the DSA forward (nsa_dsa_forward: lightning indexer, token-wise top-k,
 attention over the chosen tokens) against the fp64 oracle on the same seeded inputs."""
+import dataclasses
+
 import pytest
 import torch
 
@@ -90,3 +92,49 @@ def test_dsa_benchmark_workload_sampled():
     T = c["T"]
     toks = sorted(set([0, 1, 2046, 2047, 2048, 2049, 4095, T - 1] + torch.randint(0, T, (24,), generator=g).tolist()))
     check(x, c["top_k"], toks)
+
+
+@pytest.mark.parametrize("hi,di", [(24, 64), (12, 128)])
+def test_dsa_many_indexer_heads(hi, di):
+    """More indexer heads than the select kernel keeps in shared memory: the query fragments
+    come from global memory per head and tile (the other code path of the score tile)."""
+    x = synth.dsa_inputs(1, 600, 16, 1, 128, 128, hi, di, seed=75)
+    check(x, 96, tokens=[0, 95, 96, 97, 300, 511, 599])
+
+
+def test_dsa_exact_ties_take_the_lowest_indices():
+    """Indexer keys repeating every 5 tokens give each query only 5 distinct scores, each held
+    by ~T/5 tokens, so the k-th score is shared by many: the choice must be the lowest indices
+    among the equal ones, exactly as the oracle takes them (scores equal bit for bit on both
+    sides, since the rows are equal)."""
+    x = synth.dsa_inputs(1, 900, 16, 1, 128, 128, 2, 64, seed=76)
+    k_idx = x.k_idx.clone()
+    k_idx[0] = k_idx[0, torch.arange(900) % 5]
+    x = dataclasses.replace(x, k_idx=k_idx)
+    check(x, 100, tokens=[99, 100, 101, 250, 513, 640, 899], min_exact=1.0)
+
+
+def test_dsa_zero_weights_take_the_first_tokens():
+    """A token whose indexer weights are all zero scores every earlier token 0: it takes the
+    first top_k tokens."""
+    x = synth.dsa_inputs(1, 500, 16, 1, 128, 128, 4, 64, seed=77)
+    w = x.w_idx.clone()
+    w[0, 300] = 0
+    w[0, 450] = 0
+    x = dataclasses.replace(x, w_idx=w)
+    out, sel = run_gpu(x, 64)
+    assert sel[0, 300].tolist() == list(range(64)) and sel[0, 450].tolist() == list(range(64))
+    check(x, 64, tokens=[300, 450, 499], out_sel=(out, sel), min_exact=1.0)
+
+
+def test_dsa_32k_runs_with_workspace_of_the_chosen_tokens_only():
+    """T = 32768 with top-2048: the workspace holds only the status word and the chosen tokens
+    (O(T * top_k), no [T, T] score matrix); sampled tokens against the oracle."""
+    T, K = 32768, 2048
+    x = synth.dsa_inputs(1, T, 16, 1, 128, 128, 4, 64, seed=78)
+    cfg = nsa.make_config(mode=nsa.NSA_MODE_DSA, batch=1, seqlen=T, h_q=16, h_kv=1, d_k=128, d_v=128, top_k=K)
+    up = lambda n: (n + 255) // 256 * 256
+    assert nsa.nsa_workspace_size(cfg) == 256 + up(T * K * 4)
+    g = torch.Generator().manual_seed(79)
+    toks = sorted(set([0, K - 1, K, T - 1] + torch.randint(K, T, (12,), generator=g).tolist()))
+    check(x, K, toks)

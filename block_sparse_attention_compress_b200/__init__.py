@@ -20,9 +20,15 @@ NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
 EXPORTED = ("nsa_workspace_size", "nsa_compress", "nsa_compress_append", "nsa_compress_mlp",
             "nsa_compress_append_mlp", "nsa_forward", "nsa_forward_varlen",
-            "nsa_dsa_forward", "nsa_backward", "nsa_decode",
+            "nsa_dsa_forward", "nsa_backward", "nsa_backward_ex", "nsa_decode",
             "nsa_forward_noalloc", "nsa_device_status", "nsa_device_status_noalloc", "nsa_selftest_wait_timeout",
             "nsa_status_string")
+
+
+class NsaGrads(ctypes.Structure):
+    """Mirror of ``nsa_grads`` in include/nsa.h: the fp32 gradient outputs of nsa_backward_ex."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dq", "dk", "dv", "dgates", "dw_k", "dw_v", "db_k", "db_v", "dw_k2", "dw_v2")]
 
 
 class NsaConfig(ctypes.Structure):
@@ -79,6 +85,8 @@ def load_library() -> ctypes.CDLL:
     lib.nsa_forward.argtypes = [vp, vp, vp, vp, cfgp, vp, vp]
     lib.nsa_backward.restype = ctypes.c_int
     lib.nsa_backward.argtypes = [vp, vp, vp, vp, vp, vp, cfgp, vp, vp, vp, vp, vp, vp, vp]
+    lib.nsa_backward_ex.restype = ctypes.c_int
+    lib.nsa_backward_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, cfgp, ctypes.POINTER(NsaGrads), vp]
     lib.nsa_dsa_forward.restype = ctypes.c_int
     lib.nsa_dsa_forward.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, cfgp, vp, vp, vp]
     lib.nsa_forward_varlen.restype = ctypes.c_int
@@ -204,6 +212,19 @@ def nsa_backward(q, k, v, gates, sel_idx, dout, cfg: NsaConfig, dq, dk, dv, dgat
                                      ctypes.byref(cfg), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dgates), _ptr(dw_k),
                                      _ptr(dw_v), _stream(stream, q))
     return _check(st, "nsa_backward") if check else st
+
+
+def nsa_backward_ex(q, k, v, gates, sel_idx, dout, cfg: NsaConfig, grads: dict, cu_seqlens=None, stream=None,
+                    check: bool = True) -> int:
+    """nsa_backward for the MLP phi and packed variable-length batches (see include/nsa.h).
+    grads: dict of fp32 device tensors by nsa_grads field name (db_k, db_v, dw_k2, dw_v2 with the
+    MLP only); cu_seqlens int32 [B + 1] on the device, or None."""
+    g = NsaGrads(**{n: (_ptr(t) if t is not None else None) for n, t in grads.items()})
+    total = int(q.shape[0]) if cu_seqlens is not None else 0
+    st = load_library().nsa_backward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(gates), _ptr(sel_idx), _ptr(dout),
+                                        _ptr(cu_seqlens) if cu_seqlens is not None else None, total,
+                                        ctypes.byref(cfg), ctypes.byref(g), _stream(stream, q))
+    return _check(st, "nsa_backward_ex") if check else st
 
 
 def nsa_dsa_forward(q, k, v, q_idx, k_idx, w_idx, cfg: NsaConfig, out, sel_out=None, stream=None,

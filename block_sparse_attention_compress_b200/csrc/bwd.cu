@@ -15,6 +15,12 @@
 //   bwd_phi_dx_kernel  dX[u] += sum over the compressed blocks i covering token u of
 //                      W[(u - s*i)*d : (u - s*i + 1)*d, :] . dXc[i];
 //   bwd_phi_dw_kernel  dW[r*d + c, j] = sum over (b, h, i) of X[b, s*i + r, h, c] * dXc[b, i, h, j].
+// phi as the two-layer MLP (hidden = bf16(GELU(pre)), pre = vec(block) @ W1 + b1, Xc = hidden @ W2),
+// from dXc:
+//   bwd_mlp_dw2_kernel   dW2[j, m] = sum over the rows (b, i, h) of hidden[j] * dXc[m];
+//   bwd_mlp_dpre_kernel  dpre[j] = (sum_m dXc[m] W2[j, m]) * GELU'(pre[j]), written over pre;
+//   bwd_mlp_db_kernel    db1[j] = sum over the rows of dpre[j];
+//   then the linear kernels above with dpre for dXc and W1 for W give dW1 and dX.
 // Each warp streams its tiles through two shared-memory stages (the next tile is requested
 // before the current one is waited for); the row gradients are float4 atomics (one per lane
 // and 8 columns of a row).
@@ -95,11 +101,15 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
                 const __nv_bfloat16* __restrict__ dout, const int32_t* __restrict__ idx, float* __restrict__ dq,
                 float* __restrict__ dk, float* __restrict__ dv, float* __restrict__ dkc, float* __restrict__ dvc,
                 float* __restrict__ dgates, int T, int Hq, int Hkv, int G, int nc, int top_k, int window,
-                float scale_log2) {
+                float scale_log2, const int32_t* __restrict__ cu) {
   using SM = BwdSmem<DK, DV>;
   extern __shared__ __align__(128) uint8_t smem[];
   const int t = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
+  // sequence b's rows of q, k, v, gates, dout and the gradients start at row `base` (packed
+  // variable-length batch: cu[b]); its tokens past its length have no work
+  const int base = seq_base(cu, b, T);
+  if (t >= seq_len(cu, b, T)) return;
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(smem + SM::kQ);
   __nv_bfloat16* sDO = reinterpret_cast<__nv_bfloat16*>(smem + SM::kDO);
   __nv_bfloat16* sX = reinterpret_cast<__nv_bfloat16*>(smem + SM::kX) + warp * 256;
@@ -110,7 +120,7 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
   float* sG = sD + 16;
   int* sIdx = reinterpret_cast<int*>(smem + SM::kIdx);
   static_assert(kThreads == 256, "the dgate sums take 16 threads per head row");
-  const size_t row0 = ((size_t)b * T + t) * Hq + g * G;   // the group's first head row of this token
+  const size_t row0 = ((size_t)base + t) * Hq + g * G;   // the group's first head row of this token
   for (int e = tid; e < 16 * (DK / 8); e += kThreads) {
     const int r = e / (DK / 8), ch = e % (DK / 8);
     uint4 val = make_uint4(0, 0, 0, 0);
@@ -161,8 +171,8 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
       const int u = min(j, own) * kSel + r % kSel;
       return u <= t ? u : -1;
     };
-    const __nv_bfloat16* kb = br == 0 ? kc + ((size_t)b * nc * Hkv + g) * DK : k + ((size_t)b * T * Hkv + g) * DK;
-    const __nv_bfloat16* vb = br == 0 ? vc + ((size_t)b * nc * Hkv + g) * DV : v + ((size_t)b * T * Hkv + g) * DV;
+    const __nv_bfloat16* kb = br == 0 ? kc + ((size_t)b * nc * Hkv + g) * DK : k + ((size_t)base * Hkv + g) * DK;
+    const __nv_bfloat16* vb = br == 0 ? vc + ((size_t)b * nc * Hkv + g) * DV : v + ((size_t)base * Hkv + g) * DV;
     const int ntiles = (n + kRows - 1) / kRows;
     // Lane l loads row l & 15 of a tile (chunks of parity l >> 4) and holds that row's global
     // index, -1 when the row is masked or past n; the masks of the other rows come from it by
@@ -306,7 +316,7 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
           const int u = u_add;
           float* dst = u < 0 ? nullptr
                              : br == 0 ? dkc + (((size_t)b * nc + u) * Hkv + g) * DK
-                                       : dk + (((size_t)b * T + u) * Hkv + g) * DK;
+                                       : dk + (((size_t)base + u) * Hkv + g) * DK;
           red_rows<DK / 8>(acc, dst, scale_log2 * 0.69314718055994531f, cq);   // times the softmax scale
         } else {
           float acc[DV / 8][4];
@@ -316,7 +326,7 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
           const int u = u_add;
           float* dst = u < 0 ? nullptr
                              : br == 0 ? dvc + (((size_t)b * nc + u) * Hkv + g) * DV
-                                       : dv + (((size_t)b * T + u) * Hkv + g) * DV;
+                                       : dv + (((size_t)base + u) * Hkv + g) * DV;
           red_rows<DV / 8>(acc, dst, 1.f, cq);
         }
       }
@@ -345,11 +355,13 @@ bwd_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 template <int D>
 __global__ void __launch_bounds__(256)
 bwd_phi_dx_kernel(const __nv_bfloat16* __restrict__ w, const float* __restrict__ dxc, float* __restrict__ dx, int B,
-                  int T, int H, int nc) {
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (gw >= B * T * H) return;
-  const int h = gw % H, u = (gw / H) % T, b = gw / (H * T);
-  float* dst = dx + (((size_t)b * T + u) * H + h) * D;
+                  int T, int H, int nc, const int32_t* __restrict__ cu) {
+  const long gw = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= (long)B * T * H) return;
+  const int h = (int)(gw % H), u = (int)((gw / H) % T), b = (int)(gw / ((long)H * T));
+  if (u >= seq_len(cu, b, T)) return;
+  float* dst = dx + (((size_t)seq_base(cu, b, T) + u) * H + h) * D;
   for (int i = max(0, (u - kL) / kS); i <= u / kS && i < nc; ++i) {
     const int r = u - kS * i;
     if (r < 0 || r >= kL) continue;
@@ -374,17 +386,91 @@ bwd_phi_dx_kernel(const __nv_bfloat16* __restrict__ w, const float* __restrict__
 template <int D>
 __global__ void __launch_bounds__(256)
 bwd_phi_dw_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ dxc, float* __restrict__ dw, int B,
-                  int T, int H, int nc) {
+                  int T, int H, int nc, const int32_t* __restrict__ cu) {
   const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= (size_t)kL * D * D) return;
   const int j = (int)(e % D), rc = (int)(e / D), r = rc / D, c = rc % D;
   float acc = 0.f;
-  for (int b = 0; b < B; ++b)
-    for (int i = 0; i < nc; ++i)
+  for (int b = 0; b < B; ++b) {
+    const int base = seq_base(cu, b, T), len = seq_len(cu, b, T);
+    const int nc_b = len < kL ? 0 : min(nc, (len - kL) / kS + 1);   // the sequence's own blocks
+    for (int i = 0; i < nc_b; ++i)
       for (int h = 0; h < H; ++h)
-        acc += __bfloat162float(x[(((size_t)b * T + kS * i + r) * H + h) * D + c]) *
+        acc += __bfloat162float(x[(((size_t)base + kS * i + r) * H + h) * D + c]) *
                dxc[(((size_t)b * nc + i) * H + h) * D + j];
+  }
   dw[e] = acc;
+}
+
+// d/dx of x * Phi(x): Phi(x) + x * phi(x), with Phi the normal CDF and phi its density
+__device__ __forceinline__ float gelu_grad(float x) {
+  return 0.5f * (1.f + erff(x * 0.70710678118654752f)) + x * 0.39894228040143268f * expf(-0.5f * x * x);
+}
+
+// One warp per row: the lanes split m; each j is a warp sum, kept by lane j % 32.
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_mlp_dpre_kernel(const __nv_bfloat16* __restrict__ w2, const float* __restrict__ dxc, float* __restrict__ pre,
+                    long rows) {
+  const long gw = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (gw >= rows) return;
+  float gm[D / 32];
+#pragma unroll
+  for (int x = 0; x < D / 32; ++x) gm[x] = dxc[gw * D + x * 32 + lane];
+  float* pr = pre + gw * D;
+  for (int j = 0; j < D; ++j) {
+    const __nv_bfloat16* wr = w2 + (size_t)j * D;
+    float part = 0.f;
+#pragma unroll
+    for (int x = 0; x < D / 32; ++x) part += __bfloat162float(wr[x * 32 + lane]) * gm[x];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    if (lane == (j & 31)) pr[j] = part * gelu_grad(pr[j]);
+  }
+}
+
+// One thread per output (j, m), a loop over the rows.
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_mlp_dw2_kernel(const __nv_bfloat16* __restrict__ hidden, const float* __restrict__ dxc, float* __restrict__ dw2,
+                   long rows) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= D * D) return;
+  const int j = e / D, m = e % D;
+  float acc = 0.f;
+  for (long r = 0; r < rows; ++r) acc += __bfloat162float(hidden[r * D + j]) * dxc[r * D + m];
+  dw2[e] = acc;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256)
+bwd_mlp_db_kernel(const float* __restrict__ dpre, float* __restrict__ db, long rows) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= D) return;
+  float acc = 0.f;
+  for (long r = 0; r < rows; ++r) acc += dpre[r * D + j];
+  db[j] = acc;
+}
+
+template <int D>
+cudaError_t launch_mlp_tail(const void* w2, const void* hidden, const float* dxc, float* pre, float* dw2, float* db,
+                            long rows, cudaStream_t st) {
+  if (rows > 0) {
+    bwd_mlp_dw2_kernel<D><<<(D * D + 255) / 256, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(hidden), dxc, dw2,
+                                                                 rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    bwd_mlp_dpre_kernel<D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(w2),
+                                                                                  dxc, pre, rows);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else {
+    cudaError_t e = cudaMemsetAsync(dw2, 0, (size_t)D * D * 4, st);
+    if (e != cudaSuccess) return e;
+  }
+  bwd_mlp_db_kernel<D><<<1, 256, 0, st>>>(pre, db, rows);
+  return cudaGetLastError();
 }
 
 template <int DK, int DV>
@@ -402,31 +488,40 @@ cudaError_t launch_attn(const BwdArgs& a, cudaStream_t st) {
       static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.kc),
       static_cast<const __nv_bfloat16*>(a.vc), static_cast<const __nv_bfloat16*>(a.gates),
       static_cast<const __nv_bfloat16*>(a.dout), a.idx, a.dq, a.gk, a.gv, a.gkc, a.gvc, a.dgates, a.T, a.Hq, a.Hkv,
-      a.G, a.nc, a.top_k, a.window, a.scale_log2);
+      a.G, a.nc, a.top_k, a.window, a.scale_log2, a.cu);
   return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t launch_phi(const void* x, const void* w, const float* dxc, float* dx, float* dw, int B, int T, int H,
-                       int nc, cudaStream_t st) {
+                       int nc, const int32_t* cu, cudaStream_t st) {
   if (nc == 0) return cudaSuccess;
   const long warps = (long)B * T * H;
   bwd_phi_dx_kernel<D><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(w), dxc, dx, B, T, H, nc);
+      static_cast<const __nv_bfloat16*>(w), dxc, dx, B, T, H, nc, cu);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t n = (size_t)kL * D * D;
   bwd_phi_dw_kernel<D><<<(unsigned)((n + 255) / 256), 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), dxc, dw, B,
-                                                                    T, H, nc);
+                                                                    T, H, nc, cu);
   return cudaGetLastError();
 }
 
 cudaError_t phi_dispatch(int d, const void* x, const void* w, const float* dxc, float* dx, float* dw, int B, int T,
-                         int H, int nc, cudaStream_t st) {
+                         int H, int nc, const int32_t* cu, cudaStream_t st) {
   switch (d) {
-    case 64: return launch_phi<64>(x, w, dxc, dx, dw, B, T, H, nc, st);
-    case 128: return launch_phi<128>(x, w, dxc, dx, dw, B, T, H, nc, st);
-    case 192: return launch_phi<192>(x, w, dxc, dx, dw, B, T, H, nc, st);
+    case 64: return launch_phi<64>(x, w, dxc, dx, dw, B, T, H, nc, cu, st);
+    case 128: return launch_phi<128>(x, w, dxc, dx, dw, B, T, H, nc, cu, st);
+    case 192: return launch_phi<192>(x, w, dxc, dx, dw, B, T, H, nc, cu, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+cudaError_t mlp_tail_dispatch(int d, const void* w2, const void* hidden, const float* dxc, float* pre, float* dw2,
+                              float* db, long rows, cudaStream_t st) {
+  switch (d) {
+    case 64: return launch_mlp_tail<64>(w2, hidden, dxc, pre, dw2, db, rows, st);
+    case 128: return launch_mlp_tail<128>(w2, hidden, dxc, pre, dw2, db, rows, st);
+    case 192: return launch_mlp_tail<192>(w2, hidden, dxc, pre, dw2, db, rows, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -438,9 +533,20 @@ cudaError_t launch_backward(const BwdArgs& a, cudaStream_t st) {
   else if (a.dk == 128 && a.dv == 128) e = launch_attn<128, 128>(a, st);
   else if (a.dk == 64 && a.dv == 64) e = launch_attn<64, 64>(a, st);
   if (e != cudaSuccess) return e;
-  e = phi_dispatch(a.dk, a.k, a.w_k, a.gkc, a.gk, a.dw_k, a.B, a.T, a.Hkv, a.nc, st);
+  const float* dxk = a.gkc;
+  const float* dxv = a.gvc;
+  if (a.mlp) {   // through the MLP's second layer and GELU: dpre takes the place of dXc
+    const long rows = (long)a.B * a.nc * a.Hkv;
+    e = mlp_tail_dispatch(a.dk, a.w_k2, a.hid_k, a.gkc, a.pre_k, a.dw_k2, a.db_k, rows, st);
+    if (e != cudaSuccess) return e;
+    e = mlp_tail_dispatch(a.dv, a.w_v2, a.hid_v, a.gvc, a.pre_v, a.dw_v2, a.db_v, rows, st);
+    if (e != cudaSuccess) return e;
+    dxk = a.pre_k;
+    dxv = a.pre_v;
+  }
+  e = phi_dispatch(a.dk, a.k, a.w_k, dxk, a.gk, a.dw_k, a.B, a.T, a.Hkv, a.nc, a.cu, st);
   if (e != cudaSuccess) return e;
-  return phi_dispatch(a.dv, a.v, a.w_v, a.gvc, a.gv, a.dw_v, a.B, a.T, a.Hkv, a.nc, st);
+  return phi_dispatch(a.dv, a.v, a.w_v, dxv, a.gv, a.dw_v, a.B, a.T, a.Hkv, a.nc, a.cu, st);
 }
 
 }  // namespace nsa

@@ -32,11 +32,13 @@ constexpr int kBM = 64, kBN = 64, kBK = 64, kThreads = 128;
 // loads' latency; more for the append launch, whose few CTAs each run one long k chain.
 __device__ __forceinline__ float gelu(float x) { return 0.5f * x * (1.f + erff(x * 0.70710678118654752f)); }
 
-template <int D, int DOUT, int STAGES, bool APPEND, bool MLP1 = false, bool HID_OUT = false, bool HID_IN = false>
+template <int D, int DOUT, int STAGES, bool APPEND, bool MLP1 = false, bool HID_OUT = false, bool HID_IN = false,
+          bool PRE_F32 = false>
 __global__ void __launch_bounds__(kThreads)
 compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w, int T, int H,
                 int l, int s, int nc, __nv_bfloat16* __restrict__ out, const int32_t* __restrict__ seqlens,
-                int B, const int32_t* __restrict__ cu, const __nv_bfloat16* __restrict__ bias = nullptr) {
+                int B, const int32_t* __restrict__ cu, const __nv_bfloat16* __restrict__ bias = nullptr,
+                float* __restrict__ pre_out = nullptr) {
   extern __shared__ __align__(128) uint8_t csmem[];
   auto sA = reinterpret_cast<__nv_bfloat16(*)[kBM * kBK]>(csmem);                          // [STAGES]
   auto sB = reinterpret_cast<__nv_bfloat16(*)[kBK * kBN]>(csmem + STAGES * kBM * kBK * 2);  // [STAGES]
@@ -57,7 +59,14 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
     if (i0 >= nc_b) {   // the whole CTA: no block of this sequence, zero its rows
       for (int e = tid; e < kBM * (kBN / 8); e += kThreads) {
         const int i = i0 + e / (kBN / 8), c = (e % (kBN / 8)) * 8;
-        if (i < nc) *reinterpret_cast<uint4*>(out + (((size_t)b * nc + i) * H + h) * DOUT + n0 + c) = make_uint4(0, 0, 0, 0);
+        if (i >= nc) continue;
+        const size_t o = (((size_t)b * nc + i) * H + h) * DOUT + n0 + c;
+        if constexpr (PRE_F32) {
+          *reinterpret_cast<float4*>(pre_out + o) = make_float4(0.f, 0.f, 0.f, 0.f);
+          *reinterpret_cast<float4*>(pre_out + o + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          *reinterpret_cast<uint4*>(out + o) = make_uint4(0, 0, 0, 0);
+        }
       }
       return;
     }
@@ -141,9 +150,22 @@ compress_kernel(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __rest
     const int i = row_win(row);
     if (i < 0) {
       if (!APPEND && i0 + row < nc) {   // past this sequence's blocks: zeros
-        __nv_bfloat16* dst = out + (((size_t)b * nc + i0 + row) * H + h) * DOUT + n0;
+        const size_t o = (((size_t)b * nc + i0 + row) * H + h) * DOUT + n0;
 #pragma unroll
-        for (int j = 0; j < kBN / 8; ++j) *reinterpret_cast<uint32_t*>(dst + j * 8 + 2 * cq) = 0u;
+        for (int j = 0; j < kBN / 8; ++j) {
+          if constexpr (PRE_F32) *reinterpret_cast<float2*>(pre_out + o + j * 8 + 2 * cq) = make_float2(0.f, 0.f);
+          else *reinterpret_cast<uint32_t*>(out + o + j * 8 + 2 * cq) = 0u;
+        }
+      }
+      continue;
+    }
+    if constexpr (PRE_F32) {   // the first layer's pre-activation acc + bias, kept in fp32
+      float* dstf = pre_out + (((size_t)row_seq(row) * nc + i) * H + h) * DOUT + n0;
+#pragma unroll
+      for (int j = 0; j < kBN / 8; ++j) {
+        const int col = n0 + j * 8 + 2 * cq;
+        *reinterpret_cast<float2*>(dstf + j * 8 + 2 * cq) =
+            make_float2(acc[j][2 * half] + __bfloat162float(bias[col]), acc[j][2 * half + 1] + __bfloat162float(bias[col + 1]));
       }
       continue;
     }
@@ -209,12 +231,13 @@ cudaError_t launch_append_mlp(const void* x, const void* w1, const void* b1, con
   k1<<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w1), Lmax, H, l, s, ncmax,
                                                    static_cast<__nv_bfloat16*>(hidden), seqlens, B, nullptr,
-                                                   static_cast<const __nv_bfloat16*>(b1));
+                                                   static_cast<const __nv_bfloat16*>(b1), nullptr);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k2<<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(hidden),
                                                    static_cast<const __nv_bfloat16*>(w2), Lmax, H, l, s, ncmax,
-                                                   static_cast<__nv_bfloat16*>(out), seqlens, B, nullptr, nullptr);
+                                                   static_cast<__nv_bfloat16*>(out), seqlens, B, nullptr, nullptr,
+                                                   nullptr);
   return cudaGetLastError();
 }
 
@@ -254,6 +277,28 @@ cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* 
     case 64: return launch_append<64>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
     case 128: return launch_append<128>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
     case 192: return launch_append<192>(x, w, seqlens, B, Lmax, H, l, s, ncmax, out, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int D>
+cudaError_t launch_mlp_pre(const void* x, const void* w1, const void* b1, int B, int T, int H, int l, int s, int nc,
+                           float* pre, cudaStream_t st, const int32_t* cu) {
+  dim3 grid((nc + kBM - 1) / kBM, D / kBN, B * H);
+  compress_kernel<D, D, 2, false, false, false, false, true><<<grid, kThreads, smem_bytes(2), st>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w1), T, H, l, s, nc, nullptr, nullptr, B,
+      cu, static_cast<const __nv_bfloat16*>(b1), pre);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_compress_mlp_pre(const void* x, const void* w1, const void* b1, int B, int T, int H, int d, int l,
+                                    int s, float* pre, cudaStream_t st, const int32_t* cu) {
+  const int nc = T < l ? 0 : (T - l) / s + 1;
+  if (nc == 0 || B == 0 || H == 0) return cudaSuccess;
+  switch (d) {
+    case 64: return launch_mlp_pre<64>(x, w1, b1, B, T, H, l, s, nc, pre, st, cu);
+    case 128: return launch_mlp_pre<128>(x, w1, b1, B, T, H, l, s, nc, pre, st, cu);
+    case 192: return launch_mlp_pre<192>(x, w1, b1, B, T, H, l, s, nc, pre, st, cu);
     default: return cudaErrorInvalidValue;
   }
 }

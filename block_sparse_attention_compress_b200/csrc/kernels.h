@@ -18,6 +18,10 @@ cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, i
 cudaError_t launch_compress_mlp(const void* x, const void* w1, const void* b1, const void* w2, int B, int T, int H,
                                 int d, int l, int s, void* hidden, void* out, cudaStream_t st,
                                 const int32_t* cu = nullptr);
+// The MLP's first-layer pre-activation vec(block) @ w1 + b1 in fp32 [B, nc, H, d] (the backward's
+// GELU derivative is taken there).
+cudaError_t launch_compress_mlp_pre(const void* x, const void* w1, const void* b1, int B, int T, int H, int d, int l,
+                                    int s, float* pre, cudaStream_t st, const int32_t* cu = nullptr);
 // K1 for a growing cache: for each sequence b whose newest token (L = seqlens[b], clamped
 // to Lmax) completes window i = (L - l)/s < ncmax, out[b, i, h, :] for every head.
 cudaError_t launch_compress_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H,
@@ -135,6 +139,21 @@ struct BwdArgs {
   float* dgates;      // [B, T, Hq, 3]
   float* dw_k;        // [l*dk, dk]
   float* dw_v;        // [l*dv, dv]
+  // phi as the two-layer MLP (mlp = true): w_k/w_v and dw_k/dw_v are then the first layer's
+  bool mlp = false;
+  const void* w_k2 = nullptr;   // [dk, dk] second layer
+  const void* w_v2 = nullptr;
+  const void* hid_k = nullptr;  // [B, nc, Hkv, dk] bf16 hidden rows, as the forward computed them
+  const void* hid_v = nullptr;
+  float* pre_k = nullptr;       // [B, nc, Hkv, dk] fp32 first-layer pre-activation; overwritten by dpre
+  float* pre_v = nullptr;
+  float* dw_k2 = nullptr;       // [dk, dk]
+  float* dw_v2 = nullptr;
+  float* db_k = nullptr;        // [dk]
+  float* db_v = nullptr;
+  // Variable-length batch (cu != nullptr): sequence b's rows of q, k, v, gates, dout, dq, dk,
+  // dv and dgates are cu[b] .. cu[b+1]; idx, kc, vc and their gradients keep the [B, ...] layouts
+  const int32_t* cu = nullptr;
   int B, T, Hq, Hkv, G, dk, dv, nc, top_k, window;
   float scale_log2;
 };

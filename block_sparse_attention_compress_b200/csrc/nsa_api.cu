@@ -1,5 +1,6 @@
 // C ABI of the NSA library: argument validation, workspace carving and the
 // launch sequence on the caller's stream.  See include/nsa.h for the contract.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -76,7 +77,10 @@ FwdLayout forward_layout(const nsa_config* c) {
   L.kc = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
   L.vc = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
   L.idx = off; off = align_up(off + B * c->h_kv * T * c->top_k * 4);
-  L.acc = off; off = align_up(off + B * T * c->h_q * c->d_v * 4);
+  // the branch accumulator; the backward reuses it for the fp32 Kc/Vc gradients (and, with the
+  // MLP phi, the first layers' pre-activations), which are smaller
+  const size_t bwd_rows = B * nc * c->h_kv * (c->d_k + c->d_v) * 4 * (c->phi_mlp ? 2 : 1);
+  L.acc = off; off = align_up(off + std::max(B * T * c->h_q * c->d_v * 4, bwd_rows));
   L.redo = off; off = align_up(off + B * c->h_kv * T * 4);   // the selected branch's redo list
   if (c->phi_mlp) {
     L.hk = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
@@ -332,24 +336,31 @@ nsa_status nsa_forward_varlen(const void* q, const void* k, const void* v, const
   return nsa_forward_impl(q, k, v, gates, cfg, out, static_cast<cudaStream_t>(stream), cu_seqlens, total_tokens);
 }
 
-nsa_status nsa_backward(const void* q, const void* k, const void* v, const void* gates, const int32_t* sel_idx,
-                        const void* dout, const nsa_config* cfg, float* dq, float* dk, float* dv, float* dgates,
-                        float* dw_k, float* dw_v, void* stream) {
+namespace {
+nsa_status backward_impl(const void* q, const void* k, const void* v, const void* gates, const int32_t* sel_idx,
+                         const void* dout, const int32_t* cu, int32_t total, const nsa_config* cfg,
+                         const nsa_grads& g, cudaStream_t s) {
   nsa_status st = check_cfg(cfg);
   if (st != NSA_OK) return st;
-  if (cfg->mode != NSA_MODE_NSA || cfg->phi_mlp) return NSA_ERR_UNSUPPORTED;
-  if (!q || !k || !v || !gates || !sel_idx || !dout || !dq || !dk || !dv || !dgates || !dw_k || !dw_v)
+  if (cfg->mode != NSA_MODE_NSA) return NSA_ERR_UNSUPPORTED;
+  const bool mlp = cfg->phi_mlp != 0;
+  if (!q || !k || !v || !gates || !sel_idx || !dout || !g.dq || !g.dk || !g.dv || !g.dgates || !g.dw_k || !g.dw_v)
     return NSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dq) || !aligned16(dk) ||
-      !aligned16(dv) || (reinterpret_cast<uintptr_t>(gates) & 1u) || (reinterpret_cast<uintptr_t>(sel_idx) & 3u) ||
-      (reinterpret_cast<uintptr_t>(dgates) & 3u) || (reinterpret_cast<uintptr_t>(dw_k) & 3u) ||
-      (reinterpret_cast<uintptr_t>(dw_v) & 3u))
+  if (mlp && (!g.db_k || !g.db_v || !g.dw_k2 || !g.dw_v2)) return NSA_ERR_INVALID_ARG;
+  auto a4 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; };
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(g.dq) || !aligned16(g.dk) ||
+      !aligned16(g.dv) || (reinterpret_cast<uintptr_t>(gates) & 1u) || !a4(sel_idx) || !a4(g.dgates) ||
+      !a4(g.dw_k) || !a4(g.dw_v))
     return NSA_ERR_INVALID_ARG;
+  if (mlp && (!a4(g.db_k) || !a4(g.db_v) || !a4(g.dw_k2) || !a4(g.dw_v2))) return NSA_ERR_INVALID_ARG;
+  if (cu) {
+    if (reinterpret_cast<uintptr_t>(cu) & 3u) return NSA_ERR_INVALID_ARG;
+    if (total < 1 || (int64_t)total > (int64_t)cfg->batch * cfg->seqlen) return NSA_ERR_INVALID_ARG;
+  }
   st = check_workspace(cfg, workspace_bytes(cfg));
   if (st != NSA_OK) return st;
   const FwdLayout L = forward_layout(cfg);
   auto ws = static_cast<uint8_t*>(cfg->workspace);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   nsa::BwdArgs a{};
   a.q = q; a.k = k; a.v = v; a.gates = gates; a.dout = dout; a.idx = sel_idx;
   a.w_k = cfg->w_cmp_k; a.w_v = cfg->w_cmp_v;
@@ -359,26 +370,65 @@ nsa_status nsa_backward(const void* q, const void* k, const void* v, const void*
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.kc = ws + L.kc; a.vc = ws + L.vc;
-  a.dq = dq; a.gk = dk; a.gv = dv; a.dgates = dgates; a.dw_k = dw_k; a.dw_v = dw_v;
-  // the Kc/Vc gradients use the forward's accumulator region (it is larger)
+  a.cu = cu;
+  a.dq = g.dq; a.gk = g.dk; a.gv = g.dv; a.dgates = g.dgates; a.dw_k = g.dw_k; a.dw_v = g.dw_v;
+  // the Kc/Vc gradients (and the MLP's pre-activations) use the forward's accumulator region
   const size_t nkc = (size_t)a.B * a.nc * a.Hkv;
   a.gkc = reinterpret_cast<float*>(ws + L.acc);
   a.gvc = a.gkc + nkc * a.dk;
-  const size_t nk = (size_t)a.B * a.T * a.Hkv;
+  if (mlp) {
+    a.mlp = true;
+    a.w_k2 = cfg->w_cmp_k2; a.w_v2 = cfg->w_cmp_v2;
+    a.hid_k = ws + L.hk; a.hid_v = ws + L.hv;
+    a.pre_k = a.gvc + nkc * a.dv;
+    a.pre_v = a.pre_k + nkc * a.dk;
+    a.dw_k2 = g.dw_k2; a.dw_v2 = g.dw_v2; a.db_k = g.db_k; a.db_v = g.db_v;
+  }
+  const size_t nk = (size_t)(cu ? total : a.B * a.T) * a.Hkv;   // the packed K/V rows
+  const int l = cfg->cmp_block, cs = cfg->cmp_stride;
   cudaError_t e = cudaMemsetAsync(ws + L.err, 0, sizeof(int), s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dk, 0, nk * a.dk * 4, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, nk * a.dv * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.dk, 0, nk * a.dk * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.dv, 0, nk * a.dv * 4, s);
   if (e == cudaSuccess && nkc) e = cudaMemsetAsync(a.gkc, 0, nkc * (a.dk + a.dv) * 4, s);
   if (e == cudaSuccess && a.nc == 0) {   // no compressed block: phi's weights get no gradient
-    e = cudaMemsetAsync(dw_k, 0, (size_t)cfg->cmp_block * a.dk * a.dk * 4, s);
-    if (e == cudaSuccess) e = cudaMemsetAsync(dw_v, 0, (size_t)cfg->cmp_block * a.dv * a.dv * 4, s);
+    e = cudaMemsetAsync(g.dw_k, 0, (size_t)l * a.dk * a.dk * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g.dw_v, 0, (size_t)l * a.dv * a.dv * 4, s);
   }
-  if (e == cudaSuccess)
-    e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, cfg->cmp_block, cfg->cmp_stride, ws + L.kc, s);
-  if (e == cudaSuccess)
-    e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, cfg->cmp_block, cfg->cmp_stride, ws + L.vc, s);
+  if (mlp) {   // the compressed rows and hidden rows as the forward computed them, and pre in fp32
+    if (e == cudaSuccess)
+      e = nsa::launch_compress_mlp(k, cfg->w_cmp_k, cfg->b_cmp_k, cfg->w_cmp_k2, a.B, a.T, a.Hkv, a.dk, l, cs,
+                                   ws + L.hk, ws + L.kc, s, cu);
+    if (e == cudaSuccess)
+      e = nsa::launch_compress_mlp(v, cfg->w_cmp_v, cfg->b_cmp_v, cfg->w_cmp_v2, a.B, a.T, a.Hkv, a.dv, l, cs,
+                                   ws + L.hv, ws + L.vc, s, cu);
+    if (e == cudaSuccess)
+      e = nsa::launch_compress_mlp_pre(k, cfg->w_cmp_k, cfg->b_cmp_k, a.B, a.T, a.Hkv, a.dk, l, cs, a.pre_k, s, cu);
+    if (e == cudaSuccess)
+      e = nsa::launch_compress_mlp_pre(v, cfg->w_cmp_v, cfg->b_cmp_v, a.B, a.T, a.Hkv, a.dv, l, cs, a.pre_v, s, cu);
+  } else {
+    if (e == cudaSuccess) e = nsa::launch_compress(k, cfg->w_cmp_k, a.B, a.T, a.Hkv, a.dk, l, cs, ws + L.kc, s, cu);
+    if (e == cudaSuccess) e = nsa::launch_compress(v, cfg->w_cmp_v, a.B, a.T, a.Hkv, a.dv, l, cs, ws + L.vc, s, cu);
+  }
   if (e == cudaSuccess) e = nsa::launch_backward(a, s);
   return from_cuda(e);
+}
+}  // namespace
+
+nsa_status nsa_backward(const void* q, const void* k, const void* v, const void* gates, const int32_t* sel_idx,
+                        const void* dout, const nsa_config* cfg, float* dq, float* dk, float* dv, float* dgates,
+                        float* dw_k, float* dw_v, void* stream) {
+  if (cfg && cfg->phi_mlp) return NSA_ERR_UNSUPPORTED;   // the MLP's gradients go through nsa_backward_ex
+  nsa_grads g{};
+  g.dq = dq; g.dk = dk; g.dv = dv; g.dgates = dgates; g.dw_k = dw_k; g.dw_v = dw_v;
+  return backward_impl(q, k, v, gates, sel_idx, dout, nullptr, 0, cfg, g, static_cast<cudaStream_t>(stream));
+}
+
+nsa_status nsa_backward_ex(const void* q, const void* k, const void* v, const void* gates, const int32_t* sel_idx,
+                           const void* dout, const int32_t* cu_seqlens, int32_t total_tokens, const nsa_config* cfg,
+                           const nsa_grads* grads, void* stream) {
+  if (!grads) return NSA_ERR_INVALID_ARG;
+  return backward_impl(q, k, v, gates, sel_idx, dout, cu_seqlens, total_tokens, cfg, *grads,
+                       static_cast<cudaStream_t>(stream));
 }
 
 nsa_status nsa_dsa_forward(const void* q, const void* k, const void* v, const void* q_idx, const void* k_idx,

@@ -235,7 +235,8 @@ NSA_API nsa_status nsa_forward_varlen(const void* q, const void* k, const void* 
 
 /*
  * nsa_backward -- gradients of the NSA forward ([NOTES] §13: NSA is trained natively, forward
- * and backward).  NSA mode, linear phi (phi_mlp = 0), batch of equal lengths.
+ * and backward).  NSA mode, linear phi (phi_mlp = 0), batch of equal lengths; nsa_backward_ex
+ * takes the MLP phi and variable-length batches.
  *   q, k, v, gates  the forward's inputs (as for nsa_forward);
  *   sel_idx   int32 [B, H_kv, T, top_k]: the blocks the forward chose (its sel_idx_out).  The
  *             choice is discrete: no gradient flows through the scores and the top-k;
@@ -251,6 +252,44 @@ NSA_API nsa_status nsa_forward_varlen(const void* q, const void* k, const void* 
 NSA_API nsa_status nsa_backward(const void* q, const void* k, const void* v, const void* gates,
                                 const int32_t* sel_idx, const void* dout, const nsa_config* cfg, float* dq,
                                 float* dk, float* dv, float* dgates, float* dw_k, float* dw_v, void* stream);
+
+/*
+ * nsa_backward_ex -- nsa_backward for every shape the forward takes: phi as the two-layer MLP
+ * (cfg->phi_mlp = 1, its weights in cfg as for nsa_forward) and packed variable-length batches
+ * (cu_seqlens as for nsa_forward_varlen).
+ *   cu_seqlens    int32 [B + 1] on the device, or NULL for B sequences of cfg->seqlen tokens;
+ *   total_tokens  the packed row count (cu_seqlens[B]) when cu_seqlens is given;
+ *   q, k, v, gates, dout, and the dq, dk, dv, dgates outputs are then packed [total, ...]
+ *   like the forward's; sel_idx keeps the forward's [B, H_kv, T, top_k] layout (T =
+ *   cfg->seqlen, the longest sequence).
+ *   grads         the outputs:
+ *     dq, dk, dv, dgates, dw_k, dw_v  as for nsa_backward (with the MLP, dw_k and dw_v are the
+ *                                     first layers' gradients [l*d, d]);
+ *     db_k, db_v    fp32 [d_k], [d_v]      the first layers' bias gradients   } phi_mlp = 1
+ *     dw_k2, dw_v2  fp32 [d_k, d_k], [d_v, d_v]  the second layers' gradients } only
+ * With the MLP, the gradient goes through the second layer, GELU and the first layer:
+ * dW2 = hidden^T dXc, dpre = (dXc W2^T) * GELU'(pre), db1 = sum of dpre, and dpre then takes
+ * the place of dXc in the linear map's gradients; the bf16 rounding of the hidden rows is
+ * passed through (its derivative taken as 1).  Order of sums and reproducibility as for
+ * nsa_backward.  Status codes as for nsa_backward.
+ */
+typedef struct {
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dgates;
+  float* dw_k;
+  float* dw_v;
+  float* db_k;
+  float* db_v;
+  float* dw_k2;
+  float* dw_v2;
+} nsa_grads;
+
+NSA_API nsa_status nsa_backward_ex(const void* q, const void* k, const void* v, const void* gates,
+                                   const int32_t* sel_idx, const void* dout, const int32_t* cu_seqlens,
+                                   int32_t total_tokens, const nsa_config* cfg, const nsa_grads* grads,
+                                   void* stream);
 
 /*
  * nsa_dsa_forward -- token-wise sparse attention behind a lightning indexer (DSA; 10100.com,

@@ -153,6 +153,22 @@ def test_compress_mlp_rejects_bad_arguments(lib):
         nsa.NSA_ERR_UNSUPPORTED
 
 
+def test_backward_entry_points_check_their_arguments(lib):
+    """nsa_backward takes the linear phi only; nsa_backward_ex needs the MLP's gradient buffers
+    when phi is the MLP.  All checked before any CUDA call."""
+    c = _cfg(h_q=16, h_kv=1, d_k=192, d_v=128)
+    c.phi_mlp, c.w_cmp_k2, c.w_cmp_v2, c.b_cmp_k, c.b_cmp_v = 1, 0x7000, 0x8000, 0x9000, 0xa000
+    p = [0x10000 * (i + 1) for i in range(12)]
+    st = lib.nsa_backward(p[0], p[1], p[2], p[3], p[4], p[5], ctypes.byref(c), p[6], p[7], p[8], p[9], p[10], p[11],
+                          None)
+    assert st == nsa.NSA_ERR_UNSUPPORTED
+    g = nsa.NsaGrads(dq=p[6], dk=p[7], dv=p[8], dgates=p[9], dw_k=p[10], dw_v=p[11])   # no MLP gradients
+    st = lib.nsa_backward_ex(p[0], p[1], p[2], p[3], p[4], p[5], None, 0, ctypes.byref(c), ctypes.byref(g), None)
+    assert st == nsa.NSA_ERR_INVALID_ARG
+    assert lib.nsa_backward_ex(p[0], p[1], p[2], p[3], p[4], p[5], None, 0, ctypes.byref(c), None, None) == \
+        nsa.NSA_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(nsa, "_lib", None)
     monkeypatch.setattr(nsa, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -494,3 +494,36 @@ def test_oracle_gradients_match_finite_differences():
             fd = (loss({**base, name: up}) - loss({**base, name: dn})) / (2 * h)
             ad = leaves[name].grad.reshape(-1)[pos]
             assert abs(float(fd - ad)) <= 1e-5 * max(1.0, abs(float(ad))), (name, pos, float(fd), float(ad))
+
+
+def test_oracle_mlp_gradients_match_finite_differences():
+    """The same pin with phi as the two-layer MLP: autograd through GELU, both layers and the
+    bias against central differences (hidden rows unrounded, so the function is smooth), at a
+    few coordinates of every input, the MLP's weights and bias included.  The backward's MLP
+    gradients (dW2 = hidden^T dXc, dpre = dXc W2^T GELU'(pre), db1 = sum of dpre) are checked
+    against this autograd on the GPU."""
+    x = synth.nsa_inputs(1, 70, 4, 1, 64, 64, seed=11)
+    w_k, b_k, w_k2 = synth.phi_mlp_weights(32, 64, seed=12)
+    w_v, b_v, w_v2 = synth.phi_mlp_weights(32, 64, seed=13)
+    base = {n: t.double() for n, t in dict(q=x.q, k=x.k, v=x.v, gates=x.gates, w_k=w_k, w_v=w_v, b_k=b_k,
+                                            w_k2=w_k2, b_v=b_v, w_v2=w_v2).items()}
+    mlp_names = ("b_k", "w_k2", "b_v", "w_v2")
+    run = lambda inp, forced=None: oracle.nsa_forward(
+        *[inp[n] for n in ("q", "k", "v", "gates", "w_k", "w_v")], top_k=3, window=20, round_kc=False,
+        mlp={n: inp[n] for n in mlp_names}, forced_idx=forced)
+    forced = run(base)["idx"]
+    g = torch.Generator().manual_seed(14)
+    dout = torch.randn(run(base, forced)["out"].shape, generator=g, dtype=torch.float64)
+    loss = lambda inp: (run(inp, forced)["out"] * dout).sum()
+    leaves = {n: t.clone().requires_grad_() for n, t in base.items()}
+    loss(leaves).backward()
+    for name, t in base.items():
+        flat = t.reshape(-1)
+        for pos in torch.randint(0, flat.numel(), (3,), generator=g).tolist():
+            h = 1e-6 * max(1.0, abs(float(flat[pos])))
+            up, dn = t.clone(), t.clone()
+            up.reshape(-1)[pos] += h
+            dn.reshape(-1)[pos] -= h
+            fd = (loss({**base, name: up}) - loss({**base, name: dn})) / (2 * h)
+            ad = leaves[name].grad.reshape(-1)[pos]
+            assert abs(float(fd - ad)) <= 1e-5 * max(1.0, abs(float(ad))), (name, pos, float(fd), float(ad))

@@ -178,9 +178,12 @@ struct TopK {
 };
 
 // One instantiation per top_k (0 .. kMaxK), so that the per-thread candidate lists and the
-// merged selections live in registers.
+// merged selections live in registers.  A CTA takes 256 queries of one head (16 warps of 16,
+// each warp with its own block J), so that each tile of block means it streams through shared
+// memory serves 256 queries, and three CTAs (48 warps) share an SM.
+constexpr int kSelQ = 256, kSelThreads = 512;
 template <int KK>
-__global__ void __launch_bounds__(kThreads) moba_select_kernel(
+__global__ void __launch_bounds__(kSelThreads) moba_select_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kbar, int32_t* __restrict__ idx,
     int32_t* __restrict__ counts, int B, int T, int H, int bsz, int nblk) {
   constexpr int N = TopK<KK>::N;
@@ -188,31 +191,32 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
   __nv_bfloat16* sHi = reinterpret_cast<__nv_bfloat16*>(smem);          // [2][kKT][D]
   __nv_bfloat16* sLo = sHi + 2 * kKT * D;                               // [2][kKT][D]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gl = lane >> 2, cq = lane & 3;
-  const int t0 = blockIdx.x * kQ, h = blockIdx.y, b = blockIdx.z;
-  const int J = t0 / bsz;                      // own block, the same for the whole tile (bsz % 64 == 0)
+  const int t0 = blockIdx.x * kSelQ, h = blockIdx.y, b = blockIdx.z;
+  const int J = (t0 + warp * 16) / bsz;        // this warp's own block (bsz % 64 == 0: one per 16 rows)
+  const int Jc = min(t0 + kSelQ - 1, T - 1) / bsz;   // the CTA's largest: the blocks it streams
   const int ta = t0 + warp * 16 + gl, tb = ta + 8;
   const size_t lo_off = (size_t)B * nblk * H * D;
   const bool choose = KK > 0 && J > KK;        // else every past block is taken
   TopK<KK> k0, k1;
   k0.init();
   k1.init();
-  if (choose) {
+  if (KK > 0 && Jc > KK) {                     // the same decision for every warp of the CTA
     uint32_t qf[D / 16][4];
     load_q_frag(qf, q + (((size_t)b * T + min(ta, T - 1)) * H + h) * D,
                 q + (((size_t)b * T + min(tb, T - 1)) * H + h) * D, ta < T, tb < T, cq);
-    auto load = [&](int j0, int buf) {   // blocks j0 .. j0+63 (zeros past J)
-      for (int e = tid; e < kKT * (D / 8); e += kThreads) {
+    auto load = [&](int j0, int buf) {   // blocks j0 .. j0+63 (zeros past Jc)
+      for (int e = tid; e < kKT * (D / 8); e += kSelThreads) {
         const int r = e / (D / 8), ch = e % (D / 8);
         const int j = j0 + r;
-        const size_t src = (((size_t)b * nblk + min(j, J - 1)) * H + h) * D + ch * 8;
-        cp_async16(sHi + buf * kKT * D + SwzTile<D>::offset(r, ch), kbar + src, j < J);
-        cp_async16(sLo + buf * kKT * D + SwzTile<D>::offset(r, ch), kbar + lo_off + src, j < J);
+        const size_t src = (((size_t)b * nblk + min(j, Jc - 1)) * H + h) * D + ch * 8;
+        cp_async16(sHi + buf * kKT * D + SwzTile<D>::offset(r, ch), kbar + src, j < Jc);
+        cp_async16(sLo + buf * kKT * D + SwzTile<D>::offset(r, ch), kbar + lo_off + src, j < Jc);
       }
     };
     load(0, 0);
     cp_async_commit();
-    for (int j0 = 0, it = 0; j0 < J; j0 += kKT, ++it) {
-      if (j0 + kKT < J) load(j0 + kKT, (it + 1) & 1);
+    for (int j0 = 0, it = 0; j0 < Jc; j0 += kKT, ++it) {
+      if (j0 + kKT < Jc) load(j0 + kKT, (it + 1) & 1);
       cp_async_commit();
       cp_async_wait<1>();
       __syncthreads();
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int j = j0 + nt * 8 + 2 * cq + e;
-          if (j < J) {
+          if (choose && j < J) {
             k0.offer(s[nt][e], j);
             k1.offer(s[nt][2 + e], j);
           }
@@ -265,9 +269,16 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
         if (sel1[i] > sel1[i + 1]) { const int x = sel1[i]; sel1[i] = sel1[i + 1]; sel1[i + 1] = x; }
       }
   }
+  // the picks are counted per block in shared memory (the tile buffers are free now, and the
+  // CTA's blocks 0 .. Jc fit them: at most 16384 of 64 KB), then added to the global counts
+  // once per block: the global adds of many queries on the same popular blocks were the
+  // kernel's largest single cost
+  int32_t* hist = reinterpret_cast<int32_t*>(smem);
+  __syncthreads();
+  for (int j = tid; j <= Jc; j += kSelThreads) hist[j] = 0;
+  __syncthreads();
   if (cq == 0) {
     const int kk = min(KK, J);
-    int32_t* cnt = counts + ((size_t)b * H + h) * nblk;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int t = half ? tb : ta;
@@ -278,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
         if (i < kk) {
           const int sj = half ? sel1[i] : sel0[i];
           dst[i] = sj;
-          atomicAdd(cnt + sj, 1);
+          atomicAdd(hist + sj, 1);
         } else {
           dst[i + 1] = -1;
         }
@@ -286,6 +297,10 @@ __global__ void __launch_bounds__(kThreads) moba_select_kernel(
       dst[kk] = J;
     }
   }
+  __syncthreads();
+  int32_t* cnt = counts + ((size_t)b * H + h) * nblk;
+  for (int j = tid; j <= Jc; j += kSelThreads)
+    if (hist[j] != 0) atomicAdd(cnt + j, hist[j]);
 }
 
 // ------------------------------------------------------------------ M3
@@ -552,6 +567,7 @@ MobaLayout moba_layout(int B, int T, int H, int bsz, int top_k) {
 template <int KK>
 static cudaError_t launch_select(const MobaArgs& a, const __nv_bfloat16* q, const __nv_bfloat16* kbar, int32_t* idx,
                                  int32_t* counts, int nblk, cudaStream_t st) {
+  if ((size_t)nblk * 4 > kSelectSmem) return cudaErrorInvalidValue;   // the per-CTA pick counts
   static bool attr = false;
   if (!attr) {
     const cudaError_t e =
@@ -559,7 +575,7 @@ static cudaError_t launch_select(const MobaArgs& a, const __nv_bfloat16* q, cons
     if (e != cudaSuccess) return e;
     attr = true;
   }
-  moba_select_kernel<KK><<<dim3((a.T + kQ - 1) / kQ, a.H, a.B), kThreads, kSelectSmem, st>>>(q, kbar, idx, counts, a.B,
+  moba_select_kernel<KK><<<dim3((a.T + kSelQ - 1) / kSelQ, a.H, a.B), kSelThreads, kSelectSmem, st>>>(q, kbar, idx, counts, a.B,
                                                                                             a.T, a.H, a.bsz, nblk);
   return cudaGetLastError();
 }

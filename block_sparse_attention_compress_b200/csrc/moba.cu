@@ -343,23 +343,40 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(const int32_t* __restri
     for (int c = chunks[e]; c < chunks[e + 1]; ++c) chunk_list[c] = e;
 }
 
-__global__ void moba_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ offsets,
-                                    int32_t* __restrict__ fill, int32_t* __restrict__ list, int T, int H, int nblk,
-                                    int top_k, int bsz) {
-  const size_t n = (size_t)gridDim.y * T;   // (b*H + h) rows of T tokens
-  const int bh = blockIdx.y;
-  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < T; t += gridDim.x * blockDim.x) {
+// One CTA per 256 consecutive queries of one (b, h): the picks are counted per block in shared
+// memory, each block's range in its list is reserved with one global add per CTA, and every
+// pick then goes to its slot (the order inside a list is free: each query's result depends only
+// on its own row).
+constexpr int kScatterQ = 256;
+__global__ void __launch_bounds__(kScatterQ)
+moba_scatter_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ offsets, int32_t* __restrict__ fill,
+                    int32_t* __restrict__ list, int T, int H, int nblk, int top_k, int bsz) {
+  extern __shared__ int32_t s_slot[];   // [block]: the CTA's count, then the first slot of its range
+  const int bh = blockIdx.y, t0 = blockIdx.x * kScatterQ, t = t0 + threadIdx.x;
+  const int jc = min(t0 + kScatterQ - 1, T - 1) / bsz;   // the picks are blocks below the own block: < jc
+  for (int j = threadIdx.x; j < jc; j += kScatterQ) s_slot[j] = 0;
+  __syncthreads();
+  int pick[8], local[8];
+  int n = 0;
+  if (t < T) {
     const int32_t* row = idx + ((size_t)bh * T + t) * (top_k + 1);
     const int own = t / bsz;
     for (int s = 0; s < top_k; ++s) {
       const int j = row[s];
       if (j < 0 || j >= own) break;
-      const size_t e = (size_t)bh * nblk + j;
-      const int pos = offsets[e] + atomicAdd(&fill[e], 1);
-      list[pos] = t * 8 + s;
+      pick[n] = j;
+      local[n] = atomicAdd(&s_slot[j], 1);
+      ++n;
     }
   }
-  (void)n;
+  __syncthreads();
+  for (int j = threadIdx.x; j < jc; j += kScatterQ) {
+    const int c = s_slot[j];
+    const size_t e = (size_t)bh * nblk + j;
+    s_slot[j] = c > 0 ? offsets[e] + atomicAdd(&fill[e], c) : 0;
+  }
+  __syncthreads();
+  for (int s = 0; s < n; ++s) list[s_slot[pick[s]] + local[s]] = t * 8 + s;
 }
 
 // ------------------------------------------------------------------ M4
@@ -629,8 +646,18 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   const int cq = tc ? moba_past_tc_chunk() : kQ;   // queries per past-attention chunk
   moba_scan_kernel<<<1, 1024, 0, st>>>(counts, offsets, chunks, fill, chunk_list, E, cq);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  moba_scatter_kernel<<<dim3((a.T + 255) / 256, a.B * a.H), 256, 0, st>>>(idx, offsets, fill, list, a.T, a.H, nblk,
-                                                                         a.top_k, a.bsz);
+  {
+    const size_t smem = (size_t)nblk * 4;   // at most 16384 blocks: 64 KB
+    static bool attr = false;
+    if (!attr) {
+      e = cudaFuncSetAttribute(moba_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
+      if (e != cudaSuccess) return e;
+      attr = true;
+    }
+    if (smem > 65536) return cudaErrorInvalidValue;
+    moba_scatter_kernel<<<dim3((a.T + kScatterQ - 1) / kScatterQ, a.B * a.H), kScatterQ, smem, st>>>(
+        idx, offsets, fill, list, a.T, a.H, nblk, a.top_k, a.bsz);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
   int dev = 0, sms = 148;

@@ -27,6 +27,7 @@
 // issuing work, and frees its TMEM.
 #include <algorithm>
 #include <cfloat>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -137,33 +138,57 @@ struct TopkWarp {
   }
 
   // The selection rounds over the first M slots of each lane (slots >= M hold no candidate).
+  // The slots form groups of (up to) eight, each with its best key and slot kept in registers:
+  // a lane's best is the best of its group bests, and when a lane's slot is taken only that
+  // slot's group is scanned again.  Every comparison is strict, so equal keys keep the lowest
+  // slot, and among lanes the lowest block index wins.
   template <int K, int M>
   __device__ __forceinline__ void rounds(int nforced, int top_k, int lane) {
-    // this lane's best key and its mm (the lowest mm among equal keys), by a pairwise tree
-    uint32_t bk = 0;
-    int bm = 0;
-    auto local_best = [&]() {
-      uint32_t kt[M / 2];
-      int mt[M / 2];
+    constexpr int GS = M < 8 ? M : 8;   // slots per group
+    constexpr int NG = M / GS;          // groups
+    uint32_t gk[NG];
+    int gm[NG];
+    // group G's best (G a compile-time constant, so that every slot index is one)
+    auto group_best = [&](auto gc) {
+      constexpr int G = decltype(gc)::value;
+      uint32_t bk = key[K][G * GS];
+      int bm = G * GS;
 #pragma unroll
-      for (int i = 0; i < M / 2; ++i) {
-        const bool c = key[K][2 * i + 1] > key[K][2 * i];
-        kt[i] = c ? key[K][2 * i + 1] : key[K][2 * i];
-        mt[i] = c ? 2 * i + 1 : 2 * i;
-      }
-#pragma unroll
-      for (int w = M / 4; w >= 1; w >>= 1)
-#pragma unroll
-        for (int i = 0; i < w; ++i) {
-          const bool c = kt[2 * i + 1] > kt[2 * i];
-          kt[i] = c ? kt[2 * i + 1] : kt[2 * i];
-          mt[i] = c ? mt[2 * i + 1] : mt[2 * i];
+      for (int i = 1; i < GS; ++i)
+        if (key[K][G * GS + i] > bk) {
+          bk = key[K][G * GS + i];
+          bm = G * GS + i;
         }
-      bk = kt[0];
-      bm = mt[0];
+      gk[G] = bk;
+      gm[G] = bm;
     };
-    local_best();
+    // the group of slot mw: clear the slot and scan the group again
+    auto retake = [&](auto gc, int mw) {
+      constexpr int G = decltype(gc)::value;
+      if (mw / GS != G) return;
+#pragma unroll
+      for (int i = 0; i < GS; ++i)
+        if (G * GS + i == mw) key[K][G * GS + i] = 0u;
+      group_best(gc);
+    };
+    using G0 = std::integral_constant<int, 0>;
+    using G1 = std::integral_constant<int, (NG > 1 ? 1 : 0)>;
+    using G2 = std::integral_constant<int, (NG > 2 ? 2 : 0)>;
+    using G3 = std::integral_constant<int, (NG > 3 ? 3 : 0)>;
+    static_assert(NG <= 4, "at most 32 slots");
+    group_best(G0{});
+    if constexpr (NG > 1) group_best(G1{});
+    if constexpr (NG > 2) group_best(G2{});
+    if constexpr (NG > 3) group_best(G3{});
     for (int rr = nforced; rr < top_k; ++rr) {
+      uint32_t bk = gk[0];
+      int bm = gm[0];
+#pragma unroll
+      for (int g = 1; g < NG; ++g)
+        if (gk[g] > bk) {
+          bk = gk[g];
+          bm = gm[g];
+        }
       const uint32_t vmax = __reduce_max_sync(0xffffffffu, bk);
       if (vmax == 0u) break;
       // the lowest block index among the lanes holding the maximum
@@ -171,10 +196,10 @@ struct TopkWarp {
       if (lane == (int)(jmin & 31u)) {
         const int mw = (int)(jmin >> 5);
         taken[K] |= 1u << mw;
-#pragma unroll
-        for (int mm = 0; mm < M; ++mm)
-          if (mm == mw) key[K][mm] = 0u;
-        local_best();
+        retake(G0{}, mw);
+        if constexpr (NG > 1) retake(G1{}, mw);
+        if constexpr (NG > 2) retake(G2{}, mw);
+        if constexpr (NG > 3) retake(G3{}, mw);
       }
     }
   }

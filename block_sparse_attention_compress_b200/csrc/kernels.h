@@ -193,6 +193,10 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st);
 // Past-block attention on tcgen05 (chunks of moba_past_tc_chunk() queries; block size a
 // multiple of 128).  max_chunks bounds the chunk count written to chunks[E] on the device.
 bool moba_past_tc_supported(const MobaArgs& a);
+// Block selection on tcgen05 (128 queries per CTA as the MMA M, 64 block means per tile as N).
+bool moba_select_tc_supported(const MobaArgs& a, int nblk);
+cudaError_t launch_moba_select_tc(const MobaArgs& a, const void* kbar, int32_t* idx, int32_t* counts, int nblk,
+                                  cudaStream_t st);
 // Own block + merge on tcgen05 (same support condition).
 cudaError_t launch_moba_own_tc(const MobaArgs& a, const int32_t* idx, const __nv_bfloat16* part_o,
                                const float* part_lse, cudaStream_t st);

@@ -630,7 +630,9 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   moba_mean_kernel<<<dim3(nblk, a.H, a.B), D, 0, st>>>(k, kbar, a.B, a.T, a.H, a.bsz, nblk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  switch (a.top_k) {
+  if (moba_select_tc_supported(a, nblk)) {
+    e = launch_moba_select_tc(a, kbar, idx, counts, nblk, st);
+  } else switch (a.top_k) {
     case 0: e = launch_select<0>(a, q, kbar, idx, counts, nblk, st); break;
     case 1: e = launch_select<1>(a, q, kbar, idx, counts, nblk, st); break;
     case 2: e = launch_select<2>(a, q, kbar, idx, counts, nblk, st); break;

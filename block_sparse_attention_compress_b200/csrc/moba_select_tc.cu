@@ -6,14 +6,14 @@
 // MMA (one TMEM lane each), the past blocks' means come in tiles of 64 (the N):
 //   S = Q Kbar^T   (M = 128, N = 64, K = 128: the bf16 hi and lo halves of the fp32 means
 //                   accumulate into the same fp32 tile, so S = q . (hi + lo))
-// Warp 8 loads the queries and the mean tiles by TMA (two tiles in flight), one thread of
-// warp 9 issues the MMAs into two TMEM buffers, and warps 0-7 offer the past blocks to
-// register top-k lists (larger score first, then the lower block): warps w and w + 4 read the
-// same 32 query rows (TMEM lane quadrant w % 4), each 32 of a tile's 64 blocks, and the two
-// lists of a query are merged at the end.  The offers are the kernel's cost (with random scores
-// nearly every offer inserts in some lane of the warp), so each query's chain is split in two.
-// The picks are counted per block in shared memory (the tile buffers, free by then) and added
-// to the global counts once per block.
+// Warp 16 loads the queries and the mean tiles by TMA (two tiles in flight), one thread of
+// warp 17 issues the MMAs into two TMEM buffers, and warps 0-15 offer the past blocks to
+// register top-k lists (larger score first, then the lower block): warps w, w + 4, w + 8 and
+// w + 12 read the same 32 query rows (TMEM lane quadrant w % 4), each 16 of a tile's 64
+// blocks, and the four lists of a query are merged at the end.  The offers are the kernel's
+// cost (with random scores nearly every offer inserts in some lane of the warp), so each
+// query's chain is split in four.  The merge lists and then the per-block pick counts use the
+// tile buffers, free by then; the counts are added to the global ones once per block.
 #include <cfloat>
 
 #include "common.cuh"
@@ -26,7 +26,9 @@ namespace {
 constexpr int D = 128;
 constexpr int kRows = 128;                        // queries per CTA
 constexpr int kTileB = 64;                        // block means per tile
-constexpr int kOfferWarps = 8, kTmaWarp = 8, kMmaWarp = 9, kThreads = 320;
+constexpr int kOfferWarps = 16, kTmaWarp = 16, kMmaWarp = 17, kThreads = 576;
+constexpr int kSplit = kOfferWarps / 4;          // offer threads per query
+constexpr int kCols = kTileB / kSplit;           // a tile's blocks per offer thread
 constexpr uint32_t kQSlab = kRows * 128;          // 128 rows x 64 bf16 (128-byte swizzle): 16 KB
 constexpr uint32_t kBSlab = kTileB * 128;         // 64 rows x 64 bf16: 8 KB
 constexpr uint32_t kTileBytes = 4 * kBSlab;       // hi and lo, two 64-column slabs each: 32 KB
@@ -38,8 +40,7 @@ enum Err { kErrQ = 101, kErrFull, kErrEmpty, kErrSFull, kErrSEmpty };
 struct SelSmem {
   static constexpr uint32_t kQ = 0;                          // 2 slabs
   static constexpr uint32_t kB = kQ + 2 * kQSlab;            // [2 tiles][hi s0, hi s1, lo s0, lo s1]
-  static constexpr uint32_t kMerge = kB + 2 * kTileBytes;   // [128 rows][7] scores + [128][7] blocks
-  static constexpr uint32_t kBar = kMerge + 2 * kRows * 7 * 4;
+  static constexpr uint32_t kBar = kB + 2 * kTileBytes;
   static constexpr int kNumBars = 1 + 2 + 2 + 2 + 2;
   static constexpr uint32_t kTmemSlot = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kTmemSlot + 16;
@@ -80,7 +81,7 @@ struct TopRow {
 };
 
 template <int KK>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kb,
                       int32_t* __restrict__ idx, int32_t* __restrict__ counts, int B, int T, int H, int bsz, int nblk,
                       int* __restrict__ err) {
@@ -123,7 +124,7 @@ moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
   TopRow<KK> top;
   top.init();
-  const int half = warp >> 2;                        // offer warps: which 32 of a tile's 64 blocks
+  const int part = warp >> 2;                        // offer warps: which kCols of a tile's blocks
   const int r = 32 * (warp & 3) + lane;              // this thread's query (offer warps)
   const int t = t0 + r;
   const int J = t / bsz;                             // its own block: the past blocks are 0 .. J-1
@@ -177,7 +178,7 @@ moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
   } else {
     // ------------------------------------------------------------ offers (one query per thread)
-    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + 32 * half;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kCols * part;
     const bool mine = t < T && J > KK;
     bool ok = true;
     for (int it = 0; it < ntile; ++it) {
@@ -185,41 +186,44 @@ moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       ok = __all_sync(0xffffffffu, ok && tc::mbar_wait(s_full + buf, (it >> 1) & 1, err, kErrSFull));
       if (!ok) break;
       tc::tc_fence_after();
-      float v[kTileB / 2];
+      float v[kCols];
 #pragma unroll
-      for (int c = 0; c < kTileB / 2 / 16; ++c)
+      for (int c = 0; c < kCols / 16; ++c)
         tc::tmem_ld16(lane_addr + kTileB * buf + 16 * c, *reinterpret_cast<float(*)[16]>(v + 16 * c));
       tc::tmem_wait_ld();
       tc::tc_fence_before();
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(s_empty + buf);
       if (mine) {
-        const int j0 = it * kTileB + 32 * half;
+        const int j0 = it * kTileB + kCols * part;
 #pragma unroll
-        for (int c = 0; c < kTileB / 2; ++c)
+        for (int c = 0; c < kCols; ++c)
           if (j0 + c < J) top.offer(v[c], j0 + c);
       }
     }
   }
 
-  // the second list of each query joins the first
-  float* mv = reinterpret_cast<float*>(smem + SM::kMerge);
-  int* mj = reinterpret_cast<int*>(mv + kRows * 7);
-  if (warp < kOfferWarps && half == 1) {
+  // every tile has been read (the MMAs before the last s_full, the offers before here): the
+  // tile buffers take the other lists of each query, which join the first
+  float* mv = reinterpret_cast<float*>(sB);                    // [part - 1][row][7]
+  int* mj = reinterpret_cast<int*>(mv + (kSplit - 1) * kRows * 7);
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp < kOfferWarps && part > 0) {
 #pragma unroll
     for (int i = 0; i < TopRow<KK>::N; ++i) {
-      mv[r * 7 + i] = top.v[i];
-      mj[r * 7 + i] = top.j[i];
+      mv[((part - 1) * kRows + r) * 7 + i] = top.v[i];
+      mj[((part - 1) * kRows + r) * 7 + i] = top.j[i];
     }
   }
-  tc::tc_fence_before();
   __syncthreads();
   if (warp < 4) {
 #pragma unroll
-    for (int i = 0; i < TopRow<KK>::N; ++i) top.offer(mv[r * 7 + i], mj[r * 7 + i]);
+    for (int q = 0; q < kSplit - 1; ++q)
+#pragma unroll
+      for (int i = 0; i < TopRow<KK>::N; ++i) top.offer(mv[(q * kRows + r) * 7 + i], mj[(q * kRows + r) * 7 + i]);
   }
-  // every tile has been read (the MMAs before the last s_full, the offers before here): the tile
-  // buffers hold the pick counts of blocks 0 .. Jc
+  // then the pick counts of blocks 0 .. Jc
   int32_t* hist = reinterpret_cast<int32_t*>(sB);
   __syncthreads();
   for (int j = tid; j <= Jc; j += kThreads) hist[j] = 0;

@@ -214,9 +214,9 @@ def workload_config(c, name):
 # compressed cache stay mostly in L2.  An entry goes back to None whenever its kernel
 # changes, until it is captured again.
 NCU_DRAM_BYTES_PER_ITEM = {
-    "cmp_select": (205.892352e6 + 217.154048e6) / 32768,    # profiles/nsa_fwd_8k_kernels_ncu.md
-    "slc_attn": (501143552 + 228722944) / 32768,           # profiles/slc_attn_tc_8k_dram_ncu.md
-    "swa_combine": (494.068480e6 + 118.855680e6) / 32768,   # profiles/nsa_fwd_8k_kernels_ncu.md
+    "cmp_select": (205.892352e6 + 217.154048e6) / 32768,    # --set full capture of the three kernels
+    "slc_attn": (501143552 + 228722944) / 32768,           # dram__bytes capture of the selected branch
+    "swa_combine": (494.068480e6 + 118.855680e6) / 32768,   # --set full capture of the three kernels
 }
 
 # The selected branch gathers whole 64-token K/V blocks from L2 into shared memory; its

@@ -558,6 +558,13 @@ moba_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       plse[sl] = in ? part_lse[(((size_t)b * T + t) * H + h) * top_k + sl] : -INFINITY;
       np += in ? 1 : 0;
     }
+    {   // this thread's half rows of those partials (one 128-byte line each) on their way to L2
+        // while the own block's tiles run: the epilogue reads them after its O is complete
+      const __nv_bfloat16* po = part_o + (((size_t)b * T + (row_ok ? t : 0)) * H + h) * top_k * D + (D / 2) * gr;
+#pragma unroll
+      for (int sl = 0; sl < kMaxPast; ++sl)
+        if (sl < np) prefetch_l2(po + sl * D);
+    }
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int n = 0; n < ntiles; ++n) {

@@ -700,21 +700,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 template <int DK, int DV>
 cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   using SM = Smem<DK, DV>;
-  static bool attr = false;
-  static int sms = 0;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SM::kAlloc);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(attn_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SM::kAlloc);
-    if (e != cudaSuccess) return e;
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
+  const int sms = sm_count();
   CUtensorMap mq, mk, mv;
   const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.total};
   const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};

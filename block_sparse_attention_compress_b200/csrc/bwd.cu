@@ -476,13 +476,13 @@ cudaError_t launch_mlp_tail(const void* w2, const void* hidden, const float* dxc
 template <int DK, int DV>
 cudaError_t launch_attn(const BwdArgs& a, cudaStream_t st) {
   using SM = BwdSmem<DK, DV>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     const cudaError_t e =
         cudaFuncSetAttribute(bwd_attn_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   bwd_attn_kernel<DK, DV><<<dim3(a.T, a.Hkv, a.B), kThreads, SM::kTotal, st>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
       static_cast<const __nv_bfloat16*>(a.v), static_cast<const __nv_bfloat16*>(a.kc),

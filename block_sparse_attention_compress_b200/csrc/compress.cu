@@ -199,13 +199,13 @@ template <int D>
 cudaError_t launch_append(const void* x, const void* w, const int32_t* seqlens, int B, int Lmax, int H, int l,
                           int s, int ncmax, void* out, cudaStream_t st) {
   constexpr int kStages = 8;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     const cudaError_t e = cudaFuncSetAttribute(compress_kernel<D, D, kStages, true>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   dim3 grid((B + kBM - 1) / kBM, D / kBN, H);
   compress_kernel<D, D, kStages, true><<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w), Lmax, H, l, s, ncmax,
@@ -219,14 +219,14 @@ cudaError_t launch_append_mlp(const void* x, const void* w1, const void* b1, con
   constexpr int kStages = 8;
   auto k1 = compress_kernel<D, D, kStages, true, true, true, false>;
   auto k2 = compress_kernel<D, D, kStages, true, false, false, true>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes(kStages));
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   dim3 grid((B + kBM - 1) / kBM, D / kBN, H);
   k1<<<grid, kThreads, smem_bytes(kStages), st>>>(static_cast<const __nv_bfloat16*>(x),
                                                    static_cast<const __nv_bfloat16*>(w1), Lmax, H, l, s, ncmax,

@@ -288,13 +288,13 @@ decode_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restri
 template <int DK, int DV>
 cudaError_t launch(const DecodeArgs& a, cudaStream_t st) {
   const size_t smem = Smem<DK, DV>::kTotal;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(decode_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   dim3 grid(a.Hkv, a.B);
   decode_kernel<DK, DV><<<grid, kThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),

@@ -407,13 +407,13 @@ dsa_attn_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 template <int DK, int DV>
 cudaError_t launch_attn(const DsaArgs& a, cudaStream_t st) {
   using SM = DsaSmem<DK, DV>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     const cudaError_t e =
         cudaFuncSetAttribute(dsa_attn_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   dsa_attn_kernel<DK, DV><<<dim3(a.T, a.Hkv, a.B), kThreads, SM::kTotal, st>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
       static_cast<const __nv_bfloat16*>(a.v), a.sel, static_cast<__nv_bfloat16*>(a.out), a.T, a.Hq, a.Hkv, a.G,
@@ -424,13 +424,13 @@ cudaError_t launch_attn(const DsaArgs& a, cudaStream_t st) {
 template <int DI>
 cudaError_t launch_select(const DsaArgs& a, cudaStream_t st) {
   using SM = SelSmem<DI>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     const cudaError_t e =
         cudaFuncSetAttribute(dsa_select_kernel<DI>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kTotal);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   const int nq = (a.T + kSelRows - 1) / kSelRows;
   dsa_select_kernel<DI><<<dim3(nq, a.B), kSelThreads, SM::kTotal, st>>>(
       static_cast<const __nv_bfloat16*>(a.qi), static_cast<const __nv_bfloat16*>(a.ki),

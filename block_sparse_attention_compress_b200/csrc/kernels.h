@@ -2,12 +2,44 @@
 // launches on `st`, returns cudaGetLastError(), and expects arguments that
 // nsa_api.cu has already validated.
 #pragma once
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace nsa {
+
+// A kernel's attributes (the dynamic shared-memory limit) belong to one device: a launcher
+// keeps one of these and sets its kernels' attributes the first time it runs on each device.
+// `set` makes the calls and returns the first error; nothing is remembered after an error, so
+// the next launch tries again.  Devices past the 64th are set on every launch.
+class PerDevice {
+ public:
+  template <class F>
+  cudaError_t once(F&& set) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? uint64_t(1) << dev : 0;
+    if (bit != 0 && (done_.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+    e = set();
+    if (e == cudaSuccess && bit != 0) done_.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
+
+// SMs of the current device (the persistent kernels' grid), 148 if the query fails.
+inline int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+    return 148;
+  return sms;
+}
 
 // K1: phi for every (b, h): out [B, N_c, H, d] bf16 (l = 32, s = 16 validated).
 cudaError_t launch_compress(const void* x, const void* w, int B, int T, int H, int d, int l, int s, void* out,

@@ -585,27 +585,27 @@ template <int KK>
 static cudaError_t launch_select(const MobaArgs& a, const __nv_bfloat16* q, const __nv_bfloat16* kbar, int32_t* idx,
                                  int32_t* counts, int nblk, cudaStream_t st) {
   if ((size_t)nblk * 4 > kSelectSmem) return cudaErrorInvalidValue;   // the per-CTA pick counts
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     const cudaError_t e =
         cudaFuncSetAttribute(moba_select_kernel<KK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelectSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   moba_select_kernel<KK><<<dim3((a.T + kSelQ - 1) / kSelQ, a.H, a.B), kSelThreads, kSelectSmem, st>>>(q, kbar, idx, counts, a.B,
                                                                                             a.T, a.H, a.bsz, nblk);
   return cudaGetLastError();
 }
 
 cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e = cudaFuncSetAttribute(moba_past_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moba_own_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   const int nblk = (a.T + a.bsz - 1) / a.bsz;
   const int E = a.B * a.H * nblk;
   const MobaLayout L = moba_layout(a.B, a.T, a.H, a.bsz, a.top_k);
@@ -650,21 +650,17 @@ cudaError_t launch_moba(const MobaArgs& a, cudaStream_t st) {
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     const size_t smem = (size_t)nblk * 4;   // at most 16384 blocks: 64 KB
-    static bool attr = false;
-    if (!attr) {
-      e = cudaFuncSetAttribute(moba_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536);
-      if (e != cudaSuccess) return e;
-      attr = true;
-    }
+    static PerDevice scatter_attr;
+    e = scatter_attr.once(
+        [] { return cudaFuncSetAttribute(moba_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 65536); });
+    if (e != cudaSuccess) return e;
     if (smem > 65536) return cudaErrorInvalidValue;
     moba_scatter_kernel<<<dim3((a.T + kScatterQ - 1) / kScatterQ, a.B * a.H), kScatterQ, smem, st>>>(
         idx, offsets, fill, list, a.T, a.H, nblk, a.top_k, a.bsz);
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (a.mark) { e = a.mark(a.mark_ctx, st); if (e != cudaSuccess) return e; }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   if (a.top_k > 0 && tc) {
     // every list holds at most B*H*T*top_k entries in all: the chunk count is bounded by
     // that over the chunk size plus one partial chunk per list

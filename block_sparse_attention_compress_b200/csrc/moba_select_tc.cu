@@ -268,13 +268,13 @@ moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 template <int KK>
 cudaError_t launch_kk(const MobaArgs& a, const void* kbar, int32_t* idx, int32_t* counts, int nblk,
                       cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     const cudaError_t e = cudaFuncSetAttribute(moba_select_tc_kernel<KK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                (int)SelSmem::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   CUtensorMap mq, mkb;
   const uint64_t dq[3] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)a.B * a.T};
   const uint64_t dkb[3] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)2 * a.B * nblk};

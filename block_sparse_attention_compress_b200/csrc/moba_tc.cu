@@ -719,13 +719,13 @@ moba_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 
 cudaError_t launch_moba_own_tc(const MobaArgs& a, const int32_t* idx, const __nv_bfloat16* part_o,
                                const float* part_lse, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(moba_own_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Smem::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   CUtensorMap mq, mk, mv;
   const uint64_t d3[3] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)a.B * a.T};
   const uint64_t s3[2] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2};
@@ -750,13 +750,13 @@ cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const 
                                 const int32_t* chunks, const int32_t* chunk_list, const int32_t* list,
                                 __nv_bfloat16* part_o, float* part_lse, int nblk, int E, size_t max_chunks,
                                 cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(moba_past_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Smem::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   if (max_chunks == 0) return cudaSuccess;
   CUtensorMap mk, mv;
   const uint64_t d3[3] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)a.B * a.T};
@@ -764,13 +764,7 @@ cudaError_t launch_moba_past_tc(const MobaArgs& a, const int32_t* counts, const 
   const uint32_t box[3] = {64, 1, (uint32_t)kBlk};
   if (!make_tmap_bf16(&mk, a.k, 3, d3, s3, box) || !make_tmap_bf16(&mv, a.v, 3, d3, s3, box))
     return cudaErrorInvalidValue;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  const int sms = sm_count();
   const unsigned grid = (unsigned)std::min<size_t>(max_chunks, (size_t)sms);
   moba_past_tc_kernel<<<grid, kThreads, Smem::kAlloc, st>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), counts, offsets, chunks, chunk_list, list, part_o, part_lse, a.T,

@@ -695,8 +695,8 @@ slc_redo_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __rest
 template <int DK, int DV>
 cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   using SM = Smem<DK, DV>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(slc_attn_tc_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
     if (e == cudaSuccess)
@@ -708,9 +708,9 @@ cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(slc_redo_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)RedoSmem<DK>::kBytes);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   CUtensorMap mk, mv, mq;
   const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.total};
   const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
@@ -723,13 +723,7 @@ cudaError_t launch_tc(const FwdArgs& a, cudaStream_t st) {
   if (!make_tmap_bf16(&mk, a.k, 3, dk3, sk3, box) || !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, box) ||
       !make_tmap_bf16(&mq, a.q, 3, dq3, sq3, qbox))
     return cudaErrorInvalidValue;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  const int sms = sm_count();
   const long items = (long)a.Hkv * a.B * a.T;
   const int grid = (int)(items < sms ? items : sms);
   auto kernel = a.cu ? slc_attn_tc_kernel<DK, DV, true> : slc_attn_tc_kernel<DK, DV, false>;

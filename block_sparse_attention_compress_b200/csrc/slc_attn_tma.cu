@@ -435,16 +435,16 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 template <int DK, int DV>
 cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   using SM = Smem<DK, DV>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(slc_attn_tma_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(slc_attn_tma_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SM::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   CUtensorMap mk, mv;
   const uint64_t dk3[3] = {(uint64_t)DK, (uint64_t)a.Hkv, (uint64_t)a.total};
   const uint64_t sk3[2] = {(uint64_t)DK * 2, (uint64_t)a.Hkv * DK * 2};
@@ -459,9 +459,7 @@ cudaError_t launch_tma(const FwdArgs& a, cudaStream_t st) {
   if (!make_tmap_bf16(&mk, a.k, 3, dk3, sk3, box) || !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, box) ||
       !make_tmap_bf16(&mq, a.q, 3, dq3, sq3, qbox))
     return cudaErrorInvalidValue;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const long total = (long)a.Hkv * a.B * a.T;
   const long ctas = (total + kGroups - 1) / kGroups;
   const int grid = (int)(ctas < (long)sms * kCtasPerSm ? ctas : (long)sms * kCtasPerSm);

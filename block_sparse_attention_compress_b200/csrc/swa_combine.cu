@@ -195,13 +195,13 @@ swa_combine_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __r
 template <int DK, int DV>
 cudaError_t launch(const FwdArgs& a, cudaStream_t st) {
   const size_t smem = Smem<DK, DV>::kTotal;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(swa_combine_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   dim3 grid((a.T + kWarps - 1) / kWarps, a.Hkv, a.B);
   swa_combine_kernel<DK, DV><<<grid, kThreads, smem, st>>>(
       static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),

@@ -462,16 +462,16 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 template <int DK, int DV>
 cudaError_t launch_w(const FwdArgs& a, cudaStream_t st) {
   using SM = Smem<DK, DV>;
-  static bool attr = false;
-  if (!attr) {
+  static PerDevice attr;
+  const cudaError_t e_attr = attr.once([&] {
     cudaError_t e =
         cudaFuncSetAttribute(window_tc_kernel<DK, DV, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SM::kAlloc);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(window_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)SM::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return e;
+  });
+  if (e_attr != cudaSuccess) return e_attr;
   CUtensorMap mq, mk, mv;
   const uint64_t dq[3] = {(uint64_t)DK, (uint64_t)a.Hq, (uint64_t)a.total};
   const uint64_t sq[2] = {(uint64_t)DK * 2, (uint64_t)a.Hq * DK * 2};
@@ -484,13 +484,7 @@ cudaError_t launch_w(const FwdArgs& a, cudaStream_t st) {
   if (!make_tmap_bf16(&mq, a.q, 3, dq, sq, bq) || !make_tmap_bf16(&mk, a.k, 3, dk3, sk3, bkv) ||
       !make_tmap_bf16(&mv, a.v, 3, dv3, sv3, bkv))
     return cudaErrorInvalidValue;
-  static int sms = 0;
-  if (sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  const int sms = sm_count();
   const long items = (long)((a.T + kTok - 1) / kTok) * a.Hkv * a.B;
   const int grid = (int)(items < sms ? items : sms);
   auto kernel = a.cu ? window_tc_kernel<DK, DV, true> : window_tc_kernel<DK, DV, false>;

@@ -1,7 +1,9 @@
-// Host-side TMA descriptor construction (driver entry point looked up once).
+// Host-side TMA descriptor construction (the driver's encoder is looked up on first use and kept
+// once the lookup succeeds).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "tc.cuh"
@@ -12,20 +14,31 @@ namespace {
 using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-EncodeFn g_encode = nullptr;
-std::once_flag g_once;
+std::atomic<EncodeFn> g_encode{nullptr};
+std::mutex g_lookup;
+
+// A failed lookup is not remembered: the next call asks the driver again.
+EncodeFn encoder() {
+  EncodeFn f = g_encode.load(std::memory_order_acquire);
+  if (f) return f;
+  std::lock_guard<std::mutex> lock(g_lookup);
+  f = g_encode.load(std::memory_order_acquire);
+  if (f) return f;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess && fn != nullptr) {
+    f = reinterpret_cast<EncodeFn>(fn);
+    g_encode.store(f, std::memory_order_release);
+  }
+  return f;
+}
 }  // namespace
 
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box) {
-  std::call_once(g_once, [] {
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      g_encode = reinterpret_cast<EncodeFn>(fn);
-  });
-  if (!g_encode || rank < 1 || rank > 5) return false;
+  const EncodeFn encode = encoder();
+  if (!encode || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], st[4];
   cuuint32_t bx[5], es[5];
   for (int i = 0; i < rank; ++i) {
@@ -34,7 +47,7 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t
     es[i] = 1;
     if (i + 1 < rank) st[i] = strides_bytes[i];
   }
-  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, st, bx, es,
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, st, bx, es,
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;

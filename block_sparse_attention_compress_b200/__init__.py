@@ -15,6 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnsa.so")
 
 NSA_OK, NSA_ERR_INVALID_ARG, NSA_ERR_UNSUPPORTED, NSA_ERR_WORKSPACE, NSA_ERR_CUDA, NSA_ERR_TIMEOUT = range(6)
+NSA_CODE_CU_SEQLENS = 200   # status word: a variable-length call's cu_seqlens broke its rules
 NSA_MODE_NSA, NSA_MODE_MOBA, NSA_MODE_DSA = 0, 1, 2
 NSA_MAP_TOUCH, NSA_MAP_CONTAINED, NSA_MAP_OVERLAP = 0, 1, 2
 
@@ -246,7 +247,8 @@ def nsa_decode(q, k_cache, v_cache, kc_cache, vc_cache, seqlens, max_seqlen: int
 
 def nsa_device_status(workspace, stream=None) -> tuple[int, int]:
     """(status, word) of the workspace's status word after synchronising the stream:
-    NSA_OK with word 0, or NSA_ERR_TIMEOUT with the code of the wait that gave up."""
+    NSA_OK with word 0, NSA_ERR_INVALID_ARG with NSA_CODE_CU_SEQLENS, or NSA_ERR_TIMEOUT with
+    the code of the wait that gave up."""
     word = ctypes.c_int32(0)
     st = load_library().nsa_device_status(_ptr(workspace), ctypes.byref(word), _stream(stream, workspace))
     return st, int(word.value)

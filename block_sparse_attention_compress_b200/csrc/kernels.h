@@ -92,6 +92,13 @@ struct FwdArgs {
   int* redo_list = nullptr;
 };
 
+// Status word code: the caller's cu_seqlens broke its rules (the kernels ran on clamped ranges).
+constexpr int kErrSeqRanges = 200;
+// The checked copy of cu_seqlens [B + 1] that the kernels of a packed batch read (one warp):
+// lengths clamped to [0, T], running sum capped at total; kErrSeqRanges if it differs from cu or
+// cu[B] != total.
+cudaError_t launch_seq_ranges(const int32_t* cu, int B, int T, int total, int32_t* safe, int* err, cudaStream_t st);
+
 // First row and length of sequence b in a (possibly variable-length) batch.
 __device__ __forceinline__ int seq_base(const int32_t* cu, int b, int T) { return cu ? __ldg(cu + b) : b * T; }
 __device__ __forceinline__ int seq_len(const int32_t* cu, int b, int T) {

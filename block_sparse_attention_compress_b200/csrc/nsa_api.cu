@@ -8,6 +8,8 @@
 #include "../../include/nsa.h"
 #include "kernels.h"
 
+static_assert(nsa::kErrSeqRanges == NSA_CODE_CU_SEQLENS, "one code for the checked cu_seqlens");
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -66,7 +68,7 @@ nsa_status check_cfg(const nsa_config* c) {
 }
 
 struct FwdLayout {
-  size_t err, kc, vc, idx, acc, redo, hk, hv, total;   // hk, hv: the MLP's hidden rows (phi_mlp only)
+  size_t err, kc, vc, idx, acc, redo, cu, hk, hv, total;   // hk, hv: the MLP's hidden rows (phi_mlp only)
 };
 
 FwdLayout forward_layout(const nsa_config* c) {
@@ -82,6 +84,7 @@ FwdLayout forward_layout(const nsa_config* c) {
   const size_t bwd_rows = B * nc * c->h_kv * (c->d_k + c->d_v) * 4 * (c->phi_mlp ? 2 : 1);
   L.acc = off; off = align_up(off + std::max(B * T * c->h_q * c->d_v * 4, bwd_rows));
   L.redo = off; off = align_up(off + B * c->h_kv * T * 4);   // the selected branch's redo list
+  L.cu = off; off = align_up(off + (B + 1) * 4);              // a packed batch's checked cu_seqlens
   if (c->phi_mlp) {
     L.hk = off; off = align_up(off + B * nc * c->h_kv * c->d_k * 2);
     L.hv = off; off = align_up(off + B * nc * c->h_kv * c->d_v * 2);
@@ -177,12 +180,17 @@ nsa_status nsa_forward_impl(const void* q, const void* k, const void* v, const v
   a.err = reinterpret_cast<int*>(ws + L.err);
   a.redo_count = a.err + 1;
   a.redo_list = reinterpret_cast<int*>(ws + L.redo);
-  a.cu = cu;
   a.total = total;
   a.w_straddle = straddle_weight(cfg);
 
   StageMarks marks(cfg, 5);
   cudaError_t e = cudaMemsetAsync(a.err, 0, 2 * sizeof(int), s);   // the status word and the redo count
+  if (cu) {   // every kernel reads the checked copy
+    int32_t* safe = reinterpret_cast<int32_t*>(ws + L.cu);
+    if (e == cudaSuccess) e = nsa::launch_seq_ranges(cu, a.B, a.T, total, safe, a.err, s);
+    cu = safe;
+  }
+  a.cu = cu;
   if (e == cudaSuccess) e = marks.mark(s);
   const int l = cfg->cmp_block, st = cfg->cmp_stride;
   if (e == cudaSuccess)
@@ -237,7 +245,7 @@ nsa_status nsa_device_status(const void* workspace, int32_t* code_out, void* str
   if (cudaStreamSynchronize(s) != cudaSuccess) return NSA_ERR_CUDA;
   if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return NSA_ERR_CUDA;
   if (code_out) *code_out = word;
-  return word == 0 ? NSA_OK : NSA_ERR_TIMEOUT;
+  return word == 0 ? NSA_OK : word == NSA_CODE_CU_SEQLENS ? NSA_ERR_INVALID_ARG : NSA_ERR_TIMEOUT;
 }
 
 nsa_status nsa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, uint32_t limit_us, void* stream) {
@@ -370,7 +378,7 @@ nsa_status backward_impl(const void* q, const void* k, const void* v, const void
   const float scale = cfg->softmax_scale > 0.f ? cfg->softmax_scale : 1.f / std::sqrt((float)cfg->d_k);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.kc = ws + L.kc; a.vc = ws + L.vc;
-  a.cu = cu;
+  int32_t* safe = cu ? reinterpret_cast<int32_t*>(ws + L.cu) : nullptr;   // the checked copy of cu
   a.dq = g.dq; a.gk = g.dk; a.gv = g.dv; a.dgates = g.dgates; a.dw_k = g.dw_k; a.dw_v = g.dw_v;
   // the Kc/Vc gradients (and the MLP's pre-activations) use the forward's accumulator region
   const size_t nkc = (size_t)a.B * a.nc * a.Hkv;
@@ -387,6 +395,11 @@ nsa_status backward_impl(const void* q, const void* k, const void* v, const void
   const size_t nk = (size_t)(cu ? total : a.B * a.T) * a.Hkv;   // the packed K/V rows
   const int l = cfg->cmp_block, cs = cfg->cmp_stride;
   cudaError_t e = cudaMemsetAsync(ws + L.err, 0, sizeof(int), s);
+  if (cu) {
+    if (e == cudaSuccess) e = nsa::launch_seq_ranges(cu, a.B, a.T, total, safe, reinterpret_cast<int*>(ws + L.err), s);
+    cu = safe;
+  }
+  a.cu = cu;
   if (e == cudaSuccess) e = cudaMemsetAsync(g.dk, 0, nk * a.dk * 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(g.dv, 0, nk * a.dv * 4, s);
   if (e == cudaSuccess && nkc) e = cudaMemsetAsync(a.gkc, 0, nkc * (a.dk + a.dv) * 4, s);

@@ -48,6 +48,9 @@ typedef enum {
   NSA_ERR_TIMEOUT = 5       /* a bounded device-side wait gave up (see nsa_device_status) */
 } nsa_status;
 
+/* Status word value (nsa_device_status): the contents of cu_seqlens broke its rules. */
+#define NSA_CODE_CU_SEQLENS 200
+
 typedef enum {
   NSA_MODE_NSA = 0,   /* compressed + selected + sliding-window branches, gated sum */
   NSA_MODE_MOBA = 1,  /* MoBA: mean-pooled block keys, per-head top-k plus the own block */
@@ -217,7 +220,12 @@ NSA_API nsa_status nsa_forward(const void* q, const void* k, const void* v, cons
  *   cu_seqlens   int32 [B + 1] device: sequence b is rows cu_seqlens[b] .. cu_seqlens[b+1]-1
  *                of q, k, v, gates and out; cu_seqlens[0] = 0, non-decreasing, every length
  *                <= cfg->seqlen (empty sequences allowed), cu_seqlens[B] = total_tokens.  The
- *                contents are not checked: values outside these rules give undefined results.
+ *                contents are checked on the device, never read by the host: the kernels take
+ *                their ranges from a copy in the workspace whose lengths are clamped to
+ *                [0, cfg->seqlen] and whose running sum stops at total_tokens, so that no
+ *                contents take them outside the packed rows.  Contents outside the rules leave
+ *                NSA_CODE_CU_SEQLENS in the status word (nsa_device_status then returns
+ *                NSA_ERR_INVALID_ARG) and an output computed on the clamped ranges.
  *   total_tokens the packed row count (host), 1 <= total_tokens <= B * cfg->seqlen.
  *   q bf16 [total, H_q, d_k];  k [total, H_kv, d_k];  v [total, H_kv, d_v];
  *   gates bf16 [total, H_q, 3];  out bf16 [total, H_q, d_v].
@@ -411,8 +419,9 @@ NSA_API nsa_status nsa_forward_noalloc(const void* q, const void* k, const void*
  * wait on an mbarrier (one second); a wait that gives up writes a nonzero code to the word,
  * and the kernel stops issuing work and returns instead of hanging.
  * Synchronises `stream` (a cudaStream_t, NULL = the default stream), reads the word and
- * returns NSA_OK if it is 0, NSA_ERR_TIMEOUT otherwise (code_out, if not NULL, receives the
- * word: which wait gave up).  NSA_ERR_INVALID_ARG for a null workspace, NSA_ERR_CUDA if the
+ * returns NSA_OK if it is 0, NSA_ERR_INVALID_ARG if it is NSA_CODE_CU_SEQLENS (the contents of
+ * a variable-length call's cu_seqlens broke their rules), NSA_ERR_TIMEOUT otherwise (code_out,
+ * if not NULL, receives the word: which wait gave up).  NSA_ERR_INVALID_ARG for a null workspace, NSA_ERR_CUDA if the
  * synchronisation or the copy fails.
  */
 NSA_API nsa_status nsa_device_status(const void* workspace, int32_t* code_out, void* stream);

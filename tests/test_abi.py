@@ -80,10 +80,11 @@ def test_status_strings(lib):
 def test_workspace_size_of_the_workloads(lib):
     c = _cfg()
     # status word and redo count, kc 63*64*2, vc same, idx 1*1024*4*4, acc 1024*4*64*4, the selected
-    # branch's redo list 1*1*1024*4 (each rounded up to 256 B)
+    # branch's redo list 1*1*1024*4, a packed batch's checked cu_seqlens (B + 1)*4 (each rounded up
+    # to 256 B)
     up = lambda x: (x + 255) // 256 * 256
     assert nsa.nsa_workspace_size(c) == (256 + 2 * up(63 * 64 * 2) + up(1024 * 4 * 4) + up(1024 * 4 * 64 * 4) +
-                                         up(1024 * 4))
+                                         up(1024 * 4) + up(2 * 4))
     big = _cfg(seqlen=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512)
     assert nsa.nsa_workspace_size(big) > 65536 * 64 * 128 * 4
     assert nsa.nsa_workspace_size(_cfg(h_q=6, h_kv=4)) == 0

@@ -115,3 +115,47 @@ def test_varlen_benchmark_batch():
         sl = slice(lo, lo + L)
         check_sequence_against_oracle(q[sl], k[sl], v[sl], gates[sl], w_k, w_v, out[sl], idx[b, :, :L], top_k,
                                       window, toks, f"sequence {b} (length {L})")
+
+
+def clamped_ranges(cu, T, total):
+    """The checked copy of cu_seqlens the library's kernels read (include/nsa.h,
+    nsa_forward_varlen): each length clamped to [0, T], the running sum stopped at total."""
+    safe, run = [0], 0
+    for b in range(len(cu) - 1):
+        run = min(run + min(max(cu[b + 1] - cu[b], 0), T), total)
+        safe.append(run)
+    return safe
+
+
+@pytest.mark.parametrize("bad", [
+    [0, 400, 437, 466],   # a length above T
+    [0, 300, 200, 466],   # decreasing
+    [0, 100, 200, 900],   # cu[B] past the packed rows
+    [50, 100, 200, 300],  # cu[0] != 0
+    [0, -5, 100, 466],    # negative
+])
+def test_varlen_cu_seqlens_outside_its_rules(bad):
+    """Contents of cu_seqlens that break its rules are reported by the status word
+    (NSA_CODE_CU_SEQLENS, nsa_device_status -> NSA_ERR_INVALID_ARG), and the kernels ran on the
+    clamped ranges: the output equals, bit for bit, a call made with those ranges."""
+    import block_sparse_attention_compress_b200 as nsa
+    lengths = [300, 37, 129]
+    hq, hkv, dk, dv, top_k, window = 16, 1, 192, 128, 4, 100
+    q, k, v, gates, w_k, w_v, _ = packed_inputs(lengths, hq, hkv, dk, dv, seed=52)
+    total, T = q.shape[0], max(lengths)
+    safe = clamped_ranges(bad, T, total)
+    assert safe != bad or bad[-1] != total
+    dq, dkk, dvv, dg, wk, wv = (t.to(DEV) for t in (q, k, v, gates, w_k, w_v))
+    f = NSAForwardVarlen(len(lengths), T, hq, hkv, dk, dv, wk, wv, top_k=top_k, window=window)
+    out = f(dq, dkk, dvv, dg, torch.tensor(bad, dtype=torch.int32, device=DEV))
+    st, word = nsa.nsa_device_status(f.workspace)
+    assert (st, word) == (nsa.NSA_ERR_INVALID_ARG, nsa.NSA_CODE_CU_SEQLENS)
+    n = safe[-1]
+    ref_f = NSAForwardVarlen(len(lengths), T, hq, hkv, dk, dv, wk, wv, top_k=top_k, window=window)
+    ref = ref_f(dq[:n], dkk[:n], dvv[:n], dg[:n], torch.tensor(safe, dtype=torch.int32, device=DEV))
+    torch.cuda.synchronize()
+    assert ref_f.device_status() == 0, "the clamped ranges keep every rule"
+    assert torch.equal(out[:n].cpu(), ref.cpu())
+    for b in range(len(lengths)):
+        L = safe[b + 1] - safe[b]
+        assert torch.equal(f.idx[b, :, :L].cpu(), ref_f.idx[b, :, :L].cpu()), f"sequence {b}: chosen blocks"

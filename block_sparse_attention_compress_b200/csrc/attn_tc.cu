@@ -337,10 +337,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // before leaving, let the copies still in flight land (bounded)
       for (int i = 0; i < kKcSlots && i < fill; ++i) {
         const int f = fill - 1 - i;
-        tc::mbar_wait(kc_full + (f % kKcSlots), (f / kKcSlots) & 1, err, kErrKcFull);
+        tc::mbar_drain(kc_full + (f % kKcSlots), (f / kKcSlots) & 1);
       }
-      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_wait(vc_full + (n & 1), (n >> 1) & 1, err, kErrVcFull);
-      if (k > 0) tc::mbar_wait(bar_q, (k - 1) & 1, err, kErrQ);
+      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_drain(vc_full + (n & 1), (n >> 1) & 1);
+      if (k > 0) tc::mbar_drain(bar_q, (k - 1) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -689,6 +689,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   }
 
+  tc::settle_after_error(err);
   tc::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -204,9 +204,11 @@ moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   }
 
   // every tile has been read (the MMAs before the last s_full, the offers before here): the
-  // tile buffers take the other lists of each query, which join the first
+  // tile buffers take the other lists of each query, which join the first.  After a wait gave
+  // up, tiles may still be landing: they are let land first.
   float* mv = reinterpret_cast<float*>(sB);                    // [part - 1][row][7]
   int* mj = reinterpret_cast<int*>(mv + (kSplit - 1) * kRows * 7);
+  tc::settle_after_error(err);
   tc::tc_fence_before();
   __syncthreads();
   if (warp < kOfferWarps && part > 0) {
@@ -244,11 +246,14 @@ moba_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           sel[i + 1] = x;
         }
     int32_t* dst = idx + (((size_t)b * H + h) * T + t) * (KK + 1);
+    // a list cut short by a wait that gave up still holds its initial entries: only past
+    // blocks are written and counted (the counts and the lists built from them agree)
 #pragma unroll
     for (int i = 0; i < KK; ++i) {
       if (i < kk) {
-        dst[i] = sel[i];
-        atomicAdd(hist + sel[i], 1);
+        const bool past = sel[i] >= 0 && sel[i] < J;
+        dst[i] = past ? sel[i] : -1;
+        if (past) atomicAdd(hist + sel[i], 1);
       } else {
         dst[i + 1] = -1;
       }

@@ -187,9 +187,9 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     if (lane == 0) {   // let the copies in flight land (bounded)
       for (int i = 0; i < kKSlots && i < fill; ++i) {
         const int f = fill - 1 - i;
-        tc::mbar_wait(k_full + (f % kKSlots), (f / kKSlots) & 1, err, kErrKFull);
+        tc::mbar_drain(k_full + (f % kKSlots), (f / kKSlots) & 1);
       }
-      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull);
+      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_drain(v_full + (n & 1), (n >> 1) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -382,6 +382,7 @@ moba_past_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
   }
 
+  tc::settle_after_error(err);
   tc::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -486,9 +487,9 @@ moba_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       }
       for (int i = 0; i < kKSlots && i < fill; ++i) {   // let the copies in flight land (bounded)
         const int f = fill - 1 - i;
-        tc::mbar_wait(k_full + (f % kKSlots), (f / kKSlots) & 1, err, kErrKFull);
+        tc::mbar_drain(k_full + (f % kKSlots), (f / kKSlots) & 1);
       }
-      for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull);
+      for (int n = max(0, ntiles - 2); n < ntiles; ++n) tc::mbar_drain(v_full + (n & 1), (n >> 1) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -708,6 +709,7 @@ moba_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
   }
 
+  tc::settle_after_error(err);
   tc::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

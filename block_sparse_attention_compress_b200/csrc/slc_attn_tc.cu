@@ -566,6 +566,7 @@ slc_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     }
   }
 
+  tc::settle_after_error(err);
   tc::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -177,9 +177,9 @@ slc_attn_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     }
     if (lane == 0) {   // let copies in flight land
       for (long f = fill - 1; f >= 0 && f >= fill - kSlots; --f)
-        tc::mbar_wait(full + (f % kSlots), (uint32_t)((f / kSlots) & 1), err, 22);
+        tc::mbar_drain(full + (f % kSlots), (uint32_t)((f / kSlots) & 1));
       for (long f = qfill - 1; f >= 0 && f >= qfill - 2; --f)   // qfill = query copies issued
-        tc::mbar_wait(q_full + (f & 1), (uint32_t)((f >> 1) & 1), err, 25);
+        tc::mbar_drain(q_full + (f & 1), (uint32_t)((f >> 1) & 1));
     }
   } else {
     // ---------------------------------------------------------------- consumers

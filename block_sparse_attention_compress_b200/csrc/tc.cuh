@@ -111,6 +111,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
   return false;
 }
 
+// A producer's last look at its own copies before it leaves: waits for the phase that the
+// copies it issued complete, whatever the status word says (they land within microseconds),
+// for at most `limit_ns`.  Records nothing.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 10000000ull) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 <= limit_ns)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Once a wait of this launch (or an earlier one on the stream) gave up, copies and MMAs issued
+// before that may still be landing in this CTA's shared and tensor memory: thread 0 lets
+// `ns` pass (they finish within microseconds) before the CTA's final barrier, so that nothing
+// lands after the tensor memory is freed or the CTA has left.  Costs one load when the
+// status word is 0.
+__device__ __forceinline__ void settle_after_error(const int* err, uint64_t ns = 1000000ull) {
+  if (threadIdx.x != 0 || *(volatile const int*)err == 0) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (globaltimer_ns() - t0 < ns) __nanosleep(1000);
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_3d(void* smem, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
   asm volatile(

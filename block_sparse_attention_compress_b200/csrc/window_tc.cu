@@ -193,10 +193,10 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       // let the copies in flight land (bounded)
       for (int i = 0; i < kKSlots && i < fill; ++i) {
         const int f = fill - 1 - i;
-        tc::mbar_wait(k_full + (f % kKSlots), (f / kKSlots) & 1, err, kErrKFull);
+        tc::mbar_drain(k_full + (f % kKSlots), (f / kKSlots) & 1);
       }
-      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_wait(v_full + (n & 1), (n >> 1) & 1, err, kErrVFull);
-      if (k > 0) tc::mbar_wait(bar_q, (k - 1) & 1, err, kErrQ);
+      for (int n = max(0, vcnt - 2); n < vcnt; ++n) tc::mbar_drain(v_full + (n & 1), (n >> 1) & 1);
+      if (k > 0) tc::mbar_drain(bar_q, (k - 1) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -451,6 +451,7 @@ window_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
   }
 
+  tc::settle_after_error(err);
   tc::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {

@@ -530,7 +530,7 @@ def run_varlen_bench(args, dev, world):
             "tflops_computed": flops / (ms * 1e-3) / 1e12,
             "frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "stages_ms": {n: round(v, 4) for n, v in stages.items()},
-            "gpu_launches": len(STAGES) * args.steps}
+            "gpu_launches": (len(STAGES) + 1) * args.steps}   # + the check of cu_seqlens (one warp)
 
 
 def run_phi_mlp_bench(args, dev, world):

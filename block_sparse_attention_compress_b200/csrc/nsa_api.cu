@@ -183,15 +183,15 @@ nsa_status nsa_forward_impl(const void* q, const void* k, const void* v, const v
   a.total = total;
   a.w_straddle = straddle_weight(cfg);
 
-  StageMarks marks(cfg, 5);
-  cudaError_t e = cudaMemsetAsync(a.err, 0, 2 * sizeof(int), s);   // the status word and the redo count
+  StageMarks marks(cfg, 5);   // the first stage also holds the status word's reset and the range check
+  cudaError_t e = marks.mark(s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.err, 0, 2 * sizeof(int), s);   // the status word and the redo count
   if (cu) {   // every kernel reads the checked copy
     int32_t* safe = reinterpret_cast<int32_t*>(ws + L.cu);
     if (e == cudaSuccess) e = nsa::launch_seq_ranges(cu, a.B, a.T, total, safe, a.err, s);
     cu = safe;
   }
   a.cu = cu;
-  if (e == cudaSuccess) e = marks.mark(s);
   const int l = cfg->cmp_block, st = cfg->cmp_stride;
   if (e == cudaSuccess)
     e = cfg->phi_mlp ? nsa::launch_compress_mlp(k, cfg->w_cmp_k, cfg->b_cmp_k, cfg->w_cmp_k2, a.B, a.T, a.Hkv, a.dk, l,

@@ -103,7 +103,8 @@ typedef enum {
  *   n_stage_events handles.  When n_stage_events >= (kernels launched) + 1, event 0 is
  *                 recorded on `stream` before the first kernel and event i after the
  *                 i-th, so that cudaEventElapsedTime gives each kernel's duration.
- *                 nsa_forward has 5 stages in NSA mode (phi of K, phi of V,
+ *                 nsa_forward has 5 stages in NSA mode (phi of K, which also holds the
+ *                 status word's reset and, for a packed batch, the check of cu_seqlens; phi of V,
  *                 compressed attention + selection, selected attention, window +
  *                 combine) and 5 in MoBA mode (block means, selection, query lists,
  *                 past-block attention, own block + merge); nsa_decode has 1.

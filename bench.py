@@ -443,10 +443,11 @@ def run_decode_bench(args, dev, world):
 
 
 def run_moba_bench(args, dev, world):
-    """MoBA forward of the 128K-token, 32-head workload (stage times from the library's events)."""
+    """MoBA forward of the 128K-token, 32-head workload (stage times from the library's events);
+    --moba-seqlen takes a shorter sequence of the same shape (for a profiler capture)."""
     import block_sparse_attention_compress_b200 as nsa
     c = synth.WORKLOADS["moba_128k"]
-    B, T, H, d = 1, c["T"], c["h"], c["d"]
+    B, T, H, d = 1, args.moba_seqlen or c["T"], c["h"], c["d"]
     x = synth.moba_inputs(B, T, H, d, seed=0, device=dev)
     out = torch.empty((B, T, H, d), dtype=torch.bfloat16, device=dev)
     cfg = nsa.make_config(mode=nsa.NSA_MODE_MOBA, batch=B, seqlen=T, h_q=H, h_kv=H, d_k=d, d_v=d,
@@ -477,7 +478,8 @@ def run_moba_bench(args, dev, world):
     ms = allreduce_max(step_ms, world, dev)
     attn, score = moba_flops(T, H, d, c["block"], c["top_k"], B)
     peaks, src = load_peaks()
-    return {"workload": f"moba_128k: B=1 T={T} heads={H} d={d} block={c['block']} top_k={c['top_k']} + own block",
+    name = "moba_128k" if T == c["T"] else "moba"
+    return {"workload": f"{name}: B=1 T={T} heads={H} d={d} block={c['block']} top_k={c['top_k']} + own block",
             "ms_per_step": ms, "tokens_per_s": world * B * T / (ms * 1e-3),
             "tflops_computed": (attn + score) / (ms * 1e-3) / 1e12,
             "frac_of_bf16_peak": (attn + score) / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
@@ -777,6 +779,9 @@ def main():
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step and print its line (for a profiler capture)")
     ap.add_argument("--decode-batch", type=int, default=0, help="decode sequences (default: the workload's 32)")
+    ap.add_argument("--moba-only", action="store_true",
+                    help="time only the MoBA forward and print its line (for a profiler capture)")
+    ap.add_argument("--moba-seqlen", type=int, default=0, help="MoBA tokens (default: the workload's 131072)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -795,6 +800,13 @@ def main():
             res = run_decode_bench(args, dev, world)
             if rank == 0:
                 print(json.dumps({"metric": METRIC, "decode": res}), flush=True)
+            return
+        if args.moba_only:
+            dev = torch.device("cuda", local_rank)
+            torch.cuda.set_device(dev)
+            res = run_moba_bench(args, dev, world)
+            if rank == 0:
+                print(json.dumps({"metric": METRIC, "moba": res}), flush=True)
             return
         run_ours(args, rank, world, local_rank)
     finally:

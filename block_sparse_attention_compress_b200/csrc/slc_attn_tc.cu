@@ -24,20 +24,20 @@
 //
 // Persistent: one CTA per SM walks the items group-major (the CTAs running together share
 // one group's K/V in L2).  Warp roles:
-//   warp 8     TMA producer of keys: the item's block list (into shared memory), its 16
+//   warp 12    TMA producer of keys: the item's block list (into shared memory), its 16
 //              query rows (3-slot item ring), each pair's K (2-slot ring of 48 KB pairs).
-//   warp 10    TMA producer of values: each pair's V (2-slot ring of 32 KB pairs).  The
+//   warp 14    TMA producer of values: each pair's V (2-slot ring of 32 KB pairs).  The
 //              rings run across items.
-//   warp 9     MMA issuer (one thread): S of pair n, then the P.V of pair n - 1, so the
-//              softmax of a pair overlaps the next pair's S.  Alternate items accumulate
-//              into two O buffers, so an item's pairs overlap the previous item's epilogue.
+//   warp 13    MMA issuer (one thread): the S of pairs 0 and 1, then per step the P.V of
+//              pair n and the S of pair n + 2, so the softmax of a pair overlaps the S of the
+//              pairs after it.  Alternate items accumulate into two O buffers, so an item's
+//              pairs overlap the previous item's epilogue.
 //   warps 0-7  softmax: warp w takes TMEM lane quadrant w % 4 (32 keys of each pair) and
-//              heads 8(w / 4) .. 8(w / 4) + 7.  p = 2^(s*scale - m) with a reference m per
-//              (quadrant, head) set from the quadrant's first valid scores of the item and
-//              never moved: the keys of quadrant q reach O^T only through partials 2q and
-//              2q + 1, so the epilogue brings the quadrants to a common reference and no
-//              warp waits for another.  P^T (bf16) goes to shared memory; each thread keeps
-//              its keys' partial row sums, added up once per item.
+//              heads 8(w / 4) .. 8(w / 4) + 7.  p = 2^(s*scale - m) with one reference m per
+//              (item, head): the largest valid score of the item's first pair, agreed by the
+//              four quadrants' warps at a named barrier and never moved afterwards, so no
+//              warp waits for another after the first pair.  P^T (bf16) goes to shared
+//              memory; each thread keeps its keys' partial row sums, added up once per item.
 //   warps 8-11 epilogue, one quadrant of value columns each: acc += g_slc * O / l.
 //
 // A later score can exceed its fixed reference without bound, so p is not bounded by 1.

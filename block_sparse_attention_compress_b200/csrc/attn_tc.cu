@@ -7,15 +7,17 @@
 // consecutive tokens (longest rows first).  An item's 128 query rows (token-major, 16 heads
 // per token) are one tcgen05 M=128 tile held in shared memory.  The group's compressed
 // keys/values stream through shared memory by TMA in tiles of 128 blocks.
-//   pass A   S = Q Kc^T into TMEM (rows = (token, head)); each softmax thread owns a
-//            row and keeps its running max and sum -> log-sum-exp per row.
+//   pass A   S = Q Kc^T into TMEM (rows = (token, head)); each softmax thread keeps the
+//            running max and sum of its row's 32 columns of every tile, and the four
+//            groups' pairs are merged once per item -> log-sum-exp per row.
 //   pass B   S^T = Kc Q^T into TMEM (rows = compressed blocks, columns = (token, head)):
 //            each softmax thread owns one compressed block, forms the normalised
 //            probabilities of its 128 columns, adds each token's 16 heads in registers
 //            (the group sum), folds them into 64-token selection-block scores, and
 //            writes P^T (bf16) to shared memory; O^T = Vc^T P^T accumulates in TMEM
 //            (rows = value dims), already normalised, so no rescaling is ever needed.
-//   top-k    per token over the selection-block scores in shared memory.
+//   top-k    per token over the selection-block scores: the top-k warps copy a finished
+//            item's scores from shared memory into registers and select there.
 //   epilogue acc[t, h, :] = g_cmp * o_cmp, read from O^T (each thread one value dim).
 // Warp roles: 16 TMA producer, 17 MMA issuer (and TMEM owner), 18-19 top-k, 0-15 softmax /
 // epilogue in four groups of four (warp w owns TMEM lanes 32*(w%4)..+31; group w/4 takes 32

@@ -398,7 +398,9 @@ namespace {
 // keys from the own block's start to the CTA's last query in 128-key tiles, masked to u <= t;
 // the same TMA / MMA / softmax roles and lazy reference as the past-block kernel.  Epilogue:
 // the own-block state (O unnormalised against the reference m, row sum l) merged with the
-// query's past-block partials by their log-sum-exps; out in bf16.
+// query's past-block partials by their log-sum-exps; out in bf16.  Each softmax thread asks
+// L2 for its half rows of those partials when it starts, so that the merge does not wait for
+// DRAM.
 __global__ void __launch_bounds__(kThreads, 1)
 moba_own_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ idx,

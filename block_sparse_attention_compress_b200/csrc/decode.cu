@@ -15,7 +15,9 @@
 //   B  the selected blocks (two per warp), with one more softmax state per warp;
 //      each branch's states are merged by log-sum-exp weights;
 //   C  out = g_cmp*o_cmp + g_slc*o_slc + g_win*o_win, rounded to bf16.
-// Loads are 16-byte cp.async of whole K/V rows (coalesced, each row 384 + 256 bytes).
+// Loads are 16-byte cp.async of whole K/V rows (each row 384 + 256 bytes): a group of eight
+// lanes copies one 128-byte line of a row, so each copy instruction of a warp moves lines of
+// four rows, and each lane looks its four rows up once per tile.
 #include <cfloat>
 
 #include "common.cuh"

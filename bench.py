@@ -36,6 +36,7 @@ import synth  # noqa: E402
 
 METRIC = "NSA fwd tokens/s @T=64K and % bf16 tensor peak; decode GB/s vs HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0   # the datasheet dense bf16 rate of one B200 (context for the measured peaks)
 L, S, BSEL = 32, 16, 64
 STAGES = ["phi_k", "phi_v", "cmp_select", "slc_attn", "swa_combine"]
 
@@ -292,6 +293,8 @@ def run_ours(args, rank, world, local_rank):
         "config": workload_config(c, args.workload),
         "tflops_computed": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12,
         "frac_of_bf16_peak": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / peaks["bf16_tflops"],
+        "frac_of_bf16_sustained": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+        "frac_of_bf16_nominal": total_flops / (statistics.mean(step_ms) * 1e-3) / 1e12 / NOMINAL_BF16_TFLOPS,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                      "frac": ach / peak,
                      "traffic": (None if NCU_DRAM_BYTES_PER_ITEM.get(dom) is None

@@ -34,6 +34,8 @@ nsa_status check_cfg(const nsa_config* c) {
     return NSA_ERR_INVALID_ARG;
   if (c->h_q % c->h_kv) return NSA_ERR_INVALID_ARG;
   if (c->top_k < 0 || c->sel_block < 1) return NSA_ERR_INVALID_ARG;
+  // the kernels index (token, head) rows and take TMA row coordinates in 32 bits
+  if ((int64_t)c->batch * c->seqlen * c->h_q > (int64_t)INT32_MAX) return NSA_ERR_UNSUPPORTED;
   if (!(c->softmax_scale >= 0.f) || std::isinf(c->softmax_scale)) return NSA_ERR_INVALID_ARG;
   if (c->mode == NSA_MODE_NSA) {
     if (c->cmp_block < 1 || c->cmp_stride < 1 || c->window < 1) return NSA_ERR_INVALID_ARG;

@@ -74,7 +74,9 @@ typedef enum {
  *   mode          nsa_mode.
  *   batch, seqlen B and T of the prefill (nsa_forward); in nsa_decode,
  *                 `batch` is the number of sequences and `seqlen` the capacity
- *                 L_max of the caches (their second dimension).
+ *                 L_max of the caches (their second dimension).  Every mode needs
+ *                 batch * seqlen * h_q <= 2^31 - 1 (the kernels index rows in 32
+ *                 bits), else NSA_ERR_UNSUPPORTED.
  *   h_q, h_kv     query and KV heads; h_q % h_kv == 0.  MoBA needs h_q == h_kv.
  *   d_k, d_v      head dims.  Implemented: NSA (d_k,d_v) in {(64,64),(128,128),
  *                 (192,128)}, G <= 16, T <= 65536; MoBA d_k = d_v = 128, sel_block a

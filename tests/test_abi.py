@@ -99,6 +99,9 @@ def test_workspace_size_of_the_workloads(lib):
     big = _cfg(seqlen=65536, h_q=64, h_kv=4, d_k=192, d_v=128, top_k=16, window=512)
     assert nsa.nsa_workspace_size(big) > 65536 * 64 * 128 * 4
     assert nsa.nsa_workspace_size(_cfg(h_q=6, h_kv=4)) == 0
+    # batch * seqlen * h_q rows up to 2^31 - 1 (32-bit row indices in the kernels), not beyond
+    assert nsa.nsa_workspace_size(_cfg(batch=(1 << 31) // 4096 - 1)) > 0
+    assert nsa.nsa_workspace_size(_cfg(batch=(1 << 31) // 4096)) == 0
 
 
 @made_up_pointers
@@ -117,6 +120,7 @@ def test_workspace_size_of_the_workloads(lib):
     (dict(d_k=96, d_v=96), nsa.NSA_ERR_UNSUPPORTED),
     (dict(seqlen=65537), nsa.NSA_ERR_UNSUPPORTED),
     (dict(top_k=33), nsa.NSA_ERR_UNSUPPORTED),
+    (dict(batch=1 << 20, seqlen=1024, h_q=4), nsa.NSA_ERR_UNSUPPORTED),   # 2^32 (token, head) rows
 ])
 def test_forward_rejects_bad_configs_without_launching(lib, kw, status):
     c = _cfg(**kw)
